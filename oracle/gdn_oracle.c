@@ -1,0 +1,325 @@
+/*
+ * gdn_oracle.c -- plain fp64 CPU oracle for the gated delta rule.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The CUDA library
+ * never calls it and shares no code, header or constant with it.
+ *
+ * What it computes (the definition, written out token by token):
+ *
+ *   S_t = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *   o_t = scale * S_t q_t
+ *
+ * Source: "Inside Qwen3.8-27B: Hybrid DeltaNet Architecture, 256k Context,
+ * and 24GB Local Serving", section "Gated DeltaNet Mechanics" (the delta rule
+ * removes the old association stored under k_t before writing v_t; S_t is a
+ * d x d state of fixed size; k_t is the normalized key, v_t the value).  The
+ * displayed equation did not survive on that page; the form above is the
+ * gated delta rule it describes in words, with alpha_t = exp(g_t) the decay
+ * and beta_t the write strength.  Head layout (16 query/key heads shared by
+ * 48 value heads, head dim 128): "Qwen 3.8 27B Review: Native Vision, FP8
+ * Quantization & 1M Context in a Compact Dense Model", section "3.
+ * Architecture: Gated DeltaNet Hybrid + FP8 Quantization".
+ *
+ * Readings where the pages are silent (each one is listed in the design
+ * notes of the repository):
+ *   - S is stored Dv x Dk (row i = value dimension i, Dk contiguous), so the
+ *     write term is v k^T, the read is S k and the output is S q.
+ *   - V head h reads query/key head h / (Hv / Hqk) (contiguous groups).
+ *   - g and beta are per (token, V head); alpha = exp(g).
+ *   - o_t uses the state after token t's update.
+ *   - Each sequence starts from its own initial state (zeros if none).
+ *
+ * The update is applied row by row: with u = S_{t-1} k_t (one number per
+ * row i of S),  alpha S (I - beta k k^T) + beta v k^T
+ *             = alpha S + beta (v - alpha u) k^T,
+ * which touches row i of S only through u_i.  That identity is the only
+ * rearrangement here; it is exact algebra, and the tests check the result
+ * against the explicit matrix-product form computed independently.
+ *
+ * Also here: the chunked (WY / UT-transform) form of the same recurrence,
+ * derived from the definition above, in fp64.  It exists to show that the
+ * chunked algebra a GPU kernel follows reproduces the token-by-token
+ * definition; the tests check it against the sequential oracle.
+ *
+ * Threads: units (sequence, V head) are independent and are spread over
+ * POSIX threads; inside a unit the arithmetic order is fixed, so results do
+ * not depend on the thread count.
+ */
+#include <math.h>
+#include <pthread.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <unistd.h>
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEMORY 2
+
+typedef struct {
+    const double *q, *k, *v, *g, *beta;
+    const int64_t *cu_seqlens;
+    int num_seqs, Hqk, Hv, Dk, Dv, chunk;
+    double scale;
+    const double *initial_state; /* [N, Hv, Dv, Dk] or NULL */
+    double *final_state;         /* [N, Hv, Dv, Dk] or NULL */
+    double *o;                   /* [T, Hv, Dv] */
+    int64_t next_unit;           /* shared work counter */
+    pthread_mutex_t lock;
+    int failed;
+} job_t;
+
+/* ---- sequential definition, one (sequence n, V head h) unit ---------- */
+static void sequential_unit(const job_t *J, int n, int h, double *S)
+{
+    const int Dk = J->Dk, Dv = J->Dv, Hqk = J->Hqk, Hv = J->Hv;
+    const int j = h / (Hv / Hqk); /* query/key head of V head h */
+    const size_t sdim = (size_t)Dv * Dk;
+
+    if (J->initial_state)
+        memcpy(S, J->initial_state + ((size_t)n * Hv + h) * sdim, sdim * sizeof(double));
+    else
+        memset(S, 0, sdim * sizeof(double));
+
+    for (int64_t t = J->cu_seqlens[n]; t < J->cu_seqlens[n + 1]; ++t) {
+        const double alpha = exp(J->g[t * Hv + h]);
+        const double b = J->beta[t * Hv + h];
+        const double *kt = J->k + ((size_t)t * Hqk + j) * Dk;
+        const double *qt = J->q + ((size_t)t * Hqk + j) * Dk;
+        const double *vt = J->v + ((size_t)t * Hv + h) * Dv;
+        double *ot = J->o + ((size_t)t * Hv + h) * Dv;
+
+        for (int i = 0; i < Dv; ++i) {
+            double *Si = S + (size_t)i * Dk;
+            double u = 0.0; /* u_i = (S_{t-1} k_t)_i */
+            for (int c = 0; c < Dk; ++c) u += Si[c] * kt[c];
+            const double w = b * (vt[i] - alpha * u);
+            for (int c = 0; c < Dk; ++c) Si[c] = alpha * Si[c] + w * kt[c];
+        }
+        for (int i = 0; i < Dv; ++i) {
+            const double *Si = S + (size_t)i * Dk;
+            double acc = 0.0; /* (S_t q_t)_i */
+            for (int c = 0; c < Dk; ++c) acc += Si[c] * qt[c];
+            ot[i] = J->scale * acc;
+        }
+    }
+    if (J->final_state)
+        memcpy(J->final_state + ((size_t)n * Hv + h) * sdim, S, sdim * sizeof(double));
+}
+
+/* ---- chunked WY / UT form, one unit ----------------------------------
+ *
+ * Within a chunk of C' <= C tokens (aligned to the sequence start) with
+ * start state S0 and local prefix sums G_t = g_1 + ... + g_t:
+ *   writing w_t = beta_t (v_t - alpha_t S_{t-1} k_t), S_t = alpha_t S_{t-1} + w_t k_t^T,
+ *   S_t = e^{G_t} S0 + sum_{s<=t} e^{G_t-G_s} w_s k_s^T.
+ * Substituting into w_t gives the unit lower-triangular system
+ *   w_t + sum_{s<t} A_ts w_s = beta_t (v_t - e^{G_t} S0 k_t),
+ *   A_ts = beta_t e^{G_t-G_s} (k_t . k_s),
+ * so with Tm = (I + A)^{-1}:  W = Tm diag(beta e^G) K,  Ut = Tm diag(beta) V,
+ *   U = Ut - W S0^T            (row t of U is w_t),
+ *   o_t = e^{G_t} S0 q_t + sum_{s<=t} e^{G_t-G_s} (q_t . k_s) w_s,
+ *   S_C' = e^{G_C'} S0 + sum_s e^{G_C'-G_s} w_s k_s^T.
+ * Requires finite g (exp(G_t - G_s) of two infinite sums is undefined).
+ */
+static void chunked_unit(const job_t *J, int n, int h, double *S, double *scratch)
+{
+    const int Dk = J->Dk, Dv = J->Dv, Hqk = J->Hqk, Hv = J->Hv, C = J->chunk;
+    const int j = h / (Hv / Hqk);
+    const size_t sdim = (size_t)Dv * Dk;
+    double *G = scratch;                       /* C       */
+    double *A = G + C;                         /* C x C   */
+    double *Tm = A + (size_t)C * C;            /* C x C   */
+    double *W = Tm + (size_t)C * C;            /* C x Dk  */
+    double *U = W + (size_t)C * Dk;            /* C x Dv  */
+    double *Snew = U + (size_t)C * Dv;         /* Dv x Dk */
+
+    if (J->initial_state)
+        memcpy(S, J->initial_state + ((size_t)n * Hv + h) * sdim, sdim * sizeof(double));
+    else
+        memset(S, 0, sdim * sizeof(double));
+
+    const int64_t t0 = J->cu_seqlens[n], t1 = J->cu_seqlens[n + 1];
+    for (int64_t c0 = t0; c0 < t1; c0 += C) {
+        const int L = (int)((t1 - c0) < C ? (t1 - c0) : C);
+#define KROW(r) (J->k + ((size_t)(c0 + (r)) * Hqk + j) * Dk)
+#define QROW(r) (J->q + ((size_t)(c0 + (r)) * Hqk + j) * Dk)
+#define VROW(r) (J->v + ((size_t)(c0 + (r)) * Hv + h) * Dv)
+#define GVAL(r) (J->g[(c0 + (r)) * Hv + h])
+#define BVAL(r) (J->beta[(c0 + (r)) * Hv + h])
+        double acc = 0.0;
+        for (int r = 0; r < L; ++r) { acc += GVAL(r); G[r] = acc; }
+
+        /* A (strictly lower) */
+        for (int r = 0; r < L; ++r)
+            for (int s = 0; s < L; ++s) {
+                double a = 0.0;
+                if (s < r) {
+                    double kk = 0.0;
+                    for (int c = 0; c < Dk; ++c) kk += KROW(r)[c] * KROW(s)[c];
+                    a = BVAL(r) * exp(G[r] - G[s]) * kk;
+                }
+                A[(size_t)r * C + s] = a;
+            }
+        /* Tm = (I + A)^{-1} by forward substitution, column by column */
+        for (int col = 0; col < L; ++col)
+            for (int r = 0; r < L; ++r) {
+                double x = (r == col) ? 1.0 : 0.0;
+                for (int s = 0; s < r; ++s) x -= A[(size_t)r * C + s] * Tm[(size_t)s * C + col];
+                Tm[(size_t)r * C + col] = x;
+            }
+        /* W = Tm diag(beta e^G) K ;  U = Tm diag(beta) V - W S0^T */
+        for (int r = 0; r < L; ++r) {
+            for (int c = 0; c < Dk; ++c) {
+                double x = 0.0;
+                for (int s = 0; s < L; ++s) x += Tm[(size_t)r * C + s] * BVAL(s) * exp(G[s]) * KROW(s)[c];
+                W[(size_t)r * Dk + c] = x;
+            }
+            for (int i = 0; i < Dv; ++i) {
+                double x = 0.0;
+                for (int s = 0; s < L; ++s) x += Tm[(size_t)r * C + s] * BVAL(s) * VROW(s)[i];
+                double ws = 0.0;
+                for (int c = 0; c < Dk; ++c) ws += W[(size_t)r * Dk + c] * S[(size_t)i * Dk + c];
+                U[(size_t)r * Dv + i] = x - ws;
+            }
+        }
+        /* outputs */
+        for (int r = 0; r < L; ++r) {
+            double *ot = J->o + ((size_t)(c0 + r) * Hv + h) * Dv;
+            const double er = exp(G[r]);
+            for (int i = 0; i < Dv; ++i) {
+                double x = 0.0;
+                for (int c = 0; c < Dk; ++c) x += S[(size_t)i * Dk + c] * QROW(r)[c];
+                x *= er;
+                for (int s = 0; s <= r; ++s) {
+                    double qk = 0.0;
+                    for (int c = 0; c < Dk; ++c) qk += QROW(r)[c] * KROW(s)[c];
+                    x += exp(G[r] - G[s]) * qk * U[(size_t)s * Dv + i];
+                }
+                ot[i] = J->scale * x;
+            }
+        }
+        /* carried state */
+        const double eL = exp(G[L - 1]);
+        for (int i = 0; i < Dv; ++i)
+            for (int c = 0; c < Dk; ++c) {
+                double x = eL * S[(size_t)i * Dk + c];
+                for (int s = 0; s < L; ++s) x += exp(G[L - 1] - G[s]) * U[(size_t)s * Dv + i] * KROW(s)[c];
+                Snew[(size_t)i * Dk + c] = x;
+            }
+        memcpy(S, Snew, sdim * sizeof(double));
+#undef KROW
+#undef QROW
+#undef VROW
+#undef GVAL
+#undef BVAL
+    }
+    if (J->final_state)
+        memcpy(J->final_state + ((size_t)n * Hv + h) * sdim, S, sdim * sizeof(double));
+}
+
+static void *worker(void *arg)
+{
+    job_t *J = (job_t *)arg;
+    const size_t sdim = (size_t)J->Dv * J->Dk;
+    size_t extra = 0;
+    if (J->chunk > 0)
+        extra = (size_t)J->chunk * (1 + 2 * (size_t)J->chunk + J->Dk + J->Dv) + sdim;
+    double *S = (double *)malloc((sdim + extra) * sizeof(double));
+    if (!S) {
+        pthread_mutex_lock(&J->lock);
+        J->failed = 1;
+        pthread_mutex_unlock(&J->lock);
+        return NULL;
+    }
+    const int64_t total = (int64_t)J->num_seqs * J->Hv;
+    for (;;) {
+        pthread_mutex_lock(&J->lock);
+        const int64_t u = J->next_unit++;
+        pthread_mutex_unlock(&J->lock);
+        if (u >= total) break;
+        const int n = (int)(u / J->Hv), h = (int)(u % J->Hv);
+        if (J->chunk > 0)
+            chunked_unit(J, n, h, S, S + sdim);
+        else
+            sequential_unit(J, n, h, S);
+    }
+    free(S);
+    return NULL;
+}
+
+static int run(job_t *J, int num_threads)
+{
+    if (!J->q || !J->k || !J->v || !J->g || !J->beta || !J->cu_seqlens || !J->o) return ORACLE_BAD_ARG;
+    if (J->num_seqs < 0 || J->Hqk <= 0 || J->Hv <= 0 || J->Dk <= 0 || J->Dv <= 0) return ORACLE_BAD_ARG;
+    if (J->Hv % J->Hqk != 0) return ORACLE_BAD_ARG;
+    if (J->cu_seqlens[0] != 0) return ORACLE_BAD_ARG;
+    for (int n = 0; n < J->num_seqs; ++n)
+        if (J->cu_seqlens[n + 1] < J->cu_seqlens[n]) return ORACLE_BAD_ARG;
+
+    if (num_threads <= 0) num_threads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (num_threads <= 0) num_threads = 1;
+    const int64_t units = (int64_t)J->num_seqs * J->Hv;
+    if (num_threads > units) num_threads = (int)(units > 0 ? units : 1);
+
+    J->next_unit = 0;
+    J->failed = 0;
+    pthread_mutex_init(&J->lock, NULL);
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)num_threads);
+    if (!th) { pthread_mutex_destroy(&J->lock); return ORACLE_NO_MEMORY; }
+    int started = 0;
+    for (int i = 0; i < num_threads; ++i) {
+        if (pthread_create(&th[i], NULL, worker, J) != 0) break;
+        ++started;
+    }
+    if (started == 0) worker(J);
+    for (int i = 0; i < started; ++i) pthread_join(th[i], NULL);
+    free(th);
+    pthread_mutex_destroy(&J->lock);
+    return J->failed ? ORACLE_NO_MEMORY : ORACLE_OK;
+}
+
+/*
+ * Prefill over packed sequences.  Arrays are host fp64, row-major:
+ *   q, k [T, Hqk, Dk];  v [T, Hv, Dv];  g, beta [T, Hv];  o [T, Hv, Dv];
+ *   cu_seqlens [num_seqs + 1] (cu_seqlens[0] = 0, non-decreasing, last = T);
+ *   initial_state, final_state [num_seqs, Hv, Dv, Dk] (either may be NULL;
+ *   NULL initial state means zeros, NULL final state skips the write).
+ * chunk = 0 runs the token-by-token definition; chunk > 0 runs the chunked
+ * WY/UT form with that chunk size.  num_threads <= 0 uses every online core.
+ * Returns 0 on success, 1 on a bad argument, 2 when memory ran out.
+ */
+int gdn_oracle_prefill(const double *q, const double *k, const double *v, const double *g,
+                       const double *beta, const int64_t *cu_seqlens, int num_seqs, int Hqk,
+                       int Hv, int Dk, int Dv, double scale, const double *initial_state,
+                       double *final_state, double *o, int chunk, int num_threads)
+{
+    job_t J;
+    memset(&J, 0, sizeof(J));
+    J.q = q; J.k = k; J.v = v; J.g = g; J.beta = beta; J.cu_seqlens = cu_seqlens;
+    J.num_seqs = num_seqs; J.Hqk = Hqk; J.Hv = Hv; J.Dk = Dk; J.Dv = Dv; J.chunk = chunk;
+    J.scale = scale; J.initial_state = initial_state; J.final_state = final_state; J.o = o;
+    if (chunk < 0) return ORACLE_BAD_ARG;
+    return run(&J, num_threads);
+}
+
+/*
+ * One decode step for B sequences, one token each: the same update as the
+ * prefill applied once per (sequence b, V head h), state updated in place.
+ *   q, k [B, Hqk, Dk];  v [B, Hv, Dv];  g, beta [B, Hv];  state [B, Hv, Dv, Dk];
+ *   o [B, Hv, Dv].
+ */
+int gdn_oracle_decode_step(const double *q, const double *k, const double *v, const double *g,
+                           const double *beta, double *state, double *o, int B, int Hqk, int Hv,
+                           int Dk, int Dv, double scale, int num_threads)
+{
+    if (B < 0) return ORACLE_BAD_ARG;
+    int64_t *cu = (int64_t *)malloc(sizeof(int64_t) * ((size_t)B + 1));
+    if (!cu) return ORACLE_NO_MEMORY;
+    for (int b = 0; b <= B; ++b) cu[b] = b; /* B sequences of one token each */
+    int rc = gdn_oracle_prefill(q, k, v, g, beta, cu, B, Hqk, Hv, Dk, Dv, scale, state, state, o,
+                                0, num_threads);
+    free(cu);
+    return rc;
+}

@@ -1,0 +1,48 @@
+"""The fp64 oracle against what the definition fixes (CPU only).
+
+See tests/oracle_pins.py for what each check pins and why it is independent
+of the oracle's own code.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import oracle_pins as P
+
+
+@pytest.mark.parametrize("D", [1, 2, 4, 8])
+@pytest.mark.parametrize("T", [1, 5, 12])
+def test_product_form(oracle_lib, D, T):
+    P.check_product_form(oracle_lib, seed=D * 31 + T, T=T, Dk=D, Dv=max(1, D - 1))
+
+
+def test_product_form_gqa_and_scale(oracle_lib):
+    P.check_product_form(oracle_lib, seed=99, T=6, Hqk=2, Hv=6, Dk=3, Dv=2, scale=0.37)
+
+
+@pytest.mark.parametrize("name", [c.__name__ for c in P.ALL_CHECKS if c is not P.check_product_form])
+def test_pin(oracle_lib, name):
+    getattr(P, name)(oracle_lib)
+
+
+def test_thread_count_does_not_change_bits(oracle_lib):
+    q, k, v, g, beta, s0 = P.random_problem(11, 40, 2, 6, 8, 8, N=2)
+    cu = np.array([0, 17, 40])
+    a = oracle.prefill(q, k, v, g, beta, cu_seqlens=cu, initial_state=s0, num_threads=1)
+    b = oracle.prefill(q, k, v, g, beta, cu_seqlens=cu, initial_state=s0, num_threads=8)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_rejects_bad_cu_seqlens(oracle_lib):
+    q, k, v, g, beta, s0 = P.random_problem(12, 6, 1, 1, 2, 2, init=False)
+    with pytest.raises(ValueError):
+        oracle.prefill(q, k, v, g, beta, cu_seqlens=np.array([0, 4, 3, 6]))
+    with pytest.raises(ValueError):
+        oracle.prefill(q, k, v, g, beta, cu_seqlens=np.array([1, 6]))
+
+
+def test_empty_input(oracle_lib):
+    q, k, v, g, beta, s0 = P.random_problem(13, 0, 1, 3, 2, 2)
+    o, fin = oracle.prefill(q, k, v, g, beta, initial_state=s0)
+    assert o.shape == (0, 3, 2)
+    assert np.array_equal(fin, s0)

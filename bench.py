@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""Benchmark of the gated delta rule library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints ONE JSON line (rank 0).  A step is one prefill call over the
+Qwen3.8-27B-shaped DeltaNet layer workload (B=1, T=8192, 16 QK / 48 V heads,
+head dim 128, bf16 q/k/v, fp32 g/beta, fp32 state, zero initial state, final
+state returned).  ``value`` is prefill throughput in Mtok/s with the inputs
+resident in HBM, L2 flushed between timed steps.  The same line carries:
+  roofline     the prefill kernel against its bound (algorithmic flops or bytes
+               per launch / CUDA-event launch time, over the measured peak);
+  decode       the batched decode workload (B=64, 1000 steps, fp32 state of
+               201 MB updated in place): state GB/s against HBM peak;
+  e2e          prefill through the public API with inputs copied from pinned
+               host memory and o / final state copied back, every step;
+  cpu_baseline the fp64 oracle on the host cores (rank 0, N=1 only);
+  clocks       SM clocks and throttle reasons sampled during the timed region.
+With --gpus N under torchrun each rank runs its own independent workload
+(weak scaling, no collective on the data path); timings are the max over
+ranks.  ``--impl reference`` times the fp64 oracle instead, on the host.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+# Algorithmic work per token of one DeltaNet layer at Hqk=16, Hv=48, D=128, chunk 64.
+#   flops: per (chunk, V head): QK^T 1.05M + KK^T 1.05M (both shared by the 3 V heads
+#   of a QK head) + W 1.05M + U~ 1.05M + W S0^T 2.10M + Q S0^T 2.10M + P U 1.05M +
+#   state 2.10M  ->  7,602,176 flop per token over the layer.
+#   bytes: q 4096 + k 4096 + v 12288 (bf16) + o 24576 (fp32) + g 192 + beta 192
+#   = 45,440 per token.
+FLOP_PER_TOKEN = 7_602_176
+BYTES_PER_TOKEN = 45_440
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--decode-steps", type=int, default=1000)
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------- distributed
+class Dist:
+    """Rank bookkeeping; torch.distributed only for barriers and max-over-ranks."""
+
+    def __init__(self, backend=None):
+        import torch.distributed as dist
+
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.dist = dist if self.world > 1 else None
+        if self.dist is not None and not dist.is_initialized():
+            import datetime
+
+            dist.init_process_group(backend=backend or "nccl",
+                                    timeout=datetime.timedelta(seconds=120))
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float, device=None) -> float:
+        if self.dist is None:
+            return float(x)
+        import torch
+
+        t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None and self.dist.is_initialized():
+            self.dist.destroy_process_group()
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent workload (weak scaling)."""
+    return base + 1000 * rank
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id=None):
+        self.proc = None
+        self.gpu_id = gpu_id
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if self.gpu_id:
+            cmd += ["-i", self.gpu_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        return False
+
+    def summary(self):
+        if not getattr(self, "lines", None):
+            return None
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(PEAKS_FALLBACK), "fallback"
+
+
+def kernel_traffic(kernel_key: str, source_file: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel source changed after the counters were taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+        ent = table[kernel_key]
+        with open(source_file, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        if ent.get("source_sha") != sha:
+            return None
+        return ent["dram_bytes_per_launch"]
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+# ---------------------------------------------------------------- oracle (CPU)
+def oracle_prefill_timed(inp, ntok, num_threads=0):
+    """Time the fp64 oracle on the first ``ntok`` tokens (all heads) of a
+    single-sequence prefill workload; returns (seconds, threads used)."""
+    import numpy as np
+
+    import oracle
+
+    lib = oracle.load()
+    sl = {n: inp[n][:ntok] for n in ("q", "k", "v", "g", "beta")}
+    arrs = {n: np.ascontiguousarray(sl[n].double().numpy()) for n in sl}
+    cu = np.array([0, ntok], dtype=np.int64)
+    Hv = arrs["v"].shape[1]
+    threads = num_threads if num_threads > 0 else (os.cpu_count() or 1)
+    threads = min(threads, Hv)
+    t0 = time.perf_counter()
+    oracle.prefill(arrs["q"], arrs["k"], arrs["v"], arrs["g"], arrs["beta"], cu_seqlens=cu,
+                   num_threads=threads, want_final=True, lib=lib)
+    return time.perf_counter() - t0, threads
+
+
+# ---------------------------------------------------------------- main arms
+def workload_desc(w):
+    return (f"{w.name}: B={len(w.lengths)} T={w.total_tokens} Hqk={w.Hqk} Hv={w.Hv} D={w.D} "
+            f"{w.dtype} q/k/v, fp32 g/beta, fp32 o, fp32 state "
+            f"{'zero init' if w.init_std == 0 else 'N(0,%g) init' % w.init_std}, final state returned")
+
+
+def run_reference(args, D):
+    """The fp64 oracle timed on the host cores (rank 0 only)."""
+    import torch
+
+    from gated_deltanet_recurrence_rule_b200 import inputs
+
+    w = inputs.WORKLOADS["prefill8k"]
+    if D.rank != 0:
+        return None
+    inp = inputs.workload_inputs(w)
+    ntok = 1024
+    secs = []
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        s, threads = oracle_prefill_timed(inp, ntok)
+        if i >= args.warmup:
+            secs.append(s)
+    total = sum(secs)
+    value = ntok * len(secs) / total / 1e6
+    return {
+        "impl": "reference",
+        "metric": "GDN prefill Mtok/s (H=16/48,D=128) and decode-step state GB/s vs HBM peak",
+        "value": value, "unit": "Mtok/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total / len(secs) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "global_batch": 1, "seq_len": w.total_tokens,
+                   "parallelism": "host threads over (sequence, V head)",
+                   "sample": f"first {ntok} tokens, all 48 V heads, per step"},
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": threads, "kind": "oracle",
+                         "sample": f"first {ntok} of 8192 tokens, all 48 V heads, per step"},
+        "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def run_ours(args, D):
+    import torch
+
+    from gated_deltanet_recurrence_rule_b200 import api, inputs
+
+    dev = torch.device("cuda", D.local_rank)
+    torch.cuda.set_device(dev)
+    api.load()
+    w = inputs.WORKLOADS["prefill8k"]
+    inp = inputs.prefill_inputs(w.lengths, w.Hqk, w.Hv, w.D, dtype=w.dtype,
+                                seed=rank_seed(w.seed, D.rank))
+    T = w.total_tokens
+    x = {n: t.to(dev) for n, t in inp.items() if t is not None}
+    o = torch.empty((T, w.Hv, w.D), dtype=torch.float32, device=dev)
+    fin = torch.empty((1, w.Hv, w.D, w.D), dtype=torch.float32, device=dev)
+    ws = torch.zeros(api.prefill_workspace_size(1, T, w.Hqk, w.Hv, w.D, w.D), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # > 126 MB L2
+
+    def step():
+        api.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=x["cu_seqlens"],
+                    final_state=fin, o=o, workspace=ws)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    D.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(gpu_uuid(torch, dev)) as clk:
+        for e0, e1 in evs:
+            flush.zero_()              # outside the timed pair: L2 holds nothing of the inputs
+            e0.record(stream)
+            step()
+            e1.record(stream)
+        torch.cuda.synchronize()
+    D.barrier()
+    per_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    local_ms = sum(per_ms)
+    max_ms = D.max(local_ms, dev)
+    status = api.get_device_status(ws)
+    if status != api.GDN_OK:
+        raise RuntimeError(f"device status after timing: {api.status_string(status)}")
+    ms_per_step = max_ms / args.steps
+    value = D.world * T * args.steps / (max_ms / 1e3) / 1e6
+
+    peaks, peak_src = load_peaks()
+    kernel_ms = statistics.mean(per_ms)
+    uses_tc = _tc_path_available()
+    if uses_tc:
+        achieved = FLOP_PER_TOKEN * T / (kernel_ms / 1e3) / 1e12
+        peak = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "kernel": "gdn_prefill_tc", "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
+                "algorithmic": f"{FLOP_PER_TOKEN} flop/token x {T} tokens",
+                "traffic": kernel_traffic("prefill_tc", os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_prefill_tc.cu"))}
+    else:
+        # CUDA-core path: 3 fp32 FMAs per state element per token (read, update, output)
+        flop = 3 * 2 * w.D * w.D * w.Hv * T
+        fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        achieved = flop / (kernel_ms / 1e3) / 1e12
+        roof = {"bound": "alu", "kernel": "prefill_simt_kernel", "achieved": achieved,
+                "peak": fp32_peak, "unit": "TFLOP/s", "frac": achieved / fp32_peak,
+                "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
+                "algorithmic": f"3 FMA per state element per token = {flop} flop",
+                "traffic": kernel_traffic("prefill_simt", os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_prefill_simt.cu"))}
+    roof["hbm_bytes_algorithmic"] = BYTES_PER_TOKEN * T + w.Hv * w.D * w.D * 4
+    roof["hbm_frac"] = roof["hbm_bytes_algorithmic"] / (kernel_ms / 1e3) / 1e9 / peaks["hbm_gbs"]
+
+    out = {
+        "metric": "GDN prefill Mtok/s (H=16/48,D=128) and decode-step state GB/s vs HBM peak",
+        "value": value, "unit": "Mtok/s", "n_gpus": D.world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": workload_desc(w), "global_batch": D.world, "seq_len": T,
+                   "parallelism": f"replicas{D.world}" if D.world > 1 else "single GPU",
+                   "l2": "flushed between timed steps (256 MiB write outside the timed pair)"},
+        "roofline": roof,
+        "gpu_launches": args.steps,
+        "clocks": clk.summary(),
+    }
+
+    if not args.no_e2e:
+        out["e2e"] = _e2e(args, D, inp, dev, w, ws)
+
+    if not args.no_decode:
+        out["decode"] = _decode(args, D, dev, peaks, peak_src)
+
+    if not args.no_cpu_baseline and D.rank == 0 and D.world == 1:
+        secs, threads = oracle_prefill_timed(inp, T)
+        out["cpu_baseline"] = {"value": T / secs / 1e6, "unit": "Mtok/s", "cores": threads,
+                               "kind": "oracle",
+                               "sample": f"the whole workload ({T} tokens x {w.Hv} V heads) once, "
+                                         f"{secs:.1f} s wall"}
+    return out
+
+
+def _tc_path_available():
+    from gated_deltanet_recurrence_rule_b200 import api
+
+    return api.prefill_uses_tensor_cores(16, 48, 128, 128)
+
+
+def _e2e(args, D, inp, dev, w, ws):
+    import torch
+
+    from gated_deltanet_recurrence_rule_b200 import api
+
+    names = ("q", "k", "v", "g", "beta", "cu_seqlens")
+    host = {n: inp[n].pin_memory() for n in names}
+    devb = {n: torch.empty_like(host[n], device=dev) for n in names}
+    T = w.total_tokens
+    o_host = torch.empty((T, w.Hv, w.D), dtype=torch.float32).pin_memory()
+    f_host = torch.empty((1, w.Hv, w.D, w.D), dtype=torch.float32).pin_memory()
+    o = torch.empty((T, w.Hv, w.D), dtype=torch.float32, device=dev)
+    fin = torch.empty((1, w.Hv, w.D, w.D), dtype=torch.float32, device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_host.numel() * 4 + f_host.numel() * 4
+
+    def step():
+        for n in names:
+            devb[n].copy_(host[n], non_blocking=True)
+        api.prefill(devb["q"], devb["k"], devb["v"], devb["g"], devb["beta"],
+                    cu_seqlens=devb["cu_seqlens"], final_state=fin, o=o, workspace=ws)
+        o_host.copy_(o, non_blocking=True)
+        f_host.copy_(fin, non_blocking=True)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    ms = D.max(e0.elapsed_time(e1), dev)
+    return {"value": D.world * T * args.steps / (ms / 1e3) / 1e6, "unit": "Mtok/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / args.steps, "host_buffers": "pinned"}
+
+
+def _decode(args, D, dev, peaks, peak_src):
+    import torch
+
+    from gated_deltanet_recurrence_rule_b200 import api, inputs
+
+    w = inputs.WORKLOADS["decode64"]
+    steps = args.decode_steps
+    d = inputs.decode_inputs(w.batch, w.Hqk, w.Hv, w.D, steps=steps, dtype=w.dtype,
+                             seed=rank_seed(w.seed, D.rank), init_std=w.init_std)
+    x = {n: d[n].to(dev) for n in ("q", "k", "v", "g", "beta")}
+    S = d["state"].to(dev)
+    o = torch.empty((w.batch, w.Hv, w.D), dtype=torch.float32, device=dev)
+
+    def run(n):
+        for s in range(n):
+            api.decode_step(x["q"][s], x["k"][s], x["v"][s], x["g"][s], x["beta"][s], S, o=o)
+
+    run(min(steps, 10))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    run(steps)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    ms = D.max(e0.elapsed_time(e1), dev)
+    state_bytes = w.batch * w.Hv * w.D * w.D * 4
+    # q, k (bf16) + v (bf16) + o (fp32) + g, beta (fp32)
+    io_bytes = w.batch * (2 * w.Hqk * w.D * 2 + w.Hv * w.D * 2 + w.Hv * w.D * 4 + 2 * w.Hv * 4)
+    per_step = 2 * state_bytes + io_bytes
+    us = ms * 1e3 / steps
+    gbs = D.world * per_step * steps / (ms / 1e3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"value": gbs, "unit": "GB/s", "workload": f"decode64: B={w.batch} x 1 token, Hqk={w.Hqk} "
+            f"Hv={w.Hv} D={w.D} bf16, fp32 state {state_bytes} B in place, {steps} steps",
+            "us_per_step": us, "steps_per_s": steps / (ms / 1e3),
+            "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": gbs / D.world,
+                         "peak": peak, "unit": "GB/s", "frac": gbs / D.world / peak,
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "algorithmic": f"{per_step} B per step (state read+write {2 * state_bytes} + io {io_bytes})",
+                         "traffic": kernel_traffic("decode", os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_decode.cu"))},
+            "gpu_launches": steps}
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        # the oracle runs on the host; only rank 0 works, other ranks exit 0
+        if int(os.environ.get("RANK", "0")) != 0:
+            return 0
+        D = Dist.__new__(Dist)
+        D.rank, D.world, D.local_rank, D.dist = 0, 1, 0, None
+        out = run_reference(args, D)
+        print(json.dumps(out), flush=True)
+        return 0
+    D = Dist()
+    try:
+        out = run_ours(args, D)
+        if D.rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        D.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,155 @@
+// gdn_api.cu -- the C ABI of libgdn.so (declared in include/gdn.h).
+//
+// Host-side argument validation, status codes and kernel dispatch.  No entry
+// point allocates memory, keeps pointers between calls or synchronises,
+// except gdn_get_device_status, which synchronises the stream it is given.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+#include "gdn_common.cuh"
+
+namespace gdn {
+cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, float *state, void *o, int B, int Hqk, int Hv,
+                          int Dk, int Dv, int dtype, int o_dtype, float scale,
+                          cudaStream_t stream);
+cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, const int32_t *cu, int N, long long T_,
+                                int Hqk, int Hv, int Dk, int Dv, int dtype, int o_dtype,
+                                float scale, const float *s0, float *sfin, void *o,
+                                int32_t *status, cudaStream_t stream);
+bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype);
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const int32_t *cu, int N, long long T_,
+                              int Hqk, int Hv, int o_dtype, float scale, const float *s0,
+                              float *sfin, void *o, void *workspace, cudaStream_t stream);
+}  // namespace gdn
+
+namespace {
+
+constexpr int32_t kVersion = 100;  // 0.1.0
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+bool dtype_ok(int32_t dtype) { return dtype == GDN_DTYPE_BF16 || dtype == GDN_DTYPE_FP32; }
+
+bool dims_ok(int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, int32_t dtype) {
+  if (Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0) return false;
+  if (!dtype_ok(dtype)) return false;
+  return Dk > 0 && Dv > 0;
+}
+
+bool dims_supported(int32_t Dk, int32_t Dv) {
+  return (Dk == 64 || Dk == 128) && (Dv == 64 || Dv == 128);
+}
+
+int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(int32_t status) {
+  switch (status) {
+    case GDN_OK: return "GDN_OK";
+    case GDN_ERR_INVALID_ARG: return "GDN_ERR_INVALID_ARG: invalid argument";
+    case GDN_ERR_UNSUPPORTED: return "GDN_ERR_UNSUPPORTED: shape or dtype not supported";
+    case GDN_ERR_CUDA: return "GDN_ERR_CUDA: a CUDA call or launch failed";
+    case GDN_ERR_DEVICE_TIMEOUT: return "GDN_ERR_DEVICE_TIMEOUT: a bounded wait in a kernel ran out";
+    case GDN_ERR_BAD_SEQLENS: return "GDN_ERR_BAD_SEQLENS: cu_seqlens is not 0 = c0 <= ... <= cN = T";
+    case GDN_ERR_WORKSPACE: return "GDN_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    default: return "GDN_ERR_UNKNOWN";
+  }
+}
+
+int32_t gdn_version(void) { return kVersion; }
+
+size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t num_qk_heads,
+                                  int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
+                                  int32_t dtype) {
+  if (num_seqs < 0 || total_tokens < 0) return 0;
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return 0;
+  return gdn::kWorkspaceHeaderBytes;
+}
+
+int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
+                    int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
+                    int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, int32_t o_dtype,
+                    float scale, const float *initial_state, float *final_state, void *o,
+                    void *workspace, size_t workspace_bytes, void *stream) {
+  if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dtype_ok(o_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !g || !beta || !o) return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(g, 4) || !aligned(beta, 4))
+      return GDN_ERR_INVALID_ARG;
+  }
+  if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
+    return GDN_ERR_INVALID_ARG;
+  const size_t need = gdn_prefill_workspace_size(num_seqs, total_tokens, num_qk_heads,
+                                                 num_v_heads, head_dim_k, head_dim_v, dtype);
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+  // grid-size limits of the launches below
+  if ((int64_t)num_seqs * num_v_heads * 4 > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t *status = static_cast<int32_t *>(workspace);
+  cudaError_t e;
+  if (gdn::prefill_tc_supported(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) {
+    e = gdn::launch_prefill_tc(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_qk_heads,
+                               num_v_heads, o_dtype, scale, initial_state, final_state, o,
+                               workspace, s);
+  } else {
+    e = gdn::launch_prefill_simt(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
+                                 num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype,
+                                 scale, initial_state, final_state, o, status, s);
+  }
+  return cuda_status(e);
+}
+
+int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, float *state, void *o, int32_t batch,
+                        int32_t num_qk_heads, int32_t num_v_heads, int32_t head_dim_k,
+                        int32_t head_dim_v, int32_t dtype, int32_t o_dtype, float scale,
+                        void *stream) {
+  if (batch < 0) return GDN_ERR_INVALID_ARG;
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dtype_ok(o_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
+  if (batch == 0) return GDN_OK;
+  if ((int64_t)batch * num_v_heads > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !g || !beta || !state || !o) return GDN_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      !aligned(state, 16) || !aligned(g, 4) || !aligned(beta, 4))
+    return GDN_ERR_INVALID_ARG;
+  return cuda_status(gdn::launch_decode(q, k, v, g, beta, state, o, batch, num_qk_heads,
+                                        num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype,
+                                        scale, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t gdn_prefill_uses_tensor_cores(int32_t num_qk_heads, int32_t num_v_heads,
+                                      int32_t head_dim_k, int32_t head_dim_v, int32_t dtype) {
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return 0;
+  return gdn::prefill_tc_supported(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype) ? 1 : 0;
+}
+
+int32_t gdn_get_device_status(const void *workspace, void *stream, int32_t *status_host) {
+  if (!workspace || !status_host || !aligned(workspace, 256)) return GDN_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t value = GDN_OK;
+  cudaError_t e = cudaMemcpyAsync(&value, workspace, sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(const_cast<void *>(workspace), 0, sizeof(int32_t), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return GDN_ERR_CUDA;
+  *status_host = value;
+  return GDN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// gdn_common.cuh -- small device helpers shared by the libgdn kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdn.h"
+
+namespace gdn {
+
+// Workspace header written by gdn_prefill (first 256 bytes of the workspace).
+struct WorkspaceHeader {
+  int32_t status;       // GDN_OK or a device-detected error code (first one wins)
+  int32_t reserved0;
+  uint32_t next_unit;   // dynamic work counter of persistent kernels
+  uint32_t reserved1;
+};
+constexpr size_t kWorkspaceHeaderBytes = 256;
+
+__device__ __forceinline__ void report_status(int32_t *status, int32_t code) {
+  if (status) atomicCAS(status, GDN_OK, code);
+}
+
+// ---- element conversion ---------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+// Load 4 consecutive elements (8-byte aligned for bf16, 16-byte for fp32).
+__device__ __forceinline__ void load4(const float *p, float out[4]) {
+  const float4 x = *reinterpret_cast<const float4 *>(p);
+  out[0] = x.x; out[1] = x.y; out[2] = x.z; out[3] = x.w;
+}
+__device__ __forceinline__ void load4(const __nv_bfloat16 *p, float out[4]) {
+  const uint2 x = *reinterpret_cast<const uint2 *>(p);
+  out[0] = __uint_as_float(x.x << 16);
+  out[1] = __uint_as_float(x.x & 0xffff0000u);
+  out[2] = __uint_as_float(x.y << 16);
+  out[3] = __uint_as_float(x.y & 0xffff0000u);
+}
+
+// Streaming (evict-first) 128-bit global load / store for data touched once.
+__device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p); }
+__device__ __forceinline__ void st_stream(float4 *p, float4 v) { __stcs(p, v); }
+
+// Call f(T{}, TO{}) with the input element type T (dtype) and output element
+// type TO (o_dtype) as type tags.
+template <class F>
+__host__ auto dispatch_types(int dtype, int o_dtype, F &&f) {
+  if (dtype == GDN_DTYPE_BF16) {
+    if (o_dtype == GDN_DTYPE_BF16) return f(__nv_bfloat16{}, __nv_bfloat16{});
+    return f(__nv_bfloat16{}, float{});
+  }
+  if (o_dtype == GDN_DTYPE_BF16) return f(float{}, __nv_bfloat16{});
+  return f(float{}, float{});
+}
+
+}  // namespace gdn

@@ -1,0 +1,169 @@
+/*
+ * gdn.h -- C ABI of libgdn.so: the Gated DeltaNet recurrence (gated delta
+ * rule) on NVIDIA B200 (sm_100a).
+ *
+ * The operation.  For every sequence and every value head h, with state
+ * S (Dv x Dk, fp32) and per-token decay alpha_t = exp(g_t) and write strength
+ * beta_t:
+ *
+ *     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = scale * S_t q_t
+ *
+ * Source: "Inside Qwen3.8-27B: Hybrid DeltaNet Architecture, 256k Context,
+ * and 24GB Local Serving", section "Gated DeltaNet Mechanics" (the delta rule
+ * subtracts the association stored under the normalized key k_t before
+ * writing the value v_t; S_t is a fixed-size d x d state; prefill uses a
+ * block-parallel chunked form, inference updates the state token by token).
+ * Head layout: "Qwen 3.8 27B Review: Native Vision, FP8 Quantization & 1M
+ * Context in a Compact Dense Model", section "3. Architecture: Gated DeltaNet
+ * Hybrid + FP8 Quantization" (16 query/key heads, 48 value heads, head dim
+ * 128).
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - State layout [num_seqs, Hv, Dv, Dk], fp32, row i = value dim i, Dk
+ *     contiguous.  Read u = S k, write v k^T, output S q.
+ *   - Value head h reads query/key head h / (Hv / Hqk) (contiguous groups);
+ *     Hv must be a multiple of Hqk.  No copies are made for the sharing.
+ *   - g (= log alpha, <= 0) and beta are fp32, one per (token, value head).
+ *   - o_t uses the state after token t.
+ *   - q and k are used as given (the caller normalises them).
+ *
+ * Memory.  Every pointer argument except those named "host" is a device
+ * pointer (cudaMalloc'd or equivalent) owned by the caller; the library never
+ * allocates, frees or keeps a pointer after a call returns.  All arrays are
+ * dense row-major with the shapes given below and 16-byte-aligned bases.
+ *
+ * Ordering.  Every call enqueues work on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and returns without synchronising, except
+ * gdn_get_device_status, which synchronises that stream.
+ *
+ * Errors.  Arguments are validated on the host before any launch; an invalid
+ * call returns a nonzero status and enqueues nothing.  A failed launch
+ * returns GDN_ERR_CUDA.  Conditions only the device can see (inconsistent
+ * cu_seqlens contents, a bounded wait that ran out) are recorded in the
+ * workspace status word; read them with gdn_get_device_status.  Nothing in
+ * the library aborts, traps or throws.
+ */
+#ifndef GDN_H_
+#define GDN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes (returned as int32_t). */
+#define GDN_OK 0
+#define GDN_ERR_INVALID_ARG 1    /* null / misaligned pointer, bad size or dtype        */
+#define GDN_ERR_UNSUPPORTED 2    /* valid but not implemented (head dims, dtype combo)  */
+#define GDN_ERR_CUDA 3           /* a CUDA runtime call or launch failed                */
+#define GDN_ERR_DEVICE_TIMEOUT 4 /* device status: a bounded wait inside a kernel ran out */
+#define GDN_ERR_BAD_SEQLENS 5    /* device status: cu_seqlens not 0 = c0 <= c1 .. <= cN = T */
+#define GDN_ERR_WORKSPACE 6      /* workspace missing, misaligned or too small           */
+
+/* Element types of q, k, v (dtype) and of o (o_dtype); g, beta and the state
+ * are always fp32.  o_dtype is chosen independently: fp32 o keeps the
+ * precision the fp32 state carries (rounding o to bf16 alone costs up to
+ * 2^-8 |o| per element). */
+#define GDN_DTYPE_BF16 0
+#define GDN_DTYPE_FP32 1
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *gdn_status_string(int32_t status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t gdn_version(void);
+
+/*
+ * Bytes of device workspace gdn_prefill needs for these sizes.  The
+ * workspace holds the device status word and the work scheduler's counters;
+ * it must stay allocated and unused by anything else until the call's work on
+ * the stream has finished.  Returns 0 for invalid sizes.
+ */
+size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t num_qk_heads,
+                                  int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
+                                  int32_t dtype);
+
+/*
+ * Prefill: run the recurrence over num_seqs packed sequences.
+ *
+ * The chunked (block-parallel) form: "Inside Qwen3.8-27B ...", section "Gated
+ * DeltaNet Mechanics" (the note that prefill is rewritten into a
+ * block-parallel form for tensor cores with the state kept on chip).  Chunks
+ * of 64 tokens aligned to each sequence's first token; the result equals the
+ * token-by-token definition up to rounding.
+ *
+ *   q, k           [T, Hqk, Dk]   dtype
+ *   v              [T, Hv, Dv]    dtype
+ *   g, beta        [T, Hv]        fp32  (g = log alpha; -inf allowed: alpha = 0)
+ *   cu_seqlens     [num_seqs + 1] int32, device; 0 = c_0 <= c_1 <= ... <= c_N = T.
+ *                  Sequence n is tokens [c_n, c_{n+1}); empty sequences are allowed
+ *                  (their final state equals their initial state).
+ *   initial_state  [num_seqs, Hv, Dv, Dk] fp32, or NULL for zeros.
+ *   final_state    [num_seqs, Hv, Dv, Dk] fp32, or NULL to skip.  May be the same
+ *                  pointer as initial_state (updated in place); no other overlap
+ *                  between arguments is allowed.
+ *   o              [T, Hv, Dv]    o_dtype (output)
+ *   scale          multiplies o (1.0 for o_t = S_t q_t)
+ *   workspace      device buffer of at least gdn_prefill_workspace_size(...) bytes,
+ *                  256-byte aligned, zero-filled once before its first use.  The
+ *                  kernels leave it zeroed apart from the status word, which is
+ *                  sticky: it keeps the first device-detected error until
+ *                  gdn_get_device_status reads and clears it.
+ *
+ * Supported: Hv % Hqk == 0; Dk, Dv in {64, 128}; dtype and o_dtype each bf16
+ * or fp32.  bf16 inputs with Dk = Dv = 128 run the tensor-core (tcgen05) kernel with bf16
+ * operands and fp32 accumulation; every other case runs the fp32 CUDA-core
+ * kernel.  T = 0 or num_seqs = 0 is a valid no-op apart from copying
+ * initial_state to final_state.
+ */
+int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
+                    const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
+                    int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
+                    int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, int32_t o_dtype,
+                    float scale, const float *initial_state, float *final_state, void *o,
+                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode step: one new token for each of `batch` sequences, updating their
+ * states in place ("Inside Qwen3.8-27B ...", section "Gated DeltaNet
+ * Mechanics": in inference the state is updated token by token).
+ *
+ *   q, k     [batch, Hqk, Dk]        dtype
+ *   v        [batch, Hv, Dv]         dtype
+ *   g, beta  [batch, Hv]             fp32
+ *   state    [batch, Hv, Dv, Dk]     fp32, read and overwritten in place
+ *   o        [batch, Hv, Dv]         o_dtype (output); must not overlap state
+ *
+ * Supported: Hv % Hqk == 0; Dk, Dv in {64, 128}; dtype and o_dtype each bf16
+ * or fp32.  Needs no workspace.  batch = 0 is a valid no-op.
+ */
+int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                        const float *beta, float *state, void *o, int32_t batch,
+                        int32_t num_qk_heads, int32_t num_v_heads, int32_t head_dim_k,
+                        int32_t head_dim_v, int32_t dtype, int32_t o_dtype, float scale,
+                        void *stream);
+
+/*
+ * 1 if gdn_prefill with these sizes and dtype runs the tensor-core (tcgen05)
+ * kernel, 0 if it runs the fp32 CUDA-core kernel or the arguments are invalid.
+ * Host only; touches no device.
+ */
+int32_t gdn_prefill_uses_tensor_cores(int32_t num_qk_heads, int32_t num_v_heads,
+                                      int32_t head_dim_k, int32_t head_dim_v, int32_t dtype);
+
+/*
+ * Synchronise `stream`, read the status word kept in `workspace` (the first
+ * device-detected error of the gdn_prefill calls that used it since it was
+ * last cleared, or GDN_OK), store it in *status_host (host pointer) and clear
+ * it.  Returns GDN_OK when the read itself worked.
+ */
+int32_t gdn_get_device_status(const void *workspace, void *stream, int32_t *status_host);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H_ */

@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+The library must load, export every function include/gdn.h declares, and
+reject invalid calls with the documented status before touching the device.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_deltanet_recurrence_rule_b200 import api
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gdn.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(gdn_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from gated_deltanet_recurrence_rule_b200 import build
+
+    build.build()
+    return api.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "gdn_prefill" in names and "gdn_decode_step" in names
+    for name in names:
+        assert hasattr(lib, name), f"libgdn.so does not export {name}"
+
+
+def test_status_strings(lib):
+    for code in range(0, 7):
+        assert api.status_string(code).startswith("GDN_")
+    assert api.status_string(999) == "GDN_ERR_UNKNOWN"
+    assert lib.gdn_version() >= 100
+
+
+def test_workspace_size(lib):
+    assert api.prefill_workspace_size(1, 8192, 16, 48, 128, 128) >= 256
+    assert lib.gdn_prefill_workspace_size(-1, 10, 16, 48, 128, 128, 0) == 0
+    assert lib.gdn_prefill_workspace_size(1, 10, 16, 40, 128, 128, 0) == 0  # 40 % 16 != 0
+    assert lib.gdn_prefill_workspace_size(1, 10, 16, 48, 128, 128, 7) == 0  # bad dtype
+
+
+def _prefill(lib, **kw):
+    a = dict(q=1 << 12, k=1 << 12, v=1 << 12, g=1 << 12, beta=1 << 12, cu=1 << 12, N=1, T=16,
+             Hqk=2, Hv=6, Dk=64, Dv=64, dtype=0, odt=1, scale=1.0, s0=None, sf=None, o=1 << 12,
+             ws=1 << 12, wsb=256)
+    a.update(kw)
+    return lib.gdn_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["T"],
+                           a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"], a["odt"], a["scale"], a["s0"],
+                           a["sf"], a["o"], a["ws"], a["wsb"], None)
+
+
+def test_prefill_validation(lib):
+    # every case is rejected on the host; the fake addresses are never dereferenced
+    assert _prefill(lib, q=None) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, cu=None) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, o=None) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, v=(1 << 12) + 8) == api.GDN_ERR_INVALID_ARG  # misaligned
+    assert _prefill(lib, Hv=5) == api.GDN_ERR_INVALID_ARG            # Hv % Hqk
+    assert _prefill(lib, Hqk=0) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, dtype=3) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, odt=2) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, T=-1) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, N=-1) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, Dk=96) == api.GDN_ERR_UNSUPPORTED
+    assert _prefill(lib, Dv=256) == api.GDN_ERR_UNSUPPORTED
+    assert _prefill(lib, ws=None) == api.GDN_ERR_WORKSPACE
+    assert _prefill(lib, ws=(1 << 12) + 16) == api.GDN_ERR_WORKSPACE
+    assert _prefill(lib, wsb=8) == api.GDN_ERR_WORKSPACE
+    assert _prefill(lib, N=0, T=5) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, N=0, T=0) == api.GDN_OK                    # nothing to do
+
+
+def _decode(lib, **kw):
+    a = dict(q=1 << 12, k=1 << 12, v=1 << 12, g=1 << 12, beta=1 << 12, S=1 << 12, o=1 << 12, B=2,
+             Hqk=16, Hv=48, Dk=128, Dv=128, dtype=0, odt=1, scale=1.0)
+    a.update(kw)
+    return lib.gdn_decode_step(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S"], a["o"], a["B"],
+                               a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"], a["odt"], a["scale"],
+                               None)
+
+
+def test_decode_validation(lib):
+    assert _decode(lib, S=None) == api.GDN_ERR_INVALID_ARG
+    assert _decode(lib, k=None) == api.GDN_ERR_INVALID_ARG
+    assert _decode(lib, o=(1 << 12) + 4) == api.GDN_ERR_INVALID_ARG
+    assert _decode(lib, Hv=47) == api.GDN_ERR_INVALID_ARG
+    assert _decode(lib, B=-3) == api.GDN_ERR_INVALID_ARG
+    assert _decode(lib, Dk=32) == api.GDN_ERR_UNSUPPORTED
+    assert _decode(lib, odt=-1) == api.GDN_ERR_INVALID_ARG
+    assert _decode(lib, B=0) == api.GDN_OK
+
+
+def test_device_status_validation(lib):
+    out = ctypes.c_int32(7)
+    assert lib.gdn_get_device_status(None, None, ctypes.byref(out)) == api.GDN_ERR_INVALID_ARG
+    assert lib.gdn_get_device_status(1 << 12, None, None) == api.GDN_ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+
+    x = torch.zeros(4, 1, 64)
+    with pytest.raises(ValueError):
+        api.prefill(x, x, x, torch.zeros(4, 1), torch.zeros(4, 1))

@@ -1,0 +1,150 @@
+"""Prefill on the GPU against the fp64 oracle (through the C ABI)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_recurrence_rule_b200 import api, inputs
+from parity import TOL, assert_parity, oracle_prefill_heads, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def run_gpu(inp, scale=1.0, alias=False, o_dtype=torch.float32):
+    dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
+    fin = dev["initial_state"] if alias else None
+    o, f = api.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                       cu_seqlens=dev["cu_seqlens"], initial_state=dev["initial_state"],
+                       final_state=fin, scale=scale, o_dtype=o_dtype)
+    torch.cuda.synchronize()
+    return o, f
+
+
+def run_oracle(inp, scale=1.0):
+    return oracle.prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                          cu_seqlens=inp["cu_seqlens"], initial_state=inp["initial_state"],
+                          scale=scale)
+
+
+def test_tiny_workload():
+    """T=256, Hqk=2, Hv=6, D=64, fp32, zero initial state, seed 0."""
+    inp = inputs.workload_inputs(inputs.WORKLOADS["tiny"])
+    o, f = run_gpu(inp)
+    o_ref, f_ref = run_oracle(inp)
+    assert_parity(torch.float32, to_np(o), o_ref, to_np(f), f_ref, "tiny")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_ragged_chunks(dtype, D):
+    """Several 64-token chunks plus a ragged tail, nonzero initial state."""
+    inp = inputs.prefill_inputs([300], 2, 6, D, dtype=dtype, seed=11, init_std=0.1)
+    o, f = run_gpu(inp, scale=0.75)
+    o_ref, f_ref = run_oracle(inp, scale=0.75)
+    assert_parity(inputs.DTYPES[dtype], to_np(o), o_ref, to_np(f), f_ref, f"{dtype} D={D}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_varlen_edges(dtype):
+    """Packed sequences of length 1, 63, 64, 65, 0, 130 and 200 with their own
+    initial states."""
+    lengths = [1, 63, 64, 65, 0, 130, 200]
+    inp = inputs.prefill_inputs(lengths, 2, 6, 128, dtype=dtype, seed=12, init_std=0.05)
+    o, f = run_gpu(inp)
+    o_ref, f_ref = run_oracle(inp)
+    assert_parity(inputs.DTYPES[dtype], to_np(o), o_ref, to_np(f), f_ref, "varlen")
+    # the empty sequence returns its initial state untouched
+    assert torch.equal(f[4].cpu(), inp["initial_state"][4])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_bf16_output(dtype):
+    """o stored in bf16: checked against the rounding-aware bound."""
+    inp = inputs.prefill_inputs([257, 64, 5], 2, 6, 128, dtype=dtype, seed=18, init_std=0.1)
+    o, f = run_gpu(inp, o_dtype=torch.bfloat16)
+    assert o.dtype == torch.bfloat16
+    o_ref, f_ref = run_oracle(inp)
+    assert_parity(inputs.DTYPES[dtype], to_np(o), o_ref, to_np(f), f_ref, "bf16 o", o_bf16=True)
+
+
+def test_in_place_state():
+    """final_state may be the initial_state buffer (updated in place)."""
+    inp = inputs.prefill_inputs([129, 70], 2, 6, 128, dtype="bf16", seed=13, init_std=0.1)
+    o, f = run_gpu(inp, alias=True)
+    o_ref, f_ref = run_oracle(inp)
+    assert_parity(torch.bfloat16, to_np(o), o_ref, to_np(f), f_ref, "aliased state")
+
+
+def test_zero_tokens_copies_state():
+    inp = inputs.prefill_inputs([0, 0], 2, 6, 64, dtype="bf16", seed=14, init_std=0.1)
+    o, f = run_gpu(inp)
+    assert o.shape[0] == 0
+    assert torch.equal(f.cpu(), inp["initial_state"])
+
+
+def test_reset_and_no_write_edges():
+    """alpha = 0 on some tokens (state reset) and beta = 0 on others."""
+    inp = inputs.prefill_inputs([200], 2, 6, 128, dtype="fp32", seed=15, init_std=0.1)
+    inp["g"][[3, 64, 150]] = -float("inf")
+    inp["beta"][[10, 11, 70]] = 0.0
+    o, f = run_gpu(inp)
+    o_ref, f_ref = run_oracle(inp)
+    assert_parity(torch.float32, to_np(o), o_ref, to_np(f), f_ref, "edges")
+
+
+def test_bad_cu_seqlens_sets_device_status():
+    inp = inputs.prefill_inputs([64, 64], 2, 6, 64, dtype="bf16", seed=16)
+    dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
+    ws = torch.zeros(api.prefill_workspace_size(2, 128, 2, 6, 64, 64), dtype=torch.uint8, device=DEV)
+    bad = torch.tensor([0, 100, 90], dtype=torch.int32, device=DEV)  # decreasing
+    api.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu_seqlens=bad, workspace=ws)
+    assert api.get_device_status(ws) == api.GDN_ERR_BAD_SEQLENS
+    api.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], cu_seqlens=dev["cu_seqlens"],
+                workspace=ws)
+    assert api.get_device_status(ws) == api.GDN_OK
+
+
+def test_guard_bands_and_determinism():
+    inp = inputs.prefill_inputs([190, 3], 2, 6, 128, dtype="bf16", seed=17, init_std=0.1)
+    dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
+    T, pad = 193, 8192
+    obuf = torch.full((T * 6 * 128 + 2 * pad,), 3.0, dtype=torch.bfloat16, device=DEV)
+    o = obuf[pad:pad + T * 6 * 128].view(T, 6, 128)
+    sbuf = torch.full((2 * 6 * 128 * 128 + 2 * pad,), float("nan"), device=DEV)
+    f = sbuf[pad:pad + 2 * 6 * 128 * 128].view(2, 6, 128, 128)
+    outs = []
+    for _ in range(2):
+        api.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                    cu_seqlens=dev["cu_seqlens"], initial_state=dev["initial_state"],
+                    final_state=f, o=o)
+        torch.cuda.synchronize()
+        outs.append((o.clone(), f.clone()))
+    assert (obuf[:pad] == 3).all() and (obuf[-pad:] == 3).all()
+    assert torch.isnan(sbuf[:pad]).all() and torch.isnan(sbuf[-pad:]).all()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def _sampled_workload(name, qk_heads):
+    w = inputs.WORKLOADS[name]
+    inp = inputs.workload_inputs(w)
+    o, f = run_gpu(inp)
+    o_ref, f_ref, vh = oracle_prefill_heads(inp, qk_heads, w.Hv // w.Hqk)
+    assert_parity(torch.bfloat16, to_np(o[:, vh]), o_ref, to_np(f[:, vh]), f_ref, name)
+
+
+def test_prefill8k_sampled_heads():
+    """T=8192, 16/48 heads, D=128, bf16; oracle on QK heads 0 and 15."""
+    _sampled_workload("prefill8k", [0, 15])
+
+
+@pytest.mark.slow
+def test_long262k_sampled_heads():
+    """T=262,144, slow decay, nonzero initial state; oracle on QK head 9."""
+    _sampled_workload("long262k", [9])
+
+
+@pytest.mark.slow
+def test_varlen32_sampled_heads():
+    """32 packed sequences of 1024..32768 tokens; oracle on QK head 4."""
+    _sampled_workload("varlen32", [4])

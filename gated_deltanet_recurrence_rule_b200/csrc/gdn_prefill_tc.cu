@@ -1,15 +1,709 @@
-// gdn_prefill_tc.cu -- tensor-core (tcgen05) chunked prefill.  Not built yet:
-// every prefill call takes the CUDA-core kernel.
+// gdn_prefill_tc.cu -- chunked prefill of the gated delta rule on the
+// Blackwell tensor cores (tcgen05 + TMEM + TMA), bf16 operands, fp32 state.
+//
+// The recurrence ("Inside Qwen3.8-27B: Hybrid DeltaNet Architecture, 256k
+// Context, and 24GB Local Serving", section "Gated DeltaNet Mechanics"; the
+// note there says prefill is rewritten into a block-parallel form for tensor
+// cores while the state stays on chip):
+//     S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,  o_t = S_t q_t.
+// Chunked form for a chunk of C = 64 tokens with start state S0 (Dv x Dk),
+// local log-decay prefix sums G_t and w_t = beta_t (v_t - alpha_t S_{t-1} k_t):
+//     A_ts = beta_t e^{G_t - G_s} (k_t . k_s)   (s < t),   Tm = (I + A)^-1
+//     W  = Tm diag(beta e^G) K,   U~ = Tm diag(beta) V,   U = U~ - W S0^T
+//     O  = diag(e^G) Q S0^T + (e^{G_t - G_s} (q_t . k_s))_{s<=t} U
+//     S  = e^{G_C} S0 + U^T diag(e^{G_C - G}) K
+// Every product is computed transposed so that the 128-wide head dimension is
+// the MMA's M (full-rate 128-lane tcgen05 tiles):
+//     [Q;K] K^T        (M128 N64 K128)  -> QK^T and KK^T (exact bf16 inputs)
+//     W^T  = K^T T'^T  (M128 N64 K64),  T'  = Tm diag(beta e^G)
+//     U~^T = V^T T''^T (M128 N64 K64),  T'' = Tm diag(beta)
+//     U^T  = U~^T - S0 W^T                   (accumulated with negated A)
+//     Oi^T = S0 Q^T,   Oa^T = U^T P^T,   o_t = e^{G_t} Oi_t + Oa_t
+//     dS   = (U diag(e^{G_C - G}))^T K,   S <- e^{G_C} S + dS  (fp32 master copy)
+// Precision.  Rounding every operand to bf16 costs about 5e-2 RMS(o) in the
+// largest output errors (the 1e-2 RMS bound needs ~11 significant bits at the
+// largest outputs).  So the operands that carry computed values are split
+// into two bf16 terms, x = hi + lo with hi = bf16(x), lo = bf16(x - hi):
+// T' and T'' (2 MMAs each), S0 in the output product (2 MMAs), U and P in
+// U^T P^T (hi*hi + lo*hi + hi*lo), and U diag(e^{G_C-G}) in dS (2 MMAs).  Q,
+// K, V are exact bf16 inputs; decays are applied in fp32 (e^{G_t} on the
+// output accumulator, e^{G_C-G_t} folded into U before the split).  S0 in
+// U = U~ - W S0^T and W itself stay single bf16 (their rounding costs ~1e-3).
+// The 64x64 unit lower-triangular inverse Tm is computed in fp32 on CUDA
+// cores (16x16 diagonal blocks by forward substitution, then block rows).
+//
+// One CTA per (sequence, value head); 384 threads:
+//   warp 0      TMA producer (Q/K ring of 2, V buffer of 1, L2 prefetch ahead)
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 2      per-chunk scalars (prefix sums of g, decays, masked beta)
+//   warp 3      idle
+//   warps 4-11  256 epilogue threads: TMEM -> registers -> SMEM operands,
+//               the triangular solve, the fp32 state and the outputs.
+// Chunks run one after another (this version does not overlap the next
+// chunk's state-independent work with the current chunk's state chain).
+// Every wait is bounded; a wait that runs out sets GDN_ERR_DEVICE_TIMEOUT in
+// the workspace status word and every role leaves its loop.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "gdn_common.cuh"
+#include "gdn_sm100.cuh"
 
 namespace gdn {
+namespace tc {
 
-bool prefill_tc_supported(int, int, int, int, int) { return false; }
+using namespace sm100;
 
-cudaError_t launch_prefill_tc(const void *, const void *, const void *, const float *,
-                              const float *, const int32_t *, int, long long, int, int, int, float,
-                              const float *, float *, void *, void *, cudaStream_t) {
-  return cudaErrorNotSupported;
+constexpr int CH = 64;            // chunk length
+constexpr int HD = 128;           // head dim (Dk = Dv)
+constexpr int NTHREADS = 384;
+constexpr int NEPI = 256;         // epilogue threads
+constexpr int EPI_BAR = 1;        // named barrier id of the epilogue threads
+constexpr float LOG2E = 1.4426950408889634f;
+// alpha below e^-30 is treated as e^-30: the chunk prefix sums stay finite
+// (exp(-inf - -inf) is undefined) and e^-30 ~ 1e-13 is below fp32 resolution.
+constexpr float G_FLOOR = -30.f;
+
+// ---- shared memory map (bytes); swizzled tiles are 1024-byte aligned ----
+constexpr uint32_t QK_STAGE = 32768;   // [Q d0-63 | K d0-63 | Q d64-127 | K d64-127], 64 rows x 128 B each
+constexpr uint32_t V_STAGE = 16384;    // [V d0-63 | V d64-127]
+constexpr uint32_t OFF_QK = 0;         // 2 stages
+constexpr uint32_t OFF_V = 65536;      // 1 stage
+constexpr uint32_t OFF_S0H = 81920;    // bf16 hi(S0), K-major: 2 x (128 rows x 128 B)
+constexpr uint32_t OFF_S0L = 114688;   // bf16 lo(S0)
+// R1: one 64 KB region reused by phases of a chunk that never overlap:
+//   solve:   A fp32 [64][68] @0, Tm fp32 [64][68] @32K, Y fp32 [3][16][17] @50176
+//   W, U~:   T' hi @0, T' lo @8K, T'' hi @16K, T'' lo @24K (Tm still read)
+//   S0 W^T:  W^T bf16 MN-major (128 rows d x 64 t) @0
+//   U:       U hi @0, U lo @16K, Ukdec hi @32K, Ukdec lo @48K (K-major, 128 rows x 64 t)
+constexpr uint32_t OFF_R1 = 147456;
+constexpr uint32_t OFF_A = OFF_R1;
+constexpr uint32_t OFF_TM = OFF_R1 + 32768;
+constexpr uint32_t OFF_Y = OFF_R1 + 50176;
+constexpr uint32_t OFF_TPH = OFF_R1, OFF_TPL = OFF_R1 + 8192;
+constexpr uint32_t OFF_TQH = OFF_R1 + 16384, OFF_TQL = OFF_R1 + 24576;
+constexpr uint32_t OFF_WT = OFF_R1;
+constexpr uint32_t OFF_UH = OFF_R1, OFF_UL = OFF_R1 + 16384;
+constexpr uint32_t OFF_UKH = OFF_R1 + 32768, OFF_UKL = OFF_R1 + 49152;
+constexpr uint32_t OFF_PH = OFF_R1 + 65536;  // bf16 hi(P), K-major B: 64 rows (t) x 64 s
+constexpr uint32_t OFF_PL = OFF_PH + 8192;   // bf16 lo(P)
+constexpr uint32_t OFF_SCAL = OFF_PL + 8192;
+constexpr uint32_t SCAL_STAGE = 5 * 64 * 4;  // G2 (log2 prefix), gamma, kdec, beta; gamma_C at [256]
+constexpr uint32_t OFF_BAR = OFF_SCAL + 2 * SCAL_STAGE;
+constexpr uint32_t OFF_MISC = OFF_BAR + 192;  // [0] TMEM base, [4] abort flag, [8] drain mbarrier
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+constexpr int AST = 68;  // fp32 row stride of A and Tm (conflict-free float4 row stores)
+static_assert(OFF_R1 % 1024 == 0 && OFF_PH % 1024 == 0 && OFF_S0H % 1024 == 0, "alignment");
+static_assert(OFF_Y + 3 * 16 * 17 * 4 <= OFF_R1 + 65536, "R1 layout");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// ---- TMEM columns (fp32 accumulators, 128 lanes) ----
+constexpr uint32_t R_QK = 0;    // 64: rows 0-63 = Q K^T, rows 64-127 = K K^T
+constexpr uint32_t R_W = 64;    // 64: W^T
+constexpr uint32_t R_U = 128;   // 64: U~^T, then U^T
+constexpr uint32_t R_S = 192;   // 128: dS
+constexpr uint32_t R_OI = 320;  // 64: S0 Q^T
+constexpr uint32_t R_OA = 384;  // 64: U^T P^T
+constexpr uint32_t TMEM_COLS = 512;
+
+// ---- mbarriers ----
+enum {
+  B_FULL_QK = 0, B_EMPTY_QK = 2, B_FULL_V = 4, B_EMPTY_V = 5, B_SCAL_FULL = 6, B_SCAL_EMPTY = 8,
+  B_QK = 10, B_T = 11, B_W = 12, B_WT = 13, B_U = 14, B_UT = 15, B_S = 16, B_DONE = 17, NBAR = 18
+};
+static_assert(NBAR * 8 <= 192, "barrier area");
+
+constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, 0, 0);      // [Q;K] K^T
+constexpr uint32_t IDESC_WY = idesc_bf16(128, 64, 1, 0);      // K^T T'^T, V^T T''^T
+constexpr uint32_t IDESC_SW = idesc_bf16(128, 64, 0, 1, 1);   // -S0 W^T
+constexpr uint32_t IDESC_SQ = idesc_bf16(128, 64, 0, 0);      // S0 Q^T, U^T P^T
+constexpr uint32_t IDESC_UK = idesc_bf16(128, 128, 0, 1);     // Ukdec^T K
+
+struct Params {
+  const float *g, *beta;
+  const int32_t *cu;
+  int N, T, Hqk, Hv;
+  float scale;
+  const float *s0;
+  float *sfin;
+  void *o;
+  int32_t *status;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t sb, int i) { return sb + OFF_BAR + 8u * i; }
+
+// Unit lower-triangular inverse Tm = (I + A)^-1 of a 64x64 strictly lower A,
+// fp32, by the 256 epilogue threads.  Diagonal 16x16 blocks by forward
+// substitution (one warp per block, two lanes per column), then block rows
+// i = 1..3: Y_ij = sum_{j<=k<i} A_ik Tm_kj and Tm_ij = -Tm_ii Y_ij.
+__device__ __forceinline__ void ut_solve(const float *A, float *Tm, float *Y, int etid) {
+  const int ew = etid >> 5, lane = etid & 31;
+  if (ew < 4) {
+    const int b = ew, c = lane >> 1, hh = lane & 1;
+    float x[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) x[m] = (2 * m + hh == c) ? 1.f : 0.f;
+#pragma unroll
+    for (int s = 0; s < 16; ++s) {
+      const float xs = __shfl_sync(0xffffffffu, x[s >> 1], (c << 1) | (s & 1));
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        const int r = 2 * m + hh;
+        if (r > s) x[m] = fmaf(-A[(16 * b + r) * AST + 16 * b + s], xs, x[m]);
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 8; ++m) Tm[(16 * b + 2 * m + hh) * AST + 16 * b + c] = x[m];
+  }
+  named_bar_sync(EPI_BAR, NEPI);
+#pragma unroll
+  for (int i = 1; i < 4; ++i) {
+    for (int e = etid; e < i * 256; e += NEPI) {
+      const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+      float acc = 0.f;
+      const float *arow = A + (16 * i + r) * AST;
+      for (int q = 16 * j; q < 16 * i; q += 4) {
+        const float4 a4 = *reinterpret_cast<const float4 *>(arow + q);
+        acc = fmaf(a4.x, Tm[(q + 0) * AST + 16 * j + cc], acc);
+        acc = fmaf(a4.y, Tm[(q + 1) * AST + 16 * j + cc], acc);
+        acc = fmaf(a4.z, Tm[(q + 2) * AST + 16 * j + cc], acc);
+        acc = fmaf(a4.w, Tm[(q + 3) * AST + 16 * j + cc], acc);
+      }
+      Y[(j * 16 + r) * 17 + cc] = acc;
+    }
+    named_bar_sync(EPI_BAR, NEPI);
+    for (int e = etid; e < i * 256; e += NEPI) {
+      const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
+      const float *trow = Tm + (16 * i + r) * AST + 16 * i;
+      float acc = 0.f;
+#pragma unroll
+      for (int m = 0; m < 16; m += 4) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(trow + m);
+        acc = fmaf(t4.x, Y[(j * 16 + m + 0) * 17 + cc], acc);
+        acc = fmaf(t4.y, Y[(j * 16 + m + 1) * 17 + cc], acc);
+        acc = fmaf(t4.z, Y[(j * 16 + m + 2) * 17 + cc], acc);
+        acc = fmaf(t4.w, Y[(j * 16 + m + 3) * 17 + cc], acc);
+      }
+      Tm[(16 * i + r) * AST + 16 * j + cc] = -acc;
+    }
+    named_bar_sync(EPI_BAR, NEPI);
+  }
+}
+
+// One waiter (epilogue thread 0) for an mbarrier phase, then a named barrier;
+// returns false on abort (then every epilogue thread returns false).
+__device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, int etid,
+                                         volatile int *abort, int32_t *status) {
+  if (etid == 0) {
+    if (!mbar_wait(bar, parity, abort)) {
+      *abort = 1;
+      report_status(status, GDN_ERR_DEVICE_TIMEOUT);
+    }
+  }
+  named_bar_sync(EPI_BAR, NEPI);
+  const bool ok = (*abort == 0);
+  if (ok) tc_fence_after();
+  return ok;
+}
+
+// 8 consecutive fp32 values -> one 16-byte chunk of bf16 at `dst`.
+__device__ __forceinline__ void st_bf16x8(unsigned char *dst, const float *x) {
+  *reinterpret_cast<uint4 *>(dst) = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
+                                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
+}
+// 8 fp32 values x -> hi = bf16(x) at dst_hi and lo = bf16(x - hi) at dst_lo.
+__device__ __forceinline__ void st_split8(unsigned char *dst_hi, unsigned char *dst_lo,
+                                          const float *x) {
+  uint32_t hw[4], lw[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
+    const __nv_bfloat162 hh = __halves2bfloat162(h0, h1);
+    hw[e] = *reinterpret_cast<const uint32_t *>(&hh);
+    lw[e] = pack_bf16x2(x[2 * e] - __bfloat162float(h0), x[2 * e + 1] - __bfloat162float(h1));
+  }
+  *reinterpret_cast<uint4 *>(dst_hi) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+  *reinterpret_cast<uint4 *>(dst_lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+template <typename TO>
+__global__ void __launch_bounds__(NTHREADS, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n = blockIdx.x / p.Hv, h = blockIdx.x - n * p.Hv;
+  const int j = h / (p.Hv / p.Hqk);
+  const size_t sbase = ((size_t)n * p.Hv + h) * HD * HD;
+
+  const int c0 = p.cu[n], c1 = p.cu[n + 1];
+  if (c0 < 0 || c1 < c0 || c1 > p.T || (n == 0 && c0 != 0) || (n == p.N - 1 && c1 != p.T)) {
+    if (tid == 0) report_status(p.status, GDN_ERR_BAD_SEQLENS);
+    return;
+  }
+  const int L = c1 - c0;
+  const int nch = (L + CH - 1) / CH;
+  if (nch == 0) {  // empty sequence: final state = initial state
+    if (p.sfin)
+      for (int x = tid; x < HD * HD; x += NTHREADS) p.sfin[sbase + x] = p.s0 ? p.s0[sbase + x] : 0.f;
+    return;
+  }
+
+  const uint32_t sb = smem_addr(smem);
+  if (sb & 1023u) {  // swizzled operand tiles need 1024-byte alignment
+    if (tid == 0) report_status(p.status, GDN_ERR_UNSUPPORTED);
+    return;
+  }
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  if (tid == 0) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + OFF_MISC, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      prefetch_tensormap(&tm_v);
+      constexpr int PF = 4;  // L2 prefetch distance in chunks
+      for (int c = 0; c < PF && c < nch; ++c) {
+        const int t = c0 + c * CH;
+        tma_prefetch_3d(&tm_q, 0, j, t); tma_prefetch_3d(&tm_q, 64, j, t);
+        tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
+        tma_prefetch_3d(&tm_v, 0, h, t); tma_prefetch_3d(&tm_v, 64, h, t);
+      }
+      int issued_qk = 0, issued_v = 0;  // chunks whose loads were issued
+      for (int c = 0; c < nch; ++c) {
+        const int s = c & 1;
+        const int t0 = c0 + c * CH;
+        if (c + PF < nch) {
+          const int t = t0 + PF * CH;
+          tma_prefetch_3d(&tm_q, 0, j, t); tma_prefetch_3d(&tm_q, 64, j, t);
+          tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
+          tma_prefetch_3d(&tm_v, 0, h, t); tma_prefetch_3d(&tm_v, 64, h, t);
+        }
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c >> 1) & 1) ^ 1, abort_flag)) break;
+        const uint32_t st = sb + OFF_QK + s * QK_STAGE;
+        const uint32_t fb = bar_addr(sb, B_FULL_QK + s);
+        mbar_arrive_expect_tx(fb, QK_STAGE);
+        tma_load_3d(st + 0, &tm_q, fb, 0, j, t0);
+        tma_load_3d(st + 16384, &tm_q, fb, 64, j, t0);
+        tma_load_3d(st + 8192, &tm_k, fb, 0, j, t0);
+        tma_load_3d(st + 24576, &tm_k, fb, 64, j, t0);
+        issued_qk = c + 1;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_V), (c & 1) ^ 1, abort_flag)) break;
+        const uint32_t fv = bar_addr(sb, B_FULL_V);
+        mbar_arrive_expect_tx(fv, V_STAGE);
+        tma_load_3d(sb + OFF_V + 0, &tm_v, fv, 0, h, t0);
+        tma_load_3d(sb + OFF_V + 8192, &tm_v, fv, 64, h, t0);
+        issued_v = c + 1;
+      }
+      if (issued_qk < nch || issued_v < nch) {
+        *abort_flag = 1;
+        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+      }
+      // Let every load this thread issued land before the CTA can exit (each
+      // buffer's latest fill; earlier fills were consumed before it was issued).
+      for (int c = max(issued_qk - 2, 0); c < issued_qk; ++c)
+        mbar_wait(bar_addr(sb, B_FULL_QK + (c & 1)), (c >> 1) & 1, abort_flag, 50000000ull);
+      if (issued_v > 0)
+        mbar_wait(bar_addr(sb, B_FULL_V), (issued_v - 1) & 1, abort_flag, 50000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int s = c & 1;
+        const uint32_t ph2 = (c >> 1) & 1, ph = c & 1;
+        const uint32_t st = sb + OFF_QK + s * QK_STAGE;
+        // [Q;K] K^T
+        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), ph2, abort_flag);
+        if (ok && c > 0) ok = mbar_wait(bar_addr(sb, B_DONE), (c - 1) & 1, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16(tmem + R_QK, sdesc_sw128(st + koff, 16, 1024),
+                   sdesc_sw128(st + 8192 + koff, 16, 1024), IDESC_QK, ks > 0);
+        }
+        mma_commit(bar_addr(sb, B_QK));
+        // W^T = K^T (T'h + T'l)^T ;  U~^T = V^T (T''h + T''l)^T
+        ok = mbar_wait(bar_addr(sb, B_T), ph, abort_flag) &&
+             mbar_wait(bar_addr(sb, B_FULL_V), ph, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t bo = ((ks & 1) ? OFF_TPL : OFF_TPH) + (ks >> 1) * 32;
+          mma_bf16(tmem + R_W, sdesc_sw128(st + 8192 + (ks >> 1) * 2048, 16384, 1024),
+                   sdesc_sw128(sb + bo, 16, 1024), IDESC_WY, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t bo = ((ks & 1) ? OFF_TQL : OFF_TQH) + (ks >> 1) * 32;
+          mma_bf16(tmem + R_U, sdesc_sw128(sb + OFF_V + (ks >> 1) * 2048, 8192, 1024),
+                   sdesc_sw128(sb + bo, 16, 1024), IDESC_WY, ks > 0);
+        }
+        mma_commit(bar_addr(sb, B_W));
+        mma_commit(bar_addr(sb, B_EMPTY_V));
+        // U^T = U~^T - S0h W^T ;  Oi^T = (S0h + S0l) Q^T
+        ok = mbar_wait(bar_addr(sb, B_WT), ph, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
+          mma_bf16(tmem + R_U, sdesc_sw128(sb + OFF_S0H + koff, 16, 1024),
+                   sdesc_sw128(sb + OFF_WT + ks * 2048, 8192, 1024), IDESC_SW, 1);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks) {
+          const uint32_t koff = ((ks >> 1) >> 2) * 16384 + ((ks >> 1) & 3) * 32;
+          const uint32_t ao = (ks & 1) ? OFF_S0L : OFF_S0H;
+          mma_bf16(tmem + R_OI, sdesc_sw128(sb + ao + koff, 16, 1024),
+                   sdesc_sw128(st + koff, 16, 1024), IDESC_SQ, ks > 0);
+        }
+        mma_commit(bar_addr(sb, B_U));
+        // dS = (Ukh + Ukl)^T K ;  Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T
+        ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t ao = ((ks & 1) ? OFF_UKL : OFF_UKH) + (ks >> 1) * 32;
+          mma_bf16(tmem + R_S, sdesc_sw128(sb + ao, 16, 1024),
+                   sdesc_sw128(st + 8192 + (ks >> 1) * 2048, 16384, 1024), IDESC_UK, ks > 0);
+        }
+#pragma unroll
+        for (int ks = 0; ks < 12; ++ks) {
+          const int part = ks % 3, kk = ks / 3;  // (Uh,Ph), (Ul,Ph), (Uh,Pl)
+          const uint32_t ao = (part == 1 ? OFF_UL : OFF_UH) + kk * 32;
+          const uint32_t bo = (part == 2 ? OFF_PL : OFF_PH) + kk * 32;
+          mma_bf16(tmem + R_OA, sdesc_sw128(sb + ao, 16, 1024), sdesc_sw128(sb + bo, 16, 1024),
+                   IDESC_SQ, ks > 0);
+        }
+        mma_commit(bar_addr(sb, B_S));
+        mma_commit(bar_addr(sb, B_EMPTY_QK + s));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+      }
+      // Drain: every MMA this thread issued finishes before TMEM is freed.
+      const uint32_t drain = sb + OFF_MISC + 8;
+      mbar_init(drain, 1);
+      fence_barrier_init();
+      mma_commit(drain);
+      mbar_wait(drain, 0, abort_flag, 50000000ull);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ chunk scalars
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(bar_addr(sb, B_SCAL_EMPTY + s), ((c >> 1) & 1) ^ 1, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) { *abort_flag = 1; report_status(p.status, GDN_ERR_DEVICE_TIMEOUT); }
+        break;
+      }
+      const int t0 = c0 + c * CH;
+      const int Lc = min(CH, c1 - t0);
+      float ga = 0.f, gb = 0.f, ba = 0.f, bb = 0.f;
+      if (lane < Lc) {
+        ga = fmaxf(p.g[(size_t)(t0 + lane) * p.Hv + h], G_FLOOR);
+        ba = p.beta[(size_t)(t0 + lane) * p.Hv + h];
+      }
+      if (lane + 32 < Lc) {
+        gb = fmaxf(p.g[(size_t)(t0 + lane + 32) * p.Hv + h], G_FLOOR);
+        bb = p.beta[(size_t)(t0 + lane + 32) * p.Hv + h];
+      }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float xa = __shfl_up_sync(0xffffffffu, ga, off);
+        const float xb = __shfl_up_sync(0xffffffffu, gb, off);
+        if (lane >= off) { ga += xa; gb += xb; }
+      }
+      gb += __shfl_sync(0xffffffffu, ga, 31);
+      const float Ga = ga * LOG2E, Gb = gb * LOG2E;  // log2 of the decay prefix
+      const int last = Lc - 1;
+      const float GL = last < 32 ? __shfl_sync(0xffffffffu, Ga, last & 31)
+                                 : __shfl_sync(0xffffffffu, Gb, last & 31);
+      float *sc = reinterpret_cast<float *>(smem + OFF_SCAL + s * SCAL_STAGE);
+      sc[lane] = Ga;                 sc[lane + 32] = Gb;
+      sc[64 + lane] = exp2f(Ga);     sc[64 + lane + 32] = exp2f(Gb);
+      sc[128 + lane] = lane < Lc ? exp2f(GL - Ga) : 0.f;
+      sc[128 + lane + 32] = lane + 32 < Lc ? exp2f(GL - Gb) : 0.f;
+      sc[192 + lane] = ba;           sc[192 + lane + 32] = bb;
+      if (lane == 0) sc[256] = exp2f(GL);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(sb, B_SCAL_FULL + s));
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int etid = tid - 128;
+    const int ewg = etid >> 7;         // column half
+    const int row = etid & 127;        // TMEM lane = row of the 128-row tiles
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    float *A = reinterpret_cast<float *>(smem + OFF_A);
+    float *Tm = reinterpret_cast<float *>(smem + OFF_TM);
+    float *Y = reinterpret_cast<float *>(smem + OFF_Y);
+
+    // fp32 master state: row `row`, columns [64 ewg, 64 ewg + 64); S0 = hi + lo in SMEM
+    float S[64];
+    {
+      const float *src = p.s0 ? p.s0 + sbase + (size_t)row * HD + 64 * ewg : nullptr;
+#pragma unroll
+      for (int x = 0; x < 64; x += 4) {
+        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (src) v4 = *reinterpret_cast<const float4 *>(src + x);
+        S[x] = v4.x; S[x + 1] = v4.y; S[x + 2] = v4.z; S[x + 3] = v4.w;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint32_t off = ewg * 16384 + sw128_off(row, q);
+        st_split8(smem + OFF_S0H + off, smem + OFF_S0L + off, S + 8 * q);
+      }
+      fence_proxy_async_smem();
+    }
+
+    for (int c = 0; c < nch; ++c) {
+      const int s = c & 1;
+      const uint32_t ph = c & 1;
+      const int t0 = c0 + c * CH;
+      const int Lc = min(CH, c1 - t0);
+      const float *sc = reinterpret_cast<const float *>(smem + OFF_SCAL + s * SCAL_STAGE);
+      const float *G2 = sc, *gam = sc + 64, *kdec = sc + 128, *bet = sc + 192;
+
+      // ---- Q K^T and K K^T -> P (hi/lo) and A (fp32)
+      if (etid == 0) {
+        if (!mbar_wait(bar_addr(sb, B_SCAL_FULL + s), (c >> 1) & 1, abort_flag)) {
+          *abort_flag = 1;
+          report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+        }
+      }
+      if (!epi_wait(bar_addr(sb, B_QK), ph, etid, abort_flag, p.status)) break;
+      {
+        float v[32];
+        tmem_ld32(tl + R_QK + 32 * ewg, v);
+        tmem_wait_ld();
+        if (row < 64) {
+          const int t = row;
+          const float Gt = G2[t];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float pv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int si = 32 * ewg + 8 * q + e;
+              pv[e] = (si <= t && t < Lc) ? exp2f(Gt - G2[si]) * v[8 * q + e] : 0.f;
+            }
+            const uint32_t off = sw128_off(t, 4 * ewg + q);
+            st_split8(smem + OFF_PH + off, smem + OFF_PL + off, pv);
+          }
+        } else {
+          const int t = row - 64;
+          const float Gt = G2[t], bt = bet[t];
+          float *arow = A + t * AST + 32 * ewg;
+#pragma unroll
+          for (int x = 0; x < 32; x += 4) {
+            float a[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int si = 32 * ewg + x + e;
+              a[e] = (si < t && t < Lc) ? bt * exp2f(Gt - G2[si]) * v[x + e] : 0.f;
+            }
+            *reinterpret_cast<float4 *>(arow + x) = make_float4(a[0], a[1], a[2], a[3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      named_bar_sync(EPI_BAR, NEPI);
+
+      // ---- Tm = (I + A)^-1, then T' = Tm diag(beta gamma), T'' = Tm diag(beta), split
+      ut_solve(A, Tm, Y, etid);
+      {
+        const int t = etid >> 2, qq = etid & 3;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const int sbeg = 16 * qq + 8 * hf;
+          float tp[8], tq[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int si = sbeg + e;
+            const float m = (si <= t) ? Tm[t * AST + si] : 0.f;
+            tq[e] = m * bet[si];
+            tp[e] = tq[e] * gam[si];
+          }
+          const uint32_t off = sw128_off(t, sbeg >> 3);
+          st_split8(smem + OFF_TPH + off, smem + OFF_TPL + off, tp);
+          st_split8(smem + OFF_TQH + off, smem + OFF_TQL + off, tq);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_T));
+
+      // ---- W^T -> bf16 (MN-major B)
+      if (!epi_wait(bar_addr(sb, B_W), ph, etid, abort_flag, p.status)) break;
+      {
+        float v[32];
+        tmem_ld32(tl + R_W + 32 * ewg, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) st_bf16x8(smem + OFF_WT + sw128_off(row, 4 * ewg + q), v + 8 * q);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_WT));
+
+      // ---- U^T -> hi/lo (for P) and U^T diag(kdec) -> hi/lo (for the state)
+      if (!epi_wait(bar_addr(sb, B_U), ph, etid, abort_flag, p.status)) break;
+      {
+        float v[32];
+        tmem_ld32(tl + R_U + 32 * ewg, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t off = sw128_off(row, 4 * ewg + q);
+          st_split8(smem + OFF_UH + off, smem + OFF_UL + off, v + 8 * q);
+          float uk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) uk[e] = v[8 * q + e] * kdec[32 * ewg + 8 * q + e];
+          st_split8(smem + OFF_UKH + off, smem + OFF_UKL + off, uk);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_UT));
+
+      // ---- state: S = gamma_C S + dS (fp32), S0 <- hi/lo(S); outputs
+      if (!epi_wait(bar_addr(sb, B_S), ph, etid, abort_flag, p.status)) break;
+      {
+        const float gC = sc[256];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          float v[32];
+          tmem_ld32(tl + R_S + 64 * ewg + 32 * hf, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) S[32 * hf + x] = fmaf(gC, S[32 * hf + x], v[x]);
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint32_t off = ewg * 16384 + sw128_off(row, q);
+          st_split8(smem + OFF_S0H + off, smem + OFF_S0L + off, S + 8 * q);
+        }
+        float vi[32], va[32];
+        tmem_ld32(tl + R_OI + 32 * ewg, vi);
+        tmem_ld32(tl + R_OA + 32 * ewg, va);
+        tmem_wait_ld();
+        TO *op = static_cast<TO *>(p.o) + ((size_t)t0 * p.Hv + h) * HD + row;
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          const int t = 32 * ewg + x;
+          if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(p.scale * fmaf(gam[t], vi[x], va[x]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) {
+        mbar_arrive(bar_addr(sb, B_DONE));
+        mbar_arrive(bar_addr(sb, B_SCAL_EMPTY + s));
+      }
+    }
+    if (*abort_flag == 0 && p.sfin) {
+      float *dst = p.sfin + sbase + (size_t)row * HD + 64 * ewg;
+#pragma unroll
+      for (int x = 0; x < 64; x += 4)
+        *reinterpret_cast<float4 *>(dst + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  }
+  return fn;
+}
+
+// [T, H, 128] bf16 viewed as a 3-D tensor (d, head, token); box 64 d x 1 head x 64 tokens.
+static bool make_map(CUtensorMap *m, const void *base, int H, int T) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)H * HD * 2};
+  const cuuint32_t box[3] = {64, 1, CH};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename TO>
+static cudaError_t launch_t(const void *q, const void *k, const void *v, const Params &prm,
+                            cudaStream_t stream) {
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, q, prm.Hqk, prm.T) || !make_map(&mk, k, prm.Hqk, prm.T) ||
+      !make_map(&mv, v, prm.Hv, prm.T))
+    return cudaErrorInvalidValue;
+  auto kern = prefill_tc_kernel<TO>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)prm.N * (unsigned)prm.Hv, NTHREADS, SMEM_BYTES, stream>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace tc
+
+bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype) {
+  return dtype == GDN_DTYPE_BF16 && Dk == 128 && Dv == 128 && Hqk > 0 && Hv % Hqk == 0;
+}
+
+cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
+                              int Hv, int o_dtype, float scale, const float *s0, float *sfin,
+                              void *o, void *workspace, cudaStream_t stream) {
+  tc::Params prm;
+  prm.g = g; prm.beta = beta; prm.cu = cu; prm.N = N; prm.T = (int)T_; prm.Hqk = Hqk; prm.Hv = Hv;
+  prm.scale = scale; prm.s0 = s0; prm.sfin = sfin; prm.o = o;
+  prm.status = static_cast<int32_t *>(workspace);
+  if (o_dtype == GDN_DTYPE_BF16) return tc::launch_t<__nv_bfloat16>(q, k, v, prm, stream);
+  return tc::launch_t<float>(q, k, v, prm, stream);
 }
 
 }  // namespace gdn

@@ -101,67 +101,75 @@ def rank_seed(base: int, rank: int) -> int:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clock, max clock and throttle reasons of one GPU every
+    `period_s` (NVML) while the timed region runs."""
 
-    def __init__(self, gpu_id=None):
-        self.proc = None
-        self.gpu_id = gpu_id
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, device_index=0, period_s=0.005):
+        self.idx = device_index
+        self.period = period_s
+        self.samples = []
+        self._stop = None
 
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-               "-lms", "200"]
-        if self.gpu_id:
-            cmd += ["-i", self.gpu_id]
+        import threading
+
         try:
-            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
-                                         text=True)
-        except (OSError, ValueError):
-            self.proc = None
+            import pynvml
+
+            pynvml.nvmlInit()
+            uuid = self.idx if isinstance(self.idx, str) else None
+            self.h = (pynvml.nvmlDeviceGetHandleByUUID(uuid) if uuid else
+                      pynvml.nvmlDeviceGetHandleByIndex(int(self.idx)))
+            self.nv = pynvml
+        except Exception:
+            self.nv = None
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            nv = self.nv
+            while not self._stop.is_set():
+                try:
+                    sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    mx = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+                    get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                        nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                    rs = get_reasons(self.h)
+                    self.samples.append((sm, mx, rs))
+                except Exception:
+                    pass
+                self._stop.wait(self.period)
+
+        self._t = threading.Thread(target=loop, daemon=True)
+        self._t.start()
         return self
 
     def __exit__(self, *exc):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+        if self._stop is not None:
+            self._stop.set()
+            self._t.join(timeout=2)
         return False
 
     def summary(self):
-        if not getattr(self, "lines", None):
+        if not self.samples:
             return None
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({name for _, _, r in self.samples for name, bit in self.REASONS.items()
+                          if r & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(x[1] for x in self.samples),
+                "reasons": reasons, "samples": len(sm), "source": "nvml"}
 
 
 def gpu_uuid(torch, dev):
+    """NVML identifier of the torch device: its UUID string, else its index."""
     try:
         u = str(torch.cuda.get_device_properties(dev).uuid)
         return u if u.startswith("GPU-") else "GPU-" + u
     except Exception:
-        return None
+        return dev.index or 0
 
 
 def load_peaks():
@@ -285,7 +293,9 @@ def run_ours(args, D):
            for _ in range(args.steps)]
     D.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(gpu_uuid(torch, dev)) as clk:
+    clk = ClockSampler(gpu_uuid(torch, dev))
+    clk.__enter__()  # sampled through the prefill, e2e and decode timed regions
+    if True:
         for e0, e1 in evs:
             flush.zero_()              # outside the timed pair: L2 holds nothing of the inputs
             e0.record(stream)
@@ -304,14 +314,29 @@ def run_ours(args, D):
 
     peaks, peak_src = load_peaks()
     kernel_ms = statistics.mean(per_ms)
-    uses_tc = _tc_path_available()
-    if uses_tc:
-        achieved = FLOP_PER_TOKEN * T / (kernel_ms / 1e3) / 1e12
-        peak = peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "kernel": "gdn_prefill_tc", "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak, "peak_source": f"{peak_src} bf16_tflops (burst)",
-                "algorithmic": f"{FLOP_PER_TOKEN} flop/token x {T} tokens",
-                "traffic": kernel_traffic("prefill_tc", os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_prefill_tc.cu"))}
+    if _tc_path_available():
+        # Time floors of the two bounds; the larger one binds.
+        flops = FLOP_PER_TOKEN * T
+        hbm_bytes = BYTES_PER_TOKEN * T + w.Hv * w.D * w.D * 4
+        t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
+        t_hbm = hbm_bytes / (peaks["hbm_gbs"] * 1e9)
+        tensor_ach = flops / (kernel_ms / 1e3) / 1e12
+        hbm_ach = hbm_bytes / (kernel_ms / 1e3) / 1e9
+        src = os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_prefill_tc.cu")
+        if t_hbm >= t_tensor:
+            roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": hbm_ach / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
+                    "algorithmic": f"{BYTES_PER_TOKEN} B/token x {T} tokens + final state"}
+        else:
+            roof = {"bound": "tensor", "achieved": tensor_ach, "peak": peaks["bf16_tflops"],
+                    "unit": "TFLOP/s", "frac": tensor_ach / peaks["bf16_tflops"],
+                    "peak_source": f"{peak_src} bf16_tflops (burst)",
+                    "algorithmic": f"{FLOP_PER_TOKEN} flop/token x {T} tokens"}
+        roof.update({"kernel": "prefill_tc_kernel", "kernel_ms": kernel_ms,
+                     "tensor_frac": tensor_ach / peaks["bf16_tflops"],
+                     "tensor_achieved_tflops": tensor_ach, "hbm_frac": hbm_ach / peaks["hbm_gbs"],
+                     "floor_us": {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6},
+                     "traffic": kernel_traffic("prefill_tc", src)})
     else:
         # CUDA-core path: 3 fp32 FMAs per state element per token (read, update, output)
         flop = 3 * 2 * w.D * w.D * w.Hv * T
@@ -322,8 +347,6 @@ def run_ours(args, D):
                 "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
                 "algorithmic": f"3 FMA per state element per token = {flop} flop",
                 "traffic": kernel_traffic("prefill_simt", os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_prefill_simt.cu"))}
-    roof["hbm_bytes_algorithmic"] = BYTES_PER_TOKEN * T + w.Hv * w.D * w.D * 4
-    roof["hbm_frac"] = roof["hbm_bytes_algorithmic"] / (kernel_ms / 1e3) / 1e9 / peaks["hbm_gbs"]
 
     out = {
         "metric": "GDN prefill Mtok/s (H=16/48,D=128) and decode-step state GB/s vs HBM peak",
@@ -335,7 +358,6 @@ def run_ours(args, D):
                    "l2": "flushed between timed steps (256 MiB write outside the timed pair)"},
         "roofline": roof,
         "gpu_launches": args.steps,
-        "clocks": clk.summary(),
     }
 
     if not args.no_e2e:
@@ -343,6 +365,8 @@ def run_ours(args, D):
 
     if not args.no_decode:
         out["decode"] = _decode(args, D, dev, peaks, peak_src)
+    clk.__exit__(None, None, None)
+    out["clocks"] = clk.summary()
 
     if not args.no_cpu_baseline and D.rank == 0 and D.world == 1:
         secs, threads = oracle_prefill_timed(inp, T)

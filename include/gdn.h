@@ -127,6 +127,38 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
                     void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Prefill for callers that cannot allocate device memory.  (The pages have no
+ * counterpart; this is a calling convention of the library.)  Some callers
+ * cannot call cudaMalloc for gdn_prefill's workspace: the device allocator
+ * belongs to someone else (a framework's caching allocator, a serving
+ * runtime's memory pool), the path is real-time and must not take
+ * cudaMalloc's implicit device-wide synchronisation, or a plugin is handed
+ * only its input and output buffers.  This entry point allocates nothing: it
+ * runs gdn_prefill with a 4096-byte workspace kept in a file-scope __device__
+ * array of the library (every GPU that loads the library holds it until the
+ * process exits), and calls no cudaMalloc, cudaFree or allocating routine.
+ *
+ * Arguments are those of gdn_prefill without the workspace, plus
+ *   device_status  optional device int32 (caller's memory, NULL to discard) that
+ *                  receives this call's device-detected status (GDN_OK,
+ *                  GDN_ERR_BAD_SEQLENS or GDN_ERR_DEVICE_TIMEOUT) in stream order.
+ * Returns GDN_ERR_WORKSPACE if these sizes need more workspace than the 4096-byte
+ * built-in array; otherwise what gdn_prefill returns.
+ *
+ * The first call on each device resolves the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call before
+ * any stream capture.  Every call on a device shares the one array: each call
+ * clears its header first, and calls whose work overlaps on the GPU (other
+ * streams, other host threads without ordering) race on it.
+ */
+int32_t gdn_prefill_noalloc(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
+                            int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
+                            int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, int32_t o_dtype,
+                            float scale, const float *initial_state, float *final_state, void *o,
+                            int32_t *device_status, void *stream);
+
+/*
  * Decode step: one new token for each of `batch` sequences, updating their
  * states in place ("Inside Qwen3.8-27B ...", section "Gated DeltaNet
  * Mechanics": in inference the state is updated token by token).

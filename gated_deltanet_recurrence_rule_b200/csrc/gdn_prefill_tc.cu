@@ -132,10 +132,52 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sb, int i) { return sb + OFF_BAR + 8u * i; }
 
+// Block row I (1..3) of the inverse: for every block column j < I,
+// Y_Ij = sum_{j<=k<I} A_Ik Tm_kj, then Tm_Ij = -Tm_II Y_Ij.  Thread etid owns
+// element (r, cc) = (etid / 16, etid % 16) of every block of the row.
+template <int I>
+__device__ __forceinline__ void ut_block_row(const float *A, float *Tm, float *Y, int etid) {
+  const int r = etid >> 4, cc = etid & 15;
+  float arow[16 * I];
+#pragma unroll
+  for (int q = 0; q < 16 * I; q += 4) {
+    const float4 a4 = *reinterpret_cast<const float4 *>(A + (16 * I + r) * AST + q);
+    arow[q] = a4.x; arow[q + 1] = a4.y; arow[q + 2] = a4.z; arow[q + 3] = a4.w;
+  }
+#pragma unroll
+  for (int j = 0; j < I; ++j) {
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int q = 16 * j; q < 16 * I; q += 2) {
+      acc0 = fmaf(arow[q], Tm[q * AST + 16 * j + cc], acc0);
+      acc1 = fmaf(arow[q + 1], Tm[(q + 1) * AST + 16 * j + cc], acc1);
+    }
+    Y[(j * 16 + r) * 17 + cc] = acc0 + acc1;
+  }
+  named_bar_sync(EPI_BAR, NEPI);
+  float trow[16];
+#pragma unroll
+  for (int m = 0; m < 16; m += 4) {
+    const float4 t4 = *reinterpret_cast<const float4 *>(Tm + (16 * I + r) * AST + 16 * I + m);
+    trow[m] = t4.x; trow[m + 1] = t4.y; trow[m + 2] = t4.z; trow[m + 3] = t4.w;
+  }
+#pragma unroll
+  for (int j = 0; j < I; ++j) {
+    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+    for (int m = 0; m < 16; m += 2) {
+      acc0 = fmaf(trow[m], Y[(j * 16 + m) * 17 + cc], acc0);
+      acc1 = fmaf(trow[m + 1], Y[(j * 16 + m + 1) * 17 + cc], acc1);
+    }
+    Tm[(16 * I + r) * AST + 16 * j + cc] = -(acc0 + acc1);
+  }
+  named_bar_sync(EPI_BAR, NEPI);
+}
+
 // Unit lower-triangular inverse Tm = (I + A)^-1 of a 64x64 strictly lower A,
 // fp32, by the 256 epilogue threads.  Diagonal 16x16 blocks by forward
-// substitution (one warp per block, two lanes per column), then block rows
-// i = 1..3: Y_ij = sum_{j<=k<i} A_ik Tm_kj and Tm_ij = -Tm_ii Y_ij.
+// substitution (one warp per block, two lanes per column), then the three
+// block rows below the first.
 __device__ __forceinline__ void ut_solve(const float *A, float *Tm, float *Y, int etid) {
   const int ew = etid >> 5, lane = etid & 31;
   if (ew < 4) {
@@ -156,38 +198,9 @@ __device__ __forceinline__ void ut_solve(const float *A, float *Tm, float *Y, in
     for (int m = 0; m < 8; ++m) Tm[(16 * b + 2 * m + hh) * AST + 16 * b + c] = x[m];
   }
   named_bar_sync(EPI_BAR, NEPI);
-#pragma unroll
-  for (int i = 1; i < 4; ++i) {
-    for (int e = etid; e < i * 256; e += NEPI) {
-      const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-      float acc = 0.f;
-      const float *arow = A + (16 * i + r) * AST;
-      for (int q = 16 * j; q < 16 * i; q += 4) {
-        const float4 a4 = *reinterpret_cast<const float4 *>(arow + q);
-        acc = fmaf(a4.x, Tm[(q + 0) * AST + 16 * j + cc], acc);
-        acc = fmaf(a4.y, Tm[(q + 1) * AST + 16 * j + cc], acc);
-        acc = fmaf(a4.z, Tm[(q + 2) * AST + 16 * j + cc], acc);
-        acc = fmaf(a4.w, Tm[(q + 3) * AST + 16 * j + cc], acc);
-      }
-      Y[(j * 16 + r) * 17 + cc] = acc;
-    }
-    named_bar_sync(EPI_BAR, NEPI);
-    for (int e = etid; e < i * 256; e += NEPI) {
-      const int j = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-      const float *trow = Tm + (16 * i + r) * AST + 16 * i;
-      float acc = 0.f;
-#pragma unroll
-      for (int m = 0; m < 16; m += 4) {
-        const float4 t4 = *reinterpret_cast<const float4 *>(trow + m);
-        acc = fmaf(t4.x, Y[(j * 16 + m + 0) * 17 + cc], acc);
-        acc = fmaf(t4.y, Y[(j * 16 + m + 1) * 17 + cc], acc);
-        acc = fmaf(t4.z, Y[(j * 16 + m + 2) * 17 + cc], acc);
-        acc = fmaf(t4.w, Y[(j * 16 + m + 3) * 17 + cc], acc);
-      }
-      Tm[(16 * i + r) * AST + 16 * j + cc] = -acc;
-    }
-    named_bar_sync(EPI_BAR, NEPI);
-  }
+  ut_block_row<1>(A, Tm, Y, etid);
+  ut_block_row<2>(A, Tm, Y, etid);
+  ut_block_row<3>(A, Tm, Y, etid);
 }
 
 // One waiter (epilogue thread 0) for an mbarrier phase, then a named barrier;
@@ -211,16 +224,19 @@ __device__ __forceinline__ void st_bf16x8(unsigned char *dst, const float *x) {
   *reinterpret_cast<uint4 *>(dst) = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
                                                pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
 }
-// 8 fp32 values x -> hi = bf16(x) at dst_hi and lo = bf16(x - hi) at dst_lo.
+// 8 fp32 values x -> x = hi + lo with hi = x truncated to bf16 (high 16 bits)
+// and lo = (x - hi) truncated to bf16; |x - hi - lo| < 2^-14 |x|.  Bit
+// operations only (mask, subtract, byte permute), no conversion instructions.
 __device__ __forceinline__ void st_split8(unsigned char *dst_hi, unsigned char *dst_lo,
                                           const float *x) {
   uint32_t hw[4], lw[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
-    const __nv_bfloat162 hh = __halves2bfloat162(h0, h1);
-    hw[e] = *reinterpret_cast<const uint32_t *>(&hh);
-    lw[e] = pack_bf16x2(x[2 * e] - __bfloat162float(h0), x[2 * e + 1] - __bfloat162float(h1));
+    const uint32_t a = __float_as_uint(x[2 * e]), b = __float_as_uint(x[2 * e + 1]);
+    const float ra = x[2 * e] - __uint_as_float(a & 0xffff0000u);
+    const float rb = x[2 * e + 1] - __uint_as_float(b & 0xffff0000u);
+    hw[e] = __byte_perm(a, b, 0x7632);
+    lw[e] = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
   }
   *reinterpret_cast<uint4 *>(dst_hi) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
   *reinterpret_cast<uint4 *>(dst_lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
@@ -609,15 +625,18 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const uint32_t off = ewg * 16384 + sw128_off(row, q);
           st_split8(smem + OFF_S0H + off, smem + OFF_S0L + off, S + 8 * q);
         }
-        float vi[32], va[32];
-        tmem_ld32(tl + R_OI + 32 * ewg, vi);
-        tmem_ld32(tl + R_OA + 32 * ewg, va);
-        tmem_wait_ld();
         TO *op = static_cast<TO *>(p.o) + ((size_t)t0 * p.Hv + h) * HD + row;
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          const int t = 32 * ewg + x;
-          if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(p.scale * fmaf(gam[t], vi[x], va[x]));
+        for (int hf = 0; hf < 2; ++hf) {
+          float vi[16], va[16];
+          tmem_ld16(tl + R_OI + 32 * ewg + 16 * hf, vi);
+          tmem_ld16(tl + R_OA + 32 * ewg + 16 * hf, va);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 16; ++x) {
+            const int t = 32 * ewg + 16 * hf + x;
+            if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(p.scale * fmaf(gam[t], vi[x], va[x]));
+          }
         }
       }
       fence_proxy_async_smem();

@@ -32,12 +32,12 @@
 // The 64x64 unit lower-triangular inverse Tm is computed in fp32 on CUDA
 // cores (16x16 diagonal blocks by forward substitution, then block rows).
 //
-// One CTA per (sequence, value head); 384 threads:
+// One CTA per (sequence, value head); 640 threads:
 //   warp 0      TMA producer (Q/K ring of 2, V buffer of 1, L2 prefetch ahead)
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
 //   warp 2      per-chunk scalars (prefix sums of g, decays, masked beta)
 //   warp 3      idle
-//   warps 4-11  256 epilogue threads: TMEM -> registers -> SMEM operands,
+//   warps 4-19  512 epilogue threads: TMEM -> registers -> SMEM operands,
 //               the triangular solve, the fp32 state and the outputs.
 // Chunks run one after another (this version does not overlap the next
 // chunk's state-independent work with the current chunk's state chain).
@@ -56,8 +56,8 @@ using namespace sm100;
 
 constexpr int CH = 64;            // chunk length
 constexpr int HD = 128;           // head dim (Dk = Dv)
-constexpr int NTHREADS = 384;
-constexpr int NEPI = 256;         // epilogue threads
+constexpr int NTHREADS = 640;
+constexpr int NEPI = 512;         // epilogue threads: 4 warpgroups, one quarter of the columns each
 constexpr int EPI_BAR = 1;        // named barrier id of the epilogue threads
 constexpr float LOG2E = 1.4426950408889634f;
 // alpha below e^-30 is treated as e^-30: the chunk prefix sums stay finite
@@ -65,51 +65,52 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr float G_FLOOR = -30.f;
 
 // ---- shared memory map (bytes); swizzled tiles are 1024-byte aligned ----
+constexpr int NQK = 3, NV = 2;          // ring depths (Q/K and V)
 constexpr uint32_t QK_STAGE = 32768;   // [Q d0-63 | K d0-63 | Q d64-127 | K d64-127], 64 rows x 128 B each
 constexpr uint32_t V_STAGE = 16384;    // [V d0-63 | V d64-127]
-constexpr uint32_t OFF_QK = 0;         // 2 stages
-constexpr uint32_t OFF_V = 65536;      // 1 stage
-constexpr uint32_t OFF_S0H = 81920;    // bf16 hi(S0), K-major: 2 x (128 rows x 128 B)
-constexpr uint32_t OFF_S0L = 114688;   // bf16 lo(S0)
-// R1: one 64 KB region reused by phases of a chunk that never overlap:
+constexpr uint32_t OFF_QK = 0;
+constexpr uint32_t OFF_V = OFF_QK + NQK * QK_STAGE;
+// R1: a region reused by phases of a chunk that never overlap:
 //   solve:   A fp32 [64][68] @0, Tm fp32 [64][68] @32K, Y fp32 [3][16][17] @50176
 //   W, U~:   T' hi @0, T' lo @8K, T'' hi @16K, T'' lo @24K (Tm still read)
 //   S0 W^T:  W^T bf16 MN-major (128 rows d x 64 t) @0
-//   U:       U hi @0, U lo @16K, Ukdec hi @32K, Ukdec lo @48K (K-major, 128 rows x 64 t)
-constexpr uint32_t OFF_R1 = 147456;
+constexpr uint32_t OFF_R1 = OFF_V + NV * V_STAGE;
 constexpr uint32_t OFF_A = OFF_R1;
 constexpr uint32_t OFF_TM = OFF_R1 + 32768;
 constexpr uint32_t OFF_Y = OFF_R1 + 50176;
 constexpr uint32_t OFF_TPH = OFF_R1, OFF_TPL = OFF_R1 + 8192;
 constexpr uint32_t OFF_TQH = OFF_R1 + 16384, OFF_TQL = OFF_R1 + 24576;
 constexpr uint32_t OFF_WT = OFF_R1;
-constexpr uint32_t OFF_UH = OFF_R1, OFF_UL = OFF_R1 + 16384;
-constexpr uint32_t OFF_UKH = OFF_R1 + 32768, OFF_UKL = OFF_R1 + 49152;
-constexpr uint32_t OFF_PH = OFF_R1 + 65536;  // bf16 hi(P), K-major B: 64 rows (t) x 64 s
-constexpr uint32_t OFF_PL = OFF_PH + 8192;   // bf16 lo(P)
+constexpr uint32_t R1_BYTES = 54272;
+constexpr uint32_t OFF_PH = OFF_R1 + R1_BYTES;  // bf16 hi(P), K-major B: 64 rows (t) x 64 s
+constexpr uint32_t OFF_PL = OFF_PH + 8192;      // bf16 lo(P)
 constexpr uint32_t OFF_SCAL = OFF_PL + 8192;
 constexpr uint32_t SCAL_STAGE = 5 * 64 * 4;  // G2 (log2 prefix), gamma, kdec, beta; gamma_C at [256]
 constexpr uint32_t OFF_BAR = OFF_SCAL + 2 * SCAL_STAGE;
 constexpr uint32_t OFF_MISC = OFF_BAR + 192;  // [0] TMEM base, [4] abort flag, [8] drain mbarrier
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
 constexpr int AST = 68;  // fp32 row stride of A and Tm (conflict-free float4 row stores)
-static_assert(OFF_R1 % 1024 == 0 && OFF_PH % 1024 == 0 && OFF_S0H % 1024 == 0, "alignment");
-static_assert(OFF_Y + 3 * 16 * 17 * 4 <= OFF_R1 + 65536, "R1 layout");
+static_assert(OFF_R1 % 1024 == 0 && OFF_PH % 1024 == 0 && OFF_V % 1024 == 0, "alignment");
+static_assert(OFF_Y + 3 * 16 * 17 * 4 <= OFF_R1 + R1_BYTES, "R1 layout");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// ---- TMEM columns (fp32 accumulators, 128 lanes) ----
-constexpr uint32_t R_QK = 0;    // 64: rows 0-63 = Q K^T, rows 64-127 = K K^T
-constexpr uint32_t R_W = 64;    // 64: W^T
-constexpr uint32_t R_U = 128;   // 64: U~^T, then U^T
-constexpr uint32_t R_S = 192;   // 128: dS
-constexpr uint32_t R_OI = 320;  // 64: S0 Q^T
-constexpr uint32_t R_OA = 384;  // 64: U^T P^T
+// ---- TMEM columns (128 lanes x 512 columns of 32 bit) ----
+// Accumulators (fp32) share columns across phases of a chunk that never overlap.
+constexpr uint32_t R_QK = 0;    // 64: rows 0-63 = Q K^T, rows 64-127 = K K^T   (chunk start)
+constexpr uint32_t R_W = 64;    // 64: W^T                                      (after the solve)
+constexpr uint32_t R_S = 0;     // 128: dS                                      (chunk end)
+constexpr uint32_t R_UO = 128;  // 64: U~^T, then U^T; afterwards U^T P^T
+constexpr uint32_t R_OI = 192;  // 64: S0 Q^T
+// MMA A operands in TMEM (bf16 pairs per column; lane = row of the operand).
+constexpr uint32_t T_S0H = 256, T_S0L = 320;  // hi/lo(S0): 128 rows x 128 K (64 columns each)
+constexpr uint32_t T_UH = 384, T_UL = 416;    // hi/lo(U^T): 128 rows x 64 K (32 columns each)
+constexpr uint32_t T_UKH = 448, T_UKL = 480;  // hi/lo(U^T diag(kdec))
 constexpr uint32_t TMEM_COLS = 512;
 
 // ---- mbarriers ----
 enum {
-  B_FULL_QK = 0, B_EMPTY_QK = 2, B_FULL_V = 4, B_EMPTY_V = 5, B_SCAL_FULL = 6, B_SCAL_EMPTY = 8,
-  B_QK = 10, B_T = 11, B_W = 12, B_WT = 13, B_U = 14, B_UT = 15, B_S = 16, B_DONE = 17, NBAR = 18
+  B_FULL_QK = 0, B_EMPTY_QK = 3, B_FULL_V = 6, B_EMPTY_V = 8, B_SCAL_FULL = 10, B_SCAL_EMPTY = 12,
+  B_QK = 14, B_T = 15, B_W = 16, B_WT = 17, B_U = 18, B_UT = 19, B_S = 20, B_DONE = 21, NBAR = 22
 };
 static_assert(NBAR * 8 <= 192, "barrier area");
 
@@ -132,75 +133,112 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sb, int i) { return sb + OFF_BAR + 8u * i; }
 
-// Block row I (1..3) of the inverse: for every block column j < I,
-// Y_Ij = sum_{j<=k<I} A_Ik Tm_kj, then Tm_Ij = -Tm_II Y_Ij.  Thread etid owns
-// element (r, cc) = (etid / 16, etid % 16) of every block of the row.
-template <int I>
-__device__ __forceinline__ void ut_block_row(const float *A, float *Tm, float *Y, int etid) {
-  const int r = etid >> 4, cc = etid & 15;
-  float arow[16 * I];
+// ---- warp-level m16n8k8 tf32 MMAs with a 3-term split (x = hi + lo, hi =
+// tf32(x)): hi*hi + hi*lo + lo*hi carries ~fp32 accuracy.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+__device__ __forceinline__ void mma_tf32_16x8x8(float *d, const uint32_t *a, const uint32_t *b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// D (16x8 fp32, fragment layout) = X (16 x 8 KS, row-major, stride ldx) *
+// Y (8 KS x 8, row-major, stride ldy), with the 3-term split.
+template <int KS>
+__device__ __forceinline__ void mma3_16x8(float *d, const float *X, int ldx, const float *Y, int ldy,
+                                          int lane) {
+  const int gid = lane >> 2, tig = lane & 3;
+  float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int q = 0; q < 16 * I; q += 4) {
-    const float4 a4 = *reinterpret_cast<const float4 *>(A + (16 * I + r) * AST + q);
-    arow[q] = a4.x; arow[q + 1] = a4.y; arow[q + 2] = a4.z; arow[q + 3] = a4.w;
+  for (int ks = 0; ks < KS; ++ks) {
+    const float a0 = X[gid * ldx + 8 * ks + tig], a1 = X[(gid + 8) * ldx + 8 * ks + tig];
+    const float a2 = X[gid * ldx + 8 * ks + tig + 4], a3 = X[(gid + 8) * ldx + 8 * ks + tig + 4];
+    const float b0 = Y[(8 * ks + tig) * ldy + gid], b1 = Y[(8 * ks + tig + 4) * ldy + gid];
+    const uint32_t ah[4] = {to_tf32(a0), to_tf32(a1), to_tf32(a2), to_tf32(a3)};
+    const uint32_t al[4] = {to_tf32(a0 - __uint_as_float(ah[0])), to_tf32(a1 - __uint_as_float(ah[1])),
+                            to_tf32(a2 - __uint_as_float(ah[2])), to_tf32(a3 - __uint_as_float(ah[3]))};
+    const uint32_t bh[2] = {to_tf32(b0), to_tf32(b1)};
+    const uint32_t bl[2] = {to_tf32(b0 - __uint_as_float(bh[0])), to_tf32(b1 - __uint_as_float(bh[1]))};
+    mma_tf32_16x8x8(d, ah, bh);
+    mma_tf32_16x8x8(d1, ah, bl);
+    mma_tf32_16x8x8(d2, al, bh);
   }
 #pragma unroll
-  for (int j = 0; j < I; ++j) {
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int q = 16 * j; q < 16 * I; q += 2) {
-      acc0 = fmaf(arow[q], Tm[q * AST + 16 * j + cc], acc0);
-      acc1 = fmaf(arow[q + 1], Tm[(q + 1) * AST + 16 * j + cc], acc1);
-    }
-    Y[(j * 16 + r) * 17 + cc] = acc0 + acc1;
+  for (int e = 0; e < 4; ++e) d[e] += d1[e] + d2[e];
+}
+__device__ __forceinline__ void st_frag16x8(float *M, int ld, const float *d, float scale, int lane) {
+  const int gid = lane >> 2, tig = lane & 3;
+  M[gid * ld + 2 * tig] = scale * d[0];
+  M[gid * ld + 2 * tig + 1] = scale * d[1];
+  M[(gid + 8) * ld + 2 * tig] = scale * d[2];
+  M[(gid + 8) * ld + 2 * tig + 1] = scale * d[3];
+}
+
+// Off-diagonal blocks at block distance DIST (1..3) of the inverse: for the
+// 4 - DIST blocks (i, j = i - DIST), Y_ij = sum_{j<=k<i} A_ik Tm_kj (one
+// 16 x 16 DIST x 16 product), then Tm_ij = -Tm_ii Y_ij (16 x 16 x 16).  One warp
+// per (block, 8-column half) on the tensor cores (warp-level mma.sync).
+template <int DIST>
+__device__ __forceinline__ void ut_distance(const float *__restrict__ A, float *__restrict__ Tm,
+                                            float *__restrict__ Y, int etid) {
+  constexpr int NB = 4 - DIST;
+  const int w = etid >> 5, lane = etid & 31;
+  if (w < 2 * NB) {
+    const int j = w >> 1, i = j + DIST, nh = w & 1;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    mma3_16x8<2 * DIST>(d, A + 16 * i * AST + 16 * j, AST, Tm + 16 * j * AST + 16 * j + 8 * nh, AST, lane);
+    st_frag16x8(Y + (j * 16) * 17 + 8 * nh, 17, d, 1.f, lane);
   }
   named_bar_sync(EPI_BAR, NEPI);
-  float trow[16];
-#pragma unroll
-  for (int m = 0; m < 16; m += 4) {
-    const float4 t4 = *reinterpret_cast<const float4 *>(Tm + (16 * I + r) * AST + 16 * I + m);
-    trow[m] = t4.x; trow[m + 1] = t4.y; trow[m + 2] = t4.z; trow[m + 3] = t4.w;
-  }
-#pragma unroll
-  for (int j = 0; j < I; ++j) {
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int m = 0; m < 16; m += 2) {
-      acc0 = fmaf(trow[m], Y[(j * 16 + m) * 17 + cc], acc0);
-      acc1 = fmaf(trow[m + 1], Y[(j * 16 + m + 1) * 17 + cc], acc1);
-    }
-    Tm[(16 * I + r) * AST + 16 * j + cc] = -(acc0 + acc1);
+  if (w < 2 * NB) {
+    const int j = w >> 1, i = j + DIST, nh = w & 1;
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    mma3_16x8<2>(d, Tm + 16 * i * AST + 16 * i, AST, Y + (j * 16) * 17 + 8 * nh, 17, lane);
+    st_frag16x8(Tm + 16 * i * AST + 16 * j + 8 * nh, AST, d, -1.f, lane);
   }
   named_bar_sync(EPI_BAR, NEPI);
 }
 
 // Unit lower-triangular inverse Tm = (I + A)^-1 of a 64x64 strictly lower A,
-// fp32, by the 256 epilogue threads.  Diagonal 16x16 blocks by forward
-// substitution (one warp per block, two lanes per column), then the three
-// block rows below the first.
-__device__ __forceinline__ void ut_solve(const float *A, float *Tm, float *Y, int etid) {
-  const int ew = etid >> 5, lane = etid & 31;
-  if (ew < 4) {
-    const int b = ew, c = lane >> 1, hh = lane & 1;
-    float x[8];
+// fp32, by the epilogue threads.  The four 16x16 diagonal blocks by forward
+// substitution (four warps per block, eight lanes per column, each lane two
+// rows with their A entries in registers), then the off-diagonal blocks by
+// block distance 1, 2, 3 (each needs only blocks of smaller distance).
+__device__ __forceinline__ void ut_solve(const float *__restrict__ A, float *__restrict__ Tm,
+                                         float *__restrict__ Y, int etid) {
+  {
+    const int ew = etid >> 5, lane = etid & 31;
+    const int b = ew >> 2, c = 4 * (ew & 3) + (lane >> 3), q = lane & 7;
+    float a[2][16];
 #pragma unroll
-    for (int m = 0; m < 8; ++m) x[m] = (2 * m + hh == c) ? 1.f : 0.f;
+    for (int m = 0; m < 2; ++m)
+#pragma unroll
+      for (int s4 = 0; s4 < 16; s4 += 4) {
+        const float4 v4 = *reinterpret_cast<const float4 *>(A + (16 * b + q + 8 * m) * AST + 16 * b + s4);
+        a[m][s4] = v4.x; a[m][s4 + 1] = v4.y; a[m][s4 + 2] = v4.z; a[m][s4 + 3] = v4.w;
+      }
+    float x[2];
+#pragma unroll
+    for (int m = 0; m < 2; ++m) x[m] = (q + 8 * m == c) ? 1.f : 0.f;
 #pragma unroll
     for (int s = 0; s < 16; ++s) {
-      const float xs = __shfl_sync(0xffffffffu, x[s >> 1], (c << 1) | (s & 1));
+      const float xs = __shfl_sync(0xffffffffu, x[s >> 3], (lane & ~7) | (s & 7));
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int r = 2 * m + hh;
-        if (r > s) x[m] = fmaf(-A[(16 * b + r) * AST + 16 * b + s], xs, x[m]);
-      }
+      for (int m = 0; m < 2; ++m)
+        if (q + 8 * m > s) x[m] = fmaf(-a[m][s], xs, x[m]);
     }
 #pragma unroll
-    for (int m = 0; m < 8; ++m) Tm[(16 * b + 2 * m + hh) * AST + 16 * b + c] = x[m];
+    for (int m = 0; m < 2; ++m) Tm[(16 * b + q + 8 * m) * AST + 16 * b + c] = x[m];
   }
   named_bar_sync(EPI_BAR, NEPI);
-  ut_block_row<1>(A, Tm, Y, etid);
-  ut_block_row<2>(A, Tm, Y, etid);
-  ut_block_row<3>(A, Tm, Y, etid);
+  ut_distance<1>(A, Tm, Y, etid);
+  ut_distance<2>(A, Tm, Y, etid);
+  ut_distance<3>(A, Tm, Y, etid);
 }
 
 // One waiter (epilogue thread 0) for an mbarrier phase, then a named barrier;
@@ -240,6 +278,20 @@ __device__ __forceinline__ void st_split8(unsigned char *dst_hi, unsigned char *
   }
   *reinterpret_cast<uint4 *>(dst_hi) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
   *reinterpret_cast<uint4 *>(dst_lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+// 2n fp32 values -> packed bf16 pairs hw[n] = hi(x), lw[n] = lo(x) with the
+// same truncation split as st_split8 (for tcgen05.st into TMEM operands).
+template <int NP>
+__device__ __forceinline__ void split_words(const float *x, uint32_t *hw, uint32_t *lw) {
+#pragma unroll
+  for (int e = 0; e < NP; ++e) {
+    const uint32_t a = __float_as_uint(x[2 * e]), b = __float_as_uint(x[2 * e + 1]);
+    const float ra = x[2 * e] - __uint_as_float(a & 0xffff0000u);
+    const float rb = x[2 * e + 1] - __uint_as_float(b & 0xffff0000u);
+    hw[e] = __byte_perm(a, b, 0x7632);
+    lw[e] = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+  }
 }
 
 template <typename TO>
@@ -300,7 +352,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       int issued_qk = 0, issued_v = 0;  // chunks whose loads were issued
       for (int c = 0; c < nch; ++c) {
-        const int s = c & 1;
+        const int s = c % NQK, sv = c % NV;
         const int t0 = c0 + c * CH;
         if (c + PF < nch) {
           const int t = t0 + PF * CH;
@@ -308,7 +360,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
           tma_prefetch_3d(&tm_v, 0, h, t); tma_prefetch_3d(&tm_v, 64, h, t);
         }
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c >> 1) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag)) break;
         const uint32_t st = sb + OFF_QK + s * QK_STAGE;
         const uint32_t fb = bar_addr(sb, B_FULL_QK + s);
         mbar_arrive_expect_tx(fb, QK_STAGE);
@@ -317,11 +369,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tma_load_3d(st + 8192, &tm_k, fb, 0, j, t0);
         tma_load_3d(st + 24576, &tm_k, fb, 64, j, t0);
         issued_qk = c + 1;
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_V), (c & 1) ^ 1, abort_flag)) break;
-        const uint32_t fv = bar_addr(sb, B_FULL_V);
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_V + sv), ((c / NV) & 1) ^ 1, abort_flag)) break;
+        const uint32_t vs = sb + OFF_V + sv * V_STAGE;
+        const uint32_t fv = bar_addr(sb, B_FULL_V + sv);
         mbar_arrive_expect_tx(fv, V_STAGE);
-        tma_load_3d(sb + OFF_V + 0, &tm_v, fv, 0, h, t0);
-        tma_load_3d(sb + OFF_V + 8192, &tm_v, fv, 64, h, t0);
+        tma_load_3d(vs + 0, &tm_v, fv, 0, h, t0);
+        tma_load_3d(vs + 8192, &tm_v, fv, 64, h, t0);
         issued_v = c + 1;
       }
       if (issued_qk < nch || issued_v < nch) {
@@ -330,85 +383,87 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       // Let every load this thread issued land before the CTA can exit (each
       // buffer's latest fill; earlier fills were consumed before it was issued).
-      for (int c = max(issued_qk - 2, 0); c < issued_qk; ++c)
-        mbar_wait(bar_addr(sb, B_FULL_QK + (c & 1)), (c >> 1) & 1, abort_flag, 50000000ull);
-      if (issued_v > 0)
-        mbar_wait(bar_addr(sb, B_FULL_V), (issued_v - 1) & 1, abort_flag, 50000000ull);
+      for (int c = max(issued_qk - NQK, 0); c < issued_qk; ++c)
+        mbar_wait(bar_addr(sb, B_FULL_QK + c % NQK), (c / NQK) & 1, abort_flag, 50000000ull);
+      for (int c = max(issued_v - NV, 0); c < issued_v; ++c)
+        mbar_wait(bar_addr(sb, B_FULL_V + c % NV), (c / NV) & 1, abort_flag, 50000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
+      // Base descriptors, built once; per-MMA offsets are compile-time byte
+      // counts added to the start-address field (bytes / 16).
+      const uint64_t dQK0 = sdesc_sw128(sb + OFF_QK, 16, 1024);            // Q/K stage, K-major
+      const uint64_t dKmn0 = sdesc_sw128(sb + OFF_QK + 8192, 16384, 1024); // K as MN-major operand
+      const uint64_t dVmn0 = sdesc_sw128(sb + OFF_V, 8192, 1024);           // V as MN-major operand
+      const uint64_t dR1 = sdesc_sw128(sb + OFF_R1, 16, 1024);              // T splits (K-major)
+      const uint64_t dWT = sdesc_sw128(sb + OFF_WT, 8192, 1024);            // W^T, MN-major
+      const uint64_t dP = sdesc_sw128(sb + OFF_PH, 16, 1024);               // P hi / lo, K-major
       bool ok = true;
       for (int c = 0; c < nch && ok; ++c) {
-        const int s = c & 1;
-        const uint32_t ph2 = (c >> 1) & 1, ph = c & 1;
-        const uint32_t st = sb + OFF_QK + s * QK_STAGE;
+        const int s = c % NQK, sv = c % NV;
+        const uint32_t ph = c & 1;
+        const uint64_t dQK = dQK0 + s * (QK_STAGE >> 4), dKmn = dKmn0 + s * (QK_STAGE >> 4);
+        const uint64_t dVmn = dVmn0 + sv * (V_STAGE >> 4);
         // [Q;K] K^T
-        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), ph2, abort_flag);
+        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), (c / NQK) & 1, abort_flag);
         if (ok && c > 0) ok = mbar_wait(bar_addr(sb, B_DONE), (c - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_bf16(tmem + R_QK, sdesc_sw128(st + koff, 16, 1024),
-                   sdesc_sw128(st + 8192 + koff, 16, 1024), IDESC_QK, ks > 0);
+          const uint32_t k16 = ((ks >> 2) * 16384 + (ks & 3) * 32) >> 4;
+          mma_bf16(tmem + R_QK, dQK + k16, dQK + (8192 >> 4) + k16, IDESC_QK, ks > 0);
         }
         mma_commit(bar_addr(sb, B_QK));
         // W^T = K^T (T'h + T'l)^T ;  U~^T = V^T (T''h + T''l)^T
         ok = mbar_wait(bar_addr(sb, B_T), ph, abort_flag) &&
-             mbar_wait(bar_addr(sb, B_FULL_V), ph, abort_flag);
+             mbar_wait(bar_addr(sb, B_FULL_V + sv), (c / NV) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t bo = ((ks & 1) ? OFF_TPL : OFF_TPH) + (ks >> 1) * 32;
-          mma_bf16(tmem + R_W, sdesc_sw128(st + 8192 + (ks >> 1) * 2048, 16384, 1024),
-                   sdesc_sw128(sb + bo, 16, 1024), IDESC_WY, ks > 0);
+          const uint32_t bo = (((ks & 1) ? OFF_TPL : OFF_TPH) - OFF_R1 + (ks >> 1) * 32) >> 4;
+          mma_bf16(tmem + R_W, dKmn + (((ks >> 1) * 2048) >> 4), dR1 + bo, IDESC_WY, ks > 0);
         }
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t bo = ((ks & 1) ? OFF_TQL : OFF_TQH) + (ks >> 1) * 32;
-          mma_bf16(tmem + R_U, sdesc_sw128(sb + OFF_V + (ks >> 1) * 2048, 8192, 1024),
-                   sdesc_sw128(sb + bo, 16, 1024), IDESC_WY, ks > 0);
+          const uint32_t bo = (((ks & 1) ? OFF_TQL : OFF_TQH) - OFF_R1 + (ks >> 1) * 32) >> 4;
+          mma_bf16(tmem + R_UO, dVmn + (((ks >> 1) * 2048) >> 4), dR1 + bo, IDESC_WY, ks > 0);
         }
         mma_commit(bar_addr(sb, B_W));
-        mma_commit(bar_addr(sb, B_EMPTY_V));
-        // U^T = U~^T - S0h W^T ;  Oi^T = (S0h + S0l) Q^T
+        mma_commit(bar_addr(sb, B_EMPTY_V + sv));
+        // U^T = U~^T - S0h W^T ;  Oi^T = (S0h + S0l) Q^T   (S0 from TMEM)
         ok = mbar_wait(bar_addr(sb, B_WT), ph, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t koff = (ks >> 2) * 16384 + (ks & 3) * 32;
-          mma_bf16(tmem + R_U, sdesc_sw128(sb + OFF_S0H + koff, 16, 1024),
-                   sdesc_sw128(sb + OFF_WT + ks * 2048, 8192, 1024), IDESC_SW, 1);
-        }
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_ts(tmem + R_UO, tmem + T_S0H + 8 * ks, dWT + ((ks * 2048) >> 4), IDESC_SW, 1);
 #pragma unroll
         for (int ks = 0; ks < 16; ++ks) {
-          const uint32_t koff = ((ks >> 1) >> 2) * 16384 + ((ks >> 1) & 3) * 32;
-          const uint32_t ao = (ks & 1) ? OFF_S0L : OFF_S0H;
-          mma_bf16(tmem + R_OI, sdesc_sw128(sb + ao + koff, 16, 1024),
-                   sdesc_sw128(st + koff, 16, 1024), IDESC_SQ, ks > 0);
+          const int k = ks >> 1;
+          const uint32_t k16 = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+          mma_bf16_ts(tmem + R_OI, tmem + ((ks & 1) ? T_S0L : T_S0H) + 8 * k, dQK + k16, IDESC_SQ,
+                      ks > 0);
         }
         mma_commit(bar_addr(sb, B_U));
-        // dS = (Ukh + Ukl)^T K ;  Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T
+        // dS = (Ukh + Ukl)^T K ;  Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T   (U from TMEM)
         ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t ao = ((ks & 1) ? OFF_UKL : OFF_UKH) + (ks >> 1) * 32;
-          mma_bf16(tmem + R_S, sdesc_sw128(sb + ao, 16, 1024),
-                   sdesc_sw128(st + 8192 + (ks >> 1) * 2048, 16384, 1024), IDESC_UK, ks > 0);
+          const int kk = ks >> 1;
+          mma_bf16_ts(tmem + R_S, tmem + ((ks & 1) ? T_UKL : T_UKH) + 8 * kk,
+                      dKmn + ((kk * 2048) >> 4), IDESC_UK, ks > 0);
         }
 #pragma unroll
         for (int ks = 0; ks < 12; ++ks) {
           const int part = ks % 3, kk = ks / 3;  // (Uh,Ph), (Ul,Ph), (Uh,Pl)
-          const uint32_t ao = (part == 1 ? OFF_UL : OFF_UH) + kk * 32;
-          const uint32_t bo = (part == 2 ? OFF_PL : OFF_PH) + kk * 32;
-          mma_bf16(tmem + R_OA, sdesc_sw128(sb + ao, 16, 1024), sdesc_sw128(sb + bo, 16, 1024),
-                   IDESC_SQ, ks > 0);
+          const uint32_t bo = ((part == 2 ? OFF_PL - OFF_PH : 0) + kk * 32) >> 4;
+          mma_bf16_ts(tmem + R_UO, tmem + (part == 1 ? T_UL : T_UH) + 8 * kk, dP + bo, IDESC_SQ,
+                      ks > 0);
         }
         mma_commit(bar_addr(sb, B_S));
         mma_commit(bar_addr(sb, B_EMPTY_QK + s));
@@ -470,29 +525,28 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int etid = tid - 128;
-    const int ewg = etid >> 7;         // column half
+    const int ewq = etid >> 7;         // column quarter
     const int row = etid & 127;        // TMEM lane = row of the 128-row tiles
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     float *A = reinterpret_cast<float *>(smem + OFF_A);
     float *Tm = reinterpret_cast<float *>(smem + OFF_TM);
     float *Y = reinterpret_cast<float *>(smem + OFF_Y);
 
-    // fp32 master state: row `row`, columns [64 ewg, 64 ewg + 64); S0 = hi + lo in SMEM
-    float S[64];
+    // fp32 master state: row `row`, columns [32 ewq, 32 ewq + 32); S0 = hi + lo in TMEM
+    float S[32];
     {
-      const float *src = p.s0 ? p.s0 + sbase + (size_t)row * HD + 64 * ewg : nullptr;
+      const float *src = p.s0 ? p.s0 + sbase + (size_t)row * HD + 32 * ewq : nullptr;
 #pragma unroll
-      for (int x = 0; x < 64; x += 4) {
+      for (int x = 0; x < 32; x += 4) {
         float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
         if (src) v4 = *reinterpret_cast<const float4 *>(src + x);
         S[x] = v4.x; S[x + 1] = v4.y; S[x + 2] = v4.z; S[x + 3] = v4.w;
       }
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t off = ewg * 16384 + sw128_off(row, q);
-        st_split8(smem + OFF_S0H + off, smem + OFF_S0L + off, S + 8 * q);
-      }
-      fence_proxy_async_smem();
+      uint32_t hw[16], lw[16];
+      split_words<16>(S, hw, lw);
+      tmem_st16(tl + T_S0H + 16 * ewq, hw);
+      tmem_st16(tl + T_S0L + 16 * ewq, lw);
+      tmem_wait_st();
     }
 
     for (int c = 0; c < nch; ++c) {
@@ -512,33 +566,33 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       if (!epi_wait(bar_addr(sb, B_QK), ph, etid, abort_flag, p.status)) break;
       {
-        float v[32];
-        tmem_ld32(tl + R_QK + 32 * ewg, v);
+        float v[16];
+        tmem_ld16(tl + R_QK + 16 * ewq, v);
         tmem_wait_ld();
         if (row < 64) {
           const int t = row;
           const float Gt = G2[t];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
+          for (int q = 0; q < 2; ++q) {
             float pv[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const int si = 32 * ewg + 8 * q + e;
+              const int si = 16 * ewq + 8 * q + e;
               pv[e] = (si <= t && t < Lc) ? exp2f(Gt - G2[si]) * v[8 * q + e] : 0.f;
             }
-            const uint32_t off = sw128_off(t, 4 * ewg + q);
+            const uint32_t off = sw128_off(t, 2 * ewq + q);
             st_split8(smem + OFF_PH + off, smem + OFF_PL + off, pv);
           }
         } else {
           const int t = row - 64;
           const float Gt = G2[t], bt = bet[t];
-          float *arow = A + t * AST + 32 * ewg;
+          float *arow = A + t * AST + 16 * ewq;
 #pragma unroll
-          for (int x = 0; x < 32; x += 4) {
+          for (int x = 0; x < 16; x += 4) {
             float a[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int si = 32 * ewg + x + e;
+              const int si = 16 * ewq + x + e;
               a[e] = (si < t && t < Lc) ? bt * exp2f(Gt - G2[si]) * v[x + e] : 0.f;
             }
             *reinterpret_cast<float4 *>(arow + x) = make_float4(a[0], a[1], a[2], a[3]);
@@ -551,22 +605,26 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // ---- Tm = (I + A)^-1, then T' = Tm diag(beta gamma), T'' = Tm diag(beta), split
       ut_solve(A, Tm, Y, etid);
       {
-        const int t = etid >> 2, qq = etid & 3;
+        const int t = etid >> 3, sbeg = 8 * (etid & 7);
+        float tm[8], bt[8], gm[8], tp[8], tq[8];
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const int sbeg = 16 * qq + 8 * hf;
-          float tp[8], tq[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int si = sbeg + e;
-            const float m = (si <= t) ? Tm[t * AST + si] : 0.f;
-            tq[e] = m * bet[si];
-            tp[e] = tq[e] * gam[si];
-          }
-          const uint32_t off = sw128_off(t, sbeg >> 3);
-          st_split8(smem + OFF_TPH + off, smem + OFF_TPL + off, tp);
-          st_split8(smem + OFF_TQH + off, smem + OFF_TQL + off, tq);
+        for (int e = 0; e < 8; e += 4) {
+          const float4 a4 = *reinterpret_cast<const float4 *>(Tm + t * AST + sbeg + e);
+          const float4 b4 = *reinterpret_cast<const float4 *>(bet + sbeg + e);
+          const float4 g4 = *reinterpret_cast<const float4 *>(gam + sbeg + e);
+          tm[e] = a4.x; tm[e + 1] = a4.y; tm[e + 2] = a4.z; tm[e + 3] = a4.w;
+          bt[e] = b4.x; bt[e + 1] = b4.y; bt[e + 2] = b4.z; bt[e + 3] = b4.w;
+          gm[e] = g4.x; gm[e + 1] = g4.y; gm[e + 2] = g4.z; gm[e + 3] = g4.w;
         }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float m = (sbeg + e <= t) ? tm[e] : 0.f;
+          tq[e] = m * bt[e];
+          tp[e] = tq[e] * gm[e];
+        }
+        const uint32_t off = sw128_off(t, sbeg >> 3);
+        st_split8(smem + OFF_TPH + off, smem + OFF_TPL + off, tp);
+        st_split8(smem + OFF_TQH + off, smem + OFF_TQL + off, tq);
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -576,34 +634,34 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // ---- W^T -> bf16 (MN-major B)
       if (!epi_wait(bar_addr(sb, B_W), ph, etid, abort_flag, p.status)) break;
       {
-        float v[32];
-        tmem_ld32(tl + R_W + 32 * ewg, v);
+        float v[16];
+        tmem_ld16(tl + R_W + 16 * ewq, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) st_bf16x8(smem + OFF_WT + sw128_off(row, 4 * ewg + q), v + 8 * q);
+        for (int q = 0; q < 2; ++q) st_bf16x8(smem + OFF_WT + sw128_off(row, 2 * ewq + q), v + 8 * q);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(EPI_BAR, NEPI);
       if (etid == 0) mbar_arrive(bar_addr(sb, B_WT));
 
-      // ---- U^T -> hi/lo (for P) and U^T diag(kdec) -> hi/lo (for the state)
+      // ---- U^T -> hi/lo (for P) and U^T diag(kdec) -> hi/lo (for the state), into TMEM
       if (!epi_wait(bar_addr(sb, B_U), ph, etid, abort_flag, p.status)) break;
       {
-        float v[32];
-        tmem_ld32(tl + R_U + 32 * ewg, v);
+        float v[16];
+        tmem_ld16(tl + R_UO + 16 * ewq, v);
         tmem_wait_ld();
+        uint32_t hw[8], lw[8];
+        split_words<8>(v, hw, lw);
+        tmem_st8(tl + T_UH + 8 * ewq, hw);
+        tmem_st8(tl + T_UL + 8 * ewq, lw);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t off = sw128_off(row, 4 * ewg + q);
-          st_split8(smem + OFF_UH + off, smem + OFF_UL + off, v + 8 * q);
-          float uk[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) uk[e] = v[8 * q + e] * kdec[32 * ewg + 8 * q + e];
-          st_split8(smem + OFF_UKH + off, smem + OFF_UKL + off, uk);
-        }
+        for (int e = 0; e < 16; ++e) v[e] *= kdec[16 * ewq + e];
+        split_words<8>(v, hw, lw);
+        tmem_st8(tl + T_UKH + 8 * ewq, hw);
+        tmem_st8(tl + T_UKL + 8 * ewq, lw);
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(EPI_BAR, NEPI);
       if (etid == 0) mbar_arrive(bar_addr(sb, B_UT));
@@ -612,34 +670,31 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (!epi_wait(bar_addr(sb, B_S), ph, etid, abort_flag, p.status)) break;
       {
         const float gC = sc[256];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
+        {
           float v[32];
-          tmem_ld32(tl + R_S + 64 * ewg + 32 * hf, v);
+          tmem_ld32(tl + R_S + 32 * ewq, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int x = 0; x < 32; ++x) S[32 * hf + x] = fmaf(gC, S[32 * hf + x], v[x]);
+          for (int x = 0; x < 32; ++x) S[x] = fmaf(gC, S[x], v[x]);
         }
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint32_t off = ewg * 16384 + sw128_off(row, q);
-          st_split8(smem + OFF_S0H + off, smem + OFF_S0L + off, S + 8 * q);
+        {
+          uint32_t hw[16], lw[16];
+          split_words<16>(S, hw, lw);
+          tmem_st16(tl + T_S0H + 16 * ewq, hw);
+          tmem_st16(tl + T_S0L + 16 * ewq, lw);
         }
+        float vi[16], va[16];
+        tmem_ld16(tl + R_OI + 16 * ewq, vi);
+        tmem_ld16(tl + R_UO + 16 * ewq, va);
+        tmem_wait_ld();
         TO *op = static_cast<TO *>(p.o) + ((size_t)t0 * p.Hv + h) * HD + row;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          float vi[16], va[16];
-          tmem_ld16(tl + R_OI + 32 * ewg + 16 * hf, vi);
-          tmem_ld16(tl + R_OA + 32 * ewg + 16 * hf, va);
-          tmem_wait_ld();
-#pragma unroll
-          for (int x = 0; x < 16; ++x) {
-            const int t = 32 * ewg + 16 * hf + x;
-            if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(p.scale * fmaf(gam[t], vi[x], va[x]));
-          }
+        for (int x = 0; x < 16; ++x) {
+          const int t = 16 * ewq + x;
+          if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(p.scale * fmaf(gam[t], vi[x], va[x]));
         }
+        tmem_wait_st();
       }
-      fence_proxy_async_smem();
       tc_fence_before();
       named_bar_sync(EPI_BAR, NEPI);
       if (etid == 0) {
@@ -648,9 +703,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
     if (*abort_flag == 0 && p.sfin) {
-      float *dst = p.sfin + sbase + (size_t)row * HD + 64 * ewg;
+      float *dst = p.sfin + sbase + (size_t)row * HD + 32 * ewq;
 #pragma unroll
-      for (int x = 0; x < 64; x += 4)
+      for (int x = 0; x < 32; x += 4)
         *reinterpret_cast<float4 *>(dst + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
     }
   }

@@ -58,6 +58,8 @@ def load():
         lib.gdn_version.argtypes = []
         lib.gdn_prefill_workspace_size.restype = sz
         lib.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+        lib.gdn_prefill_workspace_size_rounds.restype = sz
+        lib.gdn_prefill_workspace_size_rounds.argtypes = [i32, i64, i32, i32, i32, i32, i32, i64]
         lib.gdn_prefill.restype = i32
         lib.gdn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32, i32,
                                     f32, vp, vp, vp, vp, sz, vp]
@@ -102,9 +104,16 @@ def _require(t, name, device, dtype=None, shape=None):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
-def prefill_workspace_size(num_seqs, total_tokens, Hqk, Hv, Dk, Dv, dtype=torch.bfloat16) -> int:
-    return int(load().gdn_prefill_workspace_size(num_seqs, total_tokens, Hqk, Hv, Dk, Dv,
-                                                 _DTYPE_CODE[dtype]))
+def prefill_workspace_size(num_seqs, total_tokens, Hqk, Hv, Dk, Dv, dtype=torch.bfloat16,
+                           chunks_per_round=0) -> int:
+    """Workspace bytes for prefill; ``chunks_per_round`` > 0 bounds it by
+    processing the packed chunk list in rounds of that many 64-token chunks."""
+    lib = load()
+    if chunks_per_round:
+        return int(lib.gdn_prefill_workspace_size_rounds(num_seqs, total_tokens, Hqk, Hv, Dk, Dv,
+                                                         _DTYPE_CODE[dtype], chunks_per_round))
+    return int(lib.gdn_prefill_workspace_size(num_seqs, total_tokens, Hqk, Hv, Dk, Dv,
+                                              _DTYPE_CODE[dtype]))
 
 
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_state=True,

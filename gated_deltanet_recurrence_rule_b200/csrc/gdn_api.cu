@@ -24,6 +24,14 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
                               const float *beta, const int32_t *cu, int N, long long T_,
                               int Hqk, int Hv, int o_dtype, float scale, const float *s0,
                               float *sfin, void *o, void *workspace, cudaStream_t stream);
+size_t twophase_workspace_bytes(int64_t N, int64_t T, int Hv);
+size_t twophase_round_workspace_bytes(int64_t N, int Hv, int64_t chunks_per_round);
+size_t twophase_min_workspace_bytes(int64_t N, int Hv);
+cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const int32_t *cu, int N, long long T_,
+                                    int Hqk, int Hv, int o_dtype, float scale, const float *s0,
+                                    float *sfin, void *o, void *workspace, size_t workspace_bytes,
+                                    cudaStream_t stream);
 }  // namespace gdn
 
 namespace {
@@ -48,6 +56,16 @@ int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_
 
 }  // namespace
 
+namespace gdn {
+// Smallest workspace gdn_prefill accepts for these sizes (the status header;
+// bf16 D=128 then runs the single-pass kernel), 0 for invalid sizes.
+size_t prefill_min_workspace_bytes(int32_t num_seqs, int64_t total_tokens, int32_t Hqk, int32_t Hv,
+                                   int32_t Dk, int32_t Dv, int32_t dtype) {
+  if (num_seqs < 0 || total_tokens < 0 || !dims_ok(Hqk, Hv, Dk, Dv, dtype)) return 0;
+  return kWorkspaceHeaderBytes;
+}
+}  // namespace gdn
+
 extern "C" {
 
 const char *gdn_status_string(int32_t status) {
@@ -70,7 +88,23 @@ size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
                                   int32_t dtype) {
   if (num_seqs < 0 || total_tokens < 0) return 0;
   if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return 0;
+  if (gdn::prefill_tc_supported(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype))
+    return gdn::twophase_workspace_bytes(num_seqs, total_tokens, num_v_heads);
   return gdn::kWorkspaceHeaderBytes;
+}
+
+size_t gdn_prefill_workspace_size_rounds(int32_t num_seqs, int64_t total_tokens,
+                                         int32_t num_qk_heads, int32_t num_v_heads,
+                                         int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                                         int64_t chunks_per_round) {
+  const size_t full = gdn_prefill_workspace_size(num_seqs, total_tokens, num_qk_heads, num_v_heads,
+                                                 head_dim_k, head_dim_v, dtype);
+  if (full == 0 || chunks_per_round < 0) return 0;
+  if (chunks_per_round == 0 ||
+      !gdn::prefill_tc_supported(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype))
+    return full;
+  const size_t r = gdn::twophase_round_workspace_bytes(num_seqs, num_v_heads, chunks_per_round);
+  return r < full ? r : full;
 }
 
 int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
@@ -93,9 +127,8 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
   }
   if ((initial_state && !aligned(initial_state, 16)) || (final_state && !aligned(final_state, 16)))
     return GDN_ERR_INVALID_ARG;
-  const size_t need = gdn_prefill_workspace_size(num_seqs, total_tokens, num_qk_heads,
-                                                 num_v_heads, head_dim_k, head_dim_v, dtype);
-  if (!workspace || !aligned(workspace, 256) || workspace_bytes < need) return GDN_ERR_WORKSPACE;
+  if (!workspace || !aligned(workspace, 256) || workspace_bytes < gdn::kWorkspaceHeaderBytes)
+    return GDN_ERR_WORKSPACE;
   // grid-size limits of the launches below
   if ((int64_t)num_seqs * num_v_heads * 4 > INT32_MAX) return GDN_ERR_UNSUPPORTED;
 
@@ -103,9 +136,17 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
   int32_t *status = static_cast<int32_t *>(workspace);
   cudaError_t e;
   if (gdn::prefill_tc_supported(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) {
-    e = gdn::launch_prefill_tc(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_qk_heads,
-                               num_v_heads, o_dtype, scale, initial_state, final_state, o,
-                               workspace, s);
+    if (workspace_bytes >= gdn::twophase_min_workspace_bytes(num_seqs, num_v_heads)) {
+      // two phases: every chunk's state-free products at once, then the state pass
+      e = gdn::launch_prefill_twophase(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
+                                       num_qk_heads, num_v_heads, o_dtype, scale, initial_state,
+                                       final_state, o, workspace, workspace_bytes, s);
+    } else {
+      // a header-only workspace: one pass, each CTA does all of a (sequence, head)
+      e = gdn::launch_prefill_tc(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
+                                 num_qk_heads, num_v_heads, o_dtype, scale, initial_state,
+                                 final_state, o, workspace, s);
+    }
   } else {
     e = gdn::launch_prefill_simt(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
                                  num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype,

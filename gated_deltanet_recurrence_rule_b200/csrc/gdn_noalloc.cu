@@ -1,8 +1,9 @@
 // gdn_noalloc.cu -- gdn_prefill_noalloc: the prefill entry point for callers
 // that cannot allocate device memory.
 //
-// gdn_prefill needs a small device workspace (its status word and scheduler
-// header).  Some callers cannot call cudaMalloc to get one: code that runs
+// gdn_prefill needs a device workspace: at least its status header (then the
+// bf16 head-dim-128 case runs the single-pass kernel), more for the faster
+// two-phase kernels.  Some callers cannot call cudaMalloc to get one: code that runs
 // where the device allocator belongs to someone else (a framework's caching
 // allocator, a serving runtime's memory pool), real-time paths that must not
 // take cudaMalloc's implicit device-wide synchronisation, and plugins that are
@@ -15,6 +16,11 @@
 #include <mutex>
 
 #include "gdn.h"
+
+namespace gdn {
+size_t prefill_min_workspace_bytes(int32_t num_seqs, int64_t total_tokens, int32_t Hqk, int32_t Hv,
+                                   int32_t Dk, int32_t Dv, int32_t dtype);
+}  // namespace gdn
 
 namespace {
 
@@ -51,8 +57,8 @@ extern "C" int32_t gdn_prefill_noalloc(const void *q, const void *k, const void 
                                        int32_t o_dtype, float scale, const float *initial_state,
                                        float *final_state, void *o, int32_t *device_status,
                                        void *stream) {
-  const size_t need = gdn_prefill_workspace_size(num_seqs, total_tokens, num_qk_heads,
-                                                 num_v_heads, head_dim_k, head_dim_v, dtype);
+  const size_t need = gdn::prefill_min_workspace_bytes(num_seqs, total_tokens, num_qk_heads,
+                                                       num_v_heads, head_dim_k, head_dim_v, dtype);
   if (need > kScratchBytes) return GDN_ERR_WORKSPACE;  // beyond the built-in scratch
   void *scratch = nullptr;
   const int32_t st = scratch_address(&scratch);

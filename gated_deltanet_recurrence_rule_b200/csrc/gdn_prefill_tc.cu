@@ -46,13 +46,16 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "gdn_chunk_ops.cuh"
 #include "gdn_common.cuh"
 #include "gdn_sm100.cuh"
+#include "gdn_twophase.cuh"
 
 namespace gdn {
 namespace tc {
 
 using namespace sm100;
+using namespace chunk;
 
 constexpr int CH = 64;            // chunk length
 constexpr int HD = 128;           // head dim (Dk = Dv)
@@ -89,7 +92,6 @@ constexpr uint32_t SCAL_STAGE = 5 * 64 * 4;  // G2 (log2 prefix), gamma, kdec, b
 constexpr uint32_t OFF_BAR = OFF_SCAL + 2 * SCAL_STAGE;
 constexpr uint32_t OFF_MISC = OFF_BAR + 192;  // [0] TMEM base, [4] abort flag, [8] drain mbarrier
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
-constexpr int AST = 68;  // fp32 row stride of A and Tm (conflict-free float4 row stores)
 static_assert(OFF_R1 % 1024 == 0 && OFF_PH % 1024 == 0 && OFF_V % 1024 == 0, "alignment");
 static_assert(OFF_Y + 3 * 16 * 17 * 4 <= OFF_R1 + R1_BYTES, "R1 layout");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -133,165 +135,9 @@ struct Params {
 
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sb, int i) { return sb + OFF_BAR + 8u * i; }
 
-// ---- warp-level m16n8k8 tf32 MMAs with a 3-term split (x = hi + lo, hi =
-// tf32(x)): hi*hi + hi*lo + lo*hi carries ~fp32 accuracy.
-__device__ __forceinline__ uint32_t to_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return r;
-}
-__device__ __forceinline__ void mma_tf32_16x8x8(float *d, const uint32_t *a, const uint32_t *b) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
-}
-// D (16x8 fp32, fragment layout) = X (16 x 8 KS, row-major, stride ldx) *
-// Y (8 KS x 8, row-major, stride ldy), with the 3-term split.
-template <int KS>
-__device__ __forceinline__ void mma3_16x8(float *d, const float *X, int ldx, const float *Y, int ldy,
-                                          int lane) {
-  const int gid = lane >> 2, tig = lane & 3;
-  float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int ks = 0; ks < KS; ++ks) {
-    const float a0 = X[gid * ldx + 8 * ks + tig], a1 = X[(gid + 8) * ldx + 8 * ks + tig];
-    const float a2 = X[gid * ldx + 8 * ks + tig + 4], a3 = X[(gid + 8) * ldx + 8 * ks + tig + 4];
-    const float b0 = Y[(8 * ks + tig) * ldy + gid], b1 = Y[(8 * ks + tig + 4) * ldy + gid];
-    const uint32_t ah[4] = {to_tf32(a0), to_tf32(a1), to_tf32(a2), to_tf32(a3)};
-    const uint32_t al[4] = {to_tf32(a0 - __uint_as_float(ah[0])), to_tf32(a1 - __uint_as_float(ah[1])),
-                            to_tf32(a2 - __uint_as_float(ah[2])), to_tf32(a3 - __uint_as_float(ah[3]))};
-    const uint32_t bh[2] = {to_tf32(b0), to_tf32(b1)};
-    const uint32_t bl[2] = {to_tf32(b0 - __uint_as_float(bh[0])), to_tf32(b1 - __uint_as_float(bh[1]))};
-    mma_tf32_16x8x8(d, ah, bh);
-    mma_tf32_16x8x8(d1, ah, bl);
-    mma_tf32_16x8x8(d2, al, bh);
-  }
-#pragma unroll
-  for (int e = 0; e < 4; ++e) d[e] += d1[e] + d2[e];
-}
-__device__ __forceinline__ void st_frag16x8(float *M, int ld, const float *d, float scale, int lane) {
-  const int gid = lane >> 2, tig = lane & 3;
-  M[gid * ld + 2 * tig] = scale * d[0];
-  M[gid * ld + 2 * tig + 1] = scale * d[1];
-  M[(gid + 8) * ld + 2 * tig] = scale * d[2];
-  M[(gid + 8) * ld + 2 * tig + 1] = scale * d[3];
-}
-
-// Off-diagonal blocks at block distance DIST (1..3) of the inverse: for the
-// 4 - DIST blocks (i, j = i - DIST), Y_ij = sum_{j<=k<i} A_ik Tm_kj (one
-// 16 x 16 DIST x 16 product), then Tm_ij = -Tm_ii Y_ij (16 x 16 x 16).  One warp
-// per (block, 8-column half) on the tensor cores (warp-level mma.sync).
-template <int DIST>
-__device__ __forceinline__ void ut_distance(const float *__restrict__ A, float *__restrict__ Tm,
-                                            float *__restrict__ Y, int etid) {
-  constexpr int NB = 4 - DIST;
-  const int w = etid >> 5, lane = etid & 31;
-  if (w < 2 * NB) {
-    const int j = w >> 1, i = j + DIST, nh = w & 1;
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    mma3_16x8<2 * DIST>(d, A + 16 * i * AST + 16 * j, AST, Tm + 16 * j * AST + 16 * j + 8 * nh, AST, lane);
-    st_frag16x8(Y + (j * 16) * 17 + 8 * nh, 17, d, 1.f, lane);
-  }
-  named_bar_sync(EPI_BAR, NEPI);
-  if (w < 2 * NB) {
-    const int j = w >> 1, i = j + DIST, nh = w & 1;
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    mma3_16x8<2>(d, Tm + 16 * i * AST + 16 * i, AST, Y + (j * 16) * 17 + 8 * nh, 17, lane);
-    st_frag16x8(Tm + 16 * i * AST + 16 * j + 8 * nh, AST, d, -1.f, lane);
-  }
-  named_bar_sync(EPI_BAR, NEPI);
-}
-
-// Unit lower-triangular inverse Tm = (I + A)^-1 of a 64x64 strictly lower A,
-// fp32, by the epilogue threads.  The four 16x16 diagonal blocks by forward
-// substitution (four warps per block, eight lanes per column, each lane two
-// rows with their A entries in registers), then the off-diagonal blocks by
-// block distance 1, 2, 3 (each needs only blocks of smaller distance).
-__device__ __forceinline__ void ut_solve(const float *__restrict__ A, float *__restrict__ Tm,
-                                         float *__restrict__ Y, int etid) {
-  {
-    const int ew = etid >> 5, lane = etid & 31;
-    const int b = ew >> 2, c = 4 * (ew & 3) + (lane >> 3), q = lane & 7;
-    float a[2][16];
-#pragma unroll
-    for (int m = 0; m < 2; ++m)
-#pragma unroll
-      for (int s4 = 0; s4 < 16; s4 += 4) {
-        const float4 v4 = *reinterpret_cast<const float4 *>(A + (16 * b + q + 8 * m) * AST + 16 * b + s4);
-        a[m][s4] = v4.x; a[m][s4 + 1] = v4.y; a[m][s4 + 2] = v4.z; a[m][s4 + 3] = v4.w;
-      }
-    float x[2];
-#pragma unroll
-    for (int m = 0; m < 2; ++m) x[m] = (q + 8 * m == c) ? 1.f : 0.f;
-#pragma unroll
-    for (int s = 0; s < 16; ++s) {
-      const float xs = __shfl_sync(0xffffffffu, x[s >> 3], (lane & ~7) | (s & 7));
-#pragma unroll
-      for (int m = 0; m < 2; ++m)
-        if (q + 8 * m > s) x[m] = fmaf(-a[m][s], xs, x[m]);
-    }
-#pragma unroll
-    for (int m = 0; m < 2; ++m) Tm[(16 * b + q + 8 * m) * AST + 16 * b + c] = x[m];
-  }
-  named_bar_sync(EPI_BAR, NEPI);
-  ut_distance<1>(A, Tm, Y, etid);
-  ut_distance<2>(A, Tm, Y, etid);
-  ut_distance<3>(A, Tm, Y, etid);
-}
-
-// One waiter (epilogue thread 0) for an mbarrier phase, then a named barrier;
-// returns false on abort (then every epilogue thread returns false).
 __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, int etid,
                                          volatile int *abort, int32_t *status) {
-  if (etid == 0) {
-    if (!mbar_wait(bar, parity, abort)) {
-      *abort = 1;
-      report_status(status, GDN_ERR_DEVICE_TIMEOUT);
-    }
-  }
-  named_bar_sync(EPI_BAR, NEPI);
-  const bool ok = (*abort == 0);
-  if (ok) tc_fence_after();
-  return ok;
-}
-
-// 8 consecutive fp32 values -> one 16-byte chunk of bf16 at `dst`.
-__device__ __forceinline__ void st_bf16x8(unsigned char *dst, const float *x) {
-  *reinterpret_cast<uint4 *>(dst) = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]),
-                                               pack_bf16x2(x[4], x[5]), pack_bf16x2(x[6], x[7]));
-}
-// 8 fp32 values x -> x = hi + lo with hi = x truncated to bf16 (high 16 bits)
-// and lo = (x - hi) truncated to bf16; |x - hi - lo| < 2^-14 |x|.  Bit
-// operations only (mask, subtract, byte permute), no conversion instructions.
-__device__ __forceinline__ void st_split8(unsigned char *dst_hi, unsigned char *dst_lo,
-                                          const float *x) {
-  uint32_t hw[4], lw[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const uint32_t a = __float_as_uint(x[2 * e]), b = __float_as_uint(x[2 * e + 1]);
-    const float ra = x[2 * e] - __uint_as_float(a & 0xffff0000u);
-    const float rb = x[2 * e + 1] - __uint_as_float(b & 0xffff0000u);
-    hw[e] = __byte_perm(a, b, 0x7632);
-    lw[e] = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
-  }
-  *reinterpret_cast<uint4 *>(dst_hi) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-  *reinterpret_cast<uint4 *>(dst_lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-}
-
-// 2n fp32 values -> packed bf16 pairs hw[n] = hi(x), lw[n] = lo(x) with the
-// same truncation split as st_split8 (for tcgen05.st into TMEM operands).
-template <int NP>
-__device__ __forceinline__ void split_words(const float *x, uint32_t *hw, uint32_t *lw) {
-#pragma unroll
-  for (int e = 0; e < NP; ++e) {
-    const uint32_t a = __float_as_uint(x[2 * e]), b = __float_as_uint(x[2 * e + 1]);
-    const float ra = x[2 * e] - __uint_as_float(a & 0xffff0000u);
-    const float rb = x[2 * e + 1] - __uint_as_float(b & 0xffff0000u);
-    hw[e] = __byte_perm(a, b, 0x7632);
-    lw[e] = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
-  }
+  return group_wait<NEPI, EPI_BAR>(bar, parity, etid, abort, status);
 }
 
 template <typename TO>
@@ -603,7 +449,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       named_bar_sync(EPI_BAR, NEPI);
 
       // ---- Tm = (I + A)^-1, then T' = Tm diag(beta gamma), T'' = Tm diag(beta), split
-      ut_solve(A, Tm, Y, etid);
+      ut_solve<NEPI, EPI_BAR>(A, Tm, Y, etid);
       {
         const int t = etid >> 3, sbeg = 8 * (etid & 7);
         float tm[8], bt[8], gm[8], tp[8], tq[8];
@@ -718,42 +564,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
 }
 
-using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  if (!fn) {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(ptr);
-  }
-  return fn;
-}
-
-// [T, H, 128] bf16 viewed as a 3-D tensor (d, head, token); box 64 d x 1 head x 64 tokens.
-static bool make_map(CUtensorMap *m, const void *base, int H, int T) {
-  EncodeFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)H, (cuuint64_t)T};
-  const cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)H * HD * 2};
-  const cuuint32_t box[3] = {64, 1, CH};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename TO>
 static cudaError_t launch_t(const void *q, const void *k, const void *v, const Params &prm,
                             cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, q, prm.Hqk, prm.T) || !make_map(&mk, k, prm.Hqk, prm.T) ||
-      !make_map(&mv, v, prm.Hv, prm.T))
+  if (!make_qkv_map(&mq, q, prm.Hqk, prm.T) || !make_qkv_map(&mk, k, prm.Hqk, prm.T) ||
+      !make_qkv_map(&mv, v, prm.Hv, prm.T))
     return cudaErrorInvalidValue;
   auto kern = prefill_tc_kernel<TO>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);

@@ -1,0 +1,574 @@
+// gdn_state_pass.cu -- phase 2 of the two-phase tensor-core prefill (the
+// inter-chunk state passing), the plan kernel that maps packed sequences to
+// global chunks, and the host driver of the two phases.
+//
+// Per (sequence, value head), chunk after chunk, with the state-free record of
+// each chunk already computed by phase 1 (gdn_wy_prep.cu):
+//     U^T  = U~^T - S0 W^T                     (M128 N64 K128; U~ added in the epilogue)
+//     Oi^T = S0 Q^T,   Oa^T = U^T P^T,   o_t = scale (e^{G_t} Oi_t + Oa_t)
+//     dS   = (U diag(e^{G_C - G}))^T K,   S <- e^{G_C} S + dS   (fp32 master copy)
+// ("Inside Qwen3.8-27B: Hybrid DeltaNet Architecture, 256k Context, and 24GB
+// Local Serving", section "Gated DeltaNet Mechanics": o_t = S_t q_t with the
+// fixed-size state kept on chip.)  The state lives in registers of the 512
+// epilogue threads (fp32) and as hi + lo bf16 operands in TMEM; only o and
+// the final state leave the SM.  The critical path of a chunk is
+//     S0 ready -> U MMA -> U epilogue -> dS MMA -> state epilogue -> S0 ready,
+// and the output MMAs (Oi, Oa) fill the tensor pipe around it.
+//
+// Packed sequences are mapped to one list of global chunks (chunks aligned to
+// each sequence start).  A workspace that cannot hold every chunk's record is
+// used in rounds of RC global chunks: phase 1 then phase 2 per round; the one
+// sequence that crosses a round boundary carries its state through the
+// workspace.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "gdn_chunk_ops.cuh"
+#include "gdn_common.cuh"
+#include "gdn_sm100.cuh"
+#include "gdn_twophase.cuh"
+
+namespace gdn {
+
+size_t wy_prep_smem_bytes();
+cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                           const float *g, const float *beta, const int32_t *cu, int T, int Hqk,
+                           int Hv, int round, int rc, const void *workspace,
+                           const tp::Layout &L, cudaStream_t stream);
+
+namespace plan {
+
+// One CTA: validates cu_seqlens, lists the non-empty sequences with the first
+// global chunk of each (exclusive scan of ceil(L_n / 64)), and writes the
+// final state of every empty sequence (= its initial state, or zeros).  Bad
+// cu_seqlens set GDN_ERR_BAD_SEQLENS and leave zero chunks to process.
+__global__ void __launch_bounds__(1024)
+plan_kernel(const int32_t *__restrict__ cu, int N, int T, int Hv, const float *__restrict__ s0,
+            float *__restrict__ sfin, tp::PlanHeader *ph, int32_t *ne_seq, int32_t *ne_cs,
+            int32_t *status) {
+  __shared__ int s_bad, s_run_ne, s_run_ch, s_nempty;
+  __shared__ int w_ne[32], w_ch[32];
+  __shared__ int s_empty[1024];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  if (tid == 0) { s_bad = 0; s_run_ne = 0; s_run_ch = 0; }
+  __syncthreads();
+  for (int i = tid; i <= N; i += blockDim.x) {
+    const int c = cu[i];
+    bool bad = c < 0 || c > T || (i == 0 && c != 0) || (i == N && c != T);
+    if (i < N && cu[i + 1] < c) bad = true;
+    if (bad) atomicOr(&s_bad, 1);
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (tid == 0) {
+      report_status(status, GDN_ERR_BAD_SEQLENS);
+      ph->n_nonempty = 0;
+      ph->total_chunks = 0;
+    }
+    return;
+  }
+  const size_t state_elems = (size_t)Hv * 128 * 128;
+  for (int base = 0; base < N; base += blockDim.x) {
+    const int n = base + tid;
+    const int L = n < N ? cu[n + 1] - cu[n] : 0;
+    const int ne = L > 0 ? 1 : 0, nc = (L + 63) / 64;
+    int ie = ne, ic = nc;  // warp-inclusive scans
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int xe = __shfl_up_sync(0xffffffffu, ie, off), xc = __shfl_up_sync(0xffffffffu, ic, off);
+      if (lane >= off) { ie += xe; ic += xc; }
+    }
+    if (lane == 31) { w_ne[wid] = ie; w_ch[wid] = ic; }
+    if (tid == 0) s_nempty = 0;
+    __syncthreads();
+    if (wid == 0) {
+      int ve = w_ne[lane], vc = w_ch[lane];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int xe = __shfl_up_sync(0xffffffffu, ve, off), xc = __shfl_up_sync(0xffffffffu, vc, off);
+        if (lane >= off) { ve += xe; vc += xc; }
+      }
+      w_ne[lane] = ve - w_ne[lane];  // exclusive warp offsets
+      w_ch[lane] = vc - w_ch[lane];
+    }
+    __syncthreads();
+    const int pe = s_run_ne + w_ne[wid] + ie - ne, pc = s_run_ch + w_ch[wid] + ic - nc;
+    if (ne) { ne_seq[pe] = n; ne_cs[pe] = pc; }
+    if (n < N && !ne && sfin) s_empty[atomicAdd(&s_nempty, 1)] = n;
+    __syncthreads();
+    if (tid == blockDim.x - 1) { s_run_ne = pe + ne; s_run_ch = pc + nc; }
+    // final state of the empty sequences of this tile = initial state (or 0)
+    for (int e = 0; e < s_nempty; ++e) {
+      const size_t off = (size_t)s_empty[e] * state_elems;
+      float4 *dst = reinterpret_cast<float4 *>(sfin + off);
+      const float4 *src = s0 ? reinterpret_cast<const float4 *>(s0 + off) : nullptr;
+      for (size_t x = tid; x < state_elems / 4; x += blockDim.x)
+        dst[x] = src ? src[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    ne_cs[s_run_ne] = s_run_ch;
+    ph->n_nonempty = s_run_ne;
+    ph->total_chunks = s_run_ch;
+  }
+}
+
+}  // namespace plan
+
+namespace sp {
+
+using namespace sm100;
+using namespace chunk;
+using tp::CH;
+using tp::HD;
+using tp::REC_BYTES;
+
+constexpr int NTHREADS = 640;
+constexpr int NEPI = 512;   // 4 column quarters x 128 rows
+constexpr int EPI_BAR = 1;
+
+// ---- shared memory map (bytes) ----
+constexpr int NQK = 2, NR = 2;         // ring depths: Q/K tiles, chunk records
+constexpr uint32_t QK_STAGE = 32768;   // [Q d0-63 | K d0-63 | Q d64-127 | K d64-127], 64 rows x 128 B each
+constexpr uint32_t OFF_QK = 0;
+constexpr uint32_t OFF_REC = NQK * QK_STAGE;
+constexpr uint32_t OFF_BAR = OFF_REC + NR * REC_BYTES;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;  // [0] TMEM base, [4] abort flag, [8] drain mbarrier
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+static_assert(OFF_REC % 1024 == 0 && REC_BYTES % 1024 == 0, "alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+enum {
+  B_FULL_QK = 0, B_EMPTY_QK = B_FULL_QK + NQK, B_FULL_R = B_EMPTY_QK + NQK, B_EMPTY_R = B_FULL_R + NR,
+  B_S0 = B_EMPTY_R + NR, B_U, B_UT, B_S, B_OA, B_OFREE, NBAR
+};
+static_assert(NBAR * 8 <= 256, "barrier area");
+
+// ---- TMEM columns (128 lanes x 512 columns of 32 bit) ----
+constexpr uint32_t R_S = 0;     // 128: U^T - U~^T in [0, 64) (chunk start), then dS (chunk end)
+constexpr uint32_t R_OI = 128;  // 64: S0 Q^T
+constexpr uint32_t R_OA = 192;  // 64: U^T P^T
+// MMA A operands in TMEM (bf16 pairs per column; lane = row of the operand).
+constexpr uint32_t T_S0H = 256, T_S0L = 320;  // hi/lo(S0): 128 rows x 128 K
+constexpr uint32_t T_UH = 384, T_UL = 416;    // hi/lo(U^T): 128 rows x 64 K
+constexpr uint32_t T_UKH = 448, T_UKL = 480;  // hi/lo(U^T diag(kdec))
+constexpr uint32_t TMEM_COLS = 512;
+
+constexpr uint32_t IDESC_SW = idesc_bf16(128, 64, 0, 1, 1);  // -S0 W^T
+constexpr uint32_t IDESC_SQ = idesc_bf16(128, 64, 0, 0);     // S0 Q^T, U^T P^T
+constexpr uint32_t IDESC_UK = idesc_bf16(128, 128, 0, 1);    // Ukdec^T K
+
+struct Params {
+  const int32_t *cu;
+  int N, Hqk, Hv;
+  int round, rc;
+  float scale;
+  const float *s0;
+  float *sfin;
+  void *o;
+  const tp::PlanHeader *plan;
+  const int32_t *ne_seq, *ne_cs;
+  const unsigned char *rec;  // this round's records, [rc][Hv]
+  float *carry;              // [2][Hv][128][128]
+  int32_t *status;
+};
+
+__device__ __forceinline__ uint32_t bar_addr(uint32_t sb, int i) { return sb + OFF_BAR + 8u * i; }
+
+template <typename TO>
+__global__ void __launch_bounds__(NTHREADS, 1)
+state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const Params p) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y;
+  // ---- which sequence and which of its chunks this CTA owns in this round
+  const int n_ne = p.plan->n_nonempty, total = p.plan->total_chunks;
+  const int g_lo = p.round * p.rc, g_hi = min(g_lo + p.rc, total);
+  if (g_lo >= g_hi) return;
+  const int kseq = tp::owner_of_chunk(p.ne_cs, n_ne, g_lo) + (int)blockIdx.x;
+  if (kseq >= n_ne) return;
+  const int cs = p.ne_cs[kseq], ce = p.ne_cs[kseq + 1];
+  if (cs >= g_hi) return;
+  const int ga = max(cs, g_lo), gb = min(ce, g_hi);
+  const int nch = gb - ga;
+  const int n = p.ne_seq[kseq];
+  const int j = h / (p.Hv / p.Hqk);
+  const int seq_begin = p.cu[n], seq_end = p.cu[n + 1];
+  const size_t hstate = (size_t)HD * HD;
+  const size_t sbase = ((size_t)n * p.Hv + h) * hstate;
+  const float *src = (ga == cs) ? (p.s0 ? p.s0 + sbase : nullptr)
+                                : p.carry + ((size_t)((p.round - 1) & 1) * p.Hv + h) * hstate;
+  float *dst = (gb == ce) ? (p.sfin ? p.sfin + sbase : nullptr)
+                          : p.carry + ((size_t)(p.round & 1) * p.Hv + h) * hstate;
+
+  const uint32_t sb = smem_addr(smem);
+  if (sb & 1023u) {  // swizzled operand tiles need 1024-byte alignment
+    if (tid == 0) report_status(p.status, GDN_ERR_UNSUPPORTED);
+    return;
+  }
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  if (tid == 0) {
+    for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
+    // a record slot is free once its MMAs completed AND the epilogue read it
+    for (int i = 0; i < NR; ++i) mbar_init(bar_addr(sb, B_EMPTY_R + i), 2);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(sb + OFF_MISC, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + OFF_MISC);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      prefetch_tensormap(&tm_q);
+      prefetch_tensormap(&tm_k);
+      constexpr int PF = 4;  // L2 prefetch distance in chunks
+      auto chunk_t0 = [&](int c) { return seq_begin + (ga - cs + c) * CH; };
+      auto chunk_rec = [&](int c) {
+        return p.rec + ((size_t)(ga + c - g_lo) * p.Hv + h) * REC_BYTES;
+      };
+      for (int c = 0; c < PF && c < nch; ++c) {
+        const int t = chunk_t0(c);
+        tma_prefetch_3d(&tm_q, 0, j, t); tma_prefetch_3d(&tm_q, 64, j, t);
+        tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
+        bulk_prefetch_l2(chunk_rec(c), REC_BYTES);
+      }
+      int issued_qk = 0, issued_r = 0;
+      for (int c = 0; c < nch; ++c) {
+        const int s = c % NQK, sr = c % NR;
+        const int t0 = chunk_t0(c);
+        if (c + PF < nch) {
+          const int t = chunk_t0(c + PF);
+          tma_prefetch_3d(&tm_q, 0, j, t); tma_prefetch_3d(&tm_q, 64, j, t);
+          tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
+          bulk_prefetch_l2(chunk_rec(c + PF), REC_BYTES);
+        }
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag)) break;
+        const uint32_t st = sb + OFF_QK + s * QK_STAGE;
+        const uint32_t fb = bar_addr(sb, B_FULL_QK + s);
+        mbar_arrive_expect_tx(fb, QK_STAGE);
+        tma_load_3d(st + 0, &tm_q, fb, 0, j, t0);
+        tma_load_3d(st + 16384, &tm_q, fb, 64, j, t0);
+        tma_load_3d(st + 8192, &tm_k, fb, 0, j, t0);
+        tma_load_3d(st + 24576, &tm_k, fb, 64, j, t0);
+        issued_qk = c + 1;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_R + sr), ((c / NR) & 1) ^ 1, abort_flag)) break;
+        const uint32_t fr = bar_addr(sb, B_FULL_R + sr);
+        mbar_arrive_expect_tx(fr, REC_BYTES);
+        bulk_load(sb + OFF_REC + sr * REC_BYTES, chunk_rec(c), REC_BYTES, fr);
+        issued_r = c + 1;
+      }
+      if (issued_qk < nch || issued_r < nch) {
+        *abort_flag = 1;
+        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+      }
+      // Every load this thread issued lands before the CTA can exit (each
+      // buffer's latest fill; earlier fills were consumed before it was issued).
+      for (int c = max(issued_qk - NQK, 0); c < issued_qk; ++c)
+        mbar_wait_landed(bar_addr(sb, B_FULL_QK + c % NQK), (c / NQK) & 1, 50000000ull);
+      for (int c = max(issued_r - NR, 0); c < issued_r; ++c)
+        mbar_wait_landed(bar_addr(sb, B_FULL_R + c % NR), (c / NR) & 1, 50000000ull);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t dQK0 = sdesc_sw128(sb + OFF_QK, 16, 1024);            // Q, K-major
+      const uint64_t dKmn0 = sdesc_sw128(sb + OFF_QK + 8192, 16384, 1024); // K as MN-major operand
+      const uint64_t dW0 = sdesc_sw128(sb + OFF_REC + tp::REC_WT, 8192, 1024);  // W^T, MN-major
+      const uint64_t dP0 = sdesc_sw128(sb + OFF_REC + tp::REC_PH, 16, 1024);    // P hi / lo, K-major
+      bool ok = true;
+      for (int c = 0; c < nch && ok; ++c) {
+        const int s = c % NQK, sr = c % NR;
+        const uint32_t ph = c & 1;
+        const uint64_t dQK = dQK0 + s * (QK_STAGE >> 4), dKmn = dKmn0 + s * (QK_STAGE >> 4);
+        const uint64_t dW = dW0 + sr * (REC_BYTES >> 4), dP = dP0 + sr * (REC_BYTES >> 4);
+        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), (c / NQK) & 1, abort_flag) &&
+             mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag) &&
+             mbar_wait(bar_addr(sb, B_S0), ph, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        // U^T - U~^T = -S0h W^T   (S0 from TMEM)
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          mma_bf16_ts(tmem + R_S, tmem + T_S0H + 8 * ks, dW + ((ks * 2048) >> 4), IDESC_SW, ks > 0);
+        mma_commit(bar_addr(sb, B_U));
+        // Oi^T = (S0h + S0l) Q^T, once the previous chunk's outputs were read
+        if (c > 0 && !(ok = mbar_wait(bar_addr(sb, B_OFREE), (c - 1) & 1, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 16; ++ks) {
+          const int k = ks >> 1;
+          const uint32_t k16 = ((k >> 2) * 16384 + (k & 3) * 32) >> 4;
+          mma_bf16_ts(tmem + R_OI, tmem + ((ks & 1) ? T_S0L : T_S0H) + 8 * k, dQK + k16, IDESC_SQ,
+                      ks > 0);
+        }
+        // dS = (Ukh + Ukl)^T K ;  Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T   (U from TMEM)
+        if (!(ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const int kk = ks >> 1;
+          mma_bf16_ts(tmem + R_S, tmem + ((ks & 1) ? T_UKL : T_UKH) + 8 * kk,
+                      dKmn + ((kk * 2048) >> 4), IDESC_UK, ks > 0);
+        }
+        mma_commit(bar_addr(sb, B_S));
+#pragma unroll
+        for (int ks = 0; ks < 12; ++ks) {
+          const int part = ks % 3, kk = ks / 3;  // (Uh,Ph), (Ul,Ph), (Uh,Pl)
+          const uint32_t bo = ((part == 2 ? tp::REC_PL - tp::REC_PH : 0) + kk * 32) >> 4;
+          mma_bf16_ts(tmem + R_OA, tmem + (part == 1 ? T_UL : T_UH) + 8 * kk, dP + bo, IDESC_SQ,
+                      ks > 0);
+        }
+        mma_commit(bar_addr(sb, B_OA));
+        mma_commit(bar_addr(sb, B_EMPTY_QK + s));
+        mma_commit(bar_addr(sb, B_EMPTY_R + sr));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+      }
+      // Drain: every MMA this thread issued finishes before TMEM is freed.
+      const uint32_t drain = sb + OFF_MISC + 8;
+      mbar_init(drain, 1);
+      fence_barrier_init();
+      mma_commit(drain);
+      mbar_wait_landed(drain, 0, 50000000ull);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ epilogue
+    const int etid = tid - 128;
+    const int ewq = etid >> 7;   // column quarter
+    const int row = etid & 127;  // TMEM lane = row (Dv index) of the 128-row tiles
+    const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+
+    // fp32 master state: row `row`, columns [32 ewq, 32 ewq + 32); S0 = hi + lo in TMEM
+    float S[32];
+    {
+      const float *srow = src ? src + (size_t)row * HD + 32 * ewq : nullptr;
+#pragma unroll
+      for (int x = 0; x < 32; x += 4) {
+        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (srow) v4 = *reinterpret_cast<const float4 *>(srow + x);
+        S[x] = v4.x; S[x + 1] = v4.y; S[x + 2] = v4.z; S[x + 3] = v4.w;
+      }
+      uint32_t hw[16], lw[16];
+      split_words<16>(S, hw, lw);
+      tmem_st16(tl + T_S0H + 16 * ewq, hw);
+      tmem_st16(tl + T_S0L + 16 * ewq, lw);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    named_bar_sync(EPI_BAR, NEPI);
+    if (etid == 0) mbar_arrive(bar_addr(sb, B_S0));
+
+    bool ok = true;
+    for (int c = 0; c < nch; ++c) {
+      const int sr = c % NR;
+      const uint32_t ph = c & 1;
+      const int t0 = seq_begin + (ga - cs + c) * CH;
+      const int Lc = min(CH, seq_end - t0);
+      const unsigned char *rb = smem + OFF_REC + sr * REC_BYTES;
+      const float *gam = reinterpret_cast<const float *>(rb + tp::REC_SC);
+      const float *kdec = gam + 64;
+
+      // ---- U = (U - U~) + U~  ->  hi/lo(U^T) and hi/lo(U^T diag(kdec)) into TMEM
+      if (etid == 0 && !mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag)) {
+        *abort_flag = 1;
+        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+      }
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_U), ph, etid, abort_flag, p.status))) break;
+      {
+        float v[16];
+        tmem_ld16(tl + R_S + 16 * ewq, v);
+        tmem_wait_ld();
+        const float *ut = reinterpret_cast<const float *>(rb + tp::REC_UT) + row;
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[x] += ut[(16 * ewq + x) * HD];
+        uint32_t hw[8], lw[8];
+        split_words<8>(v, hw, lw);
+        tmem_st8(tl + T_UH + 8 * ewq, hw);
+        tmem_st8(tl + T_UL + 8 * ewq, lw);
+#pragma unroll
+        for (int x = 0; x < 16; ++x) v[x] *= kdec[16 * ewq + x];
+        split_words<8>(v, hw, lw);
+        tmem_st8(tl + T_UKH + 8 * ewq, hw);
+        tmem_st8(tl + T_UKL + 8 * ewq, lw);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_UT));
+
+      // ---- state: S = gamma_C S + dS (fp32), S0 <- hi/lo(S)
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_S), ph, etid, abort_flag, p.status))) break;
+      {
+        const float gC = gam[128];
+        float v[32];
+        tmem_ld32(tl + R_S + 32 * ewq, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) S[x] = fmaf(gC, S[x], v[x]);
+        uint32_t hw[16], lw[16];
+        split_words<16>(S, hw, lw);
+        tmem_st16(tl + T_S0H + 16 * ewq, hw);
+        tmem_st16(tl + T_S0L + 16 * ewq, lw);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_S0));
+
+      // ---- outputs o_t = scale (e^{G_t} Oi_t + Oa_t) for t < Lc
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_OA), ph, etid, abort_flag, p.status))) break;
+      float out[16];
+      {
+        float va[16];
+        tmem_ld16(tl + R_OI + 16 * ewq, out);
+        tmem_ld16(tl + R_OA + 16 * ewq, va);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 16; ++x) out[x] = p.scale * fmaf(gam[16 * ewq + x], out[x], va[x]);
+      }
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) {
+        mbar_arrive(bar_addr(sb, B_OFREE));
+        mbar_arrive(bar_addr(sb, B_EMPTY_R + sr));
+      }
+      TO *op = static_cast<TO *>(p.o) + ((size_t)t0 * p.Hv + h) * HD + row;
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int t = 16 * ewq + x;
+        if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(out[x]);
+      }
+    }
+    if (ok && *abort_flag == 0 && dst) {
+      float *drow = dst + (size_t)row * HD + 32 * ewq;
+#pragma unroll
+      for (int x = 0; x < 32; x += 4)
+        *reinterpret_cast<float4 *>(drow + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace sp
+
+// ---------------------------------------------------------------- host side
+
+using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                              const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                              const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                              CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeFn encode_fn() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  }
+  return fn;
+}
+
+bool make_qkv_map(CUtensorMap *m, const void *base, int H, int T) {
+  EncodeFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)tp::HD, (cuuint64_t)H, (cuuint64_t)T};
+  const cuuint64_t strides[2] = {(cuuint64_t)tp::HD * 2, (cuuint64_t)H * tp::HD * 2};
+  const cuuint32_t box[3] = {64, 1, tp::CH};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+size_t twophase_workspace_bytes(int64_t N, int64_t T, int Hv) {
+  const tp::Layout L = tp::layout(N, Hv);
+  return L.fixed + (size_t)tp::chunk_bound(N, T) * L.rec_row;
+}
+
+size_t twophase_min_workspace_bytes(int64_t N, int Hv) {
+  const tp::Layout L = tp::layout(N, Hv);
+  return L.fixed + L.rec_row;
+}
+
+size_t twophase_round_workspace_bytes(int64_t N, int Hv, int64_t chunks_per_round) {
+  const tp::Layout L = tp::layout(N, Hv);
+  return L.fixed + (size_t)chunks_per_round * L.rec_row;
+}
+
+template <typename TO>
+static cudaError_t launch_state_pass(const CUtensorMap &mq, const CUtensorMap &mk,
+                                     const sp::Params &prm, int grid_x, cudaStream_t stream) {
+  auto kern = sp::state_pass_kernel<TO>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sp::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3((unsigned)grid_x, (unsigned)prm.Hv), sp::NTHREADS, sp::SMEM_BYTES, stream>>>(mq, mk, prm);
+  return cudaGetLastError();
+}
+
+// Plan, then per round: phase 1 (WY prep of every chunk of the round) and
+// phase 2 (state passing).  workspace_bytes >= twophase_min_workspace_bytes.
+cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const int32_t *cu, int N, long long T_,
+                                    int Hqk, int Hv, int o_dtype, float scale, const float *s0,
+                                    float *sfin, void *o, void *workspace, size_t workspace_bytes,
+                                    cudaStream_t stream) {
+  const int T = (int)T_;
+  const tp::Layout L = tp::layout(N, Hv);
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  int32_t *status = reinterpret_cast<int32_t *>(ws);
+  tp::PlanHeader *ph = reinterpret_cast<tp::PlanHeader *>(ws + tp::kPlanHeaderOffset);
+  int32_t *ne_seq = reinterpret_cast<int32_t *>(ws + L.plan_off);
+  int32_t *ne_cs = ne_seq + L.n_ne_capacity;
+  plan::plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, Hv, s0, sfin, ph, ne_seq, ne_cs, status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || T == 0) return e;
+
+  CUtensorMap mq, mk, mv;
+  if (!make_qkv_map(&mq, q, Hqk, T) || !make_qkv_map(&mk, k, Hqk, T) || !make_qkv_map(&mv, v, Hv, T))
+    return cudaErrorInvalidValue;
+  const int64_t bound = tp::chunk_bound(N, T);
+  const int64_t fit = (int64_t)((workspace_bytes - L.fixed) / L.rec_row);
+  const int rc = (int)std::min<int64_t>(std::min<int64_t>(bound, fit), 1 << 20);
+  const int rounds = (int)((bound + rc - 1) / rc);
+
+  sp::Params prm;
+  prm.cu = cu; prm.N = N; prm.Hqk = Hqk; prm.Hv = Hv; prm.rc = rc; prm.scale = scale;
+  prm.s0 = s0; prm.sfin = sfin; prm.o = o;
+  prm.plan = ph; prm.ne_seq = ne_seq; prm.ne_cs = ne_cs;
+  prm.rec = ws + L.rec_off;
+  prm.carry = reinterpret_cast<float *>(ws + L.carry_off);
+  prm.status = status;
+  const int grid_x = std::min(N, rc);
+  for (int r = 0; r < rounds; ++r) {
+    e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, workspace, L, stream);
+    if (e != cudaSuccess) return e;
+    prm.round = r;
+    e = (o_dtype == GDN_DTYPE_BF16) ? launch_state_pass<__nv_bfloat16>(mq, mk, prm, grid_x, stream)
+                                    : launch_state_pass<float>(mq, mk, prm, grid_x, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace gdn

@@ -77,14 +77,29 @@ const char *gdn_status_string(int32_t status);
 int32_t gdn_version(void);
 
 /*
- * Bytes of device workspace gdn_prefill needs for these sizes.  The
- * workspace holds the device status word and the work scheduler's counters;
- * it must stay allocated and unused by anything else until the call's work on
- * the stream has finished.  Returns 0 for invalid sizes.
+ * Bytes of device workspace with which gdn_prefill runs at full speed for
+ * these sizes.  The workspace holds the device status word and, for the
+ * tensor-core path, the per-chunk products of its first phase (about 65 KiB
+ * per chunk of 64 tokens and value head, plus 2 x Hv x 64 KiB of state
+ * carry).  It must stay allocated and unused by anything else until the
+ * call's work on the stream has finished.  Returns 0 for invalid sizes.
  */
 size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_t num_qk_heads,
                                   int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
                                   int32_t dtype);
+
+/*
+ * Bytes of a workspace with which the tensor-core prefill processes the packed
+ * chunk list in rounds of `chunks_per_round` chunks (of 64 tokens, across all
+ * value heads): a bounded workspace for long inputs, at the price of one
+ * launch pair per round.  0 means one round (= gdn_prefill_workspace_size);
+ * sizes that need no rounds return gdn_prefill_workspace_size.  Returns 0 for
+ * invalid sizes or a negative chunks_per_round.
+ */
+size_t gdn_prefill_workspace_size_rounds(int32_t num_seqs, int64_t total_tokens,
+                                         int32_t num_qk_heads, int32_t num_v_heads,
+                                         int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                                         int64_t chunks_per_round);
 
 /*
  * Prefill: run the recurrence over num_seqs packed sequences.
@@ -107,17 +122,25 @@ size_t gdn_prefill_workspace_size(int32_t num_seqs, int64_t total_tokens, int32_
  *                  between arguments is allowed.
  *   o              [T, Hv, Dv]    o_dtype (output)
  *   scale          multiplies o (1.0 for o_t = S_t q_t)
- *   workspace      device buffer of at least gdn_prefill_workspace_size(...) bytes,
- *                  256-byte aligned, zero-filled once before its first use.  The
- *                  kernels leave it zeroed apart from the status word, which is
- *                  sticky: it keeps the first device-detected error until
- *                  gdn_get_device_status reads and clears it.
+ *   workspace      device buffer of workspace_bytes >= 256 bytes, 256-byte aligned,
+ *                  zero-filled once before its first use.  Its first word is the
+ *                  sticky status word: it keeps the first device-detected error
+ *                  until gdn_get_device_status reads and clears it; nothing else in
+ *                  it needs to survive between calls.
  *
  * Supported: Hv % Hqk == 0; Dk, Dv in {64, 128}; dtype and o_dtype each bf16
- * or fp32.  bf16 inputs with Dk = Dv = 128 run the tensor-core (tcgen05) kernel with bf16
- * operands and fp32 accumulation; every other case runs the fp32 CUDA-core
- * kernel.  T = 0 or num_seqs = 0 is a valid no-op apart from copying
- * initial_state to final_state.
+ * or fp32.  bf16 inputs with Dk = Dv = 128 run on the tensor cores (tcgen05,
+ * bf16 operands with hi/lo splits of computed values, fp32 accumulation):
+ *   - workspace_bytes >= gdn_prefill_workspace_size(...): two phases, the
+ *     state-free products of every chunk at once (WY/UT transform), then one
+ *     pass per (sequence, value head) over its chunks for the state;
+ *   - smaller, down to the two-phase minimum (the state carry plus one chunk
+ *     per value head): the same in rounds of as many chunks as fit;
+ *   - below that (>= 256 bytes): a single-pass kernel, one CTA per (sequence,
+ *     value head) doing all of each chunk in turn (slower).
+ * Every other case runs the fp32 CUDA-core kernel, which needs 256 bytes.
+ * T = 0 or num_seqs = 0 is a valid no-op apart from copying initial_state to
+ * final_state.
  */
 int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
                     const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,

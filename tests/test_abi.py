@@ -8,6 +8,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from gated_deltanet_recurrence_rule_b200 import api
 
@@ -41,6 +42,21 @@ def test_status_strings(lib):
         assert api.status_string(code).startswith("GDN_")
     assert api.status_string(999) == "GDN_ERR_UNKNOWN"
     assert lib.gdn_version() >= 100
+
+
+def test_workspace_size_rounds(lib):
+    """Tensor-core sizes: the full workspace holds one record per (chunk,
+    value head); rounds bound it; CUDA-core sizes need only the header."""
+    full = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128)
+    assert full > 129 * 48 * 65536  # one record per chunk (bound: T/64 + N) and value head
+    r1 = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=1)
+    r4 = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=4)
+    assert 256 < r1 < r4 < full
+    assert r4 - r1 == 3 * (r4 - r1) // 3 and (r4 - r1) // 3 >= 48 * 65536
+    assert api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=10 ** 6) == full
+    assert lib.gdn_prefill_workspace_size_rounds(1, 8192, 16, 48, 128, 128, 0, -1) == 0
+    assert api.prefill_workspace_size(1, 256, 2, 6, 64, 64, torch.float32) == 256
+    assert api.prefill_workspace_size(1, 256, 2, 6, 64, 64, torch.float32, chunks_per_round=2) == 256
 
 
 def test_workspace_size(lib):

@@ -125,6 +125,42 @@ def test_guard_bands_and_determinism():
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
+def _run_ws(inp, ws):
+    dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
+    o, f = api.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                       cu_seqlens=dev["cu_seqlens"], initial_state=dev["initial_state"],
+                       workspace=ws)
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == api.GDN_OK
+    return o, f
+
+
+@pytest.mark.parametrize("rc", [1, 3, 7])
+def test_rounds_bounded_workspace(rc):
+    """A workspace for rounds of rc chunks: sequences cross round boundaries
+    (state carried through the workspace); same bits as one round, and the
+    oracle's result within tolerance."""
+    lengths = [300, 1, 0, 130, 700, 64, 65]
+    inp = inputs.prefill_inputs(lengths, 2, 6, 128, dtype="bf16", seed=19, init_std=0.1)
+    N, T = len(lengths), sum(lengths)
+    full = api.prefill_workspace_size(N, T, 2, 6, 128, 128)
+    small = api.prefill_workspace_size(N, T, 2, 6, 128, 128, chunks_per_round=rc)
+    assert small < full
+    o1, f1 = _run_ws(inp, torch.zeros(full, dtype=torch.uint8, device=DEV))
+    o2, f2 = _run_ws(inp, torch.zeros(small, dtype=torch.uint8, device=DEV))
+    assert torch.equal(o1, o2) and torch.equal(f1, f2)
+    o_ref, f_ref = run_oracle(inp)
+    assert_parity(torch.bfloat16, to_np(o2), o_ref, to_np(f2), f_ref, f"rounds of {rc}")
+
+
+def test_single_pass_header_workspace():
+    """A 256-byte workspace runs the single-pass tensor-core kernel."""
+    inp = inputs.prefill_inputs([300, 0, 65], 2, 6, 128, dtype="bf16", seed=20, init_std=0.1)
+    o, f = _run_ws(inp, torch.zeros(256, dtype=torch.uint8, device=DEV))
+    o_ref, f_ref = run_oracle(inp)
+    assert_parity(torch.bfloat16, to_np(o), o_ref, to_np(f), f_ref, "single pass")
+
+
 def _sampled_workload(name, qk_heads):
     w = inputs.WORKLOADS[name]
     inp = inputs.workload_inputs(w)

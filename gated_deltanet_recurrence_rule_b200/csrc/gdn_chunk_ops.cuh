@@ -90,9 +90,9 @@ __device__ __forceinline__ void ut_distance(const float *__restrict__ A, float *
 // Unit lower-triangular inverse Tm = (I + A)^-1 of a 64x64 strictly lower A
 // (fp32, shared memory, row stride AST), by NT = 256 or 512 threads.  The four
 // 16x16 diagonal blocks by forward substitution: column c of block b is solved
-// by one group of lanes that hold its rows (NT = 512: 8 lanes x 2 rows, A in
-// registers; NT = 256: 4 lanes x 4 rows, A read from shared memory), the
-// solved entry of step s passed by a shuffle.  Then the off-diagonal blocks by
+// by one group of lanes that hold its rows (NT = 512: 8 lanes x 2 rows; NT =
+// 256: 4 lanes x 4 rows; A read from shared memory), the solved entry of
+// step s passed by a shuffle.  Then the off-diagonal blocks by
 // block distance 1, 2, 3 (each needs only blocks of smaller distance).  Only
 // the lower triangle of Tm is written.  Y holds [3][16][17] fp32 of scratch.
 template <int NT, int BAR>
@@ -152,6 +152,23 @@ __device__ __forceinline__ void split_words(const float *x, uint32_t *hw, uint32
     lw[e] = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
   }
 }
+// The two halves of split_words separately: hi(x) words, then lo(x) words.
+template <int NP>
+__device__ __forceinline__ void hi_words(const float *x, uint32_t *hw) {
+#pragma unroll
+  for (int e = 0; e < NP; ++e)
+    hw[e] = __byte_perm(__float_as_uint(x[2 * e]), __float_as_uint(x[2 * e + 1]), 0x7632);
+}
+template <int NP>
+__device__ __forceinline__ void lo_words(const float *x, uint32_t *lw) {
+#pragma unroll
+  for (int e = 0; e < NP; ++e) {
+    const float ra = x[2 * e] - __uint_as_float(__float_as_uint(x[2 * e]) & 0xffff0000u);
+    const float rb = x[2 * e + 1] - __uint_as_float(__float_as_uint(x[2 * e + 1]) & 0xffff0000u);
+    lw[e] = __byte_perm(__float_as_uint(ra), __float_as_uint(rb), 0x7632);
+  }
+}
+
 // 8 fp32 values -> one 16-byte hi chunk and one 16-byte lo chunk.
 __device__ __forceinline__ void st_split8(unsigned char *dst_hi, unsigned char *dst_lo,
                                           const float *x) {

@@ -24,6 +24,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "gdn_chunk_ops.cuh"
 #include "gdn_common.cuh"
@@ -36,7 +37,7 @@ size_t wy_prep_smem_bytes();
 cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                            const float *g, const float *beta, const int32_t *cu, int T, int Hqk,
                            int Hv, int round, int rc, const void *workspace,
-                           const tp::Layout &L, cudaStream_t stream);
+                           const tp::Layout &L, unsigned char *rec, cudaStream_t stream);
 
 namespace plan {
 
@@ -127,8 +128,8 @@ using tp::HD;
 using tp::REC_BYTES;
 
 constexpr int NTHREADS = 640;
-constexpr int NEPI = 512;   // 4 column quarters x 128 rows
-constexpr int EPI_BAR = 1;
+constexpr int NEPI = 512;   // epilogue threads: 4 column quarters x 128 rows
+constexpr int EPI_BAR = 1;  // named barrier of the epilogue threads
 
 // ---- shared memory map (bytes) ----
 constexpr int NQK = 2, NR = 2;         // ring depths: Q/K tiles, chunk records
@@ -143,7 +144,10 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 enum {
   B_FULL_QK = 0, B_EMPTY_QK = B_FULL_QK + NQK, B_FULL_R = B_EMPTY_QK + NQK, B_EMPTY_R = B_FULL_R + NR,
-  B_S0 = B_EMPTY_R + NR, B_U, B_UT, B_S, B_OA, B_OFREE, NBAR
+  // S0 hi / lo written; U ready; U diag(kdec) split written; U split written;
+  // dS (and Oi) ready; Oa ready; the outputs of a chunk were read out of TMEM;
+  // the MMA issuer's drain
+  B_S0H = B_EMPTY_R + NR, B_S0L, B_U, B_UK, B_UO, B_S, B_OA, B_OFREE, B_DRAIN, NBAR
 };
 static_assert(NBAR * 8 <= 256, "barrier area");
 
@@ -163,7 +167,7 @@ constexpr uint32_t IDESC_UK = idesc_bf16(128, 128, 0, 1);    // Ukdec^T K
 
 struct Params {
   const int32_t *cu;
-  int N, Hqk, Hv;
+  int N, T, Hqk, Hv;
   int round, rc;
   float scale;
   const float *s0;
@@ -281,30 +285,41 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint64_t dQK0 = sdesc_sw128(sb + OFF_QK, 16, 1024);            // Q, K-major
-      const uint64_t dKmn0 = sdesc_sw128(sb + OFF_QK + 8192, 16384, 1024); // K as MN-major operand
-      const uint64_t dW0 = sdesc_sw128(sb + OFF_REC + tp::REC_WT, 8192, 1024);  // W^T, MN-major
-      const uint64_t dP0 = sdesc_sw128(sb + OFF_REC + tp::REC_PH, 16, 1024);    // P hi / lo, K-major
-      bool ok = true;
-      for (int c = 0; c < nch && ok; ++c) {
-        const int s = c % NQK, sr = c % NR;
-        const uint32_t ph = c & 1;
-        const uint64_t dQK = dQK0 + s * (QK_STAGE >> 4), dKmn = dKmn0 + s * (QK_STAGE >> 4);
-        const uint64_t dW = dW0 + sr * (REC_BYTES >> 4), dP = dP0 + sr * (REC_BYTES >> 4);
-        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), (c / NQK) & 1, abort_flag) &&
-             mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag) &&
-             mbar_wait(bar_addr(sb, B_S0), ph, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        // U^T - U~^T = -S0h W^T   (S0 from TMEM)
+    // A converged warp: lane 0 waits, one elected lane issues each group of
+    // MMAs and its commits (far fewer issue cycles than a lone diverged lane).
+    // Order per chunk: U (chain), Oi (runs while the epilogue splits U), dS
+    // (chain), Oa (runs while the epilogue updates the state).
+    const uint64_t dQK0 = sdesc_sw128(sb + OFF_QK, 16, 1024);            // Q, K-major
+    const uint64_t dKmn0 = sdesc_sw128(sb + OFF_QK + 8192, 16384, 1024); // K as MN-major operand
+    const uint64_t dW0 = sdesc_sw128(sb + OFF_REC + tp::REC_WT, 8192, 1024);  // W^T, MN-major
+    const uint64_t dP0 = sdesc_sw128(sb + OFF_REC + tp::REC_PH, 16, 1024);    // P hi / lo, K-major
+    auto wait = [&](int b, uint32_t parity) {
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(bar_addr(sb, b), parity, abort_flag);
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    };
+    bool ok = true;
+    for (int c = 0; c < nch && ok; ++c) {
+      const int s = c % NQK, sr = c % NR;
+      const uint32_t ph = c & 1;
+      const uint64_t dQK = dQK0 + s * (QK_STAGE >> 4), dKmn = dKmn0 + s * (QK_STAGE >> 4);
+      const uint64_t dW = dW0 + sr * (REC_BYTES >> 4), dP = dP0 + sr * (REC_BYTES >> 4);
+      // U^T - U~^T = -S0h W^T   (S0 hi from TMEM)
+      if (!(ok = wait(B_FULL_R + sr, (c / NR) & 1) && wait(B_S0H, ph))) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
           mma_bf16_ts(tmem + R_S, tmem + T_S0H + 8 * ks, dW + ((ks * 2048) >> 4), IDESC_SW, ks > 0);
         mma_commit(bar_addr(sb, B_U));
-        // Oi^T = (S0h + S0l) Q^T, once the previous chunk's outputs were read
-        if (c > 0 && !(ok = mbar_wait(bar_addr(sb, B_OFREE), (c - 1) & 1, abort_flag))) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      // Oi^T = (S0h + S0l) Q^T, once S0 is complete and the previous outputs were read
+      if (!(ok = wait(B_FULL_QK + s, (c / NQK) & 1) && wait(B_S0L, ph) &&
+                 (c == 0 || wait(B_OFREE, (c - 1) & 1))))
+        break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < 16; ++ks) {
           const int k = ks >> 1;
@@ -312,9 +327,12 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           mma_bf16_ts(tmem + R_OI, tmem + ((ks & 1) ? T_S0L : T_S0H) + 8 * k, dQK + k16, IDESC_SQ,
                       ks > 0);
         }
-        // dS = (Ukh + Ukl)^T K ;  Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T   (U from TMEM)
-        if (!(ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag))) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      // dS = (Ukh + Ukl)^T K   (U diag(kdec) from TMEM)
+      if (!(ok = wait(B_UK, ph))) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
           const int kk = ks >> 1;
@@ -322,6 +340,12 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                       dKmn + ((kk * 2048) >> 4), IDESC_UK, ks > 0);
         }
         mma_commit(bar_addr(sb, B_S));
+      }
+      __syncwarp();
+      // Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T   (U from TMEM)
+      if (!(ok = wait(B_UO, ph))) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
         for (int ks = 0; ks < 12; ++ks) {
           const int part = ks % 3, kk = ks / 3;  // (Uh,Ph), (Ul,Ph), (Uh,Pl)
@@ -333,23 +357,28 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mma_commit(bar_addr(sb, B_EMPTY_QK + s));
         mma_commit(bar_addr(sb, B_EMPTY_R + sr));
       }
-      if (!ok) {
-        *abort_flag = 1;
-        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
-      }
-      // Drain: every MMA this thread issued finishes before TMEM is freed.
-      const uint32_t drain = sb + OFF_MISC + 8;
-      mbar_init(drain, 1);
-      fence_barrier_init();
-      mma_commit(drain);
-      mbar_wait_landed(drain, 0, 50000000ull);
+      __syncwarp();
     }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+    }
+    // Drain: every MMA this warp issued finishes before TMEM is freed.
+    if (elect_one()) {
+      mma_commit(bar_addr(sb, B_DRAIN));
+      mbar_wait_landed(bar_addr(sb, B_DRAIN), 0, 50000000ull);
+    }
+    __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int etid = tid - 128;
     const int ewq = etid >> 7;   // column quarter
     const int row = etid & 127;  // TMEM lane = row (Dv index) of the 128-row tiles
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    auto fail = [&]() {
+      *abort_flag = 1;
+      report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+    };
 
     // fp32 master state: row `row`, columns [32 ewq, 32 ewq + 32); S0 = hi + lo in TMEM
     float S[32];
@@ -369,68 +398,116 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     tc_fence_before();
     named_bar_sync(EPI_BAR, NEPI);
-    if (etid == 0) mbar_arrive(bar_addr(sb, B_S0));
+    if (etid == 0) {
+      mbar_arrive(bar_addr(sb, B_S0H));
+      mbar_arrive(bar_addr(sb, B_S0L));
+    }
 
-    bool ok = true;
-    for (int c = 0; c < nch; ++c) {
+    // U~ of the chunk about to run, read from its record while the previous
+    // chunk's dS product runs
+    float un[16];
+    auto fetch_ut = [&](int c) {
+      const int sr = c % NR;
+      if (etid == 0 && !mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag)) fail();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (*abort_flag) return false;
+      const float *ut = reinterpret_cast<const float *>(smem + OFF_REC + sr * REC_BYTES + tp::REC_UT) + row;
+#pragma unroll
+      for (int x = 0; x < 16; ++x) un[x] = ut[(16 * ewq + x) * HD];
+      return true;
+    };
+    // The outputs of chunk c leave TMEM at the end of chunk c and go to HBM
+    // during chunk c + 1, a quarter at each of its four waits, so that the
+    // store path drains in the background.
+    float out[16];
+    int out_t0 = 0, out_Lc = 0;  // tokens of the chunk whose outputs `out` holds
+    auto store_out = [&](int part) {
+      TO *op = static_cast<TO *>(p.o) + ((size_t)out_t0 * p.Hv + h) * HD + row;
+#pragma unroll
+      for (int x = 4 * part; x < 4 * part + 4; ++x) {
+        const int t = 16 * ewq + x;
+        if (t < out_Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(out[x]);
+      }
+    };
+    bool ok = fetch_ut(0);
+    for (int c = 0; c < nch && ok; ++c) {
       const int sr = c % NR;
       const uint32_t ph = c & 1;
       const int t0 = seq_begin + (ga - cs + c) * CH;
       const int Lc = min(CH, seq_end - t0);
-      const unsigned char *rb = smem + OFF_REC + sr * REC_BYTES;
-      const float *gam = reinterpret_cast<const float *>(rb + tp::REC_SC);
+      const float *gam = reinterpret_cast<const float *>(smem + OFF_REC + sr * REC_BYTES + tp::REC_SC);
       const float *kdec = gam + 64;
 
-      // ---- U = (U - U~) + U~  ->  hi/lo(U^T) and hi/lo(U^T diag(kdec)) into TMEM
-      if (etid == 0 && !mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag)) {
-        *abort_flag = 1;
-        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
-      }
+      // ---- U = (U - U~) + U~ -> hi/lo(U^T diag(kdec)) for dS first, then hi/lo(U^T) for Oa
       if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_U), ph, etid, abort_flag, p.status))) break;
       {
         float v[16];
         tmem_ld16(tl + R_S + 16 * ewq, v);
         tmem_wait_ld();
-        const float *ut = reinterpret_cast<const float *>(rb + tp::REC_UT) + row;
 #pragma unroll
-        for (int x = 0; x < 16; ++x) v[x] += ut[(16 * ewq + x) * HD];
+        for (int x = 0; x < 16; ++x) v[x] += un[x];
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+          float w[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) w[x] = v[8 * hq + x] * kdec[16 * ewq + 8 * hq + x];
+          uint32_t hw[4], lw[4];
+          split_words<4>(w, hw, lw);
+          tmem_st4(tl + T_UKH + 8 * ewq + 4 * hq, hw);
+          tmem_st4(tl + T_UKL + 8 * ewq + 4 * hq, lw);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        named_bar_sync(EPI_BAR, NEPI);
+        if (etid == 0) mbar_arrive(bar_addr(sb, B_UK));
+        store_out(0);
         uint32_t hw[8], lw[8];
         split_words<8>(v, hw, lw);
         tmem_st8(tl + T_UH + 8 * ewq, hw);
         tmem_st8(tl + T_UL + 8 * ewq, lw);
-#pragma unroll
-        for (int x = 0; x < 16; ++x) v[x] *= kdec[16 * ewq + x];
-        split_words<8>(v, hw, lw);
-        tmem_st8(tl + T_UKH + 8 * ewq, hw);
-        tmem_st8(tl + T_UKL + 8 * ewq, lw);
         tmem_wait_st();
       }
       tc_fence_before();
       named_bar_sync(EPI_BAR, NEPI);
-      if (etid == 0) mbar_arrive(bar_addr(sb, B_UT));
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_UO));
 
-      // ---- state: S = gamma_C S + dS (fp32), S0 <- hi/lo(S)
+      store_out(1);
+
+      // ---- state: S = gamma_C S + dS (fp32); hi(S) first (the next U product), then lo(S)
       if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_S), ph, etid, abort_flag, p.status))) break;
       {
         const float gC = gam[128];
-        float v[32];
-        tmem_ld32(tl + R_S + 32 * ewq, v);
-        tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 32; ++x) S[x] = fmaf(gC, S[x], v[x]);
-        uint32_t hw[16], lw[16];
-        split_words<16>(S, hw, lw);
-        tmem_st16(tl + T_S0H + 16 * ewq, hw);
-        tmem_st16(tl + T_S0L + 16 * ewq, lw);
+        for (int hq = 0; hq < 2; ++hq) {
+          float v[16];
+          tmem_ld16(tl + R_S + 32 * ewq + 16 * hq, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 16; ++x) S[16 * hq + x] = fmaf(gC, S[16 * hq + x], v[x]);
+          uint32_t hw[8];
+          hi_words<8>(S + 16 * hq, hw);
+          tmem_st8(tl + T_S0H + 16 * ewq + 8 * hq, hw);
+        }
         tmem_wait_st();
       }
       tc_fence_before();
       named_bar_sync(EPI_BAR, NEPI);
-      if (etid == 0) mbar_arrive(bar_addr(sb, B_S0));
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_S0H));
+      store_out(2);
+#pragma unroll
+      for (int hq = 0; hq < 2; ++hq) {
+        uint32_t lw[8];
+        lo_words<8>(S + 16 * hq, lw);
+        tmem_st8(tl + T_S0L + 16 * ewq + 8 * hq, lw);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      named_bar_sync(EPI_BAR, NEPI);
+      if (etid == 0) mbar_arrive(bar_addr(sb, B_S0L));
+      store_out(3);
 
-      // ---- outputs o_t = scale (e^{G_t} Oi_t + Oa_t) for t < Lc
+      // ---- outputs o_t = scale (e^{G_t} Oi_t + Oa_t) out of TMEM
       if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_OA), ph, etid, abort_flag, p.status))) break;
-      float out[16];
       {
         float va[16];
         tmem_ld16(tl + R_OI + 16 * ewq, out);
@@ -439,24 +516,26 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
         for (int x = 0; x < 16; ++x) out[x] = p.scale * fmaf(gam[16 * ewq + x], out[x], va[x]);
       }
+      out_t0 = t0;
+      out_Lc = Lc;
       tc_fence_before();
       named_bar_sync(EPI_BAR, NEPI);
       if (etid == 0) {
         mbar_arrive(bar_addr(sb, B_OFREE));
         mbar_arrive(bar_addr(sb, B_EMPTY_R + sr));
       }
-      TO *op = static_cast<TO *>(p.o) + ((size_t)t0 * p.Hv + h) * HD + row;
-#pragma unroll
-      for (int x = 0; x < 16; ++x) {
-        const int t = 16 * ewq + x;
-        if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(out[x]);
-      }
+      // ---- the next chunk's U~, while its U product runs
+      if (c + 1 < nch && !(ok = fetch_ut(c + 1))) break;
     }
-    if (ok && *abort_flag == 0 && dst) {
-      float *drow = dst + (size_t)row * HD + 32 * ewq;
+    if (ok && *abort_flag == 0) {
 #pragma unroll
-      for (int x = 0; x < 32; x += 4)
-        *reinterpret_cast<float4 *>(drow + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
+      for (int part = 0; part < 4; ++part) store_out(part);
+      if (dst) {
+        float *drow = dst + (size_t)row * HD + 32 * ewq;
+#pragma unroll
+        for (int x = 0; x < 32; x += 4)
+          *reinterpret_cast<float4 *>(drow + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
+      }
     }
   }
 
@@ -501,9 +580,18 @@ bool make_qkv_map(CUtensorMap *m, const void *base, int H, int T) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Rounds of the pipelined schedule: about kPipeRounds rounds of at least
+// kMinRoundChunks global chunks each, records double-buffered.
+constexpr int64_t kPipeRounds = 8, kMinRoundChunks = 8;
+
+static int64_t pipelined_round_chunks(int64_t N, int64_t T) {
+  const int64_t bound = tp::chunk_bound(N, T);
+  return std::max<int64_t>(kMinRoundChunks, (bound + kPipeRounds - 1) / kPipeRounds);
+}
+
 size_t twophase_workspace_bytes(int64_t N, int64_t T, int Hv) {
   const tp::Layout L = tp::layout(N, Hv);
-  return L.fixed + (size_t)tp::chunk_bound(N, T) * L.rec_row;
+  return L.fixed + 2 * (size_t)pipelined_round_chunks(N, T) * L.rec_row;
 }
 
 size_t twophase_min_workspace_bytes(int64_t N, int Hv) {
@@ -526,8 +614,50 @@ static cudaError_t launch_state_pass(const CUtensorMap &mq, const CUtensorMap &m
   return cudaGetLastError();
 }
 
+// Internal streams and events of one device, created by its first pipelined
+// prefill and kept until the process exits: phase 1 runs on `prep`, phase 2
+// on `chain` (higher priority, so its CTAs get the SMs that free up first).
+namespace {
+constexpr int kMaxDevices = 64, kEventRing = 4;
+struct DeviceStreams {
+  bool ready = false;
+  cudaStream_t prep = nullptr, chain = nullptr;
+  cudaEvent_t start = nullptr, prep_done = nullptr, ev_p[kEventRing] = {}, ev_c[kEventRing] = {};
+};
+std::mutex g_streams_mutex;
+DeviceStreams g_streams[kMaxDevices];
+
+cudaError_t device_streams(DeviceStreams **out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  DeviceStreams &d = g_streams[dev];
+  if (!d.ready) {
+    int least = 0, greatest = 0;
+    if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&d.prep, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
+    if ((e = cudaStreamCreateWithPriority(&d.chain, cudaStreamNonBlocking, greatest)) != cudaSuccess) return e;
+    cudaEvent_t *all[] = {&d.start, &d.prep_done};
+    for (cudaEvent_t *ev : all)
+      if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+    for (int i = 0; i < kEventRing; ++i) {
+      if ((e = cudaEventCreateWithFlags(&d.ev_p[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+      if ((e = cudaEventCreateWithFlags(&d.ev_c[i], cudaEventDisableTiming)) != cudaSuccess) return e;
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return cudaSuccess;
+}
+}  // namespace
+
 // Plan, then per round: phase 1 (WY prep of every chunk of the round) and
-// phase 2 (state passing).  workspace_bytes >= twophase_min_workspace_bytes.
+// phase 2 (state passing).  With a workspace of twophase_workspace_bytes or
+// more, rounds are pipelined: phase 1 of round r + 1 runs on the SMs phase 2
+// of round r leaves free, each round's records still in L2 when phase 2 reads
+// them (two record buffers).  With less (>= twophase_min_workspace_bytes) the
+// rounds run one after another on `stream` with as many chunks as fit.
 cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const int32_t *cu, int N, long long T_,
                                     int Hqk, int Hv, int o_dtype, float scale, const float *s0,
@@ -540,35 +670,74 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
   tp::PlanHeader *ph = reinterpret_cast<tp::PlanHeader *>(ws + tp::kPlanHeaderOffset);
   int32_t *ne_seq = reinterpret_cast<int32_t *>(ws + L.plan_off);
   int32_t *ne_cs = ne_seq + L.n_ne_capacity;
-  plan::plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, Hv, s0, sfin, ph, ne_seq, ne_cs, status);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || T == 0) return e;
 
   CUtensorMap mq, mk, mv;
-  if (!make_qkv_map(&mq, q, Hqk, T) || !make_qkv_map(&mk, k, Hqk, T) || !make_qkv_map(&mv, v, Hv, T))
+  if (T > 0 && (!make_qkv_map(&mq, q, Hqk, T) || !make_qkv_map(&mk, k, Hqk, T) ||
+                !make_qkv_map(&mv, v, Hv, T)))
     return cudaErrorInvalidValue;
   const int64_t bound = tp::chunk_bound(N, T);
+  const bool pipelined = workspace_bytes >= twophase_workspace_bytes(N, T, Hv);
   const int64_t fit = (int64_t)((workspace_bytes - L.fixed) / L.rec_row);
-  const int rc = (int)std::min<int64_t>(std::min<int64_t>(bound, fit), 1 << 20);
+  const int rc = (int)std::min<int64_t>(
+      pipelined ? pipelined_round_chunks(N, T) : std::min<int64_t>(bound, fit), 1 << 20);
   const int rounds = (int)((bound + rc - 1) / rc);
 
   sp::Params prm;
-  prm.cu = cu; prm.N = N; prm.Hqk = Hqk; prm.Hv = Hv; prm.rc = rc; prm.scale = scale;
+  prm.cu = cu; prm.N = N; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.rc = rc; prm.scale = scale;
   prm.s0 = s0; prm.sfin = sfin; prm.o = o;
   prm.plan = ph; prm.ne_seq = ne_seq; prm.ne_cs = ne_cs;
-  prm.rec = ws + L.rec_off;
   prm.carry = reinterpret_cast<float *>(ws + L.carry_off);
   prm.status = status;
   const int grid_x = std::min(N, rc);
-  for (int r = 0; r < rounds; ++r) {
-    e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, workspace, L, stream);
-    if (e != cudaSuccess) return e;
-    prm.round = r;
-    e = (o_dtype == GDN_DTYPE_BF16) ? launch_state_pass<__nv_bfloat16>(mq, mk, prm, grid_x, stream)
-                                    : launch_state_pass<float>(mq, mk, prm, grid_x, stream);
-    if (e != cudaSuccess) return e;
+  auto state_pass = [&](cudaStream_t st) {
+    return (o_dtype == GDN_DTYPE_BF16) ? launch_state_pass<__nv_bfloat16>(mq, mk, prm, grid_x, st)
+                                       : launch_state_pass<float>(mq, mk, prm, grid_x, st);
+  };
+  cudaError_t e;
+
+  if (!pipelined) {
+    plan::plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, Hv, s0, sfin, ph, ne_seq, ne_cs, status);
+    if ((e = cudaGetLastError()) != cudaSuccess || T == 0) return e;
+    prm.rec = ws + L.rec_off;
+    for (int r = 0; r < rounds; ++r) {
+      e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, workspace, L, ws + L.rec_off, stream);
+      if (e != cudaSuccess) return e;
+      prm.round = r;
+      if ((e = state_pass(stream)) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
   }
-  return cudaSuccess;
+
+  // Pipelined rounds on the device's two internal streams, joined to `stream`
+  // by events (this also works while `stream` is being captured into a graph).
+  std::lock_guard<std::mutex> lock(g_streams_mutex);
+  DeviceStreams *d = nullptr;
+  if ((e = device_streams(&d)) != cudaSuccess) return e;
+  if ((e = cudaEventRecord(d->start, stream)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(d->prep, d->start, 0)) != cudaSuccess) return e;
+  if ((e = cudaStreamWaitEvent(d->chain, d->start, 0)) != cudaSuccess) return e;
+  plan::plan_kernel<<<1, 1024, 0, d->prep>>>(cu, N, T, Hv, s0, sfin, ph, ne_seq, ne_cs, status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (T == 0) {
+    if ((e = cudaEventRecord(d->prep_done, d->prep)) != cudaSuccess) return e;
+    return cudaStreamWaitEvent(stream, d->prep_done, 0);
+  }
+  for (int r = 0; r < rounds; ++r) {
+    unsigned char *rec = ws + L.rec_off + (size_t)(r & 1) * rc * L.rec_row;
+    // phase 1 of round r reuses the buffer phase 2 of round r - 2 read
+    if (r >= 2 && (e = cudaStreamWaitEvent(d->prep, d->ev_c[(r - 2) % kEventRing], 0)) != cudaSuccess)
+      return e;
+    e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, workspace, L, rec, d->prep);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaEventRecord(d->ev_p[r % kEventRing], d->prep)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(d->chain, d->ev_p[r % kEventRing], 0)) != cudaSuccess) return e;
+    prm.round = r;
+    prm.rec = rec;
+    if ((e = state_pass(d->chain)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(d->ev_c[r % kEventRing], d->chain)) != cudaSuccess) return e;
+  }
+  // phase 2 of the last round follows every earlier launch of both streams
+  return cudaStreamWaitEvent(stream, d->ev_c[(rounds - 1) % kEventRing], 0);
 }
 
 }  // namespace gdn

@@ -335,7 +335,7 @@ size_t wy_prep_smem_bytes() { return wy::SMEM_BYTES; }
 cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                            const float *g, const float *beta, const int32_t *cu, int T, int Hqk,
                            int Hv, int round, int rc, const void *workspace,
-                           const tp::Layout &L, cudaStream_t stream) {
+                           const tp::Layout &L, unsigned char *rec, cudaStream_t stream) {
   wy::Params prm;
   prm.g = g; prm.beta = beta; prm.cu = cu; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv;
   prm.round = round; prm.rc = rc;
@@ -343,7 +343,7 @@ cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const C
   prm.plan = reinterpret_cast<const tp::PlanHeader *>(ws + tp::kPlanHeaderOffset);
   prm.ne_seq = reinterpret_cast<const int32_t *>(ws + L.plan_off);
   prm.ne_cs = prm.ne_seq + L.n_ne_capacity;
-  prm.rec = ws + L.rec_off;
+  prm.rec = rec;
   prm.status = reinterpret_cast<int32_t *>(ws);
   cudaError_t e = cudaFuncSetAttribute(wy::wy_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        wy::SMEM_BYTES);

@@ -45,10 +45,11 @@ def test_status_strings(lib):
 
 
 def test_workspace_size_rounds(lib):
-    """Tensor-core sizes: the full workspace holds one record per (chunk,
-    value head); rounds bound it; CUDA-core sizes need only the header."""
+    """Tensor-core sizes: the full workspace holds two rounds of records (one
+    per chunk and value head, 8 rounds of ceil(129 / 8) = 17 chunks at T=8192);
+    smaller rounds bound it; CUDA-core sizes need only the header."""
     full = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128)
-    assert full > 129 * 48 * 65536  # one record per chunk (bound: T/64 + N) and value head
+    assert 2 * 17 * 48 * 65536 < full < 2 * 18 * 48 * 66560 + (8 << 20)
     r1 = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=1)
     r4 = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=4)
     assert 256 < r1 < r4 < full

@@ -182,21 +182,37 @@ def load_peaks():
         return dict(PEAKS_FALLBACK), "fallback"
 
 
-def kernel_traffic(kernel_key: str, source_file: str):
-    """DRAM bytes per launch from a committed ncu summary, or None when the
-    kernel source changed after the counters were taken."""
+def sources_sha(source_files) -> str:
+    h = hashlib.sha256()
+    for path in ([source_files] if isinstance(source_files, str) else source_files):
+        with open(path, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_entry(kernel_key: str, source_files):
+    """The committed ncu figures of a kernel (profiles/traffic.json), or None
+    when a source changed after the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
-            table = json.load(f)
-        ent = table[kernel_key]
-        with open(source_file, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()[:16]
-        if ent.get("source_sha") != sha:
-            return None
-        return ent["dram_bytes_per_launch"]
+            ent = json.load(f)[kernel_key]
+        return ent if ent.get("source_sha") == sources_sha(source_files) else None
     except (OSError, ValueError, KeyError):
         return None
+
+
+def kernel_traffic(kernel_key: str, source_files):
+    """DRAM bytes per launch (per step for a multi-launch entry) from a
+    committed ncu summary, or None when a source changed since."""
+    ent = traffic_entry(kernel_key, source_files)
+    return None if ent is None else ent["dram_bytes_per_launch"]
+
+
+CSRC = os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc")
+PREFILL_SOURCES = [os.path.join(CSRC, n) for n in
+                   ("gdn_twophase.cuh", "gdn_chunk_ops.cuh", "gdn_sm100.cuh", "gdn_wy_prep.cu",
+                    "gdn_state_pass.cu")]
 
 
 # ---------------------------------------------------------------- oracle (CPU)
@@ -314,6 +330,7 @@ def run_ours(args, D):
 
     peaks, peak_src = load_peaks()
     kernel_ms = statistics.mean(per_ms)
+    launches = api.prefill_launch_count(1, T, w.Hqk, w.Hv, w.D, w.D, ws.numel())
     if _tc_path_available():
         # Time floors of the two bounds; the larger one binds.
         flops = FLOP_PER_TOKEN * T
@@ -322,7 +339,6 @@ def run_ours(args, D):
         t_hbm = hbm_bytes / (peaks["hbm_gbs"] * 1e9)
         tensor_ach = flops / (kernel_ms / 1e3) / 1e12
         hbm_ach = hbm_bytes / (kernel_ms / 1e3) / 1e9
-        src = os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_prefill_tc.cu")
         if t_hbm >= t_tensor:
             roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": hbm_ach / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
@@ -332,11 +348,19 @@ def run_ours(args, D):
                     "unit": "TFLOP/s", "frac": tensor_ach / peaks["bf16_tflops"],
                     "peak_source": f"{peak_src} bf16_tflops (burst)",
                     "algorithmic": f"{FLOP_PER_TOKEN} flop/token x {T} tokens"}
-        roof.update({"kernel": "prefill_tc_kernel", "kernel_ms": kernel_ms,
+        # One prefill call is a sequence of launches (plan, then WY prep and
+        # state pass per round, on two streams, rounds pipelined): the time is
+        # the whole call's, between CUDA events on the caller's stream that
+        # bracket every launch of the step.
+        ent = traffic_entry("prefill_step", PREFILL_SOURCES)
+        roof.update({"kernel": f"prefill step: plan_kernel + wy_prep_kernel and state_pass_kernel "
+                               f"per round ({launches} launches, 2 streams, pipelined)",
+                     "kernel_ms": kernel_ms,
                      "tensor_frac": tensor_ach / peaks["bf16_tflops"],
                      "tensor_achieved_tflops": tensor_ach, "hbm_frac": hbm_ach / peaks["hbm_gbs"],
                      "floor_us": {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6},
-                     "traffic": kernel_traffic("prefill_tc", src)})
+                     "traffic": None if ent is None else ent["dram_bytes_per_launch"],
+                     "dominant": None if ent is None else ent.get("dominant")})
     else:
         # CUDA-core path: 3 fp32 FMAs per state element per token (read, update, output)
         flop = 3 * 2 * w.D * w.D * w.Hv * T
@@ -357,7 +381,7 @@ def run_ours(args, D):
                    "parallelism": f"replicas{D.world}" if D.world > 1 else "single GPU",
                    "l2": "flushed between timed steps (256 MiB write outside the timed pair)"},
         "roofline": roof,
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * launches,
     }
 
     if not args.no_e2e:

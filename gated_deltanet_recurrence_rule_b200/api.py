@@ -58,6 +58,8 @@ def load():
         lib.gdn_version.argtypes = []
         lib.gdn_prefill_workspace_size.restype = sz
         lib.gdn_prefill_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32, i32]
+        lib.gdn_prefill_launch_count.restype = i64
+        lib.gdn_prefill_launch_count.argtypes = [i32, i64, i32, i32, i32, i32, i32, sz]
         lib.gdn_prefill_workspace_size_rounds.restype = sz
         lib.gdn_prefill_workspace_size_rounds.argtypes = [i32, i64, i32, i32, i32, i32, i32, i64]
         lib.gdn_prefill.restype = i32
@@ -114,6 +116,13 @@ def prefill_workspace_size(num_seqs, total_tokens, Hqk, Hv, Dk, Dv, dtype=torch.
                                                          _DTYPE_CODE[dtype], chunks_per_round))
     return int(lib.gdn_prefill_workspace_size(num_seqs, total_tokens, Hqk, Hv, Dk, Dv,
                                               _DTYPE_CODE[dtype]))
+
+
+def prefill_launch_count(num_seqs, total_tokens, Hqk, Hv, Dk, Dv, workspace_bytes,
+                         dtype=torch.bfloat16) -> int:
+    """Kernel launches one prefill call makes with a workspace of that size."""
+    return int(load().gdn_prefill_launch_count(num_seqs, total_tokens, Hqk, Hv, Dk, Dv,
+                                               _DTYPE_CODE[dtype], workspace_bytes))
 
 
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_state=True,

@@ -27,6 +27,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
 size_t twophase_workspace_bytes(int64_t N, int64_t T, int Hv);
 size_t twophase_round_workspace_bytes(int64_t N, int Hv, int64_t chunks_per_round);
 size_t twophase_min_workspace_bytes(int64_t N, int Hv);
+int64_t twophase_launch_count(int64_t N, int64_t T, int Hv, size_t workspace_bytes);
 cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const int32_t *cu, int N, long long T_,
                                     int Hqk, int Hv, int o_dtype, float scale, const float *s0,
@@ -105,6 +106,21 @@ size_t gdn_prefill_workspace_size_rounds(int32_t num_seqs, int64_t total_tokens,
     return full;
   const size_t r = gdn::twophase_round_workspace_bytes(num_seqs, num_v_heads, chunks_per_round);
   return r < full ? r : full;
+}
+
+int64_t gdn_prefill_launch_count(int32_t num_seqs, int64_t total_tokens, int32_t num_qk_heads,
+                                 int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
+                                 int32_t dtype, size_t workspace_bytes) {
+  if (num_seqs < 0 || total_tokens < 0 ||
+      !dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype))
+    return -1;
+  if (!dims_supported(head_dim_k, head_dim_v)) return -1;
+  if (num_seqs == 0) return 0;
+  if (workspace_bytes < gdn::kWorkspaceHeaderBytes) return -1;
+  if (gdn::prefill_tc_supported(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype) &&
+      workspace_bytes >= gdn::twophase_min_workspace_bytes(num_seqs, num_v_heads))
+    return gdn::twophase_launch_count(num_seqs, total_tokens, num_v_heads, workspace_bytes);
+  return 1;  // one single-pass kernel
 }
 
 int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,

@@ -604,6 +604,18 @@ size_t twophase_round_workspace_bytes(int64_t N, int Hv, int64_t chunks_per_roun
   return L.fixed + (size_t)chunks_per_round * L.rec_row;
 }
 
+// Kernel launches of one two-phase prefill with this workspace: the plan
+// kernel, then phase 1 and phase 2 per round.
+int64_t twophase_launch_count(int64_t N, int64_t T, int Hv, size_t workspace_bytes) {
+  if (T == 0) return 1;
+  const tp::Layout L = tp::layout(N, Hv);
+  const int64_t bound = tp::chunk_bound(N, T);
+  const bool pipelined = workspace_bytes >= twophase_workspace_bytes(N, T, Hv);
+  const int64_t fit = (int64_t)((workspace_bytes - L.fixed) / L.rec_row);
+  const int64_t rc = std::min<int64_t>(pipelined ? pipelined_round_chunks(N, T) : std::min(bound, fit), 1 << 20);
+  return 1 + 2 * ((bound + rc - 1) / rc);
+}
+
 template <typename TO>
 static cudaError_t launch_state_pass(const CUtensorMap &mq, const CUtensorMap &mk,
                                      const sp::Params &prm, int grid_x, cudaStream_t stream) {

@@ -102,6 +102,15 @@ size_t gdn_prefill_workspace_size_rounds(int32_t num_seqs, int64_t total_tokens,
                                          int64_t chunks_per_round);
 
 /*
+ * Number of kernel launches one gdn_prefill call with these sizes and this
+ * workspace makes (0 for num_seqs = 0), or -1 for invalid arguments.  Host
+ * only.  For sizing CUDA graphs and for counting launches in benchmarks.
+ */
+int64_t gdn_prefill_launch_count(int32_t num_seqs, int64_t total_tokens, int32_t num_qk_heads,
+                                 int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
+                                 int32_t dtype, size_t workspace_bytes);
+
+/*
  * Prefill: run the recurrence over num_seqs packed sequences.
  *
  * The chunked (block-parallel) form: "Inside Qwen3.8-27B ...", section "Gated

@@ -60,6 +60,19 @@ def test_workspace_size_rounds(lib):
     assert api.prefill_workspace_size(1, 256, 2, 6, 64, 64, torch.float32, chunks_per_round=2) == 256
 
 
+def test_launch_count(lib):
+    """One launch for the single-pass and CUDA-core kernels; plan + two per
+    round for the two-phase kernels (8 pipelined rounds of 17 chunks at 8k)."""
+    full = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128)
+    assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, full) == 1 + 2 * 8
+    assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, 256) == 1
+    one_row = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=1)
+    assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, one_row) == 1 + 2 * 129
+    assert api.prefill_launch_count(1, 256, 2, 6, 64, 64, 256, torch.float32) == 1
+    assert api.prefill_launch_count(0, 0, 16, 48, 128, 128, full) == 0
+    assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, 100) == -1
+
+
 def test_workspace_size(lib):
     assert api.prefill_workspace_size(1, 8192, 16, 48, 128, 128) >= 256
     assert lib.gdn_prefill_workspace_size(-1, 10, 16, 48, 128, 128, 0) == 0

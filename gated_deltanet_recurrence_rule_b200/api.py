@@ -68,6 +68,9 @@ def load():
         lib.gdn_decode_step.restype = i32
         lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                         i32, f32, vp]
+        lib.gdn_decode_tokens.restype = i32
+        lib.gdn_decode_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
+                                          i32, i32, i32, i32, i32, f32, vp, vp]
         lib.gdn_prefill_uses_tensor_cores.restype = i32
         lib.gdn_prefill_uses_tensor_cores.argtypes = [i32, i32, i32, i32, i32]
         lib.gdn_get_device_status.restype = i32
@@ -208,6 +211,52 @@ def decode_step(q, k, v, g, beta, state, o=None, scale=1.0, o_dtype=torch.float3
                              B, Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], _DTYPE_CODE[o.dtype],
                              float(scale), _stream(dev))
     _check(st, "gdn_decode_step")
+    return o
+
+
+def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst_slot=None,
+                  o=None, scale=1.0, o_dtype=torch.float32, device_status=None):
+    """Several tokens per sequence against a pool of states.
+
+    q, k [B, Tn, Hqk, Dk]; v [B, Tn, Hv, Dv]; g, beta [B, Tn, Hv] fp32;
+    state_in [num_slots, Hv, Dv, Dk] fp32; state_out the same shape (default:
+    state_in, updated in place); src_slot / dst_slot [B] int32 or None (slot b /
+    the source slot); device_status an int32 device tensor of one element or
+    None.  Returns o [B, Tn, Hv, Dv] in ``o_dtype``."""
+    lib = load()
+    if not q.is_cuda:
+        raise ValueError("decode_tokens runs on a CUDA device only (q is on the CPU)")
+    dev = q.device
+    B, Tn, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[2], v.shape[3]
+    dt = q.dtype
+    if dt not in _DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dt}")
+    _require(q, "q", dev, dt)
+    _require(k, "k", dev, dt, (B, Tn, Hqk, Dk))
+    _require(v, "v", dev, dt, (B, Tn, Hv, Dv))
+    _require(g, "g", dev, torch.float32, (B, Tn, Hv))
+    _require(beta, "beta", dev, torch.float32, (B, Tn, Hv))
+    num_slots = state_in.shape[0]
+    _require(state_in, "state_in", dev, torch.float32, (num_slots, Hv, Dv, Dk))
+    if state_out is None:
+        state_out = state_in
+    _require(state_out, "state_out", dev, torch.float32, (num_slots, Hv, Dv, Dk))
+    for name, sl in (("src_slot", src_slot), ("dst_slot", dst_slot)):
+        if sl is not None:
+            _require(sl, name, dev, torch.int32, (B,))
+    if device_status is not None:
+        _require(device_status, "device_status", dev, torch.int32, (1,))
+    if o is None:
+        o = torch.empty((B, Tn, Hv, Dv), dtype=o_dtype, device=dev)
+    if o.dtype not in _DTYPE_CODE:
+        raise ValueError(f"unsupported o dtype {o.dtype}")
+    _require(o, "o", dev, None, (B, Tn, Hv, Dv))
+    st = lib.gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
+                               _ptr(state_out), _ptr(src_slot), _ptr(dst_slot), num_slots, _ptr(o),
+                               B, Tn, Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], _DTYPE_CODE[o.dtype],
+                               float(scale), _ptr(device_status), _stream(dev))
+    _check(st, "gdn_decode_tokens")
     return o
 
 

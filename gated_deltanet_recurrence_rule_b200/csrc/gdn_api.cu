@@ -19,6 +19,12 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, con
                                 int Hqk, int Hv, int Dk, int Dv, int dtype, int o_dtype,
                                 float scale, const float *s0, float *sfin, void *o,
                                 int32_t *status, cudaStream_t stream);
+int decode_tokens_max();
+cudaError_t launch_decode_tokens(const void *q, const void *k, const void *v, const float *g,
+                                 const float *beta, const float *state_in, float *state_out,
+                                 const int32_t *src_slot, const int32_t *dst_slot, int num_slots,
+                                 void *o, int B, int Tn, int Hqk, int Hv, int Dk, int Dv, int dtype,
+                                 int o_dtype, float scale, int32_t *status, cudaStream_t s);
 bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, int N, long long T_,
@@ -189,6 +195,33 @@ int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float
   return cuda_status(gdn::launch_decode(q, k, v, g, beta, state, o, batch, num_qk_heads,
                                         num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype,
                                         scale, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *state_in, float *state_out,
+                          const int32_t *src_slot, const int32_t *dst_slot, int32_t num_slots,
+                          void *o, int32_t batch, int32_t tokens, int32_t num_qk_heads,
+                          int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
+                          int32_t dtype, int32_t o_dtype, float scale, int32_t *device_status,
+                          void *stream) {
+  if (batch < 0 || tokens < 0 || num_slots < 0) return GDN_ERR_INVALID_ARG;
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dtype_ok(o_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
+  if (tokens > gdn::decode_tokens_max()) return GDN_ERR_UNSUPPORTED;
+  if (batch == 0 || tokens == 0) return GDN_OK;
+  if ((int64_t)batch * num_v_heads > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !g || !beta || !state_in || !state_out || !o) return GDN_ERR_INVALID_ARG;
+  if (!src_slot && batch > num_slots) return GDN_ERR_INVALID_ARG;  // slot b for sequence b
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 4) ||
+      !aligned(state_in, 16) || !aligned(state_out, 16) || !aligned(g, 4) || !aligned(beta, 4) ||
+      (src_slot && !aligned(src_slot, 4)) || (dst_slot && !aligned(dst_slot, 4)) ||
+      (device_status && !aligned(device_status, 4)))
+    return GDN_ERR_INVALID_ARG;
+  return cuda_status(gdn::launch_decode_tokens(
+      q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, batch, tokens,
+      num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype, scale, device_status,
+      static_cast<cudaStream_t>(stream)));
 }
 
 int32_t gdn_prefill_uses_tensor_cores(int32_t num_qk_heads, int32_t num_v_heads,

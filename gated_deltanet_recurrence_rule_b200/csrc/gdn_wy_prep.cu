@@ -81,6 +81,7 @@ struct Params {
   const int32_t *cu;
   int T, Hqk, Hv;
   int round, rc;  // this launch covers global chunks [round rc, round rc + rc)
+  int resident;   // CTAs resident at once (2 per SM): the distance to the next CTA on a slot
   const tp::PlanHeader *plan;
   const int32_t *ne_seq, *ne_cs;
   unsigned char *rec;  // this round's records, [rc][Hv]
@@ -137,6 +138,21 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_arrive_expect_tx(fv, 16384);
       tma_load_3d(sb + OFF_V + 0, &tm_v, fv, 0, h, t0);
       tma_load_3d(sb + OFF_V + 8192, &tm_v, fv, 64, h, t0);
+      // Warm L2 with the tiles of the CTA that will most likely take this
+      // slot next (CTAs start in linear order), so that its loads hit L2.
+      const int lin = (int)(blockIdx.y * gridDim.x + blockIdx.x) + p.resident;
+      if (lin < (int)(gridDim.x * gridDim.y)) {
+        const int xn = lin % (int)gridDim.x, hn = lin / (int)gridDim.x;
+        const int gn = p.round * p.rc + xn;
+        if (gn < total) {
+          const int kn = tp::owner_of_chunk(p.ne_cs, n_ne, gn);
+          const int tn = p.cu[p.ne_seq[kn]] + (gn - p.ne_cs[kn]) * CH;
+          const int jn = hn / (p.Hv / p.Hqk);
+          tma_prefetch_3d(&tm_q, 0, jn, tn); tma_prefetch_3d(&tm_q, 64, jn, tn);
+          tma_prefetch_3d(&tm_k, 0, jn, tn); tma_prefetch_3d(&tm_k, 64, jn, tn);
+          tma_prefetch_3d(&tm_v, 0, hn, tn); tma_prefetch_3d(&tm_v, 64, hn, tn);
+        }
+      }
       // both tiles land before this CTA can exit
       if (!mbar_wait_landed(fq, 0) || !mbar_wait_landed(fv, 0)) {
         *abort_flag = 1;
@@ -339,6 +355,9 @@ cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const C
   wy::Params prm;
   prm.g = g; prm.beta = beta; prm.cu = cu; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv;
   prm.round = round; prm.rc = rc;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  prm.resident = 2 * sms;
   unsigned char *ws = static_cast<unsigned char *>(const_cast<void *>(workspace));
   prm.plan = reinterpret_cast<const tp::PlanHeader *>(ws + tp::kPlanHeaderOffset);
   prm.ne_seq = reinterpret_cast<const int32_t *>(ws + L.plan_off);

@@ -211,6 +211,48 @@ int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float
                         void *stream);
 
 /*
+ * Multi-token decode over a pool of states: `tokens` new tokens for each of
+ * `batch` sequences, each sequence's state read from one slot of `state_in`
+ * and written after the last token to one slot of `state_out`.  Serves
+ * speculative verification (several drafted tokens per call, the state written
+ * to a fresh slot so that a rejected draft leaves the old one intact) and
+ * continuous batching (sequences bound to arbitrary slots, padding entries).
+ * Same rule as gdn_decode_step, applied `tokens` times in order; each state is
+ * read from HBM once and written once per call.  (The pages' inference mode
+ * updates the state token by token: "Inside Qwen3.8-27B ...", section "Gated
+ * DeltaNet Mechanics".)
+ *
+ *   q, k        [batch, tokens, Hqk, Dk]   dtype
+ *   v           [batch, tokens, Hv, Dv]    dtype
+ *   g, beta     [batch, tokens, Hv]        fp32
+ *   state_in    [num_slots, Hv, Dv, Dk]    fp32 pool read
+ *   state_out   [num_slots, Hv, Dv, Dk]    fp32 pool written; may be state_in
+ *   src_slot    [batch] int32, device: slot of sequence b in state_in; NULL means
+ *               slot b.  A negative entry marks padding: nothing is read or
+ *               written for that sequence (its o is left untouched).
+ *   dst_slot    [batch] int32, device: slot written in state_out; NULL means the
+ *               source slot.  No two sequences may write the same slot, and a
+ *               written slot must not be another sequence's source slot in the
+ *               same call when state_out == state_in.
+ *   o           [batch, tokens, Hv, Dv]    o_dtype (output)
+ *   device_status  optional device int32 (caller's memory, NULL to discard): a
+ *               slot index >= num_slots (or a negative dst_slot for a real
+ *               sequence) is recorded as GDN_ERR_INVALID_ARG there (first error
+ *               wins, as with the workspace status word) and that sequence is
+ *               skipped.
+ *
+ * Supported: 1 <= tokens <= 16; Hv % Hqk == 0; Dk, Dv in {64, 128}; dtype and
+ * o_dtype each bf16 or fp32.  batch = 0 or tokens = 0 is a valid no-op.
+ */
+int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const float *g,
+                          const float *beta, const float *state_in, float *state_out,
+                          const int32_t *src_slot, const int32_t *dst_slot, int32_t num_slots,
+                          void *o, int32_t batch, int32_t tokens, int32_t num_qk_heads,
+                          int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
+                          int32_t dtype, int32_t o_dtype, float scale, int32_t *device_status,
+                          void *stream);
+
+/*
  * 1 if gdn_prefill with these sizes and dtype runs the tensor-core (tcgen05)
  * kernel, 0 if it runs the fp32 CUDA-core kernel or the arguments are invalid.
  * Host only; touches no device.

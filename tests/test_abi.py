@@ -73,6 +73,25 @@ def test_launch_count(lib):
     assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, 100) == -1
 
 
+def test_decode_tokens_validation(lib):
+    """Host-side rejections of gdn_decode_tokens (nothing is launched)."""
+    vp = ctypes.c_void_p(256)
+    args = dict(batch=2, tokens=4, Hqk=16, Hv=48, Dk=128, Dv=128, dtype=0, o_dtype=1)
+
+    def call(**kw):
+        a = {**args, **kw}
+        return lib.gdn_decode_tokens(vp, vp, vp, vp, vp, vp, vp, None, None, 4, vp, a["batch"],
+                                     a["tokens"], a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"],
+                                     a["o_dtype"], 1.0, None, None)
+
+    assert call(tokens=17) == api.GDN_ERR_UNSUPPORTED      # more than 16 tokens
+    assert call(Dk=96) == api.GDN_ERR_UNSUPPORTED
+    assert call(Hv=40) == api.GDN_ERR_INVALID_ARG            # 40 % 16 != 0
+    assert call(tokens=-1) == api.GDN_ERR_INVALID_ARG
+    assert call(batch=0) == api.GDN_OK and call(tokens=0) == api.GDN_OK
+    assert call(batch=5) == api.GDN_ERR_INVALID_ARG          # no slot map: needs batch <= slots
+
+
 def test_workspace_size(lib):
     assert api.prefill_workspace_size(1, 8192, 16, 48, 128, 128) >= 256
     assert lib.gdn_prefill_workspace_size(-1, 10, 16, 48, 128, 128, 0) == 0

@@ -1,0 +1,89 @@
+"""Multi-token decode over a slot pool (gdn_decode_tokens) on the GPU against
+the fp64 oracle: each sequence's tokens are a prefill of that length from the
+state in its source slot, and the result lands in its destination slot."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_recurrence_rule_b200 import api, inputs
+from parity import assert_parity, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+
+
+def _case(B, Tn, Hqk, Hv, D, dtype, seed, num_slots, pool_std=0.3):
+    inp = inputs.prefill_inputs([Tn] * B, Hqk, Hv, D, dtype=dtype, seed=seed)
+    gen = torch.Generator().manual_seed(seed + 1000)
+    pool = torch.randn(num_slots, Hv, D, D, generator=gen) * pool_std
+    x = {"q": inp["q"].view(B, Tn, Hqk, D), "k": inp["k"].view(B, Tn, Hqk, D),
+         "v": inp["v"].view(B, Tn, Hv, D), "g": inp["g"].view(B, Tn, Hv),
+         "beta": inp["beta"].view(B, Tn, Hv)}
+    return inp, x, pool
+
+
+def _oracle(inp, pool, src, scale=1.0):
+    init = pool[torch.tensor(src, dtype=torch.long)]
+    return oracle.prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                          cu_seqlens=inp["cu_seqlens"], initial_state=init, scale=scale)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Tn", [1, 3, 16])
+def test_slots_against_oracle(dtype, D, Tn):
+    B, Hqk, Hv, slots = 3, 2, 6, 7
+    inp, x, pool = _case(B, Tn, Hqk, Hv, D, dtype, seed=31 + Tn, num_slots=slots)
+    src, dst = [4, 0, 6], [2, 5, 1]
+    pin = pool.to(DEV)
+    pout = torch.full_like(pin, float("nan"))
+    o = api.decode_tokens(*(x[n].to(DEV) for n in ("q", "k", "v", "g", "beta")), pin, pout,
+                          src_slot=torch.tensor(src, dtype=torch.int32, device=DEV),
+                          dst_slot=torch.tensor(dst, dtype=torch.int32, device=DEV), scale=0.5)
+    torch.cuda.synchronize()
+    o_ref, f_ref = _oracle(inp, pool, src, scale=0.5)
+    o_gpu = to_np(o).reshape(B * Tn, Hv, D)
+    assert_parity(inputs.DTYPES[dtype], o_gpu, o_ref, to_np(pout[dst]), f_ref, f"Tn={Tn}")
+    untouched = [s for s in range(slots) if s not in dst]
+    assert torch.isnan(pout[untouched]).all()          # only destination slots written
+    assert torch.equal(pin.cpu(), pool)                 # the input pool is only read
+
+
+def test_single_token_matches_decode_step():
+    """tokens = 1 with the identity slot map is the decode step, bit for bit."""
+    B, Hqk, Hv, D = 4, 2, 6, 128
+    inp, x, pool = _case(B, 1, Hqk, Hv, D, "bf16", seed=40, num_slots=B)
+    S1 = pool.to(DEV)
+    S2 = pool.to(DEV)
+    o1 = api.decode_tokens(*(x[n].to(DEV) for n in ("q", "k", "v", "g", "beta")), S1)
+    o2 = api.decode_step(*(x[n][:, 0].to(DEV) for n in ("q", "k", "v", "g", "beta")), S2)
+    torch.cuda.synchronize()
+    assert torch.equal(o1[:, 0], o2) and torch.equal(S1, S2)
+
+
+def test_in_place_padding_and_bad_slot():
+    """In place (state_out = state_in); a padding entry (-1) reads and writes
+    nothing; an out-of-range slot is reported and skipped."""
+    B, Tn, Hqk, Hv, D, slots = 4, 4, 2, 6, 128, 5
+    inp, x, pool = _case(B, Tn, Hqk, Hv, D, "bf16", seed=41, num_slots=slots)
+    src = [3, -1, 9, 0]
+    S = pool.to(DEV)
+    o = torch.full((B, Tn, Hv, D), 7.0, device=DEV)
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    api.decode_tokens(*(x[n].to(DEV) for n in ("q", "k", "v", "g", "beta")), S, o=o,
+                      src_slot=torch.tensor(src, dtype=torch.int32, device=DEV),
+                      device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == api.GDN_ERR_INVALID_ARG
+    assert (o[1] == 7).all() and (o[2] == 7).all()      # padding and bad slot untouched
+    for s in (1, 2, 4):
+        assert torch.equal(S[s].cpu(), pool[s])          # slots nobody uses stay as they were
+    keep = [0, 3]
+    o_ref, f_ref = _oracle({n: (t.view(B, Tn, *t.shape[1:])[keep].reshape(-1, *t.shape[1:])
+                                if n in ("q", "k", "v", "g", "beta") else t)
+                            for n, t in inp.items() if n != "cu_seqlens"} |
+                           {"cu_seqlens": torch.tensor([0, Tn, 2 * Tn], dtype=torch.int32)},
+                           pool, [src[b] for b in keep])
+    assert_parity(torch.bfloat16, to_np(o[keep]).reshape(-1, Hv, D), o_ref,
+                  to_np(S[[src[b] for b in keep]]), f_ref, "in place")

@@ -12,6 +12,8 @@ resident in HBM, L2 flushed between timed steps.  The same line carries:
                per launch / CUDA-event launch time, over the measured peak);
   decode       the batched decode workload (B=64, 1000 steps, fp32 state of
                201 MB updated in place): state GB/s against HBM peak;
+  decode_tokens  the same batch with 4 tokens per sequence per call through the
+               multi-token decode over a state pool: tokens/s, GB/s against HBM peak;
   e2e          prefill through the public API with inputs copied from pinned
                host memory and o / final state copied back, every step;
   cpu_baseline the fp64 oracle on the host cores (rank 0, N=1 only);
@@ -389,6 +391,7 @@ def run_ours(args, D):
 
     if not args.no_decode:
         out["decode"] = _decode(args, D, dev, peaks, peak_src)
+        out["decode_tokens"] = _decode_tokens(args, D, dev, peaks, peak_src)
     clk.__exit__(None, None, None)
     out["clocks"] = clk.summary()
 
@@ -495,6 +498,60 @@ def _decode(args, D, dev, peaks, peak_src):
                          "algorithmic": f"{per_step} B per step (state read+write {2 * state_bytes} + io {io_bytes})",
                          "traffic": kernel_traffic("decode", os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_decode.cu"))},
             "gpu_launches": steps}
+
+
+def _decode_tokens(args, D, dev, peaks, peak_src, tokens=4):
+    """Multi-token decode (gdn_decode_tokens): the decode64 batch with ``tokens``
+    new tokens per sequence per call, states updated in place in a 64-slot pool."""
+    import torch
+
+    from gated_deltanet_recurrence_rule_b200 import api, inputs
+
+    w = inputs.WORKLOADS["decode64"]
+    calls = max(args.decode_steps // tokens, 4)
+    d = inputs.decode_inputs(w.batch, w.Hqk, w.Hv, w.D, steps=calls * tokens, dtype=w.dtype,
+                             seed=rank_seed(w.seed, D.rank), init_std=w.init_std)
+
+    def per_call(t):  # [calls*tokens, B, ...] -> [calls, B, tokens, ...]
+        t = t.view(calls, tokens, *t.shape[1:])
+        return t.transpose(1, 2).contiguous().to(dev)
+
+    x = {n: per_call(d[n]) for n in ("q", "k", "v", "g", "beta")}
+    S = d["state"].to(dev)
+    o = torch.empty((w.batch, tokens, w.Hv, w.D), dtype=torch.float32, device=dev)
+
+    def run(n):
+        for c in range(n):
+            api.decode_tokens(x["q"][c], x["k"][c], x["v"][c], x["g"][c], x["beta"][c], S, o=o)
+
+    run(min(calls, 4))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    run(calls)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    ms = D.max(e0.elapsed_time(e1), dev)
+    state_bytes = w.batch * w.Hv * w.D * w.D * 4
+    io_bytes = tokens * w.batch * (2 * w.Hqk * w.D * 2 + w.Hv * w.D * 2 + w.Hv * w.D * 4 + 2 * w.Hv * 4)
+    per_call_bytes = 2 * state_bytes + io_bytes
+    gbs = D.world * per_call_bytes * calls / (ms / 1e3) / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"value": D.world * w.batch * tokens * calls / (ms / 1e3), "unit": "tokens/s",
+            "workload": f"decode64 with {tokens} tokens per sequence per call: B={w.batch}, "
+                        f"Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16, fp32 state pool of {w.batch} slots "
+                        f"in place, {calls} calls",
+            "us_per_call": ms * 1e3 / calls,
+            "roofline": {"bound": "hbm", "kernel": "decode_tokens_kernel", "achieved": gbs / D.world,
+                         "peak": peak, "unit": "GB/s", "frac": gbs / D.world / peak,
+                         "peak_source": f"{peak_src} hbm_gbs",
+                         "algorithmic": f"{per_call_bytes} B per call (state read+write {2 * state_bytes} + io {io_bytes})",
+                         "traffic": kernel_traffic("decode_tokens", os.path.join(CSRC, "gdn_decode.cu"))},
+            "gpu_launches": calls}
 
 
 def main(argv=None):

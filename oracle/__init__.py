@@ -51,6 +51,8 @@ def _bind(lib):
     lib.gdn_oracle_prefill.argtypes = [d, d, d, d, d, i64, ci, ci, ci, ci, ci, cd, d, d, d, ci, ci]
     lib.gdn_oracle_decode_step.restype = ci
     lib.gdn_oracle_decode_step.argtypes = [d, d, d, d, d, d, d, ci, ci, ci, ci, ci, cd, ci]
+    lib.gdn_oracle_round_bf16.restype = ci
+    lib.gdn_oracle_round_bf16.argtypes = [d, ctypes.c_int64]
     return lib
 
 
@@ -88,14 +90,27 @@ def _ptr(a):
     return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
 
 
+def round_bf16(x, lib=None):
+    """x rounded to the nearest bf16 value (ties to even), in fp64: the value a
+    state kept at rest in bf16 holds.  Returns a new fp64 array."""
+    lib = lib or load()
+    y = _f64(x).copy()
+    rc = lib.gdn_oracle_round_bf16(_ptr(y), int(y.size))
+    if rc != 0:
+        raise ValueError(f"gdn_oracle_round_bf16 failed with code {rc}")
+    return y
+
+
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, scale=1.0, chunk=0,
-            num_threads=0, want_final=True, lib=None):
+            num_threads=0, want_final=True, state_at_rest=None, lib=None):
     """Run the recurrence over packed sequences in fp64.
 
     q, k: [T, Hqk, Dk]; v: [T, Hv, Dv]; g, beta: [T, Hv]; cu_seqlens: [N+1]
     (default: one sequence of T tokens); initial_state: [N, Hv, Dv, Dk] or
     None (zeros).  chunk=0 is the token-by-token definition; chunk>0 the
-    chunked WY/UT form.  Returns (o [T, Hv, Dv], final_state [N, Hv, Dv, Dk]).
+    chunked WY/UT form.  state_at_rest="bf16" rounds the final state to bf16
+    (a state stored in bf16 between calls; the arithmetic stays fp64).
+    Returns (o [T, Hv, Dv], final_state [N, Hv, Dv, Dk]).
     """
     lib = lib or load()
     q, k, v, g, beta = (_f64(t) for t in (q, k, v, g, beta))
@@ -120,13 +135,18 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, scale=1.0, ch
         _ptr(s0), _ptr(fin), _ptr(o), int(chunk), int(num_threads))
     if rc != 0:
         raise ValueError(f"gdn_oracle_prefill failed with code {rc}")
+    if state_at_rest not in (None, "fp64", "bf16"):
+        raise ValueError(f"unknown state_at_rest {state_at_rest!r}")
+    if state_at_rest == "bf16" and fin is not None:
+        fin = round_bf16(fin, lib)
     return o, fin
 
 
-def decode_step(q, k, v, g, beta, state, scale=1.0, num_threads=0, lib=None):
+def decode_step(q, k, v, g, beta, state, scale=1.0, num_threads=0, state_at_rest=None, lib=None):
     """One token for each of B sequences.  q, k: [B, Hqk, Dk]; v: [B, Hv, Dv];
     g, beta: [B, Hv]; state: [B, Hv, Dv, Dk].  Returns (o [B, Hv, Dv],
-    new_state) and leaves the argument ``state`` untouched."""
+    new_state) and leaves the argument ``state`` untouched; state_at_rest="bf16"
+    rounds new_state to bf16."""
     lib = lib or load()
     q, k, v, g, beta = (_f64(t) for t in (q, k, v, g, beta))
     S = _f64(state).copy()
@@ -137,4 +157,8 @@ def decode_step(q, k, v, g, beta, state, scale=1.0, num_threads=0, lib=None):
                                     _ptr(o), B, Hqk, Hv, Dk, Dv, float(scale), int(num_threads))
     if rc != 0:
         raise ValueError(f"gdn_oracle_decode_step failed with code {rc}")
+    if state_at_rest not in (None, "fp64", "bf16"):
+        raise ValueError(f"unknown state_at_rest {state_at_rest!r}")
+    if state_at_rest == "bf16":
+        S = round_bf16(S, lib)
     return o, S

@@ -323,3 +323,32 @@ int gdn_oracle_decode_step(const double *q, const double *k, const double *v, co
     free(cu);
     return rc;
 }
+
+/*
+ * States kept at rest in bf16: round each x[i] to the nearest value of the
+ * bf16 format, ties to even, straight from fp64 (one rounding, no fp32 step).
+ * bf16 keeps 8 significant bits and the exponent range of IEEE binary32: in
+ * the binade [2^(e-1), 2^e) its values are the multiples of 2^(e-8); below
+ * 2^-126 (subnormals) the multiples of 2^-133; the largest finite value is
+ * (2 - 2^-7) 2^127, and a value that rounds above it becomes infinite.  This
+ * is IEEE 754 round-to-nearest-even applied to that format, written out.
+ * Returns 0, or 1 for a bad argument.
+ */
+int gdn_oracle_round_bf16(double *x, int64_t n)
+{
+    if (n < 0 || (n > 0 && !x)) return ORACLE_BAD_ARG;
+    const double bf16_max = ldexp(255.0, 120); /* (2 - 2^-7) 2^127 */
+    for (int64_t i = 0; i < n; ++i) {
+        const double a = x[i];
+        if (!isfinite(a) || a == 0.0) continue;
+        int e;
+        frexp(a, &e); /* a = m 2^e with 0.5 <= |m| < 1 */
+        int qexp = e - 8;
+        if (qexp < -133) qexp = -133;
+        const double r = nearbyint(ldexp(a, -qexp)); /* default rounding mode: ties to even */
+        double y = ldexp(r, qexp);
+        if (fabs(y) > bf16_max) y = copysign(INFINITY, a);
+        x[i] = y;
+    }
+    return ORACLE_OK;
+}

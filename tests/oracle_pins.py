@@ -281,8 +281,69 @@ def check_chunked(lib, seed=10):
         _close(fin, f_ref, 1e-11, f"chunked C={C} state")
 
 
+def check_round_bf16(lib, seed=11):
+    """bf16 at rest: round to nearest, ties to even, 8 significant bits.
+
+    Hand-worked values of the format (the spacing of bf16 is 2^-7 in [1, 2),
+    2^-133 below 2^-126, the largest finite value is (2 - 2^-7) 2^127), then
+    torch's own fp32 -> bf16 conversion (an independent round-to-nearest-even)
+    on random fp32 values and on constructed ties, where the fp64 -> bf16
+    rounding of the oracle must agree exactly."""
+    import torch
+
+    cases = [
+        (1 + 2 ** -8, 1.0),                       # tie between 1 and 1 + 2^-7: even is 1
+        (1 + 3 * 2 ** -8, 1 + 2 ** -6),           # tie between 1 + 2^-7 and 1 + 2^-6: even is the upper
+        (1 + 2 ** -8 + 2 ** -30, 1 + 2 ** -7),    # just above a tie
+        (-(1 + 2 ** -8 + 2 ** -30), -(1 + 2 ** -7)),
+        (1 + 2 ** -7 + 2 ** -9, 1 + 2 ** -7),     # below a tie
+        (3 * 2 ** -9 + 2 ** -40, 3 * 2 ** -9),    # binade [2^-8, 2^-7), spacing 2^-15
+        (0.5 * 2 ** -133, 0.0),                   # half the smallest subnormal: tie to even (zero)
+        (0.75 * 2 ** -133, 2 ** -133),
+        (3.2 * 2 ** -133, 3 * 2 ** -133),
+        (255 * 2 ** 120 + 2 ** 119, math.inf),    # largest finite + half a spacing: tie, overflows
+        (255 * 2 ** 120 + 2 ** 118, 255 * 2 ** 120),
+        (0.0, 0.0), (-0.0, -0.0),
+    ]
+    got = oracle.round_bf16(np.array([c[0] for c in cases]), lib)
+    for (x, want), y in zip(cases, got):
+        assert y == want and math.copysign(1, y) == math.copysign(1, want), \
+            f"round_bf16({x!r}) = {y!r}, want {want!r}"
+
+    r = _rng(seed)
+    f32 = (r.standard_normal(4096) * np.exp(r.uniform(-30, 30, 4096))).astype(np.float32)
+    bits = r.integers(0, 2 ** 16, 512, dtype=np.uint32) << 16 | np.uint32(0x8000)  # exact ties
+    bits = bits[(bits >> 23 & 0xFF) != 0xFF]                                  # finite ones
+    f32 = np.concatenate([f32, bits.view(np.float32)])
+    want = torch.from_numpy(f32).to(torch.bfloat16).to(torch.float64).numpy()
+    got = oracle.round_bf16(f32.astype(np.float64), lib)
+    bad = np.flatnonzero(~((got == want) | (np.isnan(got) & np.isnan(want))))
+    assert bad.size == 0, f"round_bf16 differs from fp32->bf16 RNE at {f32[bad[:3]]}: {got[bad[:3]]} vs {want[bad[:3]]}"
+
+
+def check_state_at_rest_bf16(lib, seed=12):
+    """With the state at rest in bf16, the returned final state is the exact
+    fp64 one rounded once: every value is a bf16 value (it survives a round
+    trip through torch.bfloat16 unchanged), lies within half a bf16 spacing of
+    the exact value, and o is untouched by the rounding."""
+    import torch
+
+    q, k, v, g, beta, s0 = random_problem(seed, T=9, Hqk=1, Hv=2, Dk=8, Dv=4, N=2)
+    cu = np.array([0, 4, 9])
+    o_ex, f_ex = oracle.prefill(q, k, v, g, beta, cu, s0, lib=lib)
+    o_r, f_r = oracle.prefill(q, k, v, g, beta, cu, s0, state_at_rest="bf16", lib=lib)
+    assert np.array_equal(o_ex, o_r), "o must not depend on how the final state is stored"
+    back = torch.from_numpy(f_r).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(back, f_r), "final state holds values that are not bf16"
+    _, e = np.frexp(f_ex)
+    half = np.ldexp(1.0, np.maximum(e - 9, -134))
+    assert (np.abs(f_r - f_ex) <= half).all(), "rounded state is not the nearest bf16 value"
+    assert not np.array_equal(f_r, f_ex), "rounding changed nothing: inputs too coarse to test it"
+
+
 ALL_CHECKS = [
     check_product_form, check_golden_scalar, check_golden_matrix, check_no_write_no_decay,
     check_exact_writeback, check_reset, check_pure_decay, check_orthonormal_memory, check_scale,
-    check_gqa_mapping, check_varlen, check_decode, check_chunked,
+    check_gqa_mapping, check_varlen, check_decode, check_chunked, check_round_bf16,
+    check_state_at_rest_bf16,
 ]

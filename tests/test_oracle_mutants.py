@@ -38,6 +38,11 @@ MUTANTS = [
     ("chunk_decay_off_by_one", "a = BVAL(r) * exp(G[r] - G[s]) * kk;", "a = BVAL(r) * exp(G[r] - G[s + 1]) * kk;"),
     ("chunk_output_strict", "for (int s = 0; s <= r; ++s) {", "for (int s = 0; s < r; ++s) {"),
     ("chunk_carry_undecayed", "double x = eL * S[(size_t)i * Dk + c];", "double x = S[(size_t)i * Dk + c];"),
+    ("bf16_ties_away", "const double r = nearbyint(ldexp(a, -qexp));", "const double r = round(ldexp(a, -qexp));"),
+    ("bf16_truncate", "const double r = nearbyint(ldexp(a, -qexp));", "const double r = trunc(ldexp(a, -qexp));"),
+    ("bf16_seven_bits", "int qexp = e - 8;", "int qexp = e - 7;"),
+    ("bf16_no_subnormal_floor", "if (qexp < -133) qexp = -133;", "if (qexp < -149) qexp = -149;"),
+    ("bf16_no_overflow", "if (fabs(y) > bf16_max) y = copysign(INFINITY, a);", "(void)bf16_max;"),
 ]
 
 

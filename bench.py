@@ -14,6 +14,9 @@ resident in HBM, L2 flushed between timed steps.  The same line carries:
                201 MB updated in place): state GB/s against HBM peak;
   decode_tokens  the same batch with 4 tokens per sequence per call through the
                multi-token decode over a state pool: tokens/s, GB/s against HBM peak;
+  decode_bf16_state, decode_tokens_bf16_state
+               the same with the state pool at rest in bf16 (fp32 arithmetic,
+               100 MB of state), 1 and 4 tokens per call;
   e2e          prefill through the public API with inputs copied from pinned
                host memory and o / final state copied back, every step;
   cpu_baseline the fp64 oracle on the host cores (rank 0, N=1 only);
@@ -392,6 +395,10 @@ def run_ours(args, D):
     if not args.no_decode:
         out["decode"] = _decode(args, D, dev, peaks, peak_src)
         out["decode_tokens"] = _decode_tokens(args, D, dev, peaks, peak_src)
+        out["decode_bf16_state"] = _decode_tokens(args, D, dev, peaks, peak_src, tokens=1,
+                                                  state_dtype="bf16")
+        out["decode_tokens_bf16_state"] = _decode_tokens(args, D, dev, peaks, peak_src,
+                                                         state_dtype="bf16")
     clk.__exit__(None, None, None)
     out["clocks"] = clk.summary()
 
@@ -500,9 +507,10 @@ def _decode(args, D, dev, peaks, peak_src):
             "gpu_launches": steps}
 
 
-def _decode_tokens(args, D, dev, peaks, peak_src, tokens=4):
+def _decode_tokens(args, D, dev, peaks, peak_src, tokens=4, state_dtype="fp32"):
     """Multi-token decode (gdn_decode_tokens): the decode64 batch with ``tokens``
-    new tokens per sequence per call, states updated in place in a 64-slot pool."""
+    new tokens per sequence per call, states updated in place in a 64-slot pool
+    kept in ``state_dtype`` (fp32, or bf16 at rest with fp32 arithmetic)."""
     import torch
 
     from gated_deltanet_recurrence_rule_b200 import api, inputs
@@ -517,7 +525,8 @@ def _decode_tokens(args, D, dev, peaks, peak_src, tokens=4):
         return t.transpose(1, 2).contiguous().to(dev)
 
     x = {n: per_call(d[n]) for n in ("q", "k", "v", "g", "beta")}
-    S = d["state"].to(dev)
+    sdt = {"fp32": torch.float32, "bf16": torch.bfloat16}[state_dtype]
+    S = d["state"].to(sdt).to(dev)
     o = torch.empty((w.batch, tokens, w.Hv, w.D), dtype=torch.float32, device=dev)
 
     def run(n):
@@ -536,21 +545,24 @@ def _decode_tokens(args, D, dev, peaks, peak_src, tokens=4):
     torch.cuda.synchronize()
     D.barrier()
     ms = D.max(e0.elapsed_time(e1), dev)
-    state_bytes = w.batch * w.Hv * w.D * w.D * 4
+    state_bytes = w.batch * w.Hv * w.D * w.D * S.element_size()
     io_bytes = tokens * w.batch * (2 * w.Hqk * w.D * 2 + w.Hv * w.D * 2 + w.Hv * w.D * 4 + 2 * w.Hv * 4)
     per_call_bytes = 2 * state_bytes + io_bytes
     gbs = D.world * per_call_bytes * calls / (ms / 1e3) / 1e9
     peak = peaks["hbm_gbs"]
+    kernel = "decode_tokens_bf16s_kernel" if state_dtype == "bf16" else "decode_tokens_kernel"
+    traffic_key = "decode_tokens" + ("" if tokens > 1 else "_1") + ("_bf16" if state_dtype == "bf16" else "")
     return {"value": D.world * w.batch * tokens * calls / (ms / 1e3), "unit": "tokens/s",
             "workload": f"decode64 with {tokens} tokens per sequence per call: B={w.batch}, "
-                        f"Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16, fp32 state pool of {w.batch} slots "
-                        f"in place, {calls} calls",
+                        f"Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16, {state_dtype} state pool of {w.batch} "
+                        f"slots in place, {calls} calls",
+            "state_dtype": state_dtype,
             "us_per_call": ms * 1e3 / calls,
-            "roofline": {"bound": "hbm", "kernel": "decode_tokens_kernel", "achieved": gbs / D.world,
+            "roofline": {"bound": "hbm", "kernel": kernel, "achieved": gbs / D.world,
                          "peak": peak, "unit": "GB/s", "frac": gbs / D.world / peak,
                          "peak_source": f"{peak_src} hbm_gbs",
                          "algorithmic": f"{per_call_bytes} B per call (state read+write {2 * state_bytes} + io {io_bytes})",
-                         "traffic": kernel_traffic("decode_tokens", os.path.join(CSRC, "gdn_decode.cu"))},
+                         "traffic": kernel_traffic(traffic_key, os.path.join(CSRC, "gdn_decode.cu"))},
             "gpu_launches": calls}
 
 

@@ -70,7 +70,7 @@ def load():
                                         i32, f32, vp]
         lib.gdn_decode_tokens.restype = i32
         lib.gdn_decode_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
-                                          i32, i32, i32, i32, i32, f32, vp, vp]
+                                          i32, i32, i32, i32, i32, i32, f32, vp, vp]
         lib.gdn_prefill_uses_tensor_cores.restype = i32
         lib.gdn_prefill_uses_tensor_cores.argtypes = [i32, i32, i32, i32, i32]
         lib.gdn_get_device_status.restype = i32
@@ -219,10 +219,11 @@ def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst
     """Several tokens per sequence against a pool of states.
 
     q, k [B, Tn, Hqk, Dk]; v [B, Tn, Hv, Dv]; g, beta [B, Tn, Hv] fp32;
-    state_in [num_slots, Hv, Dv, Dk] fp32; state_out the same shape (default:
-    state_in, updated in place); src_slot / dst_slot [B] int32 or None (slot b /
-    the source slot); device_status an int32 device tensor of one element or
-    None.  Returns o [B, Tn, Hv, Dv] in ``o_dtype``."""
+    state_in [num_slots, Hv, Dv, Dk] fp32 or bf16 (bf16: states at rest in
+    bf16, fp32 arithmetic, rounded once per call on store); state_out the same
+    shape and dtype (default: state_in, updated in place); src_slot / dst_slot
+    [B] int32 or None (slot b / the source slot); device_status an int32 device
+    tensor of one element or None.  Returns o [B, Tn, Hv, Dv] in ``o_dtype``."""
     lib = load()
     if not q.is_cuda:
         raise ValueError("decode_tokens runs on a CUDA device only (q is on the CPU)")
@@ -238,10 +239,13 @@ def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst
     _require(g, "g", dev, torch.float32, (B, Tn, Hv))
     _require(beta, "beta", dev, torch.float32, (B, Tn, Hv))
     num_slots = state_in.shape[0]
-    _require(state_in, "state_in", dev, torch.float32, (num_slots, Hv, Dv, Dk))
+    sdt = state_in.dtype
+    if sdt not in _DTYPE_CODE:
+        raise ValueError(f"unsupported state dtype {sdt}")
+    _require(state_in, "state_in", dev, sdt, (num_slots, Hv, Dv, Dk))
     if state_out is None:
         state_out = state_in
-    _require(state_out, "state_out", dev, torch.float32, (num_slots, Hv, Dv, Dk))
+    _require(state_out, "state_out", dev, sdt, (num_slots, Hv, Dv, Dk))
     for name, sl in (("src_slot", src_slot), ("dst_slot", dst_slot)):
         if sl is not None:
             _require(sl, name, dev, torch.int32, (B,))
@@ -255,7 +259,7 @@ def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst
     st = lib.gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
                                _ptr(state_out), _ptr(src_slot), _ptr(dst_slot), num_slots, _ptr(o),
                                B, Tn, Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], _DTYPE_CODE[o.dtype],
-                               float(scale), _ptr(device_status), _stream(dev))
+                               _DTYPE_CODE[sdt], float(scale), _ptr(device_status), _stream(dev))
     _check(st, "gdn_decode_tokens")
     return o
 

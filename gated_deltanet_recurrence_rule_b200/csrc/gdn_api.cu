@@ -21,10 +21,11 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, con
                                 int32_t *status, cudaStream_t stream);
 int decode_tokens_max();
 cudaError_t launch_decode_tokens(const void *q, const void *k, const void *v, const float *g,
-                                 const float *beta, const float *state_in, float *state_out,
+                                 const float *beta, const void *state_in, void *state_out,
                                  const int32_t *src_slot, const int32_t *dst_slot, int num_slots,
                                  void *o, int B, int Tn, int Hqk, int Hv, int Dk, int Dv, int dtype,
-                                 int o_dtype, float scale, int32_t *status, cudaStream_t s);
+                                 int o_dtype, int state_dtype, float scale, int32_t *status,
+                                 cudaStream_t s);
 bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, int N, long long T_,
@@ -198,15 +199,15 @@ int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float
 }
 
 int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const float *g,
-                          const float *beta, const float *state_in, float *state_out,
+                          const float *beta, const void *state_in, void *state_out,
                           const int32_t *src_slot, const int32_t *dst_slot, int32_t num_slots,
                           void *o, int32_t batch, int32_t tokens, int32_t num_qk_heads,
                           int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
-                          int32_t dtype, int32_t o_dtype, float scale, int32_t *device_status,
-                          void *stream) {
+                          int32_t dtype, int32_t o_dtype, int32_t state_dtype, float scale,
+                          int32_t *device_status, void *stream) {
   if (batch < 0 || tokens < 0 || num_slots < 0) return GDN_ERR_INVALID_ARG;
   if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
-  if (!dtype_ok(o_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dtype_ok(o_dtype) || !dtype_ok(state_dtype)) return GDN_ERR_INVALID_ARG;
   if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
   if (tokens > gdn::decode_tokens_max()) return GDN_ERR_UNSUPPORTED;
   if (batch == 0 || tokens == 0) return GDN_OK;
@@ -220,8 +221,8 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
     return GDN_ERR_INVALID_ARG;
   return cuda_status(gdn::launch_decode_tokens(
       q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, batch, tokens,
-      num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype, scale, device_status,
-      static_cast<cudaStream_t>(stream)));
+      num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype, state_dtype, scale,
+      device_status, static_cast<cudaStream_t>(stream)));
 }
 
 int32_t gdn_prefill_uses_tensor_cores(int32_t num_qk_heads, int32_t num_v_heads,

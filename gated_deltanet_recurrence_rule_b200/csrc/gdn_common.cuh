@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "gdn.h"
 
 namespace gdn {
@@ -59,6 +61,35 @@ __host__ auto dispatch_types(int dtype, int o_dtype, F &&f) {
   }
   if (o_dtype == GDN_DTYPE_BF16) return f(float{}, __nv_bfloat16{});
   return f(float{}, float{});
+}
+
+// ---- programmatic dependent launch ------------------------------------------
+// Kernels launched with launch_pdl may be scheduled while the previous kernel
+// on the stream is still finishing.  Each of them calls pdl_wait() before its
+// first global memory access: that waits until the previous grid has completed
+// and its writes are visible (a no-op when the kernel was launched normally),
+// so only launch latency and block scheduling overlap the previous kernel's
+// tail.  pdl_allow_next() lets the next such kernel be scheduled once every
+// block of this grid has started.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_next() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+__host__ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t stream, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 }  // namespace gdn

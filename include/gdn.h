@@ -225,8 +225,8 @@ int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float
  *   q, k        [batch, tokens, Hqk, Dk]   dtype
  *   v           [batch, tokens, Hv, Dv]    dtype
  *   g, beta     [batch, tokens, Hv]        fp32
- *   state_in    [num_slots, Hv, Dv, Dk]    fp32 pool read
- *   state_out   [num_slots, Hv, Dv, Dk]    fp32 pool written; may be state_in
+ *   state_in    [num_slots, Hv, Dv, Dk]    state_dtype, pool read
+ *   state_out   [num_slots, Hv, Dv, Dk]    state_dtype, pool written; may be state_in
  *   src_slot    [batch] int32, device: slot of sequence b in state_in; NULL means
  *               slot b.  A negative entry marks padding: nothing is read or
  *               written for that sequence (its o is left untouched).
@@ -235,6 +235,15 @@ int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float
  *               written slot must not be another sequence's source slot in the
  *               same call when state_out == state_in.
  *   o           [batch, tokens, Hv, Dv]    o_dtype (output)
+ *   state_dtype GDN_DTYPE_FP32, or GDN_DTYPE_BF16 for states at rest in bf16
+ *               (half the bytes per call).  The arithmetic is fp32 either way:
+ *               a bf16 state is widened exactly on load, carried in fp32 through
+ *               all `tokens` updates, and rounded to nearest even once, when it
+ *               is stored.  The fixed state of all DeltaNet layers is put at
+ *               some tens of megabytes in "Qwen3.8 Explained: 27B Multimodal,
+ *               2.4T MoE, and the VRAM Math", section "The architecture detail
+ *               that matters for VRAM"; bf16 at 48 layers x 48 heads x 128 x 128
+ *               is 72 MiB.
  *   device_status  optional device int32 (caller's memory, NULL to discard): a
  *               slot index >= num_slots (or a negative dst_slot for a real
  *               sequence) is recorded as GDN_ERR_INVALID_ARG there (first error
@@ -245,12 +254,12 @@ int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float
  * o_dtype each bf16 or fp32.  batch = 0 or tokens = 0 is a valid no-op.
  */
 int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const float *g,
-                          const float *beta, const float *state_in, float *state_out,
+                          const float *beta, const void *state_in, void *state_out,
                           const int32_t *src_slot, const int32_t *dst_slot, int32_t num_slots,
                           void *o, int32_t batch, int32_t tokens, int32_t num_qk_heads,
                           int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
-                          int32_t dtype, int32_t o_dtype, float scale, int32_t *device_status,
-                          void *stream);
+                          int32_t dtype, int32_t o_dtype, int32_t state_dtype, float scale,
+                          int32_t *device_status, void *stream);
 
 /*
  * 1 if gdn_prefill with these sizes and dtype runs the tensor-core (tcgen05)

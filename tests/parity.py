@@ -67,6 +67,24 @@ def assert_parity(dtype, o, o_ref, s=None, s_ref=None, what="", o_bf16=False):
     return eo, es
 
 
+def state_error_bf16_rest(s, s_ref, slack_rel=2e-5):
+    """Largest ratio of |s - s_ref| to the bound for states kept at rest in bf16
+    (<= 1 passes).  s_ref is the oracle's state rounded once to bf16 (fp64
+    arithmetic); s is the kernel's, computed in fp32 and rounded once.  With x
+    the exact value and x' = x + e the fp32 one (|e| <= eps), the two roundings
+    differ by at most half a bf16 spacing at each plus |e|, and a bf16 spacing
+    at y is at most 2^-7 |y|, so
+        |s - s_ref| <= 2^-7 (|s_ref| + 2 eps) + 2 eps,   eps = slack_rel * RMS(s_ref).
+    """
+    s = np.asarray(s, dtype=np.float64)
+    s_ref = np.asarray(s_ref, dtype=np.float64)
+    if not s_ref.size:
+        return 0.0
+    eps = slack_rel * float(np.sqrt(np.mean(s_ref ** 2)))
+    bound = 2.0 ** -7 * (np.abs(s_ref) + 2 * eps) + 2 * eps
+    return float((np.abs(s - s_ref) / np.maximum(bound, 1e-300)).max())
+
+
 def to_np(t):
     return t.detach().to("cpu", torch.float64).numpy()
 

@@ -76,13 +76,13 @@ def test_launch_count(lib):
 def test_decode_tokens_validation(lib):
     """Host-side rejections of gdn_decode_tokens (nothing is launched)."""
     vp = ctypes.c_void_p(256)
-    args = dict(batch=2, tokens=4, Hqk=16, Hv=48, Dk=128, Dv=128, dtype=0, o_dtype=1)
+    args = dict(batch=2, tokens=4, Hqk=16, Hv=48, Dk=128, Dv=128, dtype=0, o_dtype=1, s_dtype=1)
 
     def call(**kw):
         a = {**args, **kw}
         return lib.gdn_decode_tokens(vp, vp, vp, vp, vp, vp, vp, None, None, 4, vp, a["batch"],
                                      a["tokens"], a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"],
-                                     a["o_dtype"], 1.0, None, None)
+                                     a["o_dtype"], a["s_dtype"], 1.0, None, None)
 
     assert call(tokens=17) == api.GDN_ERR_UNSUPPORTED      # more than 16 tokens
     assert call(Dk=96) == api.GDN_ERR_UNSUPPORTED
@@ -90,6 +90,8 @@ def test_decode_tokens_validation(lib):
     assert call(tokens=-1) == api.GDN_ERR_INVALID_ARG
     assert call(batch=0) == api.GDN_OK and call(tokens=0) == api.GDN_OK
     assert call(batch=5) == api.GDN_ERR_INVALID_ARG          # no slot map: needs batch <= slots
+    assert call(s_dtype=2) == api.GDN_ERR_INVALID_ARG        # state dtype neither bf16 nor fp32
+    assert call(s_dtype=0, batch=0) == api.GDN_OK            # bf16 states accepted
 
 
 def test_workspace_size(lib):

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from gated_deltanet_recurrence_rule_b200 import api, inputs
-from parity import assert_parity, to_np
+from parity import assert_parity, state_error, state_error_bf16_rest, to_np
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -23,10 +23,11 @@ def _case(B, Tn, Hqk, Hv, D, dtype, seed, num_slots, pool_std=0.3):
     return inp, x, pool
 
 
-def _oracle(inp, pool, src, scale=1.0):
+def _oracle(inp, pool, src, scale=1.0, state_at_rest=None):
     init = pool[torch.tensor(src, dtype=torch.long)]
     return oracle.prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
-                          cu_seqlens=inp["cu_seqlens"], initial_state=init, scale=scale)
+                          cu_seqlens=inp["cu_seqlens"], initial_state=init, scale=scale,
+                          state_at_rest=state_at_rest)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
@@ -87,3 +88,62 @@ def test_in_place_padding_and_bad_slot():
                            pool, [src[b] for b in keep])
     assert_parity(torch.bfloat16, to_np(o[keep]).reshape(-1, Hv, D), o_ref,
                   to_np(S[[src[b] for b in keep]]), f_ref, "in place")
+
+
+# ---- states at rest in bf16 (fp32 arithmetic, one rounding per call) ---------
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Tn", [1, 4, 16])
+def test_bf16_state_against_oracle(dtype, D, Tn):
+    """bf16 pool: the oracle reads the same bf16 values, runs the tokens in fp64
+    and rounds the final state once; o within the input dtype's bound, the state
+    within one rounding of the oracle's (and within the bf16 bound, 5e-3, of the
+    unrounded result)."""
+    B, Hqk, Hv, slots = 3, 2, 6, 7
+    inp, x, pool = _case(B, Tn, Hqk, Hv, D, dtype, seed=51 + Tn, num_slots=slots)
+    pool = pool.to(torch.bfloat16)
+    src, dst = [4, 0, 6], [2, 5, 1]
+    pin = pool.to(DEV)
+    pout = torch.full_like(pin, float("nan"))
+    o = api.decode_tokens(*(x[n].to(DEV) for n in ("q", "k", "v", "g", "beta")), pin, pout,
+                          src_slot=torch.tensor(src, dtype=torch.int32, device=DEV),
+                          dst_slot=torch.tensor(dst, dtype=torch.int32, device=DEV), scale=0.5)
+    torch.cuda.synchronize()
+    o_ref, f_ref = _oracle(inp, pool, src, scale=0.5, state_at_rest="bf16")
+    _, f_exact = _oracle(inp, pool, src, scale=0.5)
+    s_gpu = to_np(pout[dst])
+    assert_parity(inputs.DTYPES[dtype], to_np(o).reshape(B * Tn, Hv, D), o_ref,
+                  what=f"bf16 state Tn={Tn}")
+    e = state_error_bf16_rest(s_gpu, f_ref)
+    assert e <= 1.0, f"bf16 state Tn={Tn}: {e:.3f}x the one-rounding bound"
+    # a state stored in bf16 is a bf16 quantity: the bf16 bound against the exact one
+    assert state_error(s_gpu, f_exact) <= 5e-3
+    untouched = [s for s in range(slots) if s not in dst]
+    assert torch.isnan(pout[untouched].float()).all()
+    assert torch.equal(pin.cpu(), pool)
+
+
+def test_bf16_state_many_calls():
+    """64 one-token calls and 16 four-token calls in place on a bf16 pool, each
+    followed on the oracle by one rounding of the state: the two stay within the
+    bf16-input bounds of each other (rounding flips of one bf16 spacing are the
+    only source of divergence, and the recurrence damps them)."""
+    B, Hqk, Hv, D = 4, 2, 6, 128
+    for Tn, calls in ((1, 64), (4, 16)):
+        inp, x, pool = _case(B, Tn * calls, Hqk, Hv, D, "bf16", seed=60 + Tn, num_slots=B)
+        pool = pool.to(torch.bfloat16)
+        S = pool.to(DEV)
+        ref = pool.to(torch.float64).numpy()
+        for c in range(calls):
+            sl = slice(c * Tn, (c + 1) * Tn)
+            xc = {n: x[n][:, sl].contiguous() for n in ("q", "k", "v", "g", "beta")}
+            o = api.decode_tokens(*(xc[n].to(DEV) for n in ("q", "k", "v", "g", "beta")), S)
+            o_ref, ref = oracle.prefill(
+                *(xc[n].reshape(B * Tn, *xc[n].shape[2:]) for n in ("q", "k", "v", "g", "beta")),
+                cu_seqlens=torch.arange(0, B * Tn + 1, Tn, dtype=torch.int32), initial_state=ref,
+                state_at_rest="bf16")
+        torch.cuda.synchronize()
+        assert_parity(torch.bfloat16, to_np(o).reshape(B * Tn, Hv, D), o_ref, to_np(S), ref,
+                      f"{calls} calls of {Tn}")
+        assert state_error(to_np(S), ref) <= 1e-3, f"{calls} calls of {Tn}: state diverged"

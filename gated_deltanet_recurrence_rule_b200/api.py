@@ -64,7 +64,7 @@ def load():
         lib.gdn_prefill_workspace_size_rounds.argtypes = [i32, i64, i32, i32, i32, i32, i32, i64]
         lib.gdn_prefill.restype = i32
         lib.gdn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32, i32,
-                                    f32, vp, vp, vp, vp, sz, vp]
+                                    i32, f32, vp, vp, vp, vp, sz, vp]
         lib.gdn_decode_step.restype = i32
         lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                         i32, f32, vp]
@@ -129,15 +129,18 @@ def prefill_launch_count(num_seqs, total_tokens, Hqk, Hv, Dk, Dv, workspace_byte
 
 
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_state=True,
-            final_state=None, scale=1.0, o=None, workspace=None, o_dtype=torch.float32):
+            final_state=None, scale=1.0, o=None, workspace=None, o_dtype=torch.float32,
+            state_dtype=None):
     """Chunked prefill over packed sequences on the GPU.
 
     q, k [T, Hqk, Dk]; v [T, Hv, Dv] (bf16 or fp32, same dtype); g, beta [T, Hv]
     fp32; cu_seqlens [N+1] int32 (default: one sequence of T tokens);
     o is produced in ``o_dtype`` (fp32 by default, or bf16);
-    initial_state [N, Hv, Dv, Dk] fp32 or None (zeros).  ``final_state`` may
+    initial_state [N, Hv, Dv, Dk] or None (zeros).  ``final_state`` may
     be given (it may be ``initial_state`` itself, for an in-place update);
-    otherwise one is allocated when ``output_final_state``.
+    otherwise one is allocated when ``output_final_state``.  States are fp32,
+    or bf16 kept at rest (fp32 arithmetic, the final state rounded once): the
+    dtype of the given states, else ``state_dtype`` (default fp32).
     Returns (o [T, Hv, Dv], final_state or None).
     """
     lib = load()
@@ -159,12 +162,16 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_
     _require(cu_seqlens, "cu_seqlens", dev, torch.int32)
     N = cu_seqlens.shape[0] - 1
     sshape = (N, Hv, Dv, Dk)
+    given = [t.dtype for t in (initial_state, final_state) if t is not None]
+    sdt = given[0] if given else (state_dtype or torch.float32)
+    if sdt not in _DTYPE_CODE or (state_dtype is not None and state_dtype != sdt):
+        raise ValueError(f"unsupported or inconsistent state dtype {sdt}")
     if initial_state is not None:
-        _require(initial_state, "initial_state", dev, torch.float32, sshape)
+        _require(initial_state, "initial_state", dev, sdt, sshape)
     if final_state is None and output_final_state:
-        final_state = torch.empty(sshape, dtype=torch.float32, device=dev)
+        final_state = torch.empty(sshape, dtype=sdt, device=dev)
     if final_state is not None:
-        _require(final_state, "final_state", dev, torch.float32, sshape)
+        _require(final_state, "final_state", dev, sdt, sshape)
     if o is None:
         o = torch.empty((T, Hv, Dv), dtype=o_dtype, device=dev)
     if o.dtype not in _DTYPE_CODE:
@@ -175,8 +182,8 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     _require(workspace, "workspace", dev, torch.uint8)
     st = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T,
-                         Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], _DTYPE_CODE[o.dtype], float(scale),
-                         _ptr(initial_state),
+                         Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], _DTYPE_CODE[o.dtype],
+                         _DTYPE_CODE[sdt], float(scale), _ptr(initial_state),
                          _ptr(final_state), _ptr(o), _ptr(workspace), workspace.numel(),
                          _stream(dev))
     _check(st, "gdn_prefill")

@@ -17,7 +17,7 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const int32_t *cu, int N, long long T_,
                                 int Hqk, int Hv, int Dk, int Dv, int dtype, int o_dtype,
-                                float scale, const float *s0, float *sfin, void *o,
+                                int state_dtype, float scale, const void *s0, void *sfin, void *o,
                                 int32_t *status, cudaStream_t stream);
 int decode_tokens_max();
 cudaError_t launch_decode_tokens(const void *q, const void *k, const void *v, const float *g,
@@ -28,18 +28,18 @@ cudaError_t launch_decode_tokens(const void *q, const void *k, const void *v, co
                                  cudaStream_t s);
 bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
-                              const float *beta, const int32_t *cu, int N, long long T_,
-                              int Hqk, int Hv, int o_dtype, float scale, const float *s0,
-                              float *sfin, void *o, void *workspace, cudaStream_t stream);
+                              const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
+                              int Hv, int o_dtype, int state_dtype, float scale, const void *s0,
+                              void *sfin, void *o, void *workspace, cudaStream_t stream);
 size_t twophase_workspace_bytes(int64_t N, int64_t T, int Hv);
 size_t twophase_round_workspace_bytes(int64_t N, int Hv, int64_t chunks_per_round);
 size_t twophase_min_workspace_bytes(int64_t N, int Hv);
 int64_t twophase_launch_count(int64_t N, int64_t T, int Hv, size_t workspace_bytes);
 cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const int32_t *cu, int N, long long T_,
-                                    int Hqk, int Hv, int o_dtype, float scale, const float *s0,
-                                    float *sfin, void *o, void *workspace, size_t workspace_bytes,
-                                    cudaStream_t stream);
+                                    int Hqk, int Hv, int o_dtype, int state_dtype, float scale,
+                                    const void *s0, void *sfin, void *o, void *workspace,
+                                    size_t workspace_bytes, cudaStream_t stream);
 }  // namespace gdn
 
 namespace {
@@ -134,11 +134,12 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
                     const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
                     int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
                     int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, int32_t o_dtype,
-                    float scale, const float *initial_state, float *final_state, void *o,
-                    void *workspace, size_t workspace_bytes, void *stream) {
+                    int32_t state_dtype, float scale, const void *initial_state,
+                    void *final_state, void *o, void *workspace, size_t workspace_bytes,
+                    void *stream) {
   if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
   if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
-  if (!dtype_ok(o_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dtype_ok(o_dtype) || !dtype_ok(state_dtype)) return GDN_ERR_INVALID_ARG;
   if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
   if (num_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
   if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
@@ -162,18 +163,18 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
     if (workspace_bytes >= gdn::twophase_min_workspace_bytes(num_seqs, num_v_heads)) {
       // two phases: every chunk's state-free products at once, then the state pass
       e = gdn::launch_prefill_twophase(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
-                                       num_qk_heads, num_v_heads, o_dtype, scale, initial_state,
-                                       final_state, o, workspace, workspace_bytes, s);
+                                       num_qk_heads, num_v_heads, o_dtype, state_dtype, scale,
+                                       initial_state, final_state, o, workspace, workspace_bytes, s);
     } else {
       // a header-only workspace: one pass, each CTA does all of a (sequence, head)
       e = gdn::launch_prefill_tc(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
-                                 num_qk_heads, num_v_heads, o_dtype, scale, initial_state,
-                                 final_state, o, workspace, s);
+                                 num_qk_heads, num_v_heads, o_dtype, state_dtype, scale,
+                                 initial_state, final_state, o, workspace, s);
     }
   } else {
     e = gdn::launch_prefill_simt(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
                                  num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype,
-                                 scale, initial_state, final_state, o, status, s);
+                                 state_dtype, scale, initial_state, final_state, o, status, s);
   }
   return cuda_status(e);
 }

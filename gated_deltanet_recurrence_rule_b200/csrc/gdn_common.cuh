@@ -47,6 +47,24 @@ __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float out[4]) {
   out[3] = __uint_as_float(x.y & 0xffff0000u);
 }
 
+// States of the caller kept in fp32 or, at rest, in bf16 (widened exactly on
+// load, rounded to nearest even on store).  `e` is an element index, a
+// multiple of 4; the base pointer is 16-byte aligned.
+__device__ __forceinline__ void load_state4(const void *base, size_t e, bool bf16, float out[4]) {
+  if (bf16) load4(static_cast<const __nv_bfloat16 *>(base) + e, out);
+  else load4(static_cast<const float *>(base) + e, out);
+}
+__device__ __forceinline__ void store_state4(void *base, size_t e, bool bf16, const float in[4]) {
+  if (bf16) {
+    const __nv_bfloat162 a = __floats2bfloat162_rn(in[0], in[1]);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(in[2], in[3]);
+    *reinterpret_cast<uint2 *>(static_cast<__nv_bfloat16 *>(base) + e) =
+        make_uint2(*reinterpret_cast<const uint32_t *>(&a), *reinterpret_cast<const uint32_t *>(&b));
+  } else {
+    *reinterpret_cast<float4 *>(static_cast<float *>(base) + e) = make_float4(in[0], in[1], in[2], in[3]);
+  }
+}
+
 // Streaming (evict-first) 128-bit global load / store for data touched once.
 __device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(float4 *p, float4 v) { __stcs(p, v); }

@@ -55,8 +55,8 @@ __global__ void __launch_bounds__(128)
 prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     const float *__restrict__ g, const float *__restrict__ beta,
                     const int32_t *__restrict__ cu, int N, long long Ttot, int Hqk, int Hv,
-                    int DV, float scale, const float *s0, float *sfin, TO *__restrict__ o,
-                    int32_t *status) {
+                    int DV, float scale, const void *s0, void *sfin, int state_bf16,
+                    TO *__restrict__ o, int32_t *status) {
   using C = SimtCfg<T, DK>;
   extern __shared__ __align__(16) unsigned char smem[];
   unsigned char *raw[2] = {smem, smem + C::RAW_BYTES};
@@ -88,9 +88,8 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
   const size_t srow = (((size_t)n * Hv + h) * DV + row) * DK;
 #pragma unroll
   for (int m = 0; m < C::NV4; ++m) {
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (s0) x = *reinterpret_cast<const float4 *>(s0 + srow + 16 * m + 4 * r4);
-    S[4 * m + 0] = x.x; S[4 * m + 1] = x.y; S[4 * m + 2] = x.z; S[4 * m + 3] = x.w;
+    if (s0) load_state4(s0, srow + 16 * m + 4 * r4, state_bf16, S + 4 * m);
+    else S[4 * m] = S[4 * m + 1] = S[4 * m + 2] = S[4 * m + 3] = 0.f;
   }
 
   const long long L = c1 - c0;
@@ -193,17 +192,16 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
 
   if (sfin) {
 #pragma unroll
-    for (int m = 0; m < C::NV4; ++m)
-      *reinterpret_cast<float4 *>(sfin + srow + 16 * m + 4 * r4) =
-          make_float4(S[4 * m + 0], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
+    for (int m = 0; m < C::NV4; ++m) store_state4(sfin, srow + 16 * m + 4 * r4, state_bf16, S + 4 * m);
   }
 }
 
 template <typename T, typename TO, int DK>
 static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const int32_t *cu, int N, long long T_,
-                                 int Hqk, int Hv, int Dv, float scale, const float *s0,
-                                 float *sfin, void *o, int32_t *status, cudaStream_t stream) {
+                                 int Hqk, int Hv, int Dv, float scale, const void *s0,
+                                 void *sfin, int state_bf16, void *o, int32_t *status,
+                                 cudaStream_t stream) {
   using C = SimtCfg<T, DK>;
   auto kern = prefill_simt_kernel<T, TO, DK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
@@ -211,21 +209,22 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
   const unsigned blocks = (unsigned)N * (unsigned)Hv * (unsigned)(Dv / C::ROWS);
   kern<<<blocks, C::THREADS, C::SMEM, stream>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), g, beta,
-      cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, static_cast<TO *>(o), status);
+      cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, state_bf16, static_cast<TO *>(o), status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const int32_t *cu, int N, long long T_,
                                 int Hqk, int Hv, int Dk, int Dv, int dtype, int o_dtype,
-                                float scale, const float *s0, float *sfin, void *o,
+                                int state_dtype, float scale, const void *s0, void *sfin, void *o,
                                 int32_t *status, cudaStream_t stream) {
+  const int sb = state_dtype == GDN_DTYPE_BF16;
   return dispatch_types(dtype, o_dtype, [&](auto t, auto to) {
     using T = decltype(t);
     using TO = decltype(to);
     if (Dk == 128)
-      return launch_simt_t<T, TO, 128>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, o, status, stream);
-    return launch_simt_t<T, TO, 64>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, o, status, stream);
+      return launch_simt_t<T, TO, 128>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, sb, o, status, stream);
+    return launch_simt_t<T, TO, 64>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, sb, o, status, stream);
   });
 }
 

@@ -127,8 +127,9 @@ struct Params {
   const int32_t *cu;
   int N, T, Hqk, Hv;
   float scale;
-  const float *s0;
-  float *sfin;
+  const void *s0;  // caller's initial states, fp32 or (state_bf16) bf16
+  void *sfin;      // caller's final states, same type
+  int state_bf16;
   void *o;
   int32_t *status;
 };
@@ -157,9 +158,16 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   const int L = c1 - c0;
   const int nch = (L + CH - 1) / CH;
-  if (nch == 0) {  // empty sequence: final state = initial state
-    if (p.sfin)
-      for (int x = tid; x < HD * HD; x += NTHREADS) p.sfin[sbase + x] = p.s0 ? p.s0[sbase + x] : 0.f;
+  if (nch == 0) {  // empty sequence: final state = initial state (a byte copy)
+    if (p.sfin) {
+      const int eb = p.state_bf16 ? 2 : 4;
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(p.sfin) + sbase * eb);
+      const uint4 *src = p.s0 ? reinterpret_cast<const uint4 *>(
+                                    static_cast<const unsigned char *>(p.s0) + sbase * eb)
+                              : nullptr;
+      for (int x = tid; x < HD * HD * eb / 16; x += NTHREADS)
+        dst[x] = src ? src[x] : make_uint4(0u, 0u, 0u, 0u);
+    }
     return;
   }
 
@@ -381,12 +389,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // fp32 master state: row `row`, columns [32 ewq, 32 ewq + 32); S0 = hi + lo in TMEM
     float S[32];
     {
-      const float *src = p.s0 ? p.s0 + sbase + (size_t)row * HD + 32 * ewq : nullptr;
+      const size_t e0 = sbase + (size_t)row * HD + 32 * ewq;
 #pragma unroll
       for (int x = 0; x < 32; x += 4) {
-        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (src) v4 = *reinterpret_cast<const float4 *>(src + x);
-        S[x] = v4.x; S[x + 1] = v4.y; S[x + 2] = v4.z; S[x + 3] = v4.w;
+        if (p.s0) load_state4(p.s0, e0 + x, p.state_bf16, S + x);
+        else S[x] = S[x + 1] = S[x + 2] = S[x + 3] = 0.f;
       }
       uint32_t hw[16], lw[16];
       split_words<16>(S, hw, lw);
@@ -549,10 +556,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
     if (*abort_flag == 0 && p.sfin) {
-      float *dst = p.sfin + sbase + (size_t)row * HD + 32 * ewq;
+      const size_t e0 = sbase + (size_t)row * HD + 32 * ewq;
 #pragma unroll
-      for (int x = 0; x < 32; x += 4)
-        *reinterpret_cast<float4 *>(dst + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
+      for (int x = 0; x < 32; x += 4) store_state4(p.sfin, e0 + x, p.state_bf16, S + x);
     }
   }
 
@@ -586,11 +592,12 @@ bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype) {
 
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
-                              int Hv, int o_dtype, float scale, const float *s0, float *sfin,
-                              void *o, void *workspace, cudaStream_t stream) {
+                              int Hv, int o_dtype, int state_dtype, float scale, const void *s0,
+                              void *sfin, void *o, void *workspace, cudaStream_t stream) {
   tc::Params prm;
   prm.g = g; prm.beta = beta; prm.cu = cu; prm.N = N; prm.T = (int)T_; prm.Hqk = Hqk; prm.Hv = Hv;
-  prm.scale = scale; prm.s0 = s0; prm.sfin = sfin; prm.o = o;
+  prm.scale = scale; prm.s0 = s0; prm.sfin = sfin; prm.state_bf16 = state_dtype == GDN_DTYPE_BF16;
+  prm.o = o;
   prm.status = static_cast<int32_t *>(workspace);
   if (o_dtype == GDN_DTYPE_BF16) return tc::launch_t<__nv_bfloat16>(q, k, v, prm, stream);
   return tc::launch_t<float>(q, k, v, prm, stream);

@@ -46,9 +46,9 @@ namespace plan {
 // final state of every empty sequence (= its initial state, or zeros).  Bad
 // cu_seqlens set GDN_ERR_BAD_SEQLENS and leave zero chunks to process.
 __global__ void __launch_bounds__(1024)
-plan_kernel(const int32_t *__restrict__ cu, int N, int T, int Hv, const float *__restrict__ s0,
-            float *__restrict__ sfin, tp::PlanHeader *ph, int32_t *ne_seq, int32_t *ne_cs,
-            int32_t *status) {
+plan_kernel(const int32_t *__restrict__ cu, int N, int T, int Hv, const void *__restrict__ s0,
+            void *__restrict__ sfin, size_t state_bytes, tp::PlanHeader *ph, int32_t *ne_seq,
+            int32_t *ne_cs, int32_t *status) {
   __shared__ int s_bad, s_run_ne, s_run_ch, s_nempty;
   __shared__ int w_ne[32], w_ch[32];
   __shared__ int s_empty[1024];
@@ -70,7 +70,6 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int T, int Hv, const float *_
     }
     return;
   }
-  const size_t state_elems = (size_t)Hv * 128 * 128;
   for (int base = 0; base < N; base += blockDim.x) {
     const int n = base + tid;
     const int L = n < N ? cu[n + 1] - cu[n] : 0;
@@ -101,12 +100,14 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int T, int Hv, const float *_
     __syncthreads();
     if (tid == blockDim.x - 1) { s_run_ne = pe + ne; s_run_ch = pc + nc; }
     // final state of the empty sequences of this tile = initial state (or 0)
+    // (a byte copy: the caller's states are all fp32 or all bf16)
     for (int e = 0; e < s_nempty; ++e) {
-      const size_t off = (size_t)s_empty[e] * state_elems;
-      float4 *dst = reinterpret_cast<float4 *>(sfin + off);
-      const float4 *src = s0 ? reinterpret_cast<const float4 *>(s0 + off) : nullptr;
-      for (size_t x = tid; x < state_elems / 4; x += blockDim.x)
-        dst[x] = src ? src[x] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const size_t off = (size_t)s_empty[e] * state_bytes;
+      uint4 *dst = reinterpret_cast<uint4 *>(static_cast<unsigned char *>(sfin) + off);
+      const uint4 *src =
+          s0 ? reinterpret_cast<const uint4 *>(static_cast<const unsigned char *>(s0) + off) : nullptr;
+      for (size_t x = tid; x < state_bytes / 16; x += blockDim.x)
+        dst[x] = src ? src[x] : make_uint4(0u, 0u, 0u, 0u);
     }
     __syncthreads();
   }
@@ -170,8 +171,9 @@ struct Params {
   int N, T, Hqk, Hv;
   int round, rc;
   float scale;
-  const float *s0;
-  float *sfin;
+  const void *s0;  // caller's initial states, fp32 or (state_bf16) bf16
+  void *sfin;      // caller's final states, same type
+  int state_bf16;
   void *o;
   const tp::PlanHeader *plan;
   const int32_t *ne_seq, *ne_cs;
@@ -204,10 +206,16 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int seq_begin = p.cu[n], seq_end = p.cu[n + 1];
   const size_t hstate = (size_t)HD * HD;
   const size_t sbase = ((size_t)n * p.Hv + h) * hstate;
-  const float *src = (ga == cs) ? (p.s0 ? p.s0 + sbase : nullptr)
-                                : p.carry + ((size_t)((p.round - 1) & 1) * p.Hv + h) * hstate;
-  float *dst = (gb == ce) ? (p.sfin ? p.sfin + sbase : nullptr)
-                          : p.carry + ((size_t)(p.round & 1) * p.Hv + h) * hstate;
+  // the state comes from the caller (first chunk of the sequence) or from the
+  // carry of the previous round, and goes to the caller or to the carry
+  const int ueb = p.state_bf16 ? 2 : 4;  // bytes per element of the caller's states
+  const bool src_bf16 = (ga == cs) && p.state_bf16, dst_bf16 = (gb == ce) && p.state_bf16;
+  const void *src = (ga == cs)
+      ? (p.s0 ? static_cast<const void *>(static_cast<const unsigned char *>(p.s0) + sbase * ueb) : nullptr)
+      : static_cast<const void *>(p.carry + ((size_t)((p.round - 1) & 1) * p.Hv + h) * hstate);
+  void *dst = (gb == ce)
+      ? (p.sfin ? static_cast<void *>(static_cast<unsigned char *>(p.sfin) + sbase * ueb) : nullptr)
+      : static_cast<void *>(p.carry + ((size_t)(p.round & 1) * p.Hv + h) * hstate);
 
   const uint32_t sb = smem_addr(smem);
   if (sb & 1023u) {  // swizzled operand tiles need 1024-byte alignment
@@ -383,12 +391,11 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // fp32 master state: row `row`, columns [32 ewq, 32 ewq + 32); S0 = hi + lo in TMEM
     float S[32];
     {
-      const float *srow = src ? src + (size_t)row * HD + 32 * ewq : nullptr;
+      const size_t e0 = (size_t)row * HD + 32 * ewq;
 #pragma unroll
       for (int x = 0; x < 32; x += 4) {
-        float4 v4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (srow) v4 = *reinterpret_cast<const float4 *>(srow + x);
-        S[x] = v4.x; S[x + 1] = v4.y; S[x + 2] = v4.z; S[x + 3] = v4.w;
+        if (src) load_state4(src, e0 + x, src_bf16, S + x);
+        else S[x] = S[x + 1] = S[x + 2] = S[x + 3] = 0.f;
       }
       uint32_t hw[16], lw[16];
       split_words<16>(S, hw, lw);
@@ -531,10 +538,9 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
       for (int part = 0; part < 4; ++part) store_out(part);
       if (dst) {
-        float *drow = dst + (size_t)row * HD + 32 * ewq;
+        const size_t e0 = (size_t)row * HD + 32 * ewq;
 #pragma unroll
-        for (int x = 0; x < 32; x += 4)
-          *reinterpret_cast<float4 *>(drow + x) = make_float4(S[x], S[x + 1], S[x + 2], S[x + 3]);
+        for (int x = 0; x < 32; x += 4) store_state4(dst, e0 + x, dst_bf16, S + x);
       }
     }
   }
@@ -672,9 +678,9 @@ cudaError_t device_streams(DeviceStreams **out) {
 // rounds run one after another on `stream` with as many chunks as fit.
 cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const int32_t *cu, int N, long long T_,
-                                    int Hqk, int Hv, int o_dtype, float scale, const float *s0,
-                                    float *sfin, void *o, void *workspace, size_t workspace_bytes,
-                                    cudaStream_t stream) {
+                                    int Hqk, int Hv, int o_dtype, int state_dtype, float scale,
+                                    const void *s0, void *sfin, void *o, void *workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
   const int T = (int)T_;
   const tp::Layout L = tp::layout(N, Hv);
   unsigned char *ws = static_cast<unsigned char *>(workspace);
@@ -696,7 +702,8 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
 
   sp::Params prm;
   prm.cu = cu; prm.N = N; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.rc = rc; prm.scale = scale;
-  prm.s0 = s0; prm.sfin = sfin; prm.o = o;
+  prm.s0 = s0; prm.sfin = sfin; prm.state_bf16 = state_dtype == GDN_DTYPE_BF16; prm.o = o;
+  const size_t state_bytes = (size_t)Hv * 128 * 128 * (prm.state_bf16 ? 2 : 4);
   prm.plan = ph; prm.ne_seq = ne_seq; prm.ne_cs = ne_cs;
   prm.carry = reinterpret_cast<float *>(ws + L.carry_off);
   prm.status = status;
@@ -708,7 +715,8 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
   cudaError_t e;
 
   if (!pipelined) {
-    plan::plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, Hv, s0, sfin, ph, ne_seq, ne_cs, status);
+    plan::plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, Hv, s0, sfin, state_bytes, ph, ne_seq,
+                                             ne_cs, status);
     if ((e = cudaGetLastError()) != cudaSuccess || T == 0) return e;
     prm.rec = ws + L.rec_off;
     for (int r = 0; r < rounds; ++r) {
@@ -728,7 +736,8 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
   if ((e = cudaEventRecord(d->start, stream)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(d->prep, d->start, 0)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(d->chain, d->start, 0)) != cudaSuccess) return e;
-  plan::plan_kernel<<<1, 1024, 0, d->prep>>>(cu, N, T, Hv, s0, sfin, ph, ne_seq, ne_cs, status);
+  plan::plan_kernel<<<1, 1024, 0, d->prep>>>(cu, N, T, Hv, s0, sfin, state_bytes, ph, ne_seq,
+                                             ne_cs, status);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (T == 0) {
     if ((e = cudaEventRecord(d->prep_done, d->prep)) != cudaSuccess) return e;

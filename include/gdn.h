@@ -125,10 +125,14 @@ int64_t gdn_prefill_launch_count(int32_t num_seqs, int64_t total_tokens, int32_t
  *   cu_seqlens     [num_seqs + 1] int32, device; 0 = c_0 <= c_1 <= ... <= c_N = T.
  *                  Sequence n is tokens [c_n, c_{n+1}); empty sequences are allowed
  *                  (their final state equals their initial state).
- *   initial_state  [num_seqs, Hv, Dv, Dk] fp32, or NULL for zeros.
- *   final_state    [num_seqs, Hv, Dv, Dk] fp32, or NULL to skip.  May be the same
- *                  pointer as initial_state (updated in place); no other overlap
- *                  between arguments is allowed.
+ *   state_dtype    GDN_DTYPE_FP32, or GDN_DTYPE_BF16 for states kept at rest in
+ *                  bf16: the initial state is widened exactly, the arithmetic is
+ *                  the same as with fp32 states, and the final state is rounded
+ *                  to nearest even once, when it is stored.
+ *   initial_state  [num_seqs, Hv, Dv, Dk] state_dtype, or NULL for zeros.
+ *   final_state    [num_seqs, Hv, Dv, Dk] state_dtype, or NULL to skip.  May be the
+ *                  same pointer as initial_state (updated in place); no other
+ *                  overlap between arguments is allowed.
  *   o              [T, Hv, Dv]    o_dtype (output)
  *   scale          multiplies o (1.0 for o_t = S_t q_t)
  *   workspace      device buffer of workspace_bytes >= 256 bytes, 256-byte aligned,
@@ -155,8 +159,9 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
                     const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
                     int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
                     int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, int32_t o_dtype,
-                    float scale, const float *initial_state, float *final_state, void *o,
-                    void *workspace, size_t workspace_bytes, void *stream);
+                    int32_t state_dtype, float scale, const void *initial_state,
+                    void *final_state, void *o, void *workspace, size_t workspace_bytes,
+                    void *stream);
 
 /*
  * Prefill for callers that cannot allocate device memory.  (The pages have no
@@ -170,7 +175,8 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
  * array of the library (every GPU that loads the library holds it until the
  * process exits), and calls no cudaMalloc, cudaFree or allocating routine.
  *
- * Arguments are those of gdn_prefill without the workspace, plus
+ * Arguments are those of gdn_prefill without the workspace and with fp32 states
+ * (no state_dtype), plus
  *   device_status  optional device int32 (caller's memory, NULL to discard) that
  *                  receives this call's device-detected status (GDN_OK,
  *                  GDN_ERR_BAD_SEQLENS or GDN_ERR_DEVICE_TIMEOUT) in stream order.

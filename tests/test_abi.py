@@ -103,12 +103,12 @@ def test_workspace_size(lib):
 
 def _prefill(lib, **kw):
     a = dict(q=1 << 12, k=1 << 12, v=1 << 12, g=1 << 12, beta=1 << 12, cu=1 << 12, N=1, T=16,
-             Hqk=2, Hv=6, Dk=64, Dv=64, dtype=0, odt=1, scale=1.0, s0=None, sf=None, o=1 << 12,
-             ws=1 << 12, wsb=256)
+             Hqk=2, Hv=6, Dk=64, Dv=64, dtype=0, odt=1, sdt=1, scale=1.0, s0=None, sf=None,
+             o=1 << 12, ws=1 << 12, wsb=256)
     a.update(kw)
     return lib.gdn_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["T"],
-                           a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"], a["odt"], a["scale"], a["s0"],
-                           a["sf"], a["o"], a["ws"], a["wsb"], None)
+                           a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"], a["odt"], a["sdt"],
+                           a["scale"], a["s0"], a["sf"], a["o"], a["ws"], a["wsb"], None)
 
 
 def test_prefill_validation(lib):
@@ -121,6 +121,7 @@ def test_prefill_validation(lib):
     assert _prefill(lib, Hqk=0) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, dtype=3) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, odt=2) == api.GDN_ERR_INVALID_ARG
+    assert _prefill(lib, sdt=2) == api.GDN_ERR_INVALID_ARG             # state dtype
     assert _prefill(lib, T=-1) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, N=-1) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, Dk=96) == api.GDN_ERR_UNSUPPORTED

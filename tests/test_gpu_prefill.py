@@ -5,7 +5,7 @@ import torch
 
 import oracle
 from gated_deltanet_recurrence_rule_b200 import api, inputs
-from parity import TOL, assert_parity, oracle_prefill_heads, to_np
+from parity import TOL, assert_parity, oracle_prefill_heads, state_error, state_error_bf16_rest, to_np
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -184,3 +184,97 @@ def test_long262k_sampled_heads():
 def test_varlen32_sampled_heads():
     """32 packed sequences of 1024..32768 tokens; oracle on QK head 4."""
     _sampled_workload("varlen32", [4])
+
+
+# ---- states at rest in bf16: widened on load, rounded once on store ----------
+
+def _bf16_state_case(lengths, dtype, D, seed, ws_bytes=None, alias=False):
+    """Run the prefill with bf16 states, and again with fp32 states holding the
+    same values; return both results and the oracle's."""
+    inp = inputs.prefill_inputs(lengths, 2, 6, D, dtype=dtype, seed=seed, init_std=0.1)
+    inp["initial_state"] = inp["initial_state"].to(torch.bfloat16)
+    dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
+    out = {}
+    for sdt in (torch.bfloat16, torch.float32):
+        ws = None if ws_bytes is None else torch.zeros(ws_bytes, dtype=torch.uint8, device=DEV)
+        s0 = dev["initial_state"].to(sdt, copy=True)  # each run gets its own (in-place) copy
+        o, f = api.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                           cu_seqlens=dev["cu_seqlens"], initial_state=s0,
+                           final_state=s0 if alias else None, workspace=ws)
+        torch.cuda.synchronize()
+        assert f.dtype == sdt
+        if ws is not None:
+            assert api.get_device_status(ws) == api.GDN_OK
+        out[sdt] = (o, f)
+    o_ref, f_ref = oracle.prefill(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                  cu_seqlens=inp["cu_seqlens"], initial_state=inp["initial_state"],
+                                  state_at_rest="bf16")
+    _, f_exact = run_oracle(inp)
+    return inp, out, o_ref, f_ref, f_exact
+
+
+def _check_bf16_states(inp, out, o_ref, f_ref, f_exact, dtype, slack_rel, what):
+    """Exact against the same kernel with fp32 states (o bit for bit; the bf16
+    final state is the fp32 one rounded to nearest even, bit for bit), and
+    against the oracle: o within the input dtype's bound, the state within the
+    bf16 bound of the exact one and within one rounding (plus the path's fp32
+    error, slack_rel * RMS) of the oracle's rounded state."""
+    o, f = out[torch.bfloat16]
+    o32, f32 = out[torch.float32]
+    assert torch.equal(o, o32), f"{what}: o depends on the state storage"
+    assert torch.equal(f, f32.to(torch.bfloat16)), f"{what}: bf16 state is not RNE of the fp32 one"
+    assert_parity(inputs.DTYPES[dtype], to_np(o), o_ref, what=what)
+    e = state_error_bf16_rest(to_np(f), f_ref, slack_rel=slack_rel)
+    assert e <= 1.0, f"{what}: {e:.3f}x the one-rounding bound"
+    assert state_error(to_np(f), f_exact) <= 5e-3, what
+    lengths = np.diff(inp["cu_seqlens"].numpy())
+    for n in np.flatnonzero(lengths == 0):  # empty sequences: final state = initial state, bit for bit
+        assert torch.equal(f[n].cpu(), inp["initial_state"][n]), f"{what}: empty sequence {n}"
+
+
+# fp32 state error of the tensor-core path (bf16 operands with hi/lo splits),
+# element by element, as a fraction of RMS(S)
+TC_SLACK = 2e-3
+
+
+@pytest.mark.parametrize("alias", [False, True])
+def test_bf16_states_two_phase(alias):
+    """Two-phase tensor-core prefill, full workspace, varlen with an empty
+    sequence; bf16 initial and final states (also updated in place)."""
+    lengths = [300, 0, 130, 64, 65]
+    args = _bf16_state_case(lengths, "bf16", 128, seed=71, alias=alias)
+    _check_bf16_states(*args, "bf16", TC_SLACK, f"two-phase alias={alias}")
+
+
+def test_bf16_states_rounds_carry():
+    """Rounds of 3 chunks: states cross rounds through the fp32 carry; only the
+    caller's states are bf16."""
+    lengths = [300, 1, 0, 130, 700, 64, 65]
+    N, T = len(lengths), sum(lengths)
+    ws = api.prefill_workspace_size(N, T, 2, 6, 128, 128, chunks_per_round=3)
+    args = _bf16_state_case(lengths, "bf16", 128, seed=72, ws_bytes=ws)
+    _check_bf16_states(*args, "bf16", TC_SLACK, "rounds of 3")
+
+
+def test_bf16_states_single_pass():
+    """Header-only workspace: the single-pass tensor-core kernel."""
+    args = _bf16_state_case([300, 0, 65], "bf16", 128, seed=73, ws_bytes=256)
+    _check_bf16_states(*args, "bf16", TC_SLACK, "single pass")
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_bf16_states_cuda_cores(D):
+    """fp32 inputs run the CUDA-core kernel; bf16 states there too."""
+    args = _bf16_state_case([200, 0, 77], "fp32", D, seed=74 + D)
+    _check_bf16_states(*args, "fp32", 2e-5, f"CUDA cores D={D}")
+
+
+def test_bf16_states_zero_tokens():
+    """T = 0: every sequence is empty and its bf16 final state is its initial state."""
+    inp = inputs.prefill_inputs([0, 0], 2, 6, 128, dtype="bf16", seed=75, init_std=0.1)
+    s0 = inp["initial_state"].to(torch.bfloat16).to(DEV)
+    dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
+    o, f = api.prefill(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"],
+                       cu_seqlens=dev["cu_seqlens"], initial_state=s0)
+    torch.cuda.synchronize()
+    assert torch.equal(f, s0)

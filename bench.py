@@ -216,8 +216,9 @@ def kernel_traffic(kernel_key: str, source_files):
 
 CSRC = os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc")
 PREFILL_SOURCES = [os.path.join(CSRC, n) for n in
-                   ("gdn_twophase.cuh", "gdn_chunk_ops.cuh", "gdn_sm100.cuh", "gdn_wy_prep.cu",
-                    "gdn_state_pass.cu")]
+                   ("gdn_common.cuh", "gdn_twophase.cuh", "gdn_chunk_ops.cuh", "gdn_sm100.cuh",
+                    "gdn_wy_prep.cu", "gdn_state_pass.cu")]
+DECODE_SOURCES = [os.path.join(CSRC, n) for n in ("gdn_common.cuh", "gdn_decode.cu")]
 
 
 # ---------------------------------------------------------------- oracle (CPU)
@@ -503,7 +504,7 @@ def _decode(args, D, dev, peaks, peak_src):
                          "peak": peak, "unit": "GB/s", "frac": gbs / D.world / peak,
                          "peak_source": f"{peak_src} hbm_gbs",
                          "algorithmic": f"{per_step} B per step (state read+write {2 * state_bytes} + io {io_bytes})",
-                         "traffic": kernel_traffic("decode", os.path.join(ROOT, "gated_deltanet_recurrence_rule_b200", "csrc", "gdn_decode.cu"))},
+                         "traffic": kernel_traffic("decode", DECODE_SOURCES)},
             "gpu_launches": steps}
 
 
@@ -550,7 +551,8 @@ def _decode_tokens(args, D, dev, peaks, peak_src, tokens=4, state_dtype="fp32"):
     per_call_bytes = 2 * state_bytes + io_bytes
     gbs = D.world * per_call_bytes * calls / (ms / 1e3) / 1e9
     peak = peaks["hbm_gbs"]
-    kernel = "decode_tokens_bf16s_kernel" if state_dtype == "bf16" else "decode_tokens_kernel"
+    kernel = ("decode_tokens_kernel" if state_dtype == "fp32" else
+              "decode_one_bf16s_kernel" if tokens == 1 else "decode_tokens_bf16s_kernel")
     traffic_key = "decode_tokens" + ("" if tokens > 1 else "_1") + ("_bf16" if state_dtype == "bf16" else "")
     return {"value": D.world * w.batch * tokens * calls / (ms / 1e3), "unit": "tokens/s",
             "workload": f"decode64 with {tokens} tokens per sequence per call: B={w.batch}, "
@@ -562,7 +564,7 @@ def _decode_tokens(args, D, dev, peaks, peak_src, tokens=4, state_dtype="fp32"):
                          "peak": peak, "unit": "GB/s", "frac": gbs / D.world / peak,
                          "peak_source": f"{peak_src} hbm_gbs",
                          "algorithmic": f"{per_call_bytes} B per call (state read+write {2 * state_bytes} + io {io_bytes})",
-                         "traffic": kernel_traffic(traffic_key, os.path.join(CSRC, "gdn_decode.cu"))},
+                         "traffic": kernel_traffic(traffic_key, DECODE_SOURCES)},
             "gpu_launches": calls}
 
 

@@ -46,3 +46,32 @@ def test_empty_input(oracle_lib):
     o, fin = oracle.prefill(q, k, v, g, beta, initial_state=s0)
     assert o.shape == (0, 3, 2)
     assert np.array_equal(fin, s0)
+
+
+def test_bf16_state_drift_is_bounded(oracle_lib):
+    """Tolerance study for states kept at rest in bf16 (oracle only): one token
+    per call, the state rounded to bf16 after every call, against an fp64
+    state kept throughout.  Each rounding adds relative noise of about 2^-9 and
+    the recurrence damps old noise by alpha per step, so the error settles at
+    about 2^-9 / sqrt(1 - alpha^2) instead of growing with the number of steps."""
+    r = np.random.default_rng(5)
+    B, Hv, D, steps, mu = 2, 3, 64, 256, -2.0
+    S = oracle.round_bf16(0.02 * r.standard_normal((B, Hv, D, D)))
+    exact, rest = S.copy(), S.copy()
+    err = {}
+    alphas = []
+    for t in range(1, steps + 1):
+        q = r.standard_normal((B, 1, D)); q /= np.linalg.norm(q, axis=-1, keepdims=True)
+        k = r.standard_normal((B, 1, D)); k /= np.linalg.norm(k, axis=-1, keepdims=True)
+        v = r.standard_normal((B, Hv, D))
+        beta = 1 / (1 + np.exp(-r.standard_normal((B, Hv))))
+        g = -np.log1p(np.exp(r.standard_normal((B, Hv)) + mu))
+        alphas.append(np.exp(g))
+        _, exact = oracle.decode_step(q, k, v, g, beta, exact, lib=oracle_lib)
+        _, rest = oracle.decode_step(q, k, v, g, beta, rest, state_at_rest="bf16", lib=oracle_lib)
+        if t in (64, 256):
+            err[t] = np.linalg.norm(rest - exact) / np.linalg.norm(exact)
+    a = float(np.median(np.concatenate(alphas, axis=None)))
+    level = 2.0 ** -9 / np.sqrt(1 - a * a)
+    assert 2.0 ** -11 < err[256] < 3 * level, (err, level)   # rounding happens, noise is damped
+    assert err[256] < 2 * err[64], err                       # no growth with the number of steps

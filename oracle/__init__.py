@@ -53,6 +53,8 @@ def _bind(lib):
     lib.gdn_oracle_decode_step.argtypes = [d, d, d, d, d, d, d, ci, ci, ci, ci, ci, cd, ci]
     lib.gdn_oracle_round_bf16.restype = ci
     lib.gdn_oracle_round_bf16.argtypes = [d, ctypes.c_int64]
+    lib.gdn_oracle_prologue.restype = ci
+    lib.gdn_oracle_prologue.argtypes = [d, d, d, d, ctypes.c_int64, ci, ci, ci]
     return lib
 
 
@@ -99,6 +101,22 @@ def round_bf16(x, lib=None):
     if rc != 0:
         raise ValueError(f"gdn_oracle_round_bf16 failed with code {rc}")
     return y
+
+
+def prologue(q, k, a, b, lib=None):
+    """Raw projections to the recurrence's inputs, in fp64: q, k [T, Hqk, Dk]
+    L2-normalised per (token, head) row; g = -softplus(a) and beta = sigmoid(b)
+    ([T, Hv]).  Leading dimensions may be any shape ([B, Tn, ...] for decode);
+    returns new arrays (q, k, g, beta)."""
+    lib = lib or load()
+    q, k, g, beta = (_f64(t).copy() for t in (q, k, a, b))
+    Dk, Hqk, Hv = q.shape[-1], q.shape[-2], g.shape[-1]
+    T = q.size // (Dk * Hqk)
+    assert k.shape == q.shape and beta.shape == g.shape and g.size == T * Hv
+    rc = lib.gdn_oracle_prologue(_ptr(q), _ptr(k), _ptr(g), _ptr(beta), T, Hqk, Hv, Dk)
+    if rc != 0:
+        raise ValueError(f"gdn_oracle_prologue failed with code {rc}")
+    return q, k, g, beta
 
 
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, scale=1.0, chunk=0,

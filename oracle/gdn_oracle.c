@@ -352,3 +352,41 @@ int gdn_oracle_round_bf16(double *x, int64_t n)
     }
     return ORACLE_OK;
 }
+
+/*
+ * Input prologue: from the layer's raw projections to the inputs of the
+ * recurrence, in place.  "Inside Qwen3.8-27B ...", section "Gated DeltaNet
+ * Mechanics", calls k_t the normalized key projection and makes beta_t input
+ * dependent; the maps below are the plainest readings (listed in the design
+ * notes of the repository):
+ *   q_t, k_t  <- x / |x|_2 for each (token, query/key head) row of Dk values;
+ *                a row of zeros stays zero;
+ *   g_t       <- -softplus(a_t) = -log(1 + e^{a_t}), so alpha_t = e^{g_t} lies in (0, 1);
+ *   beta_t    <- sigmoid(b_t) = 1 / (1 + e^{-b_t}), in (0, 1).
+ * On entry g and beta hold a and b ([T, Hv]); q and k are [T, Hqk, Dk].
+ * Returns 0, or 1 for a bad argument.
+ */
+int gdn_oracle_prologue(double *q, double *k, double *g, double *beta, int64_t T, int Hqk, int Hv,
+                        int Dk)
+{
+    if (T < 0 || Hqk <= 0 || Hv <= 0 || Dk <= 0) return ORACLE_BAD_ARG;
+    if (T > 0 && (!q || !k || !g || !beta)) return ORACLE_BAD_ARG;
+    double *rows[2] = {q, k};
+    for (int w = 0; w < 2; ++w) {
+        for (int64_t r = 0; r < T * Hqk; ++r) {
+            double *x = rows[w] + r * Dk;
+            double ss = 0.0;
+            for (int c = 0; c < Dk; ++c) ss += x[c] * x[c];
+            if (ss == 0.0) continue;
+            const double norm = sqrt(ss);
+            for (int c = 0; c < Dk; ++c) x[c] /= norm;
+        }
+    }
+    for (int64_t i = 0; i < T * Hv; ++i) {
+        const double a = g[i], b = beta[i];
+        /* softplus(a) = max(a, 0) + log(1 + e^{-|a|}), the same value without overflow */
+        g[i] = -(fmax(a, 0.0) + log1p(exp(-fabs(a))));
+        beta[i] = b >= 0.0 ? 1.0 / (1.0 + exp(-b)) : exp(b) / (1.0 + exp(b));
+    }
+    return ORACLE_OK;
+}

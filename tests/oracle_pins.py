@@ -341,9 +341,43 @@ def check_state_at_rest_bf16(lib, seed=12):
     assert not np.array_equal(f_r, f_ex), "rounding changed nothing: inputs too coarse to test it"
 
 
+def check_prologue(lib, seed=13):
+    """Input prologue (raw projections -> q, k, g, beta): hand-worked values and
+    the identities that fix L2 normalisation, -softplus and sigmoid."""
+    q = np.array([[[3.0, 4.0]], [[0.0, 0.0]]])
+    k = np.array([[[1.0, 0.0]], [[0.0, -2.0]]])
+    a = np.array([[0.0], [1.0]])
+    b = np.array([[0.0], [math.log(3.0)]])
+    qn, kn, g, beta = oracle.prologue(q, k, a, b, lib)
+    _close(qn, [[[0.6, 0.8]], [[0.0, 0.0]]], 1e-15, "q normalised (zero row stays zero)")
+    _close(kn, [[[1.0, 0.0]], [[0.0, -1.0]]], 1e-15, "k normalised")
+    _close(g, [[-math.log(2.0)], [-math.log1p(math.e)]], 1e-15, "g = -softplus(a)")
+    _close(beta, [[0.5], [0.75]], 1e-15, "beta = sigmoid(b)")
+
+    r = _rng(seed)
+    T, Hqk, Hv, D = 7, 2, 4, 16
+    q = r.standard_normal((T, Hqk, D)) * 3.0
+    k = r.standard_normal((T, Hqk, D)) * 0.1
+    a = np.concatenate([r.standard_normal((T - 1, Hv)) * 4.0, [[50.0, -50.0, 0.0, 700.0]]])
+    b = np.concatenate([r.standard_normal((T - 1, Hv)) * 4.0, [[50.0, -50.0, 0.0, -700.0]]])
+    qn, kn, g, beta = oracle.prologue(q, k, a, b, lib)
+    for x, xn, name in ((q, qn, "q"), (k, kn, "k")):
+        _close(np.linalg.norm(xn, axis=-1), np.ones((T, Hqk)), 1e-14, f"|{name}^| = 1")
+        _close((x * xn).sum(-1), np.linalg.norm(x, axis=-1), 1e-13, f"{name}^ along {name}")
+    _close(np.exp(g), 1.0 / (1.0 + np.exp(np.minimum(a, 700.0))), 1e-15, "alpha = e^g = 1/(1+e^a)")
+    _, _, g_neg, beta_neg = oracle.prologue(q, k, -a, -b, lib)
+    _close(g_neg - g, a, 1e-12, "softplus(a) - softplus(-a) = a")
+    _close(beta + beta_neg, np.ones_like(beta), 1e-15, "sigmoid(b) + sigmoid(-b) = 1")
+    assert g[-1, 0] == -50.0 - math.log1p(math.exp(-50.0)) and g[-1, 3] == -700.0, "large a"
+    assert 0.0 < beta[-1, 1] < 1e-21 and beta[-1, 0] == 1.0, "sigmoid tails"
+    qn2, kn2, _, _ = oracle.prologue(qn, kn, a, b, lib)
+    _close(qn2, qn, 1e-15, "normalising twice changes nothing")
+    _close(kn2, kn, 1e-15, "normalising twice changes nothing (k)")
+
+
 ALL_CHECKS = [
     check_product_form, check_golden_scalar, check_golden_matrix, check_no_write_no_decay,
     check_exact_writeback, check_reset, check_pure_decay, check_orthonormal_memory, check_scale,
     check_gqa_mapping, check_varlen, check_decode, check_chunked, check_round_bf16,
-    check_state_at_rest_bf16,
+    check_state_at_rest_bf16, check_prologue,
 ]

@@ -43,6 +43,13 @@ MUTANTS = [
     ("bf16_seven_bits", "int qexp = e - 8;", "int qexp = e - 7;"),
     ("bf16_no_subnormal_floor", "if (qexp < -133) qexp = -133;", "if (qexp < -149) qexp = -149;"),
     ("bf16_no_overflow", "if (fabs(y) > bf16_max) y = copysign(INFINITY, a);", "(void)bf16_max;"),
+    ("prologue_no_sqrt", "for (int c = 0; c < Dk; ++c) x[c] /= norm;", "for (int c = 0; c < Dk; ++c) x[c] /= ss;"),
+    ("prologue_l1_norm", "for (int c = 0; c < Dk; ++c) ss += x[c] * x[c];", "for (int c = 0; c < Dk; ++c) ss += fabs(x[c]);"),
+    ("prologue_q_only", "for (int w = 0; w < 2; ++w) {", "for (int w = 0; w < 1; ++w) {"),
+    ("prologue_relu_not_softplus", "g[i] = -(fmax(a, 0.0) + log1p(exp(-fabs(a))));", "g[i] = -(fmax(a, 0.0));"),
+    ("prologue_decay_sign", "g[i] = -(fmax(a, 0.0) + log1p(exp(-fabs(a))));", "g[i] = (fmax(a, 0.0) + log1p(exp(-fabs(a))));"),
+    ("prologue_sigmoid_of_minus_b", "beta[i] = b >= 0.0 ? 1.0 / (1.0 + exp(-b)) : exp(b) / (1.0 + exp(b));",
+     "beta[i] = b >= 0.0 ? 1.0 / (1.0 + exp(b)) : exp(-b) / (1.0 + exp(-b));"),
 ]
 
 

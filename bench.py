@@ -14,6 +14,10 @@ resident in HBM, L2 flushed between timed steps.  The same line carries:
                201 MB updated in place): state GB/s against HBM peak;
   decode_tokens  the same batch with 4 tokens per sequence per call through the
                multi-token decode over a state pool: tokens/s, GB/s against HBM peak;
+  prefill_raw_inputs
+               the same step from raw projections (normalisation and gates
+               folded into the kernels), with the prepared-input time and the
+               time with a separate PyTorch prologue for context;
   decode_bf16_state, decode_tokens_bf16_state
                the same with the state pool at rest in bf16 (fp32 arithmetic,
                100 MB of state), 1 and 4 tokens per call;
@@ -390,6 +394,9 @@ def run_ours(args, D):
         "gpu_launches": args.steps * launches,
     }
 
+    out["prefill_raw_inputs"] = _prefill_raw(args, D, dev, x, T, w, ws, fin, o, flush, ms_per_step,
+                                             launches)
+
     if not args.no_e2e:
         out["e2e"] = _e2e(args, D, inp, dev, w, ws)
 
@@ -459,6 +466,63 @@ def _e2e(args, D, inp, dev, w, ws):
     return {"value": D.world * T * args.steps / (ms / 1e3) / 1e6, "unit": "Mtok/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms / args.steps, "host_buffers": "pinned"}
+
+
+def _prefill_raw(args, D, dev, x, T, w, ws, fin, o, flush, prepared_ms, launches):
+    """The same prefill step from the layer's raw projections (GDN_INPUT_RAW):
+    q, k unnormalised, g and beta as the pre-activations a, b.  The kernels fold
+    the normalisation and the gates in; for context, the same inputs prepared by
+    separate PyTorch ops (one more pass over q, k, g, beta) before the prepared
+    prefill."""
+    import torch
+    import torch.nn.functional as F
+
+    from gated_deltanet_recurrence_rule_b200 import api
+
+    gen = torch.Generator(device=dev).manual_seed(11)
+    scale = lambda t: torch.exp(torch.randn(t.shape[:-1] + (1,), generator=gen, device=dev))
+    q = (x["q"].float() * scale(x["q"])).to(x["q"].dtype)
+    k = (x["k"].float() * scale(x["k"])).to(x["k"].dtype)
+    a = torch.log(torch.expm1(-x["g"].double())).float()     # -softplus(a) = g
+    b = torch.log(x["beta"].double() / (1 - x["beta"].double())).float()  # sigmoid(b) = beta
+
+    def fused():
+        api.prefill(q, k, x["v"], a, b, cu_seqlens=x["cu_seqlens"], final_state=fin, o=o,
+                    workspace=ws, raw_inputs=True)
+
+    def separate():
+        qn = F.normalize(q.float(), dim=-1).to(q.dtype)
+        kn = F.normalize(k.float(), dim=-1).to(k.dtype)
+        api.prefill(qn, kn, x["v"], -F.softplus(a), torch.sigmoid(b), cu_seqlens=x["cu_seqlens"],
+                    final_state=fin, o=o, workspace=ws)
+
+    stream = torch.cuda.current_stream(dev)
+    res = {}
+    for name, fn in (("fused", fused), ("separate", separate)):
+        for _ in range(max(args.warmup, 3)):
+            flush.zero_()
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        D.barrier()
+        torch.cuda.synchronize()
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        D.barrier()
+        res[name] = D.max(sum(e0.elapsed_time(e1) for e0, e1 in evs), dev) / args.steps
+    status = api.get_device_status(ws)
+    if status != api.GDN_OK:
+        raise RuntimeError(f"device status after the raw-input leg: {api.status_string(status)}")
+    return {"value": D.world * T / (res["fused"] / 1e3) / 1e6, "unit": "Mtok/s",
+            "workload": "prefill8k from raw projections (q, k unnormalised; g, beta as the "
+                        "pre-activations of -softplus and sigmoid)",
+            "ms_per_step": res["fused"], "prepared_inputs_ms_per_step": prepared_ms,
+            "separate_torch_prologue_ms_per_step": res["separate"],
+            "l2": "flushed between timed steps", "gpu_launches": args.steps * launches}
 
 
 def _decode(args, D, dev, peaks, peak_src):

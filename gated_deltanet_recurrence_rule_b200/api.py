@@ -25,6 +25,8 @@ GDN_ERR_BAD_SEQLENS = 5
 GDN_ERR_WORKSPACE = 6
 GDN_DTYPE_BF16 = 0
 GDN_DTYPE_FP32 = 1
+GDN_INPUT_PREPARED = 0
+GDN_INPUT_RAW = 1
 
 _DTYPE_CODE = {torch.bfloat16: GDN_DTYPE_BF16, torch.float32: GDN_DTYPE_FP32}
 
@@ -64,13 +66,13 @@ def load():
         lib.gdn_prefill_workspace_size_rounds.argtypes = [i32, i64, i32, i32, i32, i32, i32, i64]
         lib.gdn_prefill.restype = i32
         lib.gdn_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32, i32,
-                                    i32, f32, vp, vp, vp, vp, sz, vp]
+                                    i32, i32, f32, vp, vp, vp, vp, sz, vp]
         lib.gdn_decode_step.restype = i32
         lib.gdn_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
                                         i32, f32, vp]
         lib.gdn_decode_tokens.restype = i32
         lib.gdn_decode_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
-                                          i32, i32, i32, i32, i32, i32, f32, vp, vp]
+                                          i32, i32, i32, i32, i32, i32, i32, f32, vp, vp]
         lib.gdn_prefill_uses_tensor_cores.restype = i32
         lib.gdn_prefill_uses_tensor_cores.argtypes = [i32, i32, i32, i32, i32]
         lib.gdn_get_device_status.restype = i32
@@ -130,7 +132,7 @@ def prefill_launch_count(num_seqs, total_tokens, Hqk, Hv, Dk, Dv, workspace_byte
 
 def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_state=True,
             final_state=None, scale=1.0, o=None, workspace=None, o_dtype=torch.float32,
-            state_dtype=None):
+            state_dtype=None, raw_inputs=False):
     """Chunked prefill over packed sequences on the GPU.
 
     q, k [T, Hqk, Dk]; v [T, Hv, Dv] (bf16 or fp32, same dtype); g, beta [T, Hv]
@@ -141,6 +143,8 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_
     otherwise one is allocated when ``output_final_state``.  States are fp32,
     or bf16 kept at rest (fp32 arithmetic, the final state rounded once): the
     dtype of the given states, else ``state_dtype`` (default fp32).
+    ``raw_inputs``: q, k are raw projections (normalised in the kernels) and
+    g, beta hold a, b with g = -softplus(a), beta = sigmoid(b).
     Returns (o [T, Hv, Dv], final_state or None).
     """
     lib = load()
@@ -183,7 +187,8 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_
     _require(workspace, "workspace", dev, torch.uint8)
     st = lib.gdn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens), N, T,
                          Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], _DTYPE_CODE[o.dtype],
-                         _DTYPE_CODE[sdt], float(scale), _ptr(initial_state),
+                         _DTYPE_CODE[sdt], GDN_INPUT_RAW if raw_inputs else GDN_INPUT_PREPARED,
+                         float(scale), _ptr(initial_state),
                          _ptr(final_state), _ptr(o), _ptr(workspace), workspace.numel(),
                          _stream(dev))
     _check(st, "gdn_prefill")
@@ -222,7 +227,7 @@ def decode_step(q, k, v, g, beta, state, o=None, scale=1.0, o_dtype=torch.float3
 
 
 def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst_slot=None,
-                  o=None, scale=1.0, o_dtype=torch.float32, device_status=None):
+                  o=None, scale=1.0, o_dtype=torch.float32, device_status=None, raw_inputs=False):
     """Several tokens per sequence against a pool of states.
 
     q, k [B, Tn, Hqk, Dk]; v [B, Tn, Hv, Dv]; g, beta [B, Tn, Hv] fp32;
@@ -230,7 +235,8 @@ def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst
     bf16, fp32 arithmetic, rounded once per call on store); state_out the same
     shape and dtype (default: state_in, updated in place); src_slot / dst_slot
     [B] int32 or None (slot b / the source slot); device_status an int32 device
-    tensor of one element or None.  Returns o [B, Tn, Hv, Dv] in ``o_dtype``."""
+    tensor of one element or None.  ``raw_inputs`` as for prefill.  Returns o
+    [B, Tn, Hv, Dv] in ``o_dtype``."""
     lib = load()
     if not q.is_cuda:
         raise ValueError("decode_tokens runs on a CUDA device only (q is on the CPU)")
@@ -266,7 +272,8 @@ def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst
     st = lib.gdn_decode_tokens(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(state_in),
                                _ptr(state_out), _ptr(src_slot), _ptr(dst_slot), num_slots, _ptr(o),
                                B, Tn, Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], _DTYPE_CODE[o.dtype],
-                               _DTYPE_CODE[sdt], float(scale), _ptr(device_status), _stream(dev))
+                               _DTYPE_CODE[sdt], GDN_INPUT_RAW if raw_inputs else GDN_INPUT_PREPARED,
+                               float(scale), _ptr(device_status), _stream(dev))
     _check(st, "gdn_decode_tokens")
     return o
 

@@ -17,29 +17,30 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const int32_t *cu, int N, long long T_,
                                 int Hqk, int Hv, int Dk, int Dv, int dtype, int o_dtype,
-                                int state_dtype, float scale, const void *s0, void *sfin, void *o,
-                                int32_t *status, cudaStream_t stream);
+                                int state_dtype, int input_form, float scale, const void *s0,
+                                void *sfin, void *o, int32_t *status, cudaStream_t stream);
 int decode_tokens_max();
 cudaError_t launch_decode_tokens(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const void *state_in, void *state_out,
                                  const int32_t *src_slot, const int32_t *dst_slot, int num_slots,
                                  void *o, int B, int Tn, int Hqk, int Hv, int Dk, int Dv, int dtype,
-                                 int o_dtype, int state_dtype, float scale, int32_t *status,
-                                 cudaStream_t s);
+                                 int o_dtype, int state_dtype, int input_form, float scale,
+                                 int32_t *status, cudaStream_t s);
 bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
-                              int Hv, int o_dtype, int state_dtype, float scale, const void *s0,
-                              void *sfin, void *o, void *workspace, cudaStream_t stream);
+                              int Hv, int o_dtype, int state_dtype, int input_form, float scale,
+                              const void *s0, void *sfin, void *o, void *workspace,
+                              cudaStream_t stream);
 size_t twophase_workspace_bytes(int64_t N, int64_t T, int Hv);
 size_t twophase_round_workspace_bytes(int64_t N, int Hv, int64_t chunks_per_round);
 size_t twophase_min_workspace_bytes(int64_t N, int Hv);
 int64_t twophase_launch_count(int64_t N, int64_t T, int Hv, size_t workspace_bytes);
 cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const int32_t *cu, int N, long long T_,
-                                    int Hqk, int Hv, int o_dtype, int state_dtype, float scale,
-                                    const void *s0, void *sfin, void *o, void *workspace,
-                                    size_t workspace_bytes, cudaStream_t stream);
+                                    int Hqk, int Hv, int o_dtype, int state_dtype, int input_form,
+                                    float scale, const void *s0, void *sfin, void *o,
+                                    void *workspace, size_t workspace_bytes, cudaStream_t stream);
 }  // namespace gdn
 
 namespace {
@@ -49,6 +50,7 @@ constexpr int32_t kVersion = 100;  // 0.1.0
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 bool dtype_ok(int32_t dtype) { return dtype == GDN_DTYPE_BF16 || dtype == GDN_DTYPE_FP32; }
+bool form_ok(int32_t f) { return f == GDN_INPUT_PREPARED || f == GDN_INPUT_RAW; }
 
 bool dims_ok(int32_t Hqk, int32_t Hv, int32_t Dk, int32_t Dv, int32_t dtype) {
   if (Hqk <= 0 || Hv <= 0 || Hv % Hqk != 0) return false;
@@ -134,12 +136,12 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
                     const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
                     int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
                     int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, int32_t o_dtype,
-                    int32_t state_dtype, float scale, const void *initial_state,
-                    void *final_state, void *o, void *workspace, size_t workspace_bytes,
-                    void *stream) {
+                    int32_t state_dtype, int32_t input_form, float scale,
+                    const void *initial_state, void *final_state, void *o, void *workspace,
+                    size_t workspace_bytes, void *stream) {
   if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
   if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
-  if (!dtype_ok(o_dtype) || !dtype_ok(state_dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dtype_ok(o_dtype) || !dtype_ok(state_dtype) || !form_ok(input_form)) return GDN_ERR_INVALID_ARG;
   if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
   if (num_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
   if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
@@ -163,18 +165,20 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
     if (workspace_bytes >= gdn::twophase_min_workspace_bytes(num_seqs, num_v_heads)) {
       // two phases: every chunk's state-free products at once, then the state pass
       e = gdn::launch_prefill_twophase(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
-                                       num_qk_heads, num_v_heads, o_dtype, state_dtype, scale,
-                                       initial_state, final_state, o, workspace, workspace_bytes, s);
+                                       num_qk_heads, num_v_heads, o_dtype, state_dtype, input_form,
+                                       scale, initial_state, final_state, o, workspace,
+                                       workspace_bytes, s);
     } else {
       // a header-only workspace: one pass, each CTA does all of a (sequence, head)
       e = gdn::launch_prefill_tc(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
-                                 num_qk_heads, num_v_heads, o_dtype, state_dtype, scale,
-                                 initial_state, final_state, o, workspace, s);
+                                 num_qk_heads, num_v_heads, o_dtype, state_dtype, input_form,
+                                 scale, initial_state, final_state, o, workspace, s);
     }
   } else {
     e = gdn::launch_prefill_simt(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
                                  num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype,
-                                 state_dtype, scale, initial_state, final_state, o, status, s);
+                                 state_dtype, input_form, scale, initial_state, final_state, o,
+                                 status, s);
   }
   return cuda_status(e);
 }
@@ -204,9 +208,10 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
                           const int32_t *src_slot, const int32_t *dst_slot, int32_t num_slots,
                           void *o, int32_t batch, int32_t tokens, int32_t num_qk_heads,
                           int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
-                          int32_t dtype, int32_t o_dtype, int32_t state_dtype, float scale,
-                          int32_t *device_status, void *stream) {
+                          int32_t dtype, int32_t o_dtype, int32_t state_dtype,
+                          int32_t input_form, float scale, int32_t *device_status, void *stream) {
   if (batch < 0 || tokens < 0 || num_slots < 0) return GDN_ERR_INVALID_ARG;
+  if (!form_ok(input_form)) return GDN_ERR_INVALID_ARG;
   if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
   if (!dtype_ok(o_dtype) || !dtype_ok(state_dtype)) return GDN_ERR_INVALID_ARG;
   if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
@@ -222,8 +227,8 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
     return GDN_ERR_INVALID_ARG;
   return cuda_status(gdn::launch_decode_tokens(
       q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, batch, tokens,
-      num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype, state_dtype, scale,
-      device_status, static_cast<cudaStream_t>(stream)));
+      num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype, state_dtype, input_form,
+      scale, device_status, static_cast<cudaStream_t>(stream)));
 }
 
 int32_t gdn_prefill_uses_tensor_cores(int32_t num_qk_heads, int32_t num_v_heads,

@@ -65,6 +65,17 @@ __device__ __forceinline__ void store_state4(void *base, size_t e, bool bf16, co
   }
 }
 
+// Gates from raw inputs (GDN_INPUT_RAW): log alpha = -softplus(a), written
+// without overflow; alpha itself = e^{-softplus(a)} = 1 / (1 + e^a); beta =
+// sigmoid(b).  Large |a|, |b| saturate to the limits 0 and 1.
+__device__ __forceinline__ float log_alpha_raw(float a) {
+  return -(fmaxf(a, 0.f) + log1pf(expf(-fabsf(a))));
+}
+__device__ __forceinline__ float alpha_raw(float a) { return 1.f / (1.f + expf(a)); }
+__device__ __forceinline__ float beta_raw(float b) { return 1.f / (1.f + expf(-b)); }
+// 1 / |x| from the sum of squares, 0 for a zero row (which then stays zero).
+__device__ __forceinline__ float inv_norm(float ss) { return ss > 0.f ? 1.f / sqrtf(ss) : 0.f; }
+
 // Streaming (evict-first) 128-bit global load / store for data touched once.
 __device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p); }
 __device__ __forceinline__ void st_stream(float4 *p, float4 v) { __stcs(p, v); }

@@ -157,7 +157,7 @@ decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
                      const float *__restrict__ g, const float *__restrict__ beta,
                      const float *state_in, float *state_out, const int32_t *__restrict__ src_slot,
                      const int32_t *__restrict__ dst_slot, int num_slots, TO *__restrict__ o,
-                     int Tn, int Hqk, int Hv, float scale, int32_t *status) {
+                     int Tn, int Hqk, int Hv, float scale, int32_t *status, int raw) {
   pdl_wait();  // nothing is read before the previous kernel on the stream is done
   pdl_allow_next();
   constexpr int NV4 = DK / 32;
@@ -208,10 +208,30 @@ decode_tokens_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
   }
   for (int t = threadIdx.x; t < Tn; t += blockDim.x) {
     const size_t gi = ((size_t)b * Tn + t) * Hv + h;
-    tok[t][0] = expf(g[gi]);
-    tok[t][1] = beta[gi];
+    tok[t][0] = raw ? alpha_raw(g[gi]) : expf(g[gi]);
+    tok[t][1] = raw ? beta_raw(beta[gi]) : beta[gi];
   }
   __syncthreads();
+  if (raw) {  // unit L2 norm per token for k and q, one token per warp in turn
+    for (int t = warp; t < Tn; t += 4) {
+      float sk = 0.f, sq = 0.f;
+      for (int d = lane; d < DK; d += 32) {
+        sk = fmaf(kq[t][0][d], kq[t][0][d], sk);
+        sq = fmaf(kq[t][1][d], kq[t][1][d], sq);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      }
+      const float rk = inv_norm(sk), rq = inv_norm(sq);
+      for (int d = lane; d < DK; d += 32) {
+        kq[t][0][d] *= rk;
+        kq[t][1][d] *= rq;
+      }
+    }
+    __syncthreads();
+  }
 
 #pragma unroll
   for (int gb = 0; gb < GROUPS; gb += BATCH) {
@@ -290,7 +310,7 @@ decode_tokens_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k,
                            __nv_bfloat16 *state_out, const int32_t *__restrict__ src_slot,
                            const int32_t *__restrict__ dst_slot, int num_slots,
                            TO *__restrict__ o, int Tn, int Hqk, int Hv, float scale,
-                           int32_t *status) {
+                           int32_t *status, int raw) {
   pdl_wait();  // nothing is read before the previous kernel on the stream is done
   pdl_allow_next();
   constexpr int NU = DK / 64;  // 16-byte pieces per lane per row
@@ -318,12 +338,12 @@ decode_tokens_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k,
   const size_t rowS = (size_t)h * DV + warp * ROWS_PER_WARP;  // first row of this warp in a slot
   const __nv_bfloat16 *Sin = state_in + ((size_t)src * Hv * DV + rowS) * DK;
   __nv_bfloat16 *Sout = state_out + ((size_t)dst * Hv * DV + rowS) * DK;
-  uint4 raw[GROUPS][NU];
+  uint4 packed[GROUPS][NU];
 #pragma unroll
   for (int x = 0; x < GROUPS; ++x)
 #pragma unroll
     for (int m = 0; m < NU; ++m)
-      raw[x][m] = __ldcs(reinterpret_cast<const uint4 *>(Sin + (size_t)(x * 4 + rr) * DK + 64 * m + 8 * c8));
+      packed[x][m] = __ldcs(reinterpret_cast<const uint4 *>(Sin + (size_t)(x * 4 + rr) * DK + 64 * m + 8 * c8));
 
   // stage k_t, q_t (fp32, column d = 64 m + 8 c + 4 hf + e at 32 (2 m + hf) + 4 c + e),
   // v_t and the per-token scalars
@@ -340,11 +360,28 @@ decode_tokens_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k,
   }
   for (int t = threadIdx.x; t < Tn; t += blockDim.x) {
     const size_t gi = ((size_t)b * Tn + t) * Hv + h;
-    tok[t][0] = expf(g[gi]);
-    tok[t][1] = beta[gi];
+    tok[t][0] = raw ? alpha_raw(g[gi]) : expf(g[gi]);
+    tok[t][1] = raw ? beta_raw(beta[gi]) : beta[gi];
   }
   __syncthreads();
   for (int t = warp; t < Tn; t += 4) {  // k_t . q_t, one token per warp in turn
+    if (raw) {  // unit L2 norm for k_t and q_t first (order of columns is immaterial)
+      float sk = 0.f, sq = 0.f;
+      for (int d = lane; d < DK; d += 32) {
+        sk = fmaf(kq[t][0][d], kq[t][0][d], sk);
+        sq = fmaf(kq[t][1][d], kq[t][1][d], sq);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+      }
+      const float rk = inv_norm(sk), rq = inv_norm(sq);
+      for (int d = lane; d < DK; d += 32) {
+        kq[t][0][d] *= rk;
+        kq[t][1][d] *= rq;
+      }
+    }
     float a = 0.f;
     for (int d = lane; d < DK; d += 32) a = fmaf(kq[t][0][d], kq[t][1][d], a);
 #pragma unroll
@@ -360,8 +397,8 @@ decode_tokens_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k,
     for (int x = 0; x < STAGE; ++x)
 #pragma unroll
       for (int m = 0; m < NU; ++m) {
-        const uint32_t w[4] = {raw[gs + x][m].x, raw[gs + x][m].y, raw[gs + x][m].z,
-                               raw[gs + x][m].w};
+        const uint32_t w[4] = {packed[gs + x][m].x, packed[gs + x][m].y, packed[gs + x][m].z,
+                               packed[gs + x][m].w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
           s[x][4 * m + i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
@@ -428,7 +465,7 @@ decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                         const __nv_bfloat16 *state_in, __nv_bfloat16 *state_out,
                         const int32_t *__restrict__ src_slot, const int32_t *__restrict__ dst_slot,
                         int num_slots, TO *__restrict__ o, int Hqk, int Hv, float scale,
-                        int32_t *status) {
+                        int32_t *status, int raw) {
   pdl_wait();  // nothing is read before the previous kernel on the stream is done
   pdl_allow_next();
   constexpr int NU = DK / 64;  // 16-byte pieces per lane per row
@@ -452,12 +489,12 @@ decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
   const size_t rowS = (size_t)h * DV + warp * ROWS_PER_WARP;  // first row of this warp in a slot
   const __nv_bfloat16 *Sin = state_in + ((size_t)src * Hv * DV + rowS) * DK;
   __nv_bfloat16 *Sout = state_out + ((size_t)dst * Hv * DV + rowS) * DK;
-  uint4 raw[GROUPS][NU];
+  uint4 packed[GROUPS][NU];
 #pragma unroll
   for (int x = 0; x < GROUPS; ++x)
 #pragma unroll
     for (int m = 0; m < NU; ++m)
-      raw[x][m] = __ldcs(reinterpret_cast<const uint4 *>(Sin + (size_t)(x * 4 + rr) * DK + 64 * m + 8 * c8));
+      packed[x][m] = __ldcs(reinterpret_cast<const uint4 *>(Sin + (size_t)(x * 4 + rr) * DK + 64 * m + 8 * c8));
 
   float2 kf[E / 2], qf[E / 2];  // columns 64 m + 8 c8 + (0..7), in pairs
   const T *kp = k + ((size_t)b * Hqk + j) * DK;
@@ -472,6 +509,26 @@ decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
       kf[4 * m + 2 * hf] = make_float2(a[0], a[1]); kf[4 * m + 2 * hf + 1] = make_float2(a[2], a[3]);
       qf[4 * m + 2 * hf] = make_float2(c[0], c[1]); qf[4 * m + 2 * hf + 1] = make_float2(c[2], c[3]);
     }
+  if (raw) {  // unit L2 norm: the 8 lanes of a row group hold all Dk columns
+    float2 sk2 = make_float2(0.f, 0.f), sq2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      sk2 = __ffma2_rn(kf[e], kf[e], sk2);
+      sq2 = __ffma2_rn(qf[e], qf[e], sq2);
+    }
+    float sk = sk2.x + sk2.y, sq = sq2.x + sq2.y;
+#pragma unroll
+    for (int off = 1; off < 8; off <<= 1) {
+      sk += __shfl_xor_sync(0xffffffffu, sk, off);
+      sq += __shfl_xor_sync(0xffffffffu, sq, off);
+    }
+    const float2 rk = make_float2(inv_norm(sk), inv_norm(sk)), rq = make_float2(inv_norm(sq), inv_norm(sq));
+#pragma unroll
+    for (int e = 0; e < E / 2; ++e) {
+      kf[e] = __fmul2_rn(kf[e], rk);
+      qf[e] = __fmul2_rn(qf[e], rq);
+    }
+  }
   float2 kap2 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int e = 0; e < E / 2; ++e) kap2 = __ffma2_rn(kf[e], qf[e], kap2);
@@ -480,8 +537,8 @@ decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
   kap += __shfl_xor_sync(0xffffffffu, kap, 2);
   kap += __shfl_xor_sync(0xffffffffu, kap, 4);
 
-  const float alpha = expf(g[bh]);
-  const float bt = beta[bh];
+  const float alpha = raw ? alpha_raw(g[bh]) : expf(g[bh]);
+  const float bt = raw ? beta_raw(beta[bh]) : beta[bh];
   const float2 alpha2 = make_float2(alpha, alpha);
   const size_t row0 = (size_t)bh * DV + warp * ROWS_PER_WARP;  // o and v rows of this warp
   const float vreg = lane < ROWS_PER_WARP ? to_f32(v[row0 + lane]) : 0.f;
@@ -492,7 +549,7 @@ decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
     float2 s[E / 2];
 #pragma unroll
     for (int m = 0; m < NU; ++m) {
-      const uint32_t w[4] = {raw[x][m].x, raw[x][m].y, raw[x][m].z, raw[x][m].w};
+      const uint32_t w[4] = {packed[x][m].x, packed[x][m].y, packed[x][m].z, packed[x][m].w};
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         s[4 * m + i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
@@ -538,7 +595,7 @@ static cudaError_t launch_decode_tokens_t(const void *q, const void *k, const vo
                                           const float *g, const float *beta, const void *sin,
                                           void *sout, const int32_t *src, const int32_t *dst,
                                           int num_slots, void *o, int B, int Tn, int Hqk, int Hv,
-                                          float scale, int state_dtype, int32_t *status,
+                                          float scale, int state_dtype, int raw, int32_t *status,
                                           cudaStream_t stream) {
   const unsigned blocks = (unsigned)B * (unsigned)Hv;
   const T *qt = static_cast<const T *>(q), *kt = static_cast<const T *>(k),
@@ -548,15 +605,15 @@ static cudaError_t launch_decode_tokens_t(const void *q, const void *k, const vo
     return launch_pdl(decode_one_bf16s_kernel<T, TO, DK, DV>, blocks, 128, 0, stream, qt, kt, vt,
                       g, beta, static_cast<const __nv_bfloat16 *>(sin),
                       static_cast<__nv_bfloat16 *>(sout), src, dst, num_slots, ot, Hqk, Hv, scale,
-                      status);
+                      status, raw);
   if (state_dtype == GDN_DTYPE_BF16)
     return launch_pdl(decode_tokens_bf16s_kernel<T, TO, DK, DV>, blocks, 128, 0, stream, qt, kt,
                       vt, g, beta, static_cast<const __nv_bfloat16 *>(sin),
                       static_cast<__nv_bfloat16 *>(sout), src, dst, num_slots, ot, Tn, Hqk, Hv,
-                      scale, status);
+                      scale, status, raw);
   return launch_pdl(decode_tokens_kernel<T, TO, DK, DV>, blocks, 128, 0, stream, qt, kt, vt, g,
                     beta, static_cast<const float *>(sin), static_cast<float *>(sout), src, dst,
-                    num_slots, ot, Tn, Hqk, Hv, scale, status);
+                    num_slots, ot, Tn, Hqk, Hv, scale, status, raw);
 }
 
 int decode_tokens_max() { return kMaxTokens; }
@@ -565,18 +622,19 @@ cudaError_t launch_decode_tokens(const void *q, const void *k, const void *v, co
                                  const float *beta, const void *state_in, void *state_out,
                                  const int32_t *src_slot, const int32_t *dst_slot, int num_slots,
                                  void *o, int B, int Tn, int Hqk, int Hv, int Dk, int Dv, int dtype,
-                                 int o_dtype, int state_dtype, float scale, int32_t *status,
-                                 cudaStream_t s) {
+                                 int o_dtype, int state_dtype, int input_form, float scale,
+                                 int32_t *status, cudaStream_t s) {
+  const int raw = input_form == GDN_INPUT_RAW;
   return dispatch_types(dtype, o_dtype, [&](auto t, auto to) {
     using T = decltype(t);
     using TO = decltype(to);
     if (Dk == 128 && Dv == 128)
-      return launch_decode_tokens_t<T, TO, 128, 128>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, status, s);
+      return launch_decode_tokens_t<T, TO, 128, 128>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, raw, status, s);
     if (Dk == 128 && Dv == 64)
-      return launch_decode_tokens_t<T, TO, 128, 64>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, status, s);
+      return launch_decode_tokens_t<T, TO, 128, 64>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, raw, status, s);
     if (Dk == 64 && Dv == 128)
-      return launch_decode_tokens_t<T, TO, 64, 128>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, status, s);
-    return launch_decode_tokens_t<T, TO, 64, 64>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, status, s);
+      return launch_decode_tokens_t<T, TO, 64, 128>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, raw, status, s);
+    return launch_decode_tokens_t<T, TO, 64, 64>(q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, B, Tn, Hqk, Hv, scale, state_dtype, raw, status, s);
   });
 }
 

@@ -69,7 +69,8 @@ extern "C" int32_t gdn_prefill_noalloc(const void *q, const void *k, const void 
   if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return GDN_ERR_CUDA;
   const int32_t rc = gdn_prefill(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
                                  num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype,
-                                 o_dtype, GDN_DTYPE_FP32, scale, initial_state, final_state, o,
+                                 o_dtype, GDN_DTYPE_FP32, GDN_INPUT_PREPARED, scale, initial_state,
+                                 final_state, o,
                                  scratch, kScratchBytes, stream);
   if (rc != GDN_OK) return rc;
   if (device_status &&

@@ -55,11 +55,11 @@ __global__ void __launch_bounds__(128)
 prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                     const float *__restrict__ g, const float *__restrict__ beta,
                     const int32_t *__restrict__ cu, int N, long long Ttot, int Hqk, int Hv,
-                    int DV, float scale, const void *s0, void *sfin, int state_bf16,
+                    int DV, float scale, const void *s0, void *sfin, int state_bf16, int raw,
                     TO *__restrict__ o, int32_t *status) {
   using C = SimtCfg<T, DK>;
   extern __shared__ __align__(16) unsigned char smem[];
-  unsigned char *raw[2] = {smem, smem + C::RAW_BYTES};
+  unsigned char *stage_buf[2] = {smem, smem + C::RAW_BYTES};
   float *fq = reinterpret_cast<float *>(smem + 2 * C::RAW_BYTES);
   float *fk = fq + C::STAGE * DK;
   float *fv = fk + C::STAGE * DK;
@@ -97,7 +97,7 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
 
   // Copy the raw inputs of stage s into raw buffer s % 2.
   auto issue = [&](int s) {
-    unsigned char *buf = raw[s & 1];
+    unsigned char *buf = stage_buf[s & 1];
     const long long t0 = c0 + (long long)s * C::STAGE;
     const int cnt = (int)min((long long)C::STAGE, c1 - t0);
     constexpr int QK_CHUNKS = DK * (int)sizeof(T) / 16;  // 16-byte chunks per row
@@ -133,7 +133,7 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
     const long long t0 = c0 + (long long)st * C::STAGE;
     const int cnt = (int)min((long long)C::STAGE, c1 - t0);
     {  // convert stage st to fp32
-      const unsigned char *buf = raw[st & 1];
+      const unsigned char *buf = stage_buf[st & 1];
       const T *rq = reinterpret_cast<const T *>(buf);
       const T *rk = reinterpret_cast<const T *>(buf + C::RAW_QK);
       const T *rv = reinterpret_cast<const T *>(buf + 2 * C::RAW_QK);
@@ -151,11 +151,32 @@ prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *_
         *reinterpret_cast<float4 *>(fv + idx) = make_float4(x[0], x[1], x[2], x[3]);
       }
       if (tid < cnt) {
-        fa[tid] = expf(rg[tid]);
-        fb[tid] = rg[C::STAGE + tid];
+        fa[tid] = raw ? alpha_raw(rg[tid]) : expf(rg[tid]);
+        fb[tid] = raw ? beta_raw(rg[C::STAGE + tid]) : rg[C::STAGE + tid];
       }
     }
     __syncthreads();
+    if (raw) {  // unit L2 norm per token for k and q, one token per warp in turn
+      const int warp = tid >> 5, lane = tid & 31;
+      for (int t = warp; t < cnt; t += C::THREADS / 32) {
+        float sk = 0.f, sq = 0.f;
+        for (int d = lane; d < DK; d += 32) {
+          sk = fmaf(fk[t * DK + d], fk[t * DK + d], sk);
+          sq = fmaf(fq[t * DK + d], fq[t * DK + d], sq);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          sk += __shfl_xor_sync(0xffffffffu, sk, off);
+          sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        }
+        const float rk = inv_norm(sk), rq = inv_norm(sq);
+        for (int d = lane; d < DK; d += 32) {
+          fk[t * DK + d] *= rk;
+          fq[t * DK + d] *= rq;
+        }
+      }
+      __syncthreads();
+    }
 
     for (int t = 0; t < cnt; ++t) {
       const float *kt = fk + t * DK;
@@ -200,7 +221,7 @@ template <typename T, typename TO, int DK>
 static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, const float *g,
                                  const float *beta, const int32_t *cu, int N, long long T_,
                                  int Hqk, int Hv, int Dv, float scale, const void *s0,
-                                 void *sfin, int state_bf16, void *o, int32_t *status,
+                                 void *sfin, int state_bf16, int raw, void *o, int32_t *status,
                                  cudaStream_t stream) {
   using C = SimtCfg<T, DK>;
   auto kern = prefill_simt_kernel<T, TO, DK>;
@@ -209,22 +230,22 @@ static cudaError_t launch_simt_t(const void *q, const void *k, const void *v, co
   const unsigned blocks = (unsigned)N * (unsigned)Hv * (unsigned)(Dv / C::ROWS);
   kern<<<blocks, C::THREADS, C::SMEM, stream>>>(
       static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), g, beta,
-      cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, state_bf16, static_cast<TO *>(o), status);
+      cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, state_bf16, raw, static_cast<TO *>(o), status);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *g,
                                 const float *beta, const int32_t *cu, int N, long long T_,
                                 int Hqk, int Hv, int Dk, int Dv, int dtype, int o_dtype,
-                                int state_dtype, float scale, const void *s0, void *sfin, void *o,
-                                int32_t *status, cudaStream_t stream) {
-  const int sb = state_dtype == GDN_DTYPE_BF16;
+                                int state_dtype, int input_form, float scale, const void *s0,
+                                void *sfin, void *o, int32_t *status, cudaStream_t stream) {
+  const int sb = state_dtype == GDN_DTYPE_BF16, raw = input_form == GDN_INPUT_RAW;
   return dispatch_types(dtype, o_dtype, [&](auto t, auto to) {
     using T = decltype(t);
     using TO = decltype(to);
     if (Dk == 128)
-      return launch_simt_t<T, TO, 128>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, sb, o, status, stream);
-    return launch_simt_t<T, TO, 64>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, sb, o, status, stream);
+      return launch_simt_t<T, TO, 128>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, sb, raw, o, status, stream);
+    return launch_simt_t<T, TO, 64>(q, k, v, g, beta, cu, N, T_, Hqk, Hv, Dv, scale, s0, sfin, sb, raw, o, status, stream);
   });
 }
 

@@ -88,7 +88,7 @@ constexpr uint32_t R1_BYTES = 54272;
 constexpr uint32_t OFF_PH = OFF_R1 + R1_BYTES;  // bf16 hi(P), K-major B: 64 rows (t) x 64 s
 constexpr uint32_t OFF_PL = OFF_PH + 8192;      // bf16 lo(P)
 constexpr uint32_t OFF_SCAL = OFF_PL + 8192;
-constexpr uint32_t SCAL_STAGE = 5 * 64 * 4;  // G2 (log2 prefix), gamma, kdec, beta; gamma_C at [256]
+constexpr uint32_t SCAL_STAGE = 7 * 64 * 4;  // G2 (log2 prefix), gamma, kdec, beta; gamma_C at [256]; 1/|q|, 1/|k| at [320], [384]
 constexpr uint32_t OFF_BAR = OFF_SCAL + 2 * SCAL_STAGE;
 constexpr uint32_t OFF_MISC = OFF_BAR + 192;  // [0] TMEM base, [4] abort flag, [8] drain mbarrier
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
@@ -130,6 +130,8 @@ struct Params {
   const void *s0;  // caller's initial states, fp32 or (state_bf16) bf16
   void *sfin;      // caller's final states, same type
   int state_bf16;
+  int raw;         // GDN_INPUT_RAW: q, k normalised here, g and beta through -softplus, sigmoid
+  const void *q, *k;  // raw inputs: rows read for their norms
   void *o;
   int32_t *status;
 };
@@ -347,13 +349,45 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int t0 = c0 + c * CH;
       const int Lc = min(CH, c1 - t0);
       float ga = 0.f, gb = 0.f, ba = 0.f, bb = 0.f;
+      auto log_alpha = [&](float x) { return fmaxf(p.raw ? log_alpha_raw(x) : x, G_FLOOR); };
+      auto write_strength = [&](float x) { return p.raw ? beta_raw(x) : x; };
       if (lane < Lc) {
-        ga = fmaxf(p.g[(size_t)(t0 + lane) * p.Hv + h], G_FLOOR);
-        ba = p.beta[(size_t)(t0 + lane) * p.Hv + h];
+        ga = log_alpha(p.g[(size_t)(t0 + lane) * p.Hv + h]);
+        ba = write_strength(p.beta[(size_t)(t0 + lane) * p.Hv + h]);
       }
       if (lane + 32 < Lc) {
-        gb = fmaxf(p.g[(size_t)(t0 + lane + 32) * p.Hv + h], G_FLOOR);
-        bb = p.beta[(size_t)(t0 + lane + 32) * p.Hv + h];
+        gb = log_alpha(p.g[(size_t)(t0 + lane + 32) * p.Hv + h]);
+        bb = write_strength(p.beta[(size_t)(t0 + lane + 32) * p.Hv + h]);
+      }
+      // Raw inputs: 1/|q_t|, 1/|k_t| of rows t = lane, lane + 32 (read from global
+      // memory: the shared tiles are recycled once their MMAs are done), folded
+      // into the scalars below and in the epilogue, not into the bf16 tiles.
+      float rq[2] = {1.f, 1.f}, rk[2] = {1.f, 1.f};
+      if (p.raw) {
+#pragma unroll
+        for (int w = 0; w < 2; ++w) {
+          const int t = lane + 32 * w;
+          float sq = 0.f, sk = 0.f;
+          if (t < Lc) {
+            const size_t off = ((size_t)(t0 + t) * p.Hqk + j) * HD;
+            const uint4 *qr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.q) + off);
+            const uint4 *kr = reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(p.k) + off);
+#pragma unroll 4
+            for (int c16 = 0; c16 < HD / 8; ++c16) {
+              const uint4 xq = qr[c16], xk = kr[c16];
+              const uint32_t wq[4] = {xq.x, xq.y, xq.z, xq.w}, wk[4] = {xk.x, xk.y, xk.z, xk.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const float q0 = __uint_as_float(wq[i] << 16), q1 = __uint_as_float(wq[i] & 0xffff0000u);
+                const float k0 = __uint_as_float(wk[i] << 16), k1 = __uint_as_float(wk[i] & 0xffff0000u);
+                sq = fmaf(q0, q0, fmaf(q1, q1, sq));
+                sk = fmaf(k0, k0, fmaf(k1, k1, sk));
+              }
+            }
+          }
+          rq[w] = inv_norm(sq);
+          rk[w] = inv_norm(sk);
+        }
       }
 #pragma unroll
       for (int off = 1; off < 32; off <<= 1) {
@@ -369,10 +403,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       float *sc = reinterpret_cast<float *>(smem + OFF_SCAL + s * SCAL_STAGE);
       sc[lane] = Ga;                 sc[lane + 32] = Gb;
       sc[64 + lane] = exp2f(Ga);     sc[64 + lane + 32] = exp2f(Gb);
-      sc[128 + lane] = lane < Lc ? exp2f(GL - Ga) : 0.f;
-      sc[128 + lane + 32] = lane + 32 < Lc ? exp2f(GL - Gb) : 0.f;
+      sc[128 + lane] = lane < Lc ? exp2f(GL - Ga) * rk[0] : 0.f;
+      sc[128 + lane + 32] = lane + 32 < Lc ? exp2f(GL - Gb) * rk[1] : 0.f;
       sc[192 + lane] = ba;           sc[192 + lane + 32] = bb;
       if (lane == 0) sc[256] = exp2f(GL);
+      sc[320 + lane] = rq[0];        sc[320 + lane + 32] = rq[1];
+      sc[384 + lane] = rk[0];        sc[384 + lane + 32] = rk[1];
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_addr(sb, B_SCAL_FULL + s));
     }
@@ -408,7 +444,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int t0 = c0 + c * CH;
       const int Lc = min(CH, c1 - t0);
       const float *sc = reinterpret_cast<const float *>(smem + OFF_SCAL + s * SCAL_STAGE);
-      const float *G2 = sc, *gam = sc + 64, *kdec = sc + 128, *bet = sc + 192;
+      const float *G2 = sc, *gam = sc + 64, *kdec = sc + 128, *bet = sc + 192, *rqn = sc + 320,
+                  *rkn = sc + 384;
 
       // ---- Q K^T and K K^T -> P (hi/lo) and A (fp32)
       if (etid == 0) {
@@ -424,21 +461,21 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tmem_wait_ld();
         if (row < 64) {
           const int t = row;
-          const float Gt = G2[t];
+          const float Gt = G2[t], rq = rqn[t];
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             float pv[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int si = 16 * ewq + 8 * q + e;
-              pv[e] = (si <= t && t < Lc) ? exp2f(Gt - G2[si]) * v[8 * q + e] : 0.f;
+              pv[e] = (si <= t && t < Lc) ? exp2f(Gt - G2[si]) * v[8 * q + e] * (rq * rkn[si]) : 0.f;
             }
             const uint32_t off = sw128_off(t, 2 * ewq + q);
             st_split8(smem + OFF_PH + off, smem + OFF_PL + off, pv);
           }
         } else {
           const int t = row - 64;
-          const float Gt = G2[t], bt = bet[t];
+          const float Gt = G2[t], bt = bet[t], rk = rkn[t];
           float *arow = A + t * AST + 16 * ewq;
 #pragma unroll
           for (int x = 0; x < 16; x += 4) {
@@ -446,7 +483,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int si = 16 * ewq + x + e;
-              a[e] = (si < t && t < Lc) ? bt * exp2f(Gt - G2[si]) * v[x + e] : 0.f;
+              a[e] = (si < t && t < Lc) ? bt * exp2f(Gt - G2[si]) * v[x + e] * (rk * rkn[si]) : 0.f;
             }
             *reinterpret_cast<float4 *>(arow + x) = make_float4(a[0], a[1], a[2], a[3]);
           }
@@ -465,9 +502,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const float4 a4 = *reinterpret_cast<const float4 *>(Tm + t * AST + sbeg + e);
           const float4 b4 = *reinterpret_cast<const float4 *>(bet + sbeg + e);
           const float4 g4 = *reinterpret_cast<const float4 *>(gam + sbeg + e);
+          const float4 r4 = *reinterpret_cast<const float4 *>(rkn + sbeg + e);
           tm[e] = a4.x; tm[e + 1] = a4.y; tm[e + 2] = a4.z; tm[e + 3] = a4.w;
           bt[e] = b4.x; bt[e + 1] = b4.y; bt[e + 2] = b4.z; bt[e + 3] = b4.w;
-          gm[e] = g4.x; gm[e + 1] = g4.y; gm[e + 2] = g4.z; gm[e + 3] = g4.w;
+          gm[e] = g4.x * r4.x; gm[e + 1] = g4.y * r4.y; gm[e + 2] = g4.z * r4.z; gm[e + 3] = g4.w * r4.w;
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -544,7 +582,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
         for (int x = 0; x < 16; ++x) {
           const int t = 16 * ewq + x;
-          if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(p.scale * fmaf(gam[t], vi[x], va[x]));
+          if (t < Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(p.scale * fmaf(gam[t] * rqn[t], vi[x], va[x]));
         }
         tmem_wait_st();
       }
@@ -592,9 +630,12 @@ bool prefill_tc_supported(int Hqk, int Hv, int Dk, int Dv, int dtype) {
 
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *g,
                               const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
-                              int Hv, int o_dtype, int state_dtype, float scale, const void *s0,
-                              void *sfin, void *o, void *workspace, cudaStream_t stream) {
+                              int Hv, int o_dtype, int state_dtype, int input_form, float scale,
+                              const void *s0, void *sfin, void *o, void *workspace,
+                              cudaStream_t stream) {
   tc::Params prm;
+  prm.raw = input_form == GDN_INPUT_RAW;
+  prm.q = q; prm.k = k;
   prm.g = g; prm.beta = beta; prm.cu = cu; prm.N = N; prm.T = (int)T_; prm.Hqk = Hqk; prm.Hv = Hv;
   prm.scale = scale; prm.s0 = s0; prm.sfin = sfin; prm.state_bf16 = state_dtype == GDN_DTYPE_BF16;
   prm.o = o;

@@ -36,7 +36,7 @@ namespace gdn {
 size_t wy_prep_smem_bytes();
 cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                            const float *g, const float *beta, const int32_t *cu, int T, int Hqk,
-                           int Hv, int round, int rc, const void *workspace,
+                           int Hv, int round, int rc, int raw, const void *workspace,
                            const tp::Layout &L, unsigned char *rec, cudaStream_t stream);
 
 namespace plan {
@@ -678,10 +678,11 @@ cudaError_t device_streams(DeviceStreams **out) {
 // rounds run one after another on `stream` with as many chunks as fit.
 cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v, const float *g,
                                     const float *beta, const int32_t *cu, int N, long long T_,
-                                    int Hqk, int Hv, int o_dtype, int state_dtype, float scale,
-                                    const void *s0, void *sfin, void *o, void *workspace,
-                                    size_t workspace_bytes, cudaStream_t stream) {
+                                    int Hqk, int Hv, int o_dtype, int state_dtype, int input_form,
+                                    float scale, const void *s0, void *sfin, void *o,
+                                    void *workspace, size_t workspace_bytes, cudaStream_t stream) {
   const int T = (int)T_;
+  const int raw = input_form == GDN_INPUT_RAW;
   const tp::Layout L = tp::layout(N, Hv);
   unsigned char *ws = static_cast<unsigned char *>(workspace);
   int32_t *status = reinterpret_cast<int32_t *>(ws);
@@ -720,7 +721,8 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
     if ((e = cudaGetLastError()) != cudaSuccess || T == 0) return e;
     prm.rec = ws + L.rec_off;
     for (int r = 0; r < rounds; ++r) {
-      e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, workspace, L, ws + L.rec_off, stream);
+      e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, raw, workspace, L, ws + L.rec_off,
+                         stream);
       if (e != cudaSuccess) return e;
       prm.round = r;
       if ((e = state_pass(stream)) != cudaSuccess) return e;
@@ -748,7 +750,7 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
     // phase 1 of round r reuses the buffer phase 2 of round r - 2 read
     if (r >= 2 && (e = cudaStreamWaitEvent(d->prep, d->ev_c[(r - 2) % kEventRing], 0)) != cudaSuccess)
       return e;
-    e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, workspace, L, rec, d->prep);
+    e = launch_wy_prep(mq, mk, mv, g, beta, cu, T, Hqk, Hv, r, rc, raw, workspace, L, rec, d->prep);
     if (e != cudaSuccess) return e;
     if ((e = cudaEventRecord(d->ev_p[r % kEventRing], d->prep)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(d->chain, d->ev_p[r % kEventRing], 0)) != cudaSuccess) return e;

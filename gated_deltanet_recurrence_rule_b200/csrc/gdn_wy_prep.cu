@@ -15,6 +15,9 @@
 //     U~^T = V^T T''^T  (same shape)
 //     W^T -> record as bf16, U~ -> record as fp32, with e^{G_t},
 //     e^{G_C - G_t} and e^{G_C}.
+// With raw inputs (GDN_INPUT_RAW) g and beta pass through -softplus and
+// sigmoid here, and q, k are normalised by folding 1/|q_t|, 1/|k_t| into the
+// per-token scalars (the operand tiles keep the raw bf16 values).
 // Padded rows (t >= chunk length) get beta = 0, so their W and U~ rows are 0.
 //
 // One CTA per (chunk of the round, value head), two CTAs per SM; 384 threads:
@@ -58,8 +61,8 @@ constexpr uint32_t OFF_TPH = OFF_R1;           // hi/lo(T') over A, after the so
 constexpr uint32_t OFF_TPL = OFF_R1 + 8192;
 constexpr uint32_t OFF_TQH = OFF_QK;           // hi/lo(T'') over the Q halves, after [Q;K]K^T
 constexpr uint32_t OFF_TQL = OFF_QK + 16384;
-constexpr uint32_t OFF_SCAL = OFF_R1 + 38912;  // G2 (log2 prefix), gamma, kdec, beta [64 each]
-constexpr uint32_t OFF_BAR = OFF_SCAL + 1280;
+constexpr uint32_t OFF_SCAL = OFF_R1 + 38912;  // G2 (log2 prefix), gamma, kdec, beta, 1/|q|, 1/|k| [64 each]
+constexpr uint32_t OFF_BAR = OFF_SCAL + 1792;
 constexpr uint32_t OFF_MISC = OFF_BAR + 64;    // [0] TMEM base, [4] abort flag, [8] drain mbarrier
 constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
 static_assert(OFF_Y + 3 * 16 * 17 * 4 <= OFF_SCAL, "R1 layout");
@@ -82,6 +85,7 @@ struct Params {
   int T, Hqk, Hv;
   int round, rc;  // this launch covers global chunks [round rc, round rc + rc)
   int resident;   // CTAs resident at once (2 per SM): the distance to the next CTA on a slot
+  int raw;        // GDN_INPUT_RAW: q, k normalised here, g and beta through -softplus, sigmoid
   const tp::PlanHeader *plan;
   const int32_t *ne_seq, *ne_cs;
   unsigned char *rec;  // this round's records, [rc][Hv]
@@ -207,13 +211,15 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   } else if (warp == 2) {
     // ------------------------------------------------------------ chunk scalars
     float ga = 0.f, gb = 0.f, ba = 0.f, bb = 0.f;
+    auto log_alpha = [&](float x) { return fmaxf(p.raw ? log_alpha_raw(x) : x, G_FLOOR); };
+    auto write_strength = [&](float x) { return p.raw ? beta_raw(x) : x; };
     if (lane < Lc) {
-      ga = fmaxf(p.g[(size_t)(t0 + lane) * p.Hv + h], G_FLOOR);
-      ba = p.beta[(size_t)(t0 + lane) * p.Hv + h];
+      ga = log_alpha(p.g[(size_t)(t0 + lane) * p.Hv + h]);
+      ba = write_strength(p.beta[(size_t)(t0 + lane) * p.Hv + h]);
     }
     if (lane + 32 < Lc) {
-      gb = fmaxf(p.g[(size_t)(t0 + lane + 32) * p.Hv + h], G_FLOOR);
-      bb = p.beta[(size_t)(t0 + lane + 32) * p.Hv + h];
+      gb = log_alpha(p.g[(size_t)(t0 + lane + 32) * p.Hv + h]);
+      bb = write_strength(p.beta[(size_t)(t0 + lane + 32) * p.Hv + h]);
     }
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -234,9 +240,13 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     sc[64 + lane] = gma;  sc[64 + lane + 32] = gmb;
     sc[128 + lane] = kda; sc[128 + lane + 32] = kdb;
     sc[192 + lane] = ba;  sc[192 + lane + 32] = bb;
+    sc[256 + lane] = 1.f; sc[256 + lane + 32] = 1.f;  // 1/|q_t|, 1/|k_t|: set by the epilogue
+    sc[320 + lane] = 1.f; sc[320 + lane + 32] = 1.f;  // for raw inputs
     float *rs = reinterpret_cast<float *>(rec + tp::REC_SC);
-    rs[lane] = gma;       rs[lane + 32] = gmb;
-    rs[64 + lane] = kda;  rs[64 + lane + 32] = kdb;
+    if (!p.raw) {  // for raw inputs the epilogue writes them with the norms folded in
+      rs[lane] = gma;       rs[lane + 32] = gmb;
+      rs[64 + lane] = kda;  rs[64 + lane + 32] = kdb;
+    }
     if (lane == 0) rs[128] = exp2f(GL);
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_addr(sb, B_SCAL));
@@ -250,11 +260,42 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     float *Tm = reinterpret_cast<float *>(smem + OFF_TM);
     float *Y = reinterpret_cast<float *>(smem + OFF_Y);
     const float *sc = reinterpret_cast<const float *>(smem + OFF_SCAL);
-    const float *G2 = sc, *gam = sc + 64, *bet = sc + 192;
+    const float *G2 = sc, *gam = sc + 64, *bet = sc + 192, *rqn = sc + 256, *rkn = sc + 320;
     do {
       if (etid == 0 && !mbar_wait(bar_addr(sb, B_SCAL), 0, abort_flag)) {
         *abort_flag = 1;
         report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+      }
+      if (p.raw) {
+        // ---- raw inputs: 1/|q_t|, 1/|k_t| from the landed tiles while the first MMA
+        // runs.  Thread -> tile row etid / 2 (Q rows, then K rows) and one of its two
+        // 128-byte segments (the swizzled order within a segment does not matter to
+        // a sum of squares).  The norms are folded into the per-token scalars, not
+        // into the bf16 operand tiles: P and A gain 1/|q_t| 1/|k_s| and
+        // 1/|k_t| 1/|k_s|, T' gains 1/|k_s|, and the record's e^{G_t} and
+        // e^{G_C - G_t} gain 1/|q_t| and 1/|k_t| for the state pass.
+        if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QKF), 0, etid, abort_flag, p.status)) break;
+        const int rr = etid >> 1, t = rr & 63;
+        const unsigned char *seg = smem + OFF_QK + (rr >> 6) * 8192 + (etid & 1) * 16384 + t * 128;
+        float ss = 0.f;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = *reinterpret_cast<const uint4 *>(seg + 16 * c);
+          const uint32_t wd[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float lo = __uint_as_float(wd[i] << 16), hi = __uint_as_float(wd[i] & 0xffff0000u);
+            ss = fmaf(lo, lo, fmaf(hi, hi, ss));
+          }
+        }
+        ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+        if ((etid & 1) == 0) {
+          const float r = inv_norm(ss);
+          float *scw = reinterpret_cast<float *>(smem + OFF_SCAL);
+          float *rs = reinterpret_cast<float *>(rec + tp::REC_SC);
+          scw[256 + rr] = r;  // 1/|q_t| at [256 + t], 1/|k_t| at [320 + t]
+          rs[rr] = sc[64 + rr] * r;  // e^{G_t} / |q_t|, then e^{G_C - G_t} / |k_t|
+        }
       }
       if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QK), 0, etid, abort_flag, p.status)) break;
       // ---- Q K^T -> P (record, hi/lo), K K^T -> A (fp32, shared)
@@ -265,21 +306,21 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_wait_ld();
         if (row < 64) {
           const int t = row;
-          const float Gt = G2[t];
+          const float Gt = G2[t], rq = rqn[t];
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             float pv[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int si = 32 * half + 16 * qh + 8 * q + e;
-              pv[e] = (si <= t && t < Lc) ? exp2f(Gt - G2[si]) * v[8 * q + e] : 0.f;
+              pv[e] = (si <= t && t < Lc) ? exp2f(Gt - G2[si]) * v[8 * q + e] * (rq * rkn[si]) : 0.f;
             }
             const uint32_t off = sw128_off(t, 4 * half + 2 * qh + q);
             st_split8(rec + tp::REC_PH + off, rec + tp::REC_PL + off, pv);
           }
         } else {
           const int t = row - 64;
-          const float Gt = G2[t], bt = bet[t];
+          const float Gt = G2[t], bt = bet[t], rk = rkn[t];
           float *arow = A + t * AST + 32 * half + 16 * qh;
 #pragma unroll
           for (int x = 0; x < 16; x += 4) {
@@ -287,7 +328,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int si = 32 * half + 16 * qh + x + e;
-              a[e] = (si < t && t < Lc) ? bt * exp2f(Gt - G2[si]) * v[x + e] : 0.f;
+              a[e] = (si < t && t < Lc) ? bt * exp2f(Gt - G2[si]) * v[x + e] * (rk * rkn[si]) : 0.f;
             }
             *reinterpret_cast<float4 *>(arow + x) = make_float4(a[0], a[1], a[2], a[3]);
           }
@@ -304,7 +345,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         for (int e = 0; e < 16; ++e) {
           const float m = (sbeg + e <= t) ? Tm[t * AST + sbeg + e] : 0.f;
           tq[e] = m * bet[sbeg + e];
-          tp_[e] = tq[e] * gam[sbeg + e];
+          tp_[e] = tq[e] * (gam[sbeg + e] * rkn[sbeg + e]);
         }
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -350,10 +391,10 @@ size_t wy_prep_smem_bytes() { return wy::SMEM_BYTES; }
 
 cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
                            const float *g, const float *beta, const int32_t *cu, int T, int Hqk,
-                           int Hv, int round, int rc, const void *workspace,
+                           int Hv, int round, int rc, int raw, const void *workspace,
                            const tp::Layout &L, unsigned char *rec, cudaStream_t stream) {
   wy::Params prm;
-  prm.g = g; prm.beta = beta; prm.cu = cu; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv;
+  prm.g = g; prm.beta = beta; prm.cu = cu; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.raw = raw;
   prm.round = round; prm.rc = rc;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

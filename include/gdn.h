@@ -70,6 +70,20 @@ extern "C" {
 #define GDN_DTYPE_BF16 0
 #define GDN_DTYPE_FP32 1
 
+/* Form of the per-token inputs (input_form).
+ *   GDN_INPUT_PREPARED  q and k L2-normalised by the caller, g = log alpha,
+ *                       beta the write strength.
+ *   GDN_INPUT_RAW       the layer's raw projections: the kernels normalise each
+ *                       (token, query/key head) row of q and k to unit L2 norm
+ *                       (a zero row stays zero), read g as a with
+ *                       alpha = e^{-softplus(a)} = 1 / (1 + e^a), and beta as b
+ *                       with beta = sigmoid(b).  No normalised copy is written.
+ * "Inside Qwen3.8-27B ...", section "Gated DeltaNet Mechanics", calls k the
+ * normalized key projection and makes beta input dependent; softplus and
+ * sigmoid are the plainest maps to a decay and a write strength in (0, 1). */
+#define GDN_INPUT_PREPARED 0
+#define GDN_INPUT_RAW 1
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char *gdn_status_string(int32_t status);
 
@@ -129,6 +143,10 @@ int64_t gdn_prefill_launch_count(int32_t num_seqs, int64_t total_tokens, int32_t
  *                  bf16: the initial state is widened exactly, the arithmetic is
  *                  the same as with fp32 states, and the final state is rounded
  *                  to nearest even once, when it is stored.
+ *   input_form     GDN_INPUT_PREPARED or GDN_INPUT_RAW (see above): with raw
+ *                  inputs q and k are normalised and g, beta mapped inside the
+ *                  kernels (the tensor-core kernels fold 1/|q_t|, 1/|k_t| into
+ *                  their per-token scalars; the bf16 operand tiles stay raw).
  *   initial_state  [num_seqs, Hv, Dv, Dk] state_dtype, or NULL for zeros.
  *   final_state    [num_seqs, Hv, Dv, Dk] state_dtype, or NULL to skip.  May be the
  *                  same pointer as initial_state (updated in place); no other
@@ -159,9 +177,9 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
                     const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
                     int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
                     int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, int32_t o_dtype,
-                    int32_t state_dtype, float scale, const void *initial_state,
-                    void *final_state, void *o, void *workspace, size_t workspace_bytes,
-                    void *stream);
+                    int32_t state_dtype, int32_t input_form, float scale,
+                    const void *initial_state, void *final_state, void *o, void *workspace,
+                    size_t workspace_bytes, void *stream);
 
 /*
  * Prefill for callers that cannot allocate device memory.  (The pages have no
@@ -175,8 +193,8 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
  * array of the library (every GPU that loads the library holds it until the
  * process exits), and calls no cudaMalloc, cudaFree or allocating routine.
  *
- * Arguments are those of gdn_prefill without the workspace and with fp32 states
- * (no state_dtype), plus
+ * Arguments are those of gdn_prefill without the workspace, with fp32 states
+ * and prepared inputs (no state_dtype, no input_form), plus
  *   device_status  optional device int32 (caller's memory, NULL to discard) that
  *                  receives this call's device-detected status (GDN_OK,
  *                  GDN_ERR_BAD_SEQLENS or GDN_ERR_DEVICE_TIMEOUT) in stream order.
@@ -250,6 +268,8 @@ int32_t gdn_decode_step(const void *q, const void *k, const void *v, const float
  *               2.4T MoE, and the VRAM Math", section "The architecture detail
  *               that matters for VRAM"; bf16 at 48 layers x 48 heads x 128 x 128
  *               is 72 MiB.
+ *   input_form  GDN_INPUT_PREPARED or GDN_INPUT_RAW (q, k normalised and g,
+ *               beta mapped inside the kernel; see above).
  *   device_status  optional device int32 (caller's memory, NULL to discard): a
  *               slot index >= num_slots (or a negative dst_slot for a real
  *               sequence) is recorded as GDN_ERR_INVALID_ARG there (first error
@@ -264,8 +284,8 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
                           const int32_t *src_slot, const int32_t *dst_slot, int32_t num_slots,
                           void *o, int32_t batch, int32_t tokens, int32_t num_qk_heads,
                           int32_t num_v_heads, int32_t head_dim_k, int32_t head_dim_v,
-                          int32_t dtype, int32_t o_dtype, int32_t state_dtype, float scale,
-                          int32_t *device_status, void *stream);
+                          int32_t dtype, int32_t o_dtype, int32_t state_dtype,
+                          int32_t input_form, float scale, int32_t *device_status, void *stream);
 
 /*
  * 1 if gdn_prefill with these sizes and dtype runs the tensor-core (tcgen05)

@@ -76,13 +76,14 @@ def test_launch_count(lib):
 def test_decode_tokens_validation(lib):
     """Host-side rejections of gdn_decode_tokens (nothing is launched)."""
     vp = ctypes.c_void_p(256)
-    args = dict(batch=2, tokens=4, Hqk=16, Hv=48, Dk=128, Dv=128, dtype=0, o_dtype=1, s_dtype=1)
+    args = dict(batch=2, tokens=4, Hqk=16, Hv=48, Dk=128, Dv=128, dtype=0, o_dtype=1, s_dtype=1,
+                form=0)
 
     def call(**kw):
         a = {**args, **kw}
         return lib.gdn_decode_tokens(vp, vp, vp, vp, vp, vp, vp, None, None, 4, vp, a["batch"],
                                      a["tokens"], a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"],
-                                     a["o_dtype"], a["s_dtype"], 1.0, None, None)
+                                     a["o_dtype"], a["s_dtype"], a["form"], 1.0, None, None)
 
     assert call(tokens=17) == api.GDN_ERR_UNSUPPORTED      # more than 16 tokens
     assert call(Dk=96) == api.GDN_ERR_UNSUPPORTED
@@ -92,6 +93,8 @@ def test_decode_tokens_validation(lib):
     assert call(batch=5) == api.GDN_ERR_INVALID_ARG          # no slot map: needs batch <= slots
     assert call(s_dtype=2) == api.GDN_ERR_INVALID_ARG        # state dtype neither bf16 nor fp32
     assert call(s_dtype=0, batch=0) == api.GDN_OK            # bf16 states accepted
+    assert call(form=5) == api.GDN_ERR_INVALID_ARG           # input form neither prepared nor raw
+    assert call(form=1, batch=0) == api.GDN_OK
 
 
 def test_workspace_size(lib):
@@ -103,12 +106,12 @@ def test_workspace_size(lib):
 
 def _prefill(lib, **kw):
     a = dict(q=1 << 12, k=1 << 12, v=1 << 12, g=1 << 12, beta=1 << 12, cu=1 << 12, N=1, T=16,
-             Hqk=2, Hv=6, Dk=64, Dv=64, dtype=0, odt=1, sdt=1, scale=1.0, s0=None, sf=None,
-             o=1 << 12, ws=1 << 12, wsb=256)
+             Hqk=2, Hv=6, Dk=64, Dv=64, dtype=0, odt=1, sdt=1, form=0, scale=1.0, s0=None,
+             sf=None, o=1 << 12, ws=1 << 12, wsb=256)
     a.update(kw)
     return lib.gdn_prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], a["cu"], a["N"], a["T"],
                            a["Hqk"], a["Hv"], a["Dk"], a["Dv"], a["dtype"], a["odt"], a["sdt"],
-                           a["scale"], a["s0"], a["sf"], a["o"], a["ws"], a["wsb"], None)
+                           a["form"], a["scale"], a["s0"], a["sf"], a["o"], a["ws"], a["wsb"], None)
 
 
 def test_prefill_validation(lib):
@@ -122,6 +125,7 @@ def test_prefill_validation(lib):
     assert _prefill(lib, dtype=3) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, odt=2) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, sdt=2) == api.GDN_ERR_INVALID_ARG             # state dtype
+    assert _prefill(lib, form=2) == api.GDN_ERR_INVALID_ARG            # input form
     assert _prefill(lib, T=-1) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, N=-1) == api.GDN_ERR_INVALID_ARG
     assert _prefill(lib, Dk=96) == api.GDN_ERR_UNSUPPORTED

@@ -55,6 +55,9 @@ def _bind(lib):
     lib.gdn_oracle_round_bf16.argtypes = [d, ctypes.c_int64]
     lib.gdn_oracle_prologue.restype = ci
     lib.gdn_oracle_prologue.argtypes = [d, d, d, d, ctypes.c_int64, ci, ci, ci]
+    lib.gdn_oracle_backward.restype = ci
+    lib.gdn_oracle_backward.argtypes = [d, d, d, d, d, i64, ci, ci, ci, ci, ci, cd, d, d, d,
+                                        d, d, d, d, d, d]
     return lib
 
 
@@ -180,3 +183,33 @@ def decode_step(q, k, v, g, beta, state, scale=1.0, num_threads=0, state_at_rest
     if state_at_rest == "bf16":
         S = round_bf16(S, lib)
     return o, S
+
+
+def backward(q, k, v, g, beta, d_o, cu_seqlens=None, initial_state=None, d_final_state=None,
+             scale=1.0, lib=None):
+    """Gradients of L = <d_o, o> + <d_final_state, S_final> with respect to q,
+    k, v, g, beta and the initial state, in fp64, token by token (small inputs:
+    every state of a sequence is kept).  Shapes as for prefill; d_o [T, Hv, Dv].
+    Returns (dq, dk, dv, dg, dbeta, d_initial_state)."""
+    lib = lib or load()
+    q, k, v, g, beta, d_o = (_f64(t) for t in (q, k, v, g, beta, d_o))
+    T, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    if cu_seqlens is None:
+        cu = np.array([0, T], dtype=np.int64)
+    else:
+        if hasattr(cu_seqlens, "detach"):
+            cu_seqlens = cu_seqlens.detach().cpu().numpy()
+        cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    N = cu.shape[0] - 1
+    s0, dsf = _f64(initial_state), _f64(d_final_state)
+    dq = np.zeros_like(q); dk = np.zeros_like(k); dv = np.zeros_like(v)
+    dg = np.zeros_like(g); db = np.zeros_like(beta)
+    ds0 = np.zeros((N, Hv, Dv, Dk))
+    rc = lib.gdn_oracle_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta),
+                                 cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), N, Hqk, Hv, Dk,
+                                 Dv, float(scale), _ptr(s0), _ptr(d_o), _ptr(dsf), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), _ptr(dg), _ptr(db), _ptr(ds0))
+    if rc != 0:
+        raise ValueError(f"gdn_oracle_backward failed with code {rc}")
+    return dq, dk, dv, dg, db, ds0

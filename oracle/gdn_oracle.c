@@ -390,3 +390,119 @@ int gdn_oracle_prologue(double *q, double *k, double *g, double *beta, int64_t T
     }
     return ORACLE_OK;
 }
+
+/*
+ * Backward pass (reverse-mode derivative) of the recurrence, token by token.
+ * The forward definition is the one above; the loss L is linear in the
+ * outputs it is given gradients for: dO = dL/do [T, Hv, Dv] and, optionally,
+ * dSfin = dL/dS_final [N, Hv, Dv, Dk].  Writing G for dL/dS_t (everything that
+ * depends on S_t), u = S_{t-1} k_t, w = v_t - alpha_t u, so that
+ * S_t = alpha_t S_{t-1} + beta_t w k_t^T and o_t = scale S_t q_t, the chain
+ * rule gives, for t from the last token down to the first:
+ *   G      += scale dO_t q_t^T
+ *   dq_t    = scale S_t^T dO_t
+ *   dv_t    = beta_t G k_t
+ *   dbeta_t = w . (G k_t)
+ *   dg_t    = alpha_t ( <G, S_{t-1}> - beta_t (G k_t) . u )       (alpha = e^g)
+ *   dk_t    = beta_t G^T w - alpha_t beta_t S_{t-1}^T (G k_t)
+ *   G      <- alpha_t (G - beta_t (G k_t) k_t^T)                  (= dL/dS_{t-1})
+ * and dS0 = G at the start of the sequence.  dq and dk of a query/key head
+ * sum over the value heads that read it.  All states S_0 .. S_L of a unit are
+ * kept (fp64), so this is for small inputs.  Outputs dq, dk [T, Hqk, Dk],
+ * dv [T, Hv, Dv], dg, dbeta [T, Hv], dS0 [N, Hv, Dv, Dk] (may be NULL).
+ * Returns 0, 1 for a bad argument, 2 when memory ran out.
+ */
+int gdn_oracle_backward(const double *q, const double *k, const double *v, const double *g,
+                        const double *beta, const int64_t *cu_seqlens, int num_seqs, int Hqk,
+                        int Hv, int Dk, int Dv, double scale, const double *initial_state,
+                        const double *dO, const double *dSfin, double *dq, double *dk,
+                        double *dv, double *dg, double *dbeta, double *dS0)
+{
+    if (num_seqs < 0 || Hqk <= 0 || Hv <= 0 || Hv % Hqk || Dk <= 0 || Dv <= 0) return ORACLE_BAD_ARG;
+    const int64_t T = cu_seqlens[num_seqs];
+    const size_t sdim = (size_t)Dv * Dk;
+    memset(dq, 0, sizeof(double) * (size_t)T * Hqk * Dk);
+    memset(dk, 0, sizeof(double) * (size_t)T * Hqk * Dk);
+    int64_t Lmax = 0;
+    for (int n = 0; n < num_seqs; ++n) {
+        const int64_t L = cu_seqlens[n + 1] - cu_seqlens[n];
+        if (L < 0) return ORACLE_BAD_ARG;
+        if (L > Lmax) Lmax = L;
+    }
+    double *states = (double *)malloc(sizeof(double) * sdim * (size_t)(Lmax + 1));
+    double *G = (double *)malloc(sizeof(double) * sdim);
+    double *Gk = (double *)malloc(sizeof(double) * Dv);
+    double *u = (double *)malloc(sizeof(double) * Dv);
+    if (!states || !G || !Gk || !u) {
+        free(states); free(G); free(Gk); free(u);
+        return ORACLE_NO_MEMORY;
+    }
+    for (int n = 0; n < num_seqs; ++n) {
+        const int64_t t0 = cu_seqlens[n], L = cu_seqlens[n + 1] - t0;
+        for (int h = 0; h < Hv; ++h) {
+            const int j = h / (Hv / Hqk);
+            /* forward, keeping S_0 .. S_L */
+            if (initial_state) memcpy(states, initial_state + ((size_t)n * Hv + h) * sdim, sdim * sizeof(double));
+            else memset(states, 0, sdim * sizeof(double));
+            for (int64_t s = 0; s < L; ++s) {
+                const int64_t t = t0 + s;
+                const double alpha = exp(g[t * Hv + h]), b = beta[t * Hv + h];
+                const double *kt = k + ((size_t)t * Hqk + j) * Dk, *vt = v + ((size_t)t * Hv + h) * Dv;
+                const double *Sp = states + (size_t)s * sdim;
+                double *Sn = states + (size_t)(s + 1) * sdim;
+                for (int i = 0; i < Dv; ++i) {
+                    double ui = 0.0;
+                    for (int c = 0; c < Dk; ++c) ui += Sp[(size_t)i * Dk + c] * kt[c];
+                    const double wi = b * (vt[i] - alpha * ui);
+                    for (int c = 0; c < Dk; ++c) Sn[(size_t)i * Dk + c] = alpha * Sp[(size_t)i * Dk + c] + wi * kt[c];
+                }
+            }
+            /* backward */
+            if (dSfin) memcpy(G, dSfin + ((size_t)n * Hv + h) * sdim, sdim * sizeof(double));
+            else memset(G, 0, sdim * sizeof(double));
+            for (int64_t s = L - 1; s >= 0; --s) {
+                const int64_t t = t0 + s;
+                const double alpha = exp(g[t * Hv + h]), b = beta[t * Hv + h];
+                const double *kt = k + ((size_t)t * Hqk + j) * Dk, *qt = q + ((size_t)t * Hqk + j) * Dk;
+                const double *vt = v + ((size_t)t * Hv + h) * Dv, *dOt = dO + ((size_t)t * Hv + h) * Dv;
+                const double *Sp = states + (size_t)s * sdim, *St = states + (size_t)(s + 1) * sdim;
+                double *dqt = dq + ((size_t)t * Hqk + j) * Dk, *dkt = dk + ((size_t)t * Hqk + j) * Dk;
+                /* o_t = scale S_t q_t */
+                for (int i = 0; i < Dv; ++i)
+                    for (int c = 0; c < Dk; ++c) {
+                        G[(size_t)i * Dk + c] += scale * dOt[i] * qt[c];
+                        dqt[c] += scale * St[(size_t)i * Dk + c] * dOt[i];
+                    }
+                double sGS = 0.0, gku = 0.0, wgk = 0.0;
+                for (int i = 0; i < Dv; ++i) {
+                    double gk = 0.0, ui = 0.0;
+                    for (int c = 0; c < Dk; ++c) {
+                        gk += G[(size_t)i * Dk + c] * kt[c];
+                        ui += Sp[(size_t)i * Dk + c] * kt[c];
+                        sGS += G[(size_t)i * Dk + c] * Sp[(size_t)i * Dk + c];
+                    }
+                    Gk[i] = gk;
+                    u[i] = ui;
+                    gku += gk * ui;
+                    wgk += (vt[i] - alpha * ui) * gk;
+                }
+                for (int i = 0; i < Dv; ++i) dv[((size_t)t * Hv + h) * Dv + i] = b * Gk[i];
+                dbeta[t * Hv + h] = wgk;
+                dg[t * Hv + h] = alpha * (sGS - b * gku);
+                for (int c = 0; c < Dk; ++c) {
+                    double acc = 0.0;
+                    for (int i = 0; i < Dv; ++i)
+                        acc += b * G[(size_t)i * Dk + c] * (vt[i] - alpha * u[i]) -
+                               alpha * b * Sp[(size_t)i * Dk + c] * Gk[i];
+                    dkt[c] += acc;
+                }
+                for (int i = 0; i < Dv; ++i)
+                    for (int c = 0; c < Dk; ++c)
+                        G[(size_t)i * Dk + c] = alpha * (G[(size_t)i * Dk + c] - b * Gk[i] * kt[c]);
+            }
+            if (dS0) memcpy(dS0 + ((size_t)n * Hv + h) * sdim, G, sdim * sizeof(double));
+        }
+    }
+    free(states); free(G); free(Gk); free(u);
+    return ORACLE_OK;
+}

@@ -375,9 +375,41 @@ def check_prologue(lib, seed=13):
     _close(kn2, kn, 1e-15, "normalising twice changes nothing (k)")
 
 
+def check_backward_finite_differences(lib, seed=14, h=1e-6):
+    """The backward pass against central finite differences of the forward
+    definition: L = <dO, o> + <dS, S_final> over two packed sequences with GQA,
+    initial states and a scale; every element of q, k, v, g, beta and the
+    initial state is perturbed by +-h."""
+    r = _rng(seed)
+    cu = np.array([0, 2, 5])
+    T, N, Hqk, Hv, Dk, Dv, scale = 5, 2, 1, 2, 3, 2, 0.7
+    x = {"q": r.standard_normal((T, Hqk, Dk)), "k": 0.6 * r.standard_normal((T, Hqk, Dk)),
+         "v": r.standard_normal((T, Hv, Dv)), "g": -np.abs(r.standard_normal((T, Hv))),
+         "beta": r.uniform(0.1, 0.9, (T, Hv)), "s0": 0.5 * r.standard_normal((N, Hv, Dv, Dk))}
+    dO = r.standard_normal((T, Hv, Dv))
+    dS = r.standard_normal((N, Hv, Dv, Dk))
+
+    def loss(a):
+        o, f = oracle.prefill(a["q"], a["k"], a["v"], a["g"], a["beta"], cu_seqlens=cu,
+                              initial_state=a["s0"], scale=scale, lib=lib)
+        return float((o * dO).sum() + (f * dS).sum())
+
+    grads = oracle.backward(x["q"], x["k"], x["v"], x["g"], x["beta"], dO, cu_seqlens=cu,
+                            initial_state=x["s0"], d_final_state=dS, scale=scale, lib=lib)
+    for name, an in zip(("q", "k", "v", "g", "beta", "s0"), grads):
+        num = np.zeros_like(x[name])
+        for idx in np.ndindex(x[name].shape):
+            a = {n: t.copy() for n, t in x.items()}
+            a[name][idx] += h
+            lp = loss(a)
+            a[name][idx] -= 2 * h
+            num[idx] = (lp - loss(a)) / (2 * h)
+        _close(an, num, 1e-7, f"d{name} against finite differences")
+
+
 ALL_CHECKS = [
     check_product_form, check_golden_scalar, check_golden_matrix, check_no_write_no_decay,
     check_exact_writeback, check_reset, check_pure_decay, check_orthonormal_memory, check_scale,
     check_gqa_mapping, check_varlen, check_decode, check_chunked, check_round_bf16,
-    check_state_at_rest_bf16, check_prologue,
+    check_state_at_rest_bf16, check_prologue, check_backward_finite_differences,
 ]

@@ -48,6 +48,14 @@ MUTANTS = [
     ("prologue_q_only", "for (int w = 0; w < 2; ++w) {", "for (int w = 0; w < 1; ++w) {"),
     ("prologue_relu_not_softplus", "g[i] = -(fmax(a, 0.0) + log1p(exp(-fabs(a))));", "g[i] = -(fmax(a, 0.0));"),
     ("prologue_decay_sign", "g[i] = -(fmax(a, 0.0) + log1p(exp(-fabs(a))));", "g[i] = (fmax(a, 0.0) + log1p(exp(-fabs(a))));"),
+    ("bwd_carry_without_decay", "G[(size_t)i * Dk + c] = alpha * (G[(size_t)i * Dk + c] - b * Gk[i] * kt[c]);",
+     "G[(size_t)i * Dk + c] = (G[(size_t)i * Dk + c] - b * Gk[i] * kt[c]);"),
+    ("bwd_dk_sign", "acc += b * G[(size_t)i * Dk + c] * (vt[i] - alpha * u[i]) -",
+     "acc += b * G[(size_t)i * Dk + c] * (vt[i] - alpha * u[i]) +"),
+    ("bwd_dq_from_previous_state", "dqt[c] += scale * St[(size_t)i * Dk + c] * dOt[i];",
+     "dqt[c] += scale * Sp[(size_t)i * Dk + c] * dOt[i];"),
+    ("bwd_dg_not_chained", "dg[t * Hv + h] = alpha * (sGS - b * gku);", "dg[t * Hv + h] = (sGS - b * gku);"),
+    ("bwd_dbeta_without_decay", "wgk += (vt[i] - alpha * ui) * gk;", "wgk += (vt[i] - ui) * gk;"),
     ("prologue_sigmoid_of_minus_b", "beta[i] = b >= 0.0 ? 1.0 / (1.0 + exp(-b)) : exp(b) / (1.0 + exp(b));",
      "beta[i] = b >= 0.0 ? 1.0 / (1.0 + exp(b)) : exp(-b) / (1.0 + exp(-b));"),
 ]

@@ -18,6 +18,9 @@ resident in HBM, L2 flushed between timed steps.  The same line carries:
                the same step from raw projections (normalisation and gates
                folded into the kernels), with the prepared-input time and the
                time with a separate PyTorch prologue for context;
+  prefill_backward
+               the backward pass of the same step (gradients for q, k, v, g,
+               beta and the initial state; CUDA cores, fp32);
   decode_bf16_state, decode_tokens_bf16_state
                the same with the state pool at rest in bf16 (fp32 arithmetic,
                100 MB of state), 1 and 4 tokens per call;
@@ -62,6 +65,7 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=1000)
+    p.add_argument("--no-backward", action="store_true", help="skip the backward-pass leg")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -400,6 +404,9 @@ def run_ours(args, D):
     if not args.no_e2e:
         out["e2e"] = _e2e(args, D, inp, dev, w, ws)
 
+    if not args.no_backward:
+        out["prefill_backward"] = _backward(args, D, dev, x, T, w, peaks)
+
     if not args.no_decode:
         out["decode"] = _decode(args, D, dev, peaks, peak_src)
         out["decode_tokens"] = _decode_tokens(args, D, dev, peaks, peak_src)
@@ -523,6 +530,63 @@ def _prefill_raw(args, D, dev, x, T, w, ws, fin, o, flush, prepared_ms, launches
             "ms_per_step": res["fused"], "prepared_inputs_ms_per_step": prepared_ms,
             "separate_torch_prologue_ms_per_step": res["separate"],
             "l2": "flushed between timed steps", "gpu_launches": args.steps * launches}
+
+
+def _backward(args, D, dev, x, T, w, peaks):
+    """Backward pass of the prefill step (gdn_prefill_backward) on the same
+    workload: d_o and dL/dS_final random fp32, gradients for q, k, v, g, beta
+    and the initial state.  CUDA cores, fp32: the roofline is the fp32 FMA
+    rate."""
+    import torch
+
+    from gated_deltanet_recurrence_rule_b200 import api
+
+    gen = torch.Generator(device=dev).manual_seed(12)
+    d_o = torch.randn((T, w.Hv, w.D), generator=gen, device=dev)
+    d_sf = torch.randn((1, w.Hv, w.D, w.D), generator=gen, device=dev) * 0.1
+    ws = torch.zeros(api.prefill_backward_workspace_size(1, T, w.Hqk, w.Hv, w.D, w.D),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        return api.prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d_o,
+                                    cu_seqlens=x["cu_seqlens"], d_final_state=d_sf, workspace=ws)
+
+    steps = max(1, min(args.steps, 3))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    ms = D.max(e0.elapsed_time(e1), dev) / steps
+    status = api.get_device_status(ws)
+    if status != api.GDN_OK:
+        raise RuntimeError(f"device status after the backward leg: {api.status_string(status)}")
+    # Algorithmic fp32 work per token and value head (an FMA counts 2): the
+    # forward state S_t (u = S k, S update: 4 D^2) and the backward terms
+    # (G += dO q^T, S_t^T dO, G k, <G, S>, G^T w, S^T G k, G update: 14 D^2).
+    # The kernel's recomputation of the states from checkpoints is not counted.
+    flop = 18 * w.D * w.D * w.Hv * T
+    fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    achieved = flop / (ms / 1e3) / 1e12
+    return {"value": D.world * T / (ms / 1e3) / 1e6, "unit": "Mtok/s",
+            "workload": f"backward of prefill8k: T={T} Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16 inputs, "
+                        "fp32 d_o and dL/dS_final, zero initial state",
+            "ms_per_step": ms,
+            "roofline": {"bound": "alu", "kernel": "backward_kernel (+ group_sum_kernel x 2)",
+                         "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s",
+                         "frac": achieved / fp32_peak,
+                         "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
+                         "algorithmic": f"18 D^2 flop per token and value head = {flop} flop",
+                         "traffic": None},
+            "gpu_launches": 3 * steps}
 
 
 def _decode(args, D, dev, peaks, peak_src):

@@ -73,6 +73,12 @@ def load():
         lib.gdn_decode_tokens.restype = i32
         lib.gdn_decode_tokens.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i32, vp, i32, i32, i32,
                                           i32, i32, i32, i32, i32, i32, i32, f32, vp, vp]
+        lib.gdn_prefill_backward_workspace_size.restype = sz
+        lib.gdn_prefill_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
+        lib.gdn_prefill_backward.restype = i32
+        lib.gdn_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
+                                             i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
+                                             vp]
         lib.gdn_prefill_uses_tensor_cores.restype = i32
         lib.gdn_prefill_uses_tensor_cores.argtypes = [i32, i32, i32, i32, i32]
         lib.gdn_get_device_status.restype = i32
@@ -276,6 +282,57 @@ def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst
                                float(scale), _ptr(device_status), _stream(dev))
     _check(st, "gdn_decode_tokens")
     return o
+
+
+def prefill_backward(q, k, v, g, beta, d_o, cu_seqlens=None, initial_state=None,
+                     d_final_state=None, scale=1.0, workspace=None, want_d_initial_state=True):
+    """Gradients of the prefill (fp32 states, prepared inputs) given d_o
+    [T, Hv, Dv] fp32 and optionally d_final_state [N, Hv, Dv, Dk] fp32.
+    Returns (dq, dk, dv, dg, dbeta, d_initial_state or None), all fp32."""
+    lib = load()
+    if not q.is_cuda:
+        raise ValueError("prefill_backward runs on a CUDA device only (q is on the CPU)")
+    dev = q.device
+    T, Hqk, Dk = q.shape
+    Hv, Dv = v.shape[1], v.shape[2]
+    dt = q.dtype
+    if dt not in _DTYPE_CODE:
+        raise ValueError(f"unsupported dtype {dt}")
+    _require(q, "q", dev, dt)
+    _require(k, "k", dev, dt, (T, Hqk, Dk))
+    _require(v, "v", dev, dt, (T, Hv, Dv))
+    _require(g, "g", dev, torch.float32, (T, Hv))
+    _require(beta, "beta", dev, torch.float32, (T, Hv))
+    _require(d_o, "d_o", dev, torch.float32, (T, Hv, Dv))
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=dev)
+    _require(cu_seqlens, "cu_seqlens", dev, torch.int32)
+    N = cu_seqlens.shape[0] - 1
+    sshape = (N, Hv, Dv, Dk)
+    for name, t in (("initial_state", initial_state), ("d_final_state", d_final_state)):
+        if t is not None:
+            _require(t, name, dev, torch.float32, sshape)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk = torch.empty((T, Hqk, Dk), **f32), torch.empty((T, Hqk, Dk), **f32)
+    dv = torch.empty((T, Hv, Dv), **f32)
+    dg, db = torch.empty((T, Hv), **f32), torch.empty((T, Hv), **f32)
+    ds0 = torch.empty(sshape, **f32) if want_d_initial_state else None
+    need = lib.gdn_prefill_backward_workspace_size(N, T, Hqk, Hv, Dk, Dv)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
+    _require(workspace, "workspace", dev, torch.uint8)
+    st = lib.gdn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+                                  N, T, Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], float(scale),
+                                  _ptr(initial_state), _ptr(d_o), _ptr(d_final_state), _ptr(dq),
+                                  _ptr(dk), _ptr(dv), _ptr(dg), _ptr(db), _ptr(ds0),
+                                  _ptr(workspace), workspace.numel(), _stream(dev))
+    _check(st, "gdn_prefill_backward")
+    return dq, dk, dv, dg, db, ds0
+
+
+def prefill_backward_workspace_size(N, T, Hqk, Hv, Dk, Dv) -> int:
+    """Workspace bytes gdn_prefill_backward needs (0 for invalid sizes)."""
+    return int(load().gdn_prefill_backward_workspace_size(N, T, Hqk, Hv, Dk, Dv))
 
 
 def prefill_uses_tensor_cores(Hqk, Hv, Dk, Dv, dtype=torch.bfloat16) -> bool:

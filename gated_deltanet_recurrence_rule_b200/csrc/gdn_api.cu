@@ -41,6 +41,13 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
                                     int Hqk, int Hv, int o_dtype, int state_dtype, int input_form,
                                     float scale, const void *s0, void *sfin, void *o,
                                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
+size_t backward_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv);
+cudaError_t launch_backward(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
+                            int Hv, int Dk, int Dv, int dtype, float scale, const float *s0,
+                            const float *dO, const float *dSfin, float *dq, float *dk, float *dv,
+                            float *dg, float *dbeta, float *ds0, void *workspace,
+                            cudaStream_t stream);
 }  // namespace gdn
 
 namespace {
@@ -229,6 +236,51 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
       q, k, v, g, beta, state_in, state_out, src_slot, dst_slot, num_slots, o, batch, tokens,
       num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype, o_dtype, state_dtype, input_form,
       scale, device_status, static_cast<cudaStream_t>(stream)));
+}
+
+size_t gdn_prefill_backward_workspace_size(int32_t num_seqs, int64_t total_tokens,
+                                           int32_t num_qk_heads, int32_t num_v_heads,
+                                           int32_t head_dim_k, int32_t head_dim_v) {
+  if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return 0;
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, GDN_DTYPE_FP32)) return 0;
+  if (!dims_supported(head_dim_k, head_dim_v)) return 0;
+  return gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads, num_v_heads,
+                                       head_dim_k, head_dim_v);
+}
+
+int32_t gdn_prefill_backward(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
+                             int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
+                             int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, float scale,
+                             const float *initial_state, const float *d_o,
+                             const float *d_final_state, float *dq, float *dk, float *dv,
+                             float *dg, float *dbeta, float *d_initial_state, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+  if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
+  if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if ((int64_t)num_seqs * num_v_heads > INT32_MAX) return GDN_ERR_UNSUPPORTED;
+  if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
+  if (total_tokens > 0) {
+    if (!q || !k || !v || !g || !beta || !d_o || !dq || !dk || !dv || !dg || !dbeta)
+      return GDN_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(d_o, 16) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 4) || !aligned(g, 4) ||
+        !aligned(beta, 4) || !aligned(dg, 4) || !aligned(dbeta, 4))
+      return GDN_ERR_INVALID_ARG;
+  }
+  if ((initial_state && !aligned(initial_state, 16)) || (d_final_state && !aligned(d_final_state, 16)) ||
+      (d_initial_state && !aligned(d_initial_state, 16)))
+    return GDN_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) ||
+      workspace_bytes < gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads,
+                                                      num_v_heads, head_dim_k, head_dim_v))
+    return GDN_ERR_WORKSPACE;
+  return cuda_status(gdn::launch_backward(
+      q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_qk_heads, num_v_heads, head_dim_k,
+      head_dim_v, dtype, scale, initial_state, d_o, d_final_state, dq, dk, dv, dg, dbeta,
+      d_initial_state, workspace, static_cast<cudaStream_t>(stream)));
 }
 
 int32_t gdn_prefill_uses_tensor_cores(int32_t num_qk_heads, int32_t num_v_heads,

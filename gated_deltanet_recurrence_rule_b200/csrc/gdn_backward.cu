@@ -1,0 +1,421 @@
+// gdn_backward.cu -- backward pass of the gated delta rule (training), on CUDA
+// cores in fp32.
+//
+// The forward rule is the one of "Inside Qwen3.8-27B: Hybrid DeltaNet
+// Architecture, 256k Context, and 24GB Local Serving", section "Gated DeltaNet
+// Mechanics" (the page's note says the block form serves training too); per
+// (sequence, value head), with u = S_{t-1} k_t and w = v_t - alpha_t u,
+//   S_t = alpha_t S_{t-1} + beta_t w k_t^T,   o_t = scale S_t q_t.
+// Given dO = dL/do and dS = dL/dS_final, the chain rule runs backwards over
+// the tokens with G = dL/dS_t:
+//   G      += scale dO_t q_t^T
+//   dq_t    = scale S_t^T dO_t
+//   dv_t    = beta_t G k_t
+//   dbeta_t = w . (G k_t)
+//   dg_t    = alpha_t (<G, S_{t-1}> - beta_t (G k_t) . u)
+//   dk_t    = beta_t G^T w - alpha_t beta_t S_{t-1}^T (G k_t)
+//   G      <- alpha_t (G - beta_t (G k_t) k_t^T)
+// and dS0 = G at the start of the sequence.
+//
+// One CTA per (sequence, value head), 4 lanes per state row (4 Dv threads),
+// each lane holding Dk/4 columns of S and of G in registers:
+//   pass 1  forward from S0, storing a checkpoint of S every C tokens;
+//   pass 2  chunks last to first: the chunk's states S_{t-1} are recomputed
+//           from its checkpoint into a per-CTA scratch, then walked backwards.
+// S^T x products (dq, dk) are column sums over all rows: a recursive-halving
+// shuffle over the 8 rows of a warp, then a sum over warps in shared memory
+// (double-buffered, one block barrier per token).  dq and dk are written per
+// value head and summed over each query/key head's group by a second kernel,
+// so the result does not depend on scheduling.
+#include <algorithm>
+
+#include "gdn_common.cuh"
+
+namespace gdn {
+namespace bwd {
+
+constexpr int C = 16;  // tokens per checkpoint chunk
+
+template <int DK, int DV>
+struct Cfg {
+  static constexpr int THREADS = 4 * DV;  // 4 lanes per state row
+  static constexpr int CPL = DK / 4;      // columns per lane: 16 m + 4 r4 + (0..3)
+  static constexpr int NV4 = CPL / 4;
+  static constexpr int NW = THREADS / 32;
+  static constexpr int KEEP = CPL / 8;    // columns a lane keeps after the 8-row halving
+  // shared memory (floats)
+  static constexpr int S_Q = 0, S_K = S_Q + C * DK, S_V = S_K + C * DK, S_DO = S_V + C * DV;
+  static constexpr int S_A = S_DO + C * DV, S_B = S_A + C;
+  static constexpr int S_RED = S_B + C;                  // [2 buffers][2 vectors][NW][DK]
+  static constexpr int S_RS = S_RED + 2 * 2 * NW * DK;   // [2 buffers][3][NW]
+  static constexpr int S_BASE = S_RS + 2 * 3 * NW;       // chunk base (int)
+  static constexpr int FLOATS = S_BASE + 4;
+  static constexpr size_t SMEM = FLOATS * sizeof(float);
+};
+
+struct Params {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  const int32_t *cu;
+  int N, T, Hqk, Hv;
+  float scale;
+  const float *s0, *dO, *dSfin;
+  float *dq, *dk;  // [T, Hv, DK]: per value head (the outputs themselves when Hv == Hqk)
+  float *dv, *dg, *dbeta, *ds0;
+  float *ckpt;     // [(ceil(T / C) + N) * Hv][64 KiB states]
+  float *scratch;  // [N * Hv][C states]
+  int32_t *status;
+};
+
+// Column c = 16 m + 4 r4 + q of this lane's row, element e = 4 m + q.
+// Sum v over the 8 rows a warp holds (lane bits 2..4) by recursive halving:
+// at each level a lane keeps half of its elements and adds the partner's copy
+// of them, so afterwards it holds KEEP = CPL / 8 consecutive elements (from
+// keep_e0) summed over the 8 rows, with 7 CPL / 8 shuffles instead of 3 CPL.
+template <int CPL>
+__device__ __forceinline__ void halve8(float (&v)[CPL], int lane) {
+  constexpr int H1 = CPL / 2, H2 = CPL / 4, H3 = CPL / 8;
+  {
+    const bool up = lane & 16;
+#pragma unroll
+    for (int e = 0; e < H1; ++e) {
+      const float mine = up ? v[H1 + e] : v[e], other = up ? v[e] : v[H1 + e];
+      v[e] = mine + __shfl_xor_sync(0xffffffffu, other, 16);
+    }
+  }
+  {
+    const bool up = lane & 8;
+#pragma unroll
+    for (int e = 0; e < H2; ++e) {
+      const float mine = up ? v[H2 + e] : v[e], other = up ? v[e] : v[H2 + e];
+      v[e] = mine + __shfl_xor_sync(0xffffffffu, other, 8);
+    }
+  }
+  {
+    const bool up = lane & 4;
+#pragma unroll
+    for (int e = 0; e < H3; ++e) {
+      const float mine = up ? v[H3 + e] : v[e], other = up ? v[e] : v[H3 + e];
+      v[e] = mine + __shfl_xor_sync(0xffffffffu, other, 4);
+    }
+  }
+}
+// First element index (4 m + q) a lane keeps after halve8.
+template <int CPL>
+__device__ __forceinline__ int keep_e0(int lane) {
+  return (CPL / 2) * ((lane >> 4) & 1) + (CPL / 4) * ((lane >> 3) & 1) + (CPL / 8) * ((lane >> 2) & 1);
+}
+
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(4 * DV, 1)
+backward_kernel(const Params p) {
+  using CF = Cfg<DK, DV>;
+  constexpr int CPL = CF::CPL, NV4 = CF::NV4, NW = CF::NW, KEEP = CF::KEEP;
+  extern __shared__ __align__(16) float sm[];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int row = tid >> 2, r4 = tid & 3;
+  const int n = blockIdx.x / p.Hv, h = blockIdx.x - n * p.Hv;
+  const int j = h / (p.Hv / p.Hqk);
+
+  const int c0 = p.cu[n], c1 = p.cu[n + 1];
+  if (c0 < 0 || c1 < c0 || c1 > p.T || (n == 0 && c0 != 0) || (n == p.N - 1 && c1 != p.T)) {
+    if (tid == 0) report_status(p.status, GDN_ERR_BAD_SEQLENS);
+    return;
+  }
+  const int L = c1 - c0, nck = (L + C - 1) / C;
+  if (tid == 0) {  // first checkpoint of this sequence: chunks of the earlier sequences
+    int base = 0;
+    for (int m = 0; m < n; ++m) base += (p.cu[m + 1] - p.cu[m] + C - 1) / C;
+    reinterpret_cast<int *>(sm + CF::S_BASE)[0] = base;
+  }
+  __syncthreads();
+  const int cbase = reinterpret_cast<const int *>(sm + CF::S_BASE)[0];
+  const size_t hs = (size_t)DV * DK;
+  const size_t srow = ((size_t)n * p.Hv + h) * hs + (size_t)row * DK;
+  auto ck = [&](int c) {  // this thread's float4s of checkpoint c, laid out [NV4][THREADS]
+    return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(cbase + c) * p.Hv + h) * hs) + tid;
+  };
+  float4 *scr = reinterpret_cast<float4 *>(p.scratch + (size_t)blockIdx.x * C * hs) + tid;
+
+  float *sq = sm + CF::S_Q, *sk = sm + CF::S_K, *sv = sm + CF::S_V, *sdo = sm + CF::S_DO;
+  float *sa = sm + CF::S_A, *sb = sm + CF::S_B;
+  // stage chunk c: k (and q, dO when `full`), v, alpha, beta as fp32
+  auto stage = [&](int c, bool full) {
+    const int t0 = c0 + c * C, cnt = min(C, c1 - t0);
+    __syncthreads();  // the previous chunk's tokens are no longer read
+    for (int x = tid; x < cnt * DK; x += CF::THREADS) {
+      const int t = x / DK, d = x - t * DK;
+      const size_t off = ((size_t)(t0 + t) * p.Hqk + j) * DK + d;
+      sk[x] = to_f32(static_cast<const T *>(p.k)[off]);
+      if (full) sq[x] = to_f32(static_cast<const T *>(p.q)[off]);
+    }
+    for (int x = tid; x < cnt * DV; x += CF::THREADS) {
+      const int t = x / DV, d = x - t * DV;
+      const size_t off = ((size_t)(t0 + t) * p.Hv + h) * DV + d;
+      sv[x] = to_f32(static_cast<const T *>(p.v)[off]);
+      if (full) sdo[x] = p.dO[off];
+    }
+    if (tid < cnt) {
+      sa[tid] = expf(p.g[(size_t)(t0 + tid) * p.Hv + h]);
+      sb[tid] = p.beta[(size_t)(t0 + tid) * p.Hv + h];
+    }
+    __syncthreads();
+    return cnt;
+  };
+  auto rowdot = [&](const float (&x)[CPL], const float *vec) {  // (x . vec) over the row
+    float a = 0.f;
+#pragma unroll
+    for (int m = 0; m < NV4; ++m) {
+      const float4 y = *reinterpret_cast<const float4 *>(vec + 16 * m + 4 * r4);
+      a = fmaf(x[4 * m], y.x, a); a = fmaf(x[4 * m + 1], y.y, a);
+      a = fmaf(x[4 * m + 2], y.z, a); a = fmaf(x[4 * m + 3], y.w, a);
+    }
+    a += __shfl_xor_sync(0xffffffffu, a, 1);
+    a += __shfl_xor_sync(0xffffffffu, a, 2);
+    return a;
+  };
+  auto step = [&](float (&S)[CPL], int t) {  // S <- S_t from S_{t-1}
+    const float *kt = sk + t * DK;
+    const float u = rowdot(S, kt);
+    const float w = sb[t] * (sv[t * DV + row] - sa[t] * u);
+#pragma unroll
+    for (int m = 0; m < NV4; ++m) {
+      const float4 y = *reinterpret_cast<const float4 *>(kt + 16 * m + 4 * r4);
+      S[4 * m] = fmaf(sa[t], S[4 * m], w * y.x); S[4 * m + 1] = fmaf(sa[t], S[4 * m + 1], w * y.y);
+      S[4 * m + 2] = fmaf(sa[t], S[4 * m + 2], w * y.z); S[4 * m + 3] = fmaf(sa[t], S[4 * m + 3], w * y.w);
+    }
+  };
+
+  // ---- pass 1: forward with a checkpoint every C tokens
+  float S[CPL];
+#pragma unroll
+  for (int m = 0; m < NV4; ++m) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p.s0) x = *reinterpret_cast<const float4 *>(p.s0 + srow + 16 * m + 4 * r4);
+    S[4 * m] = x.x; S[4 * m + 1] = x.y; S[4 * m + 2] = x.z; S[4 * m + 3] = x.w;
+  }
+  for (int c = 0; c < nck; ++c) {
+    float4 *dst = ck(c);
+#pragma unroll
+    for (int m = 0; m < NV4; ++m)
+      dst[m * CF::THREADS] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
+    const int cnt = stage(c, false);
+    for (int t = 0; t < cnt; ++t) step(S, t);
+  }
+
+  // ---- pass 2: backwards
+  float G[CPL];
+#pragma unroll
+  for (int m = 0; m < NV4; ++m) {
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (p.dSfin) x = *reinterpret_cast<const float4 *>(p.dSfin + srow + 16 * m + 4 * r4);
+    G[4 * m] = x.x; G[4 * m + 1] = x.y; G[4 * m + 2] = x.z; G[4 * m + 3] = x.w;
+  }
+  float *red = sm + CF::S_RED, *rs = sm + CF::S_RS;
+  int parity = 0;
+  for (int c = nck - 1; c >= 0; --c) {
+    const int cnt = stage(c, true);
+    {  // S_{t-1} of every token of the chunk into the scratch
+      const float4 *src = ck(c);
+#pragma unroll
+      for (int m = 0; m < NV4; ++m) {
+        const float4 x = src[m * CF::THREADS];
+        S[4 * m] = x.x; S[4 * m + 1] = x.y; S[4 * m + 2] = x.z; S[4 * m + 3] = x.w;
+      }
+      for (int t = 0; t < cnt; ++t) {
+#pragma unroll
+        for (int m = 0; m < NV4; ++m)
+          scr[(t * NV4 + m) * CF::THREADS] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
+        if (t + 1 < cnt) step(S, t);
+      }
+    }
+    for (int t = cnt - 1; t >= 0; --t) {
+      const size_t tg = (size_t)(c0 + c * C + t);
+      const float alpha = sa[t], bt = sb[t];
+      const float *kt = sk + t * DK, *qt = sq + t * DK;
+      float Sp[CPL];  // S_{t-1}
+#pragma unroll
+      for (int m = 0; m < NV4; ++m) {
+        const float4 x = scr[(t * NV4 + m) * CF::THREADS];
+        Sp[4 * m] = x.x; Sp[4 * m + 1] = x.y; Sp[4 * m + 2] = x.z; Sp[4 * m + 3] = x.w;
+      }
+      const float u = rowdot(Sp, kt);
+      const float w = sv[t * DV + row] - alpha * u;  // v - alpha u (beta applied where used)
+      const float sdO = p.scale * sdo[t * DV + row], bw = bt * w;
+      float *rb = red + parity * 2 * NW * DK;
+      const int e0 = keep_e0<CPL>(lane);
+      float tmp[CPL];
+      // G += scale dO q^T;  dq partial = scale dO_i S_t[i, :],  S_t = alpha S_{t-1} + beta w k^T
+#pragma unroll
+      for (int m = 0; m < NV4; ++m) {
+        const float4 a = *reinterpret_cast<const float4 *>(kt + 16 * m + 4 * r4);
+        const float4 b = *reinterpret_cast<const float4 *>(qt + 16 * m + 4 * r4);
+        const float kk[4] = {a.x, a.y, a.z, a.w}, qq[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          G[4 * m + x] = fmaf(sdO, qq[x], G[4 * m + x]);
+          tmp[4 * m + x] = sdO * fmaf(alpha, Sp[4 * m + x], bw * kk[x]);
+        }
+      }
+      halve8<CPL>(tmp, lane);
+#pragma unroll
+      for (int x = 0; x < KEEP; ++x) {
+        const int e = e0 + x;
+        rb[warp * DK + 16 * (e >> 2) + 4 * r4 + (e & 3)] = tmp[x];
+      }
+      float sgs = 0.f;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) sgs = fmaf(G[e], Sp[e], sgs);
+      const float gk = rowdot(G, kt);
+      // dk partial = beta w G[i, :] - alpha beta Gk_i S_{t-1}[i, :]
+      const float abg = alpha * bt * gk;
+#pragma unroll
+      for (int e = 0; e < CPL; ++e) tmp[e] = fmaf(bw, G[e], -abg * Sp[e]);
+      halve8<CPL>(tmp, lane);
+#pragma unroll
+      for (int x = 0; x < KEEP; ++x) {
+        const int e = e0 + x;
+        rb[NW * DK + warp * DK + 16 * (e >> 2) + 4 * r4 + (e & 3)] = tmp[x];
+      }
+      if (r4 == 0) p.dv[(tg * p.Hv + h) * DV + row] = bt * gk;
+      // scalars: <G, S_{t-1}> (every lane), (G k) . u and w . (G k) (one lane per row)
+      float s3[3] = {sgs, r4 == 0 ? gk * u : 0.f, r4 == 0 ? w * gk : 0.f};
+#pragma unroll
+      for (int x = 0; x < 3; ++x)
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s3[x] += __shfl_xor_sync(0xffffffffu, s3[x], off);
+      if (lane == 0) {
+        rs[parity * 3 * NW + warp] = s3[0];
+        rs[parity * 3 * NW + NW + warp] = s3[1];
+        rs[parity * 3 * NW + 2 * NW + warp] = s3[2];
+      }
+      // G <- alpha (G - beta (G k) k^T), before the barrier (registers only)
+      const float bgk = bt * gk;
+#pragma unroll
+      for (int m = 0; m < NV4; ++m) {
+        const float4 a = *reinterpret_cast<const float4 *>(kt + 16 * m + 4 * r4);
+        G[4 * m] = alpha * fmaf(-bgk, a.x, G[4 * m]);
+        G[4 * m + 1] = alpha * fmaf(-bgk, a.y, G[4 * m + 1]);
+        G[4 * m + 2] = alpha * fmaf(-bgk, a.z, G[4 * m + 2]);
+        G[4 * m + 3] = alpha * fmaf(-bgk, a.w, G[4 * m + 3]);
+      }
+      __syncthreads();
+      if (tid < DK) {
+        float aq = 0.f, ak = 0.f;
+#pragma unroll
+        for (int x = 0; x < NW; ++x) {
+          aq += rb[x * DK + tid];
+          ak += rb[NW * DK + x * DK + tid];
+        }
+        p.dq[(tg * p.Hv + h) * DK + tid] = aq;
+        p.dk[(tg * p.Hv + h) * DK + tid] = ak;
+      } else if (tid == DK) {
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f;
+#pragma unroll
+        for (int x = 0; x < NW; ++x) {
+          a0 += rs[parity * 3 * NW + x];
+          a1 += rs[parity * 3 * NW + NW + x];
+          a2 += rs[parity * 3 * NW + 2 * NW + x];
+        }
+        p.dg[tg * p.Hv + h] = alpha * (a0 - bt * a1);
+        p.dbeta[tg * p.Hv + h] = a2;
+      }
+      parity ^= 1;
+    }
+  }
+  if (p.ds0) {
+#pragma unroll
+    for (int m = 0; m < NV4; ++m)
+      *reinterpret_cast<float4 *>(p.ds0 + srow + 16 * m + 4 * r4) =
+          make_float4(G[4 * m], G[4 * m + 1], G[4 * m + 2], G[4 * m + 3]);
+  }
+}
+
+// dq, dk of query/key head j = sum over its group of value heads.
+__global__ void group_sum_kernel(const float *__restrict__ part, float *__restrict__ out, int T,
+                                 int Hqk, int Hv, int DK) {
+  const int G = Hv / Hqk;
+  const size_t total = (size_t)T * Hqk * DK;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int d = (int)(i % DK);
+    const size_t tj = i / DK;
+    const int jj = (int)(tj % Hqk);
+    const size_t t = tj / Hqk;
+    float a = 0.f;
+    for (int r = 0; r < G; ++r) a += part[(t * Hv + (size_t)jj * G + r) * DK + d];
+    out[i] = a;
+  }
+}
+
+}  // namespace bwd
+
+size_t backward_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t hs = (size_t)Dv * Dk * sizeof(float);
+  size_t b = kWorkspaceHeaderBytes;
+  b += up(((size_t)((T + bwd::C - 1) / bwd::C) + (size_t)N) * Hv * hs);  // checkpoints
+  b += up((size_t)N * Hv * bwd::C * hs);                                  // per-CTA scratch
+  if (Hv != Hqk) b += 2 * up((size_t)T * Hv * Dk * sizeof(float));        // dq, dk per value head
+  return b;
+}
+
+template <typename T, int DK, int DV>
+static cudaError_t launch_bwd_t(const bwd::Params &prm, cudaStream_t stream) {
+  using CF = bwd::Cfg<DK, DV>;
+  auto kern = bwd::backward_kernel<T, DK, DV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CF::SMEM);
+  if (e != cudaSuccess) return e;
+  kern<<<(unsigned)prm.N * (unsigned)prm.Hv, CF::THREADS, CF::SMEM, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_backward(const void *q, const void *k, const void *v, const float *g,
+                            const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
+                            int Hv, int Dk, int Dv, int dtype, float scale, const float *s0,
+                            const float *dO, const float *dSfin, float *dq, float *dk, float *dv,
+                            float *dg, float *dbeta, float *ds0, void *workspace,
+                            cudaStream_t stream) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const int T = (int)T_;
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  const size_t hs = (size_t)Dv * Dk * sizeof(float);
+  bwd::Params prm;
+  prm.q = q; prm.k = k; prm.v = v; prm.g = g; prm.beta = beta; prm.cu = cu;
+  prm.N = N; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.scale = scale;
+  prm.s0 = s0; prm.dO = dO; prm.dSfin = dSfin;
+  prm.dv = dv; prm.dg = dg; prm.dbeta = dbeta; prm.ds0 = ds0;
+  prm.status = reinterpret_cast<int32_t *>(ws);
+  size_t off = kWorkspaceHeaderBytes;
+  prm.ckpt = reinterpret_cast<float *>(ws + off);
+  off += up(((size_t)((T + bwd::C - 1) / bwd::C) + (size_t)N) * Hv * hs);
+  prm.scratch = reinterpret_cast<float *>(ws + off);
+  off += up((size_t)N * Hv * bwd::C * hs);
+  float *dq_part = dq, *dk_part = dk;
+  if (Hv != Hqk) {
+    dq_part = reinterpret_cast<float *>(ws + off);
+    off += up((size_t)T * Hv * Dk * sizeof(float));
+    dk_part = reinterpret_cast<float *>(ws + off);
+  }
+  prm.dq = dq_part; prm.dk = dk_part;
+  cudaError_t e;
+  if (dtype == GDN_DTYPE_BF16) {
+    if (Dk == 128 && Dv == 128) e = launch_bwd_t<__nv_bfloat16, 128, 128>(prm, stream);
+    else if (Dk == 128 && Dv == 64) e = launch_bwd_t<__nv_bfloat16, 128, 64>(prm, stream);
+    else if (Dk == 64 && Dv == 128) e = launch_bwd_t<__nv_bfloat16, 64, 128>(prm, stream);
+    else e = launch_bwd_t<__nv_bfloat16, 64, 64>(prm, stream);
+  } else {
+    if (Dk == 128 && Dv == 128) e = launch_bwd_t<float, 128, 128>(prm, stream);
+    else if (Dk == 128 && Dv == 64) e = launch_bwd_t<float, 128, 64>(prm, stream);
+    else if (Dk == 64 && Dv == 128) e = launch_bwd_t<float, 64, 128>(prm, stream);
+    else e = launch_bwd_t<float, 64, 64>(prm, stream);
+  }
+  if (e != cudaSuccess || Hv == Hqk || T == 0) return e;
+  const size_t total = (size_t)T * Hqk * Dk;
+  const unsigned blocks = (unsigned)std::min<size_t>((total + 255) / 256, 148 * 16);
+  bwd::group_sum_kernel<<<blocks, 256, 0, stream>>>(dq_part, dq, T, Hqk, Hv, Dk);
+  bwd::group_sum_kernel<<<blocks, 256, 0, stream>>>(dk_part, dk, T, Hqk, Hv, Dk);
+  return cudaGetLastError();
+}
+
+}  // namespace gdn

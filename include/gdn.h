@@ -288,6 +288,53 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
                           int32_t input_form, float scale, int32_t *device_status, void *stream);
 
 /*
+ * Bytes of device workspace gdn_prefill_backward needs for these sizes (0 for
+ * invalid sizes): the status header, a checkpoint of every state every 16
+ * tokens (about (T/16 + num_seqs) x Hv x Dv x Dk x 4 bytes), a scratch of 16
+ * states per (sequence, value head), and per-value-head dq, dk when
+ * Hv > Hqk.
+ */
+size_t gdn_prefill_backward_workspace_size(int32_t num_seqs, int64_t total_tokens,
+                                           int32_t num_qk_heads, int32_t num_v_heads,
+                                           int32_t head_dim_k, int32_t head_dim_v);
+
+/*
+ * Backward pass of gdn_prefill (training): the gradients of a loss L with
+ * respect to q, k, v, g, beta and the initial state, given d_o = dL/do and
+ * optionally d_final_state = dL/dS_final.  Same rule, layout and sequences as
+ * gdn_prefill with fp32 states and prepared inputs (the page's note says the
+ * block form is used in training as well: "Inside Qwen3.8-27B ...", section
+ * "Gated DeltaNet Mechanics").  With u = S_{t-1} k_t, w = v_t - alpha_t u and
+ * G = dL/dS_t, going backwards over the tokens:
+ *   G += scale dO_t q_t^T;  dq_t = scale S_t^T dO_t;  dv_t = beta_t G k_t;
+ *   dbeta_t = w . G k_t;  dg_t = alpha_t (<G, S_{t-1}> - beta_t (G k_t) . u);
+ *   dk_t = beta_t G^T w - alpha_t beta_t S_{t-1}^T G k_t;
+ *   G <- alpha_t (G - beta_t (G k_t) k_t^T);  d_initial_state = G at the start.
+ * dq and dk of a query/key head sum over the value heads reading it.
+ *
+ *   q, k, v, g, beta, cu_seqlens, initial_state (fp32 or NULL), scale: as for
+ *                  gdn_prefill (prepared inputs; dtype bf16 or fp32)
+ *   d_o            [T, Hv, Dv] fp32
+ *   d_final_state  [num_seqs, Hv, Dv, Dk] fp32, or NULL for zeros
+ *   dq, dk         [T, Hqk, Dk] fp32 (outputs);  dv [T, Hv, Dv] fp32;
+ *   dg, dbeta      [T, Hv] fp32;  d_initial_state [num_seqs, Hv, Dv, Dk] fp32 or NULL
+ *   workspace      >= gdn_prefill_backward_workspace_size(...) bytes, 256-byte
+ *                  aligned; its first word is the sticky device status word
+ *                  (GDN_ERR_BAD_SEQLENS), read with gdn_get_device_status.
+ * Runs on CUDA cores in fp32: one block per (sequence, value head) with the
+ * state and G in registers, a forward pass storing checkpoints, then the
+ * chunks in reverse.  Supported: Hv % Hqk == 0; Dk, Dv in {64, 128}.
+ */
+int32_t gdn_prefill_backward(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
+                             int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
+                             int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, float scale,
+                             const float *initial_state, const float *d_o,
+                             const float *d_final_state, float *dq, float *dk, float *dv,
+                             float *dg, float *dbeta, float *d_initial_state, void *workspace,
+                             size_t workspace_bytes, void *stream);
+
+/*
  * 1 if gdn_prefill with these sizes and dtype runs the tensor-core (tcgen05)
  * kernel, 0 if it runs the fp32 CUDA-core kernel or the arguments are invalid.
  * Host only; touches no device.

@@ -169,3 +169,34 @@ def test_binding_refuses_cpu_tensors(lib):
     x = torch.zeros(4, 1, 64)
     with pytest.raises(ValueError):
         api.prefill(x, x, x, torch.zeros(4, 1), torch.zeros(4, 1))
+
+
+def test_backward_workspace_and_validation(lib):
+    """gdn_prefill_backward: workspace arithmetic and host-side rejections
+    (nothing is launched; the fake addresses are never dereferenced)."""
+    ck = 64 * 1024  # one 128 x 128 fp32 state
+    ws = api.prefill_backward_workspace_size(1, 8192, 16, 48, 128, 128)
+    need = (512 + 1) * 48 * ck + 48 * 16 * ck + 2 * 8192 * 48 * 128 * 4
+    assert need <= ws <= need + 4 * 256 + 256
+    assert api.prefill_backward_workspace_size(1, 8192, 48, 48, 128, 128) < ws  # no per-head dq, dk
+    assert lib.gdn_prefill_backward_workspace_size(1, 10, 16, 40, 128, 128) == 0  # 40 % 16
+    assert lib.gdn_prefill_backward_workspace_size(1, 10, 16, 48, 96, 128) == 0
+    vp = 1 << 12
+    a = dict(q=vp, k=vp, v=vp, g=vp, beta=vp, cu=vp, N=1, T=16, Hqk=2, Hv=6, Dk=64, Dv=64, dtype=0,
+             scale=1.0, s0=None, do=vp, dsf=None, dq=vp, dk=vp, dv=vp, dg=vp, db=vp, ds0=None,
+             ws=vp, wsb=1 << 30)
+
+    def call(**kw):
+        x = {**a, **kw}
+        return lib.gdn_prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu"], x["N"],
+                                        x["T"], x["Hqk"], x["Hv"], x["Dk"], x["Dv"], x["dtype"],
+                                        x["scale"], x["s0"], x["do"], x["dsf"], x["dq"], x["dk"],
+                                        x["dv"], x["dg"], x["db"], x["ds0"], x["ws"], x["wsb"], None)
+
+    assert call(do=None) == api.GDN_ERR_INVALID_ARG
+    assert call(dq=vp + 4) == api.GDN_ERR_INVALID_ARG          # misaligned
+    assert call(Hv=5) == api.GDN_ERR_INVALID_ARG
+    assert call(Dk=96) == api.GDN_ERR_UNSUPPORTED
+    assert call(wsb=1024) == api.GDN_ERR_WORKSPACE
+    assert call(ws=vp + 16) == api.GDN_ERR_WORKSPACE            # not 256-byte aligned
+    assert call(N=0, T=0) == api.GDN_OK

@@ -1,0 +1,76 @@
+"""Backward pass (gdn_prefill_backward) on the GPU against the fp64 oracle's
+backward, itself pinned to central finite differences of the forward rule."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_deltanet_recurrence_rule_b200 import api, inputs
+from parity import o_error, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+TOL = 1e-4  # fp32 arithmetic against fp64 on the same inputs: max|err| / RMS(ref) per gradient
+
+
+def _case(lengths, Hqk, Hv, D, dtype, seed, init=True, dsf=True, scale=0.5):
+    inp = inputs.prefill_inputs(lengths, Hqk, Hv, D, dtype=dtype, seed=seed,
+                                init_std=0.1 if init else 0.0)
+    T, N = sum(lengths), len(lengths)
+    gen = torch.Generator().manual_seed(seed + 700)
+    d_o = torch.randn(T, Hv, D, generator=gen)
+    d_sf = torch.randn(N, Hv, D, D, generator=gen) * 0.1 if dsf else None
+    dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
+    out = api.prefill_backward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], d_o.to(DEV),
+                               cu_seqlens=dev["cu_seqlens"], initial_state=dev["initial_state"],
+                               d_final_state=None if d_sf is None else d_sf.to(DEV), scale=scale)
+    torch.cuda.synchronize()
+    ref = oracle.backward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], d_o,
+                          cu_seqlens=inp["cu_seqlens"], initial_state=inp["initial_state"],
+                          d_final_state=d_sf, scale=scale)
+    return out, ref
+
+
+def _check(out, ref, what):
+    for name, a, b in zip(("dq", "dk", "dv", "dg", "dbeta", "ds0"), out, ref):
+        a = to_np(a)
+        assert np.isfinite(a).all(), f"{what}: non-finite {name}"
+        e = o_error(a, b)
+        assert e <= TOL, f"{what}: {name} max|err|/RMS = {e:.3e} > {TOL:.0e}"
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_backward_varlen_gqa(dtype, D):
+    out, ref = _case([37, 0, 50, 16], 2, 6, D, dtype, seed=101 + D)
+    _check(out, ref, f"{dtype} D={D}")
+
+
+def test_backward_mixed_dims():
+    """Dk != Dv, one value head per query/key head (dq, dk written directly)."""
+    for Dk, Dv in ((128, 64), (64, 128)):
+        inp = inputs.prefill_inputs([40, 23], 2, 2, Dk, dtype="fp32", seed=105, init_std=0.1)
+        gen = torch.Generator().manual_seed(106)
+        T = 63
+        v = torch.randn(T, 2, Dv, generator=gen)
+        s0 = torch.randn(2, 2, Dv, Dk, generator=gen) * 0.1
+        d_o = torch.randn(T, 2, Dv, generator=gen)
+        out = api.prefill_backward(inp["q"].to(DEV), inp["k"].to(DEV), v.to(DEV), inp["g"].to(DEV),
+                                   inp["beta"].to(DEV), d_o.to(DEV),
+                                   cu_seqlens=inp["cu_seqlens"].to(DEV), initial_state=s0.to(DEV))
+        torch.cuda.synchronize()
+        ref = oracle.backward(inp["q"], inp["k"], v, inp["g"], inp["beta"], d_o,
+                              cu_seqlens=inp["cu_seqlens"], initial_state=s0)
+        _check(out, ref, f"Dk={Dk} Dv={Dv}")
+
+
+def test_backward_without_states():
+    """No initial state and no final-state gradient (both NULL)."""
+    out, ref = _case([70], 1, 3, 64, "fp32", seed=107, init=False, dsf=False, scale=1.0)
+    _check(out, ref, "no states")
+
+
+def test_backward_long_sequence():
+    """1000 tokens (62 chunks of 16 plus a ragged one) at D=64."""
+    out, ref = _case([1000], 1, 2, 64, "bf16", seed=108)
+    _check(out, ref, "T=1000")

@@ -580,13 +580,14 @@ def _backward(args, D, dev, x, T, w, peaks):
             "workload": f"backward of prefill8k: T={T} Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16 inputs, "
                         "fp32 d_o and dL/dS_final, zero initial state",
             "ms_per_step": ms,
-            "roofline": {"bound": "alu", "kernel": "backward_kernel (+ group_sum_kernel x 2)",
+            "roofline": {"bound": "alu", "kernel": "backward_kernel (4 row slices per head), then "
+                                                    "group_sum_kernel x 4 for dq, dk, dg, dbeta",
                          "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s",
                          "frac": achieved / fp32_peak,
                          "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
                          "algorithmic": f"18 D^2 flop per token and value head = {flop} flop",
                          "traffic": None},
-            "gpu_launches": 3 * steps}
+            "gpu_launches": 5 * steps}  # at these sizes: 4 row slices per head, Hv > Hqk
 
 
 def _decode(args, D, dev, peaks, peak_src):

@@ -17,16 +17,20 @@
 //   G      <- alpha_t (G - beta_t (G k_t) k_t^T)
 // and dS0 = G at the start of the sequence.
 //
-// One CTA per (sequence, value head), 4 lanes per state row (4 Dv threads),
-// each lane holding Dk/4 columns of S and of G in registers:
+// Rows of S (and of G) evolve independently, so one CTA takes a slice of
+// ROWS rows of one (sequence, value head): 4 lanes per state row, each lane
+// holding Dk/4 columns of S and of G in registers.  Slices are chosen so that
+// a small batch still fills the GPU (backward_slices); sums over the rows
+// (dq, dk, dg, dbeta) are written per slice and added by a second kernel.
+// Per CTA:
 //   pass 1  forward from S0, storing a checkpoint of S every C tokens;
 //   pass 2  chunks last to first: the chunk's states S_{t-1} are recomputed
 //           from its checkpoint into a per-CTA scratch, then walked backwards.
 // S^T x products (dq, dk) are column sums over all rows: a recursive-halving
 // shuffle over the 8 rows of a warp, then a sum over warps in shared memory
-// (double-buffered, one block barrier per token).  dq and dk are written per
-// value head and summed over each query/key head's group by a second kernel,
-// so the result does not depend on scheduling.
+// (double-buffered, one block barrier per token).  The partial sums are added
+// in a fixed order by the second kernel, so the result does not depend on
+// scheduling.
 #include <algorithm>
 
 #include "gdn_common.cuh"
@@ -36,16 +40,16 @@ namespace bwd {
 
 constexpr int C = 16;  // tokens per checkpoint chunk
 
-template <int DK, int DV>
+template <int DK, int ROWS>
 struct Cfg {
-  static constexpr int THREADS = 4 * DV;  // 4 lanes per state row
+  static constexpr int THREADS = 4 * ROWS;  // 4 lanes per state row
   static constexpr int CPL = DK / 4;      // columns per lane: 16 m + 4 r4 + (0..3)
   static constexpr int NV4 = CPL / 4;
   static constexpr int NW = THREADS / 32;
   static constexpr int KEEP = CPL / 8;    // columns a lane keeps after the 8-row halving
   // shared memory (floats)
-  static constexpr int S_Q = 0, S_K = S_Q + C * DK, S_V = S_K + C * DK, S_DO = S_V + C * DV;
-  static constexpr int S_A = S_DO + C * DV, S_B = S_A + C;
+  static constexpr int S_Q = 0, S_K = S_Q + C * DK, S_V = S_K + C * DK, S_DO = S_V + C * ROWS;
+  static constexpr int S_A = S_DO + C * ROWS, S_B = S_A + C;
   static constexpr int S_RED = S_B + C;                  // [2 buffers][2 vectors][NW][DK]
   static constexpr int S_RS = S_RED + 2 * 2 * NW * DK;   // [2 buffers][3][NW]
   static constexpr int S_BASE = S_RS + 2 * 3 * NW;       // chunk base (int)
@@ -57,13 +61,14 @@ struct Params {
   const void *q, *k, *v;
   const float *g, *beta;
   const int32_t *cu;
-  int N, T, Hqk, Hv;
+  int N, T, Hqk, Hv, Dv, R;  // R slices of Dv / R rows per (sequence, value head)
   float scale;
   const float *s0, *dO, *dSfin;
-  float *dq, *dk;  // [T, Hv, DK]: per value head (the outputs themselves when Hv == Hqk)
-  float *dv, *dg, *dbeta, *ds0;
-  float *ckpt;     // [(ceil(T / C) + N) * Hv][64 KiB states]
-  float *scratch;  // [N * Hv][C states]
+  float *dq, *dk;     // [T, Hv R, DK] per slice (the outputs themselves when Hv R == Hqk)
+  float *dg, *dbeta;  // [T, Hv R] per slice (the outputs themselves when R == 1)
+  float *dv, *ds0;
+  float *ckpt;     // [(ceil(T / C) + N) * Hv][Dv x Dk states]
+  float *scratch;  // [N * Hv * R][C states of a slice]
   int32_t *status;
 };
 
@@ -106,16 +111,19 @@ __device__ __forceinline__ int keep_e0(int lane) {
   return (CPL / 2) * ((lane >> 4) & 1) + (CPL / 4) * ((lane >> 3) & 1) + (CPL / 8) * ((lane >> 2) & 1);
 }
 
-template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(4 * DV, 1)
+template <typename T, int DK, int ROWS>
+__global__ void __launch_bounds__(4 * ROWS, ROWS == 128 ? 1 : 2)
 backward_kernel(const Params p) {
-  using CF = Cfg<DK, DV>;
+  using CF = Cfg<DK, ROWS>;
   constexpr int CPL = CF::CPL, NV4 = CF::NV4, NW = CF::NW, KEEP = CF::KEEP;
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = tid >> 2, r4 = tid & 3;
-  const int n = blockIdx.x / p.Hv, h = blockIdx.x - n * p.Hv;
+  const int row = tid >> 2, r4 = tid & 3;  // row within the slice
+  const int unit = blockIdx.x / p.R, slice = blockIdx.x - unit * p.R;
+  const int n = unit / p.Hv, h = unit - n * p.Hv;
   const int j = h / (p.Hv / p.Hqk);
+  const int DV = p.Dv, rowg = slice * ROWS + row;  // row within the head
+  const int slot = h * p.R + slice;                // partial-sum slot of this CTA
 
   const int c0 = p.cu[n], c1 = p.cu[n + 1];
   if (c0 < 0 || c1 < c0 || c1 > p.T || (n == 0 && c0 != 0) || (n == p.N - 1 && c1 != p.T)) {
@@ -130,12 +138,12 @@ backward_kernel(const Params p) {
   }
   __syncthreads();
   const int cbase = reinterpret_cast<const int *>(sm + CF::S_BASE)[0];
-  const size_t hs = (size_t)DV * DK;
-  const size_t srow = ((size_t)n * p.Hv + h) * hs + (size_t)row * DK;
+  const size_t hs = (size_t)DV * DK, ss = (size_t)ROWS * DK;  // a head's / a slice's state
+  const size_t srow = ((size_t)n * p.Hv + h) * hs + (size_t)rowg * DK;
   auto ck = [&](int c) {  // this thread's float4s of checkpoint c, laid out [NV4][THREADS]
-    return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(cbase + c) * p.Hv + h) * hs) + tid;
+    return reinterpret_cast<float4 *>(p.ckpt + ((size_t)(cbase + c) * p.Hv + h) * hs + slice * ss) + tid;
   };
-  float4 *scr = reinterpret_cast<float4 *>(p.scratch + (size_t)blockIdx.x * C * hs) + tid;
+  float4 *scr = reinterpret_cast<float4 *>(p.scratch + (size_t)blockIdx.x * C * ss) + tid;
 
   float *sq = sm + CF::S_Q, *sk = sm + CF::S_K, *sv = sm + CF::S_V, *sdo = sm + CF::S_DO;
   float *sa = sm + CF::S_A, *sb = sm + CF::S_B;
@@ -149,9 +157,9 @@ backward_kernel(const Params p) {
       sk[x] = to_f32(static_cast<const T *>(p.k)[off]);
       if (full) sq[x] = to_f32(static_cast<const T *>(p.q)[off]);
     }
-    for (int x = tid; x < cnt * DV; x += CF::THREADS) {
-      const int t = x / DV, d = x - t * DV;
-      const size_t off = ((size_t)(t0 + t) * p.Hv + h) * DV + d;
+    for (int x = tid; x < cnt * ROWS; x += CF::THREADS) {
+      const int t = x / ROWS, d = x - t * ROWS;
+      const size_t off = ((size_t)(t0 + t) * p.Hv + h) * DV + slice * ROWS + d;
       sv[x] = to_f32(static_cast<const T *>(p.v)[off]);
       if (full) sdo[x] = p.dO[off];
     }
@@ -177,7 +185,7 @@ backward_kernel(const Params p) {
   auto step = [&](float (&S)[CPL], int t) {  // S <- S_t from S_{t-1}
     const float *kt = sk + t * DK;
     const float u = rowdot(S, kt);
-    const float w = sb[t] * (sv[t * DV + row] - sa[t] * u);
+    const float w = sb[t] * (sv[t * ROWS + row] - sa[t] * u);
 #pragma unroll
     for (int m = 0; m < NV4; ++m) {
       const float4 y = *reinterpret_cast<const float4 *>(kt + 16 * m + 4 * r4);
@@ -240,8 +248,8 @@ backward_kernel(const Params p) {
         Sp[4 * m] = x.x; Sp[4 * m + 1] = x.y; Sp[4 * m + 2] = x.z; Sp[4 * m + 3] = x.w;
       }
       const float u = rowdot(Sp, kt);
-      const float w = sv[t * DV + row] - alpha * u;  // v - alpha u (beta applied where used)
-      const float sdO = p.scale * sdo[t * DV + row], bw = bt * w;
+      const float w = sv[t * ROWS + row] - alpha * u;  // v - alpha u (beta applied where used)
+      const float sdO = p.scale * sdo[t * ROWS + row], bw = bt * w;
       float *rb = red + parity * 2 * NW * DK;
       const int e0 = keep_e0<CPL>(lane);
       float tmp[CPL];
@@ -277,7 +285,7 @@ backward_kernel(const Params p) {
         const int e = e0 + x;
         rb[NW * DK + warp * DK + 16 * (e >> 2) + 4 * r4 + (e & 3)] = tmp[x];
       }
-      if (r4 == 0) p.dv[(tg * p.Hv + h) * DV + row] = bt * gk;
+      if (r4 == 0) p.dv[(tg * p.Hv + h) * DV + rowg] = bt * gk;
       // scalars: <G, S_{t-1}> (every lane), (G k) . u and w . (G k) (one lane per row)
       float s3[3] = {sgs, r4 == 0 ? gk * u : 0.f, r4 == 0 ? w * gk : 0.f};
 #pragma unroll
@@ -307,9 +315,10 @@ backward_kernel(const Params p) {
           aq += rb[x * DK + tid];
           ak += rb[NW * DK + x * DK + tid];
         }
-        p.dq[(tg * p.Hv + h) * DK + tid] = aq;
-        p.dk[(tg * p.Hv + h) * DK + tid] = ak;
-      } else if (tid == DK) {
+        p.dq[(tg * p.Hv * p.R + slot) * DK + tid] = aq;
+        p.dk[(tg * p.Hv * p.R + slot) * DK + tid] = ak;
+      }
+      if (tid == 0) {  // (a block may have exactly DK threads)
         float a0 = 0.f, a1 = 0.f, a2 = 0.f;
 #pragma unroll
         for (int x = 0; x < NW; ++x) {
@@ -317,8 +326,8 @@ backward_kernel(const Params p) {
           a1 += rs[parity * 3 * NW + NW + x];
           a2 += rs[parity * 3 * NW + 2 * NW + x];
         }
-        p.dg[tg * p.Hv + h] = alpha * (a0 - bt * a1);
-        p.dbeta[tg * p.Hv + h] = a2;
+        p.dg[tg * p.Hv * p.R + slot] = alpha * (a0 - bt * a1);  // linear in the row sums
+        p.dbeta[tg * p.Hv * p.R + slot] = a2;
       }
       parity ^= 1;
     }
@@ -331,43 +340,65 @@ backward_kernel(const Params p) {
   }
 }
 
-// dq, dk of query/key head j = sum over its group of value heads.
-__global__ void group_sum_kernel(const float *__restrict__ part, float *__restrict__ out, int T,
-                                 int Hqk, int Hv, int DK) {
-  const int G = Hv / Hqk;
-  const size_t total = (size_t)T * Hqk * DK;
+// out[r][d] = sum over the `width` consecutive partial slots of group r:
+// part is [rows * width][inner], out is [rows][inner] (dq, dk: a query/key
+// head's value heads and slices; dg, dbeta: a value head's slices).
+__global__ void group_sum_kernel(const float *__restrict__ part, float *__restrict__ out,
+                                 size_t rows, int width, int inner) {
+  const size_t total = rows * inner;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
        i += (size_t)gridDim.x * blockDim.x) {
-    const int d = (int)(i % DK);
-    const size_t tj = i / DK;
-    const int jj = (int)(tj % Hqk);
-    const size_t t = tj / Hqk;
+    const size_t r = i / inner, d = i - r * inner;
+    const float *src = part + r * width * inner + d;
     float a = 0.f;
-    for (int r = 0; r < G; ++r) a += part[(t * Hv + (size_t)jj * G + r) * DK + d];
+    for (int x = 0; x < width; ++x) a += src[(size_t)x * inner];
     out[i] = a;
   }
 }
 
 }  // namespace bwd
 
+// Slices per (sequence, value head): doubled, down to 32 rows per CTA, until
+// the grid has two CTAs per SM of a B200 (148 SMs).  A function of the sizes
+// only, so the workspace query and the launch agree.
+static int backward_slices(int64_t N, int Hv, int Dv) {
+  int R = 1;
+  while (Dv / (2 * R) >= 32 && N * Hv * R < 2 * 148) R *= 2;
+  return R;
+}
+
 size_t backward_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const int R = backward_slices(N, Hv, Dv);
   const size_t hs = (size_t)Dv * Dk * sizeof(float);
   size_t b = kWorkspaceHeaderBytes;
   b += up(((size_t)((T + bwd::C - 1) / bwd::C) + (size_t)N) * Hv * hs);  // checkpoints
   b += up((size_t)N * Hv * bwd::C * hs);                                  // per-CTA scratch
-  if (Hv != Hqk) b += 2 * up((size_t)T * Hv * Dk * sizeof(float));        // dq, dk per value head
+  if ((int64_t)Hv * R != Hqk) b += 2 * up((size_t)T * Hv * R * Dk * sizeof(float));  // dq, dk
+  if (R > 1) b += 2 * up((size_t)T * Hv * R * sizeof(float));                        // dg, dbeta
   return b;
 }
 
-template <typename T, int DK, int DV>
+template <typename T, int DK, int ROWS>
 static cudaError_t launch_bwd_t(const bwd::Params &prm, cudaStream_t stream) {
-  using CF = bwd::Cfg<DK, DV>;
-  auto kern = bwd::backward_kernel<T, DK, DV>;
+  using CF = bwd::Cfg<DK, ROWS>;
+  auto kern = bwd::backward_kernel<T, DK, ROWS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CF::SMEM);
   if (e != cudaSuccess) return e;
-  kern<<<(unsigned)prm.N * (unsigned)prm.Hv, CF::THREADS, CF::SMEM, stream>>>(prm);
+  kern<<<(unsigned)prm.N * (unsigned)prm.Hv * (unsigned)prm.R, CF::THREADS, CF::SMEM, stream>>>(prm);
   return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_bwd_rows(const bwd::Params &prm, int Dk, int rows, cudaStream_t stream) {
+  if (Dk == 128) {
+    if (rows == 128) return launch_bwd_t<T, 128, 128>(prm, stream);
+    if (rows == 64) return launch_bwd_t<T, 128, 64>(prm, stream);
+    return launch_bwd_t<T, 128, 32>(prm, stream);
+  }
+  if (rows == 128) return launch_bwd_t<T, 64, 128>(prm, stream);
+  if (rows == 64) return launch_bwd_t<T, 64, 64>(prm, stream);
+  return launch_bwd_t<T, 64, 32>(prm, stream);
 }
 
 cudaError_t launch_backward(const void *q, const void *k, const void *v, const float *g,
@@ -378,43 +409,49 @@ cudaError_t launch_backward(const void *q, const void *k, const void *v, const f
                             cudaStream_t stream) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
   const int T = (int)T_;
+  const int R = backward_slices(N, Hv, Dv);
   unsigned char *ws = static_cast<unsigned char *>(workspace);
   const size_t hs = (size_t)Dv * Dk * sizeof(float);
   bwd::Params prm;
   prm.q = q; prm.k = k; prm.v = v; prm.g = g; prm.beta = beta; prm.cu = cu;
-  prm.N = N; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.scale = scale;
+  prm.N = N; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.Dv = Dv; prm.R = R; prm.scale = scale;
   prm.s0 = s0; prm.dO = dO; prm.dSfin = dSfin;
-  prm.dv = dv; prm.dg = dg; prm.dbeta = dbeta; prm.ds0 = ds0;
+  prm.dv = dv; prm.ds0 = ds0;
   prm.status = reinterpret_cast<int32_t *>(ws);
   size_t off = kWorkspaceHeaderBytes;
   prm.ckpt = reinterpret_cast<float *>(ws + off);
   off += up(((size_t)((T + bwd::C - 1) / bwd::C) + (size_t)N) * Hv * hs);
   prm.scratch = reinterpret_cast<float *>(ws + off);
   off += up((size_t)N * Hv * bwd::C * hs);
-  float *dq_part = dq, *dk_part = dk;
-  if (Hv != Hqk) {
-    dq_part = reinterpret_cast<float *>(ws + off);
-    off += up((size_t)T * Hv * Dk * sizeof(float));
-    dk_part = reinterpret_cast<float *>(ws + off);
+  const bool qk_direct = (int64_t)Hv * R == Hqk, gb_direct = R == 1;
+  prm.dq = dq; prm.dk = dk; prm.dg = dg; prm.dbeta = dbeta;
+  if (!qk_direct) {
+    prm.dq = reinterpret_cast<float *>(ws + off);
+    off += up((size_t)T * Hv * R * Dk * sizeof(float));
+    prm.dk = reinterpret_cast<float *>(ws + off);
+    off += up((size_t)T * Hv * R * Dk * sizeof(float));
   }
-  prm.dq = dq_part; prm.dk = dk_part;
-  cudaError_t e;
-  if (dtype == GDN_DTYPE_BF16) {
-    if (Dk == 128 && Dv == 128) e = launch_bwd_t<__nv_bfloat16, 128, 128>(prm, stream);
-    else if (Dk == 128 && Dv == 64) e = launch_bwd_t<__nv_bfloat16, 128, 64>(prm, stream);
-    else if (Dk == 64 && Dv == 128) e = launch_bwd_t<__nv_bfloat16, 64, 128>(prm, stream);
-    else e = launch_bwd_t<__nv_bfloat16, 64, 64>(prm, stream);
-  } else {
-    if (Dk == 128 && Dv == 128) e = launch_bwd_t<float, 128, 128>(prm, stream);
-    else if (Dk == 128 && Dv == 64) e = launch_bwd_t<float, 128, 64>(prm, stream);
-    else if (Dk == 64 && Dv == 128) e = launch_bwd_t<float, 64, 128>(prm, stream);
-    else e = launch_bwd_t<float, 64, 64>(prm, stream);
+  if (!gb_direct) {
+    prm.dg = reinterpret_cast<float *>(ws + off);
+    off += up((size_t)T * Hv * R * sizeof(float));
+    prm.dbeta = reinterpret_cast<float *>(ws + off);
   }
-  if (e != cudaSuccess || Hv == Hqk || T == 0) return e;
-  const size_t total = (size_t)T * Hqk * Dk;
-  const unsigned blocks = (unsigned)std::min<size_t>((total + 255) / 256, 148 * 16);
-  bwd::group_sum_kernel<<<blocks, 256, 0, stream>>>(dq_part, dq, T, Hqk, Hv, Dk);
-  bwd::group_sum_kernel<<<blocks, 256, 0, stream>>>(dk_part, dk, T, Hqk, Hv, Dk);
+  const int rows = Dv / R;
+  cudaError_t e = dtype == GDN_DTYPE_BF16 ? launch_bwd_rows<__nv_bfloat16>(prm, Dk, rows, stream)
+                                          : launch_bwd_rows<float>(prm, Dk, rows, stream);
+  if (e != cudaSuccess || T == 0) return e;
+  auto blocks = [](size_t total) { return (unsigned)std::min<size_t>((total + 255) / 256, 148 * 16); };
+  if (!qk_direct) {
+    const size_t rows_qk = (size_t)T * Hqk;
+    const int width = Hv / Hqk * R;
+    bwd::group_sum_kernel<<<blocks(rows_qk * Dk), 256, 0, stream>>>(prm.dq, dq, rows_qk, width, Dk);
+    bwd::group_sum_kernel<<<blocks(rows_qk * Dk), 256, 0, stream>>>(prm.dk, dk, rows_qk, width, Dk);
+  }
+  if (!gb_direct) {
+    const size_t rows_gb = (size_t)T * Hv;
+    bwd::group_sum_kernel<<<blocks(rows_gb), 256, 0, stream>>>(prm.dg, dg, rows_gb, R, 1);
+    bwd::group_sum_kernel<<<blocks(rows_gb), 256, 0, stream>>>(prm.dbeta, dbeta, rows_gb, R, 1);
+  }
   return cudaGetLastError();
 }
 

@@ -175,10 +175,15 @@ def test_backward_workspace_and_validation(lib):
     """gdn_prefill_backward: workspace arithmetic and host-side rejections
     (nothing is launched; the fake addresses are never dereferenced)."""
     ck = 64 * 1024  # one 128 x 128 fp32 state
+    # 48 heads fill few SMs: 4 row slices per head, dq/dk/dg/dbeta per slice
     ws = api.prefill_backward_workspace_size(1, 8192, 16, 48, 128, 128)
-    need = (512 + 1) * 48 * ck + 48 * 16 * ck + 2 * 8192 * 48 * 128 * 4
-    assert need <= ws <= need + 4 * 256 + 256
-    assert api.prefill_backward_workspace_size(1, 8192, 48, 48, 128, 128) < ws  # no per-head dq, dk
+    need = (512 + 1) * 48 * ck + 48 * 16 * ck + 2 * 8192 * 48 * 4 * (128 * 4 + 4)
+    assert need <= ws <= need + 6 * 256
+    # 8 sequences x 48 heads fill the GPU: one slice, dq/dk per value head only
+    ws8 = api.prefill_backward_workspace_size(8, 8192, 16, 48, 128, 128)
+    need8 = (512 + 8) * 48 * ck + 8 * 48 * 16 * ck + 2 * 8192 * 48 * 128 * 4
+    assert need8 <= ws8 <= need8 + 4 * 256
+    assert api.prefill_backward_workspace_size(8, 8192, 48, 48, 128, 128) == ws8 - 2 * 8192 * 48 * 128 * 4
     assert lib.gdn_prefill_backward_workspace_size(1, 10, 16, 40, 128, 128) == 0  # 40 % 16
     assert lib.gdn_prefill_backward_workspace_size(1, 10, 16, 48, 96, 128) == 0
     vp = 1 << 12

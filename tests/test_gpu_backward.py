@@ -74,3 +74,12 @@ def test_backward_long_sequence():
     """1000 tokens (62 chunks of 16 plus a ragged one) at D=64."""
     out, ref = _case([1000], 1, 2, 64, "bf16", seed=108)
     _check(out, ref, "T=1000")
+
+
+@pytest.mark.parametrize("Hqk,Hv,N", [(2, 6, 50), (2, 2, 150)])
+def test_backward_many_units_one_slice(Hqk, Hv, N):
+    """Enough (sequence, value head) units to fill the GPU: one slice per head,
+    dg and dbeta written directly (and dq, dk too when Hv == Hqk)."""
+    lengths = [(7 * i) % 23 for i in range(N)]  # 0 .. 22 tokens, some empty
+    out, ref = _case(lengths, Hqk, Hv, 64, "fp32", seed=109 + Hv)
+    _check(out, ref, f"{N} sequences x {Hv} heads")

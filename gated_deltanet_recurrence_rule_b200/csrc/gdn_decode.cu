@@ -458,14 +458,14 @@ decode_tokens_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k,
 // the fp32 decode step: k, q and v go straight from global memory into
 // registers (no shared memory, no block barrier) and every warp has all of its
 // rows in flight (8 KiB at Dk = Dv = 128) before the first one is used.
-template <typename T, typename TO, int DK, int DV>
-__global__ void __launch_bounds__(128, 4)
+template <typename T, typename TO, int DK, int DV, bool RAW>
+__global__ void __launch_bounds__(128, RAW ? 3 : 4)  // the prologue needs a few more registers
 decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                         const float *__restrict__ g, const float *__restrict__ beta,
                         const __nv_bfloat16 *state_in, __nv_bfloat16 *state_out,
                         const int32_t *__restrict__ src_slot, const int32_t *__restrict__ dst_slot,
                         int num_slots, TO *__restrict__ o, int Hqk, int Hv, float scale,
-                        int32_t *status, int raw) {
+                        int32_t *status) {
   pdl_wait();  // nothing is read before the previous kernel on the stream is done
   pdl_allow_next();
   constexpr int NU = DK / 64;  // 16-byte pieces per lane per row
@@ -509,7 +509,7 @@ decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
       kf[4 * m + 2 * hf] = make_float2(a[0], a[1]); kf[4 * m + 2 * hf + 1] = make_float2(a[2], a[3]);
       qf[4 * m + 2 * hf] = make_float2(c[0], c[1]); qf[4 * m + 2 * hf + 1] = make_float2(c[2], c[3]);
     }
-  if (raw) {  // unit L2 norm: the 8 lanes of a row group hold all Dk columns
+  if constexpr (RAW) {  // unit L2 norm: the 8 lanes of a row group hold all Dk columns
     float2 sk2 = make_float2(0.f, 0.f), sq2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int e = 0; e < E / 2; ++e) {
@@ -537,8 +537,8 @@ decode_one_bf16s_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
   kap += __shfl_xor_sync(0xffffffffu, kap, 2);
   kap += __shfl_xor_sync(0xffffffffu, kap, 4);
 
-  const float alpha = raw ? alpha_raw(g[bh]) : expf(g[bh]);
-  const float bt = raw ? beta_raw(beta[bh]) : beta[bh];
+  const float alpha = RAW ? alpha_raw(g[bh]) : expf(g[bh]);
+  const float bt = RAW ? beta_raw(beta[bh]) : beta[bh];
   const float2 alpha2 = make_float2(alpha, alpha);
   const size_t row0 = (size_t)bh * DV + warp * ROWS_PER_WARP;  // o and v rows of this warp
   const float vreg = lane < ROWS_PER_WARP ? to_f32(v[row0 + lane]) : 0.f;
@@ -601,11 +601,12 @@ static cudaError_t launch_decode_tokens_t(const void *q, const void *k, const vo
   const T *qt = static_cast<const T *>(q), *kt = static_cast<const T *>(k),
           *vt = static_cast<const T *>(v);
   TO *ot = static_cast<TO *>(o);
-  if (state_dtype == GDN_DTYPE_BF16 && Tn == 1)
-    return launch_pdl(decode_one_bf16s_kernel<T, TO, DK, DV>, blocks, 128, 0, stream, qt, kt, vt,
-                      g, beta, static_cast<const __nv_bfloat16 *>(sin),
-                      static_cast<__nv_bfloat16 *>(sout), src, dst, num_slots, ot, Hqk, Hv, scale,
-                      status, raw);
+  if (state_dtype == GDN_DTYPE_BF16 && Tn == 1)  // the input form is compiled in: registers are tight
+    return launch_pdl(raw ? decode_one_bf16s_kernel<T, TO, DK, DV, true>
+                          : decode_one_bf16s_kernel<T, TO, DK, DV, false>,
+                      blocks, 128, 0, stream, qt, kt, vt, g, beta,
+                      static_cast<const __nv_bfloat16 *>(sin), static_cast<__nv_bfloat16 *>(sout),
+                      src, dst, num_slots, ot, Hqk, Hv, scale, status);
   if (state_dtype == GDN_DTYPE_BF16)
     return launch_pdl(decode_tokens_bf16s_kernel<T, TO, DK, DV>, blocks, 128, 0, stream, qt, kt,
                       vt, g, beta, static_cast<const __nv_bfloat16 *>(sin),

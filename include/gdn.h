@@ -20,17 +20,20 @@
  * 128).
  *
  * Conventions fixed by this library where the pages are silent:
- *   - State layout [num_seqs, Hv, Dv, Dk], fp32, row i = value dim i, Dk
- *     contiguous.  Read u = S k, write v k^T, output S q.
+ *   - State layout [num_seqs, Hv, Dv, Dk], fp32 (or bf16 at rest where a
+ *     state_dtype says so), row i = value dim i, Dk contiguous.  Read u = S k,
+ *     write v k^T, output S q.
  *   - Value head h reads query/key head h / (Hv / Hqk) (contiguous groups);
  *     Hv must be a multiple of Hqk.  No copies are made for the sharing.
  *   - g (= log alpha, <= 0) and beta are fp32, one per (token, value head).
  *   - o_t uses the state after token t.
- *   - q and k are used as given (the caller normalises them).
+ *   - q and k are used as given (the caller normalises them), unless an
+ *     input_form of GDN_INPUT_RAW asks the kernels to do it.
  *
  * Memory.  Every pointer argument except those named "host" is a device
  * pointer (cudaMalloc'd or equivalent) owned by the caller; the library never
- * allocates, frees or keeps a pointer after a call returns.  All arrays are
+ * allocates device memory, frees or keeps a pointer after a call returns (the
+ * pipelined prefill keeps two internal streams and a few events per device).  All arrays are
  * dense row-major with the shapes given below and 16-byte-aligned bases.
  *
  * Ordering.  Every call enqueues work on `stream` (a cudaStream_t; NULL is
@@ -63,10 +66,11 @@ extern "C" {
 #define GDN_ERR_BAD_SEQLENS 5    /* device status: cu_seqlens not 0 = c0 <= c1 .. <= cN = T */
 #define GDN_ERR_WORKSPACE 6      /* workspace missing, misaligned or too small           */
 
-/* Element types of q, k, v (dtype) and of o (o_dtype); g, beta and the state
- * are always fp32.  o_dtype is chosen independently: fp32 o keeps the
- * precision the fp32 state carries (rounding o to bf16 alone costs up to
- * 2^-8 |o| per element). */
+/* Element types of q, k, v (dtype), of o (o_dtype) and of the states kept
+ * between calls (state_dtype, where an entry point takes one; fp32 elsewhere);
+ * g and beta are always fp32.  o_dtype is chosen independently: fp32 o keeps
+ * the precision the fp32 arithmetic carries (rounding o to bf16 alone costs up
+ * to 2^-8 |o| per element). */
 #define GDN_DTYPE_BF16 0
 #define GDN_DTYPE_FP32 1
 

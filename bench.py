@@ -419,10 +419,15 @@ def run_ours(args, D):
 
     if not args.no_cpu_baseline and D.rank == 0 and D.world == 1:
         secs, threads = oracle_prefill_timed(inp, T)
+        n1 = 1024  # one core, a bounded sample: the first 1024 tokens, all heads
+        secs1, _ = oracle_prefill_timed(inp, n1, num_threads=1)
         out["cpu_baseline"] = {"value": T / secs / 1e6, "unit": "Mtok/s", "cores": threads,
                                "kind": "oracle",
                                "sample": f"the whole workload ({T} tokens x {w.Hv} V heads) once, "
-                                         f"{secs:.1f} s wall"}
+                                         f"{secs:.1f} s wall",
+                               "single_core": {"value": n1 / secs1 / 1e6, "unit": "Mtok/s",
+                                               "sample": f"first {n1} tokens x {w.Hv} V heads, "
+                                                         f"1 thread, {secs1:.1f} s wall"}}
     return out
 
 
@@ -619,6 +624,33 @@ def _decode(args, D, dev, peaks, peak_src):
     torch.cuda.synchronize()
     D.barrier()
     ms = D.max(e0.elapsed_time(e1), dev)
+    # The same steps replayed from a CUDA graph of 100 steps (launches with
+    # their programmatic-dependent-launch edges captured; fresh inputs per step).
+    chunk = min(100, steps)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        run(1)  # warm the binding on the capture stream
+    stream.wait_stream(side)
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph):
+        for s_ in range(chunk):
+            api.decode_step(x["q"][s_], x["k"][s_], x["v"][s_], x["g"][s_], x["beta"][s_], S, o=o)
+    graph.replay()
+    torch.cuda.synchronize()
+    reps = max(1, steps // chunk)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier()
+    torch.cuda.synchronize()
+    g0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    g1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    ms_graph = D.max(g0.elapsed_time(g1), dev) / (reps * chunk)
+    del graph
     state_bytes = w.batch * w.Hv * w.D * w.D * 4
     # q, k (bf16) + v (bf16) + o (fp32) + g, beta (fp32)
     io_bytes = w.batch * (2 * w.Hqk * w.D * 2 + w.Hv * w.D * 2 + w.Hv * w.D * 4 + 2 * w.Hv * 4)
@@ -629,6 +661,8 @@ def _decode(args, D, dev, peaks, peak_src):
     return {"value": gbs, "unit": "GB/s", "workload": f"decode64: B={w.batch} x 1 token, Hqk={w.Hqk} "
             f"Hv={w.Hv} D={w.D} bf16, fp32 state {state_bytes} B in place, {steps} steps",
             "us_per_step": us, "steps_per_s": steps / (ms / 1e3),
+            "us_per_step_cuda_graph": ms_graph * 1e3,
+            "value_cuda_graph": D.world * per_step / (ms_graph / 1e3) / 1e9,
             "roofline": {"bound": "hbm", "kernel": "decode_step_kernel", "achieved": gbs / D.world,
                          "peak": peak, "unit": "GB/s", "frac": gbs / D.world / peak,
                          "peak_source": f"{peak_src} hbm_gbs",

@@ -438,46 +438,80 @@ def _tc_path_available():
 
 
 def _e2e(args, D, inp, dev, w, ws):
+    """The prefill through the public API with host buffers: every step copies
+    its inputs from pinned host memory to the device and its o and final state
+    back.  Consecutive steps are pipelined on three streams (upload of step
+    i+1, prefill of step i, download of step i-1) with double-buffered device
+    inputs and outputs, so PCIe's two directions and the GPU work overlap."""
     import torch
 
     from gated_deltanet_recurrence_rule_b200 import api
 
     names = ("q", "k", "v", "g", "beta", "cu_seqlens")
     host = {n: inp[n].pin_memory() for n in names}
-    devb = {n: torch.empty_like(host[n], device=dev) for n in names}
     T = w.total_tokens
-    o_host = torch.empty((T, w.Hv, w.D), dtype=torch.float32).pin_memory()
-    f_host = torch.empty((1, w.Hv, w.D, w.D), dtype=torch.float32).pin_memory()
-    o = torch.empty((T, w.Hv, w.D), dtype=torch.float32, device=dev)
-    fin = torch.empty((1, w.Hv, w.D, w.D), dtype=torch.float32, device=dev)
+    devb = [{n: torch.empty_like(host[n], device=dev) for n in names} for _ in range(2)]
+    o = [torch.empty((T, w.Hv, w.D), dtype=torch.float32, device=dev) for _ in range(2)]
+    fin = [torch.empty((1, w.Hv, w.D, w.D), dtype=torch.float32, device=dev) for _ in range(2)]
+    o_host = [torch.empty((T, w.Hv, w.D), dtype=torch.float32).pin_memory() for _ in range(2)]
+    f_host = [torch.empty((1, w.Hv, w.D, w.D), dtype=torch.float32).pin_memory() for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o_host.numel() * 4 + f_host.numel() * 4
+    d2h = o_host[0].numel() * 4 + f_host[0].numel() * 4
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    ev = lambda: torch.cuda.Event()
+    ev_in, ev_comp, ev_out = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    state = {"i": 0}
 
     def step():
-        for n in names:
-            devb[n].copy_(host[n], non_blocking=True)
-        api.prefill(devb["q"], devb["k"], devb["v"], devb["g"], devb["beta"],
-                    cu_seqlens=devb["cu_seqlens"], final_state=fin, o=o, workspace=ws)
-        o_host.copy_(o, non_blocking=True)
-        f_host.copy_(fin, non_blocking=True)
+        i = state["i"]
+        b = i % 2
+        state["i"] += 1
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[b])           # step i-2 no longer reads devb[b]
+            for n in names:
+                devb[b][n].copy_(host[n], non_blocking=True)
+            ev_in[b].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in[b])
+            if i >= 2:
+                s_comp.wait_event(ev_out[b])          # step i-2's o, final state are on the host
+            x = devb[b]
+            api.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=x["cu_seqlens"],
+                        final_state=fin[b], o=o[b], workspace=ws)
+            ev_comp[b].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[b])
+            o_host[b].copy_(o[b], non_blocking=True)
+            f_host[b].copy_(fin[b], non_blocking=True)
+            ev_out[b].record(s_out)
 
-    for _ in range(max(args.warmup, 3)):
-        step()
+    main = torch.cuda.current_stream(dev)
+
+    def run(n):
+        for st in (s_in, s_comp, s_out):
+            st.wait_stream(main)
+        for _ in range(n):
+            step()
+        for st in (s_in, s_comp, s_out):
+            main.wait_stream(st)
+
+    run(max(args.warmup, 3))
     torch.cuda.synchronize()
-    stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     D.barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(args.steps):
-        step()
-    e1.record(stream)
+    e0.record(main)
+    run(args.steps)
+    e1.record(main)
     torch.cuda.synchronize()
     D.barrier()
     ms = D.max(e0.elapsed_time(e1), dev)
     return {"value": D.world * T * args.steps / (ms / 1e3) / 1e6, "unit": "Mtok/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "ms_per_step": ms / args.steps, "host_buffers": "pinned"}
+            "ms_per_step": ms / args.steps, "host_buffers": "pinned",
+            "pipelined": "upload of step i+1, prefill of step i and download of step i-1 on "
+                         "three streams, device buffers doubled"}
 
 
 def _prefill_raw(args, D, dev, x, T, w, ws, fin, o, flush, prepared_ms, launches):

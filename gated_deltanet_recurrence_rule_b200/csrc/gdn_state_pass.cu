@@ -588,7 +588,7 @@ bool make_qkv_map(CUtensorMap *m, const void *base, int H, int T) {
 
 // Rounds of the pipelined schedule: about kPipeRounds rounds of at least
 // kMinRoundChunks global chunks each, records double-buffered.
-constexpr int64_t kPipeRounds = 8, kMinRoundChunks = 8;
+constexpr int64_t kPipeRounds = 6, kMinRoundChunks = 8;
 
 static int64_t pipelined_round_chunks(int64_t N, int64_t T) {
   const int64_t bound = tp::chunk_bound(N, T);

@@ -46,10 +46,10 @@ def test_status_strings(lib):
 
 def test_workspace_size_rounds(lib):
     """Tensor-core sizes: the full workspace holds two rounds of records (one
-    per chunk and value head, 8 rounds of ceil(129 / 8) = 17 chunks at T=8192);
+    per chunk and value head, 6 rounds of ceil(129 / 6) = 22 chunks at T=8192);
     smaller rounds bound it; CUDA-core sizes need only the header."""
     full = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128)
-    assert 2 * 17 * 48 * 65536 < full < 2 * 18 * 48 * 66560 + (8 << 20)
+    assert 2 * 22 * 48 * 65536 < full < 2 * 23 * 48 * 66560 + (8 << 20)
     r1 = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=1)
     r4 = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=4)
     assert 256 < r1 < r4 < full
@@ -62,9 +62,9 @@ def test_workspace_size_rounds(lib):
 
 def test_launch_count(lib):
     """One launch for the single-pass and CUDA-core kernels; plan + two per
-    round for the two-phase kernels (8 pipelined rounds of 17 chunks at 8k)."""
+    round for the two-phase kernels (6 pipelined rounds of 22 chunks at 8k)."""
     full = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128)
-    assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, full) == 1 + 2 * 8
+    assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, full) == 1 + 2 * 6
     assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, 256) == 1
     one_row = api.prefill_workspace_size(1, 8192, 16, 48, 128, 128, chunks_per_round=1)
     assert api.prefill_launch_count(1, 8192, 16, 48, 128, 128, one_row) == 1 + 2 * 129

@@ -625,7 +625,8 @@ def _backward(args, D, dev, x, T, w, peaks):
                          "frac": achieved / fp32_peak,
                          "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
                          "algorithmic": f"18 D^2 flop per token and value head = {flop} flop",
-                         "traffic": None},
+                         "traffic": kernel_traffic("prefill_backward", [os.path.join(CSRC, n) for n in
+                                                                          ("gdn_common.cuh", "gdn_backward.cu")])},
             "gpu_launches": 5 * steps}  # at these sizes: 4 row slices per head, Hv > Hqk
 
 

@@ -40,13 +40,14 @@ namespace bwd {
 
 constexpr int C = 16;  // tokens per checkpoint chunk
 
-template <int DK, int ROWS>
+template <int DK, int ROWS, int LPR>
 struct Cfg {
-  static constexpr int THREADS = 4 * ROWS;  // 4 lanes per state row
-  static constexpr int CPL = DK / 4;      // columns per lane: 16 m + 4 r4 + (0..3)
+  static constexpr int THREADS = LPR * ROWS;  // LPR lanes per state row
+  static constexpr int CPL = DK / LPR;        // columns per lane: 4 LPR m + 4 r + (0..3)
   static constexpr int NV4 = CPL / 4;
   static constexpr int NW = THREADS / 32;
-  static constexpr int KEEP = CPL / 8;    // columns a lane keeps after the 8-row halving
+  static constexpr int RPW = 32 / LPR;        // rows per warp
+  static constexpr int KEEP = CPL / RPW;      // columns a lane keeps after the row halving
   // shared memory (floats)
   static constexpr int S_Q = 0, S_K = S_Q + C * DK, S_V = S_K + C * DK, S_DO = S_V + C * ROWS;
   static constexpr int S_A = S_DO + C * ROWS, S_B = S_A + C;
@@ -72,53 +73,49 @@ struct Params {
   int32_t *status;
 };
 
-// Column c = 16 m + 4 r4 + q of this lane's row, element e = 4 m + q.
-// Sum v over the 8 rows a warp holds (lane bits 2..4) by recursive halving:
-// at each level a lane keeps half of its elements and adds the partner's copy
-// of them, so afterwards it holds KEEP = CPL / 8 consecutive elements (from
-// keep_e0) summed over the 8 rows, with 7 CPL / 8 shuffles instead of 3 CPL.
-template <int CPL>
-__device__ __forceinline__ void halve8(float (&v)[CPL], int lane) {
-  constexpr int H1 = CPL / 2, H2 = CPL / 4, H3 = CPL / 8;
-  {
-    const bool up = lane & 16;
+// Column c = 4 LPR m + 4 r + q of this lane's row (r = lane % LPR), element
+// e = 4 m + q.  Sum v over the 32 / LPR rows a warp holds (lane bits log2(LPR)
+// .. 4) by recursive halving: at each level a lane keeps half of its elements
+// and adds the partner's copy of them, so afterwards it holds CPL / (32 / LPR)
+// consecutive elements (from keep_e0) summed over the warp's rows, with far
+// fewer shuffles than one reduction per element.
+template <int CPL, int LPR>
+__device__ __forceinline__ void halve_rows(float (&v)[CPL], int lane) {
+  int width = CPL;
 #pragma unroll
-    for (int e = 0; e < H1; ++e) {
-      const float mine = up ? v[H1 + e] : v[e], other = up ? v[e] : v[H1 + e];
-      v[e] = mine + __shfl_xor_sync(0xffffffffu, other, 16);
-    }
-  }
-  {
-    const bool up = lane & 8;
+  for (int b = 16; b >= LPR; b >>= 1) {
+    width >>= 1;
+    const bool up = lane & b;
 #pragma unroll
-    for (int e = 0; e < H2; ++e) {
-      const float mine = up ? v[H2 + e] : v[e], other = up ? v[e] : v[H2 + e];
-      v[e] = mine + __shfl_xor_sync(0xffffffffu, other, 8);
-    }
-  }
-  {
-    const bool up = lane & 4;
-#pragma unroll
-    for (int e = 0; e < H3; ++e) {
-      const float mine = up ? v[H3 + e] : v[e], other = up ? v[e] : v[H3 + e];
-      v[e] = mine + __shfl_xor_sync(0xffffffffu, other, 4);
+    for (int e = 0; e < CPL / 2; ++e) {
+      if (e < width) {
+        const float mine = up ? v[width + e] : v[e], other = up ? v[e] : v[width + e];
+        v[e] = mine + __shfl_xor_sync(0xffffffffu, other, b);
+      }
     }
   }
 }
-// First element index (4 m + q) a lane keeps after halve8.
-template <int CPL>
+// First element index (4 m + q) a lane keeps after halve_rows.
+template <int CPL, int LPR>
 __device__ __forceinline__ int keep_e0(int lane) {
-  return (CPL / 2) * ((lane >> 4) & 1) + (CPL / 4) * ((lane >> 3) & 1) + (CPL / 8) * ((lane >> 2) & 1);
+  int e0 = 0, width = CPL;
+#pragma unroll
+  for (int b = 16; b >= LPR; b >>= 1) {
+    width >>= 1;
+    if (lane & b) e0 += width;
+  }
+  return e0;
 }
 
-template <typename T, int DK, int ROWS>
-__global__ void __launch_bounds__(4 * ROWS, ROWS == 128 ? 1 : 2)
+template <typename T, int DK, int ROWS, int LPR>
+__global__ void __launch_bounds__(LPR * ROWS, LPR * ROWS >= 512 ? 1 : 2)
 backward_kernel(const Params p) {
-  using CF = Cfg<DK, ROWS>;
+  using CF = Cfg<DK, ROWS, LPR>;
   constexpr int CPL = CF::CPL, NV4 = CF::NV4, NW = CF::NW, KEEP = CF::KEEP;
+  constexpr int CS = 4 * LPR;  // column stride between a lane's float4s
   extern __shared__ __align__(16) float sm[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = tid >> 2, r4 = tid & 3;  // row within the slice
+  const int row = tid / LPR, r4 = tid % LPR;  // row within the slice, lane within the row
   const int unit = blockIdx.x / p.R, slice = blockIdx.x - unit * p.R;
   const int n = unit / p.Hv, h = unit - n * p.Hv;
   const int j = h / (p.Hv / p.Hqk);
@@ -174,12 +171,12 @@ backward_kernel(const Params p) {
     float a = 0.f;
 #pragma unroll
     for (int m = 0; m < NV4; ++m) {
-      const float4 y = *reinterpret_cast<const float4 *>(vec + 16 * m + 4 * r4);
+      const float4 y = *reinterpret_cast<const float4 *>(vec + CS * m + 4 * r4);
       a = fmaf(x[4 * m], y.x, a); a = fmaf(x[4 * m + 1], y.y, a);
       a = fmaf(x[4 * m + 2], y.z, a); a = fmaf(x[4 * m + 3], y.w, a);
     }
-    a += __shfl_xor_sync(0xffffffffu, a, 1);
-    a += __shfl_xor_sync(0xffffffffu, a, 2);
+#pragma unroll
+    for (int off = 1; off < LPR; off <<= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
     return a;
   };
   auto step = [&](float (&S)[CPL], int t) {  // S <- S_t from S_{t-1}
@@ -188,7 +185,7 @@ backward_kernel(const Params p) {
     const float w = sb[t] * (sv[t * ROWS + row] - sa[t] * u);
 #pragma unroll
     for (int m = 0; m < NV4; ++m) {
-      const float4 y = *reinterpret_cast<const float4 *>(kt + 16 * m + 4 * r4);
+      const float4 y = *reinterpret_cast<const float4 *>(kt + CS * m + 4 * r4);
       S[4 * m] = fmaf(sa[t], S[4 * m], w * y.x); S[4 * m + 1] = fmaf(sa[t], S[4 * m + 1], w * y.y);
       S[4 * m + 2] = fmaf(sa[t], S[4 * m + 2], w * y.z); S[4 * m + 3] = fmaf(sa[t], S[4 * m + 3], w * y.w);
     }
@@ -199,7 +196,7 @@ backward_kernel(const Params p) {
 #pragma unroll
   for (int m = 0; m < NV4; ++m) {
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (p.s0) x = *reinterpret_cast<const float4 *>(p.s0 + srow + 16 * m + 4 * r4);
+    if (p.s0) x = *reinterpret_cast<const float4 *>(p.s0 + srow + CS * m + 4 * r4);
     S[4 * m] = x.x; S[4 * m + 1] = x.y; S[4 * m + 2] = x.z; S[4 * m + 3] = x.w;
   }
   for (int c = 0; c < nck; ++c) {
@@ -216,7 +213,7 @@ backward_kernel(const Params p) {
 #pragma unroll
   for (int m = 0; m < NV4; ++m) {
     float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (p.dSfin) x = *reinterpret_cast<const float4 *>(p.dSfin + srow + 16 * m + 4 * r4);
+    if (p.dSfin) x = *reinterpret_cast<const float4 *>(p.dSfin + srow + CS * m + 4 * r4);
     G[4 * m] = x.x; G[4 * m + 1] = x.y; G[4 * m + 2] = x.z; G[4 * m + 3] = x.w;
   }
   float *red = sm + CF::S_RED, *rs = sm + CF::S_RS;
@@ -251,13 +248,13 @@ backward_kernel(const Params p) {
       const float w = sv[t * ROWS + row] - alpha * u;  // v - alpha u (beta applied where used)
       const float sdO = p.scale * sdo[t * ROWS + row], bw = bt * w;
       float *rb = red + parity * 2 * NW * DK;
-      const int e0 = keep_e0<CPL>(lane);
+      const int e0 = keep_e0<CPL, LPR>(lane);
       float tmp[CPL];
       // G += scale dO q^T;  dq partial = scale dO_i S_t[i, :],  S_t = alpha S_{t-1} + beta w k^T
 #pragma unroll
       for (int m = 0; m < NV4; ++m) {
-        const float4 a = *reinterpret_cast<const float4 *>(kt + 16 * m + 4 * r4);
-        const float4 b = *reinterpret_cast<const float4 *>(qt + 16 * m + 4 * r4);
+        const float4 a = *reinterpret_cast<const float4 *>(kt + CS * m + 4 * r4);
+        const float4 b = *reinterpret_cast<const float4 *>(qt + CS * m + 4 * r4);
         const float kk[4] = {a.x, a.y, a.z, a.w}, qq[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
@@ -265,11 +262,11 @@ backward_kernel(const Params p) {
           tmp[4 * m + x] = sdO * fmaf(alpha, Sp[4 * m + x], bw * kk[x]);
         }
       }
-      halve8<CPL>(tmp, lane);
+      halve_rows<CPL, LPR>(tmp, lane);
 #pragma unroll
       for (int x = 0; x < KEEP; ++x) {
         const int e = e0 + x;
-        rb[warp * DK + 16 * (e >> 2) + 4 * r4 + (e & 3)] = tmp[x];
+        rb[warp * DK + CS * (e >> 2) + 4 * r4 + (e & 3)] = tmp[x];
       }
       float sgs = 0.f;
 #pragma unroll
@@ -279,11 +276,11 @@ backward_kernel(const Params p) {
       const float abg = alpha * bt * gk;
 #pragma unroll
       for (int e = 0; e < CPL; ++e) tmp[e] = fmaf(bw, G[e], -abg * Sp[e]);
-      halve8<CPL>(tmp, lane);
+      halve_rows<CPL, LPR>(tmp, lane);
 #pragma unroll
       for (int x = 0; x < KEEP; ++x) {
         const int e = e0 + x;
-        rb[NW * DK + warp * DK + 16 * (e >> 2) + 4 * r4 + (e & 3)] = tmp[x];
+        rb[NW * DK + warp * DK + CS * (e >> 2) + 4 * r4 + (e & 3)] = tmp[x];
       }
       if (r4 == 0) p.dv[(tg * p.Hv + h) * DV + rowg] = bt * gk;
       // scalars: <G, S_{t-1}> (every lane), (G k) . u and w . (G k) (one lane per row)
@@ -301,7 +298,7 @@ backward_kernel(const Params p) {
       const float bgk = bt * gk;
 #pragma unroll
       for (int m = 0; m < NV4; ++m) {
-        const float4 a = *reinterpret_cast<const float4 *>(kt + 16 * m + 4 * r4);
+        const float4 a = *reinterpret_cast<const float4 *>(kt + CS * m + 4 * r4);
         G[4 * m] = alpha * fmaf(-bgk, a.x, G[4 * m]);
         G[4 * m + 1] = alpha * fmaf(-bgk, a.y, G[4 * m + 1]);
         G[4 * m + 2] = alpha * fmaf(-bgk, a.z, G[4 * m + 2]);
@@ -335,7 +332,7 @@ backward_kernel(const Params p) {
   if (p.ds0) {
 #pragma unroll
     for (int m = 0; m < NV4; ++m)
-      *reinterpret_cast<float4 *>(p.ds0 + srow + 16 * m + 4 * r4) =
+      *reinterpret_cast<float4 *>(p.ds0 + srow + CS * m + 4 * r4) =
           make_float4(G[4 * m], G[4 * m + 1], G[4 * m + 2], G[4 * m + 3]);
   }
 }
@@ -381,8 +378,11 @@ size_t backward_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, int Dk, i
 
 template <typename T, int DK, int ROWS>
 static cudaError_t launch_bwd_t(const bwd::Params &prm, cudaStream_t stream) {
-  using CF = bwd::Cfg<DK, ROWS>;
-  auto kern = bwd::backward_kernel<T, DK, ROWS>;
+  // 8 lanes per row for slices of up to 64 rows (twice the warps of 4 lanes for
+  // this latency-bound walk), 4 for whole 128-row heads (registers)
+  constexpr int LPR = ROWS <= 64 ? 8 : 4;
+  using CF = bwd::Cfg<DK, ROWS, LPR>;
+  auto kern = bwd::backward_kernel<T, DK, ROWS, LPR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)CF::SMEM);
   if (e != cudaSuccess) return e;
   kern<<<(unsigned)prm.N * (unsigned)prm.Hv * (unsigned)prm.R, CF::THREADS, CF::SMEM, stream>>>(prm);

@@ -66,6 +66,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--no-backward", action="store_true", help="skip the backward-pass leg")
+    p.add_argument("--varlen", action="store_true",
+                   help="add a leg on the varlen32 workload (32 sequences, ~556k tokens, ~20 GB)")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -406,6 +408,8 @@ def run_ours(args, D):
 
     if not args.no_backward:
         out["prefill_backward"] = _backward(args, D, dev, x, T, w, peaks)
+    if args.varlen:
+        out["prefill_varlen32"] = _varlen(args, D, dev, peaks)
 
     if not args.no_decode:
         out["decode"] = _decode(args, D, dev, peaks, peak_src)
@@ -569,6 +573,55 @@ def _prefill_raw(args, D, dev, x, T, w, ws, fin, o, flush, prepared_ms, launches
             "ms_per_step": res["fused"], "prepared_inputs_ms_per_step": prepared_ms,
             "separate_torch_prologue_ms_per_step": res["separate"],
             "l2": "flushed between timed steps", "gpu_launches": args.steps * launches}
+
+
+def _varlen(args, D, dev, peaks):
+    """The prefill on the varlen32 workload: 32 packed sequences of 1k to 32k
+    tokens with their own initial states, final states returned.  Unlike
+    prefill8k (one chain of chunks per value head) it gives the state pass many
+    chains at once, so it shows what the two phases cost in SM time."""
+    import torch
+
+    from gated_deltanet_recurrence_rule_b200 import api, inputs
+
+    w = inputs.WORKLOADS["varlen32"]
+    inp = inputs.workload_inputs(w)
+    x = {n: t.to(dev) for n, t in inp.items() if t is not None}
+    T, N = w.total_tokens, len(w.lengths)
+    o = torch.empty((T, w.Hv, w.D), dtype=torch.float32, device=dev)
+    fin = torch.empty((N, w.Hv, w.D, w.D), dtype=torch.float32, device=dev)
+    ws = torch.zeros(api.prefill_workspace_size(N, T, w.Hqk, w.Hv, w.D, w.D), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        api.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=x["cu_seqlens"],
+                    initial_state=x["initial_state"], final_state=fin, o=o, workspace=ws)
+
+    step()
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 3))
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    D.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    ms = D.max(e0.elapsed_time(e1), dev) / steps
+    if api.get_device_status(ws) != api.GDN_OK:
+        raise RuntimeError("device status after the varlen leg")
+    hbm_bytes = BYTES_PER_TOKEN * T + 2 * N * w.Hv * w.D * w.D * 4
+    gbs = hbm_bytes / (ms / 1e3) / 1e9
+    return {"value": D.world * T / (ms / 1e3) / 1e6, "unit": "Mtok/s", "ms_per_step": ms,
+            "workload": f"varlen32: N={N} T={T} Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16, fp32 o, "
+                        "N(0,0.02) initial states, final states returned",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"],
+                         "algorithmic": f"{BYTES_PER_TOKEN} B/token x {T} + initial and final states"},
+            "gpu_launches": steps * api.prefill_launch_count(N, T, w.Hqk, w.Hv, w.D, w.D, ws.numel())}
 
 
 def _backward(args, D, dev, x, T, w, peaks):

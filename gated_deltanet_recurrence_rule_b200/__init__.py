@@ -6,14 +6,21 @@ the seeded input generator.  Importing the package does not load the CUDA
 library; the first call does, and fails loudly if it is missing.
 """
 from .api import (  # noqa: F401
+    GDN_INPUT_PREPARED,
+    GDN_INPUT_RAW,
     GDNError,
     decode_step,
+    decode_tokens,
     get_device_status,
     lib_path,
     prefill,
+    prefill_backward,
+    prefill_backward_workspace_size,
+    prefill_launch_count,
     prefill_uses_tensor_cores,
     prefill_workspace_size,
 )
 
-__all__ = ["prefill", "decode_step", "prefill_workspace_size", "prefill_uses_tensor_cores", "get_device_status", "GDNError",
-           "lib_path"]
+__all__ = ["prefill", "prefill_backward", "decode_step", "decode_tokens", "prefill_workspace_size",
+           "prefill_backward_workspace_size", "prefill_launch_count", "prefill_uses_tensor_cores",
+           "get_device_status", "GDNError", "GDN_INPUT_PREPARED", "GDN_INPUT_RAW", "lib_path"]

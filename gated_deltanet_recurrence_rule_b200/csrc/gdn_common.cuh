@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 #include "gdn.h"
@@ -90,6 +91,33 @@ __host__ auto dispatch_types(int dtype, int o_dtype, F &&f) {
   }
   if (o_dtype == GDN_DTYPE_BF16) return f(float{}, __nv_bfloat16{});
   return f(float{}, float{});
+}
+
+// ---- host-side caches ----------------------------------------------------------
+// A kernel's dynamic shared memory limit is set once per device (the attribute
+// persists); later calls skip the runtime call.  `flags` is one static array
+// per kernel, indexed by device.
+template <typename K>
+__host__ cudaError_t set_smem_once(K kernel, int bytes, std::atomic<bool> (&flags)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && flags[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev >= 0 && dev < 64) flags[dev].store(true, std::memory_order_release);
+  return e;
+}
+// Multiprocessor count of the current device, queried once per device.
+__host__ inline int sm_count() {
+  static std::atomic<int> counts[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  int n = counts[dev].load(std::memory_order_acquire);
+  if (n == 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    counts[dev].store(n, std::memory_order_release);
+  }
+  return n;
 }
 
 // ---- programmatic dependent launch ------------------------------------------

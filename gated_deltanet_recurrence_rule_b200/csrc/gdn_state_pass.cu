@@ -563,15 +563,18 @@ using EncodeFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, vo
                               CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeFn encode_fn() {
-  static EncodeFn fn = nullptr;
-  if (!fn) {
+  static std::atomic<EncodeFn> fn{nullptr};
+  EncodeFn f = fn.load(std::memory_order_acquire);
+  if (!f) {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeFn>(ptr);
+        q == cudaDriverEntryPointSuccess) {
+      f = reinterpret_cast<EncodeFn>(ptr);
+      fn.store(f, std::memory_order_release);
+    }
   }
-  return fn;
+  return f;
 }
 
 bool make_qkv_map(CUtensorMap *m, const void *base, int H, int T) {
@@ -626,7 +629,8 @@ template <typename TO>
 static cudaError_t launch_state_pass(const CUtensorMap &mq, const CUtensorMap &mk,
                                      const sp::Params &prm, int grid_x, cudaStream_t stream) {
   auto kern = sp::state_pass_kernel<TO>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, sp::SMEM_BYTES);
+  static std::atomic<bool> smem_set[64];
+  cudaError_t e = set_smem_once(kern, (int)sp::SMEM_BYTES, smem_set);
   if (e != cudaSuccess) return e;
   kern<<<dim3((unsigned)grid_x, (unsigned)prm.Hv), sp::NTHREADS, sp::SMEM_BYTES, stream>>>(mq, mk, prm);
   return cudaGetLastError();

@@ -396,17 +396,15 @@ cudaError_t launch_wy_prep(const CUtensorMap &mq, const CUtensorMap &mk, const C
   wy::Params prm;
   prm.g = g; prm.beta = beta; prm.cu = cu; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.raw = raw;
   prm.round = round; prm.rc = rc;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  prm.resident = 2 * sms;
+  prm.resident = 2 * sm_count();
   unsigned char *ws = static_cast<unsigned char *>(const_cast<void *>(workspace));
   prm.plan = reinterpret_cast<const tp::PlanHeader *>(ws + tp::kPlanHeaderOffset);
   prm.ne_seq = reinterpret_cast<const int32_t *>(ws + L.plan_off);
   prm.ne_cs = prm.ne_seq + L.n_ne_capacity;
   prm.rec = rec;
   prm.status = reinterpret_cast<int32_t *>(ws);
-  cudaError_t e = cudaFuncSetAttribute(wy::wy_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       wy::SMEM_BYTES);
+  static std::atomic<bool> smem_set[64];
+  cudaError_t e = set_smem_once(wy::wy_prep_kernel, (int)wy::SMEM_BYTES, smem_set);
   if (e != cudaSuccess) return e;
   wy::wy_prep_kernel<<<dim3((unsigned)rc, (unsigned)Hv), wy::NTHREADS, wy::SMEM_BYTES, stream>>>(
       mq, mk, mv, prm);

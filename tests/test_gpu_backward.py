@@ -13,9 +13,11 @@ DEV = torch.device("cuda:0")
 TOL = 1e-4  # fp32 arithmetic against fp64 on the same inputs: max|err| / RMS(ref) per gradient
 
 
-def _case(lengths, Hqk, Hv, D, dtype, seed, init=True, dsf=True, scale=0.5):
+def _case(lengths, Hqk, Hv, D, dtype, seed, init=True, dsf=True, scale=0.5, edit=None):
     inp = inputs.prefill_inputs(lengths, Hqk, Hv, D, dtype=dtype, seed=seed,
                                 init_std=0.1 if init else 0.0)
+    if edit is not None:
+        edit(inp)
     T, N = sum(lengths), len(lengths)
     gen = torch.Generator().manual_seed(seed + 700)
     d_o = torch.randn(T, Hv, D, generator=gen)
@@ -44,6 +46,19 @@ def _check(out, ref, what):
 def test_backward_varlen_gqa(dtype, D):
     out, ref = _case([37, 0, 50, 16], 2, 6, D, dtype, seed=101 + D)
     _check(out, ref, f"{dtype} D={D}")
+
+
+def test_backward_degenerate_gates():
+    """alpha = 0 (g = -inf) on single tokens, at the first and last token of a
+    16-token checkpoint interval and on a run; g = 0 on a stretch; beta = 0 and
+    beta = 1 on others."""
+    def edit(inp):
+        inp["g"][[0, 5, 15, 16, 17, 18, 60, 75]] = -float("inf")
+        inp["g"][30:45] = 0.0
+        inp["beta"][[3, 4, 50, 80]] = 0.0
+        inp["beta"][[7, 33, 90]] = 1.0
+    out, ref = _case([70, 40], 2, 6, 64, "fp32", seed=111, edit=edit)
+    _check(out, ref, "gates")
 
 
 def test_backward_mixed_dims():

@@ -124,6 +124,40 @@ def test_bf16_state_against_oracle(dtype, D, Tn):
     assert torch.equal(pin.cpu(), pool)
 
 
+@pytest.mark.parametrize("sdt", ["fp32", "bf16"])
+@pytest.mark.parametrize("Tn", [1, 4])
+def test_degenerate_gates(sdt, Tn):
+    """alpha = 0 (g = -inf, the state resets), g = 0, beta = 0 and beta = 1 on
+    chosen (sequence, token) pairs, against the oracle, on the fp32-pool and
+    bf16-pool kernels."""
+    B, Hqk, Hv, D, slots = 4, 2, 6, 128, 4
+    inp, x, pool = _case(B, Tn, Hqk, Hv, D, "bf16", seed=81 + Tn, num_slots=slots)
+    g, beta = inp["g"].view(B, Tn, Hv), inp["beta"].view(B, Tn, Hv)
+    g[0, 0] = -float("inf")
+    g[1, Tn - 1] = -float("inf")
+    g[2] = 0.0
+    beta[1, 0] = 0.0
+    beta[2, Tn - 1] = 1.0
+    beta[3] = 0.0
+    if sdt == "bf16":
+        pool = pool.to(torch.bfloat16)
+    src = [0, 1, 2, 3]
+    S = pool.to(DEV)
+    o = api.decode_tokens(*(x[n].to(DEV) for n in ("q", "k", "v", "g", "beta")), S)
+    torch.cuda.synchronize()
+    o_gpu = to_np(o).reshape(B * Tn, Hv, D)
+    assert np.isfinite(o_gpu).all() and torch.isfinite(S.float()).all()
+    if sdt == "fp32":
+        o_ref, f_ref = _oracle(inp, pool, src)
+        assert_parity(torch.bfloat16, o_gpu, o_ref, to_np(S), f_ref, f"gates fp32 pool Tn={Tn}")
+    else:
+        o_ref, f_ref = _oracle(inp, pool, src, state_at_rest="bf16")
+        _, f_exact = _oracle(inp, pool, src)
+        assert_parity(torch.bfloat16, o_gpu, o_ref, what=f"gates bf16 pool Tn={Tn}")
+        assert state_error_bf16_rest(to_np(S), f_ref) <= 1.0
+        assert state_error(to_np(S), f_exact) <= 5e-3
+
+
 def test_bf16_state_many_calls():
     """64 one-token calls and 16 four-token calls in place on a bf16 pool, each
     followed on the oracle by one rounding of the state: the two stay within the

@@ -93,6 +93,27 @@ def test_reset_and_no_write_edges():
     assert_parity(torch.float32, to_np(o), o_ref, to_np(f), f_ref, "edges")
 
 
+@pytest.mark.parametrize("path", ["cuda_cores", "two_phase", "single_pass"])
+def test_degenerate_gates(path):
+    """alpha = 0 (g = -inf, the state resets) on single tokens, on the first and
+    last token of a chunk and on a run of tokens; g = 0 (no decay) on a
+    stretch; beta = 0 (no write) and beta = 1 (the key direction is replaced)
+    on others; in both sequences of a packed batch, on every prefill path."""
+    dtype = "fp32" if path == "cuda_cores" else "bf16"
+    inp = inputs.prefill_inputs([260, 70], 2, 6, 128, dtype=dtype, seed=31, init_std=0.1)
+    inp["g"][[3, 64, 127, 128, 129, 130, 200, 261]] = -float("inf")
+    inp["g"][140:180] = 0.0
+    inp["beta"][[10, 11, 70, 262]] = 0.0
+    inp["beta"][[20, 90, 191, 300]] = 1.0
+    if path == "single_pass":
+        o, f = _run_ws(inp, torch.zeros(256, dtype=torch.uint8, device=DEV))
+    else:
+        o, f = run_gpu(inp)
+    o_ref, f_ref = run_oracle(inp)
+    assert np.isfinite(to_np(o)).all() and np.isfinite(to_np(f)).all()
+    assert_parity(inputs.DTYPES[dtype], to_np(o), o_ref, to_np(f), f_ref, f"gates {path}")
+
+
 def test_bad_cu_seqlens_sets_device_status():
     inp = inputs.prefill_inputs([64, 64], 2, 6, 64, dtype="bf16", seed=16)
     dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}

@@ -68,3 +68,57 @@ def test_capture_and_replay_match_eager():
     assert torch.equal(graphed[2], eager[2]) and torch.equal(pool_g, pool_e)
     for name in ("dq", "dk", "dv", "dg", "db", "ds0"):
         assert torch.equal(graphed[3][name], eager[3][name]), name
+
+
+def test_serving_loop_replays():
+    """A serving loop's graph: raw-input prefill into bf16 states, then decode
+    steps on fp32 states and one-token calls on a bf16 pool, both in place.
+    Replayed three times, the graph gives the same bits as three rounds of the
+    eager calls (the in-place states advance on every replay)."""
+    B, Hqk, Hv, D = 4, 2, 6, 128
+    pin = inputs.prefill_inputs([200, 64], Hqk, Hv, D, dtype="bf16", seed=94, init_std=0.1)
+    x = {n: t.to(DEV) for n, t in pin.items()}
+    T, N = x["q"].shape[0], 2
+    s0 = x["initial_state"].to(torch.bfloat16)
+    ws = torch.zeros(api.prefill_workspace_size(N, T, Hqk, Hv, D, D), dtype=torch.uint8, device=DEV)
+    dx = inputs.prefill_inputs([1] * B, Hqk, Hv, D, dtype="bf16", seed=95)
+    d = {n: dx[n].to(DEV) for n in ("q", "k", "v", "g", "beta")}
+    gen = torch.Generator().manual_seed(96)
+    st0 = (torch.randn(B, Hv, D, D, generator=gen) * 0.3).to(DEV)
+    pool0 = st0.to(torch.bfloat16)
+    dt = {n: t.view(B, 1, *t.shape[1:]) for n, t in d.items()}
+
+    def buffers():
+        return {"o": torch.empty(T, Hv, D, device=DEV),
+                "f": torch.empty(N, Hv, D, D, dtype=torch.bfloat16, device=DEV),
+                "S": st0.clone(), "pool": pool0.clone(),
+                "od": torch.empty(B, Hv, D, device=DEV), "ot": torch.empty(B, 1, Hv, D, device=DEV)}
+
+    def calls(b):
+        api.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=x["cu_seqlens"],
+                    initial_state=s0, final_state=b["f"], o=b["o"], workspace=ws, raw_inputs=True)
+        api.decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], b["S"], o=b["od"])
+        api.decode_tokens(dt["q"], dt["k"], dt["v"], dt["g"], dt["beta"], b["pool"], o=b["ot"])
+
+    eager = buffers()
+    for _ in range(3):
+        calls(eager)
+    torch.cuda.synchronize()
+
+    graphed = buffers()
+    side = torch.cuda.Stream(DEV)
+    side.wait_stream(torch.cuda.current_stream(DEV))
+    with torch.cuda.stream(side):  # warm-up off the capture, on copies of the states
+        warm = buffers()
+        calls(warm)
+    torch.cuda.current_stream(DEV).wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        calls(graphed)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    assert api.get_device_status(ws) == api.GDN_OK
+    for name in ("o", "f", "S", "pool", "od", "ot"):
+        assert torch.equal(graphed[name], eager[name]), name

@@ -618,7 +618,8 @@ def _varlen(args, D, dev, peaks):
     """The prefill on the varlen32 workload: 32 packed sequences of 1k to 32k
     tokens with their own initial states, final states returned.  Unlike
     prefill8k (one chain of chunks per value head) it gives the state pass many
-    chains at once, so it shows what the two phases cost in SM time."""
+    chains at once, so it shows what the two phases cost in SM time.  The
+    single-pass kernel (chosen by a header-only workspace) is timed beside it."""
     import torch
 
     from gated_deltanet_recurrence_rule_b200 import api, inputs
@@ -629,29 +630,34 @@ def _varlen(args, D, dev, peaks):
     T, N = w.total_tokens, len(w.lengths)
     o = torch.empty((T, w.Hv, w.D), dtype=torch.float32, device=dev)
     fin = torch.empty((N, w.Hv, w.D, w.D), dtype=torch.float32, device=dev)
-    ws = torch.zeros(api.prefill_workspace_size(N, T, w.Hqk, w.Hv, w.D, w.D), dtype=torch.uint8,
-                     device=dev)
-
-    def step():
-        api.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=x["cu_seqlens"],
-                    initial_state=x["initial_state"], final_state=fin, o=o, workspace=ws)
-
-    step()
-    torch.cuda.synchronize()
+    full = torch.zeros(api.prefill_workspace_size(N, T, w.Hqk, w.Hv, w.D, w.D), dtype=torch.uint8,
+                       device=dev)
+    header = torch.zeros(256, dtype=torch.uint8, device=dev)  # selects the single-pass kernel
     steps = max(1, min(args.steps, 3))
     stream = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    D.barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
+
+    def timed(ws):
+        def step():
+            api.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=x["cu_seqlens"],
+                        initial_state=x["initial_state"], final_state=fin, o=o, workspace=ws)
+
         step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    D.barrier()
-    ms = D.max(e0.elapsed_time(e1), dev) / steps
-    if api.get_device_status(ws) != api.GDN_OK:
-        raise RuntimeError("device status after the varlen leg")
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        D.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        D.barrier()
+        if api.get_device_status(ws) != api.GDN_OK:
+            raise RuntimeError("device status after the varlen leg")
+        return D.max(e0.elapsed_time(e1), dev) / steps
+
+    ms = timed(full)
+    ms_single = timed(header)
     hbm_bytes = BYTES_PER_TOKEN * T + 2 * N * w.Hv * w.D * w.D * 4
     gbs = hbm_bytes / (ms / 1e3) / 1e9
     return {"value": D.world * T / (ms / 1e3) / 1e6, "unit": "Mtok/s", "ms_per_step": ms,
@@ -660,7 +666,11 @@ def _varlen(args, D, dev, peaks):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"],
                          "algorithmic": f"{BYTES_PER_TOKEN} B/token x {T} + initial and final states"},
-            "gpu_launches": steps * api.prefill_launch_count(N, T, w.Hqk, w.Hv, w.D, w.D, ws.numel())}
+            "gpu_launches": steps * api.prefill_launch_count(N, T, w.Hqk, w.Hv, w.D, w.D, full.numel()),
+            "single_pass": {"value": D.world * T / (ms_single / 1e3) / 1e6, "unit": "Mtok/s",
+                            "ms_per_step": ms_single,
+                            "how": "the same call with a 256-byte workspace: one CTA per (sequence, "
+                                   "value head) runs all its chunks"}}
 
 
 def _backward(args, D, dev, x, T, w, peaks):

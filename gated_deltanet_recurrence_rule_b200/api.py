@@ -151,6 +151,11 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, output_final_
     dtype of the given states, else ``state_dtype`` (default fp32).
     ``raw_inputs``: q, k are raw projections (normalised in the kernels) and
     g, beta hold a, b with g = -softplus(a), beta = sigmoid(b).
+    ``workspace``: a zero-filled uint8 CUDA tensor, reused across calls, or
+    None (one of ``prefill_workspace_size`` bytes is allocated).  Its size
+    selects the tensor-core schedule: full size runs the two phases; a
+    256-byte one runs the single-pass kernel, which is faster for batches of
+    many sequences of similar length and slower for a few long ones.
     Returns (o [T, Hv, Dv], final_state or None).
     """
     lib = load()

@@ -10,8 +10,13 @@ state returned), captured once in a CUDA graph and replayed; the same call
 launched eagerly is reported beside it (``eager``).  ``value`` is prefill
 throughput in Mtok/s with the inputs resident in HBM, L2 flushed between timed
 steps.  The same line carries:
-  roofline     the prefill kernel against its bound (algorithmic flops or bytes
-               per launch / CUDA-event launch time, over the measured peak);
+  roofline     the prefill call against the tensor-core roofline (algorithmic
+               flops / CUDA-event time over the measured bf16 peak), with the
+               HBM fractions for fp32 o and for bf16 o beside it;
+  prefill_long262k, prefill_varlen32
+               the prefill on the long-context (262,144 tokens, slow decay,
+               nonzero initial state updated in place) and the variable-length
+               (32 packed sequences) workloads, each with its own roofline;
   decode       the batched decode workload (B=64, 1000 steps, fp32 state of
                201 MB updated in place): state GB/s against HBM peak;
   decode_tokens  the same batch with 4 tokens per sequence per call through the
@@ -41,7 +46,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -57,6 +61,8 @@ if ROOT not in sys.path:
 #   = 45,440 per token.
 FLOP_PER_TOKEN = 7_602_176
 BYTES_PER_TOKEN = 45_440
+# The same with o in bf16 (the input dtype): o 12288 B/token instead of 24576.
+BYTES_PER_TOKEN_BF16_O = 33_152
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -68,8 +74,8 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--no-backward", action="store_true", help="skip the backward-pass leg")
-    p.add_argument("--varlen", action="store_true",
-                   help="add a leg on the varlen32 workload (32 sequences, ~556k tokens, ~20 GB)")
+    p.add_argument("--no-long", action="store_true",
+                   help="skip the long262k and varlen32 prefill legs (~20 GB of device memory)")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -381,22 +387,7 @@ def run_ours(args, D):
     kernel_ms = statistics.mean(graph_per_ms)
     launches = api.prefill_launch_count(1, T, w.Hqk, w.Hv, w.D, w.D, ws.numel())
     if _tc_path_available():
-        # Time floors of the two bounds; the larger one binds.
-        flops = FLOP_PER_TOKEN * T
-        hbm_bytes = BYTES_PER_TOKEN * T + w.Hv * w.D * w.D * 4
-        t_tensor = flops / (peaks["bf16_tflops"] * 1e12)
-        t_hbm = hbm_bytes / (peaks["hbm_gbs"] * 1e9)
-        tensor_ach = flops / (kernel_ms / 1e3) / 1e12
-        hbm_ach = hbm_bytes / (kernel_ms / 1e3) / 1e9
-        if t_hbm >= t_tensor:
-            roof = {"bound": "hbm", "achieved": hbm_ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": hbm_ach / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs",
-                    "algorithmic": f"{BYTES_PER_TOKEN} B/token x {T} tokens + final state"}
-        else:
-            roof = {"bound": "tensor", "achieved": tensor_ach, "peak": peaks["bf16_tflops"],
-                    "unit": "TFLOP/s", "frac": tensor_ach / peaks["bf16_tflops"],
-                    "peak_source": f"{peak_src} bf16_tflops (burst)",
-                    "algorithmic": f"{FLOP_PER_TOKEN} flop/token x {T} tokens"}
+        roof = prefill_roofline(T, w.Hv, w.D, kernel_ms, peaks, peak_src, state_io=1)
         # One prefill call is a sequence of launches (plan, then WY prep and
         # state pass per round, on two streams, rounds pipelined): the time is
         # the whole call's, between CUDA events on the caller's stream that
@@ -405,9 +396,6 @@ def run_ours(args, D):
         roof.update({"kernel": f"prefill step: plan_kernel + wy_prep_kernel and state_pass_kernel "
                                f"per round ({launches} launches, 2 streams, pipelined)",
                      "kernel_ms": kernel_ms,
-                     "tensor_frac": tensor_ach / peaks["bf16_tflops"],
-                     "tensor_achieved_tflops": tensor_ach, "hbm_frac": hbm_ach / peaks["hbm_gbs"],
-                     "floor_us": {"tensor": t_tensor * 1e6, "hbm": t_hbm * 1e6},
                      "traffic": None if ent is None else ent["dram_bytes_per_launch"],
                      "dominant": None if ent is None else ent.get("dominant")})
     else:
@@ -447,8 +435,10 @@ def run_ours(args, D):
 
     if not args.no_backward:
         out["prefill_backward"] = _backward(args, D, dev, x, T, w, peaks)
-    if args.varlen:
-        out["prefill_varlen32"] = _varlen(args, D, dev, peaks)
+    if not args.no_long:
+        out["prefill_long262k"] = _prefill_leg(args, D, dev, peaks, peak_src, "long262k")
+        out["prefill_varlen32"] = _prefill_leg(args, D, dev, peaks, peak_src, "varlen32",
+                                               single_pass=True)
 
     if not args.no_decode:
         out["decode"] = _decode(args, D, dev, peaks, peak_src)
@@ -472,6 +462,34 @@ def run_ours(args, D):
                                                "sample": f"first {n1} tokens x {w.Hv} V heads, "
                                                          f"1 thread, {secs1:.1f} s wall"}}
     return out
+
+
+def prefill_roofline(T, Hv, D, ms, peaks, peak_src, state_io):
+    """Roofline of one tensor-core prefill call of T tokens taking ``ms``.
+    The fraction is tensor-pipe utilisation: algorithmic flops over time
+    against the measured bf16 dense (burst) peak.  Beside it the HBM
+    fractions for the two readings of the output bytes (fp32 o as written,
+    45,440 B/token; bf16 o, 33,152 B/token) plus ``state_io`` states of
+    Hv x D x D fp32 per sequence-call (final, or initial and final)."""
+    flops = FLOP_PER_TOKEN * T
+    state_bytes = state_io * Hv * D * D * 4
+    b32 = BYTES_PER_TOKEN * T + state_bytes
+    b16 = BYTES_PER_TOKEN_BF16_O * T + state_bytes
+    sec = ms / 1e3
+    tensor_ach = flops / sec / 1e12
+    return {"bound": "tensor", "achieved": tensor_ach, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": tensor_ach / peaks["bf16_tflops"],
+            "peak_source": f"{peak_src} bf16_tflops (burst; the call is timed alone)",
+            "algorithmic": f"{FLOP_PER_TOKEN} flop/token x {T} tokens",
+            "tensor_frac": tensor_ach / peaks["bf16_tflops"],
+            "tensor_achieved_tflops": tensor_ach,
+            "hbm_frac": b32 / sec / 1e9 / peaks["hbm_gbs"],
+            "hbm_algorithmic": f"{BYTES_PER_TOKEN} B/token (fp32 o) x {T} + states",
+            "hbm_frac_bf16_o": b16 / sec / 1e9 / peaks["hbm_gbs"],
+            "hbm_algorithmic_bf16_o": f"{BYTES_PER_TOKEN_BF16_O} B/token (bf16 o) x {T} + states",
+            "floor_us": {"tensor": flops / (peaks["bf16_tflops"] * 1e12) * 1e6,
+                         "hbm_fp32_o": b32 / (peaks["hbm_gbs"] * 1e9) * 1e6,
+                         "hbm_bf16_o": b16 / (peaks["hbm_gbs"] * 1e9) * 1e6}}
 
 
 def _tc_path_available():
@@ -614,22 +632,27 @@ def _prefill_raw(args, D, dev, x, T, w, ws, fin, o, flush, prepared_ms, launches
             "l2": "flushed between timed steps", "gpu_launches": args.steps * launches}
 
 
-def _varlen(args, D, dev, peaks):
-    """The prefill on the varlen32 workload: 32 packed sequences of 1k to 32k
-    tokens with their own initial states, final states returned.  Unlike
-    prefill8k (one chain of chunks per value head) it gives the state pass many
-    chains at once, so it shows what the two phases cost in SM time.  The
-    single-pass kernel (chosen by a header-only workspace) is timed beside it."""
+def _prefill_leg(args, D, dev, peaks, peak_src, name, single_pass=False):
+    """The prefill on another named workload: long262k (one 262,144-token
+    sequence, slow decay, nonzero initial state returned as the final state in
+    place) or varlen32 (32 packed sequences of 1k to 32k tokens with their own
+    initial states, final states returned).  Unlike prefill8k, varlen32 gives
+    the state pass many chains at once, so it shows what the two phases cost in
+    SM time; there the single-pass kernel (chosen by a header-only workspace) is
+    timed beside it.  Inputs are larger than L2, so no flush is needed."""
     import torch
 
     from gated_deltanet_recurrence_rule_b200 import api, inputs
 
-    w = inputs.WORKLOADS["varlen32"]
-    inp = inputs.workload_inputs(w)
+    w = inputs.WORKLOADS[name]
+    inp = inputs.prefill_inputs(w.lengths, w.Hqk, w.Hv, w.D, dtype=w.dtype,
+                                seed=rank_seed(w.seed, D.rank), g_mu=w.g_mu, init_std=w.init_std)
     x = {n: t.to(dev) for n, t in inp.items() if t is not None}
+    del inp
     T, N = w.total_tokens, len(w.lengths)
     o = torch.empty((T, w.Hv, w.D), dtype=torch.float32, device=dev)
-    fin = torch.empty((N, w.Hv, w.D, w.D), dtype=torch.float32, device=dev)
+    # the final state overwrites the initial state in place (a resumable prefill)
+    state = x["initial_state"]
     full = torch.zeros(api.prefill_workspace_size(N, T, w.Hqk, w.Hv, w.D, w.D), dtype=torch.uint8,
                        device=dev)
     header = torch.zeros(256, dtype=torch.uint8, device=dev)  # selects the single-pass kernel
@@ -639,9 +662,10 @@ def _varlen(args, D, dev, peaks):
     def timed(ws):
         def step():
             api.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], cu_seqlens=x["cu_seqlens"],
-                        initial_state=x["initial_state"], final_state=fin, o=o, workspace=ws)
+                        initial_state=state, final_state=state, o=o, workspace=ws)
 
-        step()
+        for _ in range(2):
+            step()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         D.barrier()
@@ -653,24 +677,23 @@ def _varlen(args, D, dev, peaks):
         torch.cuda.synchronize()
         D.barrier()
         if api.get_device_status(ws) != api.GDN_OK:
-            raise RuntimeError("device status after the varlen leg")
+            raise RuntimeError(f"device status after the {name} leg")
         return D.max(e0.elapsed_time(e1), dev) / steps
 
     ms = timed(full)
-    ms_single = timed(header)
-    hbm_bytes = BYTES_PER_TOKEN * T + 2 * N * w.Hv * w.D * w.D * 4
-    gbs = hbm_bytes / (ms / 1e3) / 1e9
-    return {"value": D.world * T / (ms / 1e3) / 1e6, "unit": "Mtok/s", "ms_per_step": ms,
-            "workload": f"varlen32: N={N} T={T} Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16, fp32 o, "
-                        "N(0,0.02) initial states, final states returned",
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"],
-                         "algorithmic": f"{BYTES_PER_TOKEN} B/token x {T} + initial and final states"},
-            "gpu_launches": steps * api.prefill_launch_count(N, T, w.Hqk, w.Hv, w.D, w.D, full.numel()),
-            "single_pass": {"value": D.world * T / (ms_single / 1e3) / 1e6, "unit": "Mtok/s",
-                            "ms_per_step": ms_single,
-                            "how": "the same call with a 256-byte workspace: one CTA per (sequence, "
-                                   "value head) runs all its chunks"}}
+    out = {"value": D.world * T / (ms / 1e3) / 1e6, "unit": "Mtok/s", "ms_per_step": ms,
+           "workload": workload_desc(w) + ", final state written over the initial state",
+           "roofline": prefill_roofline(T, w.Hv, w.D, ms, peaks, peak_src, state_io=2 * N),
+           "gpu_launches": steps * api.prefill_launch_count(N, T, w.Hqk, w.Hv, w.D, w.D,
+                                                            full.numel()),
+           "warmup": 2, "steps": steps, "l2": "inputs larger than L2"}
+    if single_pass:
+        ms_single = timed(header)
+        out["single_pass"] = {"value": D.world * T / (ms_single / 1e3) / 1e6, "unit": "Mtok/s",
+                              "ms_per_step": ms_single,
+                              "how": "the same call with a 256-byte workspace: one CTA per "
+                                     "(sequence, value head) runs all its chunks"}
+    return out
 
 
 def _backward(args, D, dev, x, T, w, peaks):
@@ -795,6 +818,12 @@ def _decode(args, D, dev, peaks, peak_src):
     us = ms * 1e3 / steps
     gbs = D.world * per_step * steps / (ms / 1e3) / 1e9
     peak = peaks["hbm_gbs"]
+    traffic = kernel_traffic("decode", DECODE_SOURCES)
+    note = None
+    if traffic:
+        note = (f"ncu counts {traffic / 1e6:.1f} MB of DRAM traffic per launch against "
+                f"{per_step / 1e6:.1f} MB algorithmic: back to back, L2 still holds part of the "
+                f"state written by the previous step, so part of this fraction is L2 residency")
     return {"value": gbs, "unit": "GB/s", "workload": f"decode64: B={w.batch} x 1 token, Hqk={w.Hqk} "
             f"Hv={w.Hv} D={w.D} bf16, fp32 state {state_bytes} B in place, {steps} steps",
             "us_per_step": us, "steps_per_s": steps / (ms / 1e3),
@@ -804,7 +833,7 @@ def _decode(args, D, dev, peaks, peak_src):
                          "peak": peak, "unit": "GB/s", "frac": gbs / D.world / peak,
                          "peak_source": f"{peak_src} hbm_gbs",
                          "algorithmic": f"{per_step} B per step (state read+write {2 * state_bytes} + io {io_bytes})",
-                         "traffic": kernel_traffic("decode", DECODE_SOURCES)},
+                         "traffic": traffic, "note": note},
             "gpu_launches": steps}
 
 

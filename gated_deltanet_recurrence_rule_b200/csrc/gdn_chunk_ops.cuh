@@ -178,20 +178,31 @@ __device__ __forceinline__ void st_split8(unsigned char *dst_hi, unsigned char *
   *reinterpret_cast<uint4 *>(dst_lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
 
+// Whether any thread of a group of NT threads (named barrier BAR) saw the
+// CTA's abort flag set or failed a wait itself.  Every thread reads the flag
+// before the barrier and the barrier ORs the readings, so all threads of the
+// group get the same answer even when another role sets the flag meanwhile
+// (a group that split on it would leave some threads waiting at a later
+// barrier that the others never reach).
+template <int NT, int BAR>
+__device__ __forceinline__ bool group_aborted(volatile int *abort, bool failed_here = false) {
+  return named_bar_or(BAR, NT, failed_here || *abort != 0);
+}
+
 // One waiter (thread 0 of the group) for an mbarrier phase, then a named
-// barrier of the NT group threads; returns false on abort (then every thread
-// of the group returns false).
+// barrier of the NT group threads; returns false on abort, and then for every
+// thread of the group.
 template <int NT, int BAR>
 __device__ __forceinline__ bool group_wait(uint32_t bar, uint32_t parity, int gtid,
-                                           volatile int *abort, int32_t *status) {
-  if (gtid == 0) {
-    if (!mbar_wait(bar, parity, abort)) {
-      *abort = 1;
-      report_status(status, GDN_ERR_DEVICE_TIMEOUT);
-    }
+                                           volatile int *abort, int32_t *status,
+                                           uint64_t timeout_ns) {
+  bool failed = false;
+  if (gtid == 0 && !mbar_wait(bar, parity, abort, timeout_ns)) {
+    *abort = 1;
+    report_status(status, GDN_ERR_DEVICE_TIMEOUT);
+    failed = true;
   }
-  named_bar_sync(BAR, NT);
-  const bool ok = (*abort == 0);
+  const bool ok = !group_aborted<NT, BAR>(abort, failed);
   if (ok) tc_fence_after();
   return ok;
 }

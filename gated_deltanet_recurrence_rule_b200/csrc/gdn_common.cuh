@@ -14,15 +14,23 @@ namespace gdn {
 
 // Workspace header written by gdn_prefill (first 256 bytes of the workspace).
 struct WorkspaceHeader {
-  int32_t status;       // GDN_OK or a device-detected error code (first one wins)
-  int32_t reserved0;
-  uint32_t next_unit;   // dynamic work counter of persistent kernels
+  int32_t status;         // GDN_OK or a device-detected error code (first one wins)
+  uint32_t wait_limit_us; // bounded-wait limit of the kernels in microseconds; 0 = 2 s
+  uint32_t next_unit;     // dynamic work counter of persistent kernels
   uint32_t reserved1;
 };
 constexpr size_t kWorkspaceHeaderBytes = 256;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ void report_status(int32_t *status, int32_t code) {
   if (status) atomicCAS(status, GDN_OK, code);
+}
+
+// The wait limit the caller left in the workspace header (`status` is the
+// workspace base), in nanoseconds; 2 s when the field is 0.
+__device__ __forceinline__ uint64_t wait_limit_ns(const int32_t *status) {
+  const uint32_t us = status ? reinterpret_cast<const WorkspaceHeader *>(status)->wait_limit_us : 0u;
+  return us ? (uint64_t)us * 1000ull : kDefaultWaitLimitNs;
 }
 
 // ---- element conversion ---------------------------------------------------

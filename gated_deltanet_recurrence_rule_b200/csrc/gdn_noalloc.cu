@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "gdn.h"
+#include "gdn_common.cuh"
 
 namespace gdn {
 size_t prefill_min_workspace_bytes(int32_t num_seqs, int64_t total_tokens, int32_t Hqk, int32_t Hv,
@@ -25,7 +26,11 @@ size_t prefill_min_workspace_bytes(int32_t num_seqs, int64_t total_tokens, int32
 namespace {
 
 // Every GPU that loads the library holds this array until the process exits.
-constexpr size_t kScratchBytes = 4096;
+// It is exactly the workspace header (status word, wait limit, scheduler
+// counters): the most gdn_prefill_noalloc ever needs, because with no more
+// workspace than that gdn_prefill runs its single-pass kernels.
+constexpr size_t kScratchBytes = gdn::kWorkspaceHeaderBytes;
+static_assert(kScratchBytes >= gdn::kWorkspaceHeaderBytes, "the scratch holds the workspace header");
 static __device__ __align__(256) unsigned char g_prefill_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -64,9 +69,9 @@ extern "C" int32_t gdn_prefill_noalloc(const void *q, const void *k, const void 
   const int32_t st = scratch_address(&scratch);
   if (st != GDN_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // The scratch keeps the previous call's contents: its header (status word
-  // and scheduler counters) must start every call at zero.
-  if (cudaMemsetAsync(scratch, 0, 256, s) != cudaSuccess) return GDN_ERR_CUDA;
+  // The scratch keeps the previous call's contents: its header (status word,
+  // wait limit and scheduler counters) must start every call at zero.
+  if (cudaMemsetAsync(scratch, 0, gdn::kWorkspaceHeaderBytes, s) != cudaSuccess) return GDN_ERR_CUDA;
   const int32_t rc = gdn_prefill(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens,
                                  num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype,
                                  o_dtype, GDN_DTYPE_FP32, GDN_INPUT_PREPARED, scale, initial_state,

@@ -139,8 +139,8 @@ struct Params {
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sb, int i) { return sb + OFF_BAR + 8u * i; }
 
 __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, int etid,
-                                         volatile int *abort, int32_t *status) {
-  return group_wait<NEPI, EPI_BAR>(bar, parity, etid, abort, status);
+                                         volatile int *abort, int32_t *status, uint64_t tmo) {
+  return group_wait<NEPI, EPI_BAR>(bar, parity, etid, abort, status, tmo);
 }
 
 template <typename TO>
@@ -179,6 +179,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     return;
   }
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  const uint64_t tmo = wait_limit_ns(p.status);
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
     *abort_flag = 0;
@@ -216,7 +217,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
           tma_prefetch_3d(&tm_v, 0, h, t); tma_prefetch_3d(&tm_v, 64, h, t);
         }
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag, tmo)) break;
         const uint32_t st = sb + OFF_QK + s * QK_STAGE;
         const uint32_t fb = bar_addr(sb, B_FULL_QK + s);
         mbar_arrive_expect_tx(fb, QK_STAGE);
@@ -225,7 +226,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tma_load_3d(st + 8192, &tm_k, fb, 0, j, t0);
         tma_load_3d(st + 24576, &tm_k, fb, 64, j, t0);
         issued_qk = c + 1;
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_V + sv), ((c / NV) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_V + sv), ((c / NV) & 1) ^ 1, abort_flag, tmo)) break;
         const uint32_t vs = sb + OFF_V + sv * V_STAGE;
         const uint32_t fv = bar_addr(sb, B_FULL_V + sv);
         mbar_arrive_expect_tx(fv, V_STAGE);
@@ -240,9 +241,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       // Let every load this thread issued land before the CTA can exit (each
       // buffer's latest fill; earlier fills were consumed before it was issued).
       for (int c = max(issued_qk - NQK, 0); c < issued_qk; ++c)
-        mbar_wait(bar_addr(sb, B_FULL_QK + c % NQK), (c / NQK) & 1, abort_flag, 50000000ull);
+        mbar_wait_landed(bar_addr(sb, B_FULL_QK + c % NQK), (c / NQK) & 1, 50000000ull);
       for (int c = max(issued_v - NV, 0); c < issued_v; ++c)
-        mbar_wait(bar_addr(sb, B_FULL_V + c % NV), (c / NV) & 1, abort_flag, 50000000ull);
+        mbar_wait_landed(bar_addr(sb, B_FULL_V + c % NV), (c / NV) & 1, 50000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -262,8 +263,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint64_t dQK = dQK0 + s * (QK_STAGE >> 4), dKmn = dKmn0 + s * (QK_STAGE >> 4);
         const uint64_t dVmn = dVmn0 + sv * (V_STAGE >> 4);
         // [Q;K] K^T
-        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), (c / NQK) & 1, abort_flag);
-        if (ok && c > 0) ok = mbar_wait(bar_addr(sb, B_DONE), (c - 1) & 1, abort_flag);
+        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), (c / NQK) & 1, abort_flag, tmo);
+        if (ok && c > 0) ok = mbar_wait(bar_addr(sb, B_DONE), (c - 1) & 1, abort_flag, tmo);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -273,8 +274,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         mma_commit(bar_addr(sb, B_QK));
         // W^T = K^T (T'h + T'l)^T ;  U~^T = V^T (T''h + T''l)^T
-        ok = mbar_wait(bar_addr(sb, B_T), ph, abort_flag) &&
-             mbar_wait(bar_addr(sb, B_FULL_V + sv), (c / NV) & 1, abort_flag);
+        ok = mbar_wait(bar_addr(sb, B_T), ph, abort_flag, tmo) &&
+             mbar_wait(bar_addr(sb, B_FULL_V + sv), (c / NV) & 1, abort_flag, tmo);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -290,7 +291,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mma_commit(bar_addr(sb, B_W));
         mma_commit(bar_addr(sb, B_EMPTY_V + sv));
         // U^T = U~^T - S0h W^T ;  Oi^T = (S0h + S0l) Q^T   (S0 from TMEM)
-        ok = mbar_wait(bar_addr(sb, B_WT), ph, abort_flag);
+        ok = mbar_wait(bar_addr(sb, B_WT), ph, abort_flag, tmo);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -305,7 +306,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         mma_commit(bar_addr(sb, B_U));
         // dS = (Ukh + Ukl)^T K ;  Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T   (U from TMEM)
-        ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag);
+        ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag, tmo);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -333,14 +334,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_init(drain, 1);
       fence_barrier_init();
       mma_commit(drain);
-      mbar_wait(drain, 0, abort_flag, 50000000ull);
+      mbar_wait_landed(drain, 0, 50000000ull);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------ chunk scalars
     for (int c = 0; c < nch; ++c) {
       const int s = c & 1;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar_addr(sb, B_SCAL_EMPTY + s), ((c >> 1) & 1) ^ 1, abort_flag);
+      if (lane == 0) ok = mbar_wait(bar_addr(sb, B_SCAL_EMPTY + s), ((c >> 1) & 1) ^ 1, abort_flag, tmo);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) { *abort_flag = 1; report_status(p.status, GDN_ERR_DEVICE_TIMEOUT); }
@@ -449,12 +450,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
       // ---- Q K^T and K K^T -> P (hi/lo) and A (fp32)
       if (etid == 0) {
-        if (!mbar_wait(bar_addr(sb, B_SCAL_FULL + s), (c >> 1) & 1, abort_flag)) {
+        if (!mbar_wait(bar_addr(sb, B_SCAL_FULL + s), (c >> 1) & 1, abort_flag, tmo)) {
           *abort_flag = 1;
           report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
         }
       }
-      if (!epi_wait(bar_addr(sb, B_QK), ph, etid, abort_flag, p.status)) break;
+      if (!epi_wait(bar_addr(sb, B_QK), ph, etid, abort_flag, p.status, tmo)) break;
       {
         float v[16];
         tmem_ld16(tl + R_QK + 16 * ewq, v);
@@ -523,7 +524,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (etid == 0) mbar_arrive(bar_addr(sb, B_T));
 
       // ---- W^T -> bf16 (MN-major B)
-      if (!epi_wait(bar_addr(sb, B_W), ph, etid, abort_flag, p.status)) break;
+      if (!epi_wait(bar_addr(sb, B_W), ph, etid, abort_flag, p.status, tmo)) break;
       {
         float v[16];
         tmem_ld16(tl + R_W + 16 * ewq, v);
@@ -537,7 +538,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (etid == 0) mbar_arrive(bar_addr(sb, B_WT));
 
       // ---- U^T -> hi/lo (for P) and U^T diag(kdec) -> hi/lo (for the state), into TMEM
-      if (!epi_wait(bar_addr(sb, B_U), ph, etid, abort_flag, p.status)) break;
+      if (!epi_wait(bar_addr(sb, B_U), ph, etid, abort_flag, p.status, tmo)) break;
       {
         float v[16];
         tmem_ld16(tl + R_UO + 16 * ewq, v);
@@ -558,7 +559,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (etid == 0) mbar_arrive(bar_addr(sb, B_UT));
 
       // ---- state: S = gamma_C S + dS (fp32), S0 <- hi/lo(S); outputs
-      if (!epi_wait(bar_addr(sb, B_S), ph, etid, abort_flag, p.status)) break;
+      if (!epi_wait(bar_addr(sb, B_S), ph, etid, abort_flag, p.status, tmo)) break;
       {
         const float gC = sc[256];
         {

@@ -223,6 +223,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     return;
   }
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  const uint64_t tmo = wait_limit_ns(p.status);
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
     // a record slot is free once its MMAs completed AND the epilogue read it
@@ -265,7 +266,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
           bulk_prefetch_l2(chunk_rec(c + PF), REC_BYTES);
         }
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag, tmo)) break;
         const uint32_t st = sb + OFF_QK + s * QK_STAGE;
         const uint32_t fb = bar_addr(sb, B_FULL_QK + s);
         mbar_arrive_expect_tx(fb, QK_STAGE);
@@ -274,7 +275,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tma_load_3d(st + 8192, &tm_k, fb, 0, j, t0);
         tma_load_3d(st + 24576, &tm_k, fb, 64, j, t0);
         issued_qk = c + 1;
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_R + sr), ((c / NR) & 1) ^ 1, abort_flag)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_R + sr), ((c / NR) & 1) ^ 1, abort_flag, tmo)) break;
         const uint32_t fr = bar_addr(sb, B_FULL_R + sr);
         mbar_arrive_expect_tx(fr, REC_BYTES);
         bulk_load(sb + OFF_REC + sr * REC_BYTES, chunk_rec(c), REC_BYTES, fr);
@@ -303,7 +304,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint64_t dP0 = sdesc_sw128(sb + OFF_REC + tp::REC_PH, 16, 1024);    // P hi / lo, K-major
     auto wait = [&](int b, uint32_t parity) {
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar_addr(sb, b), parity, abort_flag);
+      if (lane == 0) ok = mbar_wait(bar_addr(sb, b), parity, abort_flag, tmo);
       return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
     bool ok = true;
@@ -415,9 +416,12 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float un[16];
     auto fetch_ut = [&](int c) {
       const int sr = c % NR;
-      if (etid == 0 && !mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag)) fail();
-      named_bar_sync(EPI_BAR, NEPI);
-      if (*abort_flag) return false;
+      bool failed = false;
+      if (etid == 0 && !mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag, tmo)) {
+        fail();
+        failed = true;
+      }
+      if (group_aborted<NEPI, EPI_BAR>(abort_flag, failed)) return false;
       const float *ut = reinterpret_cast<const float *>(smem + OFF_REC + sr * REC_BYTES + tp::REC_UT) + row;
 #pragma unroll
       for (int x = 0; x < 16; ++x) un[x] = ut[(16 * ewq + x) * HD];
@@ -446,7 +450,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float *kdec = gam + 64;
 
       // ---- U = (U - U~) + U~ -> hi/lo(U^T diag(kdec)) for dS first, then hi/lo(U^T) for Oa
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_U), ph, etid, abort_flag, p.status))) break;
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_U), ph, etid, abort_flag, p.status, tmo))) break;
       {
         float v[16];
         tmem_ld16(tl + R_S + 16 * ewq, v);
@@ -481,7 +485,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       store_out(1);
 
       // ---- state: S = gamma_C S + dS (fp32); hi(S) first (the next U product), then lo(S)
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_S), ph, etid, abort_flag, p.status))) break;
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_S), ph, etid, abort_flag, p.status, tmo))) break;
       {
         const float gC = gam[128];
 #pragma unroll
@@ -514,7 +518,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       store_out(3);
 
       // ---- outputs o_t = scale (e^{G_t} Oi_t + Oa_t) out of TMEM
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_OA), ph, etid, abort_flag, p.status))) break;
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_OA), ph, etid, abort_flag, p.status, tmo))) break;
       {
         float va[16];
         tmem_ld16(tl + R_OI + 16 * ewq, out);
@@ -636,26 +640,39 @@ static cudaError_t launch_state_pass(const CUtensorMap &mq, const CUtensorMap &m
   return cudaGetLastError();
 }
 
-// Internal streams and events of one device, created by its first pipelined
-// prefill and kept until the process exits: phase 1 runs on `prep`, phase 2
-// on `chain` (higher priority, so its CTAs get the SMs that free up first).
+// Internal streams and events of the pipelined schedule: phase 1 runs on
+// `prep`, phase 2 on `chain` (higher priority, so its CTAs get the SMs that
+// free up first).  One pair per (device, caller stream), for up to
+// kPairsPerDevice caller streams per device, created by the first pipelined
+// prefill issued on that caller stream and kept until the process exits, so
+// prefills issued on different caller streams do not queue behind one
+// another.  Further caller streams share the device's first pair (their
+// prefills are then ordered after one another, which is correct but not
+// concurrent).
 namespace {
-constexpr int kMaxDevices = 64, kEventRing = 4;
+constexpr int kMaxDevices = 64, kEventRing = 4, kPairsPerDevice = 8;
 struct DeviceStreams {
   bool ready = false;
+  cudaStream_t owner = nullptr;  // the caller stream this pair serves
   cudaStream_t prep = nullptr, chain = nullptr;
   cudaEvent_t start = nullptr, prep_done = nullptr, ev_p[kEventRing] = {}, ev_c[kEventRing] = {};
 };
 std::mutex g_streams_mutex;
-DeviceStreams g_streams[kMaxDevices];
+DeviceStreams g_streams[kMaxDevices][kPairsPerDevice];
 
-cudaError_t device_streams(DeviceStreams **out) {
+cudaError_t device_streams(cudaStream_t caller, DeviceStreams **out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  DeviceStreams &d = g_streams[dev];
+  int slot = 0;  // the caller's pair, else the first free one, else the shared first one
+  for (int i = 0; i < kPairsPerDevice; ++i) {
+    if (g_streams[dev][i].ready && g_streams[dev][i].owner == caller) { slot = i; break; }
+    if (!g_streams[dev][i].ready) { slot = i; break; }
+  }
+  DeviceStreams &d = g_streams[dev][slot];
   if (!d.ready) {
+    d.owner = caller;
     int least = 0, greatest = 0;
     if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
     if ((e = cudaStreamCreateWithPriority(&d.prep, cudaStreamNonBlocking, least)) != cudaSuccess) return e;
@@ -738,7 +755,7 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
   // by events (this also works while `stream` is being captured into a graph).
   std::lock_guard<std::mutex> lock(g_streams_mutex);
   DeviceStreams *d = nullptr;
-  if ((e = device_streams(&d)) != cudaSuccess) return e;
+  if ((e = device_streams(stream, &d)) != cudaSuccess) return e;
   if ((e = cudaEventRecord(d->start, stream)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(d->prep, d->start, 0)) != cudaSuccess) return e;
   if ((e = cudaStreamWaitEvent(d->chain, d->start, 0)) != cudaSuccess) return e;

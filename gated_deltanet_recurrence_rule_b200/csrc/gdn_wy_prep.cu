@@ -116,6 +116,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     return;
   }
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+  const uint64_t tmo = wait_limit_ns(p.status);
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
     *abort_flag = 0;
@@ -171,7 +172,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const uint64_t dVmn = sdesc_sw128(sb + OFF_V, 8192, 1024);           // V^T, MN-major
       const uint64_t dTP = sdesc_sw128(sb + OFF_TPH, 16, 1024);            // T', K-major
       const uint64_t dTQ = sdesc_sw128(sb + OFF_TQH, 16, 1024);            // T'', K-major
-      bool ok = mbar_wait(bar_addr(sb, B_QKF), 0, abort_flag);
+      bool ok = mbar_wait(bar_addr(sb, B_QKF), 0, abort_flag, tmo);
       if (ok) {
         tc_fence_after();
 #pragma unroll
@@ -180,7 +181,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mma_bf16(tmem + R_QK, dQK + k16, dQK + (8192 >> 4) + k16, IDESC_QK, ks > 0);
         }
         mma_commit(bar_addr(sb, B_QK));
-        ok = mbar_wait(bar_addr(sb, B_T), 0, abort_flag) && mbar_wait(bar_addr(sb, B_VF), 0, abort_flag);
+        ok = mbar_wait(bar_addr(sb, B_T), 0, abort_flag, tmo) && mbar_wait(bar_addr(sb, B_VF), 0, abort_flag, tmo);
       }
       if (ok) {
         tc_fence_after();
@@ -262,7 +263,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const float *sc = reinterpret_cast<const float *>(smem + OFF_SCAL);
     const float *G2 = sc, *gam = sc + 64, *bet = sc + 192, *rqn = sc + 256, *rkn = sc + 320;
     do {
-      if (etid == 0 && !mbar_wait(bar_addr(sb, B_SCAL), 0, abort_flag)) {
+      if (etid == 0 && !mbar_wait(bar_addr(sb, B_SCAL), 0, abort_flag, tmo)) {
         *abort_flag = 1;
         report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
       }
@@ -274,7 +275,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // into the bf16 operand tiles: P and A gain 1/|q_t| 1/|k_s| and
         // 1/|k_t| 1/|k_s|, T' gains 1/|k_s|, and the record's e^{G_t} and
         // e^{G_C - G_t} gain 1/|q_t| and 1/|k_t| for the state pass.
-        if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QKF), 0, etid, abort_flag, p.status)) break;
+        if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QKF), 0, etid, abort_flag, p.status, tmo)) break;
         const int rr = etid >> 1, t = rr & 63;
         const unsigned char *seg = smem + OFF_QK + (rr >> 6) * 8192 + (etid & 1) * 16384 + t * 128;
         float ss = 0.f;
@@ -297,7 +298,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           rs[rr] = sc[64 + rr] * r;  // e^{G_t} / |q_t|, then e^{G_C - G_t} / |k_t|
         }
       }
-      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QK), 0, etid, abort_flag, p.status)) break;
+      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QK), 0, etid, abort_flag, p.status, tmo)) break;
       // ---- Q K^T -> P (record, hi/lo), K K^T -> A (fp32, shared)
 #pragma unroll
       for (int qh = 0; qh < 2; ++qh) {
@@ -360,7 +361,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (etid == 0) mbar_arrive(bar_addr(sb, B_T));
 
       // ---- W^T -> record (bf16 MN-major image), U~ -> record (fp32 [t][d])
-      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_W), 0, etid, abort_flag, p.status)) break;
+      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_W), 0, etid, abort_flag, p.status, tmo)) break;
       {
         float v[32];
         tmem_ld32(tl + R_W + 32 * half, v);

@@ -32,9 +32,13 @@
  *
  * Memory.  Every pointer argument except those named "host" is a device
  * pointer (cudaMalloc'd or equivalent) owned by the caller; the library never
- * allocates device memory, frees or keeps a pointer after a call returns (the
- * pipelined prefill keeps two internal streams and a few events per device).  All arrays are
- * dense row-major with the shapes given below and 16-byte-aligned bases.
+ * allocates device memory, frees or keeps a pointer after a call returns.  The
+ * pipelined prefill (see gdn_prefill) keeps two internal streams and a few
+ * events per (device, caller stream) for up to 8 caller streams per device,
+ * created on first use and kept until the process exits; prefills issued on
+ * further caller streams share the device's first pair and are then ordered
+ * after one another (correct, but not concurrent).  All arrays are dense
+ * row-major with the shapes given below and 16-byte-aligned bases.
  *
  * Ordering.  Every call enqueues work on `stream` (a cudaStream_t; NULL is
  * the legacy default stream) and returns without synchronising, except
@@ -160,15 +164,24 @@ int64_t gdn_prefill_launch_count(int32_t num_seqs, int64_t total_tokens, int32_t
  *   workspace      device buffer of workspace_bytes >= 256 bytes, 256-byte aligned,
  *                  zero-filled once before its first use.  Its first word is the
  *                  sticky status word: it keeps the first device-detected error
- *                  until gdn_get_device_status reads and clears it; nothing else in
- *                  it needs to survive between calls.
+ *                  until gdn_get_device_status reads and clears it.  Its second
+ *                  word (uint32, byte offset 4) is the limit of the kernels'
+ *                  bounded waits in microseconds, 0 for the default of 2 s; a
+ *                  wait that runs out sets GDN_ERR_DEVICE_TIMEOUT, the kernel
+ *                  drains its own copies and MMAs, frees its tensor memory and
+ *                  returns, and o and final_state of that call are undefined
+ *                  (tests set a limit of a microsecond to take that path).
+ *                  Nothing else in it needs to survive between calls.
  *
  * Supported: Hv % Hqk == 0; Dk, Dv in {64, 128}; dtype and o_dtype each bf16
  * or fp32.  bf16 inputs with Dk = Dv = 128 run on the tensor cores (tcgen05,
  * bf16 operands with hi/lo splits of computed values, fp32 accumulation):
  *   - workspace_bytes >= gdn_prefill_workspace_size(...): two phases, the
  *     state-free products of every chunk at once (WY/UT transform), then one
- *     pass per (sequence, value head) over its chunks for the state;
+ *     pass per (sequence, value head) over its chunks for the state, in
+ *     pipelined rounds on the two internal streams of the caller's stream
+ *     (joined to `stream` by events, so the call stays stream-ordered and can
+ *     be captured in a CUDA graph);
  *   - smaller, down to the two-phase minimum (the state carry plus one chunk
  *     per value head): the same in rounds of as many chunks as fit;
  *   - below that (>= 256 bytes): a single-pass kernel, one CTA per (sequence,
@@ -198,23 +211,30 @@ int32_t gdn_prefill(const void *q, const void *k, const void *v, const float *g,
  * runtime's memory pool), the path is real-time and must not take
  * cudaMalloc's implicit device-wide synchronisation, or a plugin is handed
  * only its input and output buffers.  This entry point allocates nothing: it
- * runs gdn_prefill with a 4096-byte workspace kept in a file-scope __device__
- * array of the library (every GPU that loads the library holds it until the
- * process exits), and calls no cudaMalloc, cudaFree or allocating routine.
+ * runs gdn_prefill with a 256-byte workspace (the status header) kept in a
+ * file-scope __device__ array of the library (every GPU that loads the
+ * library holds it until the process exits), and calls no cudaMalloc, cudaFree
+ * or allocating routine.  With that workspace bf16 inputs at head dim 128 take
+ * the single-pass tensor-core kernel and every other case the CUDA-core
+ * kernel; the faster two-phase kernels need more workspace than any fixed
+ * array could hold for long inputs.
  *
  * Arguments are those of gdn_prefill without the workspace, with fp32 states
  * and prepared inputs (no state_dtype, no input_form), plus
  *   device_status  optional device int32 (caller's memory, NULL to discard) that
  *                  receives this call's device-detected status (GDN_OK,
  *                  GDN_ERR_BAD_SEQLENS or GDN_ERR_DEVICE_TIMEOUT) in stream order.
- * Returns GDN_ERR_WORKSPACE if these sizes need more workspace than the 4096-byte
+ * Returns GDN_ERR_WORKSPACE if these sizes need more workspace than the 256-byte
  * built-in array; otherwise what gdn_prefill returns.
  *
  * The first call on each device resolves the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call before
- * any stream capture.  Every call on a device shares the one array: each call
- * clears its header first, and calls whose work overlaps on the GPU (other
- * streams, other host threads without ordering) race on it.
+ * (cudaGetSymbolAddress) with that device current and keeps it for the life
+ * of the process; make that first call before any stream capture.  A reset of
+ * the device's primary context (cudaDeviceReset) invalidates that address: do
+ * not call this entry point on a device after resetting it.  Every call on a
+ * device shares the one array: each call clears its header first, and calls
+ * whose work overlaps on the GPU (other streams, other host threads without
+ * ordering) race on it.
  */
 int32_t gdn_prefill_noalloc(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,

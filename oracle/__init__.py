@@ -163,14 +163,23 @@ def prefill(q, k, v, g, beta, cu_seqlens=None, initial_state=None, scale=1.0, ch
     return o, fin
 
 
-def decode_step(q, k, v, g, beta, state, scale=1.0, num_threads=0, state_at_rest=None, lib=None):
+def decode_step(q, k, v, g, beta, state, scale=1.0, num_threads=0, state_at_rest=None, lib=None,
+                in_place=False):
     """One token for each of B sequences.  q, k: [B, Hqk, Dk]; v: [B, Hv, Dv];
     g, beta: [B, Hv]; state: [B, Hv, Dv, Dk].  Returns (o [B, Hv, Dv],
-    new_state) and leaves the argument ``state`` untouched; state_at_rest="bf16"
-    rounds new_state to bf16."""
+    new_state) and leaves the argument ``state`` untouched, unless
+    ``in_place`` is set: then ``state`` must be a C-contiguous fp64 array,
+    which is updated and returned (no copy, for long runs over large
+    batches); state_at_rest="bf16" rounds new_state to bf16."""
     lib = lib or load()
     q, k, v, g, beta = (_f64(t) for t in (q, k, v, g, beta))
-    S = _f64(state).copy()
+    if in_place:
+        if not (isinstance(state, np.ndarray) and state.dtype == np.float64
+                and state.flags["C_CONTIGUOUS"]):
+            raise ValueError("in_place needs a C-contiguous float64 state array")
+        S = state
+    else:
+        S = _f64(state).copy()
     B, Hqk, Dk = q.shape
     Hv, Dv = v.shape[1], v.shape[2]
     o = np.zeros((B, Hv, Dv), dtype=np.float64)
@@ -181,7 +190,10 @@ def decode_step(q, k, v, g, beta, state, scale=1.0, num_threads=0, state_at_rest
     if state_at_rest not in (None, "fp64", "bf16"):
         raise ValueError(f"unknown state_at_rest {state_at_rest!r}")
     if state_at_rest == "bf16":
-        S = round_bf16(S, lib)
+        if in_place:
+            S[...] = round_bf16(S, lib)
+        else:
+            S = round_bf16(S, lib)
     return o, S
 
 

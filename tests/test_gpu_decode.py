@@ -67,36 +67,23 @@ def test_decode_guard_bands():
 
 def test_decode64_thousand_steps():
     """The batched decode workload (B=64, 16/48 heads, D=128, bf16, fp32
-    state ~N(0, 0.02^2)) for 1000 consecutive steps.  The whole state is
-    checked against the oracle after the first step; six (sequence, head)
-    units are tracked by the oracle through all 1000 steps, with o checked
-    at every step and the state after steps 1, 10, 100 and 1000."""
+    state ~N(0, 0.02^2)) for 1000 consecutive steps, the whole batch tracked
+    by the oracle: o of every (sequence, head) checked at every step, and the
+    whole state after steps 1, 10, 100 and 1000."""
     w = inputs.WORKLOADS["decode64"]
     d = inputs.workload_inputs(w)
-    B, Hqk, Hv, D = w.batch, w.Hqk, w.Hv, w.D
-    G = Hv // Hqk
     S = d["state"].to(DEV)
     dev_in = {n: d[n].to(DEV) for n in ("q", "k", "v", "g", "beta")}
-    units = [(0, 0), (0, 47), (17, 22), (31, 5), (63, 0), (63, 46)]
-    ub = [b for b, _ in units]
-    uh = [h for _, h in units]
-    uj = [h // G for h in uh]
-    S_u = d["state"][ub, uh].double().numpy()[:, None]  # [U, 1, D, D]
+    S_ref = d["state"].double().numpy().copy()  # oracle state, updated in place
     to, ts = TOL[torch.bfloat16]
     worst_o = 0.0
     for s in range(w.steps):
         o = api.decode_step(dev_in["q"][s], dev_in["k"][s], dev_in["v"][s], dev_in["g"][s],
                             dev_in["beta"][s], S)
-        if s == 0:
-            o_full, S_full = oracle.decode_step(d["q"][0], d["k"][0], d["v"][0], d["g"][0],
-                                                d["beta"][0], d["state"])
-            assert_parity(torch.bfloat16, to_np(o), o_full, to_np(S), S_full, "full batch, step 1")
-        o_u, S_u = oracle.decode_step(d["q"][s][ub, uj][:, None], d["k"][s][ub, uj][:, None],
-                                      d["v"][s][ub, uh][:, None], d["g"][s][ub, uh][:, None],
-                                      d["beta"][s][ub, uh][:, None], S_u)
-        og = to_np(o[ub, uh])
-        worst_o = max(worst_o, o_error(og, o_u[:, 0]))
+        o_ref, _ = oracle.decode_step(d["q"][s], d["k"][s], d["v"][s], d["g"][s], d["beta"][s],
+                                      S_ref, in_place=True)
+        worst_o = max(worst_o, o_error(to_np(o), o_ref))
         assert worst_o <= to, f"step {s + 1}: o error {worst_o:.3e}"
         if s + 1 in (1, 10, 100, 1000):
-            es = state_error(to_np(S[ub, uh]), S_u[:, 0])
-            assert es <= ts, f"step {s + 1}: state error {es:.3e}"
+            es = state_error(to_np(S), S_ref)
+            assert es <= ts, f"step {s + 1}: whole-batch state error {es:.3e}"

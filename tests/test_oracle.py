@@ -75,3 +75,23 @@ def test_bf16_state_drift_is_bounded(oracle_lib):
     level = 2.0 ** -9 / np.sqrt(1 - a * a)
     assert 2.0 ** -11 < err[256] < 3 * level, (err, level)   # rounding happens, noise is damped
     assert err[256] < 2 * err[64], err                       # no growth with the number of steps
+
+
+def test_decode_step_in_place_matches_copy(oracle_lib):
+    """The wrapper's in-place mode only avoids the copy: same bits as the
+    copying mode over several steps, with and without bf16 rounding at rest."""
+    r = np.random.default_rng(21)
+    B, Hqk, Hv, D = 3, 2, 6, 8
+    for rest in (None, "bf16"):
+        S_copy = r.standard_normal((B, Hv, D, D)) * 0.1
+        S_in = S_copy.copy()
+        for _ in range(4):
+            q, k = r.standard_normal((B, Hqk, D)), r.standard_normal((B, Hqk, D))
+            v = r.standard_normal((B, Hv, D))
+            g, beta = -r.random((B, Hv)), r.random((B, Hv))
+            o1, S_copy = oracle.decode_step(q, k, v, g, beta, S_copy, state_at_rest=rest)
+            o2, S_ret = oracle.decode_step(q, k, v, g, beta, S_in, state_at_rest=rest, in_place=True)
+            assert S_ret is S_in
+            assert np.array_equal(o1, o2) and np.array_equal(S_copy, S_in)
+    with pytest.raises(ValueError):
+        oracle.decode_step(q, k, v, g, beta, S_in.astype(np.float32), in_place=True)

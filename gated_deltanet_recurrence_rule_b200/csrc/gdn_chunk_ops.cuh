@@ -178,31 +178,31 @@ __device__ __forceinline__ void st_split8(unsigned char *dst_hi, unsigned char *
   *reinterpret_cast<uint4 *>(dst_lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
 
-// Whether any thread of a group of NT threads (named barrier BAR) saw the
-// CTA's abort flag set or failed a wait itself.  Every thread reads the flag
-// before the barrier and the barrier ORs the readings, so all threads of the
-// group get the same answer even when another role sets the flag meanwhile
-// (a group that split on it would leave some threads waiting at a later
-// barrier that the others never reach).
-template <int NT, int BAR>
-__device__ __forceinline__ bool group_aborted(volatile int *abort, bool failed_here = false) {
-  return named_bar_or(BAR, NT, failed_here || *abort != 0);
-}
+// Control words of a CTA in shared memory, as the tensor-core kernels lay
+// them out: [0] the CTA's abort flag (any role may set it at any time), [1]
+// the wait limit in microseconds, [2] the epilogue group's own abort word.
+// The group acts only on [2], which nothing but the group's waiting thread
+// writes, and only before the named barrier that publishes it: every thread
+// of the group then reads the same value, so the group never splits across
+// its named barriers (an abort seen only through [0] would let some threads
+// leave while others wait at a barrier they never reach).
+constexpr int CTL_ABORT = 0, CTL_LIMIT = 1, CTL_GROUP = 2;
 
 // One waiter (thread 0 of the group) for an mbarrier phase, then a named
-// barrier of the NT group threads; returns false on abort, and then for every
-// thread of the group.
+// barrier of the NT group threads; returns false once the group has given up,
+// and then for every thread of the group.  (A waiter that gave up outside
+// this helper sets both abort words: the group then stops here at the latest,
+// whether or not this phase completed.)
 template <int NT, int BAR>
 __device__ __forceinline__ bool group_wait(uint32_t bar, uint32_t parity, int gtid,
-                                           volatile int *abort, int32_t *status,
-                                           uint64_t timeout_ns) {
-  bool failed = false;
-  if (gtid == 0 && !mbar_wait(bar, parity, abort, timeout_ns)) {
-    *abort = 1;
+                                           volatile int *ctl, int32_t *status) {
+  if (gtid == 0 && !mbar_wait(bar, parity, ctl)) {
+    ctl[CTL_ABORT] = 1;
+    ctl[CTL_GROUP] = 1;
     report_status(status, GDN_ERR_DEVICE_TIMEOUT);
-    failed = true;
   }
-  const bool ok = !group_aborted<NT, BAR>(abort, failed);
+  named_bar_sync(BAR, NT);
+  const bool ok = ctl[CTL_GROUP] == 0;
   if (ok) tc_fence_after();
   return ok;
 }

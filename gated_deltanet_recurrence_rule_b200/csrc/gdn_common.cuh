@@ -20,17 +20,15 @@ struct WorkspaceHeader {
   uint32_t reserved1;
 };
 constexpr size_t kWorkspaceHeaderBytes = 256;
-constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ void report_status(int32_t *status, int32_t code) {
   if (status) atomicCAS(status, GDN_OK, code);
 }
 
 // The wait limit the caller left in the workspace header (`status` is the
-// workspace base), in nanoseconds; 2 s when the field is 0.
-__device__ __forceinline__ uint64_t wait_limit_ns(const int32_t *status) {
-  const uint32_t us = status ? reinterpret_cast<const WorkspaceHeader *>(status)->wait_limit_us : 0u;
-  return us ? (uint64_t)us * 1000ull : kDefaultWaitLimitNs;
+// workspace base), in microseconds; 0 means the default of 2 s.
+__device__ __forceinline__ uint32_t header_wait_limit_us(const int32_t *status) {
+  return status ? reinterpret_cast<const volatile WorkspaceHeader *>(status)->wait_limit_us : 0u;
 }
 
 // ---- element conversion ---------------------------------------------------

@@ -90,8 +90,8 @@ constexpr uint32_t OFF_PL = OFF_PH + 8192;      // bf16 lo(P)
 constexpr uint32_t OFF_SCAL = OFF_PL + 8192;
 constexpr uint32_t SCAL_STAGE = 7 * 64 * 4;  // G2 (log2 prefix), gamma, kdec, beta; gamma_C at [256]; 1/|q|, 1/|k| at [320], [384]
 constexpr uint32_t OFF_BAR = OFF_SCAL + 2 * SCAL_STAGE;
-constexpr uint32_t OFF_MISC = OFF_BAR + 192;  // [0] TMEM base, [4] abort flag, [8] drain mbarrier
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+constexpr uint32_t OFF_MISC = OFF_BAR + 192;  // [0] TMEM base, [4] control words (chunk::CTL_*), [16] drain mbarrier
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 24;
 static_assert(OFF_R1 % 1024 == 0 && OFF_PH % 1024 == 0 && OFF_V % 1024 == 0, "alignment");
 static_assert(OFF_Y + 3 * 16 * 17 * 4 <= OFF_R1 + R1_BYTES, "R1 layout");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -139,8 +139,8 @@ struct Params {
 __device__ __forceinline__ uint32_t bar_addr(uint32_t sb, int i) { return sb + OFF_BAR + 8u * i; }
 
 __device__ __forceinline__ bool epi_wait(uint32_t bar, uint32_t parity, int etid,
-                                         volatile int *abort, int32_t *status, uint64_t tmo) {
-  return group_wait<NEPI, EPI_BAR>(bar, parity, etid, abort, status, tmo);
+                                         volatile int *ctl, int32_t *status) {
+  return group_wait<NEPI, EPI_BAR>(bar, parity, etid, ctl, status);
 }
 
 template <typename TO>
@@ -179,10 +179,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     return;
   }
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  const uint64_t tmo = wait_limit_ns(p.status);
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
-    *abort_flag = 0;
+    abort_flag[CTL_ABORT] = 0;
+    abort_flag[CTL_LIMIT] = 0;  // 2 s until warp 3 has read the header
+    abort_flag[CTL_GROUP] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -217,7 +218,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
           tma_prefetch_3d(&tm_v, 0, h, t); tma_prefetch_3d(&tm_v, 64, h, t);
         }
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag, tmo)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag)) break;
         const uint32_t st = sb + OFF_QK + s * QK_STAGE;
         const uint32_t fb = bar_addr(sb, B_FULL_QK + s);
         mbar_arrive_expect_tx(fb, QK_STAGE);
@@ -226,7 +227,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tma_load_3d(st + 8192, &tm_k, fb, 0, j, t0);
         tma_load_3d(st + 24576, &tm_k, fb, 64, j, t0);
         issued_qk = c + 1;
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_V + sv), ((c / NV) & 1) ^ 1, abort_flag, tmo)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_V + sv), ((c / NV) & 1) ^ 1, abort_flag)) break;
         const uint32_t vs = sb + OFF_V + sv * V_STAGE;
         const uint32_t fv = bar_addr(sb, B_FULL_V + sv);
         mbar_arrive_expect_tx(fv, V_STAGE);
@@ -263,8 +264,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint64_t dQK = dQK0 + s * (QK_STAGE >> 4), dKmn = dKmn0 + s * (QK_STAGE >> 4);
         const uint64_t dVmn = dVmn0 + sv * (V_STAGE >> 4);
         // [Q;K] K^T
-        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), (c / NQK) & 1, abort_flag, tmo);
-        if (ok && c > 0) ok = mbar_wait(bar_addr(sb, B_DONE), (c - 1) & 1, abort_flag, tmo);
+        ok = mbar_wait(bar_addr(sb, B_FULL_QK + s), (c / NQK) & 1, abort_flag);
+        if (ok && c > 0) ok = mbar_wait(bar_addr(sb, B_DONE), (c - 1) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -274,8 +275,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         mma_commit(bar_addr(sb, B_QK));
         // W^T = K^T (T'h + T'l)^T ;  U~^T = V^T (T''h + T''l)^T
-        ok = mbar_wait(bar_addr(sb, B_T), ph, abort_flag, tmo) &&
-             mbar_wait(bar_addr(sb, B_FULL_V + sv), (c / NV) & 1, abort_flag, tmo);
+        ok = mbar_wait(bar_addr(sb, B_T), ph, abort_flag) &&
+             mbar_wait(bar_addr(sb, B_FULL_V + sv), (c / NV) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -291,7 +292,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mma_commit(bar_addr(sb, B_W));
         mma_commit(bar_addr(sb, B_EMPTY_V + sv));
         // U^T = U~^T - S0h W^T ;  Oi^T = (S0h + S0l) Q^T   (S0 from TMEM)
-        ok = mbar_wait(bar_addr(sb, B_WT), ph, abort_flag, tmo);
+        ok = mbar_wait(bar_addr(sb, B_WT), ph, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -306,7 +307,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         mma_commit(bar_addr(sb, B_U));
         // dS = (Ukh + Ukl)^T K ;  Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T   (U from TMEM)
-        ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag, tmo);
+        ok = mbar_wait(bar_addr(sb, B_UT), ph, abort_flag);
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -330,7 +331,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
       }
       // Drain: every MMA this thread issued finishes before TMEM is freed.
-      const uint32_t drain = sb + OFF_MISC + 8;
+      const uint32_t drain = sb + OFF_MISC + 16;
       mbar_init(drain, 1);
       fence_barrier_init();
       mma_commit(drain);
@@ -341,7 +342,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int c = 0; c < nch; ++c) {
       const int s = c & 1;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar_addr(sb, B_SCAL_EMPTY + s), ((c >> 1) & 1) ^ 1, abort_flag, tmo);
+      if (lane == 0) ok = mbar_wait(bar_addr(sb, B_SCAL_EMPTY + s), ((c >> 1) & 1) ^ 1, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) { *abort_flag = 1; report_status(p.status, GDN_ERR_DEVICE_TIMEOUT); }
@@ -413,6 +414,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_addr(sb, B_SCAL_FULL + s));
     }
+  } else if (warp == 3) {
+    // the caller's wait limit (a global load kept off the other roles' start)
+    if (lane == 0) abort_flag[CTL_LIMIT] = (int)header_wait_limit_us(p.status);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int etid = tid - 128;
@@ -450,12 +454,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
       // ---- Q K^T and K K^T -> P (hi/lo) and A (fp32)
       if (etid == 0) {
-        if (!mbar_wait(bar_addr(sb, B_SCAL_FULL + s), (c >> 1) & 1, abort_flag, tmo)) {
-          *abort_flag = 1;
+        if (!mbar_wait(bar_addr(sb, B_SCAL_FULL + s), (c >> 1) & 1, abort_flag)) {
+          abort_flag[CTL_ABORT] = 1;
+          abort_flag[CTL_GROUP] = 1;  // the group's waiter: the next group wait gives up
           report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
         }
       }
-      if (!epi_wait(bar_addr(sb, B_QK), ph, etid, abort_flag, p.status, tmo)) break;
+      if (!epi_wait(bar_addr(sb, B_QK), ph, etid, abort_flag, p.status)) break;
       {
         float v[16];
         tmem_ld16(tl + R_QK + 16 * ewq, v);
@@ -524,7 +529,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (etid == 0) mbar_arrive(bar_addr(sb, B_T));
 
       // ---- W^T -> bf16 (MN-major B)
-      if (!epi_wait(bar_addr(sb, B_W), ph, etid, abort_flag, p.status, tmo)) break;
+      if (!epi_wait(bar_addr(sb, B_W), ph, etid, abort_flag, p.status)) break;
       {
         float v[16];
         tmem_ld16(tl + R_W + 16 * ewq, v);
@@ -538,7 +543,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (etid == 0) mbar_arrive(bar_addr(sb, B_WT));
 
       // ---- U^T -> hi/lo (for P) and U^T diag(kdec) -> hi/lo (for the state), into TMEM
-      if (!epi_wait(bar_addr(sb, B_U), ph, etid, abort_flag, p.status, tmo)) break;
+      if (!epi_wait(bar_addr(sb, B_U), ph, etid, abort_flag, p.status)) break;
       {
         float v[16];
         tmem_ld16(tl + R_UO + 16 * ewq, v);
@@ -559,7 +564,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (etid == 0) mbar_arrive(bar_addr(sb, B_UT));
 
       // ---- state: S = gamma_C S + dS (fp32), S0 <- hi/lo(S); outputs
-      if (!epi_wait(bar_addr(sb, B_S), ph, etid, abort_flag, p.status, tmo)) break;
+      if (!epi_wait(bar_addr(sb, B_S), ph, etid, abort_flag, p.status)) break;
       {
         const float gC = sc[256];
         {

@@ -55,17 +55,24 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase with the given parity to complete, with try_wait (the
 // waiting thread is suspended between checks and takes no issue slots from
-// the warps doing the work).  Gives up (returns false) after `timeout_ns` or
-// as soon as *abort becomes nonzero, so a lost arrival can never hang the GPU.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          uint64_t timeout_ns = 2000000000ull) {
+// the warps doing the work).  `ctl` points at the CTA's control words in
+// shared memory: ctl[0] its abort flag, ctl[1] the wait limit in microseconds
+// (0 for the default of 2 s).  Gives up (returns false) once the limit has
+// passed or as soon as the abort flag is set, so a lost arrival can never hang
+// the GPU.  Only the slow path reads them; with the default limit they are
+// checked every 64 attempts, with a set limit after every attempt (a suspended
+// try_wait can outlast a limit of a few microseconds).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *ctl) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t us = static_cast<uint32_t>(ctl[1]);
+  const uint64_t limit_ns = us ? (uint64_t)us * 1000ull : 2000000000ull;
+  const uint32_t every = us ? 0u : 63u;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > timeout_ns) return false;
+    if ((i & every) == 0) {
+      if (ctl[0]) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
 }
@@ -90,18 +97,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
-// Named barrier that also ORs one predicate over the `nthreads` threads: every
-// thread gets the same result, so a group can take a uniform branch on it.
-__device__ __forceinline__ bool named_bar_or(uint32_t id, uint32_t nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{ .reg .pred p, q; setp.ne.u32 p, %1, 0; barrier.red.or.pred q, %2, %3, p; selp.u32 %0, 1, 0, q; }"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 // One lane of a converged warp (the same lane for the same active mask).
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred;

@@ -138,8 +138,8 @@ constexpr uint32_t QK_STAGE = 32768;   // [Q d0-63 | K d0-63 | Q d64-127 | K d64
 constexpr uint32_t OFF_QK = 0;
 constexpr uint32_t OFF_REC = NQK * QK_STAGE;
 constexpr uint32_t OFF_BAR = OFF_REC + NR * REC_BYTES;
-constexpr uint32_t OFF_MISC = OFF_BAR + 256;  // [0] TMEM base, [4] abort flag, [8] drain mbarrier
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+constexpr uint32_t OFF_MISC = OFF_BAR + 256;  // [0] TMEM base, [4] control words (chunk::CTL_*), [16] drain mbarrier
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 24;
 static_assert(OFF_REC % 1024 == 0 && REC_BYTES % 1024 == 0, "alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -223,12 +223,13 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     return;
   }
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  const uint64_t tmo = wait_limit_ns(p.status);
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
     // a record slot is free once its MMAs completed AND the epilogue read it
     for (int i = 0; i < NR; ++i) mbar_init(bar_addr(sb, B_EMPTY_R + i), 2);
-    *abort_flag = 0;
+    abort_flag[CTL_ABORT] = 0;
+    abort_flag[CTL_LIMIT] = 0;  // 2 s until warp 3 has read the header
+    abort_flag[CTL_GROUP] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -266,7 +267,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tma_prefetch_3d(&tm_k, 0, j, t); tma_prefetch_3d(&tm_k, 64, j, t);
           bulk_prefetch_l2(chunk_rec(c + PF), REC_BYTES);
         }
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag, tmo)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_QK + s), ((c / NQK) & 1) ^ 1, abort_flag)) break;
         const uint32_t st = sb + OFF_QK + s * QK_STAGE;
         const uint32_t fb = bar_addr(sb, B_FULL_QK + s);
         mbar_arrive_expect_tx(fb, QK_STAGE);
@@ -275,7 +276,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tma_load_3d(st + 8192, &tm_k, fb, 0, j, t0);
         tma_load_3d(st + 24576, &tm_k, fb, 64, j, t0);
         issued_qk = c + 1;
-        if (!mbar_wait(bar_addr(sb, B_EMPTY_R + sr), ((c / NR) & 1) ^ 1, abort_flag, tmo)) break;
+        if (!mbar_wait(bar_addr(sb, B_EMPTY_R + sr), ((c / NR) & 1) ^ 1, abort_flag)) break;
         const uint32_t fr = bar_addr(sb, B_FULL_R + sr);
         mbar_arrive_expect_tx(fr, REC_BYTES);
         bulk_load(sb + OFF_REC + sr * REC_BYTES, chunk_rec(c), REC_BYTES, fr);
@@ -304,7 +305,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint64_t dP0 = sdesc_sw128(sb + OFF_REC + tp::REC_PH, 16, 1024);    // P hi / lo, K-major
     auto wait = [&](int b, uint32_t parity) {
       int ok = 1;
-      if (lane == 0) ok = mbar_wait(bar_addr(sb, b), parity, abort_flag, tmo);
+      if (lane == 0) ok = mbar_wait(bar_addr(sb, b), parity, abort_flag);
       return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
     bool ok = true;
@@ -378,16 +379,15 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mbar_wait_landed(bar_addr(sb, B_DRAIN), 0, 50000000ull);
     }
     __syncwarp();
+  } else if (warp == 3) {
+    // the caller's wait limit (a global load kept off the other roles' start)
+    if (lane == 0) abort_flag[CTL_LIMIT] = (int)header_wait_limit_us(p.status);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int etid = tid - 128;
     const int ewq = etid >> 7;   // column quarter
     const int row = etid & 127;  // TMEM lane = row (Dv index) of the 128-row tiles
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
-    auto fail = [&]() {
-      *abort_flag = 1;
-      report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
-    };
 
     // fp32 master state: row `row`, columns [32 ewq, 32 ewq + 32); S0 = hi + lo in TMEM
     float S[32];
@@ -416,12 +416,9 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     float un[16];
     auto fetch_ut = [&](int c) {
       const int sr = c % NR;
-      bool failed = false;
-      if (etid == 0 && !mbar_wait(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, abort_flag, tmo)) {
-        fail();
-        failed = true;
-      }
-      if (group_aborted<NEPI, EPI_BAR>(abort_flag, failed)) return false;
+      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, etid, abort_flag,
+                                     p.status))
+        return false;
       const float *ut = reinterpret_cast<const float *>(smem + OFF_REC + sr * REC_BYTES + tp::REC_UT) + row;
 #pragma unroll
       for (int x = 0; x < 16; ++x) un[x] = ut[(16 * ewq + x) * HD];
@@ -450,7 +447,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float *kdec = gam + 64;
 
       // ---- U = (U - U~) + U~ -> hi/lo(U^T diag(kdec)) for dS first, then hi/lo(U^T) for Oa
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_U), ph, etid, abort_flag, p.status, tmo))) break;
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_U), ph, etid, abort_flag, p.status))) break;
       {
         float v[16];
         tmem_ld16(tl + R_S + 16 * ewq, v);
@@ -485,7 +482,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       store_out(1);
 
       // ---- state: S = gamma_C S + dS (fp32); hi(S) first (the next U product), then lo(S)
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_S), ph, etid, abort_flag, p.status, tmo))) break;
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_S), ph, etid, abort_flag, p.status))) break;
       {
         const float gC = gam[128];
 #pragma unroll
@@ -518,7 +515,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       store_out(3);
 
       // ---- outputs o_t = scale (e^{G_t} Oi_t + Oa_t) out of TMEM
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_OA), ph, etid, abort_flag, p.status, tmo))) break;
+      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_OA), ph, etid, abort_flag, p.status))) break;
       {
         float va[16];
         tmem_ld16(tl + R_OI + 16 * ewq, out);

@@ -63,8 +63,8 @@ constexpr uint32_t OFF_TQH = OFF_QK;           // hi/lo(T'') over the Q halves, 
 constexpr uint32_t OFF_TQL = OFF_QK + 16384;
 constexpr uint32_t OFF_SCAL = OFF_R1 + 38912;  // G2 (log2 prefix), gamma, kdec, beta, 1/|q|, 1/|k| [64 each]
 constexpr uint32_t OFF_BAR = OFF_SCAL + 1792;
-constexpr uint32_t OFF_MISC = OFF_BAR + 64;    // [0] TMEM base, [4] abort flag, [8] drain mbarrier
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 16;
+constexpr uint32_t OFF_MISC = OFF_BAR + 64;    // [0] TMEM base, [4] control words (chunk::CTL_*), [16] drain mbarrier
+constexpr uint32_t SMEM_BYTES = OFF_MISC + 24;
 static_assert(OFF_Y + 3 * 16 * 17 * 4 <= OFF_SCAL, "R1 layout");
 static_assert(OFF_R1 % 1024 == 0 && OFF_TPL % 1024 == 0 && OFF_V % 1024 == 0, "alignment");
 static_assert(2 * SMEM_BYTES <= 232448 - 2048, "two CTAs per SM");
@@ -116,10 +116,11 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     return;
   }
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
-  const uint64_t tmo = wait_limit_ns(p.status);
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
-    *abort_flag = 0;
+    abort_flag[CTL_ABORT] = 0;
+    abort_flag[CTL_LIMIT] = 0;  // 2 s until warp 3 has read the header
+    abort_flag[CTL_GROUP] = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -172,7 +173,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const uint64_t dVmn = sdesc_sw128(sb + OFF_V, 8192, 1024);           // V^T, MN-major
       const uint64_t dTP = sdesc_sw128(sb + OFF_TPH, 16, 1024);            // T', K-major
       const uint64_t dTQ = sdesc_sw128(sb + OFF_TQH, 16, 1024);            // T'', K-major
-      bool ok = mbar_wait(bar_addr(sb, B_QKF), 0, abort_flag, tmo);
+      bool ok = mbar_wait(bar_addr(sb, B_QKF), 0, abort_flag);
       if (ok) {
         tc_fence_after();
 #pragma unroll
@@ -181,7 +182,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           mma_bf16(tmem + R_QK, dQK + k16, dQK + (8192 >> 4) + k16, IDESC_QK, ks > 0);
         }
         mma_commit(bar_addr(sb, B_QK));
-        ok = mbar_wait(bar_addr(sb, B_T), 0, abort_flag, tmo) && mbar_wait(bar_addr(sb, B_VF), 0, abort_flag, tmo);
+        ok = mbar_wait(bar_addr(sb, B_T), 0, abort_flag) && mbar_wait(bar_addr(sb, B_VF), 0, abort_flag);
       }
       if (ok) {
         tc_fence_after();
@@ -203,7 +204,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
       }
       // Drain: every MMA this thread issued finishes before TMEM is freed.
-      const uint32_t drain = sb + OFF_MISC + 8;
+      const uint32_t drain = sb + OFF_MISC + 16;
       mbar_init(drain, 1);
       fence_barrier_init();
       mma_commit(drain);
@@ -251,6 +252,9 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (lane == 0) rs[128] = exp2f(GL);
     __syncwarp();
     if (lane == 0) mbar_arrive(bar_addr(sb, B_SCAL));
+  } else if (warp == 3) {
+    // the caller's wait limit (a global load kept off the other roles' start)
+    if (lane == 0) abort_flag[CTL_LIMIT] = (int)header_wait_limit_us(p.status);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
     const int etid = tid - 128;
@@ -263,8 +267,9 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const float *sc = reinterpret_cast<const float *>(smem + OFF_SCAL);
     const float *G2 = sc, *gam = sc + 64, *bet = sc + 192, *rqn = sc + 256, *rkn = sc + 320;
     do {
-      if (etid == 0 && !mbar_wait(bar_addr(sb, B_SCAL), 0, abort_flag, tmo)) {
-        *abort_flag = 1;
+      if (etid == 0 && !mbar_wait(bar_addr(sb, B_SCAL), 0, abort_flag)) {
+        abort_flag[CTL_ABORT] = 1;
+        abort_flag[CTL_GROUP] = 1;  // the group's waiter: the next group wait gives up
         report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
       }
       if (p.raw) {
@@ -275,7 +280,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // into the bf16 operand tiles: P and A gain 1/|q_t| 1/|k_s| and
         // 1/|k_t| 1/|k_s|, T' gains 1/|k_s|, and the record's e^{G_t} and
         // e^{G_C - G_t} gain 1/|q_t| and 1/|k_t| for the state pass.
-        if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QKF), 0, etid, abort_flag, p.status, tmo)) break;
+        if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QKF), 0, etid, abort_flag, p.status)) break;
         const int rr = etid >> 1, t = rr & 63;
         const unsigned char *seg = smem + OFF_QK + (rr >> 6) * 8192 + (etid & 1) * 16384 + t * 128;
         float ss = 0.f;
@@ -298,7 +303,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           rs[rr] = sc[64 + rr] * r;  // e^{G_t} / |q_t|, then e^{G_C - G_t} / |k_t|
         }
       }
-      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QK), 0, etid, abort_flag, p.status, tmo)) break;
+      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_QK), 0, etid, abort_flag, p.status)) break;
       // ---- Q K^T -> P (record, hi/lo), K K^T -> A (fp32, shared)
 #pragma unroll
       for (int qh = 0; qh < 2; ++qh) {
@@ -361,7 +366,7 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       if (etid == 0) mbar_arrive(bar_addr(sb, B_T));
 
       // ---- W^T -> record (bf16 MN-major image), U~ -> record (fp32 [t][d])
-      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_W), 0, etid, abort_flag, p.status, tmo)) break;
+      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_W), 0, etid, abort_flag, p.status)) break;
       {
         float v[32];
         tmem_ld32(tl + R_W + 32 * half, v);

@@ -130,7 +130,6 @@ using tp::REC_BYTES;
 
 constexpr int NTHREADS = 640;
 constexpr int NEPI = 512;   // epilogue threads: 4 column quarters x 128 rows
-constexpr int EPI_BAR = 1;  // named barrier of the epilogue threads
 
 // ---- shared memory map (bytes) ----
 constexpr int NQK = 2, NR = 2;         // ring depths: Q/K tiles, chunk records
@@ -225,8 +224,11 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
-    // a record slot is free once its MMAs completed AND the epilogue read it
-    for (int i = 0; i < NR; ++i) mbar_init(bar_addr(sb, B_EMPTY_R + i), 2);
+    // barriers the 16 epilogue warps arrive on, one arrival per warp
+    for (int b : {(int)B_S0H, (int)B_S0L, (int)B_UK, (int)B_UO, (int)B_OFREE})
+      mbar_init(bar_addr(sb, b), NEPI / 32);
+    // a record slot is free once its MMAs completed AND every epilogue warp read it
+    for (int i = 0; i < NR; ++i) mbar_init(bar_addr(sb, B_EMPTY_R + i), 1 + NEPI / 32);
     abort_flag[CTL_ABORT] = 0;
     abort_flag[CTL_LIMIT] = 0;  // 2 s until warp 3 has read the header
     abort_flag[CTL_GROUP] = 0;
@@ -384,10 +386,30 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (lane == 0) abort_flag[CTL_LIMIT] = (int)header_wait_limit_us(p.status);
   } else if (warp >= 4) {
     // ------------------------------------------------------------ epilogue
+    // 16 warps, each on its own: a warp waits for an MMA group through its
+    // lane 0 and signals the MMA issuer by one arrival per warp (the barriers
+    // the issuer waits on count 16), so no barrier spans the epilogue warps
+    // and a slow warp delays only the MMAs that need its columns.
     const int etid = tid - 128;
     const int ewq = etid >> 7;   // column quarter
     const int row = etid & 127;  // TMEM lane = row (Dv index) of the 128-row tiles
     const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+    auto warp_wait = [&](int b, uint32_t parity) {
+      int ok = 1;
+      if (lane == 0 && !(ok = mbar_wait(bar_addr(sb, b), parity, abort_flag))) {
+        abort_flag[CTL_ABORT] = 1;
+        report_status(p.status, GDN_ERR_DEVICE_TIMEOUT);
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok) tc_fence_after();
+      return ok != 0;
+    };
+    // after this warp's tcgen05.st have completed (tmem_wait_st)
+    auto warp_signal = [&](int b) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(sb, b));
+    };
 
     // fp32 master state: row `row`, columns [32 ewq, 32 ewq + 32); S0 = hi + lo in TMEM
     float S[32];
@@ -404,21 +426,15 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tmem_st16(tl + T_S0L + 16 * ewq, lw);
       tmem_wait_st();
     }
-    tc_fence_before();
-    named_bar_sync(EPI_BAR, NEPI);
-    if (etid == 0) {
-      mbar_arrive(bar_addr(sb, B_S0H));
-      mbar_arrive(bar_addr(sb, B_S0L));
-    }
+    warp_signal(B_S0H);
+    warp_signal(B_S0L);
 
     // U~ of the chunk about to run, read from its record while the previous
     // chunk's dS product runs
     float un[16];
     auto fetch_ut = [&](int c) {
       const int sr = c % NR;
-      if (!group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_FULL_R + sr), (c / NR) & 1, etid, abort_flag,
-                                     p.status))
-        return false;
+      if (!warp_wait(B_FULL_R + sr, (c / NR) & 1)) return false;
       const float *ut = reinterpret_cast<const float *>(smem + OFF_REC + sr * REC_BYTES + tp::REC_UT) + row;
 #pragma unroll
       for (int x = 0; x < 16; ++x) un[x] = ut[(16 * ewq + x) * HD];
@@ -428,14 +444,13 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // during chunk c + 1, a quarter at each of its four waits, so that the
     // store path drains in the background.
     float out[16];
-    int out_t0 = 0, out_Lc = 0;  // tokens of the chunk whose outputs `out` holds
+    int out_t0 = 0, out_n = 0;  // this thread's first token of the chunk whose outputs `out`
+                                // holds, and how many of its 16 tokens that chunk has
     auto store_out = [&](int part) {
       TO *op = static_cast<TO *>(p.o) + ((size_t)out_t0 * p.Hv + h) * HD + row;
 #pragma unroll
-      for (int x = 4 * part; x < 4 * part + 4; ++x) {
-        const int t = 16 * ewq + x;
-        if (t < out_Lc) op[(size_t)t * p.Hv * HD] = from_f32<TO>(out[x]);
-      }
+      for (int x = 4 * part; x < 4 * part + 4; ++x)
+        if (x < out_n) op[(size_t)x * p.Hv * HD] = from_f32<TO>(out[x]);
     };
     bool ok = fetch_ut(0);
     for (int c = 0; c < nch && ok; ++c) {
@@ -447,27 +462,32 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float *kdec = gam + 64;
 
       // ---- U = (U - U~) + U~ -> hi/lo(U^T diag(kdec)) for dS first, then hi/lo(U^T) for Oa
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_U), ph, etid, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(B_U, ph))) break;
       {
         float v[16];
         tmem_ld16(tl + R_S + 16 * ewq, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int x = 0; x < 16; ++x) v[x] += un[x];
+        for (int x = 0; x < 16; x += 2) {
+          const float2 a = __fadd2_rn(make_float2(v[x], v[x + 1]), make_float2(un[x], un[x + 1]));
+          v[x] = a.x; v[x + 1] = a.y;
+        }
 #pragma unroll
         for (int hq = 0; hq < 2; ++hq) {
-          float w[8];
-#pragma unroll
-          for (int x = 0; x < 8; ++x) w[x] = v[8 * hq + x] * kdec[16 * ewq + 8 * hq + x];
+          const float4 ka = *reinterpret_cast<const float4 *>(kdec + 16 * ewq + 8 * hq);
+          const float4 kb = *reinterpret_cast<const float4 *>(kdec + 16 * ewq + 8 * hq + 4);
+          const float2 w0 = __fmul2_rn(make_float2(v[8 * hq + 0], v[8 * hq + 1]), make_float2(ka.x, ka.y));
+          const float2 w1 = __fmul2_rn(make_float2(v[8 * hq + 2], v[8 * hq + 3]), make_float2(ka.z, ka.w));
+          const float2 w2 = __fmul2_rn(make_float2(v[8 * hq + 4], v[8 * hq + 5]), make_float2(kb.x, kb.y));
+          const float2 w3 = __fmul2_rn(make_float2(v[8 * hq + 6], v[8 * hq + 7]), make_float2(kb.z, kb.w));
+          const float w[8] = {w0.x, w0.y, w1.x, w1.y, w2.x, w2.y, w3.x, w3.y};
           uint32_t hw[4], lw[4];
           split_words<4>(w, hw, lw);
           tmem_st4(tl + T_UKH + 8 * ewq + 4 * hq, hw);
           tmem_st4(tl + T_UKL + 8 * ewq + 4 * hq, lw);
         }
         tmem_wait_st();
-        tc_fence_before();
-        named_bar_sync(EPI_BAR, NEPI);
-        if (etid == 0) mbar_arrive(bar_addr(sb, B_UK));
+        warp_signal(B_UK);
         store_out(0);
         uint32_t hw[8], lw[8];
         split_words<8>(v, hw, lw);
@@ -475,32 +495,32 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tmem_st8(tl + T_UL + 8 * ewq, lw);
         tmem_wait_st();
       }
-      tc_fence_before();
-      named_bar_sync(EPI_BAR, NEPI);
-      if (etid == 0) mbar_arrive(bar_addr(sb, B_UO));
-
+      warp_signal(B_UO);
       store_out(1);
 
       // ---- state: S = gamma_C S + dS (fp32); hi(S) first (the next U product), then lo(S)
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_S), ph, etid, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(B_S, ph))) break;
       {
         const float gC = gam[128];
+        const float2 g2 = make_float2(gC, gC);
 #pragma unroll
         for (int hq = 0; hq < 2; ++hq) {
           float v[16];
           tmem_ld16(tl + R_S + 32 * ewq + 16 * hq, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int x = 0; x < 16; ++x) S[16 * hq + x] = fmaf(gC, S[16 * hq + x], v[x]);
+          for (int x = 0; x < 16; x += 2) {
+            const float2 a = __ffma2_rn(g2, make_float2(S[16 * hq + x], S[16 * hq + x + 1]),
+                                        make_float2(v[x], v[x + 1]));
+            S[16 * hq + x] = a.x; S[16 * hq + x + 1] = a.y;
+          }
           uint32_t hw[8];
           hi_words<8>(S + 16 * hq, hw);
           tmem_st8(tl + T_S0H + 16 * ewq + 8 * hq, hw);
         }
         tmem_wait_st();
       }
-      tc_fence_before();
-      named_bar_sync(EPI_BAR, NEPI);
-      if (etid == 0) mbar_arrive(bar_addr(sb, B_S0H));
+      warp_signal(B_S0H);
       store_out(2);
 #pragma unroll
       for (int hq = 0; hq < 2; ++hq) {
@@ -509,33 +529,37 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tmem_st8(tl + T_S0L + 16 * ewq + 8 * hq, lw);
       }
       tmem_wait_st();
-      tc_fence_before();
-      named_bar_sync(EPI_BAR, NEPI);
-      if (etid == 0) mbar_arrive(bar_addr(sb, B_S0L));
+      warp_signal(B_S0L);
       store_out(3);
 
       // ---- outputs o_t = scale (e^{G_t} Oi_t + Oa_t) out of TMEM
-      if (!(ok = group_wait<NEPI, EPI_BAR>(bar_addr(sb, B_OA), ph, etid, abort_flag, p.status))) break;
+      if (!(ok = warp_wait(B_OA, ph))) break;
       {
         float va[16];
         tmem_ld16(tl + R_OI + 16 * ewq, out);
         tmem_ld16(tl + R_OA + 16 * ewq, va);
         tmem_wait_ld();
+        const float2 sc2 = make_float2(p.scale, p.scale);
 #pragma unroll
-        for (int x = 0; x < 16; ++x) out[x] = p.scale * fmaf(gam[16 * ewq + x], out[x], va[x]);
+        for (int x = 0; x < 16; x += 4) {
+          const float4 g4 = *reinterpret_cast<const float4 *>(gam + 16 * ewq + x);
+          const float2 a = __ffma2_rn(make_float2(g4.x, g4.y), make_float2(out[x], out[x + 1]),
+                                      make_float2(va[x], va[x + 1]));
+          const float2 b = __ffma2_rn(make_float2(g4.z, g4.w), make_float2(out[x + 2], out[x + 3]),
+                                      make_float2(va[x + 2], va[x + 3]));
+          const float2 a2 = __fmul2_rn(sc2, a), b2 = __fmul2_rn(sc2, b);
+          out[x] = a2.x; out[x + 1] = a2.y; out[x + 2] = b2.x; out[x + 3] = b2.y;
+        }
       }
-      out_t0 = t0;
-      out_Lc = Lc;
-      tc_fence_before();
-      named_bar_sync(EPI_BAR, NEPI);
-      if (etid == 0) {
-        mbar_arrive(bar_addr(sb, B_OFREE));
-        mbar_arrive(bar_addr(sb, B_EMPTY_R + sr));
-      }
+      out_t0 = t0 + 16 * ewq;
+      out_n = min(16, Lc - 16 * ewq);
+      warp_signal(B_OFREE);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_addr(sb, B_EMPTY_R + sr));  // this warp is done with the record
       // ---- the next chunk's U~, while its U product runs
       if (c + 1 < nch && !(ok = fetch_ut(c + 1))) break;
     }
-    if (ok && *abort_flag == 0) {
+    if (ok && abort_flag[CTL_ABORT] == 0) {
 #pragma unroll
       for (int part = 0; part < 4; ++part) store_out(part);
       if (dst) {

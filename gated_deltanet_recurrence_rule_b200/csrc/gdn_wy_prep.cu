@@ -122,6 +122,17 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     abort_flag[CTL_LIMIT] = 0;  // 2 s until warp 3 has read the header
     abort_flag[CTL_GROUP] = 0;
     fence_barrier_init();
+    // the tiles first: their latency then overlaps the TMEM allocation and
+    // the CTA-wide barrier below
+    const uint32_t fq = bar_addr(sb, B_QKF), fv = bar_addr(sb, B_VF);
+    mbar_arrive_expect_tx(fq, 32768);
+    tma_load_3d(sb + OFF_QK + 0, &tm_q, fq, 0, j, t0);
+    tma_load_3d(sb + OFF_QK + 8192, &tm_k, fq, 0, j, t0);
+    tma_load_3d(sb + OFF_QK + 16384, &tm_q, fq, 64, j, t0);
+    tma_load_3d(sb + OFF_QK + 24576, &tm_k, fq, 64, j, t0);
+    mbar_arrive_expect_tx(fv, 16384);
+    tma_load_3d(sb + OFF_V + 0, &tm_v, fv, 0, h, t0);
+    tma_load_3d(sb + OFF_V + 8192, &tm_v, fv, 64, h, t0);
   }
   if (warp == 1) {
     tmem_alloc(sb + OFF_MISC, TMEM_COLS);
@@ -136,14 +147,6 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------------------------------------ TMA loads
     if (lane == 0) {
       const uint32_t fq = bar_addr(sb, B_QKF), fv = bar_addr(sb, B_VF);
-      mbar_arrive_expect_tx(fq, 32768);
-      tma_load_3d(sb + OFF_QK + 0, &tm_q, fq, 0, j, t0);
-      tma_load_3d(sb + OFF_QK + 8192, &tm_k, fq, 0, j, t0);
-      tma_load_3d(sb + OFF_QK + 16384, &tm_q, fq, 64, j, t0);
-      tma_load_3d(sb + OFF_QK + 24576, &tm_k, fq, 64, j, t0);
-      mbar_arrive_expect_tx(fv, 16384);
-      tma_load_3d(sb + OFF_V + 0, &tm_v, fv, 0, h, t0);
-      tma_load_3d(sb + OFF_V + 8192, &tm_v, fv, 64, h, t0);
       // Warm L2 with the tiles of the CTA that will most likely take this
       // slot next (CTAs start in linear order), so that its loads hit L2.
       const int lin = (int)(blockIdx.y * gridDim.x + blockIdx.x) + p.resident;

@@ -181,3 +181,47 @@ def test_bf16_state_many_calls():
         assert_parity(torch.bfloat16, to_np(o).reshape(B * Tn, Hv, D), o_ref, to_np(S), ref,
                       f"{calls} calls of {Tn}")
         assert state_error(to_np(S), ref) <= 1e-3, f"{calls} calls of {Tn}: state diverged"
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("in_place", [False, True])
+def test_bf16_pool_many_units(D, in_place):
+    """A batch large enough that the bf16-pool kernel's persistent CTAs take
+    several (sequence, head) units each, double-buffering their states: a
+    shuffled slot map, padding entries and an invalid slot mixed in, against
+    the oracle (one rounding at rest) unit by unit."""
+    B, Hqk, Hv, Tn = 300, 2, 6, 3
+    slots = B + 20
+    inp, x, pool = _case(B, Tn, Hqk, Hv, D, "bf16", seed=95 + D, num_slots=slots)
+    pool = pool.to(torch.bfloat16)
+    perm = torch.randperm(slots, generator=torch.Generator().manual_seed(7)).tolist()
+    src = perm[:B]
+    pad = set(range(5, B, 37))           # padding entries
+    bad = 11                             # a real sequence with an invalid source slot
+    src = [-1 if b in pad else s for b, s in enumerate(src)]
+    src[bad] = slots + 3
+    # destinations (out of place): distinct slots of another permutation
+    dst = list(src) if in_place else perm[::-1][:B]
+    pin = pool.to(DEV)
+    pout = pin if in_place else torch.full_like(pin, float("nan"))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o = torch.full((B, Tn, Hv, D), 7.0, device=DEV)
+    api.decode_tokens(*(x[n].to(DEV) for n in ("q", "k", "v", "g", "beta")), pin, pout,
+                      src_slot=torch.tensor(src, dtype=torch.int32, device=DEV),
+                      dst_slot=None if in_place else torch.tensor(dst, dtype=torch.int32, device=DEV),
+                      o=o, device_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == api.GDN_ERR_INVALID_ARG      # the invalid slot, reported
+    real = [b for b in range(B) if b not in pad and b != bad]
+    for b in pad | {bad}:
+        assert (o[b] == 7).all()                                # skipped: o untouched
+    idx = torch.tensor(real)
+    sub = inputs.prefill_inputs([Tn] * len(real), Hqk, Hv, D, dtype="bf16", seed=0)
+    for n in ("q", "k", "v", "g", "beta"):
+        sub[n] = x[n][idx].reshape(len(real) * Tn, *x[n].shape[2:]).contiguous()
+    sub["cu_seqlens"] = torch.arange(0, len(real) * Tn + 1, Tn, dtype=torch.int32)
+    o_ref, f_ref = _oracle(sub, pool, [src[b] for b in real], state_at_rest="bf16")
+    assert_parity(torch.bfloat16, to_np(o[idx]).reshape(len(real) * Tn, Hv, D), o_ref,
+                  what="many units")
+    s_gpu = to_np(pout[torch.tensor([src[b] if in_place else dst[b] for b in real])])
+    assert state_error_bf16_rest(s_gpu, f_ref) <= 1.0

@@ -75,10 +75,13 @@ def load():
                                           i32, i32, i32, i32, i32, i32, i32, f32, vp, vp]
         lib.gdn_prefill_backward_workspace_size.restype = sz
         lib.gdn_prefill_backward_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
-        lib.gdn_prefill_backward.restype = i32
-        lib.gdn_prefill_backward.argtypes = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32,
-                                             i32, f32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz,
-                                             vp]
+        lib.gdn_prefill_backward_workspace_size_sequential.restype = sz
+        lib.gdn_prefill_backward_workspace_size_sequential.argtypes = [i32, i64, i32, i32, i32, i32]
+        bwd_args = [vp, vp, vp, vp, vp, vp, i32, i64, i32, i32, i32, i32, i32, f32, vp, vp, vp, vp,
+                    vp, vp, vp, vp, vp, vp, sz, vp]
+        for name in ("gdn_prefill_backward", "gdn_prefill_backward_sequential"):
+            getattr(lib, name).restype = i32
+            getattr(lib, name).argtypes = bwd_args
         lib.gdn_prefill_uses_tensor_cores.restype = i32
         lib.gdn_prefill_uses_tensor_cores.argtypes = [i32, i32, i32, i32, i32]
         lib.gdn_get_device_status.restype = i32
@@ -290,10 +293,14 @@ def decode_tokens(q, k, v, g, beta, state_in, state_out=None, src_slot=None, dst
 
 
 def prefill_backward(q, k, v, g, beta, d_o, cu_seqlens=None, initial_state=None,
-                     d_final_state=None, scale=1.0, workspace=None, want_d_initial_state=True):
+                     d_final_state=None, scale=1.0, workspace=None, want_d_initial_state=True,
+                     sequential=False):
     """Gradients of the prefill (fp32 states, prepared inputs) given d_o
     [T, Hv, Dv] fp32 and optionally d_final_state [N, Hv, Dv, Dk] fp32.
-    Returns (dq, dk, dv, dg, dbeta, d_initial_state or None), all fp32."""
+    Returns (dq, dk, dv, dg, dbeta, d_initial_state or None), all fp32.
+    ``sequential`` calls gdn_prefill_backward_sequential (token by token);
+    otherwise gdn_prefill_backward, which runs the chunk form when the
+    workspace is large enough (the default one is)."""
     lib = load()
     if not q.is_cuda:
         raise ValueError("prefill_backward runs on a CUDA device only (q is on the CPU)")
@@ -322,22 +329,29 @@ def prefill_backward(q, k, v, g, beta, d_o, cu_seqlens=None, initial_state=None,
     dv = torch.empty((T, Hv, Dv), **f32)
     dg, db = torch.empty((T, Hv), **f32), torch.empty((T, Hv), **f32)
     ds0 = torch.empty(sshape, **f32) if want_d_initial_state else None
-    need = lib.gdn_prefill_backward_workspace_size(N, T, Hqk, Hv, Dk, Dv)
+    size_fn = (lib.gdn_prefill_backward_workspace_size_sequential if sequential
+               else lib.gdn_prefill_backward_workspace_size)
+    need = size_fn(N, T, Hqk, Hv, Dk, Dv)
     if workspace is None:
         workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=dev)
     _require(workspace, "workspace", dev, torch.uint8)
-    st = lib.gdn_prefill_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
+    fn = lib.gdn_prefill_backward_sequential if sequential else lib.gdn_prefill_backward
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(cu_seqlens),
                                   N, T, Hqk, Hv, Dk, Dv, _DTYPE_CODE[dt], float(scale),
                                   _ptr(initial_state), _ptr(d_o), _ptr(d_final_state), _ptr(dq),
                                   _ptr(dk), _ptr(dv), _ptr(dg), _ptr(db), _ptr(ds0),
                                   _ptr(workspace), workspace.numel(), _stream(dev))
-    _check(st, "gdn_prefill_backward")
+    _check(st, "gdn_prefill_backward_sequential" if sequential else "gdn_prefill_backward")
     return dq, dk, dv, dg, db, ds0
 
 
-def prefill_backward_workspace_size(N, T, Hqk, Hv, Dk, Dv) -> int:
-    """Workspace bytes gdn_prefill_backward needs (0 for invalid sizes)."""
-    return int(load().gdn_prefill_backward_workspace_size(N, T, Hqk, Hv, Dk, Dv))
+def prefill_backward_workspace_size(N, T, Hqk, Hv, Dk, Dv, sequential=False) -> int:
+    """Workspace bytes gdn_prefill_backward needs for the chunk form, or with
+    ``sequential`` the token-by-token form (0 for invalid sizes)."""
+    lib = load()
+    fn = (lib.gdn_prefill_backward_workspace_size_sequential if sequential
+          else lib.gdn_prefill_backward_workspace_size)
+    return int(fn(N, T, Hqk, Hv, Dk, Dv))
 
 
 def prefill_uses_tensor_cores(Hqk, Hv, Dk, Dv, dtype=torch.bfloat16) -> bool:

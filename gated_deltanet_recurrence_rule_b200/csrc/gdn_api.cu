@@ -3,6 +3,7 @@
 // Host-side argument validation, status codes and kernel dispatch.  No entry
 // point allocates memory, keeps pointers between calls or synchronises,
 // except gdn_get_device_status, which synchronises the stream it is given.
+#include <algorithm>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -42,6 +43,13 @@ cudaError_t launch_prefill_twophase(const void *q, const void *k, const void *v,
                                     float scale, const void *s0, void *sfin, void *o,
                                     void *workspace, size_t workspace_bytes, cudaStream_t stream);
 size_t backward_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv);
+size_t backward_chunked_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv);
+cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const int32_t *cu, int N, long long T, int Hqk,
+                                    int Hv, int Dk, int Dv, int dtype, float scale, const float *s0,
+                                    const float *dO, const float *dSfin, float *dq, float *dk,
+                                    float *dv, float *dg, float *dbeta, float *ds0, void *workspace,
+                                    cudaStream_t stream);
 cudaError_t launch_backward(const void *q, const void *k, const void *v, const float *g,
                             const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
                             int Hv, int Dk, int Dv, int dtype, float scale, const float *s0,
@@ -244,22 +252,39 @@ size_t gdn_prefill_backward_workspace_size(int32_t num_seqs, int64_t total_token
   if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return 0;
   if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, GDN_DTYPE_FP32)) return 0;
   if (!dims_supported(head_dim_k, head_dim_v)) return 0;
-  return gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads, num_v_heads,
-                                       head_dim_k, head_dim_v);
+  return std::max(gdn::backward_chunked_workspace_bytes(num_seqs, total_tokens, num_qk_heads,
+                                                        num_v_heads, head_dim_k, head_dim_v),
+                  gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads, num_v_heads,
+                                                head_dim_k, head_dim_v));
 }
 
-int32_t gdn_prefill_backward(const void *q, const void *k, const void *v, const float *g,
-                             const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
-                             int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
-                             int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, float scale,
-                             const float *initial_state, const float *d_o,
-                             const float *d_final_state, float *dq, float *dk, float *dv,
-                             float *dg, float *dbeta, float *d_initial_state, void *workspace,
-                             size_t workspace_bytes, void *stream) {
+size_t gdn_prefill_backward_workspace_size_sequential(int32_t num_seqs, int64_t total_tokens,
+                                                      int32_t num_qk_heads, int32_t num_v_heads,
+                                                      int32_t head_dim_k, int32_t head_dim_v) {
+  if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return 0;
+  if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, GDN_DTYPE_FP32)) return 0;
+  if (!dims_supported(head_dim_k, head_dim_v)) return 0;
+  return gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads, num_v_heads, head_dim_k,
+                                       head_dim_v);
+}
+
+namespace {
+
+constexpr int32_t kNothingToDo = -1;  // valid call with no sequences: return GDN_OK, launch nothing
+
+// Host checks shared by both backward entry points: GDN_OK to proceed,
+// kNothingToDo, or an error code.
+int32_t check_backward(const void *q, const void *k, const void *v, const float *g,
+                       const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
+                       int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
+                       int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                       const float *initial_state, const float *d_o, const float *d_final_state,
+                       const float *dq, const float *dk, const float *dv, const float *dg,
+                       const float *dbeta, const float *d_initial_state, const void *workspace) {
   if (num_seqs < 0 || total_tokens < 0 || total_tokens > INT32_MAX) return GDN_ERR_INVALID_ARG;
   if (!dims_ok(num_qk_heads, num_v_heads, head_dim_k, head_dim_v, dtype)) return GDN_ERR_INVALID_ARG;
   if (!dims_supported(head_dim_k, head_dim_v)) return GDN_ERR_UNSUPPORTED;
-  if (num_seqs == 0) return total_tokens == 0 ? GDN_OK : GDN_ERR_INVALID_ARG;
+  if (num_seqs == 0) return total_tokens == 0 ? kNothingToDo : GDN_ERR_INVALID_ARG;
   if ((int64_t)num_seqs * num_v_heads > INT32_MAX) return GDN_ERR_UNSUPPORTED;
   if (!cu_seqlens || !aligned(cu_seqlens, 4)) return GDN_ERR_INVALID_ARG;
   if (total_tokens > 0) {
@@ -273,8 +298,54 @@ int32_t gdn_prefill_backward(const void *q, const void *k, const void *v, const 
   if ((initial_state && !aligned(initial_state, 16)) || (d_final_state && !aligned(d_final_state, 16)) ||
       (d_initial_state && !aligned(d_initial_state, 16)))
     return GDN_ERR_INVALID_ARG;
-  if (!workspace || !aligned(workspace, 256) ||
-      workspace_bytes < gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads,
+  if (!workspace || !aligned(workspace, 256)) return GDN_ERR_WORKSPACE;
+  return GDN_OK;
+}
+
+}  // namespace
+
+int32_t gdn_prefill_backward(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
+                             int64_t total_tokens, int32_t num_qk_heads, int32_t num_v_heads,
+                             int32_t head_dim_k, int32_t head_dim_v, int32_t dtype, float scale,
+                             const float *initial_state, const float *d_o,
+                             const float *d_final_state, float *dq, float *dk, float *dv,
+                             float *dg, float *dbeta, float *d_initial_state, void *workspace,
+                             size_t workspace_bytes, void *stream) {
+  const int32_t c = check_backward(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_qk_heads,
+                                   num_v_heads, head_dim_k, head_dim_v, dtype, initial_state, d_o,
+                                   d_final_state, dq, dk, dv, dg, dbeta, d_initial_state, workspace);
+  if (c != GDN_OK) return c == kNothingToDo ? GDN_OK : c;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (workspace_bytes >= gdn::backward_chunked_workspace_bytes(num_seqs, total_tokens, num_qk_heads,
+                                                              num_v_heads, head_dim_k, head_dim_v))
+    return cuda_status(gdn::launch_backward_chunked(
+        q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_qk_heads, num_v_heads, head_dim_k,
+        head_dim_v, dtype, scale, initial_state, d_o, d_final_state, dq, dk, dv, dg, dbeta,
+        d_initial_state, workspace, st));
+  if (workspace_bytes >= gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads,
+                                                       num_v_heads, head_dim_k, head_dim_v))
+    return cuda_status(gdn::launch_backward(
+        q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_qk_heads, num_v_heads, head_dim_k,
+        head_dim_v, dtype, scale, initial_state, d_o, d_final_state, dq, dk, dv, dg, dbeta,
+        d_initial_state, workspace, st));
+  return GDN_ERR_WORKSPACE;
+}
+
+int32_t gdn_prefill_backward_sequential(const void *q, const void *k, const void *v, const float *g,
+                                        const float *beta, const int32_t *cu_seqlens,
+                                        int32_t num_seqs, int64_t total_tokens,
+                                        int32_t num_qk_heads, int32_t num_v_heads,
+                                        int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                                        float scale, const float *initial_state, const float *d_o,
+                                        const float *d_final_state, float *dq, float *dk,
+                                        float *dv, float *dg, float *dbeta, float *d_initial_state,
+                                        void *workspace, size_t workspace_bytes, void *stream) {
+  const int32_t c = check_backward(q, k, v, g, beta, cu_seqlens, num_seqs, total_tokens, num_qk_heads,
+                                   num_v_heads, head_dim_k, head_dim_v, dtype, initial_state, d_o,
+                                   d_final_state, dq, dk, dv, dg, dbeta, d_initial_state, workspace);
+  if (c != GDN_OK) return c == kNothingToDo ? GDN_OK : c;
+  if (workspace_bytes < gdn::backward_workspace_bytes(num_seqs, total_tokens, num_qk_heads,
                                                       num_v_heads, head_dim_k, head_dim_v))
     return GDN_ERR_WORKSPACE;
   return cuda_status(gdn::launch_backward(

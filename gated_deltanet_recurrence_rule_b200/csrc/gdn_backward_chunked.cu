@@ -1,0 +1,875 @@
+// gdn_backward_chunked.cu -- backward pass of the gated delta rule in the
+// chunked (WY/UT) form: the gradients of a loss with respect to q, k, v, g,
+// beta and the initial state, fp32-accurate, with the dense products of every
+// chunk on the tensor cores.
+//
+// The forward rule is the one of "Inside Qwen3.8-27B: Hybrid DeltaNet
+// Architecture, 256k Context, and 24GB Local Serving", section "Gated DeltaNet
+// Mechanics", whose note says the block-parallel form serves training as well
+// as prefill.  For a chunk of C = 64 tokens with start state S0 (Dv x Dk),
+// local log-decay prefix sums G_t, gamma_t = e^{G_t}, kdec_t = e^{G_last -
+// G_t}, gamma_C = e^{G_last} and E_ts = e^{G_t - G_s} (s <= t):
+//   A = strict_lower(diag(beta) (E . K K^T)),   Tm = (I + A)^-1
+//   W = Tm diag(beta gamma) K,   U~ = Tm diag(beta) V,   U = U~ - W S0^T
+//   P = E . Q K^T (s <= t),      O = scale (diag(gamma) Q S0^T + P U)
+//   S1 = gamma_C S0 + U^T diag(kdec) K
+// Reverse mode, with dO' = scale dO and dS1 = dL/dS1 (the state after the
+// chunk), first the chain over the chunks, last to first:
+//   dU  = P^T dO' + diag(kdec) K dS1^T
+//   dS0 = gamma_C dS1 + dO'^T diag(gamma) Q - dU^T W
+// then, for every chunk independently:
+//   dQ  = diag(gamma) dO' S0 + (dP . E) K,        dP = lower(dO' U^T)
+//   dW  = -dU S0,   dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T
+//   X = Tm^T dW,    Y = Tm^T dU,                  dA = strict_lower(-Tm^T dT Tm^T)
+//   dK  = diag(kdec) U dS1 + (dP . E)^T Q + diag(beta gamma) X + (B + B^T) K,
+//         B = diag(beta) (dA . E)
+//   dV  = diag(beta) Y
+//   dbeta_t = gamma_t X_t.k_t + Y_t.v_t + sum_s dA_ts (E . K K^T)_ts
+//   dG_t from every e^{G} factor (gamma, kdec, gamma_C, E in P and A), and
+//   dg_s = sum_{t >= s} dG_t within the chunk.
+// dq and dk of a query/key head sum over the value heads that read it.
+//
+// Launches (one stream):
+//   plan         validates cu_seqlens, lists the non-empty sequences and
+//                their first chunk; d_initial_state of an empty sequence is
+//                d_final_state (or zero)
+//   prep         per (chunk, value head): P, E . K K^T, Tm, W, U~, G
+//   fwd_chain    per (sequence, value head, 32 rows of the state): the state
+//                at every chunk start (S0) and U, in chunk order
+//   rev_chain    per (sequence, value head, 32 rows): dS1 and dU, chunks last
+//                to first, and d_initial_state
+//   grads_state  per (chunk, value head): the products with S0 and dS1
+//   grads_local  per (chunk, value head): the 64 x 64 algebra, then dq, dk
+//                (per value head), dv, dg, dbeta
+//   group sums   dq, dk over the value heads of each query/key head
+// Rows of S and of dS evolve independently (the chains never mix rows), so
+// each chain CTA owns 32 of the Dv rows.  Every product runs on warp-level
+// m16n8k8 tf32 tensor-core MMAs with both operands split into hi = tf32(x)
+// and lo = tf32(x - hi) and three products (hi*hi + hi*lo + lo*hi), which
+// keeps about fp32 accuracy.  Per-row sums go through fixed-order partials,
+// so results do not depend on scheduling.
+#include <algorithm>
+
+#include "gdn_chunk_ops.cuh"
+#include "gdn_common.cuh"
+#include "gdn_twophase.cuh"
+
+namespace gdn {
+
+cudaError_t launch_plan(const int32_t *cu, int N, int T, int Hv, const void *s0, void *sfin,
+                        size_t state_bytes, tp::PlanHeader *ph, int32_t *ne_seq, int32_t *ne_cs,
+                        int32_t *status, cudaStream_t stream);
+cudaError_t launch_group_sum(const float *part, float *out, size_t rows, int width, int inner,
+                             cudaStream_t stream);
+
+namespace cbwd {
+
+constexpr int C = 64;         // chunk length
+constexpr int NT = 256;       // threads per CTA (8 warps)
+constexpr int SL = 32;        // state rows per chain CTA
+constexpr int LD64 = 68;      // fp32 row stride of 64 x 64 tiles in shared memory
+constexpr float kGmin = -30.f;  // g clamp: alpha >= e^-30, so prefix sums stay finite
+
+struct Params {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  const int32_t *cu;
+  int N, T, Hqk, Hv;
+  float scale;
+  const float *s0, *dO, *dSf;
+  float *dq, *dk;  // outputs, or per-value-head partials [T, Hv, Dk] when Hv > Hqk
+  float *dv, *dg, *dbeta, *ds0;
+  const tp::PlanHeader *ph;
+  const int32_t *ne_seq, *ne_cs;
+  // per unit u = chunk * Hv + value head
+  float *Tm, *P, *EKK;      // [u][64][64]
+  float *W, *dQp, *dKp, *dW;  // [u][64][Dk]
+  float *Ut, *U, *dU;       // [u][64][Dv]
+  float *S0, *dS1;          // [u][Dv][Dk]
+  double *G;                // [u][64] prefix sums of the clamped log-decays (fp64: differences
+                            // of large sums stay exact when gates are near zero)
+  float *sc;                // [u][3][64]: dgamma (from S0), dkdec, dgamma_C at [2][0]
+};
+
+// ---- tensor-core building block -------------------------------------------
+// acc[t] (a 16 x 8 fragment) += X[16][8 KS] * Y[8 KS][8 t .. 8 t + 7] for t <
+// NTL tiles in a row.  X(r, c) and Y(r, c) read single elements; each is split
+// once per k step.  Fragment element e of tile t sits at row gid + 8 (e >> 1),
+// column 8 t + 2 tig + (e & 1) (gid = lane / 4, tig = lane % 4).
+template <int KS, int NTL, class FX, class FY>
+__device__ __forceinline__ void mma3_rows(float (&acc)[NTL][4], FX X, FY Y, int lane) {
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll 2
+  for (int ks = 0; ks < KS; ++ks) {
+    const int k0 = 8 * ks + tig;
+    const float a[4] = {X(gid, k0), X(gid + 8, k0), X(gid, k0 + 4), X(gid + 8, k0 + 4)};
+    uint32_t ah[4], al[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      ah[e] = chunk::to_tf32(a[e]);
+      al[e] = chunk::to_tf32(a[e] - __uint_as_float(ah[e]));
+    }
+#pragma unroll
+    for (int t = 0; t < NTL; ++t) {
+      const float b0 = Y(k0, 8 * t + gid), b1 = Y(k0 + 4, 8 * t + gid);
+      const uint32_t bh[2] = {chunk::to_tf32(b0), chunk::to_tf32(b1)};
+      const uint32_t bl[2] = {chunk::to_tf32(b0 - __uint_as_float(bh[0])),
+                              chunk::to_tf32(b1 - __uint_as_float(bh[1]))};
+      chunk::mma_tf32_16x8x8(acc[t], al, bh);
+      chunk::mma_tf32_16x8x8(acc[t], ah, bl);
+      chunk::mma_tf32_16x8x8(acc[t], ah, bh);
+    }
+  }
+}
+
+template <int NTL>
+__device__ __forceinline__ void zero_acc(float (&acc)[NTL][4]) {
+#pragma unroll
+  for (int t = 0; t < NTL; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+}
+
+// Call f(row, col, value&) for every element of a lane's fragments; rows from
+// r0, columns from c0.
+template <int NTL, class F>
+__device__ __forceinline__ void for_frag(float (&acc)[NTL][4], int r0, int c0, int lane, F f) {
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int t = 0; t < NTL; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) f(r0 + gid + 8 * (e >> 1), c0 + 8 * t + 2 * tig + (e & 1), acc[t][e]);
+}
+
+// Sum of the two rows (gid, gid + 8) a lane holds over the warp's columns:
+// returned in every lane of the quad.
+template <int NTL, class F>
+__device__ __forceinline__ void quad_row_sums(float (&acc)[NTL][4], F weight, int r0, int c0,
+                                              int lane, float &s_lo, float &s_hi) {
+  const int gid = lane >> 2, tig = lane & 3;
+  float a = 0.f, b = 0.f;
+#pragma unroll
+  for (int t = 0; t < NTL; ++t)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int r = r0 + gid + 8 * (e >> 1), c = c0 + 8 * t + 2 * tig + (e & 1);
+      const float x = acc[t][e] * weight(r, c);
+      if (e < 2) a += x; else b += x;
+    }
+  a += __shfl_xor_sync(0xffffffffu, a, 1);
+  a += __shfl_xor_sync(0xffffffffu, a, 2);
+  b += __shfl_xor_sync(0xffffffffu, b, 1);
+  b += __shfl_xor_sync(0xffffffffu, b, 2);
+  s_lo = a;
+  s_hi = b;
+}
+
+// ---- tile loads -------------------------------------------------------------
+// dst[r][0..COLS) (row stride ld floats) = mul * src[r * stride + 0..COLS) for
+// r < valid, zeros for valid <= r < ROWS.  COLS % 4 == 0; src 8- or 16-byte
+// aligned per row.
+template <int ROWS, int COLS, typename TI>
+__device__ __forceinline__ void load_tile(float *dst, int ld, const TI *src, size_t stride,
+                                          int valid, float mul, int tid) {
+  constexpr int V4 = COLS / 4;
+  for (int x = tid; x < ROWS * V4; x += NT) {
+    const int r = x / V4, c = 4 * (x - r * V4);
+    float f[4] = {0.f, 0.f, 0.f, 0.f};
+    if (r < valid) {
+      load4(src + (size_t)r * stride + c, f);
+      f[0] *= mul; f[1] *= mul; f[2] *= mul; f[3] *= mul;
+    }
+    *reinterpret_cast<float4 *>(dst + r * ld + c) = make_float4(f[0], f[1], f[2], f[3]);
+  }
+}
+// dst[r * stride + c] = src[r][c] (row stride ld) for r < ROWS, c < COLS.
+template <int ROWS, int COLS>
+__device__ __forceinline__ void store_tile(float *dst, size_t stride, const float *src, int ld,
+                                           int tid) {
+  constexpr int V4 = COLS / 4;
+  for (int x = tid; x < ROWS * V4; x += NT) {
+    const int r = x / V4, c = 4 * (x - r * V4);
+    *reinterpret_cast<float4 *>(dst + (size_t)r * stride + c) =
+        *reinterpret_cast<const float4 *>(src + r * ld + c);
+  }
+}
+
+struct ChunkPos {
+  int n, start, len;
+};
+// Sequence, first token and length of global chunk c; false past the last chunk.
+__device__ __forceinline__ bool chunk_pos(const Params &p, int c, ChunkPos &cp) {
+  if (c >= p.ph->total_chunks) return false;
+  const int kk = tp::owner_of_chunk(p.ne_cs, p.ph->n_nonempty, c);
+  const int n = p.ne_seq[kk];
+  cp.n = n;
+  cp.start = p.cu[n] + C * (c - p.ne_cs[kk]);
+  cp.len = min(C, p.cu[n + 1] - cp.start);
+  return true;
+}
+
+// ---- prep: P, E . K K^T, Tm, W, U~ and G of one (chunk, value head) ----------
+template <int DK, int DV>
+struct PrepSmem {
+  static constexpr int LQ = DK + 4, LK = DK + 4, LV = DV + 8;
+  static constexpr int OQ = 0, OK = OQ + C * LQ, OV = OK + C * LK, OA = OV + C * LV,
+                       OT = OA + C * LD64, OY = OT + C * LD64, OG = OY + 3 * 16 * 17,
+                       OB = OG + 2 * C, OBG = OB + C, FLOATS = OBG + C;
+  static constexpr size_t BYTES = FLOATS * sizeof(float);
+};
+
+template <typename TI, int DK, int DV>
+__global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
+  using L = PrepSmem<DK, DV>;
+  extern __shared__ __align__(16) float sm[];
+  float *Qs = sm + L::OQ, *Ks = sm + L::OK, *Vs = sm + L::OV, *As = sm + L::OA, *Ts = sm + L::OT;
+  float *Ysc = sm + L::OY, *sB = sm + L::OB, *sBG = sm + L::OBG;
+  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  ChunkPos cp;
+  if (!chunk_pos(p, blockIdx.x, cp)) return;
+  const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk);
+  const size_t u = (size_t)blockIdx.x * p.Hv + h;
+  const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k),
+           *v = static_cast<const TI *>(p.v);
+  load_tile<C, DK>(Qs, L::LQ, q + ((size_t)cp.start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, cp.len, 1.f, tid);
+  load_tile<C, DK>(Ks, L::LK, k + ((size_t)cp.start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, cp.len, 1.f, tid);
+  load_tile<C, DV>(Vs, L::LV, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, cp.len, 1.f, tid);
+  for (int x = tid; x < C * LD64; x += NT) Ts[x] = 0.f;
+  if (w == 0) {  // prefix sums of the clamped log-decays (2 tokens per lane)
+    const int t0 = 2 * lane;
+    float g0 = 0.f, g1 = 0.f, b0 = 0.f, b1 = 0.f;
+    if (t0 < cp.len) { g0 = fmaxf(p.g[(size_t)(cp.start + t0) * p.Hv + h], kGmin); b0 = p.beta[(size_t)(cp.start + t0) * p.Hv + h]; }
+    if (t0 + 1 < cp.len) { g1 = fmaxf(p.g[(size_t)(cp.start + t0 + 1) * p.Hv + h], kGmin); b1 = p.beta[(size_t)(cp.start + t0 + 1) * p.Hv + h]; }
+    double s = (double)g0 + (double)g1;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const double x = __shfl_up_sync(0xffffffffu, s, off);
+      if (lane >= off) s += x;
+    }
+    const double G1 = s, G0 = s - g1;
+    sG[t0] = G0; sG[t0 + 1] = G1;
+    sB[t0] = b0; sB[t0 + 1] = b1;
+    sBG[t0] = b0 * expf((float)G0); sBG[t0 + 1] = b1 * expf((float)G1);
+    p.G[u * C + t0] = G0;
+    p.G[u * C + t0 + 1] = G1;
+  }
+  __syncthreads();
+  {  // QK^T and KK^T: warp rows 16 (w & 3), columns 32 (w >> 2)
+    const int r0 = 16 * (w & 3), c0 = 32 * (w >> 2);
+    float aq[4][4], ak[4][4];
+    zero_acc(aq);
+    zero_acc(ak);
+    mma3_rows<DK / 8>(aq, [&](int r, int c) { return Qs[(r0 + r) * L::LQ + c]; },
+                      [&](int r, int c) { return Ks[(c0 + c) * L::LK + r]; }, lane);
+    mma3_rows<DK / 8>(ak, [&](int r, int c) { return Ks[(r0 + r) * L::LK + c]; },
+                      [&](int r, int c) { return Ks[(c0 + c) * L::LK + r]; }, lane);
+    float *P = p.P + u * C * C, *EKK = p.EKK + u * C * C;
+    const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const int i = r0 + gid + 8 * hr, j = c0 + 8 * t + 2 * tig;
+        float pv[2], ev[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float E = (i >= j + e) ? expf((float)(sG[i] - sG[j + e])) : 0.f;
+          pv[e] = (i >= j + e) ? E * aq[t][2 * hr + e] : 0.f;
+          ev[e] = (i > j + e) ? E * ak[t][2 * hr + e] : 0.f;
+          As[i * LD64 + j + e] = sB[i] * ev[e];
+        }
+        *reinterpret_cast<float2 *>(P + i * C + j) = make_float2(pv[0], pv[1]);
+        *reinterpret_cast<float2 *>(EKK + i * C + j) = make_float2(ev[0], ev[1]);
+      }
+  }
+  __syncthreads();
+  chunk::ut_solve<NT, 1>(As, Ts, Ysc, tid);  // ends with a barrier of all NT threads
+  store_tile<C, C>(p.Tm + u * C * C, C, Ts, LD64, tid);
+  {  // W = Tm diag(beta gamma) K and U~ = Tm diag(beta) V: rows 16 (w & 3), column halves
+    const int r0 = 16 * (w & 3);
+    {
+      const int c0 = (w >> 2) * (DK / 2);
+      float acc[DK / 16][4];
+      zero_acc(acc);
+      mma3_rows<C / 8>(acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c]; },
+                       [&](int r, int c) { return sBG[r] * Ks[r * L::LK + c0 + c]; }, lane);
+      float *W = p.W + u * C * DK;
+      for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { W[i * DK + c] = x; });
+    }
+    {
+      const int c0 = (w >> 2) * (DV / 2);
+      float acc[DV / 16][4];
+      zero_acc(acc);
+      mma3_rows<C / 8>(acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c]; },
+                       [&](int r, int c) { return sB[r] * Vs[r * L::LV + c0 + c]; }, lane);
+      float *Ut = p.Ut + u * C * DV;
+      for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { Ut[i * DV + c] = x; });
+    }
+  }
+}
+
+// ---- forward chain: S0 and U of every chunk, per 32 rows of the state ---------
+template <int DK, int DV>
+struct FwdSmem {
+  static constexpr int LS = DK + 4, LW = DK + 4, LK = DK + 8, LU = SL + 8;
+  static constexpr int OS = 0, OW = OS + SL * LS, OK = OW + C * LW, OU = OK + C * LK,
+                       OG = OU + C * LU, OKD = OG + 2 * C, FLOATS = OKD + C;
+  static constexpr size_t BYTES = FLOATS * sizeof(float);
+};
+
+template <typename TI, int DK, int DV>
+__global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
+  using L = FwdSmem<DK, DV>;
+  extern __shared__ __align__(16) float sm[];
+  float *S = sm + L::OS, *Ws = sm + L::OW, *Ks = sm + L::OK, *Us = sm + L::OU, *sKd = sm + L::OKD;
+  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int kk = blockIdx.x;
+  if (kk >= p.ph->n_nonempty) return;
+  const int n = p.ne_seq[kk], c0 = p.ne_cs[kk], nch = p.ne_cs[kk + 1] - c0;
+  const int cs = p.cu[n], Lseq = p.cu[n + 1] - cs;
+  const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk), v0 = SL * blockIdx.z;
+  const TI *k = static_cast<const TI *>(p.k);
+  const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;  // first state row of this slice
+  if (p.s0) load_tile<SL, DK>(S, L::LS, p.s0 + srow * DK, DK, SL, 1.f, tid);
+  else for (int x = tid; x < SL * L::LS; x += NT) S[x] = 0.f;
+  for (int j = 0; j < nch; ++j) {
+    const size_t u = (size_t)(c0 + j) * p.Hv + h;
+    const int start = cs + C * j, len = min(C, Lseq - C * j);
+    load_tile<C, DK>(Ws, L::LW, p.W + u * C * DK, DK, C, 1.f, tid);
+    load_tile<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, 1.f, tid);
+    load_tile<C, SL>(Us, L::LU, p.Ut + u * C * DV + v0, DV, C, 1.f, tid);
+    if (tid < C) sG[tid] = p.G[u * C + tid];
+    store_tile<SL, DK>(p.S0 + (u * DV + v0) * DK, DK, S, L::LS, tid);
+    __syncthreads();
+    if (tid < C) sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
+    {  // U = U~ - W S^T: rows 16 (w & 3), state rows 16 (w >> 2)
+      const int r0 = 16 * (w & 3), vb = 16 * (w >> 2);
+      float acc[2][4];
+      zero_acc(acc);
+      mma3_rows<DK / 8>(acc, [&](int r, int c) { return Ws[(r0 + r) * L::LW + c]; },
+                        [&](int r, int c) { return S[(vb + c) * L::LS + r]; }, lane);
+      float *Ug = p.U + u * C * DV + v0;
+      for_frag(acc, r0, vb, lane, [&](int i, int c, float &x) {
+        const float uu = Us[i * L::LU + c] - x;
+        Us[i * L::LU + c] = uu;
+        Ug[i * DV + c] = uu;
+      });
+    }
+    __syncthreads();
+    if (j + 1 < nch) {  // S <- gamma_C S + U^T diag(kdec) K: state rows 16 (w & 1), columns DK / 4 (w >> 1)
+      const float gC = expf((float)sG[len - 1]);
+      const int r0 = 16 * (w & 1), kb = (w >> 1) * (DK / 4);
+      float acc[DK / 32][4];
+      for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * S[r * L::LS + c]; });
+      mma3_rows<C / 8>(acc, [&](int r, int c) { return Us[c * L::LU + r0 + r] * sKd[c]; },
+                       [&](int r, int c) { return Ks[r * L::LK + kb + c]; }, lane);
+      for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { S[r * L::LS + c] = x; });
+      __syncthreads();
+    }
+  }
+}
+
+// ---- reverse chain: dS1 and dU of every chunk, last to first ------------------
+template <int DK, int DV>
+struct RevSmem {
+  static constexpr int LS = DK + 4, LK = DK + 4, LQ = DK + 8, LW = DK + 8, LO = SL + 8;
+  static constexpr int OS = 0, OP = OS + SL * LS, OO = OP + C * LD64, OK = OO + C * LO,
+                       OQ = OK + C * LK, OW = OQ + C * LQ, OU = OW + C * LW, OG = OU + C * LO,
+                       OGM = OG + 2 * C, OKD = OGM + C, FLOATS = OKD + C;
+  static constexpr size_t BYTES = FLOATS * sizeof(float);
+};
+
+template <typename TI, int DK, int DV>
+__global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
+  using L = RevSmem<DK, DV>;
+  extern __shared__ __align__(16) float sm[];
+  float *dS = sm + L::OS, *Ps = sm + L::OP, *dOs = sm + L::OO, *Ks = sm + L::OK, *Qs = sm + L::OQ,
+        *Ws = sm + L::OW, *dUs = sm + L::OU, *sGm = sm + L::OGM, *sKd = sm + L::OKD;
+  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int kk = blockIdx.x;
+  if (kk >= p.ph->n_nonempty) return;
+  const int n = p.ne_seq[kk], c0 = p.ne_cs[kk], nch = p.ne_cs[kk + 1] - c0;
+  const int cs = p.cu[n], Lseq = p.cu[n + 1] - cs;
+  const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk), v0 = SL * blockIdx.z;
+  const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
+  const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;
+  if (p.dSf) load_tile<SL, DK>(dS, L::LS, p.dSf + srow * DK, DK, SL, 1.f, tid);
+  else for (int x = tid; x < SL * L::LS; x += NT) dS[x] = 0.f;
+  for (int j = nch - 1; j >= 0; --j) {
+    const size_t u = (size_t)(c0 + j) * p.Hv + h;
+    const int start = cs + C * j, len = min(C, Lseq - C * j);
+    load_tile<C, C>(Ps, LD64, p.P + u * C * C, C, C, 1.f, tid);
+    load_tile<C, SL>(dOs, L::LO, p.dO + ((size_t)start * p.Hv + h) * DV + v0, (size_t)p.Hv * DV, len,
+                     p.scale, tid);
+    load_tile<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, 1.f, tid);
+    load_tile<C, DK>(Qs, L::LQ, q + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, 1.f, tid);
+    load_tile<C, DK>(Ws, L::LW, p.W + u * C * DK, DK, C, 1.f, tid);
+    if (tid < C) sG[tid] = p.G[u * C + tid];
+    store_tile<SL, DK>(p.dS1 + (u * DV + v0) * DK, DK, dS, L::LS, tid);
+    __syncthreads();
+    if (tid < C) {
+      sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
+      sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
+    }
+    __syncthreads();
+    {  // dU = P^T dO' + diag(kdec) K dS^T: rows 16 (w & 3), state rows 16 (w >> 2)
+      const int r0 = 16 * (w & 3), vb = 16 * (w >> 2);
+      float a1[2][4], a2[2][4];
+      zero_acc(a1);
+      zero_acc(a2);
+      mma3_rows<C / 8>(a1, [&](int r, int c) { return Ps[c * LD64 + r0 + r]; },
+                       [&](int r, int c) { return dOs[r * L::LO + vb + c]; }, lane);
+      mma3_rows<DK / 8>(a2, [&](int r, int c) { return Ks[(r0 + r) * L::LK + c]; },
+                        [&](int r, int c) { return dS[(vb + c) * L::LS + r]; }, lane);
+      float *dUg = p.dU + u * C * DV + v0;
+      const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = r0 + gid + 8 * (e >> 1), c = vb + 8 * t + 2 * tig + (e & 1);
+          const float x = a1[t][e] + sKd[i] * a2[t][e];
+          dUs[i * L::LO + c] = x;
+          dUg[i * DV + c] = x;
+        }
+    }
+    __syncthreads();
+    {  // dS <- gamma_C dS + dO'^T diag(gamma) Q - dU^T W: state rows 16 (w & 1), columns DK / 4 (w >> 1)
+      const float gC = expf((float)sG[len - 1]);
+      const int r0 = 16 * (w & 1), kb = (w >> 1) * (DK / 4);
+      float acc[DK / 32][4];
+      for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * dS[r * L::LS + c]; });
+      mma3_rows<C / 8>(acc, [&](int r, int c) { return dOs[c * L::LO + r0 + r] * sGm[c]; },
+                       [&](int r, int c) { return Qs[r * L::LQ + kb + c]; }, lane);
+      mma3_rows<C / 8>(acc, [&](int r, int c) { return -dUs[c * L::LO + r0 + r]; },
+                       [&](int r, int c) { return Ws[r * L::LW + kb + c]; }, lane);
+      for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { dS[r * L::LS + c] = x; });
+    }
+    __syncthreads();
+  }
+  if (p.ds0) store_tile<SL, DK>(p.ds0 + srow * DK, DK, dS, L::LS, tid);
+}
+
+// ---- products with S0 and dS1 of one (chunk, value head) ----------------------
+template <int DK, int DV>
+struct StateGradSmem {
+  static constexpr int LS = DK + 8, LM = DV + 4;
+  static constexpr int OS0 = 0, OS1 = OS0 + DV * LS, OM = OS1 + DV * LS, OG = OM + C * LM,
+                       OR = OG + 2 * C, FLOATS = OR + 4 * C + 8;
+  static constexpr size_t BYTES = FLOATS * sizeof(float);
+};
+
+template <typename TI, int DK, int DV>
+__global__ void __launch_bounds__(NT) grads_state_kernel(const Params p) {
+  using L = StateGradSmem<DK, DV>;
+  extern __shared__ __align__(16) float sm[];
+  float *S0s = sm + L::OS0, *S1s = sm + L::OS1, *Ms = sm + L::OM, *red = sm + L::OR;
+  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  ChunkPos cp;
+  if (!chunk_pos(p, blockIdx.x, cp)) return;
+  const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk);
+  const size_t u = (size_t)blockIdx.x * p.Hv + h;
+  const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
+  const TI *qc = q + ((size_t)cp.start * p.Hqk + hk) * DK, *kc = k + ((size_t)cp.start * p.Hqk + hk) * DK;
+  const size_t qstride = (size_t)p.Hqk * DK;
+  load_tile<DV, DK>(S0s, L::LS, p.S0 + u * DV * DK, DK, DV, 1.f, tid);
+  load_tile<DV, DK>(S1s, L::LS, p.dS1 + u * DV * DK, DK, DV, 1.f, tid);
+  load_tile<C, DV>(Ms, L::LM, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, cp.len,
+                   p.scale, tid);
+  if (tid < C) sG[tid] = p.G[u * C + tid];
+  __syncthreads();
+  const int len = cp.len;
+  {  // <dS1, S0>: fixed-order partials per thread, then per warp, then over warps
+    float s = 0.f;
+    for (int x = tid; x < DV * DK; x += NT) {
+      const int r = x / DK, c = x - r * DK;
+      s = fmaf(S0s[r * L::LS + c], S1s[r * L::LS + c], s);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+    if (lane == 0) red[4 * C + w] = s;
+  }
+  const int r0 = 16 * (w & 3), cb = (w >> 2) * (DK / 2), half = w >> 2;
+  const int gid = lane >> 2, tig = lane & 3;
+  float acc[DK / 16][4];
+  // dO' S0: dQ part diag(gamma) dO' S0 and dgamma_t = q_t . (dO' S0)_t
+  zero_acc(acc);
+  mma3_rows<DV / 8>(acc, [&](int r, int c) { return Ms[(r0 + r) * L::LM + c]; },
+                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
+  {
+    float slo, shi;
+    quad_row_sums(acc, [&](int i, int c) { return i < len ? to_f32(qc[(size_t)i * qstride + c]) : 0.f; },
+                  r0, cb, lane, slo, shi);
+    if (tig == 0) { red[half * C + r0 + gid] = slo; red[half * C + r0 + gid + 8] = shi; }
+    float *dQp = p.dQp + u * C * DK;
+    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) {
+      dQp[i * DK + c] = i < len ? expf((float)sG[i]) * x : 0.f;
+    });
+  }
+  __syncthreads();
+  load_tile<C, DV>(Ms, L::LM, p.dU + u * C * DV, DV, C, 1.f, tid);
+  __syncthreads();
+  zero_acc(acc);  // dW = -dU S0
+  mma3_rows<DV / 8>(acc, [&](int r, int c) { return Ms[(r0 + r) * L::LM + c]; },
+                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
+  {
+    float *dW = p.dW + u * C * DK;
+    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) { dW[i * DK + c] = -x; });
+  }
+  __syncthreads();
+  load_tile<C, DV>(Ms, L::LM, p.U + u * C * DV, DV, C, 1.f, tid);
+  __syncthreads();
+  zero_acc(acc);  // U dS1: dK part diag(kdec) U dS1 and dkdec_t = k_t . (U dS1)_t
+  mma3_rows<DV / 8>(acc, [&](int r, int c) { return Ms[(r0 + r) * L::LM + c]; },
+                    [&](int r, int c) { return S1s[r * L::LS + cb + c]; }, lane);
+  {
+    float slo, shi;
+    quad_row_sums(acc, [&](int i, int c) { return i < len ? to_f32(kc[(size_t)i * qstride + c]) : 0.f; },
+                  r0, cb, lane, slo, shi);
+    if (tig == 0) { red[(2 + half) * C + r0 + gid] = slo; red[(2 + half) * C + r0 + gid + 8] = shi; }
+    float *dKp = p.dKp + u * C * DK;
+    const double Gl = sG[len - 1];
+    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) {
+      dKp[i * DK + c] = i < len ? expf((float)(Gl - sG[i])) * x : 0.f;
+    });
+  }
+  __syncthreads();
+  float *sc = p.sc + u * 3 * C;
+  if (tid < C) {
+    sc[tid] = red[tid] + red[C + tid];
+    sc[C + tid] = red[2 * C + tid] + red[3 * C + tid];
+  }
+  if (tid == 0) {
+    float s = 0.f;
+    for (int x = 0; x < NT / 32; ++x) s += red[4 * C + x];
+    sc[2 * C] = s;
+  }
+}
+
+// ---- the 64 x 64 algebra of one (chunk, value head), and its outputs -----------
+template <int DK, int DV>
+struct LocalSmem {
+  static constexpr int LA = (DK > DV ? DK : DV) + 4;  // dO', then dW
+  static constexpr int LB = DV + 4;                   // U, then dU
+  static constexpr int LC = DK + 4;                   // K
+  static constexpr int LD = (DK > DV ? DK : DV) + 4;  // V, then Q
+  static constexpr int OA = 0, OB = OA + C * LA, OC = OB + C * LB, OD = OC + C * LC,
+                       O1 = OD + C * LD, O2 = O1 + C * LD64, O3 = O2 + C * LD64, O4 = O3 + C * LD64,
+                       O5 = O4 + C * LD64, OV = O5 + C * LD64, NVEC = 13, FLOATS = OV + NVEC * C;
+  static constexpr size_t BYTES = FLOATS * sizeof(float);
+};
+
+template <typename TI, int DK, int DV>
+__global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
+  using L = LocalSmem<DK, DV>;
+  extern __shared__ __align__(16) float sm[];
+  float *RA = sm + L::OA, *RB = sm + L::OB, *RC = sm + L::OC, *RD = sm + L::OD;
+  float *S1 = sm + L::O1, *S2 = sm + L::O2, *S3 = sm + L::O3, *S4 = sm + L::O4, *S5 = sm + L::O5;
+  float *vec = sm + L::OV;
+  // per-row vectors: G (fp64), beta, gamma, kdec, xk (2 halves), yv (2 halves), rP, cP, rM, cM
+  double *sG = reinterpret_cast<double *>(vec);
+  float *sB = vec + 2 * C, *sGm = vec + 3 * C, *sKd = vec + 4 * C, *sXK = vec + 5 * C,
+        *sYV = vec + 7 * C, *sRP = vec + 9 * C, *sCP = vec + 10 * C, *sRM = vec + 11 * C,
+        *sCM = vec + 12 * C;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int gid = lane >> 2, tig = lane & 3;
+  ChunkPos cp;
+  if (!chunk_pos(p, blockIdx.x, cp)) return;
+  const int h = blockIdx.y, Gq = p.Hv / p.Hqk, hk = h / Gq;
+  const size_t u = (size_t)blockIdx.x * p.Hv + h;
+  const int len = cp.len;
+  const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k),
+           *v = static_cast<const TI *>(p.v);
+  const size_t qoff = ((size_t)cp.start * p.Hqk + hk) * DK, qstride = (size_t)p.Hqk * DK;
+  // step 1: dP = lower(dO' U^T); S2 = dP . E, S1 = dP . P
+  load_tile<C, DV>(RA, L::LA, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len,
+                   p.scale, tid);
+  load_tile<C, DV>(RB, L::LB, p.U + u * C * DV, DV, C, 1.f, tid);
+  load_tile<C, C>(S1, LD64, p.P + u * C * C, C, C, 1.f, tid);
+  if (tid < C) {
+    sG[tid] = p.G[u * C + tid];
+    sB[tid] = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
+  }
+  __syncthreads();
+  if (tid < C) {
+    sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
+    sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
+  }
+  const int r0 = 16 * (w & 3), half = w >> 2, c64 = 32 * half;
+  {
+    float acc[4][4];
+    zero_acc(acc);
+    mma3_rows<DV / 8>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
+                      [&](int r, int c) { return RB[(c64 + c) * L::LB + r]; }, lane);
+    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) {
+      const float dp = i >= j ? x : 0.f;
+      S2[i * LD64 + j] = i >= j ? dp * expf((float)(sG[i] - sG[j])) : 0.f;
+      S1[i * LD64 + j] = dp * S1[i * LD64 + j];
+    });
+  }
+  __syncthreads();
+  // step 2: dT, X = Tm^T dW (dK part, x.k), Y = Tm^T dU (dv, y.v)
+  load_tile<C, DK>(RA, L::LA, p.dW + u * C * DK, DK, C, 1.f, tid);
+  load_tile<C, DV>(RB, L::LB, p.dU + u * C * DV, DV, C, 1.f, tid);
+  load_tile<C, DK>(RC, L::LC, k + qoff, qstride, len, 1.f, tid);
+  load_tile<C, DV>(RD, L::LD, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, 1.f, tid);
+  load_tile<C, C>(S3, LD64, p.Tm + u * C * C, C, C, 1.f, tid);
+  __syncthreads();
+  {  // dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T
+    float acc[4][4];
+    zero_acc(acc);
+    mma3_rows<DK / 8>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
+                      [&](int r, int c) { return sB[c64 + c] * sGm[c64 + c] * RC[(c64 + c) * L::LC + r]; }, lane);
+    mma3_rows<DV / 8>(acc, [&](int r, int c) { return RB[(r0 + r) * L::LB + c]; },
+                      [&](int r, int c) { return sB[c64 + c] * RD[(c64 + c) * L::LD + r]; }, lane);
+    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = x; });
+  }
+  const int cbk = half * (DK / 2), cbv = half * (DV / 2);
+  float dK[DK / 16][4];
+  {  // X = Tm^T dW
+    zero_acc(dK);
+    mma3_rows<C / 8>(dK, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+                     [&](int r, int c) { return RA[r * L::LA + cbk + c]; }, lane);
+    float slo, shi;
+    quad_row_sums(dK, [&](int i, int c) { return RC[i * L::LC + c]; }, r0, cbk, lane, slo, shi);
+    if (tig == 0) { sXK[half * C + r0 + gid] = slo; sXK[half * C + r0 + gid + 8] = shi; }
+    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x *= sB[i] * sGm[i]; });
+  }
+  {  // Y = Tm^T dU: dv = diag(beta) Y
+    float acc[DV / 16][4];
+    zero_acc(acc);
+    mma3_rows<C / 8>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+                     [&](int r, int c) { return RB[r * L::LB + cbv + c]; }, lane);
+    float slo, shi;
+    quad_row_sums(acc, [&](int i, int c) { return RD[i * L::LD + c]; }, r0, cbv, lane, slo, shi);
+    if (tig == 0) { sYV[half * C + r0 + gid] = slo; sYV[half * C + r0 + gid + 8] = shi; }
+    float *dv = p.dv + ((size_t)cp.start * p.Hv + h) * DV;
+    for_frag(acc, r0, cbv, lane, [&](int i, int c, float &x) {
+      if (i < len) dv[(size_t)i * p.Hv * DV + c] = sB[i] * x;
+    });
+  }
+  __syncthreads();
+  {  // Z = dT Tm^T -> S5
+    float acc[4][4];
+    zero_acc(acc);
+    mma3_rows<C / 8>(acc, [&](int r, int c) { return S4[(r0 + r) * LD64 + c]; },
+                     [&](int r, int c) { return S3[(c64 + c) * LD64 + r]; }, lane);
+    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S5[i * LD64 + j] = x; });
+  }
+  __syncthreads();
+  {  // dA = strict_lower(-Tm^T Z) -> S4
+    float acc[4][4];
+    zero_acc(acc);
+    mma3_rows<C / 8>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+                     [&](int r, int c) { return S5[r * LD64 + c64 + c]; }, lane);
+    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = i > j ? -x : 0.f; });
+  }
+  __syncthreads();
+  load_tile<C, C>(S5, LD64, p.EKK + u * C * C, C, C, 1.f, tid);
+  load_tile<C, DK>(RD, L::LD, q + qoff, qstride, len, 1.f, tid);
+  __syncthreads();
+  // S4 <- B = diag(beta) (dA . E); S5 <- dA . (E . K K^T)
+  for (int x = tid; x < C * C; x += NT) {
+    const int i = x >> 6, j = x & 63;
+    const float da = S4[i * LD64 + j];
+    S4[i * LD64 + j] = i > j ? sB[i] * da * expf((float)(sG[i] - sG[j])) : 0.f;
+    S5[i * LD64 + j] = da * S5[i * LD64 + j];
+  }
+  __syncthreads();
+  if (tid < C) {  // row sums
+    float a = 0.f, b = 0.f;
+    for (int j = 0; j < C; ++j) { a += S1[tid * LD64 + j]; b += S5[tid * LD64 + j]; }
+    sRP[tid] = a;
+    sRM[tid] = b;
+  } else if (tid < 2 * C) {  // column sums
+    const int j = tid - C;
+    float a = 0.f, b = 0.f;
+    for (int i = 0; i < C; ++i) { a += S1[i * LD64 + j]; b += sB[i] * S5[i * LD64 + j]; }
+    sCP[j] = a;
+    sCM[j] = b;
+  }
+  {  // dq (this value head's part) = diag(gamma) dO' S0 + (dP . E) K
+    float acc[DK / 16][4];
+    const float *dQp = p.dQp + u * C * DK;
+    for_frag(acc, r0, cbk, lane, [&](int i, int c, float &x) { x = dQp[i * DK + c]; });
+    mma3_rows<C / 8>(acc, [&](int r, int c) { return S2[(r0 + r) * LD64 + c]; },
+                     [&](int r, int c) { return RC[r * L::LC + cbk + c]; }, lane);
+    const bool direct = Gq == 1;
+    float *dst = direct ? p.dq + qoff : p.dq + ((size_t)cp.start * p.Hv + h) * DK;
+    const size_t rs = direct ? qstride : (size_t)p.Hv * DK;
+    for_frag(acc, r0, cbk, lane, [&](int i, int c, float &x) {
+      if (i < len) dst[(size_t)i * rs + c] = x;
+    });
+  }
+  {  // dk = diag(kdec) U dS1 + diag(beta gamma) X + (dP . E)^T Q + (B + B^T) K
+    const float *dKp = p.dKp + u * C * DK;
+    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x += dKp[i * DK + c]; });
+    mma3_rows<C / 8>(dK, [&](int r, int c) { return S2[c * LD64 + r0 + r]; },
+                     [&](int r, int c) { return RD[r * L::LD + cbk + c]; }, lane);
+    mma3_rows<C / 8>(dK, [&](int r, int c) { return S4[(r0 + r) * LD64 + c] + S4[c * LD64 + r0 + r]; },
+                     [&](int r, int c) { return RC[r * L::LC + cbk + c]; }, lane);
+    const bool direct = Gq == 1;
+    float *dst = direct ? p.dk + qoff : p.dk + ((size_t)cp.start * p.Hv + h) * DK;
+    const size_t rs = direct ? qstride : (size_t)p.Hv * DK;
+    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) {
+      if (i < len) dst[(size_t)i * rs + c] = x;
+    });
+  }
+  __syncthreads();
+  if (w == 0) {  // dG, then dg (suffix sums) and dbeta; two tokens per lane
+    const float *sc = p.sc + u * 3 * C;
+    const float dgC = sc[2 * C];
+    float dG[2], db[2], kk2 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int i = 2 * lane + e;
+      const float xk = sXK[i] + sXK[C + i], yv = sYV[i] + sYV[C + i];
+      const float dgam = sc[i] + sB[i] * xk, dkd = sc[C + i];
+      db[e] = sGm[i] * xk + yv + sRM[i];
+      dG[e] = (sRP[i] - sCP[i]) + (sB[i] * sRM[i] - sCM[i]) + dgam * sGm[i] - dkd * sKd[i];
+      kk2 += dkd * sKd[i];
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) kk2 += __shfl_xor_sync(0xffffffffu, kk2, off);
+    const float gC = expf((float)sG[len - 1]);
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      if (2 * lane + e == len - 1) dG[e] += kk2 + dgC * gC;
+    // suffix sums over the chunk's tokens (rows >= len hold zeros)
+    float s = dG[0] + dG[1];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float x = __shfl_down_sync(0xffffffffu, s, off);
+      if (lane + off < 32) s += x;
+    }
+    const float suf1 = s - dG[0], suf0 = s;  // suffix from token 2 lane + 1, from 2 lane
+    const float sf[2] = {suf0, suf1};
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int i = 2 * lane + e;
+      if (i < len) {
+        p.dg[(size_t)(cp.start + i) * p.Hv + h] = sf[e];
+        p.dbeta[(size_t)(cp.start + i) * p.Hv + h] = db[e];
+      }
+    }
+  }
+}
+
+}  // namespace cbwd
+
+// Chunk-form backward workspace: header and plan, then the per-unit arrays,
+// then the per-value-head dq, dk partials when Hv > Hqk.
+struct CbwdLayout {
+  size_t plan, Tm, P, EKK, W, dQp, dKp, dW, Ut, U, dU, S0, dS1, G, sc, dqh, dkh, total;
+};
+
+static CbwdLayout cbwd_layout(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const size_t units = (size_t)tp::chunk_bound(N, T) * Hv, f = sizeof(float), C = cbwd::C;
+  CbwdLayout L;
+  size_t o = kWorkspaceHeaderBytes;
+  L.plan = o;  o += up(sizeof(int32_t) * (2 * (size_t)N + 1));
+  L.Tm = o;    o += up(units * C * C * f);
+  L.P = o;     o += up(units * C * C * f);
+  L.EKK = o;   o += up(units * C * C * f);
+  L.W = o;     o += up(units * C * Dk * f);
+  L.dQp = o;   o += up(units * C * Dk * f);
+  L.dKp = o;   o += up(units * C * Dk * f);
+  L.dW = o;    o += up(units * C * Dk * f);
+  L.Ut = o;    o += up(units * C * Dv * f);
+  L.U = o;     o += up(units * C * Dv * f);
+  L.dU = o;    o += up(units * C * Dv * f);
+  L.S0 = o;    o += up(units * (size_t)Dv * Dk * f);
+  L.dS1 = o;   o += up(units * (size_t)Dv * Dk * f);
+  L.G = o;     o += up(units * C * sizeof(double));
+  L.sc = o;    o += up(units * 3 * C * f);
+  L.dqh = L.dkh = 0;
+  if (Hv != Hqk) {
+    L.dqh = o; o += up((size_t)T * Hv * Dk * f);
+    L.dkh = o; o += up((size_t)T * Hv * Dk * f);
+  }
+  L.total = o;
+  return L;
+}
+
+size_t backward_chunked_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv) {
+  return cbwd_layout(N, T, Hqk, Hv, Dk, Dv).total;
+}
+
+namespace {
+
+template <typename K>
+cudaError_t launch_k(K kern, dim3 grid, size_t smem, const cbwd::Params &prm, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
+  kern<<<grid, cbwd::NT, smem, stream>>>(prm);
+  return cudaGetLastError();
+}
+
+template <typename TI, int DK, int DV>
+cudaError_t run_chunked(const cbwd::Params &prm, int64_t chunks, cudaStream_t stream) {
+  using namespace cbwd;
+  const dim3 per_chunk((unsigned)chunks, (unsigned)prm.Hv), per_seq((unsigned)prm.N, (unsigned)prm.Hv, DV / SL);
+  cudaError_t e;
+  if ((e = launch_k(prep_kernel<TI, DK, DV>, per_chunk, PrepSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  if ((e = launch_k(fwd_chain_kernel<TI, DK, DV>, per_seq, FwdSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  if ((e = launch_k(grads_state_kernel<TI, DK, DV>, per_chunk, StateGradSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  return launch_k(grads_local_kernel<TI, DK, DV>, per_chunk, LocalSmem<DK, DV>::BYTES, prm, stream);
+}
+
+template <typename TI>
+cudaError_t run_chunked_dims(const cbwd::Params &prm, int Dk, int Dv, int64_t chunks, cudaStream_t stream) {
+  if (Dk == 128 && Dv == 128) return run_chunked<TI, 128, 128>(prm, chunks, stream);
+  if (Dk == 128 && Dv == 64) return run_chunked<TI, 128, 64>(prm, chunks, stream);
+  if (Dk == 64 && Dv == 128) return run_chunked<TI, 64, 128>(prm, chunks, stream);
+  return run_chunked<TI, 64, 64>(prm, chunks, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v, const float *g,
+                                    const float *beta, const int32_t *cu, int N, long long T_, int Hqk,
+                                    int Hv, int Dk, int Dv, int dtype, float scale, const float *s0,
+                                    const float *dO, const float *dSfin, float *dq, float *dk,
+                                    float *dv, float *dg, float *dbeta, float *ds0, void *workspace,
+                                    cudaStream_t stream) {
+  const int T = (int)T_;
+  unsigned char *ws = static_cast<unsigned char *>(workspace);
+  const CbwdLayout L = cbwd_layout(N, T, Hqk, Hv, Dk, Dv);
+  int32_t *status = reinterpret_cast<int32_t *>(ws);
+  auto *ph = reinterpret_cast<tp::PlanHeader *>(ws + tp::kPlanHeaderOffset);
+  int32_t *ne_seq = reinterpret_cast<int32_t *>(ws + L.plan), *ne_cs = ne_seq + N;
+  cudaError_t e = launch_plan(cu, N, T, Hv, dSfin, ds0, (size_t)Hv * Dv * Dk * sizeof(float), ph, ne_seq,
+                              ne_cs, status, stream);
+  if (e != cudaSuccess || T == 0) return e;
+  auto F = [&](size_t off) { return reinterpret_cast<float *>(ws + off); };
+  cbwd::Params prm;
+  prm.q = q; prm.k = k; prm.v = v; prm.g = g; prm.beta = beta; prm.cu = cu;
+  prm.N = N; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.scale = scale;
+  prm.s0 = s0; prm.dO = dO; prm.dSf = dSfin;
+  prm.dq = Hv == Hqk ? dq : F(L.dqh);
+  prm.dk = Hv == Hqk ? dk : F(L.dkh);
+  prm.dv = dv; prm.dg = dg; prm.dbeta = dbeta; prm.ds0 = ds0;
+  prm.ph = ph; prm.ne_seq = ne_seq; prm.ne_cs = ne_cs;
+  prm.Tm = F(L.Tm); prm.P = F(L.P); prm.EKK = F(L.EKK);
+  prm.W = F(L.W); prm.dQp = F(L.dQp); prm.dKp = F(L.dKp); prm.dW = F(L.dW);
+  prm.Ut = F(L.Ut); prm.U = F(L.U); prm.dU = F(L.dU);
+  prm.S0 = F(L.S0); prm.dS1 = F(L.dS1); prm.sc = F(L.sc);
+  prm.G = reinterpret_cast<double *>(ws + L.G);
+  const int64_t chunks = tp::chunk_bound(N, T);
+  e = dtype == GDN_DTYPE_BF16 ? run_chunked_dims<__nv_bfloat16>(prm, Dk, Dv, chunks, stream)
+                              : run_chunked_dims<float>(prm, Dk, Dv, chunks, stream);
+  if (e != cudaSuccess) return e;
+  if (Hv != Hqk) {
+    const size_t rows_qk = (size_t)T * Hqk;
+    if ((e = launch_group_sum(prm.dq, dq, rows_qk, Hv / Hqk, Dk, stream)) != cudaSuccess) return e;
+    if ((e = launch_group_sum(prm.dk, dk, rows_qk, Hv / Hqk, Dk, stream)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace gdn

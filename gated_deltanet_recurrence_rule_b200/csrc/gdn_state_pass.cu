@@ -120,6 +120,18 @@ plan_kernel(const int32_t *__restrict__ cu, int N, int T, int Hv, const void *__
 
 }  // namespace plan
 
+// One plan_kernel launch (also used by the chunk-form backward, which passes
+// dL/dS_final and dL/dS_initial as the initial and final states, so that an
+// empty sequence gets dL/dS_initial = dL/dS_final).  state_bytes is one
+// sequence's states: Hv x Dv x Dk x element size.
+cudaError_t launch_plan(const int32_t *cu, int N, int T, int Hv, const void *s0, void *sfin,
+                        size_t state_bytes, tp::PlanHeader *ph, int32_t *ne_seq, int32_t *ne_cs,
+                        int32_t *status, cudaStream_t stream) {
+  plan::plan_kernel<<<1, 1024, 0, stream>>>(cu, N, T, Hv, s0, sfin, state_bytes, ph, ne_seq, ne_cs,
+                                           status);
+  return cudaGetLastError();
+}
+
 namespace sp {
 
 using namespace sm100;

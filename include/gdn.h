@@ -317,15 +317,32 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
                           int32_t input_form, float scale, int32_t *device_status, void *stream);
 
 /*
- * Bytes of device workspace gdn_prefill_backward needs for these sizes (0 for
- * invalid sizes): the status header, a checkpoint of every state every 16
- * tokens (about (T/16 + num_seqs) x Hv x Dv x Dk x 4 bytes), a scratch of 16
- * states per (sequence, value head), and per-value-head dq, dk when
- * Hv > Hqk.
+ * Bytes of device workspace gdn_prefill_backward needs to run the chunk-form
+ * backward (0 for invalid sizes): the status header and plan, then per
+ * (64-token chunk, value head) the chunk's fp32 intermediates (Tm, P and
+ * E . K K^T at 64 x 64; W, U~, U, dU, dW and two partial gradients at 64 x D;
+ * the state and dL/dstate at the chunk's boundaries, Dv x Dk each; about
+ * (T/64 + num_seqs) x Hv x (2 Dv Dk + 5 x 64 D + 3 x 64 x 64) x 4 bytes), and
+ * per-value-head dq, dk when Hv > Hqk.  At 8192 tokens, 48 value heads and
+ * D = 128 that is about 2.9 GB.  The value is at least the sequential size
+ * below, so a workspace of this size always runs the chunk form.
  */
 size_t gdn_prefill_backward_workspace_size(int32_t num_seqs, int64_t total_tokens,
                                            int32_t num_qk_heads, int32_t num_v_heads,
                                            int32_t head_dim_k, int32_t head_dim_v);
+
+/*
+ * Bytes of device workspace the sequential (token-by-token) backward needs
+ * (0 for invalid sizes): the status header, a checkpoint of every state
+ * every 16 tokens (about (T/16 + num_seqs) x Hv x Dv x Dk x 4 bytes), a
+ * scratch of 16 states per (sequence, value head), and per-value-head dq, dk
+ * when Hv > Hqk.  gdn_prefill_backward runs the sequential form when its
+ * workspace holds at least this many bytes but fewer than
+ * gdn_prefill_backward_workspace_size.
+ */
+size_t gdn_prefill_backward_workspace_size_sequential(int32_t num_seqs, int64_t total_tokens,
+                                                      int32_t num_qk_heads, int32_t num_v_heads,
+                                                      int32_t head_dim_k, int32_t head_dim_v);
 
 /*
  * Backward pass of gdn_prefill (training): the gradients of a loss L with
@@ -333,13 +350,30 @@ size_t gdn_prefill_backward_workspace_size(int32_t num_seqs, int64_t total_token
  * optionally d_final_state = dL/dS_final.  Same rule, layout and sequences as
  * gdn_prefill with fp32 states and prepared inputs (the page's note says the
  * block form is used in training as well: "Inside Qwen3.8-27B ...", section
- * "Gated DeltaNet Mechanics").  With u = S_{t-1} k_t, w = v_t - alpha_t u and
- * G = dL/dS_t, going backwards over the tokens:
- *   G += scale dO_t q_t^T;  dq_t = scale S_t^T dO_t;  dv_t = beta_t G k_t;
- *   dbeta_t = w . G k_t;  dg_t = alpha_t (<G, S_{t-1}> - beta_t (G k_t) . u);
- *   dk_t = beta_t G^T w - alpha_t beta_t S_{t-1}^T G k_t;
- *   G <- alpha_t (G - beta_t (G k_t) k_t^T);  d_initial_state = G at the start.
- * dq and dk of a query/key head sum over the value heads reading it.
+ * "Gated DeltaNet Mechanics").
+ *
+ * Two algorithms, chosen by the workspace size, both fp32-accurate:
+ *   - chunk form (workspace >= gdn_prefill_backward_workspace_size): the
+ *     reverse mode of the chunked WY/UT form.  Per 64-token chunk with
+ *     E_ts = e^{G_t - G_s}, P = E . Q K^T, Tm = (I + A)^-1 and
+ *     U = U~ - W S0^T as in gdn_prefill, going backwards over the chunks
+ *     with dO' = scale d_o and dS1 = dL/d(state after the chunk):
+ *       dU = P^T dO' + diag(kdec) K dS1^T;
+ *       dS0 = gamma_C dS1 + dO'^T diag(gamma) Q - dU^T W;
+ *     then every chunk on its own: dQ, dK, dV, dbeta and dG through the
+ *     products of the WY/UT transform (dA = -Tm^T dT Tm^T) and dg as suffix
+ *     sums of dG within the chunk.  The dense products run on tensor cores
+ *     (tf32 with a 3-term hi/lo split of both operands, about fp32
+ *     accuracy).  g is clamped at -30 as in the tensor-core prefill.
+ *   - sequential (at least gdn_prefill_backward_workspace_size_sequential
+ *     bytes): the token-by-token rule on CUDA cores.  With u = S_{t-1} k_t,
+ *     w = v_t - alpha_t u and G = dL/dS_t, going backwards over the tokens:
+ *       G += scale dO_t q_t^T;  dq_t = scale S_t^T dO_t;  dv_t = beta_t G k_t;
+ *       dbeta_t = w . G k_t;  dg_t = alpha_t (<G, S_{t-1}> - beta_t (G k_t) . u);
+ *       dk_t = beta_t G^T w - alpha_t beta_t S_{t-1}^T G k_t;
+ *       G <- alpha_t (G - beta_t (G k_t) k_t^T);  d_initial_state = G at the start.
+ * dq and dk of a query/key head sum over the value heads reading it, in a
+ * fixed order (results do not depend on scheduling).
  *
  *   q, k, v, g, beta, cu_seqlens, initial_state (fp32 or NULL), scale: as for
  *                  gdn_prefill (prepared inputs; dtype bf16 or fp32)
@@ -347,12 +381,11 @@ size_t gdn_prefill_backward_workspace_size(int32_t num_seqs, int64_t total_token
  *   d_final_state  [num_seqs, Hv, Dv, Dk] fp32, or NULL for zeros
  *   dq, dk         [T, Hqk, Dk] fp32 (outputs);  dv [T, Hv, Dv] fp32;
  *   dg, dbeta      [T, Hv] fp32;  d_initial_state [num_seqs, Hv, Dv, Dk] fp32 or NULL
- *   workspace      >= gdn_prefill_backward_workspace_size(...) bytes, 256-byte
- *                  aligned; its first word is the sticky device status word
- *                  (GDN_ERR_BAD_SEQLENS), read with gdn_get_device_status.
- * Runs on CUDA cores in fp32: one block per (sequence, value head) with the
- * state and G in registers, a forward pass storing checkpoints, then the
- * chunks in reverse.  Supported: Hv % Hqk == 0; Dk, Dv in {64, 128}.
+ *   workspace      256-byte aligned, sized as above; its first word is the
+ *                  sticky device status word (GDN_ERR_BAD_SEQLENS), read with
+ *                  gdn_get_device_status.  Smaller than the sequential size:
+ *                  GDN_ERR_WORKSPACE.
+ * Supported: Hv % Hqk == 0; Dk, Dv in {64, 128}.
  */
 int32_t gdn_prefill_backward(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, const int32_t *cu_seqlens, int32_t num_seqs,
@@ -362,6 +395,21 @@ int32_t gdn_prefill_backward(const void *q, const void *k, const void *v, const 
                              const float *d_final_state, float *dq, float *dk, float *dv,
                              float *dg, float *dbeta, float *d_initial_state, void *workspace,
                              size_t workspace_bytes, void *stream);
+
+/*
+ * The sequential backward on its own, whatever the workspace size: same
+ * arguments and results as gdn_prefill_backward; the workspace must hold at
+ * least gdn_prefill_backward_workspace_size_sequential bytes.
+ */
+int32_t gdn_prefill_backward_sequential(const void *q, const void *k, const void *v, const float *g,
+                                        const float *beta, const int32_t *cu_seqlens,
+                                        int32_t num_seqs, int64_t total_tokens,
+                                        int32_t num_qk_heads, int32_t num_v_heads,
+                                        int32_t head_dim_k, int32_t head_dim_v, int32_t dtype,
+                                        float scale, const float *initial_state, const float *d_o,
+                                        const float *d_final_state, float *dq, float *dk,
+                                        float *dv, float *dg, float *dbeta, float *d_initial_state,
+                                        void *workspace, size_t workspace_bytes, void *stream);
 
 /*
  * 1 if gdn_prefill with these sizes and dtype runs the tensor-core (tcgen05)

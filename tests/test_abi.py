@@ -175,15 +175,29 @@ def test_backward_workspace_and_validation(lib):
     """gdn_prefill_backward: workspace arithmetic and host-side rejections
     (nothing is launched; the fake addresses are never dereferenced)."""
     ck = 64 * 1024  # one 128 x 128 fp32 state
-    # 48 heads fill few SMs: 4 row slices per head, dq/dk/dg/dbeta per slice
-    ws = api.prefill_backward_workspace_size(1, 8192, 16, 48, 128, 128)
+    # sequential form.  48 heads fill few SMs: 4 row slices per head, dq/dk/dg/dbeta per slice
+    ws = api.prefill_backward_workspace_size(1, 8192, 16, 48, 128, 128, sequential=True)
     need = (512 + 1) * 48 * ck + 48 * 16 * ck + 2 * 8192 * 48 * 4 * (128 * 4 + 4)
     assert need <= ws <= need + 6 * 256
     # 8 sequences x 48 heads fill the GPU: one slice, dq/dk per value head only
-    ws8 = api.prefill_backward_workspace_size(8, 8192, 16, 48, 128, 128)
+    ws8 = api.prefill_backward_workspace_size(8, 8192, 16, 48, 128, 128, sequential=True)
     need8 = (512 + 8) * 48 * ck + 8 * 48 * 16 * ck + 2 * 8192 * 48 * 128 * 4
     assert need8 <= ws8 <= need8 + 4 * 256
-    assert api.prefill_backward_workspace_size(8, 8192, 48, 48, 128, 128) == ws8 - 2 * 8192 * 48 * 128 * 4
+    assert (api.prefill_backward_workspace_size(8, 8192, 48, 48, 128, 128, sequential=True)
+            == ws8 - 2 * 8192 * 48 * 128 * 4)
+    # chunk form: per (chunk, value head) 3 tiles of 64 x 64, 7 of 64 x 128, the state and its
+    # gradient (128 x 128 each), 3 x 64 fp32 scalars and 64 fp64 log-decay sums; chunks bounded
+    # by ceil(T / 64) + N
+    # (the reported size is the larger of the two forms, so it always runs the chunk form)
+    per_unit = 4 * (3 * 64 * 64 + 7 * 64 * 128 + 2 * 128 * 128 + 3 * 64) + 8 * 64  # G in fp64
+    wsc1 = api.prefill_backward_workspace_size(1, 8192, 16, 48, 128, 128)
+    needc1 = (128 + 1) * 48 * per_unit + 2 * 8192 * 48 * 128 * 4
+    assert wsc1 == max(ws, wsc1) and (wsc1 == ws or needc1 <= wsc1 <= needc1 + 20 * 256)
+    wsc8 = api.prefill_backward_workspace_size(8, 8192, 16, 48, 128, 128)
+    needc8 = (128 + 8) * 48 * per_unit + 2 * 8192 * 48 * 128 * 4
+    assert wsc8 > ws8 and needc8 <= wsc8 <= needc8 + 20 * 256
+    assert (api.prefill_backward_workspace_size(8, 8192, 48, 48, 128, 128)
+            == wsc8 - 2 * 8192 * 48 * 128 * 4)
     assert lib.gdn_prefill_backward_workspace_size(1, 10, 16, 40, 128, 128) == 0  # 40 % 16
     assert lib.gdn_prefill_backward_workspace_size(1, 10, 16, 48, 96, 128) == 0
     vp = 1 << 12
@@ -191,17 +205,18 @@ def test_backward_workspace_and_validation(lib):
              scale=1.0, s0=None, do=vp, dsf=None, dq=vp, dk=vp, dv=vp, dg=vp, db=vp, ds0=None,
              ws=vp, wsb=1 << 30)
 
-    def call(**kw):
-        x = {**a, **kw}
-        return lib.gdn_prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu"], x["N"],
-                                        x["T"], x["Hqk"], x["Hv"], x["Dk"], x["Dv"], x["dtype"],
-                                        x["scale"], x["s0"], x["do"], x["dsf"], x["dq"], x["dk"],
-                                        x["dv"], x["dg"], x["db"], x["ds0"], x["ws"], x["wsb"], None)
+    for fn in (lib.gdn_prefill_backward, lib.gdn_prefill_backward_sequential):
+        def call(**kw):
+            x = {**a, **kw}
+            return fn(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu"], x["N"], x["T"], x["Hqk"],
+                      x["Hv"], x["Dk"], x["Dv"], x["dtype"], x["scale"], x["s0"], x["do"], x["dsf"],
+                      x["dq"], x["dk"], x["dv"], x["dg"], x["db"], x["ds0"], x["ws"], x["wsb"], None)
 
-    assert call(do=None) == api.GDN_ERR_INVALID_ARG
-    assert call(dq=vp + 4) == api.GDN_ERR_INVALID_ARG          # misaligned
-    assert call(Hv=5) == api.GDN_ERR_INVALID_ARG
-    assert call(Dk=96) == api.GDN_ERR_UNSUPPORTED
-    assert call(wsb=1024) == api.GDN_ERR_WORKSPACE
-    assert call(ws=vp + 16) == api.GDN_ERR_WORKSPACE            # not 256-byte aligned
-    assert call(N=0, T=0) == api.GDN_OK
+        assert call(do=None) == api.GDN_ERR_INVALID_ARG
+        assert call(dq=vp + 4) == api.GDN_ERR_INVALID_ARG          # misaligned
+        assert call(Hv=5) == api.GDN_ERR_INVALID_ARG
+        assert call(Dk=96) == api.GDN_ERR_UNSUPPORTED
+        assert call(wsb=1024) == api.GDN_ERR_WORKSPACE
+        assert call(ws=vp + 16) == api.GDN_ERR_WORKSPACE            # not 256-byte aligned
+        assert call(N=0, T=0) == api.GDN_OK
+        assert call(N=0, T=5) == api.GDN_ERR_INVALID_ARG

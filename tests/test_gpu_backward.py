@@ -1,5 +1,7 @@
-"""Backward pass (gdn_prefill_backward) on the GPU against the fp64 oracle's
-backward, itself pinned to central finite differences of the forward rule."""
+"""Backward pass on the GPU against the fp64 oracle's backward, itself pinned to
+central finite differences of the forward rule.  Every case runs both
+algorithms: the chunk form (gdn_prefill_backward with its full workspace) and
+the sequential one (gdn_prefill_backward_sequential)."""
 import numpy as np
 import pytest
 import torch
@@ -13,7 +15,12 @@ DEV = torch.device("cuda:0")
 TOL = 1e-4  # fp32 arithmetic against fp64 on the same inputs: max|err| / RMS(ref) per gradient
 
 
-def _case(lengths, Hqk, Hv, D, dtype, seed, init=True, dsf=True, scale=0.5, edit=None):
+@pytest.fixture(params=["chunked", "sequential"])
+def algo(request):
+    return request.param
+
+
+def _case(lengths, Hqk, Hv, D, dtype, seed, algo, init=True, dsf=True, scale=0.5, edit=None):
     inp = inputs.prefill_inputs(lengths, Hqk, Hv, D, dtype=dtype, seed=seed,
                                 init_std=0.1 if init else 0.0)
     if edit is not None:
@@ -25,7 +32,8 @@ def _case(lengths, Hqk, Hv, D, dtype, seed, init=True, dsf=True, scale=0.5, edit
     dev = {n: (t.to(DEV) if t is not None else None) for n, t in inp.items()}
     out = api.prefill_backward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], d_o.to(DEV),
                                cu_seqlens=dev["cu_seqlens"], initial_state=dev["initial_state"],
-                               d_final_state=None if d_sf is None else d_sf.to(DEV), scale=scale)
+                               d_final_state=None if d_sf is None else d_sf.to(DEV), scale=scale,
+                               sequential=algo == "sequential")
     torch.cuda.synchronize()
     ref = oracle.backward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], d_o,
                           cu_seqlens=inp["cu_seqlens"], initial_state=inp["initial_state"],
@@ -43,12 +51,20 @@ def _check(out, ref, what):
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_backward_varlen_gqa(dtype, D):
-    out, ref = _case([37, 0, 50, 16], 2, 6, D, dtype, seed=101 + D)
-    _check(out, ref, f"{dtype} D={D}")
+def test_backward_varlen_gqa(dtype, D, algo):
+    out, ref = _case([37, 0, 50, 16], 2, 6, D, dtype, seed=101 + D, algo=algo)
+    _check(out, ref, f"{algo} {dtype} D={D}")
 
 
-def test_backward_degenerate_gates():
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_backward_chunk_boundaries(dtype, algo):
+    """Sequences of exactly one chunk, one chunk plus a token, two chunks plus
+    one, a single token and several chunks with a ragged tail, at D=128."""
+    out, ref = _case([64, 65, 129, 1, 200], 2, 6, 128, dtype, seed=121, algo=algo)
+    _check(out, ref, f"{algo} {dtype} chunk boundaries")
+
+
+def test_backward_degenerate_gates(algo):
     """alpha = 0 (g = -inf) on single tokens, at the first and last token of a
     16-token checkpoint interval and on a run; g = 0 on a stretch; beta = 0 and
     beta = 1 on others."""
@@ -57,11 +73,11 @@ def test_backward_degenerate_gates():
         inp["g"][30:45] = 0.0
         inp["beta"][[3, 4, 50, 80]] = 0.0
         inp["beta"][[7, 33, 90]] = 1.0
-    out, ref = _case([70, 40], 2, 6, 64, "fp32", seed=111, edit=edit)
-    _check(out, ref, "gates")
+    out, ref = _case([70, 40], 2, 6, 64, "fp32", seed=111, algo=algo, edit=edit)
+    _check(out, ref, f"{algo} gates")
 
 
-def test_backward_mixed_dims():
+def test_backward_mixed_dims(algo):
     """Dk != Dv, one value head per query/key head (dq, dk written directly)."""
     for Dk, Dv in ((128, 64), (64, 128)):
         inp = inputs.prefill_inputs([40, 23], 2, 2, Dk, dtype="fp32", seed=105, init_std=0.1)
@@ -72,29 +88,31 @@ def test_backward_mixed_dims():
         d_o = torch.randn(T, 2, Dv, generator=gen)
         out = api.prefill_backward(inp["q"].to(DEV), inp["k"].to(DEV), v.to(DEV), inp["g"].to(DEV),
                                    inp["beta"].to(DEV), d_o.to(DEV),
-                                   cu_seqlens=inp["cu_seqlens"].to(DEV), initial_state=s0.to(DEV))
+                                   cu_seqlens=inp["cu_seqlens"].to(DEV), initial_state=s0.to(DEV),
+                                   sequential=algo == "sequential")
         torch.cuda.synchronize()
         ref = oracle.backward(inp["q"], inp["k"], v, inp["g"], inp["beta"], d_o,
                               cu_seqlens=inp["cu_seqlens"], initial_state=s0)
-        _check(out, ref, f"Dk={Dk} Dv={Dv}")
+        _check(out, ref, f"{algo} Dk={Dk} Dv={Dv}")
 
 
-def test_backward_without_states():
+def test_backward_without_states(algo):
     """No initial state and no final-state gradient (both NULL)."""
-    out, ref = _case([70], 1, 3, 64, "fp32", seed=107, init=False, dsf=False, scale=1.0)
-    _check(out, ref, "no states")
+    out, ref = _case([70], 1, 3, 64, "fp32", seed=107, algo=algo, init=False, dsf=False, scale=1.0)
+    _check(out, ref, f"{algo} no states")
 
 
-def test_backward_long_sequence():
-    """1000 tokens (62 chunks of 16 plus a ragged one) at D=64."""
-    out, ref = _case([1000], 1, 2, 64, "bf16", seed=108)
-    _check(out, ref, "T=1000")
+def test_backward_long_sequence(algo):
+    """1000 tokens (15 chunks of 64 plus a ragged one; 62 checkpoint intervals
+    of 16 plus one for the sequential form) at D=64."""
+    out, ref = _case([1000], 1, 2, 64, "bf16", seed=108, algo=algo)
+    _check(out, ref, f"{algo} T=1000")
 
 
 @pytest.mark.parametrize("Hqk,Hv,N", [(2, 6, 50), (2, 2, 150)])
-def test_backward_many_units_one_slice(Hqk, Hv, N):
+def test_backward_many_units_one_slice(Hqk, Hv, N, algo):
     """Enough (sequence, value head) units to fill the GPU: one slice per head,
     dg and dbeta written directly (and dq, dk too when Hv == Hqk)."""
     lengths = [(7 * i) % 23 for i in range(N)]  # 0 .. 22 tokens, some empty
-    out, ref = _case(lengths, Hqk, Hv, 64, "fp32", seed=109 + Hv)
-    _check(out, ref, f"{N} sequences x {Hv} heads")
+    out, ref = _case(lengths, Hqk, Hv, 64, "fp32", seed=109 + Hv, algo=algo)
+    _check(out, ref, f"{algo} {N} sequences x {Hv} heads")

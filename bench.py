@@ -696,11 +696,28 @@ def _prefill_leg(args, D, dev, peaks, peak_src, name, single_pass=False):
     return out
 
 
+# Algorithmic flops of the chunk-form backward per (64-token chunk, value head)
+# at head dim D (an FMA counts 2; the solve of the 64 x 64 triangular system,
+# the elementwise work and the 3-term split of every tensor-core product are
+# not counted).  Each term is one matrix product of the algebra:
+#   prep         Q K^T, K K^T, W = Tm (.) K, U~ = Tm (.) V          4 x 64.64.D
+#   forward      U = U~ - W S0^T, S1 = g S0 + U^T (.) K             2 x 64.D.D
+#   reverse      P^T dO', K dS1^T, dO'^T (.) Q, dU^T W              64.64.D + 3 x 64.D.D
+#   state grads  dO' S0, dU S0, U dS1                               3 x 64.D.D
+#   local grads  dO' U^T, dW K^T, dU V^T, Tm^T dW, Tm^T dU,
+#                (dP.E) K, (dP.E)^T Q, (B + B^T) K                  8 x 64.64.D
+#                dT Tm^T, Tm^T Z                                    2 x 64.64.64
+def backward_chunk_flops(D: int, C: int = 64) -> int:
+    return 2 * (13 * C * C * D + 8 * C * D * D + 2 * C * C * C)
+
+
 def _backward(args, D, dev, x, T, w, peaks):
-    """Backward pass of the prefill step (gdn_prefill_backward) on the same
-    workload: d_o and dL/dS_final random fp32, gradients for q, k, v, g, beta
-    and the initial state.  CUDA cores, fp32: the roofline is the fp32 FMA
-    rate."""
+    """Backward pass of the prefill step on the same workload: d_o and
+    dL/dS_final random fp32, gradients for q, k, v, g, beta and the initial
+    state.  The leg's value is the chunk form (gdn_prefill_backward with its
+    full workspace, tf32 tensor-core products with a 3-term split); the
+    sequential CUDA-core form (gdn_prefill_backward_sequential) is timed
+    beside it."""
     import torch
 
     from gated_deltanet_recurrence_rule_b200 import api
@@ -708,51 +725,73 @@ def _backward(args, D, dev, x, T, w, peaks):
     gen = torch.Generator(device=dev).manual_seed(12)
     d_o = torch.randn((T, w.Hv, w.D), generator=gen, device=dev)
     d_sf = torch.randn((1, w.Hv, w.D, w.D), generator=gen, device=dev) * 0.1
-    ws = torch.zeros(api.prefill_backward_workspace_size(1, T, w.Hqk, w.Hv, w.D, w.D),
-                     dtype=torch.uint8, device=dev)
-
-    def step():
-        return api.prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d_o,
-                                    cu_seqlens=x["cu_seqlens"], d_final_state=d_sf, workspace=ws)
-
     steps = max(1, min(args.steps, 3))
-    for _ in range(2):
-        step()
-    torch.cuda.synchronize()
     stream = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    D.barrier()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(steps):
-        step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    D.barrier()
-    ms = D.max(e0.elapsed_time(e1), dev) / steps
-    status = api.get_device_status(ws)
-    if status != api.GDN_OK:
-        raise RuntimeError(f"device status after the backward leg: {api.status_string(status)}")
-    # Algorithmic fp32 work per token and value head (an FMA counts 2): the
-    # forward state S_t (u = S k, S update: 4 D^2) and the backward terms
-    # (G += dO q^T, S_t^T dO, G k, <G, S>, G^T w, S^T G k, G update: 14 D^2).
-    # The kernel's recomputation of the states from checkpoints is not counted.
-    flop = 18 * w.D * w.D * w.Hv * T
-    fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+
+    def timed(sequential):
+        ws = torch.zeros(api.prefill_backward_workspace_size(1, T, w.Hqk, w.Hv, w.D, w.D,
+                                                             sequential=sequential),
+                         dtype=torch.uint8, device=dev)
+
+        def step():
+            return api.prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], d_o,
+                                        cu_seqlens=x["cu_seqlens"], d_final_state=d_sf,
+                                        workspace=ws, sequential=sequential)
+
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        D.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        D.barrier()
+        ms = D.max(e0.elapsed_time(e1), dev) / steps
+        status = api.get_device_status(ws)
+        if status != api.GDN_OK:
+            raise RuntimeError(f"device status after the backward leg: {api.status_string(status)}")
+        del ws
+        return ms
+
+    ms = timed(False)
+    ms_seq = timed(True)
+    units = -(-T // 64) * w.Hv
+    flop = backward_chunk_flops(w.D) * units
+    # tf32 dense peak from the measured bf16 GEMM and the nominal tf32 : bf16 ratio (1.1 : 2.25)
+    tf32_peak = peaks["bf16_tflops"] * 1.1 / 2.25
     achieved = flop / (ms / 1e3) / 1e12
+    # the sequential form: 18 D^2 fp32 flop per token and value head on CUDA cores
+    seq_flop = 18 * w.D * w.D * w.Hv * T
+    fp32_peak = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    seq_ach = seq_flop / (ms_seq / 1e3) / 1e12
+    bwd_sources = [os.path.join(CSRC, n) for n in ("gdn_common.cuh", "gdn_chunk_ops.cuh", "gdn_sm100.cuh",
+                                                   "gdn_twophase.cuh", "gdn_backward_chunked.cu")]
     return {"value": D.world * T / (ms / 1e3) / 1e6, "unit": "Mtok/s",
             "workload": f"backward of prefill8k: T={T} Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16 inputs, "
                         "fp32 d_o and dL/dS_final, zero initial state",
             "ms_per_step": ms,
-            "roofline": {"bound": "alu", "kernel": "backward_kernel (4 row slices per head), then "
-                                                    "group_sum_kernel x 4 for dq, dk, dg, dbeta",
-                         "achieved": achieved, "peak": fp32_peak, "unit": "TFLOP/s",
-                         "frac": achieved / fp32_peak,
-                         "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
-                         "algorithmic": f"18 D^2 flop per token and value head = {flop} flop",
-                         "traffic": kernel_traffic("prefill_backward", [os.path.join(CSRC, n) for n in
-                                                                          ("gdn_common.cuh", "gdn_backward.cu")])},
-            "gpu_launches": 5 * steps}  # at these sizes: 4 row slices per head, Hv > Hqk
+            "roofline": {"bound": "tensor", "kernel": "chunk form: plan, prep, forward chain, reverse "
+                                                      "chain, state grads, local grads, 2 group sums",
+                         "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
+                         "frac": achieved / tf32_peak,
+                         "peak_source": "measured bf16_tflops x nominal tf32/bf16 (1.1/2.25); "
+                                        "warp-level m16n8k8 tf32 MMAs, each product issued 3 times "
+                                        "(hi/lo split)",
+                         "algorithmic": f"{backward_chunk_flops(w.D)} flop per (64-token chunk, value head)"
+                                        f" x {units} = {flop} flop",
+                         "traffic": kernel_traffic("prefill_backward_chunked", bwd_sources)},
+            "sequential": {"ms_per_step": ms_seq, "value": D.world * T / (ms_seq / 1e3) / 1e6,
+                           "unit": "Mtok/s",
+                           "roofline": {"bound": "alu", "achieved": seq_ach, "peak": fp32_peak,
+                                        "unit": "TFLOP/s", "frac": seq_ach / fp32_peak,
+                                        "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
+                                        "algorithmic": f"18 D^2 flop per token and value head = {seq_flop} flop"},
+                           "gpu_launches": 5 * steps},
+            "gpu_launches": 8 * steps}  # plan, 5 chunk-form kernels, 2 group sums (Hv > Hqk)
 
 
 def _decode(args, D, dev, peaks, peak_src):

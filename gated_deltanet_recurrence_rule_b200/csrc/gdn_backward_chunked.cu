@@ -34,19 +34,21 @@
 //                their first chunk; d_initial_state of an empty sequence is
 //                d_final_state (or zero)
 //   prep         per (chunk, value head): P, E . K K^T, Tm, W, U~, G
-//   fwd_chain    per (sequence, value head, 32 rows of the state): the state
+//   fwd_chain    per (sequence, value head, 64 rows of the state): the state
 //                at every chunk start (S0) and U, in chunk order
-//   rev_chain    per (sequence, value head, 32 rows): dS1 and dU, chunks last
+//   rev_chain    per (sequence, value head, 64 rows): dS1 and dU, chunks last
 //                to first, and d_initial_state
 //   grads_state  per (chunk, value head): the products with S0 and dS1
 //   grads_local  per (chunk, value head): the 64 x 64 algebra, then dq, dk
 //                (per value head), dv, dg, dbeta
 //   group sums   dq, dk over the value heads of each query/key head
 // Rows of S and of dS evolve independently (the chains never mix rows), so
-// each chain CTA owns 32 of the Dv rows.  Every product runs on warp-level
-// m16n8k8 tf32 tensor-core MMAs with both operands split into hi = tf32(x)
-// and lo = tf32(x - hi) and three products (hi*hi + hi*lo + lo*hi), which
-// keeps about fp32 accuracy.  Per-row sums go through fixed-order partials,
+// each chain CTA owns 64 of the Dv rows.  Tiles move global -> shared with
+// cp.async, all of a step's copies in flight at once, and the chains fetch
+// a chunk's tiles while the previous chunk computes where buffers allow.  Every product runs on warp-level
+// m16n8k8 tf32 tensor-core MMAs with both operands split into hi (x with the
+// low 13 mantissa bits cleared) and lo = x - hi, and three products (hi*hi +
+// hi*lo + lo*hi), which keeps about fp32 accuracy.  Per-row sums go through fixed-order partials,
 // so results do not depend on scheduling.
 #include <algorithm>
 
@@ -66,7 +68,7 @@ namespace cbwd {
 
 constexpr int C = 64;         // chunk length
 constexpr int NT = 256;       // threads per CTA (8 warps)
-constexpr int SL = 32;        // state rows per chain CTA
+constexpr int SL = 64;        // state rows per chain CTA
 constexpr int LD64 = 68;      // fp32 row stride of 64 x 64 tiles in shared memory
 constexpr float kGmin = -30.f;  // g clamp: alpha >= e^-30, so prefix sums stay finite
 
@@ -92,6 +94,17 @@ struct Params {
 };
 
 // ---- tensor-core building block -------------------------------------------
+// Split of an fp32 value for the 3-term tf32 products: hi keeps the sign,
+// exponent and the 10 mantissa bits a tf32 operand holds (the low 13 bits
+// cleared, |x - hi| < 2^-10 |x|); lo = x - hi is exact in fp32 and goes to the
+// MMA as is, which reads only its tf32 bits (|error| < 2^-10 |lo|).  So
+// hi*hi' + hi*lo' + lo*hi' is within about 2^-19 of x*y, with bit operations
+// and one subtraction instead of conversions.
+__device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xffffe000u; }
+__device__ __forceinline__ uint32_t tf32_lo(float x, uint32_t hi) {
+  return __float_as_uint(x - __uint_as_float(hi));
+}
+
 // acc[t] (a 16 x 8 fragment) += X[16][8 KS] * Y[8 KS][8 t .. 8 t + 7] for t <
 // NTL tiles in a row.  X(r, c) and Y(r, c) read single elements; each is split
 // once per k step.  Fragment element e of tile t sits at row gid + 8 (e >> 1),
@@ -106,15 +119,14 @@ __device__ __forceinline__ void mma3_rows(float (&acc)[NTL][4], FX X, FY Y, int 
     uint32_t ah[4], al[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-      ah[e] = chunk::to_tf32(a[e]);
-      al[e] = chunk::to_tf32(a[e] - __uint_as_float(ah[e]));
+      ah[e] = tf32_hi(a[e]);
+      al[e] = tf32_lo(a[e], ah[e]);
     }
 #pragma unroll
     for (int t = 0; t < NTL; ++t) {
       const float b0 = Y(k0, 8 * t + gid), b1 = Y(k0 + 4, 8 * t + gid);
-      const uint32_t bh[2] = {chunk::to_tf32(b0), chunk::to_tf32(b1)};
-      const uint32_t bl[2] = {chunk::to_tf32(b0 - __uint_as_float(bh[0])),
-                              chunk::to_tf32(b1 - __uint_as_float(bh[1]))};
+      const uint32_t bh[2] = {tf32_hi(b0), tf32_hi(b1)};
+      const uint32_t bl[2] = {tf32_lo(b0, bh[0]), tf32_lo(b1, bh[1])};
       chunk::mma_tf32_16x8x8(acc[t], al, bh);
       chunk::mma_tf32_16x8x8(acc[t], ah, bl);
       chunk::mma_tf32_16x8x8(acc[t], ah, bh);
@@ -162,22 +174,29 @@ __device__ __forceinline__ void quad_row_sums(float (&acc)[NTL][4], F weight, in
   s_hi = b;
 }
 
-// ---- tile loads -------------------------------------------------------------
-// dst[r][0..COLS) (row stride ld floats) = mul * src[r * stride + 0..COLS) for
-// r < valid, zeros for valid <= r < ROWS.  COLS % 4 == 0; src 8- or 16-byte
-// aligned per row.
-template <int ROWS, int COLS, typename TI>
-__device__ __forceinline__ void load_tile(float *dst, int ld, const TI *src, size_t stride,
-                                          int valid, float mul, int tid) {
-  constexpr int V4 = COLS / 4;
-  for (int x = tid; x < ROWS * V4; x += NT) {
-    const int r = x / V4, c = 4 * (x - r * V4);
-    float f[4] = {0.f, 0.f, 0.f, 0.f};
-    if (r < valid) {
-      load4(src + (size_t)r * stride + c, f);
-      f[0] *= mul; f[1] *= mul; f[2] *= mul; f[3] *= mul;
-    }
-    *reinterpret_cast<float4 *>(dst + r * ld + c) = make_float4(f[0], f[1], f[2], f[3]);
+// ---- asynchronous tile copies -----------------------------------------------
+// 16 bytes global -> shared, or 16 zero bytes when !ok (the source is then
+// not read).
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool ok) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(sm100::smem_addr(dst)),
+               "l"(src), "r"(ok ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+// dst[r][0..COLS) (row stride ld elements) <- src[r * stride + 0..COLS) for r
+// < valid, zeros for valid <= r < ROWS.  Rows of dst and src 16-byte aligned.
+template <int ROWS, int COLS, typename E>
+__device__ __forceinline__ void tile_async(E *dst, int ld, const E *src, size_t stride, int valid,
+                                           int tid) {
+  constexpr int PER = 16 / sizeof(E), V = COLS / PER;
+  for (int x = tid; x < ROWS * V; x += NT) {
+    const int r = x / V, c = PER * (x - r * V);
+    const bool ok = r < valid;
+    cp_async16(dst + r * ld + c, ok ? src + (size_t)r * stride + c : src, ok);
   }
 }
 // dst[r * stride + c] = src[r][c] (row stride ld) for r < ROWS, c < COLS.
@@ -191,6 +210,17 @@ __device__ __forceinline__ void store_tile(float *dst, size_t stride, const floa
         *reinterpret_cast<const float4 *>(src + r * ld + c);
   }
 }
+template <int ROWS, int COLS>
+__device__ __forceinline__ void zero_tile(float *dst, int ld, int tid) {
+  for (int x = tid; x < ROWS * COLS; x += NT) dst[(x / COLS) * ld + x % COLS] = 0.f;
+}
+
+// Row stride (elements) of an input tile kept in its own type in shared
+// memory: conflict-free for the fragment reads of mma3_rows in both
+// orientations.
+template <typename E>
+constexpr int in_ld(int D) { return sizeof(E) == 2 ? D + 8 : D + 4; }
+constexpr size_t up16(size_t x) { return (x + 15) & ~(size_t)15; }
 
 struct ChunkPos {
   int n, start, len;
@@ -207,22 +237,25 @@ __device__ __forceinline__ bool chunk_pos(const Params &p, int c, ChunkPos &cp) 
 }
 
 // ---- prep: P, E . K K^T, Tm, W, U~ and G of one (chunk, value head) ----------
-template <int DK, int DV>
+template <typename TI, int DK, int DV>
 struct PrepSmem {
-  static constexpr int LQ = DK + 4, LK = DK + 4, LV = DV + 8;
-  static constexpr int OQ = 0, OK = OQ + C * LQ, OV = OK + C * LK, OA = OV + C * LV,
-                       OT = OA + C * LD64, OY = OT + C * LD64, OG = OY + 3 * 16 * 17,
-                       OB = OG + 2 * C, OBG = OB + C, FLOATS = OBG + C;
-  static constexpr size_t BYTES = FLOATS * sizeof(float);
+  static constexpr int LQ = in_ld<TI>(DK), LV = in_ld<TI>(DV);
+  static constexpr size_t OQ = 0, OK = OQ + up16(C * LQ * sizeof(TI)), OV = OK + up16(C * LQ * sizeof(TI)),
+                          OA = OV + up16(C * LV * sizeof(TI)), OT = OA + C * LD64 * 4,
+                          OY = OT + C * LD64 * 4, OG = OY + up16(3 * 16 * 17 * 4), OB = OG + C * 8,
+                          OBG = OB + C * 4, BYTES = OBG + C * 4;
 };
 
 template <typename TI, int DK, int DV>
 __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
-  using L = PrepSmem<DK, DV>;
-  extern __shared__ __align__(16) float sm[];
-  float *Qs = sm + L::OQ, *Ks = sm + L::OK, *Vs = sm + L::OV, *As = sm + L::OA, *Ts = sm + L::OT;
-  float *Ysc = sm + L::OY, *sB = sm + L::OB, *sBG = sm + L::OBG;
-  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  using L = PrepSmem<TI, DK, DV>;
+  extern __shared__ __align__(16) unsigned char smb[];
+  TI *Qs = reinterpret_cast<TI *>(smb + L::OQ), *Ks = reinterpret_cast<TI *>(smb + L::OK),
+     *Vs = reinterpret_cast<TI *>(smb + L::OV);
+  float *As = reinterpret_cast<float *>(smb + L::OA), *Ts = reinterpret_cast<float *>(smb + L::OT),
+        *Ysc = reinterpret_cast<float *>(smb + L::OY), *sB = reinterpret_cast<float *>(smb + L::OB),
+        *sBG = reinterpret_cast<float *>(smb + L::OBG);
+  double *sG = reinterpret_cast<double *>(smb + L::OG);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   ChunkPos cp;
   if (!chunk_pos(p, blockIdx.x, cp)) return;
@@ -230,11 +263,13 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
   const size_t u = (size_t)blockIdx.x * p.Hv + h;
   const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k),
            *v = static_cast<const TI *>(p.v);
-  load_tile<C, DK>(Qs, L::LQ, q + ((size_t)cp.start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, cp.len, 1.f, tid);
-  load_tile<C, DK>(Ks, L::LK, k + ((size_t)cp.start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, cp.len, 1.f, tid);
-  load_tile<C, DV>(Vs, L::LV, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, cp.len, 1.f, tid);
-  for (int x = tid; x < C * LD64; x += NT) Ts[x] = 0.f;
-  if (w == 0) {  // prefix sums of the clamped log-decays (2 tokens per lane)
+  const size_t qoff = ((size_t)cp.start * p.Hqk + hk) * DK, qstride = (size_t)p.Hqk * DK;
+  tile_async<C, DK>(Qs, L::LQ, q + qoff, qstride, cp.len, tid);
+  tile_async<C, DK>(Ks, L::LQ, k + qoff, qstride, cp.len, tid);
+  tile_async<C, DV>(Vs, L::LV, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, cp.len, tid);
+  cp_commit();
+  zero_tile<C, C>(Ts, LD64, tid);
+  if (w == 0) {  // prefix sums of the clamped log-decays, in fp64 (2 tokens per lane)
     const int t0 = 2 * lane;
     float g0 = 0.f, g1 = 0.f, b0 = 0.f, b1 = 0.f;
     if (t0 < cp.len) { g0 = fmaxf(p.g[(size_t)(cp.start + t0) * p.Hv + h], kGmin); b0 = p.beta[(size_t)(cp.start + t0) * p.Hv + h]; }
@@ -252,16 +287,17 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
     p.G[u * C + t0] = G0;
     p.G[u * C + t0 + 1] = G1;
   }
+  cp_wait<0>();
   __syncthreads();
   {  // QK^T and KK^T: warp rows 16 (w & 3), columns 32 (w >> 2)
     const int r0 = 16 * (w & 3), c0 = 32 * (w >> 2);
     float aq[4][4], ak[4][4];
     zero_acc(aq);
     zero_acc(ak);
-    mma3_rows<DK / 8>(aq, [&](int r, int c) { return Qs[(r0 + r) * L::LQ + c]; },
-                      [&](int r, int c) { return Ks[(c0 + c) * L::LK + r]; }, lane);
-    mma3_rows<DK / 8>(ak, [&](int r, int c) { return Ks[(r0 + r) * L::LK + c]; },
-                      [&](int r, int c) { return Ks[(c0 + c) * L::LK + r]; }, lane);
+    mma3_rows<DK / 8>(aq, [&](int r, int c) { return to_f32(Qs[(r0 + r) * L::LQ + c]); },
+                      [&](int r, int c) { return to_f32(Ks[(c0 + c) * L::LQ + r]); }, lane);
+    mma3_rows<DK / 8>(ak, [&](int r, int c) { return to_f32(Ks[(r0 + r) * L::LQ + c]); },
+                      [&](int r, int c) { return to_f32(Ks[(c0 + c) * L::LQ + r]); }, lane);
     float *P = p.P + u * C * C, *EKK = p.EKK + u * C * C;
     const int gid = lane >> 2, tig = lane & 3;
 #pragma unroll
@@ -291,7 +327,7 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
       float acc[DK / 16][4];
       zero_acc(acc);
       mma3_rows<C / 8>(acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c]; },
-                       [&](int r, int c) { return sBG[r] * Ks[r * L::LK + c0 + c]; }, lane);
+                       [&](int r, int c) { return sBG[r] * to_f32(Ks[r * L::LQ + c0 + c]); }, lane);
       float *W = p.W + u * C * DK;
       for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { W[i * DK + c] = x; });
     }
@@ -300,28 +336,30 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
       float acc[DV / 16][4];
       zero_acc(acc);
       mma3_rows<C / 8>(acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c]; },
-                       [&](int r, int c) { return sB[r] * Vs[r * L::LV + c0 + c]; }, lane);
+                       [&](int r, int c) { return sB[r] * to_f32(Vs[r * L::LV + c0 + c]); }, lane);
       float *Ut = p.Ut + u * C * DV;
       for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { Ut[i * DV + c] = x; });
     }
   }
 }
 
-// ---- forward chain: S0 and U of every chunk, per 32 rows of the state ---------
-template <int DK, int DV>
+// ---- forward chain: S0 and U of every chunk, per SL rows of the state ---------
+template <typename TI, int DK, int DV>
 struct FwdSmem {
-  static constexpr int LS = DK + 4, LW = DK + 4, LK = DK + 8, LU = SL + 8;
-  static constexpr int OS = 0, OW = OS + SL * LS, OK = OW + C * LW, OU = OK + C * LK,
-                       OG = OU + C * LU, OKD = OG + 2 * C, FLOATS = OKD + C;
-  static constexpr size_t BYTES = FLOATS * sizeof(float);
+  static constexpr int LS = DK + 4, LW = DK + 4, LK = in_ld<TI>(DK), LU = SL + 8;
+  static constexpr size_t OS = 0, OW = OS + SL * LS * 4, OK = OW + C * LW * 4,
+                          OU = OK + up16(C * LK * sizeof(TI)), OG = OU + C * LU * 4, OKD = OG + C * 8,
+                          BYTES = OKD + C * 4;
 };
 
 template <typename TI, int DK, int DV>
 __global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
-  using L = FwdSmem<DK, DV>;
-  extern __shared__ __align__(16) float sm[];
-  float *S = sm + L::OS, *Ws = sm + L::OW, *Ks = sm + L::OK, *Us = sm + L::OU, *sKd = sm + L::OKD;
-  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  using L = FwdSmem<TI, DK, DV>;
+  extern __shared__ __align__(16) unsigned char smb[];
+  float *S = reinterpret_cast<float *>(smb + L::OS), *Ws = reinterpret_cast<float *>(smb + L::OW),
+        *Us = reinterpret_cast<float *>(smb + L::OU), *sKd = reinterpret_cast<float *>(smb + L::OKD);
+  TI *Ks = reinterpret_cast<TI *>(smb + L::OK);
+  double *sG = reinterpret_cast<double *>(smb + L::OG);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int kk = blockIdx.x;
   if (kk >= p.ph->n_nonempty) return;
@@ -330,21 +368,24 @@ __global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
   const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk), v0 = SL * blockIdx.z;
   const TI *k = static_cast<const TI *>(p.k);
   const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;  // first state row of this slice
-  if (p.s0) load_tile<SL, DK>(S, L::LS, p.s0 + srow * DK, DK, SL, 1.f, tid);
-  else for (int x = tid; x < SL * L::LS; x += NT) S[x] = 0.f;
+  if (p.s0) tile_async<SL, DK>(S, L::LS, p.s0 + srow * DK, DK, SL, tid);
+  else zero_tile<SL, DK>(S, L::LS, tid);
+  tile_async<C, DK>(Ws, L::LW, p.W + (size_t)c0 * p.Hv * C * DK + (size_t)h * C * DK, DK, C, tid);
+  const int r0 = 16 * (w & 3);
   for (int j = 0; j < nch; ++j) {
     const size_t u = (size_t)(c0 + j) * p.Hv + h;
     const int start = cs + C * j, len = min(C, Lseq - C * j);
-    load_tile<C, DK>(Ws, L::LW, p.W + u * C * DK, DK, C, 1.f, tid);
-    load_tile<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, 1.f, tid);
-    load_tile<C, SL>(Us, L::LU, p.Ut + u * C * DV + v0, DV, C, 1.f, tid);
-    if (tid < C) sG[tid] = p.G[u * C + tid];
-    store_tile<SL, DK>(p.S0 + (u * DV + v0) * DK, DK, S, L::LS, tid);
+    tile_async<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, tid);
+    tile_async<C, SL>(Us, L::LU, p.Ut + u * C * DV + v0, DV, C, tid);
+    tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+    cp_commit();
+    cp_wait<0>();
     __syncthreads();
+    store_tile<SL, DK>(p.S0 + (u * DV + v0) * DK, DK, S, L::LS, tid);
     if (tid < C) sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
-    {  // U = U~ - W S^T: rows 16 (w & 3), state rows 16 (w >> 2)
-      const int r0 = 16 * (w & 3), vb = 16 * (w >> 2);
-      float acc[2][4];
+    {  // U = U~ - W S^T: token rows 16 (w & 3), state rows 32 (w >> 2)
+      const int vb = 32 * (w >> 2);
+      float acc[4][4];
       zero_acc(acc);
       mma3_rows<DK / 8>(acc, [&](int r, int c) { return Ws[(r0 + r) * L::LW + c]; },
                         [&](int r, int c) { return S[(vb + c) * L::LS + r]; }, lane);
@@ -356,13 +397,16 @@ __global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
       });
     }
     __syncthreads();
-    if (j + 1 < nch) {  // S <- gamma_C S + U^T diag(kdec) K: state rows 16 (w & 1), columns DK / 4 (w >> 1)
+    if (j + 1 < nch) {
+      tile_async<C, DK>(Ws, L::LW, p.W + (u + p.Hv) * C * DK, DK, C, tid);  // next chunk's W
+      cp_commit();
+      // S <- gamma_C S + U^T diag(kdec) K: state rows 16 (w & 3), columns DK / 2 (w >> 2)
       const float gC = expf((float)sG[len - 1]);
-      const int r0 = 16 * (w & 1), kb = (w >> 1) * (DK / 4);
-      float acc[DK / 32][4];
+      const int kb = (w >> 2) * (DK / 2);
+      float acc[DK / 16][4];
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * S[r * L::LS + c]; });
       mma3_rows<C / 8>(acc, [&](int r, int c) { return Us[c * L::LU + r0 + r] * sKd[c]; },
-                       [&](int r, int c) { return Ks[r * L::LK + kb + c]; }, lane);
+                       [&](int r, int c) { return to_f32(Ks[r * L::LK + kb + c]); }, lane);
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { S[r * L::LS + c] = x; });
       __syncthreads();
     }
@@ -370,23 +414,26 @@ __global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
 }
 
 // ---- reverse chain: dS1 and dU of every chunk, last to first ------------------
-template <int DK, int DV>
+template <typename TI, int DK, int DV>
 struct RevSmem {
-  static constexpr int LS = DK + 4, LK = DK + 4, LQ = DK + 8, LW = DK + 8, LO = SL + 8;
-  static constexpr int OS = 0, OP = OS + SL * LS, OO = OP + C * LD64, OK = OO + C * LO,
-                       OQ = OK + C * LK, OW = OQ + C * LQ, OU = OW + C * LW, OG = OU + C * LO,
-                       OGM = OG + 2 * C, OKD = OGM + C, FLOATS = OKD + C;
-  static constexpr size_t BYTES = FLOATS * sizeof(float);
+  static constexpr int LS = DK + 4, LK = in_ld<TI>(DK), LW = DK + 8, LO = SL + 8;
+  static constexpr size_t OS = 0, OP = OS + SL * LS * 4, OO = OP + C * LD64 * 4, OK = OO + C * LO * 4,
+                          OQ = OK + up16(C * LK * sizeof(TI)), OW = OQ + up16(C * LK * sizeof(TI)),
+                          OU = OW + C * LW * 4, OG = OU + C * LO * 4, OGM = OG + C * 8,
+                          BYTES = OGM + C * 4;
 };
 
 template <typename TI, int DK, int DV>
 __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
-  using L = RevSmem<DK, DV>;
-  extern __shared__ __align__(16) float sm[];
-  float *dS = sm + L::OS, *Ps = sm + L::OP, *dOs = sm + L::OO, *Ks = sm + L::OK, *Qs = sm + L::OQ,
-        *Ws = sm + L::OW, *dUs = sm + L::OU, *sGm = sm + L::OGM, *sKd = sm + L::OKD;
-  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  using L = RevSmem<TI, DK, DV>;
+  extern __shared__ __align__(16) unsigned char smb[];
+  float *dS = reinterpret_cast<float *>(smb + L::OS), *Ps = reinterpret_cast<float *>(smb + L::OP),
+        *dOs = reinterpret_cast<float *>(smb + L::OO), *Ws = reinterpret_cast<float *>(smb + L::OW),
+        *dUs = reinterpret_cast<float *>(smb + L::OU), *sGm = reinterpret_cast<float *>(smb + L::OGM);
+  TI *Ks = reinterpret_cast<TI *>(smb + L::OK), *Qs = reinterpret_cast<TI *>(smb + L::OQ);
+  double *sG = reinterpret_cast<double *>(smb + L::OG);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int gid = lane >> 2;
   const int kk = blockIdx.x;
   if (kk >= p.ph->n_nonempty) return;
   const int n = p.ne_seq[kk], c0 = p.ne_cs[kk], nch = p.ne_cs[kk + 1] - c0;
@@ -394,54 +441,69 @@ __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
   const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk), v0 = SL * blockIdx.z;
   const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
   const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;
-  if (p.dSf) load_tile<SL, DK>(dS, L::LS, p.dSf + srow * DK, DK, SL, 1.f, tid);
-  else for (int x = tid; x < SL * L::LS; x += NT) dS[x] = 0.f;
+  const size_t qstride = (size_t)p.Hqk * DK;
+  const float scale = p.scale;
+  if (p.dSf) tile_async<SL, DK>(dS, L::LS, p.dSf + srow * DK, DK, SL, tid);
+  else zero_tile<SL, DK>(dS, L::LS, tid);
+  {  // P and K of the last chunk (later ones are fetched one chunk ahead)
+    const size_t u = (size_t)(c0 + nch - 1) * p.Hv + h;
+    const int start = cs + C * (nch - 1), len = min(C, Lseq - C * (nch - 1));
+    tile_async<C, C>(Ps, LD64, p.P + u * C * C, C, C, tid);
+    tile_async<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
+  }
+  const int r0 = 16 * (w & 3);
   for (int j = nch - 1; j >= 0; --j) {
     const size_t u = (size_t)(c0 + j) * p.Hv + h;
     const int start = cs + C * j, len = min(C, Lseq - C * j);
-    load_tile<C, C>(Ps, LD64, p.P + u * C * C, C, C, 1.f, tid);
-    load_tile<C, SL>(dOs, L::LO, p.dO + ((size_t)start * p.Hv + h) * DV + v0, (size_t)p.Hv * DV, len,
-                     p.scale, tid);
-    load_tile<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, 1.f, tid);
-    load_tile<C, DK>(Qs, L::LQ, q + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, 1.f, tid);
-    load_tile<C, DK>(Ws, L::LW, p.W + u * C * DK, DK, C, 1.f, tid);
-    if (tid < C) sG[tid] = p.G[u * C + tid];
+    tile_async<C, SL>(dOs, L::LO, p.dO + ((size_t)start * p.Hv + h) * DV + v0, (size_t)p.Hv * DV, len, tid);
+    tile_async<C, DK>(Qs, L::LK, q + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
+    tile_async<C, DK>(Ws, L::LW, p.W + u * C * DK, DK, C, tid);
+    tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+    cp_commit();
+    cp_wait<0>();
+    __syncthreads();
     store_tile<SL, DK>(p.dS1 + (u * DV + v0) * DK, DK, dS, L::LS, tid);
-    __syncthreads();
-    if (tid < C) {
-      sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
-      sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
-    }
-    __syncthreads();
-    {  // dU = P^T dO' + diag(kdec) K dS^T: rows 16 (w & 3), state rows 16 (w >> 2)
-      const int r0 = 16 * (w & 3), vb = 16 * (w >> 2);
-      float a1[2][4], a2[2][4];
+    if (tid < C) sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
+    {  // dU = P^T dO' + diag(kdec) K dS^T: token rows 16 (w & 3), state rows 32 (w >> 2)
+      const int vb = 32 * (w >> 2);
+      float a1[4][4], a2[4][4];
       zero_acc(a1);
       zero_acc(a2);
       mma3_rows<C / 8>(a1, [&](int r, int c) { return Ps[c * LD64 + r0 + r]; },
                        [&](int r, int c) { return dOs[r * L::LO + vb + c]; }, lane);
-      mma3_rows<DK / 8>(a2, [&](int r, int c) { return Ks[(r0 + r) * L::LK + c]; },
+      mma3_rows<DK / 8>(a2, [&](int r, int c) { return to_f32(Ks[(r0 + r) * L::LK + c]); },
                         [&](int r, int c) { return dS[(vb + c) * L::LS + r]; }, lane);
+      const double Gl = sG[len - 1];
+      const int i0 = r0 + gid, i1 = i0 + 8;
+      const float kd0 = i0 < len ? expf((float)(Gl - sG[i0])) : 0.f;
+      const float kd1 = i1 < len ? expf((float)(Gl - sG[i1])) : 0.f;
       float *dUg = p.dU + u * C * DV + v0;
-      const int gid = lane >> 2, tig = lane & 3;
+      const int tig = lane & 3;
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+      for (int t = 0; t < 4; ++t)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = r0 + gid + 8 * (e >> 1), c = vb + 8 * t + 2 * tig + (e & 1);
-          const float x = a1[t][e] + sKd[i] * a2[t][e];
+          const float x = scale * a1[t][e] + (e < 2 ? kd0 : kd1) * a2[t][e];
           dUs[i * L::LO + c] = x;
           dUg[i * DV + c] = x;
         }
     }
     __syncthreads();
-    {  // dS <- gamma_C dS + dO'^T diag(gamma) Q - dU^T W: state rows 16 (w & 1), columns DK / 4 (w >> 1)
+    if (j > 0) {  // the previous chunk's P and K into the freed buffers
+      const size_t up = u - p.Hv;
+      const int sp = start - C;
+      tile_async<C, C>(Ps, LD64, p.P + up * C * C, C, C, tid);
+      tile_async<C, DK>(Ks, L::LK, k + ((size_t)sp * p.Hqk + hk) * DK, qstride, C, tid);
+      cp_commit();
+    }
+    {  // dS <- gamma_C dS + dO'^T diag(gamma) Q - dU^T W: state rows 16 (w & 3), columns DK / 2 (w >> 2)
       const float gC = expf((float)sG[len - 1]);
-      const int r0 = 16 * (w & 1), kb = (w >> 1) * (DK / 4);
-      float acc[DK / 32][4];
+      const int kb = (w >> 2) * (DK / 2);
+      float acc[DK / 16][4];
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * dS[r * L::LS + c]; });
-      mma3_rows<C / 8>(acc, [&](int r, int c) { return dOs[c * L::LO + r0 + r] * sGm[c]; },
-                       [&](int r, int c) { return Qs[r * L::LQ + kb + c]; }, lane);
+      mma3_rows<C / 8>(acc, [&](int r, int c) { return scale * dOs[c * L::LO + r0 + r] * sGm[c]; },
+                       [&](int r, int c) { return to_f32(Qs[r * L::LK + kb + c]); }, lane);
       mma3_rows<C / 8>(acc, [&](int r, int c) { return -dUs[c * L::LO + r0 + r]; },
                        [&](int r, int c) { return Ws[r * L::LW + kb + c]; }, lane);
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { dS[r * L::LS + c] = x; });
@@ -455,17 +517,19 @@ __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
 template <int DK, int DV>
 struct StateGradSmem {
   static constexpr int LS = DK + 8, LM = DV + 4;
-  static constexpr int OS0 = 0, OS1 = OS0 + DV * LS, OM = OS1 + DV * LS, OG = OM + C * LM,
-                       OR = OG + 2 * C, FLOATS = OR + 4 * C + 8;
-  static constexpr size_t BYTES = FLOATS * sizeof(float);
+  static constexpr size_t OS0 = 0, OS1 = OS0 + DV * LS * 4, OM1 = OS1 + DV * LS * 4,
+                          OM2 = OM1 + C * LM * 4, OG = OM2 + C * LM * 4, OR = OG + C * 8,
+                          BYTES = OR + (4 * C + 8) * 4;
 };
 
 template <typename TI, int DK, int DV>
 __global__ void __launch_bounds__(NT) grads_state_kernel(const Params p) {
   using L = StateGradSmem<DK, DV>;
-  extern __shared__ __align__(16) float sm[];
-  float *S0s = sm + L::OS0, *S1s = sm + L::OS1, *Ms = sm + L::OM, *red = sm + L::OR;
-  double *sG = reinterpret_cast<double *>(sm + L::OG);
+  extern __shared__ __align__(16) unsigned char smb[];
+  float *S0s = reinterpret_cast<float *>(smb + L::OS0), *S1s = reinterpret_cast<float *>(smb + L::OS1),
+        *M1 = reinterpret_cast<float *>(smb + L::OM1), *M2 = reinterpret_cast<float *>(smb + L::OM2),
+        *red = reinterpret_cast<float *>(smb + L::OR);
+  double *sG = reinterpret_cast<double *>(smb + L::OG);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   ChunkPos cp;
   if (!chunk_pos(p, blockIdx.x, cp)) return;
@@ -474,13 +538,46 @@ __global__ void __launch_bounds__(NT) grads_state_kernel(const Params p) {
   const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
   const TI *qc = q + ((size_t)cp.start * p.Hqk + hk) * DK, *kc = k + ((size_t)cp.start * p.Hqk + hk) * DK;
   const size_t qstride = (size_t)p.Hqk * DK;
-  load_tile<DV, DK>(S0s, L::LS, p.S0 + u * DV * DK, DK, DV, 1.f, tid);
-  load_tile<DV, DK>(S1s, L::LS, p.dS1 + u * DV * DK, DK, DV, 1.f, tid);
-  load_tile<C, DV>(Ms, L::LM, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, cp.len,
-                   p.scale, tid);
-  if (tid < C) sG[tid] = p.G[u * C + tid];
-  __syncthreads();
   const int len = cp.len;
+  tile_async<DV, DK>(S0s, L::LS, p.S0 + u * DV * DK, DK, DV, tid);
+  tile_async<C, DV>(M1, L::LM, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
+  tile_async<C, DV>(M2, L::LM, p.dU + u * C * DV, DV, C, tid);
+  tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+  cp_commit();
+  tile_async<DV, DK>(S1s, L::LS, p.dS1 + u * DV * DK, DK, DV, tid);
+  cp_commit();
+  cp_wait<1>();
+  __syncthreads();
+  const int r0 = 16 * (w & 3), cb = (w >> 2) * (DK / 2), half = w >> 2;
+  const int gid = lane >> 2, tig = lane & 3;
+  const float scale = p.scale;
+  float acc[DK / 16][4];
+  // dO S0: dQ part diag(gamma) dO' S0 and dgamma_t = q_t . (dO' S0)_t
+  zero_acc(acc);
+  mma3_rows<DV / 8>(acc, [&](int r, int c) { return M1[(r0 + r) * L::LM + c]; },
+                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
+  {
+    float slo, shi;
+    quad_row_sums(acc, [&](int i, int c) { return i < len ? to_f32(qc[(size_t)i * qstride + c]) : 0.f; },
+                  r0, cb, lane, slo, shi);
+    if (tig == 0) { red[half * C + r0 + gid] = scale * slo; red[half * C + r0 + gid + 8] = scale * shi; }
+    float *dQp = p.dQp + u * C * DK;
+    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) {
+      dQp[i * DK + c] = i < len ? scale * expf((float)sG[i]) * x : 0.f;
+    });
+  }
+  zero_acc(acc);  // dW = -dU S0
+  mma3_rows<DV / 8>(acc, [&](int r, int c) { return M2[(r0 + r) * L::LM + c]; },
+                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
+  {
+    float *dW = p.dW + u * C * DK;
+    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) { dW[i * DK + c] = -x; });
+  }
+  __syncthreads();
+  tile_async<C, DV>(M1, L::LM, p.U + u * C * DV, DV, C, tid);
+  cp_commit();
+  cp_wait<0>();
+  __syncthreads();
   {  // <dS1, S0>: fixed-order partials per thread, then per warp, then over warps
     float s = 0.f;
     for (int x = tid; x < DV * DK; x += NT) {
@@ -491,38 +588,8 @@ __global__ void __launch_bounds__(NT) grads_state_kernel(const Params p) {
     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
     if (lane == 0) red[4 * C + w] = s;
   }
-  const int r0 = 16 * (w & 3), cb = (w >> 2) * (DK / 2), half = w >> 2;
-  const int gid = lane >> 2, tig = lane & 3;
-  float acc[DK / 16][4];
-  // dO' S0: dQ part diag(gamma) dO' S0 and dgamma_t = q_t . (dO' S0)_t
-  zero_acc(acc);
-  mma3_rows<DV / 8>(acc, [&](int r, int c) { return Ms[(r0 + r) * L::LM + c]; },
-                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
-  {
-    float slo, shi;
-    quad_row_sums(acc, [&](int i, int c) { return i < len ? to_f32(qc[(size_t)i * qstride + c]) : 0.f; },
-                  r0, cb, lane, slo, shi);
-    if (tig == 0) { red[half * C + r0 + gid] = slo; red[half * C + r0 + gid + 8] = shi; }
-    float *dQp = p.dQp + u * C * DK;
-    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) {
-      dQp[i * DK + c] = i < len ? expf((float)sG[i]) * x : 0.f;
-    });
-  }
-  __syncthreads();
-  load_tile<C, DV>(Ms, L::LM, p.dU + u * C * DV, DV, C, 1.f, tid);
-  __syncthreads();
-  zero_acc(acc);  // dW = -dU S0
-  mma3_rows<DV / 8>(acc, [&](int r, int c) { return Ms[(r0 + r) * L::LM + c]; },
-                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
-  {
-    float *dW = p.dW + u * C * DK;
-    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) { dW[i * DK + c] = -x; });
-  }
-  __syncthreads();
-  load_tile<C, DV>(Ms, L::LM, p.U + u * C * DV, DV, C, 1.f, tid);
-  __syncthreads();
   zero_acc(acc);  // U dS1: dK part diag(kdec) U dS1 and dkdec_t = k_t . (U dS1)_t
-  mma3_rows<DV / 8>(acc, [&](int r, int c) { return Ms[(r0 + r) * L::LM + c]; },
+  mma3_rows<DV / 8>(acc, [&](int r, int c) { return M1[(r0 + r) * L::LM + c]; },
                     [&](int r, int c) { return S1s[r * L::LS + cb + c]; }, lane);
   {
     float slo, shi;
@@ -549,30 +616,34 @@ __global__ void __launch_bounds__(NT) grads_state_kernel(const Params p) {
 }
 
 // ---- the 64 x 64 algebra of one (chunk, value head), and its outputs -----------
-template <int DK, int DV>
+template <typename TI, int DK, int DV>
 struct LocalSmem {
-  static constexpr int LA = (DK > DV ? DK : DV) + 4;  // dO', then dW
-  static constexpr int LB = DV + 4;                   // U, then dU
-  static constexpr int LC = DK + 4;                   // K
-  static constexpr int LD = (DK > DV ? DK : DV) + 4;  // V, then Q
-  static constexpr int OA = 0, OB = OA + C * LA, OC = OB + C * LB, OD = OC + C * LC,
-                       O1 = OD + C * LD, O2 = O1 + C * LD64, O3 = O2 + C * LD64, O4 = O3 + C * LD64,
-                       O5 = O4 + C * LD64, OV = O5 + C * LD64, NVEC = 13, FLOATS = OV + NVEC * C;
-  static constexpr size_t BYTES = FLOATS * sizeof(float);
+  static constexpr int DM = DK > DV ? DK : DV;
+  static constexpr int LA = DM + 4;           // dO, then dW (fp32)
+  static constexpr int LB = DV + 4;           // U, then dU (fp32)
+  static constexpr int LC = in_ld<TI>(DK);    // K
+  static constexpr int LD = in_ld<TI>(DM);    // V, then Q
+  static constexpr size_t OA = 0, OB = OA + C * LA * 4, OC = OB + C * LB * 4,
+                          OD = OC + up16(C * LC * sizeof(TI)), O1 = OD + up16(C * LD * sizeof(TI)),
+                          O2 = O1 + C * LD64 * 4, O3 = O2 + C * LD64 * 4, O4 = O3 + C * LD64 * 4,
+                          O5 = O4 + C * LD64 * 4, OG = O5 + C * LD64 * 4, OV = OG + C * 8,
+                          NVEC = 11, BYTES = OV + NVEC * C * 4;
 };
 
 template <typename TI, int DK, int DV>
 __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
-  using L = LocalSmem<DK, DV>;
-  extern __shared__ __align__(16) float sm[];
-  float *RA = sm + L::OA, *RB = sm + L::OB, *RC = sm + L::OC, *RD = sm + L::OD;
-  float *S1 = sm + L::O1, *S2 = sm + L::O2, *S3 = sm + L::O3, *S4 = sm + L::O4, *S5 = sm + L::O5;
-  float *vec = sm + L::OV;
-  // per-row vectors: G (fp64), beta, gamma, kdec, xk (2 halves), yv (2 halves), rP, cP, rM, cM
-  double *sG = reinterpret_cast<double *>(vec);
-  float *sB = vec + 2 * C, *sGm = vec + 3 * C, *sKd = vec + 4 * C, *sXK = vec + 5 * C,
-        *sYV = vec + 7 * C, *sRP = vec + 9 * C, *sCP = vec + 10 * C, *sRM = vec + 11 * C,
-        *sCM = vec + 12 * C;
+  using L = LocalSmem<TI, DK, DV>;
+  extern __shared__ __align__(16) unsigned char smb[];
+  float *RA = reinterpret_cast<float *>(smb + L::OA), *RB = reinterpret_cast<float *>(smb + L::OB);
+  TI *RC = reinterpret_cast<TI *>(smb + L::OC), *RD = reinterpret_cast<TI *>(smb + L::OD);
+  float *S1 = reinterpret_cast<float *>(smb + L::O1), *S2 = reinterpret_cast<float *>(smb + L::O2),
+        *S3 = reinterpret_cast<float *>(smb + L::O3), *S4 = reinterpret_cast<float *>(smb + L::O4),
+        *S5 = reinterpret_cast<float *>(smb + L::O5);
+  double *sG = reinterpret_cast<double *>(smb + L::OG);
+  float *vec = reinterpret_cast<float *>(smb + L::OV);
+  // per-row vectors: beta, gamma, kdec, xk (2 halves), yv (2 halves), rP, cP, rM, cM
+  float *sB = vec, *sGm = vec + C, *sKd = vec + 2 * C, *sXK = vec + 3 * C, *sYV = vec + 5 * C,
+        *sRP = vec + 7 * C, *sCP = vec + 8 * C, *sRM = vec + 9 * C, *sCM = vec + 10 * C;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int gid = lane >> 2, tig = lane & 3;
   ChunkPos cp;
@@ -583,47 +654,49 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k),
            *v = static_cast<const TI *>(p.v);
   const size_t qoff = ((size_t)cp.start * p.Hqk + hk) * DK, qstride = (size_t)p.Hqk * DK;
-  // step 1: dP = lower(dO' U^T); S2 = dP . E, S1 = dP . P
-  load_tile<C, DV>(RA, L::LA, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len,
-                   p.scale, tid);
-  load_tile<C, DV>(RB, L::LB, p.U + u * C * DV, DV, C, 1.f, tid);
-  load_tile<C, C>(S1, LD64, p.P + u * C * C, C, C, 1.f, tid);
-  if (tid < C) {
-    sG[tid] = p.G[u * C + tid];
-    sB[tid] = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
-  }
+  const float scale = p.scale;
+  tile_async<C, DV>(RA, L::LA, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
+  tile_async<C, DV>(RB, L::LB, p.U + u * C * DV, DV, C, tid);
+  tile_async<C, C>(S1, LD64, p.P + u * C * C, C, C, tid);
+  tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+  cp_commit();
+  tile_async<C, DK>(RC, L::LC, k + qoff, qstride, len, tid);
+  tile_async<C, DV>(RD, L::LD, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
+  tile_async<C, C>(S3, LD64, p.Tm + u * C * C, C, C, tid);
+  cp_commit();
+  if (tid < C) sB[tid] = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
+  cp_wait<1>();
   __syncthreads();
   if (tid < C) {
     sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
     sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
   }
   const int r0 = 16 * (w & 3), half = w >> 2, c64 = 32 * half;
-  {
+  {  // step 1: dP = lower(dO' U^T); S2 = dP . E, S1 = dP . P
     float acc[4][4];
     zero_acc(acc);
     mma3_rows<DV / 8>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
                       [&](int r, int c) { return RB[(c64 + c) * L::LB + r]; }, lane);
     for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) {
-      const float dp = i >= j ? x : 0.f;
+      const float dp = i >= j ? scale * x : 0.f;
       S2[i * LD64 + j] = i >= j ? dp * expf((float)(sG[i] - sG[j])) : 0.f;
       S1[i * LD64 + j] = dp * S1[i * LD64 + j];
     });
   }
   __syncthreads();
-  // step 2: dT, X = Tm^T dW (dK part, x.k), Y = Tm^T dU (dv, y.v)
-  load_tile<C, DK>(RA, L::LA, p.dW + u * C * DK, DK, C, 1.f, tid);
-  load_tile<C, DV>(RB, L::LB, p.dU + u * C * DV, DV, C, 1.f, tid);
-  load_tile<C, DK>(RC, L::LC, k + qoff, qstride, len, 1.f, tid);
-  load_tile<C, DV>(RD, L::LD, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, 1.f, tid);
-  load_tile<C, C>(S3, LD64, p.Tm + u * C * C, C, C, 1.f, tid);
+  tile_async<C, DK>(RA, L::LA, p.dW + u * C * DK, DK, C, tid);
+  tile_async<C, DV>(RB, L::LB, p.dU + u * C * DV, DV, C, tid);
+  cp_commit();
+  cp_wait<0>();
   __syncthreads();
-  {  // dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T
+  {  // step 2: dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T -> S4
     float acc[4][4];
     zero_acc(acc);
     mma3_rows<DK / 8>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
-                      [&](int r, int c) { return sB[c64 + c] * sGm[c64 + c] * RC[(c64 + c) * L::LC + r]; }, lane);
+                      [&](int r, int c) { return sB[c64 + c] * sGm[c64 + c] * to_f32(RC[(c64 + c) * L::LC + r]); },
+                      lane);
     mma3_rows<DV / 8>(acc, [&](int r, int c) { return RB[(r0 + r) * L::LB + c]; },
-                      [&](int r, int c) { return sB[c64 + c] * RD[(c64 + c) * L::LD + r]; }, lane);
+                      [&](int r, int c) { return sB[c64 + c] * to_f32(RD[(c64 + c) * L::LD + r]); }, lane);
     for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = x; });
   }
   const int cbk = half * (DK / 2), cbv = half * (DV / 2);
@@ -633,7 +706,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     mma3_rows<C / 8>(dK, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
                      [&](int r, int c) { return RA[r * L::LA + cbk + c]; }, lane);
     float slo, shi;
-    quad_row_sums(dK, [&](int i, int c) { return RC[i * L::LC + c]; }, r0, cbk, lane, slo, shi);
+    quad_row_sums(dK, [&](int i, int c) { return to_f32(RC[i * L::LC + c]); }, r0, cbk, lane, slo, shi);
     if (tig == 0) { sXK[half * C + r0 + gid] = slo; sXK[half * C + r0 + gid + 8] = shi; }
     for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x *= sB[i] * sGm[i]; });
   }
@@ -643,7 +716,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     mma3_rows<C / 8>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
                      [&](int r, int c) { return RB[r * L::LB + cbv + c]; }, lane);
     float slo, shi;
-    quad_row_sums(acc, [&](int i, int c) { return RD[i * L::LD + c]; }, r0, cbv, lane, slo, shi);
+    quad_row_sums(acc, [&](int i, int c) { return to_f32(RD[i * L::LD + c]); }, r0, cbv, lane, slo, shi);
     if (tig == 0) { sYV[half * C + r0 + gid] = slo; sYV[half * C + r0 + gid + 8] = shi; }
     float *dv = p.dv + ((size_t)cp.start * p.Hv + h) * DV;
     for_frag(acc, r0, cbv, lane, [&](int i, int c, float &x) {
@@ -651,6 +724,8 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     });
   }
   __syncthreads();
+  tile_async<C, DK>(RD, L::LD, q + qoff, qstride, len, tid);  // V is no longer needed
+  cp_commit();
   {  // Z = dT Tm^T -> S5
     float acc[4][4];
     zero_acc(acc);
@@ -667,8 +742,9 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = i > j ? -x : 0.f; });
   }
   __syncthreads();
-  load_tile<C, C>(S5, LD64, p.EKK + u * C * C, C, C, 1.f, tid);
-  load_tile<C, DK>(RD, L::LD, q + qoff, qstride, len, 1.f, tid);
+  tile_async<C, C>(S5, LD64, p.EKK + u * C * C, C, C, tid);
+  cp_commit();
+  cp_wait<0>();
   __syncthreads();
   // S4 <- B = diag(beta) (dA . E); S5 <- dA . (E . K K^T)
   for (int x = tid; x < C * C; x += NT) {
@@ -695,7 +771,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     const float *dQp = p.dQp + u * C * DK;
     for_frag(acc, r0, cbk, lane, [&](int i, int c, float &x) { x = dQp[i * DK + c]; });
     mma3_rows<C / 8>(acc, [&](int r, int c) { return S2[(r0 + r) * LD64 + c]; },
-                     [&](int r, int c) { return RC[r * L::LC + cbk + c]; }, lane);
+                     [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
     const bool direct = Gq == 1;
     float *dst = direct ? p.dq + qoff : p.dq + ((size_t)cp.start * p.Hv + h) * DK;
     const size_t rs = direct ? qstride : (size_t)p.Hv * DK;
@@ -707,9 +783,9 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     const float *dKp = p.dKp + u * C * DK;
     for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x += dKp[i * DK + c]; });
     mma3_rows<C / 8>(dK, [&](int r, int c) { return S2[c * LD64 + r0 + r]; },
-                     [&](int r, int c) { return RD[r * L::LD + cbk + c]; }, lane);
+                     [&](int r, int c) { return to_f32(RD[r * L::LD + cbk + c]); }, lane);
     mma3_rows<C / 8>(dK, [&](int r, int c) { return S4[(r0 + r) * LD64 + c] + S4[c * LD64 + r0 + r]; },
-                     [&](int r, int c) { return RC[r * L::LC + cbk + c]; }, lane);
+                     [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
     const bool direct = Gq == 1;
     float *dst = direct ? p.dk + qoff : p.dk + ((size_t)cp.start * p.Hv + h) * DK;
     const size_t rs = direct ? qstride : (size_t)p.Hv * DK;
@@ -744,8 +820,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
       const float x = __shfl_down_sync(0xffffffffu, s, off);
       if (lane + off < 32) s += x;
     }
-    const float suf1 = s - dG[0], suf0 = s;  // suffix from token 2 lane + 1, from 2 lane
-    const float sf[2] = {suf0, suf1};
+    const float sf[2] = {s, s - dG[0]};  // suffix from token 2 lane, from 2 lane + 1
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int i = 2 * lane + e;
@@ -814,11 +889,11 @@ cudaError_t run_chunked(const cbwd::Params &prm, int64_t chunks, cudaStream_t st
   using namespace cbwd;
   const dim3 per_chunk((unsigned)chunks, (unsigned)prm.Hv), per_seq((unsigned)prm.N, (unsigned)prm.Hv, DV / SL);
   cudaError_t e;
-  if ((e = launch_k(prep_kernel<TI, DK, DV>, per_chunk, PrepSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
-  if ((e = launch_k(fwd_chain_kernel<TI, DK, DV>, per_seq, FwdSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
-  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  if ((e = launch_k(prep_kernel<TI, DK, DV>, per_chunk, PrepSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  if ((e = launch_k(fwd_chain_kernel<TI, DK, DV>, per_seq, FwdSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
   if ((e = launch_k(grads_state_kernel<TI, DK, DV>, per_chunk, StateGradSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
-  return launch_k(grads_local_kernel<TI, DK, DV>, per_chunk, LocalSmem<DK, DV>::BYTES, prm, stream);
+  return launch_k(grads_local_kernel<TI, DK, DV>, per_chunk, LocalSmem<TI, DK, DV>::BYTES, prm, stream);
 }
 
 template <typename TI>

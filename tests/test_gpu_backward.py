@@ -116,3 +116,41 @@ def test_backward_many_units_one_slice(Hqk, Hv, N, algo):
     lengths = [(7 * i) % 23 for i in range(N)]  # 0 .. 22 tokens, some empty
     out, ref = _case(lengths, Hqk, Hv, 64, "fp32", seed=109 + Hv, algo=algo)
     _check(out, ref, f"{algo} {N} sequences x {Hv} heads")
+
+
+@pytest.mark.slow
+def test_backward_prefill8k_all_heads():
+    """The bench's backward workload at full size (8192 tokens, 16/48 heads,
+    D=128, bf16 inputs) with an initial state and dL/dS_final, chunk form,
+    every gradient element of every head against the oracle.  The oracle runs
+    one query/key head (its 3 value heads) per call, calls in threads."""
+    from concurrent.futures import ThreadPoolExecutor
+    import os
+
+    w = inputs.WORKLOADS["prefill8k"]
+    inp = inputs.prefill_inputs(w.lengths, w.Hqk, w.Hv, w.D, dtype=w.dtype, seed=w.seed, init_std=0.02)
+    T, G = sum(w.lengths), w.Hv // w.Hqk
+    gen = torch.Generator().manual_seed(131)
+    d_o = torch.randn(T, w.Hv, w.D, generator=gen)
+    d_sf = torch.randn(1, w.Hv, w.D, w.D, generator=gen) * 0.1
+    dev = {n: t.to(DEV) for n, t in inp.items() if t is not None}
+    out = api.prefill_backward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], d_o.to(DEV),
+                               cu_seqlens=dev["cu_seqlens"], initial_state=dev["initial_state"],
+                               d_final_state=d_sf.to(DEV))
+    torch.cuda.synchronize()
+
+    def ref(hk):
+        qs, vs = slice(hk, hk + 1), slice(G * hk, G * hk + G)
+        return hk, oracle.backward(inp["q"][:, qs], inp["k"][:, qs], inp["v"][:, vs], inp["g"][:, vs],
+                                   inp["beta"][:, vs], d_o[:, vs], cu_seqlens=inp["cu_seqlens"],
+                                   initial_state=inp["initial_state"][:, vs], d_final_state=d_sf[:, vs])
+
+    workers = max(1, min(8, (os.cpu_count() or 1)))
+    with ThreadPoolExecutor(workers) as ex:
+        results = list(ex.map(ref, range(w.Hqk)))
+    full = [np.zeros(tuple(t.shape)) for t in out]
+    for hk, r in results:
+        qs, vs = slice(hk, hk + 1), slice(G * hk, G * hk + G)
+        full[0][:, qs], full[1][:, qs], full[2][:, vs] = r[0], r[1], r[2]
+        full[3][:, vs], full[4][:, vs], full[5][:, vs] = r[3], r[4], r[5]
+    _check(out, full, "prefill8k all heads")

@@ -74,6 +74,9 @@ def parse_args(argv=None):
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--decode-steps", type=int, default=1000)
     p.add_argument("--no-backward", action="store_true", help="skip the backward-pass leg")
+    p.add_argument("--backward-tokens", type=int, default=0,
+                   help="run the backward leg on the first N tokens of the workload (small "
+                        "profiling captures); 0 = all")
     p.add_argument("--no-long", action="store_true",
                    help="skip the long262k and varlen32 prefill legs (~20 GB of device memory)")
     p.add_argument("--no-decode", action="store_true")
@@ -722,6 +725,10 @@ def _backward(args, D, dev, x, T, w, peaks):
 
     from gated_deltanet_recurrence_rule_b200 import api
 
+    if 0 < args.backward_tokens < T:
+        T = args.backward_tokens
+        x = {n: (t[:T] if n in ("q", "k", "v", "g", "beta") else t) for n, t in x.items()}
+        x["cu_seqlens"] = torch.tensor([0, T], dtype=torch.int32, device=dev)
     gen = torch.Generator(device=dev).manual_seed(12)
     d_o = torch.randn((T, w.Hv, w.D), generator=gen, device=dev)
     d_sf = torch.randn((1, w.Hv, w.D, w.D), generator=gen, device=dev) * 0.1

@@ -44,12 +44,13 @@
 //   group sums   dq, dk over the value heads of each query/key head
 // Rows of S and of dS evolve independently (the chains never mix rows), so
 // each chain CTA owns 64 of the Dv rows.  Tiles move global -> shared with
-// cp.async, all of a step's copies in flight at once, and the chains fetch
-// a chunk's tiles while the previous chunk computes where buffers allow.  Every product runs on warp-level
-// m16n8k8 tf32 tensor-core MMAs with both operands split into hi (x with the
-// low 13 mantissa bits cleared) and lo = x - hi, and three products (hi*hi +
-// hi*lo + lo*hi), which keeps about fp32 accuracy.  Per-row sums go through fixed-order partials,
-// so results do not depend on scheduling.
+// cp.async, all of a step's copies in flight at once, and the chains fetch a
+// chunk's tiles while the previous chunk computes where buffers allow.
+// Every product runs on warp-level m16n8k8 tf32 tensor-core MMAs with both
+// operands split into hi (x with the low 13 mantissa bits cleared) and
+// lo = x - hi, and three products (hi*hi + hi*lo + lo*hi), which keeps about
+// fp32 accuracy.  Per-row sums go through fixed-order partials, so results do
+// not depend on scheduling.
 #include <algorithm>
 
 #include "gdn_chunk_ops.cuh"

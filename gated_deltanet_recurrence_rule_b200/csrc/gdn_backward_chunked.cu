@@ -29,7 +29,8 @@
 //   dg_s = sum_{t >= s} dG_t within the chunk.
 // dq and dk of a query/key head sum over the value heads that read it.
 //
-// Launches (one stream):
+// Launches (the two chains on the caller stream's internal pair, beside each
+// other; the rest on the caller's stream):
 //   plan         validates cu_seqlens, lists the non-empty sequences and
 //                their first chunk; d_initial_state of an empty sequence is
 //                d_final_state (or zero)
@@ -64,6 +65,8 @@ cudaError_t launch_plan(const int32_t *cu, int N, int T, int Hv, const void *s0,
                         int32_t *status, cudaStream_t stream);
 cudaError_t launch_group_sum(const float *part, float *out, size_t rows, int width, int inner,
                              cudaStream_t stream);
+cudaError_t internal_streams_fork(cudaStream_t caller, cudaStream_t *lo, cudaStream_t *hi);
+cudaError_t internal_streams_join(cudaStream_t caller);
 
 namespace cbwd {
 
@@ -92,6 +95,7 @@ struct Params {
   double *G;                // [u][64] prefix sums of the clamped log-decays (fp64: differences
                             // of large sums stay exact when gates are near zero)
   float *sc;                // [u][3][64]: dgamma (from S0), dkdec, dgamma_C at [2][0]
+  int32_t *status;          // workspace header: status word, then the wait limit
 };
 
 // ---- tensor-core building block -------------------------------------------
@@ -514,94 +518,282 @@ __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
   if (p.ds0) store_tile<SL, DK>(p.ds0 + srow * DK, DK, dS, L::LS, tid);
 }
 
-// ---- products with S0 and dS1 of one (chunk, value head) ----------------------
+// ---- tcgen05 building blocks -----------------------------------------------
+// Operands of the 5th-generation tensor-core products are bf16 images in
+// shared memory, 128-byte swizzled, each fp32 value split into hi =
+// bf16(x) and lo = bf16(x - hi) (both rounded to nearest, |x - hi - lo| <=
+// 2^-18 |x|); a product is hi*hi' + hi*lo' + lo*hi' (3 MMAs per K step,
+// about 2^-16 relative), accumulated in fp32 in tensor memory.
+//   K-major image of an R x K operand (R = 128 rows): K blocks of 64 columns,
+//   R x 128 bytes each; element (r, k) at block k / 64, sw128_off(r, (k % 64) / 8).
+//   MN-major image of a K x N operand: N blocks of 64 columns, K x 128 bytes
+//   each; element (k, n) at block n / 64, sw128_off(k, (n % 64) / 8).
+// Both store 8 consecutive elements of a row as one 16-byte chunk.
+__device__ __forceinline__ void split8_bf16(const float *x, uint4 &hi, uint4 &lo) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(x[2 * e], x[2 * e + 1]);
+    const float2 hf = __bfloat1622float2(hb);
+    const __nv_bfloat162 lb = __floats2bfloat162_rn(x[2 * e] - hf.x, x[2 * e + 1] - hf.y);
+    h[e] = *reinterpret_cast<const uint32_t *>(&hb);
+    l[e] = *reinterpret_cast<const uint32_t *>(&lb);
+  }
+  hi = make_uint4(h[0], h[1], h[2], h[3]);
+  lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+// Store the split of x[0..8) as chunk `chunk` of row `row` of the images
+// whose blocks start at hi_base / lo_base (block already selected).
+__device__ __forceinline__ void st_img8(unsigned char *hi_base, unsigned char *lo_base, int row,
+                                        int chunk, const float *x) {
+  uint4 h, l;
+  split8_bf16(x, h, l);
+  const uint32_t off = sm100::sw128_off((uint32_t)row, (uint32_t)chunk);
+  *reinterpret_cast<uint4 *>(hi_base + off) = h;
+  *reinterpret_cast<uint4 *>(lo_base + off) = l;
+}
+// 8 consecutive fp32 values from global memory (16-byte aligned), or zeros.
+__device__ __forceinline__ void ld8(const float *src, bool ok, float *x) {
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f), b = a;
+  if (ok) {
+    a = *reinterpret_cast<const float4 *>(src);
+    b = *reinterpret_cast<const float4 *>(src + 4);
+  }
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+// 3-term product D (+)= A B over KSTEPS K steps of 16, A K-major (blocks of
+// 64 K at a_blk bytes), B MN-major (K rows of 128 bytes, N blocks at b_lbo).
+// Issued by one thread.
+template <int KSTEPS>
+__device__ __forceinline__ void umma3_kmaj_mn(uint32_t d_tmem, uint32_t a_hi, uint32_t a_lo,
+                                              uint32_t a_blk, uint32_t b_hi, uint32_t b_lo,
+                                              uint32_t b_lbo, uint32_t idesc, bool accumulate) {
+#pragma unroll
+  for (int ks = 0; ks < KSTEPS; ++ks) {
+    const uint32_t ao = (ks >> 2) * a_blk + (ks & 3) * 32, bo = ks * 2048;
+    const uint64_t ah = sm100::sdesc_sw128(a_hi + ao, 16, 1024), al = sm100::sdesc_sw128(a_lo + ao, 16, 1024);
+    const uint64_t bh = sm100::sdesc_sw128(b_hi + bo, b_lbo, 1024), bl = sm100::sdesc_sw128(b_lo + bo, b_lbo, 1024);
+    sm100::mma_bf16(d_tmem, al, bh, idesc, (accumulate || ks > 0) ? 1u : 0u);
+    sm100::mma_bf16(d_tmem, ah, bl, idesc, 1u);
+    sm100::mma_bf16(d_tmem, ah, bh, idesc, 1u);
+  }
+}
+// Every thread waits for an mbarrier phase (bounded); false when it gave up,
+// which is recorded in the status word.  No thread leaves early, so the
+// CTA-wide barriers that follow are reached by all.
+__device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, volatile int *ctl, int32_t *status) {
+  if (sm100::mbar_wait(bar, parity, ctl)) {
+    sm100::tc_fence_after();
+    return true;
+  }
+  ctl[0] = 1;
+  report_status(status, GDN_ERR_DEVICE_TIMEOUT);
+  return false;
+}
+
+// ---- products with S0 and dS1 of one (chunk, value head), on tcgen05 ----------
+// D1 = [dO; dU] S0 (M = 128: rows 0-63 the chunk's dO, rows 64-127 its dU),
+// then D2 = U dS1 (rows 0-63; rows 64-127 of that A image still hold dU and
+// are not read), both N = Dk, K = Dv, accumulators in tensor memory:
+//   dQ part  diag(scale gamma) (dO S0),  dgamma_t = scale q_t . (dO S0)_t
+//   dW       -(dU S0)
+//   dK part  diag(kdec) (U dS1),         dkdec_t = k_t . (U dS1)_t
+//   dgamma_C = <dS1, S0>
+// One thread issues the MMAs; all threads build the operand images and read
+// the results (warp w reads TMEM lanes 32 (w % 4) .. + 31 and one column half).
 template <int DK, int DV>
 struct StateGradSmem {
-  static constexpr int LS = DK + 8, LM = DV + 4;
-  static constexpr size_t OS0 = 0, OS1 = OS0 + DV * LS * 4, OM1 = OS1 + DV * LS * 4,
-                          OM2 = OM1 + C * LM * 4, OG = OM2 + C * LM * 4, OR = OG + C * 8,
-                          BYTES = OR + (4 * C + 8) * 4;
+  static constexpr uint32_t A_BLK = 128 * 128;            // one 64-column K block of a 128-row image
+  static constexpr uint32_t A_BYTES = (DV / 64) * A_BLK;  // [dO; dU], then U
+  static constexpr uint32_t B_LBO = DV * 128;             // one 64-column N block of the MN-major image
+  static constexpr uint32_t B_BYTES = (DK / 64) * B_LBO;  // S0, then dS1
+  static constexpr uint32_t OAH = 0, OAL = A_BYTES, OBH = 2 * A_BYTES, OBL = OBH + B_BYTES,
+                            OG = OBL + B_BYTES, ORED = OG + C * 8, OBAR = ORED + (4 * C + 8) * 4,
+                            OMISC = OBAR + 16, BYTES = OMISC + 32;
+  static constexpr uint32_t TMEM_COLS = 2 * DK;  // 128 or 256
 };
 
 template <typename TI, int DK, int DV>
-__global__ void __launch_bounds__(NT) grads_state_kernel(const Params p) {
+__global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
   using L = StateGradSmem<DK, DV>;
-  extern __shared__ __align__(16) unsigned char smb[];
-  float *S0s = reinterpret_cast<float *>(smb + L::OS0), *S1s = reinterpret_cast<float *>(smb + L::OS1),
-        *M1 = reinterpret_cast<float *>(smb + L::OM1), *M2 = reinterpret_cast<float *>(smb + L::OM2),
-        *red = reinterpret_cast<float *>(smb + L::OR);
-  double *sG = reinterpret_cast<double *>(smb + L::OG);
+  extern __shared__ __align__(1024) unsigned char smb[];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   ChunkPos cp;
   if (!chunk_pos(p, blockIdx.x, cp)) return;
+  const uint32_t sb = sm100::smem_addr(smb);
+  if (sb & 1023u) {  // swizzled operand images need 1024-byte alignment
+    if (tid == 0) report_status(p.status, GDN_ERR_UNSUPPORTED);
+    return;
+  }
   const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk);
   const size_t u = (size_t)blockIdx.x * p.Hv + h;
-  const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
-  const TI *qc = q + ((size_t)cp.start * p.Hqk + hk) * DK, *kc = k + ((size_t)cp.start * p.Hqk + hk) * DK;
-  const size_t qstride = (size_t)p.Hqk * DK;
   const int len = cp.len;
-  tile_async<DV, DK>(S0s, L::LS, p.S0 + u * DV * DK, DK, DV, tid);
-  tile_async<C, DV>(M1, L::LM, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
-  tile_async<C, DV>(M2, L::LM, p.dU + u * C * DV, DV, C, tid);
-  tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
-  cp_commit();
-  tile_async<DV, DK>(S1s, L::LS, p.dS1 + u * DV * DK, DK, DV, tid);
-  cp_commit();
-  cp_wait<1>();
-  __syncthreads();
-  const int r0 = 16 * (w & 3), cb = (w >> 2) * (DK / 2), half = w >> 2;
-  const int gid = lane >> 2, tig = lane & 3;
-  const float scale = p.scale;
-  float acc[DK / 16][4];
-  // dO S0: dQ part diag(gamma) dO' S0 and dgamma_t = q_t . (dO' S0)_t
-  zero_acc(acc);
-  mma3_rows<DV / 8>(acc, [&](int r, int c) { return M1[(r0 + r) * L::LM + c]; },
-                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
-  {
-    float slo, shi;
-    quad_row_sums(acc, [&](int i, int c) { return i < len ? to_f32(qc[(size_t)i * qstride + c]) : 0.f; },
-                  r0, cb, lane, slo, shi);
-    if (tig == 0) { red[half * C + r0 + gid] = scale * slo; red[half * C + r0 + gid + 8] = scale * shi; }
-    float *dQp = p.dQp + u * C * DK;
-    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) {
-      dQp[i * DK + c] = i < len ? scale * expf((float)sG[i]) * x : 0.f;
-    });
+  volatile int *ctl = reinterpret_cast<volatile int *>(smb + L::OMISC + 4);
+  const uint32_t bar_mma = sb + L::OBAR, bar_drain = sb + L::OBAR + 8;
+  double *sG = reinterpret_cast<double *>(smb + L::OG);
+  float *red = reinterpret_cast<float *>(smb + L::ORED);
+  unsigned char *AH = smb + L::OAH, *AL = smb + L::OAL, *BH = smb + L::OBH, *BL = smb + L::OBL;
+  if (tid == 0) {
+    sm100::mbar_init(bar_mma, 1);
+    sm100::mbar_init(bar_drain, 1);
+    ctl[0] = 0;
+    ctl[1] = (int)header_wait_limit_us(p.status);
+    sm100::fence_barrier_init();
   }
-  zero_acc(acc);  // dW = -dU S0
-  mma3_rows<DV / 8>(acc, [&](int r, int c) { return M2[(r0 + r) * L::LM + c]; },
-                    [&](int r, int c) { return S0s[r * L::LS + cb + c]; }, lane);
-  {
-    float *dW = p.dW + u * C * DK;
-    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) { dW[i * DK + c] = -x; });
+  if (w == 0) {
+    sm100::tmem_alloc(sb + L::OMISC, L::TMEM_COLS);
+    sm100::tmem_relinquish();
   }
-  __syncthreads();
-  tile_async<C, DV>(M1, L::LM, p.U + u * C * DV, DV, C, tid);
-  cp_commit();
-  cp_wait<0>();
-  __syncthreads();
-  {  // <dS1, S0>: fixed-order partials per thread, then per warp, then over warps
-    float s = 0.f;
-    for (int x = tid; x < DV * DK; x += NT) {
-      const int r = x / DK, c = x - r * DK;
-      s = fmaf(S0s[r * L::LS + c], S1s[r * L::LS + c], s);
+  if (tid < C) sG[tid] = p.G[u * C + tid];
+  const float *S0g = p.S0 + u * DV * DK, *S1g = p.dS1 + u * DV * DK;
+  {  // A image [dO; dU]
+    constexpr int AC = DV / 8, ITEMS = 128 * AC / NT;
+    const float *dOc = p.dO + ((size_t)cp.start * p.Hv + h) * DV, *dUc = p.dU + u * C * DV;
+    const size_t dOs = (size_t)p.Hv * DV;
+    float x[ITEMS][8];
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
+      ld8(r < C ? dOc + (size_t)r * dOs + 8 * c : dUc + (size_t)(r - C) * DV + 8 * c, r >= C || r < len, x[it]);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) red[4 * C + w] = s;
+    for (int it = 0; it < ITEMS; ++it) {
+      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
+      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, x[it]);
+    }
   }
-  zero_acc(acc);  // U dS1: dK part diag(kdec) U dS1 and dkdec_t = k_t . (U dS1)_t
-  mma3_rows<DV / 8>(acc, [&](int r, int c) { return M1[(r0 + r) * L::LM + c]; },
-                    [&](int r, int c) { return S1s[r * L::LS + cb + c]; }, lane);
+  {  // B image S0 (MN-major: K row v, N columns k)
+    constexpr int BC = DK / 8, ITEMS = DV * BC / NT;
+    float x[ITEMS][8];
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
+      ld8(S0g + (size_t)v * DK + 8 * c, true, x[it]);
+    }
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
+      st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, x[it]);
+    }
+  }
+  sm100::fence_proxy_async_smem();
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smb + L::OMISC);
+  constexpr uint32_t IDESC = sm100::idesc_bf16(128, DK, 0, 1);
+  if (tid == 0) {
+    umma3_kmaj_mn<DV / 16>(tmem, sb + L::OAH, sb + L::OAL, L::A_BLK, sb + L::OBH, sb + L::OBL, L::B_LBO,
+                           IDESC, false);
+    sm100::mma_commit(bar_mma);
+  }
+  cta_wait(bar_mma, 0, ctl, p.status);
+  {  // A image U (rows 0-63), B image dS1, and <dS1, S0>
+    constexpr int AC = DV / 8, ITEMS = C * AC / NT;
+    const float *Uc = p.U + u * C * DV;
+    float x[ITEMS][8];
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
+      ld8(Uc + (size_t)r * DV + 8 * c, true, x[it]);
+    }
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
+      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, x[it]);
+    }
+  }
   {
-    float slo, shi;
-    quad_row_sums(acc, [&](int i, int c) { return i < len ? to_f32(kc[(size_t)i * qstride + c]) : 0.f; },
-                  r0, cb, lane, slo, shi);
-    if (tig == 0) { red[(2 + half) * C + r0 + gid] = slo; red[(2 + half) * C + r0 + gid + 8] = shi; }
-    float *dKp = p.dKp + u * C * DK;
-    const double Gl = sG[len - 1];
-    for_frag(acc, r0, cb, lane, [&](int i, int c, float &x) {
-      dKp[i * DK + c] = i < len ? expf((float)(Gl - sG[i])) * x : 0.f;
-    });
+    constexpr int BC = DK / 8, ITEMS = DV * BC / NT, HALF = ITEMS / 2 > 0 ? ITEMS / 2 : 1;
+    float dot = 0.f;
+#pragma unroll
+    for (int part = 0; part < ITEMS / HALF; ++part) {
+      float x[HALF][8], y[HALF][8];
+#pragma unroll
+      for (int it = 0; it < HALF; ++it) {
+        const int idx = tid + NT * (part * HALF + it), v = idx / BC, c = idx % BC;
+        ld8(S1g + (size_t)v * DK + 8 * c, true, x[it]);
+        ld8(S0g + (size_t)v * DK + 8 * c, true, y[it]);
+      }
+#pragma unroll
+      for (int it = 0; it < HALF; ++it) {
+        const int idx = tid + NT * (part * HALF + it), v = idx / BC, c = idx % BC;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dot = fmaf(x[it][e], y[it][e], dot);
+        st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, x[it]);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    if (lane == 0) red[4 * C + w] = dot;
+  }
+  sm100::fence_proxy_async_smem();
+  sm100::tc_fence_before();
+  __syncthreads();
+  sm100::tc_fence_after();
+  if (tid == 0) {
+    umma3_kmaj_mn<DV / 16>(tmem + DK, sb + L::OAH, sb + L::OAL, L::A_BLK, sb + L::OBH, sb + L::OBL,
+                           L::B_LBO, IDESC, false);
+    sm100::mma_commit(bar_mma);
+  }
+  // D1 while D2 runs: warp w reads TMEM lanes 32 (w % 4) .. + 31 (its rows),
+  // columns [half Dk / 2, + Dk / 2) in blocks of 32
+  const int qd = w & 3, half = w >> 2, row = 32 * qd + lane;
+  const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+  const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
+  const size_t qoff = ((size_t)cp.start * p.Hqk + hk) * DK, qstride = (size_t)p.Hqk * DK;
+  const float scale = p.scale;
+  {
+    float acc_g = 0.f;
+    const float gam = row < len ? expf((float)sG[row < C ? row : 0]) : 0.f;
+#pragma unroll
+    for (int cc = 0; cc < DK / 64; ++cc) {
+      const int col = half * (DK / 2) + 32 * cc;
+      float v[32];
+      sm100::tmem_ld32(tl + col, v);
+      sm100::tmem_wait_ld();
+      if (row < C) {  // dQ part and dgamma
+        float *dst = p.dQp + (u * C + row) * DK + col;
+        const TI *qr = q + qoff + (size_t)row * qstride + col;
+#pragma unroll
+        for (int x = 0; x < 32; x += 4) {
+          *reinterpret_cast<float4 *>(dst + x) =
+              make_float4(scale * gam * v[x], scale * gam * v[x + 1], scale * gam * v[x + 2], scale * gam * v[x + 3]);
+          if (row < len)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc_g = fmaf(to_f32(qr[x + e]), v[x + e], acc_g);
+        }
+      } else {  // dW = -(dU S0)
+        float *dst = p.dW + (u * C + row - C) * DK + col;
+#pragma unroll
+        for (int x = 0; x < 32; x += 4)
+          *reinterpret_cast<float4 *>(dst + x) = make_float4(-v[x], -v[x + 1], -v[x + 2], -v[x + 3]);
+      }
+    }
+    if (row < C) red[half * C + row] = scale * acc_g;
+  }
+  cta_wait(bar_mma, 1, ctl, p.status);
+  if (qd < 2) {  // D2 rows 0-63: dK part and dkdec
+    float acc_k = 0.f;
+    const float kd = row < len ? expf((float)(sG[len - 1] - sG[row])) : 0.f;
+#pragma unroll
+    for (int cc = 0; cc < DK / 64; ++cc) {
+      const int col = half * (DK / 2) + 32 * cc;
+      float v[32];
+      sm100::tmem_ld32(tl + DK + col, v);
+      sm100::tmem_wait_ld();
+      float *dst = p.dKp + (u * C + row) * DK + col;
+      const TI *kr = k + qoff + (size_t)row * qstride + col;
+#pragma unroll
+      for (int x = 0; x < 32; x += 4) {
+        *reinterpret_cast<float4 *>(dst + x) = make_float4(kd * v[x], kd * v[x + 1], kd * v[x + 2], kd * v[x + 3]);
+        if (row < len)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc_k = fmaf(to_f32(kr[x + e]), v[x + e], acc_k);
+      }
+    }
+    red[(2 + half) * C + row] = acc_k;
   }
   __syncthreads();
   float *sc = p.sc + u * 3 * C;
@@ -613,6 +805,15 @@ __global__ void __launch_bounds__(NT) grads_state_kernel(const Params p) {
     float s = 0.f;
     for (int x = 0; x < NT / 32; ++x) s += red[4 * C + x];
     sc[2 * C] = s;
+    // every MMA this thread issued has finished before the columns are freed
+    sm100::mma_commit(bar_drain);
+    sm100::mbar_wait_landed(bar_drain, 0, 50000000ull);
+  }
+  sm100::tc_fence_before();
+  __syncthreads();
+  if (w == 0) {
+    sm100::tc_fence_after();
+    sm100::tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
 
@@ -891,8 +1092,14 @@ cudaError_t run_chunked(const cbwd::Params &prm, int64_t chunks, cudaStream_t st
   const dim3 per_chunk((unsigned)chunks, (unsigned)prm.Hv), per_seq((unsigned)prm.N, (unsigned)prm.Hv, DV / SL);
   cudaError_t e;
   if ((e = launch_k(prep_kernel<TI, DK, DV>, per_chunk, PrepSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
-  if ((e = launch_k(fwd_chain_kernel<TI, DK, DV>, per_seq, FwdSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
-  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
+  // The two chains do not depend on each other: the reverse one (a whole SM
+  // per CTA) on the high-priority internal stream, the forward one (two CTAs
+  // fit on an SM) beside it on the SMs left.
+  cudaStream_t lo = nullptr, hi = nullptr;
+  if ((e = internal_streams_fork(stream, &lo, &hi)) != cudaSuccess) return e;
+  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<TI, DK, DV>::BYTES, prm, hi)) != cudaSuccess) return e;
+  if ((e = launch_k(fwd_chain_kernel<TI, DK, DV>, per_seq, FwdSmem<TI, DK, DV>::BYTES, prm, lo)) != cudaSuccess) return e;
+  if ((e = internal_streams_join(stream)) != cudaSuccess) return e;
   if ((e = launch_k(grads_state_kernel<TI, DK, DV>, per_chunk, StateGradSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
   return launch_k(grads_local_kernel<TI, DK, DV>, per_chunk, LocalSmem<TI, DK, DV>::BYTES, prm, stream);
 }
@@ -935,6 +1142,7 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
   prm.W = F(L.W); prm.dQp = F(L.dQp); prm.dKp = F(L.dKp); prm.dW = F(L.dW);
   prm.Ut = F(L.Ut); prm.U = F(L.U); prm.dU = F(L.dU);
   prm.S0 = F(L.S0); prm.dS1 = F(L.dS1); prm.sc = F(L.sc);
+  prm.status = status;
   prm.G = reinterpret_cast<double *>(ws + L.G);
   const int64_t chunks = tp::chunk_bound(N, T);
   e = dtype == GDN_DTYPE_BF16 ? run_chunked_dims<__nv_bfloat16>(prm, Dk, Dv, chunks, stream)

@@ -72,6 +72,7 @@ namespace cbwd {
 
 constexpr int C = 64;         // chunk length
 constexpr int NT = 256;       // threads per CTA (8 warps)
+constexpr int NTR = 512;      // threads of a reverse-chain CTA (16 warps: one CTA per SM)
 constexpr int SL = 64;        // state rows per chain CTA
 constexpr int LD64 = 68;      // fp32 row stride of 64 x 64 tiles in shared memory
 constexpr float kGmin = -30.f;  // g clamp: alpha >= e^-30, so prefix sums stay finite
@@ -194,30 +195,30 @@ __device__ __forceinline__ void cp_wait() {
 }
 // dst[r][0..COLS) (row stride ld elements) <- src[r * stride + 0..COLS) for r
 // < valid, zeros for valid <= r < ROWS.  Rows of dst and src 16-byte aligned.
-template <int ROWS, int COLS, typename E>
+template <int ROWS, int COLS, int NTH = NT, typename E>
 __device__ __forceinline__ void tile_async(E *dst, int ld, const E *src, size_t stride, int valid,
                                            int tid) {
   constexpr int PER = 16 / sizeof(E), V = COLS / PER;
-  for (int x = tid; x < ROWS * V; x += NT) {
+  for (int x = tid; x < ROWS * V; x += NTH) {
     const int r = x / V, c = PER * (x - r * V);
     const bool ok = r < valid;
     cp_async16(dst + r * ld + c, ok ? src + (size_t)r * stride + c : src, ok);
   }
 }
 // dst[r * stride + c] = src[r][c] (row stride ld) for r < ROWS, c < COLS.
-template <int ROWS, int COLS>
+template <int ROWS, int COLS, int NTH = NT>
 __device__ __forceinline__ void store_tile(float *dst, size_t stride, const float *src, int ld,
                                            int tid) {
   constexpr int V4 = COLS / 4;
-  for (int x = tid; x < ROWS * V4; x += NT) {
+  for (int x = tid; x < ROWS * V4; x += NTH) {
     const int r = x / V4, c = 4 * (x - r * V4);
     *reinterpret_cast<float4 *>(dst + (size_t)r * stride + c) =
         *reinterpret_cast<const float4 *>(src + r * ld + c);
   }
 }
-template <int ROWS, int COLS>
+template <int ROWS, int COLS, int NTH = NT>
 __device__ __forceinline__ void zero_tile(float *dst, int ld, int tid) {
-  for (int x = tid; x < ROWS * COLS; x += NT) dst[(x / COLS) * ld + x % COLS] = 0.f;
+  for (int x = tid; x < ROWS * COLS; x += NTH) dst[(x / COLS) * ld + x % COLS] = 0.f;
 }
 
 // Row stride (elements) of an input tile kept in its own type in shared
@@ -429,7 +430,7 @@ struct RevSmem {
 };
 
 template <typename TI, int DK, int DV>
-__global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
+__global__ void __launch_bounds__(NTR) rev_chain_kernel(const Params p) {
   using L = RevSmem<TI, DK, DV>;
   extern __shared__ __align__(16) unsigned char smb[];
   float *dS = reinterpret_cast<float *>(smb + L::OS), *Ps = reinterpret_cast<float *>(smb + L::OP),
@@ -448,30 +449,30 @@ __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
   const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;
   const size_t qstride = (size_t)p.Hqk * DK;
   const float scale = p.scale;
-  if (p.dSf) tile_async<SL, DK>(dS, L::LS, p.dSf + srow * DK, DK, SL, tid);
-  else zero_tile<SL, DK>(dS, L::LS, tid);
+  if (p.dSf) tile_async<SL, DK, NTR>(dS, L::LS, p.dSf + srow * DK, DK, SL, tid);
+  else zero_tile<SL, DK, NTR>(dS, L::LS, tid);
   {  // P and K of the last chunk (later ones are fetched one chunk ahead)
     const size_t u = (size_t)(c0 + nch - 1) * p.Hv + h;
     const int start = cs + C * (nch - 1), len = min(C, Lseq - C * (nch - 1));
-    tile_async<C, C>(Ps, LD64, p.P + u * C * C, C, C, tid);
-    tile_async<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
+    tile_async<C, C, NTR>(Ps, LD64, p.P + u * C * C, C, C, tid);
+    tile_async<C, DK, NTR>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
   }
   const int r0 = 16 * (w & 3);
   for (int j = nch - 1; j >= 0; --j) {
     const size_t u = (size_t)(c0 + j) * p.Hv + h;
     const int start = cs + C * j, len = min(C, Lseq - C * j);
-    tile_async<C, SL>(dOs, L::LO, p.dO + ((size_t)start * p.Hv + h) * DV + v0, (size_t)p.Hv * DV, len, tid);
-    tile_async<C, DK>(Qs, L::LK, q + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
-    tile_async<C, DK>(Ws, L::LW, p.W + u * C * DK, DK, C, tid);
-    tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+    tile_async<C, SL, NTR>(dOs, L::LO, p.dO + ((size_t)start * p.Hv + h) * DV + v0, (size_t)p.Hv * DV, len, tid);
+    tile_async<C, DK, NTR>(Qs, L::LK, q + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
+    tile_async<C, DK, NTR>(Ws, L::LW, p.W + u * C * DK, DK, C, tid);
+    tile_async<1, C, NTR>(sG, C, p.G + u * C, 0, 1, tid);
     cp_commit();
     cp_wait<0>();
     __syncthreads();
-    store_tile<SL, DK>(p.dS1 + (u * DV + v0) * DK, DK, dS, L::LS, tid);
+    store_tile<SL, DK, NTR>(p.dS1 + (u * DV + v0) * DK, DK, dS, L::LS, tid);
     if (tid < C) sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
-    {  // dU = P^T dO' + diag(kdec) K dS^T: token rows 16 (w & 3), state rows 32 (w >> 2)
-      const int vb = 32 * (w >> 2);
-      float a1[4][4], a2[4][4];
+    {  // dU = P^T dO' + diag(kdec) K dS^T: token rows 16 (w & 3), state rows 16 (w >> 2)
+      const int vb = 16 * (w >> 2);
+      float a1[2][4], a2[2][4];
       zero_acc(a1);
       zero_acc(a2);
       mma3_rows<C / 8>(a1, [&](int r, int c) { return Ps[c * LD64 + r0 + r]; },
@@ -485,7 +486,7 @@ __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
       float *dUg = p.dU + u * C * DV + v0;
       const int tig = lane & 3;
 #pragma unroll
-      for (int t = 0; t < 4; ++t)
+      for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = r0 + gid + 8 * (e >> 1), c = vb + 8 * t + 2 * tig + (e & 1);
@@ -498,14 +499,14 @@ __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
     if (j > 0) {  // the previous chunk's P and K into the freed buffers
       const size_t up = u - p.Hv;
       const int sp = start - C;
-      tile_async<C, C>(Ps, LD64, p.P + up * C * C, C, C, tid);
-      tile_async<C, DK>(Ks, L::LK, k + ((size_t)sp * p.Hqk + hk) * DK, qstride, C, tid);
+      tile_async<C, C, NTR>(Ps, LD64, p.P + up * C * C, C, C, tid);
+      tile_async<C, DK, NTR>(Ks, L::LK, k + ((size_t)sp * p.Hqk + hk) * DK, qstride, C, tid);
       cp_commit();
     }
-    {  // dS <- gamma_C dS + dO'^T diag(gamma) Q - dU^T W: state rows 16 (w & 3), columns DK / 2 (w >> 2)
+    {  // dS <- gamma_C dS + dO'^T diag(gamma) Q - dU^T W: state rows 16 (w & 3), columns DK / 4 (w >> 2)
       const float gC = expf((float)sG[len - 1]);
-      const int kb = (w >> 2) * (DK / 2);
-      float acc[DK / 16][4];
+      const int kb = (w >> 2) * (DK / 4);
+      float acc[DK / 32][4];
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * dS[r * L::LS + c]; });
       mma3_rows<C / 8>(acc, [&](int r, int c) { return scale * dOs[c * L::LO + r0 + r] * sGm[c]; },
                        [&](int r, int c) { return to_f32(Qs[r * L::LK + kb + c]); }, lane);
@@ -515,7 +516,7 @@ __global__ void __launch_bounds__(NT) rev_chain_kernel(const Params p) {
     }
     __syncthreads();
   }
-  if (p.ds0) store_tile<SL, DK>(p.ds0 + srow * DK, DK, dS, L::LS, tid);
+  if (p.ds0) store_tile<SL, DK, NTR>(p.ds0 + srow * DK, DK, dS, L::LS, tid);
 }
 
 // ---- tcgen05 building blocks -----------------------------------------------
@@ -1078,11 +1079,12 @@ size_t backward_chunked_workspace_bytes(int64_t N, int64_t T, int Hqk, int Hv, i
 namespace {
 
 template <typename K>
-cudaError_t launch_k(K kern, dim3 grid, size_t smem, const cbwd::Params &prm, cudaStream_t stream) {
+cudaError_t launch_k(K kern, dim3 grid, size_t smem, const cbwd::Params &prm, cudaStream_t stream,
+                     int threads = cbwd::NT) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (grid.x == 0 || grid.y == 0 || grid.z == 0) return cudaSuccess;
-  kern<<<grid, cbwd::NT, smem, stream>>>(prm);
+  kern<<<grid, threads, smem, stream>>>(prm);
   return cudaGetLastError();
 }
 
@@ -1097,7 +1099,7 @@ cudaError_t run_chunked(const cbwd::Params &prm, int64_t chunks, cudaStream_t st
   // fit on an SM) beside it on the SMs left.
   cudaStream_t lo = nullptr, hi = nullptr;
   if ((e = internal_streams_fork(stream, &lo, &hi)) != cudaSuccess) return e;
-  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<TI, DK, DV>::BYTES, prm, hi)) != cudaSuccess) return e;
+  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<TI, DK, DV>::BYTES, prm, hi, NTR)) != cudaSuccess) return e;
   if ((e = launch_k(fwd_chain_kernel<TI, DK, DV>, per_seq, FwdSmem<TI, DK, DV>::BYTES, prm, lo)) != cudaSuccess) return e;
   if ((e = internal_streams_join(stream)) != cudaSuccess) return e;
   if ((e = launch_k(grads_state_kernel<TI, DK, DV>, per_chunk, StateGradSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;

@@ -47,10 +47,11 @@
 // each chain CTA owns 64 of the Dv rows.  Tiles move global -> shared with
 // cp.async, all of a step's copies in flight at once, and the chains fetch a
 // chunk's tiles while the previous chunk computes where buffers allow.
-// Every product runs on warp-level m16n8k8 tf32 tensor-core MMAs with both
-// operands split into hi (x with the low 13 mantissa bits cleared) and
-// lo = x - hi, and three products (hi*hi + hi*lo + lo*hi), which keeps about
-// fp32 accuracy.  Per-row sums go through fixed-order partials, so results do
+// Products run on tensor cores at about fp32 accuracy: fp32 operands split
+// into hi and lo parts and three products hi*hi + hi*lo + lo*hi, a raw bf16
+// input used as it is (its lo part is zero).  The state gradients run on
+// tcgen05 (bf16 hi/lo images, TMEM accumulators); the rest on warp-level MMAs,
+// m16n8k16 bf16 where an operand is a raw bf16 input, m16n8k8 tf32 otherwise.  Per-row sums go through fixed-order partials, so results do
 // not depend on scheduling.
 #include <algorithm>
 
@@ -100,42 +101,88 @@ struct Params {
 };
 
 // ---- tensor-core building block -------------------------------------------
+// Warp-level m16n8k16 bf16 MMA with fp32 accumulation.
+__device__ __forceinline__ void mma_bf16_16x8x16(float *d, const uint32_t *a, const uint32_t *b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// Split of two fp32 values into packed bf16 pairs hi = bf16(x) and lo =
+// bf16(x - hi), both rounded to nearest: |x - hi - lo| <= 2^-18 |x|.
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 hf = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+  hi = *reinterpret_cast<const uint32_t *>(&h);
+  lo = *reinterpret_cast<const uint32_t *>(&l);
+}
+
 // Split of an fp32 value for the 3-term tf32 products: hi keeps the sign,
 // exponent and the 10 mantissa bits a tf32 operand holds (the low 13 bits
 // cleared, |x - hi| < 2^-10 |x|); lo = x - hi is exact in fp32 and goes to the
 // MMA as is, which reads only its tf32 bits (|error| < 2^-10 |lo|).  So
-// hi*hi' + hi*lo' + lo*hi' is within about 2^-19 of x*y, with bit operations
-// and one subtraction instead of conversions.
+// hi*hi' + hi*lo' + lo*hi' is within about 2^-18 of x*y.
 __device__ __forceinline__ uint32_t tf32_hi(float x) { return __float_as_uint(x) & 0xffffe000u; }
 __device__ __forceinline__ uint32_t tf32_lo(float x, uint32_t hi) {
   return __float_as_uint(x - __uint_as_float(hi));
 }
 
-// acc[t] (a 16 x 8 fragment) += X[16][8 KS] * Y[8 KS][8 t .. 8 t + 7] for t <
-// NTL tiles in a row.  X(r, c) and Y(r, c) read single elements; each is split
-// once per k step.  Fragment element e of tile t sits at row gid + 8 (e >> 1),
-// column 8 t + 2 tig + (e & 1) (gid = lane / 4, tig = lane % 4).
-template <int KS, int NTL, class FX, class FY>
+// acc[t] (a 16 x 8 fragment) += X[16][KDIM] * Y[KDIM][8 t .. 8 t + 7] for t <
+// NTL tiles in a row, on warp-level tensor-core MMAs.  X(r, c) and Y(r, c)
+// read single elements; each is split once per k step.  Fragment element e
+// of tile t sits at row gid + 8 (e >> 1), column 8 t + 2 tig + (e & 1) (gid =
+// lane / 4, tig = lane % 4) for both MMA shapes used:
+//   - an operand marked exact holds bf16 values already (a raw bf16 input):
+//     m16n8k16 bf16 MMAs, the other operand split into bf16 hi + lo (rounded
+//     to nearest, |x - hi - lo| <= 2^-18 |x|): two MMAs per k step, one when
+//     both operands are exact;
+//   - otherwise m16n8k8 tf32 MMAs with both operands split (tf32_hi, tf32_lo)
+//     and three products per k step.
+template <int KDIM, int NTL, bool XEXACT = false, bool YEXACT = false, class FX, class FY>
 __device__ __forceinline__ void mma3_rows(float (&acc)[NTL][4], FX X, FY Y, int lane) {
   const int gid = lane >> 2, tig = lane & 3;
+  if constexpr (XEXACT || YEXACT) {
 #pragma unroll 2
-  for (int ks = 0; ks < KS; ++ks) {
-    const int k0 = 8 * ks + tig;
-    const float a[4] = {X(gid, k0), X(gid + 8, k0), X(gid, k0 + 4), X(gid + 8, k0 + 4)};
-    uint32_t ah[4], al[4];
+    for (int ks = 0; ks < KDIM / 16; ++ks) {
+      const int k0 = 16 * ks + 2 * tig;
+      uint32_t ah[4], al[4];
+      split2(X(gid, k0), X(gid, k0 + 1), ah[0], al[0]);
+      split2(X(gid + 8, k0), X(gid + 8, k0 + 1), ah[1], al[1]);
+      split2(X(gid, k0 + 8), X(gid, k0 + 9), ah[2], al[2]);
+      split2(X(gid + 8, k0 + 8), X(gid + 8, k0 + 9), ah[3], al[3]);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      ah[e] = tf32_hi(a[e]);
-      al[e] = tf32_lo(a[e], ah[e]);
+      for (int t = 0; t < NTL; ++t) {
+        const int n = 8 * t + gid;
+        uint32_t bh[2], bl[2];
+        split2(Y(k0, n), Y(k0 + 1, n), bh[0], bl[0]);
+        split2(Y(k0 + 8, n), Y(k0 + 9, n), bh[1], bl[1]);
+        if (!XEXACT) mma_bf16_16x8x16(acc[t], al, bh);
+        if (!YEXACT) mma_bf16_16x8x16(acc[t], ah, bl);
+        mma_bf16_16x8x16(acc[t], ah, bh);
+      }
     }
+  } else {
+#pragma unroll 2
+    for (int ks = 0; ks < KDIM / 8; ++ks) {
+      const int k0 = 8 * ks + tig;
+      const float a[4] = {X(gid, k0), X(gid + 8, k0), X(gid, k0 + 4), X(gid + 8, k0 + 4)};
+      uint32_t ah[4], al[4];
 #pragma unroll
-    for (int t = 0; t < NTL; ++t) {
-      const float b0 = Y(k0, 8 * t + gid), b1 = Y(k0 + 4, 8 * t + gid);
-      const uint32_t bh[2] = {tf32_hi(b0), tf32_hi(b1)};
-      const uint32_t bl[2] = {tf32_lo(b0, bh[0]), tf32_lo(b1, bh[1])};
-      chunk::mma_tf32_16x8x8(acc[t], al, bh);
-      chunk::mma_tf32_16x8x8(acc[t], ah, bl);
-      chunk::mma_tf32_16x8x8(acc[t], ah, bh);
+      for (int e = 0; e < 4; ++e) {
+        ah[e] = tf32_hi(a[e]);
+        al[e] = tf32_lo(a[e], ah[e]);
+      }
+#pragma unroll
+      for (int t = 0; t < NTL; ++t) {
+        const float b0 = Y(k0, 8 * t + gid), b1 = Y(k0 + 4, 8 * t + gid);
+        const uint32_t bh[2] = {tf32_hi(b0), tf32_hi(b1)};
+        const uint32_t bl[2] = {tf32_lo(b0, bh[0]), tf32_lo(b1, bh[1])};
+        chunk::mma_tf32_16x8x8(acc[t], al, bh);
+        chunk::mma_tf32_16x8x8(acc[t], ah, bl);
+        chunk::mma_tf32_16x8x8(acc[t], ah, bh);
+      }
     }
   }
 }
@@ -300,9 +347,10 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
     float aq[4][4], ak[4][4];
     zero_acc(aq);
     zero_acc(ak);
-    mma3_rows<DK / 8>(aq, [&](int r, int c) { return to_f32(Qs[(r0 + r) * L::LQ + c]); },
+    constexpr bool EX = sizeof(TI) == 2;  // raw bf16 inputs are exact bf16 operands
+    mma3_rows<DK, 4, EX, EX>(aq, [&](int r, int c) { return to_f32(Qs[(r0 + r) * L::LQ + c]); },
                       [&](int r, int c) { return to_f32(Ks[(c0 + c) * L::LQ + r]); }, lane);
-    mma3_rows<DK / 8>(ak, [&](int r, int c) { return to_f32(Ks[(r0 + r) * L::LQ + c]); },
+    mma3_rows<DK, 4, EX, EX>(ak, [&](int r, int c) { return to_f32(Ks[(r0 + r) * L::LQ + c]); },
                       [&](int r, int c) { return to_f32(Ks[(c0 + c) * L::LQ + r]); }, lane);
     float *P = p.P + u * C * C, *EKK = p.EKK + u * C * C;
     const int gid = lane >> 2, tig = lane & 3;
@@ -332,8 +380,9 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
       const int c0 = (w >> 2) * (DK / 2);
       float acc[DK / 16][4];
       zero_acc(acc);
-      mma3_rows<C / 8>(acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c]; },
-                       [&](int r, int c) { return sBG[r] * to_f32(Ks[r * L::LQ + c0 + c]); }, lane);
+      mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(
+          acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c] * sBG[c]; },
+          [&](int r, int c) { return to_f32(Ks[r * L::LQ + c0 + c]); }, lane);
       float *W = p.W + u * C * DK;
       for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { W[i * DK + c] = x; });
     }
@@ -341,8 +390,9 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
       const int c0 = (w >> 2) * (DV / 2);
       float acc[DV / 16][4];
       zero_acc(acc);
-      mma3_rows<C / 8>(acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c]; },
-                       [&](int r, int c) { return sB[r] * to_f32(Vs[r * L::LV + c0 + c]); }, lane);
+      mma3_rows<C, DV / 16, false, sizeof(TI) == 2>(
+          acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c] * sB[c]; },
+          [&](int r, int c) { return to_f32(Vs[r * L::LV + c0 + c]); }, lane);
       float *Ut = p.Ut + u * C * DV;
       for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { Ut[i * DV + c] = x; });
     }
@@ -393,7 +443,7 @@ __global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
       const int vb = 32 * (w >> 2);
       float acc[4][4];
       zero_acc(acc);
-      mma3_rows<DK / 8>(acc, [&](int r, int c) { return Ws[(r0 + r) * L::LW + c]; },
+      mma3_rows<DK>(acc, [&](int r, int c) { return Ws[(r0 + r) * L::LW + c]; },
                         [&](int r, int c) { return S[(vb + c) * L::LS + r]; }, lane);
       float *Ug = p.U + u * C * DV + v0;
       for_frag(acc, r0, vb, lane, [&](int i, int c, float &x) {
@@ -411,7 +461,7 @@ __global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
       const int kb = (w >> 2) * (DK / 2);
       float acc[DK / 16][4];
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * S[r * L::LS + c]; });
-      mma3_rows<C / 8>(acc, [&](int r, int c) { return Us[c * L::LU + r0 + r] * sKd[c]; },
+      mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(acc, [&](int r, int c) { return Us[c * L::LU + r0 + r] * sKd[c]; },
                        [&](int r, int c) { return to_f32(Ks[r * L::LK + kb + c]); }, lane);
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { S[r * L::LS + c] = x; });
       __syncthreads();
@@ -475,9 +525,9 @@ __global__ void __launch_bounds__(NTR) rev_chain_kernel(const Params p) {
       float a1[2][4], a2[2][4];
       zero_acc(a1);
       zero_acc(a2);
-      mma3_rows<C / 8>(a1, [&](int r, int c) { return Ps[c * LD64 + r0 + r]; },
+      mma3_rows<C>(a1, [&](int r, int c) { return Ps[c * LD64 + r0 + r]; },
                        [&](int r, int c) { return dOs[r * L::LO + vb + c]; }, lane);
-      mma3_rows<DK / 8>(a2, [&](int r, int c) { return to_f32(Ks[(r0 + r) * L::LK + c]); },
+      mma3_rows<DK, 2, sizeof(TI) == 2, false>(a2, [&](int r, int c) { return to_f32(Ks[(r0 + r) * L::LK + c]); },
                         [&](int r, int c) { return dS[(vb + c) * L::LS + r]; }, lane);
       const double Gl = sG[len - 1];
       const int i0 = r0 + gid, i1 = i0 + 8;
@@ -508,9 +558,9 @@ __global__ void __launch_bounds__(NTR) rev_chain_kernel(const Params p) {
       const int kb = (w >> 2) * (DK / 4);
       float acc[DK / 32][4];
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * dS[r * L::LS + c]; });
-      mma3_rows<C / 8>(acc, [&](int r, int c) { return scale * dOs[c * L::LO + r0 + r] * sGm[c]; },
+      mma3_rows<C, DK / 32, false, sizeof(TI) == 2>(acc, [&](int r, int c) { return scale * dOs[c * L::LO + r0 + r] * sGm[c]; },
                        [&](int r, int c) { return to_f32(Qs[r * L::LK + kb + c]); }, lane);
-      mma3_rows<C / 8>(acc, [&](int r, int c) { return -dUs[c * L::LO + r0 + r]; },
+      mma3_rows<C>(acc, [&](int r, int c) { return -dUs[c * L::LO + r0 + r]; },
                        [&](int r, int c) { return Ws[r * L::LW + kb + c]; }, lane);
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { dS[r * L::LS + c] = x; });
     }
@@ -878,7 +928,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   {  // step 1: dP = lower(dO' U^T); S2 = dP . E, S1 = dP . P
     float acc[4][4];
     zero_acc(acc);
-    mma3_rows<DV / 8>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
+    mma3_rows<DV>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
                       [&](int r, int c) { return RB[(c64 + c) * L::LB + r]; }, lane);
     for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) {
       const float dp = i >= j ? scale * x : 0.f;
@@ -893,20 +943,29 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   cp_wait<0>();
   __syncthreads();
   {  // step 2: dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T -> S4
-    float acc[4][4];
-    zero_acc(acc);
-    mma3_rows<DK / 8>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
-                      [&](int r, int c) { return sB[c64 + c] * sGm[c64 + c] * to_f32(RC[(c64 + c) * L::LC + r]); },
-                      lane);
-    mma3_rows<DV / 8>(acc, [&](int r, int c) { return RB[(r0 + r) * L::LB + c]; },
-                      [&](int r, int c) { return sB[c64 + c] * to_f32(RD[(c64 + c) * L::LD + r]); }, lane);
-    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = x; });
+    // (dW K^T and dU V^T with the raw inputs, then the column scales)
+    constexpr bool EX = sizeof(TI) == 2;
+    float a1[4][4], a2[4][4];
+    zero_acc(a1);
+    zero_acc(a2);
+    mma3_rows<DK, 4, false, EX>(a1, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
+                                     [&](int r, int c) { return to_f32(RC[(c64 + c) * L::LC + r]); }, lane);
+    mma3_rows<DV, 4, false, EX>(a2, [&](int r, int c) { return RB[(r0 + r) * L::LB + c]; },
+                                     [&](int r, int c) { return to_f32(RD[(c64 + c) * L::LD + r]); }, lane);
+    const int tig = lane & 3;
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = r0 + gid + 8 * (e >> 1), j = c64 + 8 * t + 2 * tig + (e & 1);
+        S4[i * LD64 + j] = sB[j] * (sGm[j] * a1[t][e] + a2[t][e]);
+      }
   }
   const int cbk = half * (DK / 2), cbv = half * (DV / 2);
   float dK[DK / 16][4];
   {  // X = Tm^T dW
     zero_acc(dK);
-    mma3_rows<C / 8>(dK, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+    mma3_rows<C>(dK, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
                      [&](int r, int c) { return RA[r * L::LA + cbk + c]; }, lane);
     float slo, shi;
     quad_row_sums(dK, [&](int i, int c) { return to_f32(RC[i * L::LC + c]); }, r0, cbk, lane, slo, shi);
@@ -916,7 +975,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   {  // Y = Tm^T dU: dv = diag(beta) Y
     float acc[DV / 16][4];
     zero_acc(acc);
-    mma3_rows<C / 8>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+    mma3_rows<C>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
                      [&](int r, int c) { return RB[r * L::LB + cbv + c]; }, lane);
     float slo, shi;
     quad_row_sums(acc, [&](int i, int c) { return to_f32(RD[i * L::LD + c]); }, r0, cbv, lane, slo, shi);
@@ -932,7 +991,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   {  // Z = dT Tm^T -> S5
     float acc[4][4];
     zero_acc(acc);
-    mma3_rows<C / 8>(acc, [&](int r, int c) { return S4[(r0 + r) * LD64 + c]; },
+    mma3_rows<C>(acc, [&](int r, int c) { return S4[(r0 + r) * LD64 + c]; },
                      [&](int r, int c) { return S3[(c64 + c) * LD64 + r]; }, lane);
     for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S5[i * LD64 + j] = x; });
   }
@@ -940,7 +999,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   {  // dA = strict_lower(-Tm^T Z) -> S4
     float acc[4][4];
     zero_acc(acc);
-    mma3_rows<C / 8>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+    mma3_rows<C>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
                      [&](int r, int c) { return S5[r * LD64 + c64 + c]; }, lane);
     for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = i > j ? -x : 0.f; });
   }
@@ -973,7 +1032,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     float acc[DK / 16][4];
     const float *dQp = p.dQp + u * C * DK;
     for_frag(acc, r0, cbk, lane, [&](int i, int c, float &x) { x = dQp[i * DK + c]; });
-    mma3_rows<C / 8>(acc, [&](int r, int c) { return S2[(r0 + r) * LD64 + c]; },
+    mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(acc, [&](int r, int c) { return S2[(r0 + r) * LD64 + c]; },
                      [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
     const bool direct = Gq == 1;
     float *dst = direct ? p.dq + qoff : p.dq + ((size_t)cp.start * p.Hv + h) * DK;
@@ -985,9 +1044,9 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   {  // dk = diag(kdec) U dS1 + diag(beta gamma) X + (dP . E)^T Q + (B + B^T) K
     const float *dKp = p.dKp + u * C * DK;
     for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x += dKp[i * DK + c]; });
-    mma3_rows<C / 8>(dK, [&](int r, int c) { return S2[c * LD64 + r0 + r]; },
+    mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S2[c * LD64 + r0 + r]; },
                      [&](int r, int c) { return to_f32(RD[r * L::LD + cbk + c]); }, lane);
-    mma3_rows<C / 8>(dK, [&](int r, int c) { return S4[(r0 + r) * LD64 + c] + S4[c * LD64 + r0 + r]; },
+    mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S4[(r0 + r) * LD64 + c] + S4[c * LD64 + r0 + r]; },
                      [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
     const bool direct = Gq == 1;
     float *dst = direct ? p.dk + qoff : p.dk + ((size_t)cp.start * p.Hv + h) * DK;

@@ -29,22 +29,22 @@
 //   dg_s = sum_{t >= s} dG_t within the chunk.
 // dq and dk of a query/key head sum over the value heads that read it.
 //
-// Launches (the two chains on the caller stream's internal pair, beside each
-// other; the rest on the caller's stream):
+// Launches (one stream):
 //   plan         validates cu_seqlens, lists the non-empty sequences and
 //                their first chunk; d_initial_state of an empty sequence is
 //                d_final_state (or zero)
 //   prep         per (chunk, value head): P, E . K K^T, Tm, W, U~, G
-//   fwd_chain    per (sequence, value head, 64 rows of the state): the state
-//                at every chunk start (S0) and U, in chunk order
-//   rev_chain    per (sequence, value head, 64 rows): dS1 and dU, chunks last
-//                to first, and d_initial_state
+//   chains       one launch of both chains, which do not depend on each
+//                other: per (sequence, value head, 64 state rows) the reverse
+//                one (dS1 and dU per chunk, last to first, and
+//                d_initial_state), then per (sequence, value head) the
+//                forward one (the state at every chunk start S0, and U)
 //   grads_state  per (chunk, value head): the products with S0 and dS1
 //   grads_local  per (chunk, value head): the 64 x 64 algebra, then dq, dk
 //                (per value head), dv, dg, dbeta
 //   group sums   dq, dk over the value heads of each query/key head
-// Rows of S and of dS evolve independently (the chains never mix rows), so
-// each chain CTA owns 64 of the Dv rows.  Tiles move global -> shared with
+// Rows of S and of dS evolve independently (the chains never mix rows), so a
+// reverse-chain CTA owns 64 of the Dv rows.  Tiles move global -> shared with
 // cp.async, all of a step's copies in flight at once, and the chains fetch a
 // chunk's tiles while the previous chunk computes where buffers allow.
 // Products run on tensor cores at about fp32 accuracy: fp32 operands split
@@ -66,8 +66,6 @@ cudaError_t launch_plan(const int32_t *cu, int N, int T, int Hv, const void *s0,
                         int32_t *status, cudaStream_t stream);
 cudaError_t launch_group_sum(const float *part, float *out, size_t rows, int width, int inner,
                              cudaStream_t stream);
-cudaError_t internal_streams_fork(cudaStream_t caller, cudaStream_t *lo, cudaStream_t *hi);
-cudaError_t internal_streams_join(cudaStream_t caller);
 
 namespace cbwd {
 
@@ -399,53 +397,53 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
   }
 }
 
-// ---- forward chain: S0 and U of every chunk, per SL rows of the state ---------
+// ---- forward chain: S0 and U of every chunk, a whole head (Dv state rows) ----
 template <typename TI, int DK, int DV>
 struct FwdSmem {
-  static constexpr int LS = DK + 4, LW = DK + 4, LK = in_ld<TI>(DK), LU = SL + 8;
-  static constexpr size_t OS = 0, OW = OS + SL * LS * 4, OK = OW + C * LW * 4,
+  static constexpr int LS = DK + 4, LW = DK + 4, LK = in_ld<TI>(DK), LU = DV + 8;
+  static constexpr size_t OS = 0, OW = OS + DV * LS * 4, OK = OW + C * LW * 4,
                           OU = OK + up16(C * LK * sizeof(TI)), OG = OU + C * LU * 4, OKD = OG + C * 8,
                           BYTES = OKD + C * 4;
 };
 
+// One CTA of NTR threads per (non-empty sequence kk, value head h).
 template <typename TI, int DK, int DV>
-__global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
+__device__ __forceinline__ void fwd_chain_body(const Params &p, unsigned char *smb, int kk, int h) {
   using L = FwdSmem<TI, DK, DV>;
-  extern __shared__ __align__(16) unsigned char smb[];
+  constexpr int NW = NTR / 32;               // 16 warps
+  constexpr int RG = DV / 16, CG = NW / RG;  // state update: row groups x column groups
   float *S = reinterpret_cast<float *>(smb + L::OS), *Ws = reinterpret_cast<float *>(smb + L::OW),
         *Us = reinterpret_cast<float *>(smb + L::OU), *sKd = reinterpret_cast<float *>(smb + L::OKD);
   TI *Ks = reinterpret_cast<TI *>(smb + L::OK);
   double *sG = reinterpret_cast<double *>(smb + L::OG);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int kk = blockIdx.x;
   if (kk >= p.ph->n_nonempty) return;
   const int n = p.ne_seq[kk], c0 = p.ne_cs[kk], nch = p.ne_cs[kk + 1] - c0;
   const int cs = p.cu[n], Lseq = p.cu[n + 1] - cs;
-  const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk), v0 = SL * blockIdx.z;
+  const int hk = h / (p.Hv / p.Hqk);
   const TI *k = static_cast<const TI *>(p.k);
-  const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;  // first state row of this slice
-  if (p.s0) tile_async<SL, DK>(S, L::LS, p.s0 + srow * DK, DK, SL, tid);
-  else zero_tile<SL, DK>(S, L::LS, tid);
-  tile_async<C, DK>(Ws, L::LW, p.W + (size_t)c0 * p.Hv * C * DK + (size_t)h * C * DK, DK, C, tid);
-  const int r0 = 16 * (w & 3);
+  const size_t srow = ((size_t)n * p.Hv + h) * DV;  // first state row of the head
+  if (p.s0) tile_async<DV, DK, NTR>(S, L::LS, p.s0 + srow * DK, DK, DV, tid);
+  else zero_tile<DV, DK, NTR>(S, L::LS, tid);
+  tile_async<C, DK, NTR>(Ws, L::LW, p.W + ((size_t)c0 * p.Hv + h) * C * DK, DK, C, tid);
   for (int j = 0; j < nch; ++j) {
     const size_t u = (size_t)(c0 + j) * p.Hv + h;
     const int start = cs + C * j, len = min(C, Lseq - C * j);
-    tile_async<C, DK>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, tid);
-    tile_async<C, SL>(Us, L::LU, p.Ut + u * C * DV + v0, DV, C, tid);
-    tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+    tile_async<C, DK, NTR>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, tid);
+    tile_async<C, DV, NTR>(Us, L::LU, p.Ut + u * C * DV, DV, C, tid);
+    tile_async<1, C, NTR>(sG, C, p.G + u * C, 0, 1, tid);
     cp_commit();
     cp_wait<0>();
     __syncthreads();
-    store_tile<SL, DK>(p.S0 + (u * DV + v0) * DK, DK, S, L::LS, tid);
+    store_tile<DV, DK, NTR>(p.S0 + u * DV * DK, DK, S, L::LS, tid);
     if (tid < C) sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
-    {  // U = U~ - W S^T: token rows 16 (w & 3), state rows 32 (w >> 2)
-      const int vb = 32 * (w >> 2);
-      float acc[4][4];
+    {  // U = U~ - W S^T: token rows 16 (w & 3), state rows DV / 4 (w >> 2)
+      const int r0 = 16 * (w & 3), vb = (w >> 2) * (DV / 4);
+      float acc[DV / 32][4];
       zero_acc(acc);
       mma3_rows<DK>(acc, [&](int r, int c) { return Ws[(r0 + r) * L::LW + c]; },
-                        [&](int r, int c) { return S[(vb + c) * L::LS + r]; }, lane);
-      float *Ug = p.U + u * C * DV + v0;
+                    [&](int r, int c) { return S[(vb + c) * L::LS + r]; }, lane);
+      float *Ug = p.U + u * C * DV;
       for_frag(acc, r0, vb, lane, [&](int i, int c, float &x) {
         const float uu = Us[i * L::LU + c] - x;
         Us[i * L::LU + c] = uu;
@@ -454,15 +452,16 @@ __global__ void __launch_bounds__(NT) fwd_chain_kernel(const Params p) {
     }
     __syncthreads();
     if (j + 1 < nch) {
-      tile_async<C, DK>(Ws, L::LW, p.W + (u + p.Hv) * C * DK, DK, C, tid);  // next chunk's W
+      tile_async<C, DK, NTR>(Ws, L::LW, p.W + (u + p.Hv) * C * DK, DK, C, tid);  // next chunk's W
       cp_commit();
-      // S <- gamma_C S + U^T diag(kdec) K: state rows 16 (w & 3), columns DK / 2 (w >> 2)
+      // S <- gamma_C S + U^T diag(kdec) K: state rows 16 (w % RG), columns DK / CG (w / RG)
       const float gC = expf((float)sG[len - 1]);
-      const int kb = (w >> 2) * (DK / 2);
-      float acc[DK / 16][4];
+      const int r0 = 16 * (w % RG), kb = (w / RG) * (DK / CG);
+      float acc[DK / CG / 8][4];
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { x = gC * S[r * L::LS + c]; });
-      mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(acc, [&](int r, int c) { return Us[c * L::LU + r0 + r] * sKd[c]; },
-                       [&](int r, int c) { return to_f32(Ks[r * L::LK + kb + c]); }, lane);
+      mma3_rows<C, DK / CG / 8, false, sizeof(TI) == 2>(
+          acc, [&](int r, int c) { return Us[c * L::LU + r0 + r] * sKd[c]; },
+          [&](int r, int c) { return to_f32(Ks[r * L::LK + kb + c]); }, lane);
       for_frag(acc, r0, kb, lane, [&](int r, int c, float &x) { S[r * L::LS + c] = x; });
       __syncthreads();
     }
@@ -479,10 +478,11 @@ struct RevSmem {
                           BYTES = OGM + C * 4;
 };
 
+// One CTA of NTR threads per (non-empty sequence kk, value head h, SL state
+// rows from v0).
 template <typename TI, int DK, int DV>
-__global__ void __launch_bounds__(NTR) rev_chain_kernel(const Params p) {
+__device__ __forceinline__ void rev_chain_body(const Params &p, unsigned char *smb, int kk, int h, int v0) {
   using L = RevSmem<TI, DK, DV>;
-  extern __shared__ __align__(16) unsigned char smb[];
   float *dS = reinterpret_cast<float *>(smb + L::OS), *Ps = reinterpret_cast<float *>(smb + L::OP),
         *dOs = reinterpret_cast<float *>(smb + L::OO), *Ws = reinterpret_cast<float *>(smb + L::OW),
         *dUs = reinterpret_cast<float *>(smb + L::OU), *sGm = reinterpret_cast<float *>(smb + L::OGM);
@@ -490,11 +490,10 @@ __global__ void __launch_bounds__(NTR) rev_chain_kernel(const Params p) {
   double *sG = reinterpret_cast<double *>(smb + L::OG);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int gid = lane >> 2;
-  const int kk = blockIdx.x;
   if (kk >= p.ph->n_nonempty) return;
   const int n = p.ne_seq[kk], c0 = p.ne_cs[kk], nch = p.ne_cs[kk + 1] - c0;
   const int cs = p.cu[n], Lseq = p.cu[n + 1] - cs;
-  const int h = blockIdx.y, hk = h / (p.Hv / p.Hqk), v0 = SL * blockIdx.z;
+  const int hk = h / (p.Hv / p.Hqk);
   const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
   const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;
   const size_t qstride = (size_t)p.Hqk * DK;
@@ -567,6 +566,32 @@ __global__ void __launch_bounds__(NTR) rev_chain_kernel(const Params p) {
     __syncthreads();
   }
   if (p.ds0) store_tile<SL, DK, NTR>(p.ds0 + srow * DK, DK, dS, L::LS, tid);
+}
+
+// ---- both chains in one launch ----------------------------------------------
+// The two chains do not depend on each other.  CTAs [0, N Hv Dv / SL) run the
+// reverse chain (SL rows each), the next N Hv the forward chain (a whole head
+// each); CTAs start in index order, so at 48 heads all 144 share one wave, one
+// per SM, whatever the scheduler does with separate launches.
+template <typename TI, int DK, int DV>
+struct ChainSmem {
+  static constexpr size_t F = FwdSmem<TI, DK, DV>::BYTES, R = RevSmem<TI, DK, DV>::BYTES;
+  static constexpr size_t BYTES = F > R ? F : R;
+};
+
+template <typename TI, int DK, int DV>
+__global__ void __launch_bounds__(NTR, 1) chains_kernel(const Params p) {
+  extern __shared__ __align__(16) unsigned char smb[];
+  constexpr int R = DV / SL;
+  const int nrev = p.N * p.Hv * R;
+  int b = blockIdx.x;
+  if (b < nrev) {
+    const int kk = b / (p.Hv * R), rem = b - kk * (p.Hv * R);
+    rev_chain_body<TI, DK, DV>(p, smb, kk, rem / R, SL * (rem % R));
+  } else {
+    b -= nrev;
+    fwd_chain_body<TI, DK, DV>(p, smb, b / p.Hv, b % p.Hv);
+  }
 }
 
 // ---- tcgen05 building blocks -----------------------------------------------
@@ -1150,17 +1175,11 @@ cudaError_t launch_k(K kern, dim3 grid, size_t smem, const cbwd::Params &prm, cu
 template <typename TI, int DK, int DV>
 cudaError_t run_chunked(const cbwd::Params &prm, int64_t chunks, cudaStream_t stream) {
   using namespace cbwd;
-  const dim3 per_chunk((unsigned)chunks, (unsigned)prm.Hv), per_seq((unsigned)prm.N, (unsigned)prm.Hv, DV / SL);
+  const dim3 per_chunk((unsigned)chunks, (unsigned)prm.Hv);
   cudaError_t e;
   if ((e = launch_k(prep_kernel<TI, DK, DV>, per_chunk, PrepSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
-  // The two chains do not depend on each other: the reverse one (a whole SM
-  // per CTA) on the high-priority internal stream, the forward one (two CTAs
-  // fit on an SM) beside it on the SMs left.
-  cudaStream_t lo = nullptr, hi = nullptr;
-  if ((e = internal_streams_fork(stream, &lo, &hi)) != cudaSuccess) return e;
-  if ((e = launch_k(rev_chain_kernel<TI, DK, DV>, per_seq, RevSmem<TI, DK, DV>::BYTES, prm, hi, NTR)) != cudaSuccess) return e;
-  if ((e = launch_k(fwd_chain_kernel<TI, DK, DV>, per_seq, FwdSmem<TI, DK, DV>::BYTES, prm, lo)) != cudaSuccess) return e;
-  if ((e = internal_streams_join(stream)) != cudaSuccess) return e;
+  const dim3 chains((unsigned)(prm.N * prm.Hv * (DV / SL + 1)));
+  if ((e = launch_k(chains_kernel<TI, DK, DV>, chains, ChainSmem<TI, DK, DV>::BYTES, prm, stream, NTR)) != cudaSuccess) return e;
   if ((e = launch_k(grads_state_kernel<TI, DK, DV>, per_chunk, StateGradSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
   return launch_k(grads_local_kernel<TI, DK, DV>, per_chunk, LocalSmem<TI, DK, DV>::BYTES, prm, stream);
 }

@@ -716,34 +716,6 @@ cudaError_t device_streams(cudaStream_t caller, DeviceStreams **out) {
 }
 }  // namespace
 
-// Fork: everything issued to `caller` so far is followed by the caller's two
-// internal streams (`lo` of the lowest, `hi` of the highest priority), for
-// work that runs beside each other.  Join: `caller` then waits for everything
-// issued to both.  (Used by the chunk-form backward for its two chains; works
-// while `caller` is being captured into a graph.)
-cudaError_t internal_streams_fork(cudaStream_t caller, cudaStream_t *lo, cudaStream_t *hi) {
-  std::lock_guard<std::mutex> lock(g_streams_mutex);
-  DeviceStreams *d = nullptr;
-  cudaError_t e;
-  if ((e = device_streams(caller, &d)) != cudaSuccess) return e;
-  if ((e = cudaEventRecord(d->start, caller)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(d->prep, d->start, 0)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(d->chain, d->start, 0)) != cudaSuccess) return e;
-  *lo = d->prep;
-  *hi = d->chain;
-  return cudaSuccess;
-}
-cudaError_t internal_streams_join(cudaStream_t caller) {
-  std::lock_guard<std::mutex> lock(g_streams_mutex);
-  DeviceStreams *d = nullptr;
-  cudaError_t e;
-  if ((e = device_streams(caller, &d)) != cudaSuccess) return e;
-  if ((e = cudaEventRecord(d->prep_done, d->prep)) != cudaSuccess) return e;
-  if ((e = cudaEventRecord(d->ev_c[0], d->chain)) != cudaSuccess) return e;
-  if ((e = cudaStreamWaitEvent(caller, d->prep_done, 0)) != cudaSuccess) return e;
-  return cudaStreamWaitEvent(caller, d->ev_c[0], 0);
-}
-
 // Plan, then per round: phase 1 (WY prep of every chunk of the round) and
 // phase 2 (state passing).  With a workspace of twophase_workspace_bytes or
 // more, rounds are pipelined: phase 1 of round r + 1 runs on the SMs phase 2

@@ -781,13 +781,15 @@ def _backward(args, D, dev, x, T, w, peaks):
             "workload": f"backward of prefill8k: T={T} Hqk={w.Hqk} Hv={w.Hv} D={w.D} bf16 inputs, "
                         "fp32 d_o and dL/dS_final, zero initial state",
             "ms_per_step": ms,
-            "roofline": {"bound": "tensor", "kernel": "chunk form: plan, prep, forward chain, reverse "
-                                                      "chain, state grads, local grads, 2 group sums",
+            "roofline": {"bound": "tensor", "kernel": "chunk form: plan, prep, both chains (one launch), "
+                                                      "state grads, local grads, 2 group sums",
                          "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
                          "frac": achieved / tf32_peak,
-                         "peak_source": "measured bf16_tflops x nominal tf32/bf16 (1.1/2.25); "
-                                        "warp-level m16n8k8 tf32 MMAs, each product issued 3 times "
-                                        "(hi/lo split)",
+                         "peak_source": "measured bf16_tflops x nominal tf32/bf16 (1.1/2.25); products "
+                                        "at about fp32 accuracy: state gradients on tcgen05 (bf16 "
+                                        "hi/lo, 3 MMAs per step), the rest warp-level (m16n8k16 "
+                                        "bf16 with an exact input operand, 2 MMAs per step; "
+                                        "m16n8k8 tf32 hi/lo, 3 per step)",
                          "algorithmic": f"{backward_chunk_flops(w.D)} flop per (64-token chunk, value head)"
                                         f" x {units} = {flop} flop",
                          "traffic": kernel_traffic("prefill_backward_chunked", bwd_sources)},
@@ -798,7 +800,7 @@ def _backward(args, D, dev, x, T, w, peaks):
                                         "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
                                         "algorithmic": f"18 D^2 flop per token and value head = {seq_flop} flop"},
                            "gpu_launches": 5 * steps},
-            "gpu_launches": 8 * steps}  # plan, 5 chunk-form kernels, 2 group sums (Hv > Hqk)
+            "gpu_launches": 7 * steps}  # plan, 4 chunk-form kernels, 2 group sums (Hv > Hqk)
 
 
 def _decode(args, D, dev, peaks, peak_src):

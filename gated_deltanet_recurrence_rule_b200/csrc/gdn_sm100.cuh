@@ -196,17 +196,6 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// D[tmem] (+)= A[tmem] * B[smem desc], tf32 inputs (fp32 bit patterns whose
-// low 13 mantissa bits are ignored), fp32 accumulate.  A in tensor memory:
-// lane i = row i, 32-bit column c = K element c; one K=8 step spans 8 columns.
-__device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p; }" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 // Arrive once on `bar` when every tcgen05 operation issued so far by this
 // thread has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -221,17 +210,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_
          | (1u << 7)                      // A format bf16
          | (1u << 10)                     // B format bf16
          | (uint32_t(neg_a) << 13)        // negate A
-         | (uint32_t(a_mn) << 15)         // A major
-         | (uint32_t(b_mn) << 16)         // B major
-         | (uint32_t(N >> 3) << 17)       // N / 8
-         | (uint32_t(M >> 4) << 24);      // M / 16
-}
-
-// Instruction descriptor of kind::tf32 with tf32 A/B and fp32 D (same fields).
-__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N, int a_mn, int b_mn) {
-  return (1u << 4)                        // D format fp32
-         | (2u << 7)                      // A format tf32
-         | (2u << 10)                     // B format tf32
          | (uint32_t(a_mn) << 15)         // A major
          | (uint32_t(b_mn) << 16)         // B major
          | (uint32_t(N >> 3) << 17)       // N / 8

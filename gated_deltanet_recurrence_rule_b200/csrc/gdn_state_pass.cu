@@ -5,7 +5,7 @@
 // Per (sequence, value head), chunk after chunk, with the state-free record of
 // each chunk already computed by phase 1 (gdn_wy_prep.cu):
 //     U^T  = U~^T - S0 W^T                     (M128 N64 K128; U~ added in the epilogue)
-//     Oi^T = S0 Q^T,   Oa^T = U^T P^T (tf32),   o_t = scale (e^{G_t} Oi_t + Oa_t)
+//     Oi^T = S0 Q^T,   Oa^T = U^T P^T,   o_t = scale (e^{G_t} Oi_t + Oa_t)
 //     dS   = (U diag(e^{G_C - G}))^T K,   S <- e^{G_C} S + dS   (fp32 master copy)
 // ("Inside Qwen3.8-27B: Hybrid DeltaNet Architecture, 256k Context, and 24GB
 // Local Serving", section "Gated DeltaNet Mechanics": o_t = S_t q_t with the
@@ -156,10 +156,10 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 enum {
   B_FULL_QK = 0, B_EMPTY_QK = B_FULL_QK + NQK, B_FULL_R = B_EMPTY_QK + NQK, B_EMPTY_R = B_FULL_R + NR,
-  // S0 hi / lo written; U ready; U (tf32) and U diag(kdec) (hi/lo) written;
+  // S0 hi / lo written; U ready; U diag(kdec) split written; U split written;
   // dS (and Oi) ready; Oa ready; the outputs of a chunk were read out of TMEM;
   // the MMA issuer's drain
-  B_S0H = B_EMPTY_R + NR, B_S0L, B_U, B_UK, B_S, B_OA, B_OFREE, B_DRAIN, NBAR
+  B_S0H = B_EMPTY_R + NR, B_S0L, B_U, B_UK, B_UO, B_S, B_OA, B_OFREE, B_DRAIN, NBAR
 };
 static_assert(NBAR * 8 <= 256, "barrier area");
 
@@ -169,13 +169,12 @@ constexpr uint32_t R_OI = 128;  // 64: S0 Q^T
 constexpr uint32_t R_OA = 192;  // 64: U^T P^T
 // MMA A operands in TMEM (bf16 pairs per column; lane = row of the operand).
 constexpr uint32_t T_S0H = 256, T_S0L = 320;  // hi/lo(S0): 128 rows x 128 K
-constexpr uint32_t T_UF = 384;                // U^T rounded to tf32: 128 rows x 64 K
+constexpr uint32_t T_UH = 384, T_UL = 416;    // hi/lo(U^T): 128 rows x 64 K
 constexpr uint32_t T_UKH = 448, T_UKL = 480;  // hi/lo(U^T diag(kdec))
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t IDESC_SW = idesc_bf16(128, 64, 0, 1, 1);  // -S0 W^T
-constexpr uint32_t IDESC_SQ = idesc_bf16(128, 64, 0, 0);     // S0 Q^T
-constexpr uint32_t IDESC_UP = idesc_tf32(128, 64, 0, 0);     // U^T P^T
+constexpr uint32_t IDESC_SQ = idesc_bf16(128, 64, 0, 0);     // S0 Q^T, U^T P^T
 constexpr uint32_t IDESC_UK = idesc_bf16(128, 128, 0, 1);    // Ukdec^T K
 
 struct Params {
@@ -238,7 +237,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (tid == 0) {
     for (int i = 0; i < NBAR; ++i) mbar_init(bar_addr(sb, i), 1);
     // barriers the 16 epilogue warps arrive on, one arrival per warp
-    for (int b : {(int)B_S0H, (int)B_S0L, (int)B_UK, (int)B_OFREE})
+    for (int b : {(int)B_S0H, (int)B_S0L, (int)B_UK, (int)B_UO, (int)B_OFREE})
       mbar_init(bar_addr(sb, b), NEPI / 32);
     // a record slot is free once its MMAs completed AND every epilogue warp read it
     for (int i = 0; i < NR; ++i) mbar_init(bar_addr(sb, B_EMPTY_R + i), 1 + NEPI / 32);
@@ -317,7 +316,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint64_t dQK0 = sdesc_sw128(sb + OFF_QK, 16, 1024);            // Q, K-major
     const uint64_t dKmn0 = sdesc_sw128(sb + OFF_QK + 8192, 16384, 1024); // K as MN-major operand
     const uint64_t dW0 = sdesc_sw128(sb + OFF_REC + tp::REC_WT, 8192, 1024);  // W^T, MN-major
-    const uint64_t dP0 = sdesc_sw128(sb + OFF_REC + tp::REC_P, 16, 1024);     // P tf32, K-major
+    const uint64_t dP0 = sdesc_sw128(sb + OFF_REC + tp::REC_PH, 16, 1024);    // P hi / lo, K-major
     auto wait = [&](int b, uint32_t parity) {
       int ok = 1;
       if (lane == 0) ok = mbar_wait(bar_addr(sb, b), parity, abort_flag);
@@ -354,8 +353,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
       }
       __syncwarp();
-      // dS = (Ukh + Ukl)^T K   (U diag(kdec) from TMEM), then Oa^T = U^T P^T in tf32
-      // (U from TMEM); the state epilogue starts when dS is done
+      // dS = (Ukh + Ukl)^T K   (U diag(kdec) from TMEM)
       if (!(ok = wait(B_UK, ph))) break;
       tc_fence_after();
       if (elect_one()) {
@@ -366,10 +364,19 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                       dKmn + ((kk * 2048) >> 4), IDESC_UK, ks > 0);
         }
         mma_commit(bar_addr(sb, B_S));
+      }
+      __syncwarp();
+      // Oa^T = Uh Ph^T + Ul Ph^T + Uh Pl^T   (U from TMEM)
+      if (!(ok = wait(B_UO, ph))) break;
+      tc_fence_after();
+      if (elect_one()) {
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks)  // K = 64 tokens in steps of 8: P block ks / 4, 32 B per step
-          mma_tf32_ts(tmem + R_OA, tmem + T_UF + 8 * ks, dP + (((ks >> 2) * 8192 + (ks & 3) * 32) >> 4),
-                      IDESC_UP, ks > 0);
+        for (int ks = 0; ks < 12; ++ks) {
+          const int part = ks % 3, kk = ks / 3;  // (Uh,Ph), (Ul,Ph), (Uh,Pl)
+          const uint32_t bo = ((part == 2 ? tp::REC_PL - tp::REC_PH : 0) + kk * 32) >> 4;
+          mma_bf16_ts(tmem + R_OA, tmem + (part == 1 ? T_UL : T_UH) + 8 * kk, dP + bo, IDESC_SQ,
+                      ks > 0);
+        }
         mma_commit(bar_addr(sb, B_OA));
         mma_commit(bar_addr(sb, B_EMPTY_QK + s));
         mma_commit(bar_addr(sb, B_EMPTY_R + sr));
@@ -466,7 +473,7 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float *gam = reinterpret_cast<const float *>(smem + OFF_REC + sr * REC_BYTES + tp::REC_SC);
       const float *kdec = gam + 64;
 
-      // ---- U = (U - U~) + U~ -> U^T rounded to tf32 for Oa, hi/lo(U^T diag(kdec)) for dS
+      // ---- U = (U - U~) + U~ -> hi/lo(U^T diag(kdec)) for dS first, then hi/lo(U^T) for Oa
       if (!(ok = warp_wait(B_U, ph))) break;
       {
         float v[16];
@@ -491,15 +498,16 @@ state_pass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tmem_st4(tl + T_UKH + 8 * ewq + 4 * hq, hw);
           tmem_st4(tl + T_UKL + 8 * ewq + 4 * hq, lw);
         }
-        // U for the Oa product, rounded to tf32 (nearest); v is dead after this
-        uint32_t uf[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) uf[x] = to_tf32(v[x]);
-        tmem_st16(tl + T_UF + 16 * ewq, uf);
+        tmem_wait_st();
+        warp_signal(B_UK);
+        store_out(0);
+        uint32_t hw[8], lw[8];
+        split_words<8>(v, hw, lw);
+        tmem_st8(tl + T_UH + 8 * ewq, hw);
+        tmem_st8(tl + T_UL + 8 * ewq, lw);
         tmem_wait_st();
       }
-      warp_signal(B_UK);
-      store_out(0);
+      warp_signal(B_UO);
       store_out(1);
 
       // ---- state: S = gamma_C S + dS (fp32); hi(S) first (the next U product), then lo(S)

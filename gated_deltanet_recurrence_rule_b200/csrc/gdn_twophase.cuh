@@ -34,8 +34,8 @@ constexpr int HD = 128;  // head dim (Dk = Dv)
 // tiles (swizzle phase taken from the row index), so one bulk copy to a
 // 1024-byte aligned shared address yields MMA-ready operands.
 constexpr uint32_t REC_WT = 0;       // W^T bf16, MN-major: 128 rows (d) x 64 t
-constexpr uint32_t REC_P = 16384;    // P as tf32 (fp32 images), K-major: two 8 KiB blocks of
-                                     // 64 rows (t) x 32 s, block b holding s in [32 b, 32 b + 32)
+constexpr uint32_t REC_PH = 16384;   // hi(P) bf16, K-major: 64 rows (t) x 64 s
+constexpr uint32_t REC_PL = 24576;   // lo(P) = bf16(P - hi(P))
 constexpr uint32_t REC_UT = 32768;   // U~ fp32 [64 t][128 d], row-major
 constexpr uint32_t REC_SC = 65536;   // fp32: gamma_t = e^{G_t} [64], kdec_t = e^{G_C - G_t} [64], e^{G_C}
 constexpr uint32_t REC_BYTES = 66560;

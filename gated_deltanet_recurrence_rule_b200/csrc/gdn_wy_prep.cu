@@ -7,7 +7,7 @@
 // 256k Context, and 24GB Local Serving", section "Gated DeltaNet Mechanics":
 // the decay alpha_t = e^{g_t} scales the whole state, beta_t the write):
 //     [Q;K] K^T                 one M128 N64 K128 MMA: rows 0-63 Q K^T, 64-127 K K^T
-//     P_ts = e^{G_t-G_s} q_t.k_s (s <= t)          -> record, rounded to tf32
+//     P_ts = e^{G_t-G_s} q_t.k_s (s <= t)          -> record, bf16 hi + lo
 //     A_ts = beta_t e^{G_t-G_s} k_t.k_s (s < t)    -> shared memory, fp32
 //     Tm = (I + A)^-1                              fp32 on CUDA cores
 //     T' = Tm diag(beta e^G),  T'' = Tm diag(beta) -> bf16 hi + lo operand tiles
@@ -324,13 +324,8 @@ wy_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
               const int si = 32 * half + 16 * qh + 8 * q + e;
               pv[e] = (si <= t && t < Lc) ? exp2f(Gt - G2[si]) * v[8 * q + e] * (rq * rkn[si]) : 0.f;
             }
-            // tf32 image, K-major: block `half` holds s in [32 half, 32 half + 32)
-#pragma unroll
-            for (int e0 = 0; e0 < 8; e0 += 4) {
-              const uint32_t off = half * 8192 + sw128_off(t, 4 * qh + 2 * q + e0 / 4);
-              *reinterpret_cast<uint4 *>(rec + tp::REC_P + off) =
-                  make_uint4(to_tf32(pv[e0]), to_tf32(pv[e0 + 1]), to_tf32(pv[e0 + 2]), to_tf32(pv[e0 + 3]));
-            }
+            const uint32_t off = sw128_off(t, 4 * half + 2 * qh + q);
+            st_split8(rec + tp::REC_PH + off, rec + tp::REC_PL + off, pv);
           }
         } else {
           const int t = row - 64;

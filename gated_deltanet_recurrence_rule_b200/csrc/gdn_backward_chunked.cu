@@ -723,34 +723,30 @@ __global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
   }
   if (tid < C) sG[tid] = p.G[u * C + tid];
   const float *S0g = p.S0 + u * DV * DK, *S1g = p.dS1 + u * DV * DK;
-  {  // A image [dO; dU]
-    constexpr int AC = DV / 8, ITEMS = 128 * AC / NT;
+  {  // A image [dO; dU] and B image S0 (MN-major: K row v, N columns k), all loads in flight at once
+    constexpr int AC = DV / 8, AI = 128 * AC / NT, BC = DK / 8, BI = DV * BC / NT;
     const float *dOc = p.dO + ((size_t)cp.start * p.Hv + h) * DV, *dUc = p.dU + u * C * DV;
     const size_t dOs = (size_t)p.Hv * DV;
-    float x[ITEMS][8];
+    float xa[AI][8], xb[BI][8];
 #pragma unroll
-    for (int it = 0; it < ITEMS; ++it) {
+    for (int it = 0; it < AI; ++it) {
       const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      ld8(r < C ? dOc + (size_t)r * dOs + 8 * c : dUc + (size_t)(r - C) * DV + 8 * c, r >= C || r < len, x[it]);
+      ld8(r < C ? dOc + (size_t)r * dOs + 8 * c : dUc + (size_t)(r - C) * DV + 8 * c, r >= C || r < len, xa[it]);
     }
 #pragma unroll
-    for (int it = 0; it < ITEMS; ++it) {
+    for (int it = 0; it < BI; ++it) {
+      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
+      ld8(S0g + (size_t)v * DK + 8 * c, true, xb[it]);
+    }
+#pragma unroll
+    for (int it = 0; it < AI; ++it) {
       const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, x[it]);
-    }
-  }
-  {  // B image S0 (MN-major: K row v, N columns k)
-    constexpr int BC = DK / 8, ITEMS = DV * BC / NT;
-    float x[ITEMS][8];
-#pragma unroll
-    for (int it = 0; it < ITEMS; ++it) {
-      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
-      ld8(S0g + (size_t)v * DK + 8 * c, true, x[it]);
+      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, xa[it]);
     }
 #pragma unroll
-    for (int it = 0; it < ITEMS; ++it) {
+    for (int it = 0; it < BI; ++it) {
       const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
-      st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, x[it]);
+      st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, xb[it]);
     }
   }
   sm100::fence_proxy_async_smem();
@@ -764,41 +760,41 @@ __global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
                            IDESC, false);
     sm100::mma_commit(bar_mma);
   }
-  cta_wait(bar_mma, 0, ctl, p.status);
-  {  // A image U (rows 0-63), B image dS1, and <dS1, S0>
-    constexpr int AC = DV / 8, ITEMS = C * AC / NT;
+  {  // U (A rows 0-63) and dS1 (B), loaded while the first product runs, stored once it is
+     // done; <dS1, S0> from the S0 image (hi + lo) each dS1 element replaces
+    constexpr int AC = DV / 8, AI = C * AC / NT, BC = DK / 8, BI = DV * BC / NT;
     const float *Uc = p.U + u * C * DV;
-    float x[ITEMS][8];
+    float xa[AI][8], xb[BI][8];
 #pragma unroll
-    for (int it = 0; it < ITEMS; ++it) {
+    for (int it = 0; it < AI; ++it) {
       const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      ld8(Uc + (size_t)r * DV + 8 * c, true, x[it]);
+      ld8(Uc + (size_t)r * DV + 8 * c, true, xa[it]);
     }
 #pragma unroll
-    for (int it = 0; it < ITEMS; ++it) {
-      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, x[it]);
+    for (int it = 0; it < BI; ++it) {
+      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
+      ld8(S1g + (size_t)v * DK + 8 * c, true, xb[it]);
     }
-  }
-  {
-    constexpr int BC = DK / 8, ITEMS = DV * BC / NT, HALF = ITEMS / 2 > 0 ? ITEMS / 2 : 1;
+    cta_wait(bar_mma, 0, ctl, p.status);
+#pragma unroll
+    for (int it = 0; it < AI; ++it) {
+      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
+      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, xa[it]);
+    }
     float dot = 0.f;
 #pragma unroll
-    for (int part = 0; part < ITEMS / HALF; ++part) {
-      float x[HALF][8], y[HALF][8];
+    for (int it = 0; it < BI; ++it) {
+      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
+      const uint32_t off = sm100::sw128_off((uint32_t)v, (uint32_t)(c & 7)) + (c >> 3) * L::B_LBO;
+      const uint4 hv = *reinterpret_cast<const uint4 *>(BH + off), lv = *reinterpret_cast<const uint4 *>(BL + off);
+      const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-      for (int it = 0; it < HALF; ++it) {
-        const int idx = tid + NT * (part * HALF + it), v = idx / BC, c = idx % BC;
-        ld8(S1g + (size_t)v * DK + 8 * c, true, x[it]);
-        ld8(S0g + (size_t)v * DK + 8 * c, true, y[it]);
+      for (int e = 0; e < 4; ++e) {
+        const float s0a = __uint_as_float(hw[e] << 16) + __uint_as_float(lw[e] << 16);
+        const float s0b = __uint_as_float(hw[e] & 0xffff0000u) + __uint_as_float(lw[e] & 0xffff0000u);
+        dot = fmaf(xb[it][2 * e], s0a, fmaf(xb[it][2 * e + 1], s0b, dot));
       }
-#pragma unroll
-      for (int it = 0; it < HALF; ++it) {
-        const int idx = tid + NT * (part * HALF + it), v = idx / BC, c = idx % BC;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) dot = fmaf(x[it][e], y[it][e], dot);
-        st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, x[it]);
-      }
+      st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, xb[it]);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);

@@ -65,7 +65,9 @@ __device__ __forceinline__ void st_frag16x8(float *M, int ld, const float *d, fl
 // Off-diagonal 16x16 blocks at block distance DIST (1..3) of the inverse: for
 // the 4 - DIST blocks (i, j = i - DIST), Y_ij = sum_{j<=k<i} A_ik Tm_kj (one
 // 16 x 16 DIST x 16 product), then Tm_ij = -Tm_ii Y_ij (16 x 16 x 16).  One warp
-// per (block, 8-column half); NT threads (>= 192) meet at named barrier BAR.
+// per (block, 8-column half): the second product reads only the 8 columns of
+// Y_ij the same warp wrote, so a warp barrier separates the two; NT threads
+// (>= 192) meet at named barrier BAR once the distance is done.
 template <int DIST, int NT, int BAR>
 __device__ __forceinline__ void ut_distance(const float *__restrict__ A, float *__restrict__ Tm,
                                             float *__restrict__ Y, int etid) {
@@ -76,13 +78,10 @@ __device__ __forceinline__ void ut_distance(const float *__restrict__ A, float *
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     mma3_16x8<2 * DIST>(d, A + 16 * i * AST + 16 * j, AST, Tm + 16 * j * AST + 16 * j + 8 * nh, AST, lane);
     st_frag16x8(Y + (j * 16) * 17 + 8 * nh, 17, d, 1.f, lane);
-  }
-  named_bar_sync(BAR, NT);
-  if (w < 2 * NB) {
-    const int j = w >> 1, i = j + DIST, nh = w & 1;
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-    mma3_16x8<2>(d, Tm + 16 * i * AST + 16 * i, AST, Y + (j * 16) * 17 + 8 * nh, 17, lane);
-    st_frag16x8(Tm + 16 * i * AST + 16 * j + 8 * nh, AST, d, -1.f, lane);
+    __syncwarp();
+    float e[4] = {0.f, 0.f, 0.f, 0.f};
+    mma3_16x8<2>(e, Tm + 16 * i * AST + 16 * i, AST, Y + (j * 16) * 17 + 8 * nh, 17, lane);
+    st_frag16x8(Tm + 16 * i * AST + 16 * j + 8 * nh, AST, e, -1.f, lane);
   }
   named_bar_sync(BAR, NT);
 }
@@ -93,7 +92,8 @@ __device__ __forceinline__ void ut_distance(const float *__restrict__ A, float *
 // by one group of lanes that hold its rows (NT = 512: 8 lanes x 2 rows; NT =
 // 256: 4 lanes x 4 rows; A read from shared memory), the solved entry of
 // step s passed by a shuffle.  Then the off-diagonal blocks by
-// block distance 1, 2, 3 (each needs only blocks of smaller distance).  Only
+// block distance 1, 2, 3 (each needs only blocks of smaller distance), one
+// block-wide barrier per distance.  Only
 // the lower triangle of Tm is written.  Y holds [3][16][17] fp32 of scratch.
 template <int NT, int BAR>
 __device__ __forceinline__ void ut_solve(const float *__restrict__ A, float *__restrict__ Tm,

@@ -363,8 +363,12 @@ size_t gdn_prefill_backward_workspace_size_sequential(int32_t num_seqs, int64_t 
  *     then every chunk on its own: dQ, dK, dV, dbeta and dG through the
  *     products of the WY/UT transform (dA = -Tm^T dT Tm^T) and dg as suffix
  *     sums of dG within the chunk.  The dense products run on tensor cores
- *     (tf32 with a 3-term hi/lo split of both operands, about fp32
- *     accuracy).  g is clamped at -30 as in the tensor-core prefill.
+ *     at about fp32 accuracy: fp32 operands split into hi and lo parts and
+ *     three products (hi*hi + hi*lo + lo*hi), raw bf16 inputs used as they
+ *     are; the products with the chunk states on tcgen05, the rest as
+ *     warp-level MMAs.  g is clamped at -30 as in the tensor-core prefill.
+ *     The forward and reverse chains run in one launch; the call is
+ *     stream-ordered on `stream` (it can be captured in a CUDA graph).
  *   - sequential (at least gdn_prefill_backward_workspace_size_sequential
  *     bytes): the token-by-token rule on CUDA cores.  With u = S_{t-1} k_t,
  *     w = v_t - alpha_t u and G = dL/dS_t, going backwards over the tokens:

@@ -96,6 +96,27 @@ def test_backward_mixed_dims(algo):
         _check(out, ref, f"{algo} Dk={Dk} Dv={Dv}")
 
 
+@pytest.mark.parametrize("Dk,Dv", [(128, 64), (64, 128)])
+def test_backward_mixed_dims_gqa(Dk, Dv, algo):
+    """Dk != Dv with 3 value heads per query/key head (dq, dk summed over each
+    group), bf16 inputs, chunk boundaries inside both sequences."""
+    inp = inputs.prefill_inputs([150, 64], 1, 3, Dk, dtype="bf16", seed=151, init_std=0.1)
+    gen = torch.Generator().manual_seed(152)
+    T = 214
+    v = torch.randn(T, 3, Dv, generator=gen).to(torch.bfloat16)
+    s0 = torch.randn(2, 3, Dv, Dk, generator=gen) * 0.1
+    d_o = torch.randn(T, 3, Dv, generator=gen)
+    d_sf = torch.randn(2, 3, Dv, Dk, generator=gen) * 0.1
+    out = api.prefill_backward(inp["q"].to(DEV), inp["k"].to(DEV), v.to(DEV), inp["g"].to(DEV),
+                               inp["beta"].to(DEV), d_o.to(DEV), cu_seqlens=inp["cu_seqlens"].to(DEV),
+                               initial_state=s0.to(DEV), d_final_state=d_sf.to(DEV), scale=0.7,
+                               sequential=algo == "sequential")
+    torch.cuda.synchronize()
+    ref = oracle.backward(inp["q"], inp["k"], v, inp["g"], inp["beta"], d_o, cu_seqlens=inp["cu_seqlens"],
+                          initial_state=s0, d_final_state=d_sf, scale=0.7)
+    _check(out, ref, f"{algo} GQA Dk={Dk} Dv={Dv}")
+
+
 def test_backward_without_states(algo):
     """No initial state and no final-state gradient (both NULL)."""
     out, ref = _case([70], 1, 3, 64, "fp32", seed=107, algo=algo, init=False, dsf=False, scale=1.0)

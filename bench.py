@@ -782,7 +782,7 @@ def _backward(args, D, dev, x, T, w, peaks):
                         "fp32 d_o and dL/dS_final, zero initial state",
             "ms_per_step": ms,
             "roofline": {"bound": "tensor", "kernel": "chunk form: plan, prep, both chains (one launch), "
-                                                      "state grads, local grads, 2 group sums",
+                                                      "state grads, local grads (dq, dk summed in it)",
                          "achieved": achieved, "peak": tf32_peak, "unit": "TFLOP/s",
                          "frac": achieved / tf32_peak,
                          "peak_source": "measured bf16_tflops x nominal tf32/bf16 (1.1/2.25); products "
@@ -800,7 +800,7 @@ def _backward(args, D, dev, x, T, w, peaks):
                                         "peak_source": "148 SMs x 128 fp32 FMA/clk x 2 x max SM clock",
                                         "algorithmic": f"18 D^2 flop per token and value head = {seq_flop} flop"},
                            "gpu_launches": 5 * steps},
-            "gpu_launches": 7 * steps}  # plan, 4 chunk-form kernels, 2 group sums (Hv > Hqk)
+            "gpu_launches": 5 * steps}  # plan, prep, chains, state grads, local grads
 
 
 def _decode(args, D, dev, peaks, peak_src):

@@ -355,16 +355,6 @@ __global__ void group_sum_kernel(const float *__restrict__ part, float *__restri
 
 }  // namespace bwd
 
-// out[r][d] = sum of the `width` partial rows of group r (see group_sum_kernel).
-cudaError_t launch_group_sum(const float *part, float *out, size_t rows, int width, int inner,
-                             cudaStream_t stream) {
-  const size_t total = rows * (size_t)inner;
-  if (total == 0) return cudaSuccess;
-  const unsigned blocks = (unsigned)std::min<size_t>((total + 255) / 256, 148 * 16);
-  bwd::group_sum_kernel<<<blocks, 256, 0, stream>>>(part, out, rows, width, inner);
-  return cudaGetLastError();
-}
-
 // Slices per (sequence, value head): doubled, down to 32 rows per CTA, until
 // the grid has two CTAs per SM of a B200 (148 SMs).  A function of the sizes
 // only, so the workspace query and the launch agree.

@@ -40,9 +40,9 @@
 //                d_initial_state), then per (sequence, value head) the
 //                forward one (the state at every chunk start S0, and U)
 //   grads_state  per (chunk, value head): the products with S0 and dS1
-//   grads_local  per (chunk, value head): the 64 x 64 algebra, then dq, dk
-//                (per value head), dv, dg, dbeta
-//   group sums   dq, dk over the value heads of each query/key head
+//   grads_local  per (chunk, query/key head), its value heads in turn: the
+//                64 x 64 algebra, dv, dg, dbeta, and dq, dk summed over the
+//                group in registers (fixed order)
 // Rows of S and of dS evolve independently (the chains never mix rows), so a
 // reverse-chain CTA owns 64 of the Dv rows.  Tiles move global -> shared with
 // cp.async, all of a step's copies in flight at once, and the chains fetch a
@@ -64,8 +64,6 @@ namespace gdn {
 cudaError_t launch_plan(const int32_t *cu, int N, int T, int Hv, const void *s0, void *sfin,
                         size_t state_bytes, tp::PlanHeader *ph, int32_t *ne_seq, int32_t *ne_cs,
                         int32_t *status, cudaStream_t stream);
-cudaError_t launch_group_sum(const float *part, float *out, size_t rows, int width, int inner,
-                             cudaStream_t stream);
 
 namespace cbwd {
 
@@ -83,7 +81,7 @@ struct Params {
   int N, T, Hqk, Hv;
   float scale;
   const float *s0, *dO, *dSf;
-  float *dq, *dk;  // outputs, or per-value-head partials [T, Hv, Dk] when Hv > Hqk
+  float *dq, *dk;  // [T, Hqk, Dk] outputs
   float *dv, *dg, *dbeta, *ds0;
   const tp::PlanHeader *ph;
   const int32_t *ne_seq, *ne_cs;
@@ -922,205 +920,215 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   const int gid = lane >> 2, tig = lane & 3;
   ChunkPos cp;
   if (!chunk_pos(p, blockIdx.x, cp)) return;
-  const int h = blockIdx.y, Gq = p.Hv / p.Hqk, hk = h / Gq;
-  const size_t u = (size_t)blockIdx.x * p.Hv + h;
+  const int hk = blockIdx.y, Gq = p.Hv / p.Hqk;
   const int len = cp.len;
   const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k),
            *v = static_cast<const TI *>(p.v);
   const size_t qoff = ((size_t)cp.start * p.Hqk + hk) * DK, qstride = (size_t)p.Hqk * DK;
   const float scale = p.scale;
-  tile_async<C, DV>(RA, L::LA, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
-  tile_async<C, DV>(RB, L::LB, p.U + u * C * DV, DV, C, tid);
-  tile_async<C, C>(S1, LD64, p.P + u * C * C, C, C, tid);
-  tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
-  cp_commit();
-  tile_async<C, DK>(RC, L::LC, k + qoff, qstride, len, tid);
-  tile_async<C, DV>(RD, L::LD, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
-  tile_async<C, C>(S3, LD64, p.Tm + u * C * C, C, C, tid);
-  cp_commit();
-  if (tid < C) sB[tid] = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
-  cp_wait<1>();
-  __syncthreads();
-  if (tid < C) {
-    sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
-    sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
-  }
   const int r0 = 16 * (w & 3), half = w >> 2, c64 = 32 * half;
-  {  // step 1: dP = lower(dO' U^T); S2 = dP . E, S1 = dP . P
-    float acc[4][4];
-    zero_acc(acc);
-    mma3_rows<DV>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
-                      [&](int r, int c) { return RB[(c64 + c) * L::LB + r]; }, lane);
-    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) {
-      const float dp = i >= j ? scale * x : 0.f;
-      S2[i * LD64 + j] = i >= j ? dp * expf((float)(sG[i] - sG[j])) : 0.f;
-      S1[i * LD64 + j] = dp * S1[i * LD64 + j];
-    });
-  }
-  __syncthreads();
-  tile_async<C, DK>(RA, L::LA, p.dW + u * C * DK, DK, C, tid);
-  tile_async<C, DV>(RB, L::LB, p.dU + u * C * DV, DV, C, tid);
-  cp_commit();
-  cp_wait<0>();
-  __syncthreads();
-  {  // step 2: dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T -> S4
-    // (dW K^T and dU V^T with the raw inputs, then the column scales)
-    constexpr bool EX = sizeof(TI) == 2;
-    float a1[4][4], a2[4][4];
-    zero_acc(a1);
-    zero_acc(a2);
-    mma3_rows<DK, 4, false, EX>(a1, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
-                                     [&](int r, int c) { return to_f32(RC[(c64 + c) * L::LC + r]); }, lane);
-    mma3_rows<DV, 4, false, EX>(a2, [&](int r, int c) { return RB[(r0 + r) * L::LB + c]; },
-                                     [&](int r, int c) { return to_f32(RD[(c64 + c) * L::LD + r]); }, lane);
-    const int tig = lane & 3;
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = r0 + gid + 8 * (e >> 1), j = c64 + 8 * t + 2 * tig + (e & 1);
-        S4[i * LD64 + j] = sB[j] * (sGm[j] * a1[t][e] + a2[t][e]);
-      }
-  }
   const int cbk = half * (DK / 2), cbv = half * (DV / 2);
-  float dK[DK / 16][4];
-  {  // X = Tm^T dW
-    zero_acc(dK);
-    mma3_rows<C>(dK, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
-                     [&](int r, int c) { return RA[r * L::LA + cbk + c]; }, lane);
-    float slo, shi;
-    quad_row_sums(dK, [&](int i, int c) { return to_f32(RC[i * L::LC + c]); }, r0, cbk, lane, slo, shi);
-    if (tig == 0) { sXK[half * C + r0 + gid] = slo; sXK[half * C + r0 + gid + 8] = shi; }
-    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x *= sB[i] * sGm[i]; });
-  }
-  {  // Y = Tm^T dU: dv = diag(beta) Y
-    float acc[DV / 16][4];
-    zero_acc(acc);
-    mma3_rows<C>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
-                     [&](int r, int c) { return RB[r * L::LB + cbv + c]; }, lane);
-    float slo, shi;
-    quad_row_sums(acc, [&](int i, int c) { return to_f32(RD[i * L::LD + c]); }, r0, cbv, lane, slo, shi);
-    if (tig == 0) { sYV[half * C + r0 + gid] = slo; sYV[half * C + r0 + gid + 8] = shi; }
-    float *dv = p.dv + ((size_t)cp.start * p.Hv + h) * DV;
-    for_frag(acc, r0, cbv, lane, [&](int i, int c, float &x) {
-      if (i < len) dv[(size_t)i * p.Hv * DV + c] = sB[i] * x;
-    });
-  }
-  __syncthreads();
-  tile_async<C, DK>(RD, L::LD, q + qoff, qstride, len, tid);  // V is no longer needed
-  cp_commit();
-  {  // Z = dT Tm^T -> S5
-    float acc[4][4];
-    zero_acc(acc);
-    mma3_rows<C>(acc, [&](int r, int c) { return S4[(r0 + r) * LD64 + c]; },
-                     [&](int r, int c) { return S3[(c64 + c) * LD64 + r]; }, lane);
-    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S5[i * LD64 + j] = x; });
-  }
-  __syncthreads();
-  {  // dA = strict_lower(-Tm^T Z) -> S4
-    float acc[4][4];
-    zero_acc(acc);
-    mma3_rows<C>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
-                     [&](int r, int c) { return S5[r * LD64 + c64 + c]; }, lane);
-    for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = i > j ? -x : 0.f; });
-  }
-  __syncthreads();
-  tile_async<C, C>(S5, LD64, p.EKK + u * C * C, C, C, tid);
-  cp_commit();
-  cp_wait<0>();
-  __syncthreads();
-  // S4 <- B = diag(beta) (dA . E); S5 <- dA . (E . K K^T)
-  for (int x = tid; x < C * C; x += NT) {
-    const int i = x >> 6, j = x & 63;
-    const float da = S4[i * LD64 + j];
-    S4[i * LD64 + j] = i > j ? sB[i] * da * expf((float)(sG[i] - sG[j])) : 0.f;
-    S5[i * LD64 + j] = da * S5[i * LD64 + j];
-  }
-  __syncthreads();
-  if (tid < C) {  // row sums
-    float a = 0.f, b = 0.f;
-    for (int j = 0; j < C; ++j) { a += S1[tid * LD64 + j]; b += S5[tid * LD64 + j]; }
-    sRP[tid] = a;
-    sRM[tid] = b;
-  } else if (tid < 2 * C) {  // column sums
-    const int j = tid - C;
-    float a = 0.f, b = 0.f;
-    for (int i = 0; i < C; ++i) { a += S1[i * LD64 + j]; b += sB[i] * S5[i * LD64 + j]; }
-    sCP[j] = a;
-    sCM[j] = b;
-  }
-  {  // dq (this value head's part) = diag(gamma) dO' S0 + (dP . E) K
-    float acc[DK / 16][4];
-    const float *dQp = p.dQp + u * C * DK;
-    for_frag(acc, r0, cbk, lane, [&](int i, int c, float &x) { x = dQp[i * DK + c]; });
-    mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(acc, [&](int r, int c) { return S2[(r0 + r) * LD64 + c]; },
-                     [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
-    const bool direct = Gq == 1;
-    float *dst = direct ? p.dq + qoff : p.dq + ((size_t)cp.start * p.Hv + h) * DK;
-    const size_t rs = direct ? qstride : (size_t)p.Hv * DK;
-    for_frag(acc, r0, cbk, lane, [&](int i, int c, float &x) {
-      if (i < len) dst[(size_t)i * rs + c] = x;
-    });
-  }
-  {  // dk = diag(kdec) U dS1 + diag(beta gamma) X + (dP . E)^T Q + (B + B^T) K
-    const float *dKp = p.dKp + u * C * DK;
-    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x += dKp[i * DK + c]; });
-    mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S2[c * LD64 + r0 + r]; },
-                     [&](int r, int c) { return to_f32(RD[r * L::LD + cbk + c]); }, lane);
-    mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S4[(r0 + r) * LD64 + c] + S4[c * LD64 + r0 + r]; },
-                     [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
-    const bool direct = Gq == 1;
-    float *dst = direct ? p.dk + qoff : p.dk + ((size_t)cp.start * p.Hv + h) * DK;
-    const size_t rs = direct ? qstride : (size_t)p.Hv * DK;
-    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) {
-      if (i < len) dst[(size_t)i * rs + c] = x;
-    });
-  }
-  __syncthreads();
-  if (w == 0) {  // dG, then dg (suffix sums) and dbeta; two tokens per lane
-    const float *sc = p.sc + u * 3 * C;
-    const float dgC = sc[2 * C];
-    float dG[2], db[2], kk2 = 0.f;
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int i = 2 * lane + e;
-      const float xk = sXK[i] + sXK[C + i], yv = sYV[i] + sYV[C + i];
-      const float dgam = sc[i] + sB[i] * xk, dkd = sc[C + i];
-      db[e] = sGm[i] * xk + yv + sRM[i];
-      dG[e] = (sRP[i] - sCP[i]) + (sB[i] * sRM[i] - sCM[i]) + dgam * sGm[i] - dkd * sKd[i];
-      kk2 += dkd * sKd[i];
+  // dq and dk of the query/key head: the value heads of its group add their
+  // parts in order, in registers
+  float dQ[DK / 16][4], dK[DK / 16][4];
+  zero_acc(dQ);
+  zero_acc(dK);
+  for (int gi = 0; gi < Gq; ++gi) {
+    const int h = hk * Gq + gi;
+    const size_t u = (size_t)blockIdx.x * p.Hv + h;
+    tile_async<C, DV>(RA, L::LA, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
+    tile_async<C, DV>(RB, L::LB, p.U + u * C * DV, DV, C, tid);
+    tile_async<C, C>(S1, LD64, p.P + u * C * C, C, C, tid);
+    tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+    cp_commit();
+    if (gi == 0) tile_async<C, DK>(RC, L::LC, k + qoff, qstride, len, tid);  // K serves the group
+    tile_async<C, DV>(RD, L::LD, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
+    tile_async<C, C>(S3, LD64, p.Tm + u * C * C, C, C, tid);
+    cp_commit();
+    if (tid < C) sB[tid] = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
+    cp_wait<1>();
+    __syncthreads();
+    if (tid < C) {
+      sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
+      sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) kk2 += __shfl_xor_sync(0xffffffffu, kk2, off);
-    const float gC = expf((float)sG[len - 1]);
-#pragma unroll
-    for (int e = 0; e < 2; ++e)
-      if (2 * lane + e == len - 1) dG[e] += kk2 + dgC * gC;
-    // suffix sums over the chunk's tokens (rows >= len hold zeros)
-    float s = dG[0] + dG[1];
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const float x = __shfl_down_sync(0xffffffffu, s, off);
-      if (lane + off < 32) s += x;
+    {  // step 1: dP = lower(dO' U^T); S2 = dP . E, S1 = dP . P
+      float acc[4][4];
+      zero_acc(acc);
+      mma3_rows<DV>(acc, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
+                        [&](int r, int c) { return RB[(c64 + c) * L::LB + r]; }, lane);
+      for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) {
+        const float dp = i >= j ? scale * x : 0.f;
+        S2[i * LD64 + j] = i >= j ? dp * expf((float)(sG[i] - sG[j])) : 0.f;
+        S1[i * LD64 + j] = dp * S1[i * LD64 + j];
+      });
     }
-    const float sf[2] = {s, s - dG[0]};  // suffix from token 2 lane, from 2 lane + 1
+    __syncthreads();
+    tile_async<C, DK>(RA, L::LA, p.dW + u * C * DK, DK, C, tid);
+    tile_async<C, DV>(RB, L::LB, p.dU + u * C * DV, DV, C, tid);
+    cp_commit();
+    cp_wait<0>();
+    __syncthreads();
+    {  // step 2: dT = dW (diag(beta gamma) K)^T + dU (diag(beta) V)^T -> S4
+      // (dW K^T and dU V^T with the raw inputs, then the column scales)
+      constexpr bool EX = sizeof(TI) == 2;
+      float a1[4][4], a2[4][4];
+      zero_acc(a1);
+      zero_acc(a2);
+      mma3_rows<DK, 4, false, EX>(a1, [&](int r, int c) { return RA[(r0 + r) * L::LA + c]; },
+                                       [&](int r, int c) { return to_f32(RC[(c64 + c) * L::LC + r]); }, lane);
+      mma3_rows<DV, 4, false, EX>(a2, [&](int r, int c) { return RB[(r0 + r) * L::LB + c]; },
+                                       [&](int r, int c) { return to_f32(RD[(c64 + c) * L::LD + r]); }, lane);
+      const int tig = lane & 3;
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int i = 2 * lane + e;
-      if (i < len) {
-        p.dg[(size_t)(cp.start + i) * p.Hv + h] = sf[e];
-        p.dbeta[(size_t)(cp.start + i) * p.Hv + h] = db[e];
+      for (int t = 0; t < 4; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = r0 + gid + 8 * (e >> 1), j = c64 + 8 * t + 2 * tig + (e & 1);
+          S4[i * LD64 + j] = sB[j] * (sGm[j] * a1[t][e] + a2[t][e]);
+        }
+    }
+    {  // X = Tm^T dW; dK += diag(beta gamma) X
+      float xa[DK / 16][4];
+      zero_acc(xa);
+      mma3_rows<C>(xa, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+                       [&](int r, int c) { return RA[r * L::LA + cbk + c]; }, lane);
+      float slo, shi;
+      quad_row_sums(xa, [&](int i, int c) { return to_f32(RC[i * L::LC + c]); }, r0, cbk, lane, slo, shi);
+      if (tig == 0) { sXK[half * C + r0 + gid] = slo; sXK[half * C + r0 + gid + 8] = shi; }
+#pragma unroll
+      for (int t = 0; t < DK / 16; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = r0 + gid + 8 * (e >> 1);
+          dK[t][e] = fmaf(sB[i] * sGm[i], xa[t][e], dK[t][e]);
+        }
+    }
+    {  // Y = Tm^T dU: dv = diag(beta) Y
+      float acc[DV / 16][4];
+      zero_acc(acc);
+      mma3_rows<C>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+                       [&](int r, int c) { return RB[r * L::LB + cbv + c]; }, lane);
+      float slo, shi;
+      quad_row_sums(acc, [&](int i, int c) { return to_f32(RD[i * L::LD + c]); }, r0, cbv, lane, slo, shi);
+      if (tig == 0) { sYV[half * C + r0 + gid] = slo; sYV[half * C + r0 + gid + 8] = shi; }
+      float *dv = p.dv + ((size_t)cp.start * p.Hv + h) * DV;
+      for_frag(acc, r0, cbv, lane, [&](int i, int c, float &x) {
+        if (i < len) dv[(size_t)i * p.Hv * DV + c] = sB[i] * x;
+      });
+    }
+    __syncthreads();
+    tile_async<C, DK>(RD, L::LD, q + qoff, qstride, len, tid);  // V is no longer needed
+    cp_commit();
+    {  // Z = dT Tm^T -> S5
+      float acc[4][4];
+      zero_acc(acc);
+      mma3_rows<C>(acc, [&](int r, int c) { return S4[(r0 + r) * LD64 + c]; },
+                       [&](int r, int c) { return S3[(c64 + c) * LD64 + r]; }, lane);
+      for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S5[i * LD64 + j] = x; });
+    }
+    __syncthreads();
+    {  // dA = strict_lower(-Tm^T Z) -> S4
+      float acc[4][4];
+      zero_acc(acc);
+      mma3_rows<C>(acc, [&](int r, int c) { return S3[c * LD64 + r0 + r]; },
+                       [&](int r, int c) { return S5[r * LD64 + c64 + c]; }, lane);
+      for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = i > j ? -x : 0.f; });
+    }
+    __syncthreads();
+    tile_async<C, C>(S5, LD64, p.EKK + u * C * C, C, C, tid);
+    cp_commit();
+    cp_wait<0>();
+    __syncthreads();
+    // S4 <- B = diag(beta) (dA . E); S5 <- dA . (E . K K^T)
+    for (int x = tid; x < C * C; x += NT) {
+      const int i = x >> 6, j = x & 63;
+      const float da = S4[i * LD64 + j];
+      S4[i * LD64 + j] = i > j ? sB[i] * da * expf((float)(sG[i] - sG[j])) : 0.f;
+      S5[i * LD64 + j] = da * S5[i * LD64 + j];
+    }
+    __syncthreads();
+    if (tid < C) {  // row sums
+      float a = 0.f, b = 0.f;
+      for (int j = 0; j < C; ++j) { a += S1[tid * LD64 + j]; b += S5[tid * LD64 + j]; }
+      sRP[tid] = a;
+      sRM[tid] = b;
+    } else if (tid < 2 * C) {  // column sums
+      const int j = tid - C;
+      float a = 0.f, b = 0.f;
+      for (int i = 0; i < C; ++i) { a += S1[i * LD64 + j]; b += sB[i] * S5[i * LD64 + j]; }
+      sCP[j] = a;
+      sCM[j] = b;
+    }
+    {  // dq += diag(gamma) dO' S0 + (dP . E) K (this value head's parts)
+      const float *dQp = p.dQp + u * C * DK;
+      for_frag(dQ, r0, cbk, lane, [&](int i, int c, float &x) { x += dQp[i * DK + c]; });
+      mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dQ, [&](int r, int c) { return S2[(r0 + r) * LD64 + c]; },
+                       [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
+    }
+    {  // dk += diag(kdec) U dS1 + (dP . E)^T Q + (B + B^T) K (diag(beta gamma) X is in already)
+      const float *dKp = p.dKp + u * C * DK;
+      for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x += dKp[i * DK + c]; });
+      mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S2[c * LD64 + r0 + r]; },
+                       [&](int r, int c) { return to_f32(RD[r * L::LD + cbk + c]); }, lane);
+      mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S4[(r0 + r) * LD64 + c] + S4[c * LD64 + r0 + r]; },
+                       [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
+    }
+    __syncthreads();
+    if (w == 0) {  // dG, then dg (suffix sums) and dbeta; two tokens per lane
+      const float *sc = p.sc + u * 3 * C;
+      const float dgC = sc[2 * C];
+      float dG[2], db[2], kk2 = 0.f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = 2 * lane + e;
+        const float xk = sXK[i] + sXK[C + i], yv = sYV[i] + sYV[C + i];
+        const float dgam = sc[i] + sB[i] * xk, dkd = sc[C + i];
+        db[e] = sGm[i] * xk + yv + sRM[i];
+        dG[e] = (sRP[i] - sCP[i]) + (sB[i] * sRM[i] - sCM[i]) + dgam * sGm[i] - dkd * sKd[i];
+        kk2 += dkd * sKd[i];
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) kk2 += __shfl_xor_sync(0xffffffffu, kk2, off);
+      const float gC = expf((float)sG[len - 1]);
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (2 * lane + e == len - 1) dG[e] += kk2 + dgC * gC;
+      // suffix sums over the chunk's tokens (rows >= len hold zeros)
+      float s = dG[0] + dG[1];
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const float x = __shfl_down_sync(0xffffffffu, s, off);
+        if (lane + off < 32) s += x;
+      }
+      const float sf[2] = {s, s - dG[0]};  // suffix from token 2 lane, from 2 lane + 1
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int i = 2 * lane + e;
+        if (i < len) {
+          p.dg[(size_t)(cp.start + i) * p.Hv + h] = sf[e];
+          p.dbeta[(size_t)(cp.start + i) * p.Hv + h] = db[e];
+        }
       }
     }
+    __syncthreads();  // the next value head reuses every buffer but K
+  }
+  {  // dq and dk of the query/key head
+    float *dq = p.dq + qoff, *dk = p.dk + qoff;
+    for_frag(dQ, r0, cbk, lane, [&](int i, int c, float &x) {
+      if (i < len) dq[(size_t)i * qstride + c] = x;
+    });
+    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) {
+      if (i < len) dk[(size_t)i * qstride + c] = x;
+    });
   }
 }
 
 }  // namespace cbwd
 
-// Chunk-form backward workspace: header and plan, then the per-unit arrays,
-// then the per-value-head dq, dk partials when Hv > Hqk.
+// Chunk-form backward workspace: header and plan, then the per-unit arrays.
 struct CbwdLayout {
-  size_t plan, Tm, P, EKK, W, dQp, dKp, dW, Ut, U, dU, S0, dS1, G, sc, dqh, dkh, total;
+  size_t plan, Tm, P, EKK, W, dQp, dKp, dW, Ut, U, dU, S0, dS1, G, sc, total;
 };
 
 static CbwdLayout cbwd_layout(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int Dv) {
@@ -1143,11 +1151,6 @@ static CbwdLayout cbwd_layout(int64_t N, int64_t T, int Hqk, int Hv, int Dk, int
   L.dS1 = o;   o += up(units * (size_t)Dv * Dk * f);
   L.G = o;     o += up(units * C * sizeof(double));
   L.sc = o;    o += up(units * 3 * C * f);
-  L.dqh = L.dkh = 0;
-  if (Hv != Hqk) {
-    L.dqh = o; o += up((size_t)T * Hv * Dk * f);
-    L.dkh = o; o += up((size_t)T * Hv * Dk * f);
-  }
   L.total = o;
   return L;
 }
@@ -1177,7 +1180,8 @@ cudaError_t run_chunked(const cbwd::Params &prm, int64_t chunks, cudaStream_t st
   const dim3 chains((unsigned)(prm.N * prm.Hv * (DV / SL + 1)));
   if ((e = launch_k(chains_kernel<TI, DK, DV>, chains, ChainSmem<TI, DK, DV>::BYTES, prm, stream, NTR)) != cudaSuccess) return e;
   if ((e = launch_k(grads_state_kernel<TI, DK, DV>, per_chunk, StateGradSmem<DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
-  return launch_k(grads_local_kernel<TI, DK, DV>, per_chunk, LocalSmem<TI, DK, DV>::BYTES, prm, stream);
+  const dim3 per_group((unsigned)chunks, (unsigned)prm.Hqk);
+  return launch_k(grads_local_kernel<TI, DK, DV>, per_group, LocalSmem<TI, DK, DV>::BYTES, prm, stream);
 }
 
 template <typename TI>
@@ -1210,8 +1214,8 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
   prm.q = q; prm.k = k; prm.v = v; prm.g = g; prm.beta = beta; prm.cu = cu;
   prm.N = N; prm.T = T; prm.Hqk = Hqk; prm.Hv = Hv; prm.scale = scale;
   prm.s0 = s0; prm.dO = dO; prm.dSf = dSfin;
-  prm.dq = Hv == Hqk ? dq : F(L.dqh);
-  prm.dk = Hv == Hqk ? dk : F(L.dkh);
+  prm.dq = dq;
+  prm.dk = dk;
   prm.dv = dv; prm.dg = dg; prm.dbeta = dbeta; prm.ds0 = ds0;
   prm.ph = ph; prm.ne_seq = ne_seq; prm.ne_cs = ne_cs;
   prm.Tm = F(L.Tm); prm.P = F(L.P); prm.EKK = F(L.EKK);
@@ -1223,13 +1227,7 @@ cudaError_t launch_backward_chunked(const void *q, const void *k, const void *v,
   const int64_t chunks = tp::chunk_bound(N, T);
   e = dtype == GDN_DTYPE_BF16 ? run_chunked_dims<__nv_bfloat16>(prm, Dk, Dv, chunks, stream)
                               : run_chunked_dims<float>(prm, Dk, Dv, chunks, stream);
-  if (e != cudaSuccess) return e;
-  if (Hv != Hqk) {
-    const size_t rows_qk = (size_t)T * Hqk;
-    if ((e = launch_group_sum(prm.dq, dq, rows_qk, Hv / Hqk, Dk, stream)) != cudaSuccess) return e;
-    if ((e = launch_group_sum(prm.dk, dk, rows_qk, Hv / Hqk, Dk, stream)) != cudaSuccess) return e;
-  }
-  return cudaSuccess;
+  return e;
 }
 
 }  // namespace gdn

@@ -322,9 +322,8 @@ int32_t gdn_decode_tokens(const void *q, const void *k, const void *v, const flo
  * (64-token chunk, value head) the chunk's fp32 intermediates (Tm, P and
  * E . K K^T at 64 x 64; W, U~, U, dU, dW and two partial gradients at 64 x D;
  * the state and dL/dstate at the chunk's boundaries, Dv x Dk each; about
- * (T/64 + num_seqs) x Hv x (2 Dv Dk + 5 x 64 D + 3 x 64 x 64) x 4 bytes), and
- * per-value-head dq, dk when Hv > Hqk.  At 8192 tokens, 48 value heads and
- * D = 128 that is about 2.9 GB.  The value is at least the sequential size
+ * (T/64 + num_seqs) x Hv x (2 Dv Dk + 7 x 64 D + 3 x 64 x 64) x 4 bytes).  At
+ * 8192 tokens, 48 value heads and D = 128 that is about 2.8 GB.  The value is at least the sequential size
  * below, so a workspace of this size always runs the chunk form.
  */
 size_t gdn_prefill_backward_workspace_size(int32_t num_seqs, int64_t total_tokens,

@@ -636,6 +636,27 @@ __device__ __forceinline__ void ld8(const float *src, bool ok, float *x) {
   x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
   x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
+// 32 consecutive input elements (16-byte aligned) as fp32, by 16-byte loads.
+__device__ __forceinline__ void ld32(const float *src, float *x) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 a = *reinterpret_cast<const float4 *>(src + 4 * i);
+    x[4 * i] = a.x; x[4 * i + 1] = a.y; x[4 * i + 2] = a.z; x[4 * i + 3] = a.w;
+  }
+}
+__device__ __forceinline__ void ld32(const __nv_bfloat16 *src, float *x) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 a = *reinterpret_cast<const uint4 *>(src + 8 * i);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      x[8 * i + 2 * e] = __uint_as_float(w[e] << 16);
+      x[8 * i + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
+    }
+  }
+}
+
 // 3-term product D (+)= A B over KSTEPS K steps of 16, A K-major (blocks of
 // 64 K at a_blk bytes), B MN-major (K rows of 128 bytes, N blocks at b_lbo).
 // Issued by one thread.
@@ -820,19 +841,19 @@ __global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
 #pragma unroll
     for (int cc = 0; cc < DK / 64; ++cc) {
       const int col = half * (DK / 2) + 32 * cc;
-      float v[32];
+      float v[32], qv[32];
+      if (row < len) ld32(q + qoff + (size_t)row * qstride + col, qv);  // in flight beside the TMEM read
       sm100::tmem_ld32(tl + col, v);
       sm100::tmem_wait_ld();
       if (row < C) {  // dQ part and dgamma
         float *dst = p.dQp + (u * C + row) * DK + col;
-        const TI *qr = q + qoff + (size_t)row * qstride + col;
 #pragma unroll
         for (int x = 0; x < 32; x += 4) {
           *reinterpret_cast<float4 *>(dst + x) =
               make_float4(scale * gam * v[x], scale * gam * v[x + 1], scale * gam * v[x + 2], scale * gam * v[x + 3]);
           if (row < len)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc_g = fmaf(to_f32(qr[x + e]), v[x + e], acc_g);
+            for (int e = 0; e < 4; ++e) acc_g = fmaf(qv[x + e], v[x + e], acc_g);
         }
       } else {  // dW = -(dU S0)
         float *dst = p.dW + (u * C + row - C) * DK + col;
@@ -850,17 +871,17 @@ __global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
 #pragma unroll
     for (int cc = 0; cc < DK / 64; ++cc) {
       const int col = half * (DK / 2) + 32 * cc;
-      float v[32];
+      float v[32], kv[32];
+      if (row < len) ld32(k + qoff + (size_t)row * qstride + col, kv);  // in flight beside the TMEM read
       sm100::tmem_ld32(tl + DK + col, v);
       sm100::tmem_wait_ld();
       float *dst = p.dKp + (u * C + row) * DK + col;
-      const TI *kr = k + qoff + (size_t)row * qstride + col;
 #pragma unroll
       for (int x = 0; x < 32; x += 4) {
         *reinterpret_cast<float4 *>(dst + x) = make_float4(kd * v[x], kd * v[x + 1], kd * v[x + 2], kd * v[x + 3]);
         if (row < len)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc_k = fmaf(to_f32(kr[x + e]), v[x + e], acc_k);
+          for (int e = 0; e < 4; ++e) acc_k = fmaf(kv[x + e], v[x + e], acc_k);
       }
     }
     red[(2 + half) * C + row] = acc_k;

@@ -291,7 +291,7 @@ int32_t check_backward(const void *q, const void *k, const void *v, const float 
     if (!q || !k || !v || !g || !beta || !d_o || !dq || !dk || !dv || !dg || !dbeta)
       return GDN_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(d_o, 16) ||
-        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 4) || !aligned(g, 4) ||
+        !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(g, 4) ||
         !aligned(beta, 4) || !aligned(dg, 4) || !aligned(dbeta, 4))
       return GDN_ERR_INVALID_ARG;
   }

@@ -200,6 +200,33 @@ __device__ __forceinline__ void for_frag(float (&acc)[NTL][4], int r0, int c0, i
     for (int e = 0; e < 4; ++e) f(r0 + gid + 8 * (e >> 1), c0 + 8 * t + 2 * tig + (e & 1), acc[t][e]);
 }
 
+// Fragment-position loads and stores of an fp32 matrix M (row stride ld):
+// the two adjacent columns a lane holds per row go as one 8-byte access.
+template <int NTL>
+__device__ __forceinline__ void frag_ld(float (&dst)[NTL][4], const float *M, size_t ld, int r0, int c0,
+                                        int lane) {
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int t = 0; t < NTL; ++t) {
+    const float2 a = *reinterpret_cast<const float2 *>(M + (size_t)(r0 + gid) * ld + c0 + 8 * t + 2 * tig);
+    const float2 b = *reinterpret_cast<const float2 *>(M + (size_t)(r0 + gid + 8) * ld + c0 + 8 * t + 2 * tig);
+    dst[t][0] = a.x; dst[t][1] = a.y; dst[t][2] = b.x; dst[t][3] = b.y;
+  }
+}
+// Rows >= valid are not written.
+template <int NTL>
+__device__ __forceinline__ void frag_st(const float (&src)[NTL][4], float *M, size_t ld, int r0, int c0,
+                                        int lane, int valid) {
+  const int gid = lane >> 2, tig = lane & 3;
+#pragma unroll
+  for (int t = 0; t < NTL; ++t) {
+    if (r0 + gid < valid)
+      *reinterpret_cast<float2 *>(M + (size_t)(r0 + gid) * ld + c0 + 8 * t + 2 * tig) = make_float2(src[t][0], src[t][1]);
+    if (r0 + gid + 8 < valid)
+      *reinterpret_cast<float2 *>(M + (size_t)(r0 + gid + 8) * ld + c0 + 8 * t + 2 * tig) = make_float2(src[t][2], src[t][3]);
+  }
+}
+
 // Sum of the two rows (gid, gid + 8) a lane holds over the warp's columns:
 // returned in every lane of the quad.
 template <int NTL, class F>
@@ -967,6 +994,9 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     tile_async<C, C>(S3, LD64, p.Tm + u * C * C, C, C, tid);
     cp_commit();
     if (tid < C) sB[tid] = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
+    float qp[DK / 16][4], kp[DK / 16][4];  // this head's state-gradient parts, in flight early
+    frag_ld(qp, p.dQp + u * C * DK, DK, r0, cbk, lane);
+    frag_ld(kp, p.dKp + u * C * DK, DK, r0, cbk, lane);
     cp_wait<1>();
     __syncthreads();
     if (tid < C) {
@@ -1033,10 +1063,8 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
       float slo, shi;
       quad_row_sums(acc, [&](int i, int c) { return to_f32(RD[i * L::LD + c]); }, r0, cbv, lane, slo, shi);
       if (tig == 0) { sYV[half * C + r0 + gid] = slo; sYV[half * C + r0 + gid + 8] = shi; }
-      float *dv = p.dv + ((size_t)cp.start * p.Hv + h) * DV;
-      for_frag(acc, r0, cbv, lane, [&](int i, int c, float &x) {
-        if (i < len) dv[(size_t)i * p.Hv * DV + c] = sB[i] * x;
-      });
+      for_frag(acc, r0, cbv, lane, [&](int i, int c, float &x) { x *= sB[i]; });
+      frag_st(acc, p.dv + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, r0, cbv, lane, len);
     }
     __syncthreads();
     tile_async<C, DK>(RD, L::LD, q + qoff, qstride, len, tid);  // V is no longer needed
@@ -1082,14 +1110,18 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
       sCM[j] = b;
     }
     {  // dq += diag(gamma) dO' S0 + (dP . E) K (this value head's parts)
-      const float *dQp = p.dQp + u * C * DK;
-      for_frag(dQ, r0, cbk, lane, [&](int i, int c, float &x) { x += dQp[i * DK + c]; });
+#pragma unroll
+      for (int t = 0; t < DK / 16; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dQ[t][e] += qp[t][e];
       mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dQ, [&](int r, int c) { return S2[(r0 + r) * LD64 + c]; },
                        [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
     }
     {  // dk += diag(kdec) U dS1 + (dP . E)^T Q + (B + B^T) K (diag(beta gamma) X is in already)
-      const float *dKp = p.dKp + u * C * DK;
-      for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) { x += dKp[i * DK + c]; });
+#pragma unroll
+      for (int t = 0; t < DK / 16; ++t)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dK[t][e] += kp[t][e];
       mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S2[c * LD64 + r0 + r]; },
                        [&](int r, int c) { return to_f32(RD[r * L::LD + cbk + c]); }, lane);
       mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(dK, [&](int r, int c) { return S4[(r0 + r) * LD64 + c] + S4[c * LD64 + r0 + r]; },
@@ -1134,15 +1166,8 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     }
     __syncthreads();  // the next value head reuses every buffer but K
   }
-  {  // dq and dk of the query/key head
-    float *dq = p.dq + qoff, *dk = p.dk + qoff;
-    for_frag(dQ, r0, cbk, lane, [&](int i, int c, float &x) {
-      if (i < len) dq[(size_t)i * qstride + c] = x;
-    });
-    for_frag(dK, r0, cbk, lane, [&](int i, int c, float &x) {
-      if (i < len) dk[(size_t)i * qstride + c] = x;
-    });
-  }
+  frag_st(dQ, p.dq + qoff, qstride, r0, cbk, lane, len);  // dq and dk of the query/key head
+  frag_st(dK, p.dk + qoff, qstride, r0, cbk, lane, len);
 }
 
 }  // namespace cbwd

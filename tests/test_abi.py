@@ -214,6 +214,7 @@ def test_backward_workspace_and_validation(lib):
 
         assert call(do=None) == api.GDN_ERR_INVALID_ARG
         assert call(dq=vp + 4) == api.GDN_ERR_INVALID_ARG          # misaligned
+        assert call(dv=vp + 8) == api.GDN_ERR_INVALID_ARG          # bases are 16-byte aligned
         assert call(Hv=5) == api.GDN_ERR_INVALID_ARG
         assert call(Dk=96) == api.GDN_ERR_UNSUPPORTED
         assert call(wsb=1024) == api.GDN_ERR_WORKSPACE

@@ -406,8 +406,7 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
       mma3_rows<C, DK / 16, false, sizeof(TI) == 2>(
           acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c] * sBG[c]; },
           [&](int r, int c) { return to_f32(Ks[r * L::LQ + c0 + c]); }, lane);
-      float *W = p.W + u * C * DK;
-      for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { W[i * DK + c] = x; });
+      frag_st(acc, p.W + u * C * DK, DK, r0, c0, lane, C);
     }
     {
       const int c0 = (w >> 2) * (DV / 2);
@@ -416,8 +415,7 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
       mma3_rows<C, DV / 16, false, sizeof(TI) == 2>(
           acc, [&](int r, int c) { return Ts[(r0 + r) * LD64 + c] * sB[c]; },
           [&](int r, int c) { return to_f32(Vs[r * L::LV + c0 + c]); }, lane);
-      float *Ut = p.Ut + u * C * DV;
-      for_frag(acc, r0, c0, lane, [&](int i, int c, float &x) { Ut[i * DV + c] = x; });
+      frag_st(acc, p.Ut + u * C * DV, DV, r0, c0, lane, C);
     }
   }
 }
@@ -468,12 +466,11 @@ __device__ __forceinline__ void fwd_chain_body(const Params &p, unsigned char *s
       zero_acc(acc);
       mma3_rows<DK>(acc, [&](int r, int c) { return Ws[(r0 + r) * L::LW + c]; },
                     [&](int r, int c) { return S[(vb + c) * L::LS + r]; }, lane);
-      float *Ug = p.U + u * C * DV;
       for_frag(acc, r0, vb, lane, [&](int i, int c, float &x) {
-        const float uu = Us[i * L::LU + c] - x;
-        Us[i * L::LU + c] = uu;
-        Ug[i * DV + c] = uu;
+        x = Us[i * L::LU + c] - x;
+        Us[i * L::LU + c] = x;
       });
+      frag_st(acc, p.U + u * C * DV, DV, r0, vb, lane, C);
     }
     __syncthreads();
     if (j + 1 < nch) {
@@ -557,17 +554,16 @@ __device__ __forceinline__ void rev_chain_body(const Params &p, unsigned char *s
       const int i0 = r0 + gid, i1 = i0 + 8;
       const float kd0 = i0 < len ? expf((float)(Gl - sG[i0])) : 0.f;
       const float kd1 = i1 < len ? expf((float)(Gl - sG[i1])) : 0.f;
-      float *dUg = p.dU + u * C * DV + v0;
       const int tig = lane & 3;
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int i = r0 + gid + 8 * (e >> 1), c = vb + 8 * t + 2 * tig + (e & 1);
-          const float x = scale * a1[t][e] + (e < 2 ? kd0 : kd1) * a2[t][e];
-          dUs[i * L::LO + c] = x;
-          dUg[i * DV + c] = x;
+          a1[t][e] = scale * a1[t][e] + (e < 2 ? kd0 : kd1) * a2[t][e];
+          dUs[i * L::LO + c] = a1[t][e];
         }
+      frag_st(a1, p.dU + u * C * DV + v0, DV, r0, vb, lane, C);
     }
     __syncthreads();
     if (j > 0) {  // the previous chunk's P and K into the freed buffers

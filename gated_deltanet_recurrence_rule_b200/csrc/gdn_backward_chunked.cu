@@ -421,24 +421,26 @@ __global__ void __launch_bounds__(NT) prep_kernel(const Params p) {
 }
 
 // ---- forward chain: S0 and U of every chunk, a whole head (Dv state rows) ----
+// With bf16 inputs the K, U~ and G tiles are double-buffered: chunk j + 1's
+// are in flight while chunk j computes (fp32 inputs do not fit twice).
 template <typename TI, int DK, int DV>
 struct FwdSmem {
+  static constexpr int NB = sizeof(TI) == 2 ? 2 : 1;
   static constexpr int LS = DK + 4, LW = DK + 4, LK = in_ld<TI>(DK), LU = DV + 8;
-  static constexpr size_t OS = 0, OW = OS + DV * LS * 4, OK = OW + C * LW * 4,
-                          OU = OK + up16(C * LK * sizeof(TI)), OG = OU + C * LU * 4, OKD = OG + C * 8,
-                          BYTES = OKD + C * 4;
+  static constexpr size_t KB = up16(C * LK * sizeof(TI)), UB = C * LU * 4;
+  static constexpr size_t OS = 0, OW = OS + DV * LS * 4, OK = OW + C * LW * 4, OU = OK + NB * KB,
+                          OG = OU + NB * UB, OKD = OG + NB * C * 8, BYTES = OKD + C * 4;
 };
 
 // One CTA of NTR threads per (non-empty sequence kk, value head h).
 template <typename TI, int DK, int DV>
 __device__ __forceinline__ void fwd_chain_body(const Params &p, unsigned char *smb, int kk, int h) {
   using L = FwdSmem<TI, DK, DV>;
+  constexpr int NB = L::NB;
   constexpr int NW = NTR / 32;               // 16 warps
   constexpr int RG = DV / 16, CG = NW / RG;  // state update: row groups x column groups
   float *S = reinterpret_cast<float *>(smb + L::OS), *Ws = reinterpret_cast<float *>(smb + L::OW),
-        *Us = reinterpret_cast<float *>(smb + L::OU), *sKd = reinterpret_cast<float *>(smb + L::OKD);
-  TI *Ks = reinterpret_cast<TI *>(smb + L::OK);
-  double *sG = reinterpret_cast<double *>(smb + L::OG);
+        *sKd = reinterpret_cast<float *>(smb + L::OKD);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   if (kk >= p.ph->n_nonempty) return;
   const int n = p.ne_seq[kk], c0 = p.ne_cs[kk], nch = p.ne_cs[kk + 1] - c0;
@@ -446,18 +448,35 @@ __device__ __forceinline__ void fwd_chain_body(const Params &p, unsigned char *s
   const int hk = h / (p.Hv / p.Hqk);
   const TI *k = static_cast<const TI *>(p.k);
   const size_t srow = ((size_t)n * p.Hv + h) * DV;  // first state row of the head
+  auto Kb = [&](int j) { return reinterpret_cast<TI *>(smb + L::OK + (j % NB) * L::KB); };
+  auto Ub = [&](int j) { return reinterpret_cast<float *>(smb + L::OU + (j % NB) * L::UB); };
+  auto Gb = [&](int j) { return reinterpret_cast<double *>(smb + L::OG + (j % NB) * C * 8); };
+  auto issue_tiles = [&](int j) {  // K, U~ and G of chunk j, one commit group
+    const size_t u = (size_t)(c0 + j) * p.Hv + h;
+    const int start = cs + C * j, len = min(C, Lseq - C * j);
+    tile_async<C, DK, NTR>(Kb(j), L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, tid);
+    tile_async<C, DV, NTR>(Ub(j), L::LU, p.Ut + u * C * DV, DV, C, tid);
+    tile_async<1, C, NTR>(Gb(j), C, p.G + u * C, 0, 1, tid);
+    cp_commit();
+  };
   if (p.s0) tile_async<DV, DK, NTR>(S, L::LS, p.s0 + srow * DK, DK, DV, tid);
   else zero_tile<DV, DK, NTR>(S, L::LS, tid);
   tile_async<C, DK, NTR>(Ws, L::LW, p.W + ((size_t)c0 * p.Hv + h) * C * DK, DK, C, tid);
+  issue_tiles(0);  // S0, the first W and chunk 0's tiles in one group
   for (int j = 0; j < nch; ++j) {
     const size_t u = (size_t)(c0 + j) * p.Hv + h;
-    const int start = cs + C * j, len = min(C, Lseq - C * j);
-    tile_async<C, DK, NTR>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, (size_t)p.Hqk * DK, len, tid);
-    tile_async<C, DV, NTR>(Us, L::LU, p.Ut + u * C * DV, DV, C, tid);
-    tile_async<1, C, NTR>(sG, C, p.G + u * C, 0, 1, tid);
-    cp_commit();
-    cp_wait<0>();
+    const int len = min(C, Lseq - C * j);
+    if (NB == 2 && j + 1 < nch) {
+      issue_tiles(j + 1);  // into the buffers chunk j - 1 used
+      cp_wait<1>();
+    } else {
+      if (NB == 1 && j > 0) issue_tiles(j);
+      cp_wait<0>();
+    }
     __syncthreads();
+    TI *Ks = Kb(j);
+    float *Us = Ub(j);
+    const double *sG = Gb(j);
     store_tile<DV, DK, NTR>(p.S0 + u * DV * DK, DK, S, L::LS, tid);
     if (tid < C) sKd[tid] = tid < len ? expf((float)(sG[len - 1] - sG[tid])) : 0.f;
     {  // U = U~ - W S^T: token rows 16 (w & 3), state rows DV / 4 (w >> 2)

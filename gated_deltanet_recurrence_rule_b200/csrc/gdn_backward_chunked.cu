@@ -510,13 +510,18 @@ __device__ __forceinline__ void fwd_chain_body(const Params &p, unsigned char *s
 }
 
 // ---- reverse chain: dS1 and dU of every chunk, last to first ------------------
+// P and K are fetched one chunk ahead into single buffers (the dU product is
+// their only reader).  With bf16 inputs dO, Q, W and G are double-buffered:
+// chunk j - 1's are in flight while chunk j computes.
 template <typename TI, int DK, int DV>
 struct RevSmem {
+  static constexpr int NB = sizeof(TI) == 2 ? 2 : 1;
   static constexpr int LS = DK + 4, LK = in_ld<TI>(DK), LW = DK + 8, LO = SL + 8;
-  static constexpr size_t OS = 0, OP = OS + SL * LS * 4, OO = OP + C * LD64 * 4, OK = OO + C * LO * 4,
-                          OQ = OK + up16(C * LK * sizeof(TI)), OW = OQ + up16(C * LK * sizeof(TI)),
-                          OU = OW + C * LW * 4, OG = OU + C * LO * 4, OGM = OG + C * 8,
-                          BYTES = OGM + C * 4;
+  static constexpr size_t KB = up16(C * LK * sizeof(TI)), OB = C * LO * 4, WB = C * LW * 4;
+  static constexpr size_t OS = 0, OP = OS + SL * LS * 4, OK = OP + C * LD64 * 4, OU = OK + KB,
+                          OO = OU + OB, OQ = OO + NB * OB, OW = OQ + NB * KB, OG = OW + NB * WB,
+                          OGM = OG + NB * C * 8, BYTES = OGM + C * 4;
+  static_assert(BYTES <= 232448, "reverse chain above the 227 KB of shared memory a CTA may use");
 };
 
 // One CTA of NTR threads per (non-empty sequence kk, value head h, SL state
@@ -524,11 +529,10 @@ struct RevSmem {
 template <typename TI, int DK, int DV>
 __device__ __forceinline__ void rev_chain_body(const Params &p, unsigned char *smb, int kk, int h, int v0) {
   using L = RevSmem<TI, DK, DV>;
+  constexpr int NB = L::NB;
   float *dS = reinterpret_cast<float *>(smb + L::OS), *Ps = reinterpret_cast<float *>(smb + L::OP),
-        *dOs = reinterpret_cast<float *>(smb + L::OO), *Ws = reinterpret_cast<float *>(smb + L::OW),
         *dUs = reinterpret_cast<float *>(smb + L::OU), *sGm = reinterpret_cast<float *>(smb + L::OGM);
-  TI *Ks = reinterpret_cast<TI *>(smb + L::OK), *Qs = reinterpret_cast<TI *>(smb + L::OQ);
-  double *sG = reinterpret_cast<double *>(smb + L::OG);
+  TI *Ks = reinterpret_cast<TI *>(smb + L::OK);
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int gid = lane >> 2;
   if (kk >= p.ph->n_nonempty) return;
@@ -539,6 +543,19 @@ __device__ __forceinline__ void rev_chain_body(const Params &p, unsigned char *s
   const size_t srow = ((size_t)n * p.Hv + h) * DV + v0;
   const size_t qstride = (size_t)p.Hqk * DK;
   const float scale = p.scale;
+  auto Ob = [&](int j) { return reinterpret_cast<float *>(smb + L::OO + (j % NB) * L::OB); };
+  auto Qb = [&](int j) { return reinterpret_cast<TI *>(smb + L::OQ + (j % NB) * L::KB); };
+  auto Wb = [&](int j) { return reinterpret_cast<float *>(smb + L::OW + (j % NB) * L::WB); };
+  auto Gb = [&](int j) { return reinterpret_cast<double *>(smb + L::OG + (j % NB) * C * 8); };
+  auto issue_tiles = [&](int j) {  // dO, Q, W and G of chunk j, one commit group
+    const size_t u = (size_t)(c0 + j) * p.Hv + h;
+    const int start = cs + C * j, len = min(C, Lseq - C * j);
+    tile_async<C, SL, NTR>(Ob(j), L::LO, p.dO + ((size_t)start * p.Hv + h) * DV + v0, (size_t)p.Hv * DV, len, tid);
+    tile_async<C, DK, NTR>(Qb(j), L::LK, q + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
+    tile_async<C, DK, NTR>(Wb(j), L::LW, p.W + u * C * DK, DK, C, tid);
+    tile_async<1, C, NTR>(Gb(j), C, p.G + u * C, 0, 1, tid);
+    cp_commit();
+  };
   if (p.dSf) tile_async<SL, DK, NTR>(dS, L::LS, p.dSf + srow * DK, DK, SL, tid);
   else zero_tile<SL, DK, NTR>(dS, L::LS, tid);
   {  // P and K of the last chunk (later ones are fetched one chunk ahead)
@@ -547,17 +564,22 @@ __device__ __forceinline__ void rev_chain_body(const Params &p, unsigned char *s
     tile_async<C, C, NTR>(Ps, LD64, p.P + u * C * C, C, C, tid);
     tile_async<C, DK, NTR>(Ks, L::LK, k + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
   }
+  issue_tiles(nch - 1);  // the final-state gradient, the last P, K and tiles in one group
   const int r0 = 16 * (w & 3);
   for (int j = nch - 1; j >= 0; --j) {
     const size_t u = (size_t)(c0 + j) * p.Hv + h;
     const int start = cs + C * j, len = min(C, Lseq - C * j);
-    tile_async<C, SL, NTR>(dOs, L::LO, p.dO + ((size_t)start * p.Hv + h) * DV + v0, (size_t)p.Hv * DV, len, tid);
-    tile_async<C, DK, NTR>(Qs, L::LK, q + ((size_t)start * p.Hqk + hk) * DK, qstride, len, tid);
-    tile_async<C, DK, NTR>(Ws, L::LW, p.W + u * C * DK, DK, C, tid);
-    tile_async<1, C, NTR>(sG, C, p.G + u * C, 0, 1, tid);
-    cp_commit();
-    cp_wait<0>();
+    if (NB == 2 && j > 0) {
+      issue_tiles(j - 1);  // into the buffers chunk j + 1 used
+      cp_wait<1>();
+    } else {
+      if (NB == 1 && j < nch - 1) issue_tiles(j);
+      cp_wait<0>();
+    }
     __syncthreads();
+    const float *dOs = Ob(j), *Ws = Wb(j);
+    const TI *Qs = Qb(j);
+    const double *sG = Gb(j);
     store_tile<SL, DK, NTR>(p.dS1 + (u * DV + v0) * DK, DK, dS, L::LS, tid);
     if (tid < C) sGm[tid] = tid < len ? expf((float)sG[tid]) : 0.f;
     {  // dU = P^T dO' + diag(kdec) K dS^T: token rows 16 (w & 3), state rows 16 (w >> 2)

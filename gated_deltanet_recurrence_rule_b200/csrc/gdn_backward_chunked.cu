@@ -752,30 +752,84 @@ __device__ __forceinline__ bool cta_wait(uint32_t bar, uint32_t parity, volatile
 }
 
 // ---- products with S0 and dS1 of one (chunk, value head), on tcgen05 ----------
-// D1 = [dO; dU] S0 (M = 128: rows 0-63 the chunk's dO, rows 64-127 its dU),
-// then D2 = U dS1 (rows 0-63; rows 64-127 of that A image still hold dU and
-// are not read), both N = Dk, K = Dv, accumulators in tensor memory:
+// D1 = [dO; dU] S0 (M = 128: rows 0-63 the chunk's dO, rows 64-127 its dU) and
+// D2 = U dS1 (rows 0-63; rows 64-127 of that A image hold stale rows and are
+// not read), both N = Dk, K = Dv, accumulators in tensor memory:
 //   dQ part  diag(scale gamma) (dO S0),  dgamma_t = scale q_t . (dO S0)_t
 //   dW       -(dU S0)
 //   dK part  diag(kdec) (U dS1),         dkdec_t = k_t . (U dS1)_t
 //   dgamma_C = <dS1, S0>
-// One thread issues the MMAs; all threads build the operand images and read
-// the results (warp w reads TMEM lanes 32 (w % 4) .. + 31 and one column half).
+// K runs in halves of 64 (one operand image each), so a CTA holds 64 KB of
+// images and two CTAs share an SM (and its 512 TMEM columns): one's loads run
+// beside the other's products and epilogue.  Order at Dv = 128: D1 half 0,
+// D2 half 0, D2 half 1, D1 half 1; each B image is read back for <dS1, S0>
+// by the step that overwrites it with its partner (S0 half 0 by dS1 half 0,
+// dS1 half 1 by S0 half 1).  One thread issues the MMAs; all threads build
+// the images and read the results (warp w: TMEM lanes 32 (w % 4) .. + 31).
 template <int DK, int DV>
 struct StateGradSmem {
-  static constexpr uint32_t A_BLK = 128 * 128;            // one 64-column K block of a 128-row image
-  static constexpr uint32_t A_BYTES = (DV / 64) * A_BLK;  // [dO; dU], then U
-  static constexpr uint32_t B_LBO = DV * 128;             // one 64-column N block of the MN-major image
-  static constexpr uint32_t B_BYTES = (DK / 64) * B_LBO;  // S0, then dS1
+  static constexpr int NKH = DV / 64;                     // K halves
+  static constexpr uint32_t A_BYTES = 128 * 128;          // 128 rows x 64 K, K-major
+  static constexpr uint32_t B_LBO = 64 * 128;             // one 64-column N block of 64 K rows, MN-major
+  static constexpr uint32_t B_BYTES = (DK / 64) * B_LBO;
   static constexpr uint32_t OAH = 0, OAL = A_BYTES, OBH = 2 * A_BYTES, OBL = OBH + B_BYTES,
                             OG = OBL + B_BYTES, ORED = OG + C * 8, OBAR = ORED + (4 * C + 8) * 4,
-                            OMISC = OBAR + 16, BYTES = OMISC + 32;
+                            OMISC = OBAR + 16, USED = OMISC + 32;
+  // at least 78 KB: no third CTA on an SM whose TMEM two of them fill
+  static constexpr uint32_t BYTES = USED > 78 * 1024 ? USED : 78 * 1024;
   static constexpr uint32_t TMEM_COLS = 2 * DK;  // 128 or 256
 };
 
+// Rows of 8-element chunks, NT threads, N items each: item it of thread tid is
+// chunk (tid + NT it) % CPR of row (tid + NT it) / CPR.
+template <int CPR>
+__device__ __forceinline__ void item_pos(int tid, int it, int &r, int &c) {
+  const int idx = tid + NT * it;
+  r = idx / CPR;
+  c = idx % CPR;
+}
+// Store x (rows of 64 K columns) into the A image (K-major, one K block).
+template <int N>
+__device__ __forceinline__ void st_a_items(unsigned char *AH, unsigned char *AL, const float (&x)[N][8], int tid) {
+#pragma unroll
+  for (int it = 0; it < N; ++it) {
+    int r, c;
+    item_pos<8>(tid, it, r, c);
+    st_img8(AH, AL, r, c, x[it]);
+  }
+}
+// Store x (64 K rows x DK, MN-major) into the B image; with DOT, first add
+// <old image, x> to dot (the old value rebuilt as hi + lo).
+template <int N, int DK, bool DOT>
+__device__ __forceinline__ void st_b_items(unsigned char *BH, unsigned char *BL, uint32_t lbo, const float (&x)[N][8],
+                                           int tid, float &dot) {
+#pragma unroll
+  for (int it = 0; it < N; ++it) {
+    int v, c;
+    item_pos<DK / 8>(tid, it, v, c);
+    const uint32_t off = sm100::sw128_off((uint32_t)v, (uint32_t)(c & 7)) + (c >> 3) * lbo;
+    if (DOT) {
+      const uint4 hv = *reinterpret_cast<const uint4 *>(BH + off), lv = *reinterpret_cast<const uint4 *>(BL + off);
+      const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float o0 = __uint_as_float(hw[e] << 16) + __uint_as_float(lw[e] << 16);
+        const float o1 = __uint_as_float(hw[e] & 0xffff0000u) + __uint_as_float(lw[e] & 0xffff0000u);
+        dot = fmaf(x[it][2 * e], o0, fmaf(x[it][2 * e + 1], o1, dot));
+      }
+    }
+    uint4 hi, lo;
+    split8_bf16(x[it], hi, lo);
+    *reinterpret_cast<uint4 *>(BH + off) = hi;
+    *reinterpret_cast<uint4 *>(BL + off) = lo;
+  }
+}
+
 template <typename TI, int DK, int DV>
-__global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
+__global__ void __launch_bounds__(NT, 2) grads_state_kernel(const Params p) {
   using L = StateGradSmem<DK, DV>;
+  constexpr int NKH = L::NKH;
+  constexpr int AI = 128 * 8 / NT, UI = C * 8 / NT, BI = 64 * (DK / 8) / NT;  // items per thread
   extern __shared__ __align__(1024) unsigned char smb[];
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   ChunkPos cp;
@@ -805,101 +859,100 @@ __global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
     sm100::tmem_relinquish();
   }
   if (tid < C) sG[tid] = p.G[u * C + tid];
-  const float *S0g = p.S0 + u * DV * DK, *S1g = p.dS1 + u * DV * DK;
-  {  // A image [dO; dU] and B image S0 (MN-major: K row v, N columns k), all loads in flight at once
-    constexpr int AC = DV / 8, AI = 128 * AC / NT, BC = DK / 8, BI = DV * BC / NT;
-    const float *dOc = p.dO + ((size_t)cp.start * p.Hv + h) * DV, *dUc = p.dU + u * C * DV;
-    const size_t dOs = (size_t)p.Hv * DV;
-    float xa[AI][8], xb[BI][8];
+  const float *S0g = p.S0 + u * DV * DK, *S1g = p.dS1 + u * DV * DK, *Uc = p.U + u * C * DV;
+  const float *dOc = p.dO + ((size_t)cp.start * p.Hv + h) * DV, *dUc = p.dU + u * C * DV;
+  const size_t dOs = (size_t)p.Hv * DV;
+  // loads of one K half (value columns [64 kh, + 64)) into registers
+  auto ld_dodu = [&](int kh, float (&x)[AI][8]) {
 #pragma unroll
     for (int it = 0; it < AI; ++it) {
-      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      ld8(r < C ? dOc + (size_t)r * dOs + 8 * c : dUc + (size_t)(r - C) * DV + 8 * c, r >= C || r < len, xa[it]);
+      int r, c;
+      item_pos<8>(tid, it, r, c);
+      const int col = 64 * kh + 8 * c;
+      ld8(r < C ? dOc + (size_t)r * dOs + col : dUc + (size_t)(r - C) * DV + col, r >= C || r < len, x[it]);
     }
+  };
+  auto ld_u = [&](int kh, float (&x)[UI][8]) {
+#pragma unroll
+    for (int it = 0; it < UI; ++it) {
+      int r, c;
+      item_pos<8>(tid, it, r, c);
+      ld8(Uc + (size_t)r * DV + 64 * kh + 8 * c, true, x[it]);
+    }
+  };
+  auto ld_state = [&](const float *Sg, int kh, float (&x)[BI][8]) {
 #pragma unroll
     for (int it = 0; it < BI; ++it) {
-      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
-      ld8(S0g + (size_t)v * DK + 8 * c, true, xb[it]);
+      int v, c;
+      item_pos<DK / 8>(tid, it, v, c);
+      ld8(Sg + (size_t)(64 * kh + v) * DK + 8 * c, true, x[it]);
     }
-#pragma unroll
-    for (int it = 0; it < AI; ++it) {
-      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, xa[it]);
-    }
-#pragma unroll
-    for (int it = 0; it < BI; ++it) {
-      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
-      st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, xb[it]);
-    }
-  }
-  sm100::fence_proxy_async_smem();
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smb + L::OMISC);
+  };
   constexpr uint32_t IDESC = sm100::idesc_bf16(128, DK, 0, 1);
-  if (tid == 0) {
-    umma3_kmaj_mn<DV / 16>(tmem, sb + L::OAH, sb + L::OAL, L::A_BLK, sb + L::OBH, sb + L::OBL, L::B_LBO,
-                           IDESC, false);
-    sm100::mma_commit(bar_mma);
-  }
-  {  // U (A rows 0-63) and dS1 (B), loaded while the first product runs, stored once it is
-     // done; <dS1, S0> from the S0 image (hi + lo) each dS1 element replaces
-    constexpr int AC = DV / 8, AI = C * AC / NT, BC = DK / 8, BI = DV * BC / NT;
-    const float *Uc = p.U + u * C * DV;
+  uint32_t tmem = 0;
+  // images written -> visible to the tensor cores -> one thread issues
+  auto issue = [&](uint32_t col, bool acc) {
+    sm100::fence_proxy_async_smem();
+    sm100::tc_fence_before();
+    __syncthreads();
+    sm100::tc_fence_after();
+    tmem = *reinterpret_cast<volatile uint32_t *>(smb + L::OMISC);
+    if (tid == 0) {
+      umma3_kmaj_mn<4>(tmem + col, sb + L::OAH, sb + L::OAL, L::A_BYTES, sb + L::OBH, sb + L::OBL, L::B_LBO,
+                       IDESC, acc);
+      sm100::mma_commit(bar_mma);
+    }
+  };
+  float dot = 0.f;
+  {  // D1 half 0: [dO; dU] and S0
     float xa[AI][8], xb[BI][8];
-#pragma unroll
-    for (int it = 0; it < AI; ++it) {
-      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      ld8(Uc + (size_t)r * DV + 8 * c, true, xa[it]);
-    }
-#pragma unroll
-    for (int it = 0; it < BI; ++it) {
-      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
-      ld8(S1g + (size_t)v * DK + 8 * c, true, xb[it]);
-    }
+    ld_dodu(0, xa);
+    ld_state(S0g, 0, xb);
+    st_a_items(AH, AL, xa, tid);
+    st_b_items<BI, DK, false>(BH, BL, L::B_LBO, xb, tid, dot);
+  }
+  issue(0, false);
+  {  // D2 half 0: U and dS1 (loaded while D1 runs), <dS1, S0> over half 0
+    float xa[UI][8], xb[BI][8];
+    ld_u(0, xa);
+    ld_state(S1g, 0, xb);
     cta_wait(bar_mma, 0, ctl, p.status);
-#pragma unroll
-    for (int it = 0; it < AI; ++it) {
-      const int idx = tid + NT * it, r = idx / AC, c = idx % AC;
-      st_img8(AH + (c >> 3) * L::A_BLK, AL + (c >> 3) * L::A_BLK, r, c & 7, xa[it]);
-    }
-    float dot = 0.f;
-#pragma unroll
-    for (int it = 0; it < BI; ++it) {
-      const int idx = tid + NT * it, v = idx / BC, c = idx % BC;
-      const uint32_t off = sm100::sw128_off((uint32_t)v, (uint32_t)(c & 7)) + (c >> 3) * L::B_LBO;
-      const uint4 hv = *reinterpret_cast<const uint4 *>(BH + off), lv = *reinterpret_cast<const uint4 *>(BL + off);
-      const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float s0a = __uint_as_float(hw[e] << 16) + __uint_as_float(lw[e] << 16);
-        const float s0b = __uint_as_float(hw[e] & 0xffff0000u) + __uint_as_float(lw[e] & 0xffff0000u);
-        dot = fmaf(xb[it][2 * e], s0a, fmaf(xb[it][2 * e + 1], s0b, dot));
-      }
-      st_img8(BH + (c >> 3) * L::B_LBO, BL + (c >> 3) * L::B_LBO, v, c & 7, xb[it]);
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-    if (lane == 0) red[4 * C + w] = dot;
+    st_a_items(AH, AL, xa, tid);
+    st_b_items<BI, DK, true>(BH, BL, L::B_LBO, xb, tid, dot);
   }
-  sm100::fence_proxy_async_smem();
-  sm100::tc_fence_before();
-  __syncthreads();
-  sm100::tc_fence_after();
-  if (tid == 0) {
-    umma3_kmaj_mn<DV / 16>(tmem + DK, sb + L::OAH, sb + L::OAL, L::A_BLK, sb + L::OBH, sb + L::OBL,
-                           L::B_LBO, IDESC, false);
-    sm100::mma_commit(bar_mma);
+  issue(DK, false);
+  if (NKH == 2) {
+    {  // D2 half 1
+      float xa[UI][8], xb[BI][8];
+      ld_u(1, xa);
+      ld_state(S1g, 1, xb);
+      cta_wait(bar_mma, 1, ctl, p.status);
+      st_a_items(AH, AL, xa, tid);
+      st_b_items<BI, DK, false>(BH, BL, L::B_LBO, xb, tid, dot);
+    }
+    issue(DK, true);
+    {  // D1 half 1, <S0, dS1> over half 1
+      float xa[AI][8], xb[BI][8];
+      ld_dodu(1, xa);
+      ld_state(S0g, 1, xb);
+      cta_wait(bar_mma, 0, ctl, p.status);
+      st_a_items(AH, AL, xa, tid);
+      st_b_items<BI, DK, true>(BH, BL, L::B_LBO, xb, tid, dot);
+    }
+    issue(0, true);
   }
-  // D1 while D2 runs: warp w reads TMEM lanes 32 (w % 4) .. + 31 (its rows),
-  // columns [half Dk / 2, + Dk / 2) in blocks of 32
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+  if (lane == 0) red[4 * C + w] = dot;
+  // Epilogue: the finished accumulator first, then, after the last commit
+  // (parity 1 in both orders), the other.  Warp w reads its rows and the
+  // columns [half Dk / 2, + Dk / 2) in blocks of 32.
   const int qd = w & 3, half = w >> 2, row = 32 * qd + lane;
   const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
   const TI *q = static_cast<const TI *>(p.q), *k = static_cast<const TI *>(p.k);
   const size_t qoff = ((size_t)cp.start * p.Hqk + hk) * DK, qstride = (size_t)p.Hqk * DK;
   const float scale = p.scale;
-  {
+  auto read_d1 = [&]() {
     float acc_g = 0.f;
     const float gam = row < len ? expf((float)sG[row < C ? row : 0]) : 0.f;
 #pragma unroll
@@ -927,9 +980,9 @@ __global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
       }
     }
     if (row < C) red[half * C + row] = scale * acc_g;
-  }
-  cta_wait(bar_mma, 1, ctl, p.status);
-  if (qd < 2) {  // D2 rows 0-63: dK part and dkdec
+  };
+  auto read_d2 = [&]() {
+    if (qd >= 2) return;  // D2 rows 0-63: dK part and dkdec
     float acc_k = 0.f;
     const float kd = row < len ? expf((float)(sG[len - 1] - sG[row])) : 0.f;
 #pragma unroll
@@ -949,6 +1002,15 @@ __global__ void __launch_bounds__(NT, 1) grads_state_kernel(const Params p) {
       }
     }
     red[(2 + half) * C + row] = acc_k;
+  };
+  if (NKH == 2) {
+    read_d2();
+    cta_wait(bar_mma, 1, ctl, p.status);
+    read_d1();
+  } else {
+    read_d1();
+    cta_wait(bar_mma, 1, ctl, p.status);
+    read_d2();
   }
   __syncthreads();
   float *sc = p.sc + u * 3 * C;

@@ -1045,7 +1045,7 @@ struct LocalSmem {
   static constexpr size_t OA = 0, OB = OA + C * LA * 4, OC = OB + C * LB * 4,
                           OD = OC + up16(C * LC * sizeof(TI)), O1 = OD + up16(C * LD * sizeof(TI)),
                           O2 = O1 + C * LD64 * 4, O3 = O2 + C * LD64 * 4, O4 = O3 + C * LD64 * 4,
-                          O5 = O4 + C * LD64 * 4, OG = O5 + C * LD64 * 4, OV = OG + C * 8,
+                          O5 = O4 + C * LD64 * 4, OG = O5 + C * LD64 * 4, OV = OG + 2 * C * 8,
                           NVEC = 11, BYTES = OV + NVEC * C * 4;
 };
 
@@ -1058,7 +1058,7 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   float *S1 = reinterpret_cast<float *>(smb + L::O1), *S2 = reinterpret_cast<float *>(smb + L::O2),
         *S3 = reinterpret_cast<float *>(smb + L::O3), *S4 = reinterpret_cast<float *>(smb + L::O4),
         *S5 = reinterpret_cast<float *>(smb + L::O5);
-  double *sG = reinterpret_cast<double *>(smb + L::OG);
+  double *sGb = reinterpret_cast<double *>(smb + L::OG);  // G of this value head and the next
   float *vec = reinterpret_cast<float *>(smb + L::OV);
   // per-row vectors: beta, gamma, kdec, xk (2 halves), yv (2 halves), rP, cP, rM, cM
   float *sB = vec, *sGm = vec + C, *sKd = vec + 2 * C, *sXK = vec + 3 * C, *sYV = vec + 5 * C,
@@ -1080,19 +1080,29 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
   float dQ[DK / 16][4], dK[DK / 16][4];
   zero_acc(dQ);
   zero_acc(dK);
+  // dO, U, P, G and beta of value head gi + 1 are fetched while head gi
+  // computes, each once its buffer is free (dO after the Y step, U after the
+  // E.KK^T step, P after the row sums; G into the other of two buffers, beta
+  // into a register)
+  const float *dOg = p.dO + (size_t)cp.start * p.Hv * DV;
+  const size_t dOs = (size_t)p.Hv * DV;
+  float bnext = 0.f;
   for (int gi = 0; gi < Gq; ++gi) {
     const int h = hk * Gq + gi;
     const size_t u = (size_t)blockIdx.x * p.Hv + h;
-    tile_async<C, DV>(RA, L::LA, p.dO + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
-    tile_async<C, DV>(RB, L::LB, p.U + u * C * DV, DV, C, tid);
-    tile_async<C, C>(S1, LD64, p.P + u * C * C, C, C, tid);
-    tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+    double *sG = sGb + (gi & 1) * C;
+    if (gi == 0) {
+      tile_async<C, DV>(RA, L::LA, dOg + (size_t)h * DV, dOs, len, tid);
+      tile_async<C, DV>(RB, L::LB, p.U + u * C * DV, DV, C, tid);
+      tile_async<C, C>(S1, LD64, p.P + u * C * C, C, C, tid);
+      tile_async<1, C>(sG, C, p.G + u * C, 0, 1, tid);
+    }
     cp_commit();
     if (gi == 0) tile_async<C, DK>(RC, L::LC, k + qoff, qstride, len, tid);  // K serves the group
     tile_async<C, DV>(RD, L::LD, v + ((size_t)cp.start * p.Hv + h) * DV, (size_t)p.Hv * DV, len, tid);
     tile_async<C, C>(S3, LD64, p.Tm + u * C * C, C, C, tid);
     cp_commit();
-    if (tid < C) sB[tid] = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
+    if (tid < C) sB[tid] = gi > 0 ? bnext : tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h] : 0.f;
     float qp[DK / 16][4], kp[DK / 16][4];  // this head's state-gradient parts, in flight early
     frag_ld(qp, p.dQp + u * C * DK, DK, r0, cbk, lane);
     frag_ld(kp, p.dKp + u * C * DK, DK, r0, cbk, lane);
@@ -1167,6 +1177,12 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
     }
     __syncthreads();
     tile_async<C, DK>(RD, L::LD, q + qoff, qstride, len, tid);  // V is no longer needed
+    tile_async<C, C>(RB, LD64, p.EKK + u * C * C, C, C, tid);   // dU is done with too
+    if (gi + 1 < Gq) {
+      tile_async<C, DV>(RA, L::LA, dOg + (size_t)(h + 1) * DV, dOs, len, tid);
+      tile_async<1, C>(sGb + ((gi + 1) & 1) * C, C, p.G + (u + 1) * C, 0, 1, tid);
+      if (tid < C) bnext = tid < len ? p.beta[(size_t)(cp.start + tid) * p.Hv + h + 1] : 0.f;
+    }
     cp_commit();
     {  // Z = dT Tm^T -> S5
       float acc[4][4];
@@ -1183,19 +1199,18 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
                        [&](int r, int c) { return S5[r * LD64 + c64 + c]; }, lane);
       for_frag(acc, r0, c64, lane, [&](int i, int j, float &x) { S4[i * LD64 + j] = i > j ? -x : 0.f; });
     }
-    __syncthreads();
-    tile_async<C, C>(S5, LD64, p.EKK + u * C * C, C, C, tid);
-    cp_commit();
     cp_wait<0>();
     __syncthreads();
-    // S4 <- B = diag(beta) (dA . E); S5 <- dA . (E . K K^T)
+    // S4 <- B = diag(beta) (dA . E); S5 <- dA . (E . K K^T), E . K K^T in RB
     for (int x = tid; x < C * C; x += NT) {
       const int i = x >> 6, j = x & 63;
       const float da = S4[i * LD64 + j];
       S4[i * LD64 + j] = i > j ? sB[i] * da * expf((float)(sG[i] - sG[j])) : 0.f;
-      S5[i * LD64 + j] = da * S5[i * LD64 + j];
+      S5[i * LD64 + j] = da * RB[i * LD64 + j];
     }
     __syncthreads();
+    if (gi + 1 < Gq) tile_async<C, DV>(RB, L::LB, p.U + (u + 1) * C * DV, DV, C, tid);
+    cp_commit();
     if (tid < C) {  // row sums
       float a = 0.f, b = 0.f;
       for (int j = 0; j < C; ++j) { a += S1[tid * LD64 + j]; b += S5[tid * LD64 + j]; }
@@ -1227,6 +1242,8 @@ __global__ void __launch_bounds__(NT) grads_local_kernel(const Params p) {
                        [&](int r, int c) { return to_f32(RC[r * L::LC + cbk + c]); }, lane);
     }
     __syncthreads();
+    if (gi + 1 < Gq) tile_async<C, C>(S1, LD64, p.P + (u + 1) * C * C, C, C, tid);
+    cp_commit();
     if (w == 0) {  // dG, then dg (suffix sums) and dbeta; two tokens per lane
       const float *sc = p.sc + u * 3 * C;
       const float dgC = sc[2 * C];

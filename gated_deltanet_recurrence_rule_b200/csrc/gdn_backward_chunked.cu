@@ -1336,6 +1336,10 @@ cudaError_t launch_k(K kern, dim3 grid, size_t smem, const cbwd::Params &prm, cu
 template <typename TI, int DK, int DV>
 cudaError_t run_chunked(const cbwd::Params &prm, int64_t chunks, cudaStream_t stream) {
   using namespace cbwd;
+  constexpr size_t kMaxSmem = 232448;  // 227 KB, the most dynamic shared memory a CTA may use
+  static_assert(PrepSmem<TI, DK, DV>::BYTES <= kMaxSmem && ChainSmem<TI, DK, DV>::BYTES <= kMaxSmem &&
+                    StateGradSmem<DK, DV>::BYTES <= kMaxSmem && LocalSmem<TI, DK, DV>::BYTES <= kMaxSmem,
+                "a backward kernel needs more shared memory than a CTA may use");
   const dim3 per_chunk((unsigned)chunks, (unsigned)prm.Hv);
   cudaError_t e;
   if ((e = launch_k(prep_kernel<TI, DK, DV>, per_chunk, PrepSmem<TI, DK, DV>::BYTES, prm, stream)) != cudaSuccess) return e;
